@@ -1,0 +1,337 @@
+"""Benchmark of the KV-vector quantization hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Workload (default): 65,536 KV vectors, d = 128, fp16, rows = Gaussian direction
+x LogNormal(0, 0.5) norm with 4 outlier channels x10 (seeded synthetic data,
+one independent shard per rank). One step runs the fused quantize+dequantize
+roundtrip for RotorQuant (and TurboQuant-mse when built) at b = 2, 3, 4 over
+the batch. The headline `value` is the RotorQuant b = 3 roundtrip throughput
+in million vectors per second, summed over ranks (weak scaling, no
+collective on the data path). L2 is flushed (256 MiB write) before every timed
+launch; launches are timed with CUDA events on the launching stream and the
+max over ranks is taken.
+
+`--impl reference` times the float64 CPU oracle on a bounded sample of the
+same workload instead (rank 0 only).
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+N_VEC = 65536
+D = 128
+BITS = (2, 3, 4)
+HEADLINE_BITS = 3
+LARGE_ROWS = 4194304  # 1 GiB of fp16 input at d = 128
+
+
+def rq_bytes_per_vector(d, bits, in_bytes=2, out_bytes=2):
+    """Algorithmic bytes of the fused roundtrip: x in, packed codes + norm out, x_hat out."""
+    G = -(-d // 3)
+    W = -(-(3 * G * bits) // 32)
+    return d * in_bytes + 4 * W + 4 + d * out_bytes
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return j.get("hbm_gbs"), "measured"
+    return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_oracle_rate(n_sample, bits=HEADLINE_BITS, seed=0):
+    """Vectors/s of the oracle's RQ roundtrip on the host (bounded sample)."""
+    from kv_cache_vector_rq_b200 import synth
+    from oracle import codebook, params, rq
+
+    x = synth.lognormal(n_sample, D, seed=seed).float().numpy().astype(np.float64)
+    rot = params.rotors(D, 1)
+    c, _, _ = codebook.lloyd_max(D, bits)
+    t0 = time.perf_counter()
+    rq.roundtrip(x, rot, c, bits)
+    dt = time.perf_counter() - t0
+    return n_sample / dt, dt
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    sample = 2048
+    for _ in range(args.warmup):
+        cpu_oracle_rate(256)
+    times = []
+    for k in range(args.steps):
+        rate, dt = cpu_oracle_rate(sample, seed=k)
+        times.append(dt)
+    t = sum(times) / len(times)
+    value = sample / t / 1e6
+    line = {
+        "impl": "reference", "metric": "quantize+dequantize Mvec/s at d=128 3-bit", "value": value,
+        "unit": "Mvec/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "65536 x d128 fp16 KV vectors (LogNormal norms, 4 outlier channels x10), "
+                               "RotorQuant 3-bit quantize+dequantize", "sample_rows_per_step": sample},
+        "cpu_baseline": {"value": value, "unit": "Mvec/s", "cores": 1, "kind": "oracle",
+                         "sample": "%d rows of the workload per step, float64 numpy oracle" % sample},
+        "e2e": {"value": value, "unit": "Mvec/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="kvrq", choices=["kvrq", "reference"])
+    ap.add_argument("--no-large", action="store_true", help="skip the 1 GiB HBM-roofline leg")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import kv_cache_vector_rq_b200 as kvrq
+    from kv_cache_vector_rq_b200 import synth
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---------------------------------------------------------------- inputs and parameters
+    x = synth.lognormal(N_VEC, D, seed=1000 + rank, dtype=torch.float16, device=dev)
+    rot = torch.from_numpy(kvrq.rq_rotors_init(D, 1).astype(np.float32)).to(dev)
+    cbs = {b: torch.from_numpy(kvrq.tq_codebook_init(D, b)[0].astype(np.float32)).to(dev) for b in BITS}
+    W = {b: kvrq.packed_words(3 * kvrq.rq_groups(D), b) for b in BITS}
+    codes = {b: torch.empty((N_VEC, W[b]), dtype=torch.int32, device=dev) for b in BITS}
+    norms = torch.empty(N_VEC, dtype=torch.float32, device=dev)
+    xhat = torch.empty_like(x)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    legs = [("rq", b) for b in BITS]
+
+    def run_leg(leg):
+        kind, b = leg
+        if kind == "rq":
+            kvrq.rq_quantize_dequantize(x, rot, cbs[b], b, codes=codes[b], norms=norms, xhat=xhat, stream=stream)
+
+    # ---------------------------------------------------------------- warm-up
+    for _ in range(args.warmup):
+        for leg in legs:
+            run_leg(leg)
+    torch.cuda.synchronize()
+    kvrq.device_status()
+
+    # ---------------------------------------------------------------- timed region
+    ev = {leg: [] for leg in legs}
+    launches = 0
+    barrier()
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter()
+    with ClockSampler(local) as clk:
+        for _ in range(args.steps):
+            for leg in legs:
+                flush.zero_()
+                s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                s.record(stream)
+                run_leg(leg)
+                e.record(stream)
+                ev[leg].append((s, e))
+                launches += 1
+        torch.cuda.synchronize()
+    barrier()
+    wall = time.perf_counter() - t_wall
+    kvrq.device_status()
+
+    leg_ms = {leg: max_over_ranks(sum(s.elapsed_time(e) for s, e in ev[leg]) / args.steps) for leg in legs}
+    step_ms = sum(leg_ms.values())
+    head = ("rq", HEADLINE_BITS)
+    head_ms = leg_ms[head]
+    value = N_VEC * world / (head_ms * 1e-3) / 1e6
+
+    peak, peak_kind = measured_peaks()
+    bpv = rq_bytes_per_vector(D, HEADLINE_BITS)
+    achieved = bpv * N_VEC / (head_ms * 1e-3) / 1e9
+    legs_out = {}
+    for (kind, b), ms in leg_ms.items():
+        legs_out["%s_b%d" % (kind, b)] = {
+            "ms": ms, "Mvec_s": N_VEC / (ms * 1e-3) / 1e6,
+            "GB_s": rq_bytes_per_vector(D, b) * N_VEC / (ms * 1e-3) / 1e9}
+
+    # ---------------------------------------------------------------- end to end through the public API
+    x_host = x.to("cpu").pin_memory()
+    codes_h = torch.empty((N_VEC, W[HEADLINE_BITS]), dtype=torch.int32).pin_memory()
+    norms_h = torch.empty(N_VEC, dtype=torch.float32).pin_memory()
+    xhat_h = torch.empty_like(x_host).pin_memory()
+    xd = torch.empty_like(x)
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        xd.copy_(x_host, non_blocking=True)
+        kvrq.rq_quantize_dequantize(xd, rot, cbs[HEADLINE_BITS], HEADLINE_BITS, codes=codes[HEADLINE_BITS],
+                                    norms=norms, xhat=xhat, stream=stream)
+        codes_h.copy_(codes[HEADLINE_BITS], non_blocking=True)
+        norms_h.copy_(norms, non_blocking=True)
+        xhat_h.copy_(xhat, non_blocking=True)
+        e.record(stream)
+        e.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(s.elapsed_time(e))
+    e2e = max_over_ranks(sum(e2e_ms) / len(e2e_ms))
+    h2d = x_host.numel() * 2
+    d2h = codes_h.numel() * 4 + norms_h.numel() * 4 + xhat_h.numel() * 2
+
+    # ---------------------------------------------------------------- 1 GiB leg (HBM roofline, inputs >> L2)
+    large = None
+    if not args.no_large:
+        del flush
+        xl = synth.lognormal(LARGE_ROWS, D, seed=2000 + rank, dtype=torch.float16, device=dev)
+        cl = torch.empty((LARGE_ROWS, W[HEADLINE_BITS]), dtype=torch.int32, device=dev)
+        nl = torch.empty(LARGE_ROWS, dtype=torch.float32, device=dev)
+        ol = torch.empty_like(xl)
+        for _ in range(3):
+            kvrq.rq_quantize_dequantize(xl, rot, cbs[HEADLINE_BITS], HEADLINE_BITS, codes=cl, norms=nl, xhat=ol)
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(10):
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            kvrq.rq_quantize_dequantize(xl, rot, cbs[HEADLINE_BITS], HEADLINE_BITS, codes=cl, norms=nl, xhat=ol)
+            e.record(stream)
+            ts.append((s, e))
+        torch.cuda.synchronize()
+        lms = max_over_ranks(sum(s.elapsed_time(e) for s, e in ts) / len(ts))
+        gbs = bpv * LARGE_ROWS / (lms * 1e-3) / 1e9
+        large = {"rows": LARGE_ROWS, "ms": lms, "Mvec_s": LARGE_ROWS / (lms * 1e-3) / 1e6, "GB_s": gbs,
+                 "frac_of_peak": gbs / peak, "frac_of_8TBs": gbs / 8000.0}
+        del xl, cl, nl, ol
+
+    cpu = None
+    if rank == 0:
+        rate, dt = cpu_oracle_rate(1024)
+        n_s = int(min(16384, max(1024, rate * 10)))
+        rate, dt = cpu_oracle_rate(n_s)
+        cpu = {"value": rate / 1e6, "unit": "Mvec/s", "cores": 1, "kind": "oracle",
+               "sample": "%d rows of the workload, RotorQuant 3-bit roundtrip, float64 numpy oracle (%.1f s)" % (
+                   n_s, dt)}
+
+    if rank == 0:
+        line = {
+            "metric": "quantize+dequantize Mvec/s at d=128 3-bit", "value": value, "unit": "Mvec/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": "65536 x d128 fp16 KV vectors (LogNormal(0,0.5) norms, 4 outlier channels x10), "
+                                   "fused quantize+dequantize, RotorQuant b=2,3,4; headline RotorQuant b=3",
+                       "n_vectors_per_gpu": N_VEC, "d": D, "io_dtype": "fp16", "l2": "flushed (256 MiB write) "
+                       "before every timed launch", "parallelism": "independent shard per GPU (weak scaling)"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+                         "kernel": "rq_row_kernel<__half, 3, RQ_QDQ>", "bytes_per_vector": bpv},
+            "legs": legs_out,
+            "hbm_1gib": large,
+            "e2e": {"value": N_VEC * world / (e2e * 1e-3) / 1e6, "unit": "Mvec/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms": e2e},
+            "gpu_launches": launches,
+            "clocks": clk.summary(),
+            "cpu_baseline": cpu,
+            "wall_s_timed_region": wall,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

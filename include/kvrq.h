@@ -1,0 +1,158 @@
+/*
+ * kvrq -- online vector quantization of KV-cache vectors on NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libkvrq.so. Every hot-path call launches hand-written CUDA kernels
+ * asynchronously on the given stream and returns a status; nothing here
+ * allocates device memory, and no call synchronises the device except
+ * kvrq_device_status().
+ *
+ * Sources of the method (cited by page title and section):
+ *   [RQ]  "TurboQuant + RotorQuant" (README of the RotorQuant repository),
+ *         sections "How TurboQuant Works", "How RotorQuant Works",
+ *         "FMA Count (d=128)", "Codebook Calibration Fix",
+ *         "Post-Prefill Quantization", "The Fused CUDA Kernel",
+ *         "Non-Commutative Algebra Bug Fix", "Triton Kernels".
+ *   [TQB] "TurboQuant 论文解读" (TurboQuant paper walkthrough), sections
+ *         "随机旋转（Lemma 1）", "Beta 分布", "MSE 标量量化（Theorem 1）",
+ *         "QJL 内积无偏估计（Theorem 2）", "简单复现 demo".
+ *   [TQA] arXiv 2504.19874 summary page, section "方法" (Algorithms 1 and 2).
+ *   [PQ]  "TurboQuant и PolarQuant: математика квантизации KV-кэша в LLM",
+ *         paragraph on building codebooks with Lloyd's algorithm.
+ *
+ * Conventions shared by all calls
+ * -------------------------------
+ *  - stream: a cudaStream_t passed as void* (NULL = legacy default stream).
+ *  - Device pointers are caller-owned and must stay valid until the stream
+ *    reaches the call. Vector/tile pointers must be 16-byte aligned; row
+ *    strides (ld*) are in elements (words for packed codes) and must make
+ *    every row start 16-byte aligned unless a call says otherwise.
+ *  - Packed codes: per row one little-endian bit stream, code j in bits
+ *    [j*b, j*b+b) (LSB first), cut into 32-bit words; a row holds
+ *    kvrq_packed_words(n_codes, b) words and unused high bits are zero.
+ *  - QJL signs: bit j of a row is 1 for sign +1 and 0 for -1 (sign(0) = +1),
+ *    m/32 words per row.
+ *  - n == 0 is a no-op returning KVRQ_OK (after argument checks).
+ *  - Arguments are validated on the host before any launch; a bad argument
+ *    returns KVRQ_EINVAL / KVRQ_EUNSUPPORTED and launches nothing. A failed
+ *    launch returns KVRQ_ECUDA. kvrq_last_error_string() explains the last
+ *    non-OK status of the calling thread.
+ *  - Kernels that wait on barriers bound every wait; on time-out they record
+ *    KVRQ_ETIMEOUT in a device status word, which kvrq_device_status() reads.
+ */
+#ifndef KVRQ_H
+#define KVRQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KVRQ_OK = 0,
+  KVRQ_EINVAL = 1,       /* bad pointer, size, stride or alignment */
+  KVRQ_EUNSUPPORTED = 2, /* valid but not implemented (e.g. bits outside 1..4) */
+  KVRQ_ECUDA = 3,        /* a CUDA runtime/driver call failed */
+  KVRQ_ENOCONV = 4,      /* Lloyd-Max did not converge within max_iter */
+  KVRQ_ETIMEOUT = 5      /* a bounded device-side wait ran out */
+} kvrq_status;
+
+typedef enum { KVRQ_F32 = 0, KVRQ_F16 = 1, KVRQ_BF16 = 2 } kvrq_dtype;
+
+typedef enum { KVRQ_RQ_MSE = 0, KVRQ_TQ_MSE = 1, KVRQ_TQ_PROD = 2 } kvrq_method;
+
+/* Version string of the library. */
+const char* kvrq_version(void);
+
+/* Message for the last non-OK status returned on this thread ("" if none). */
+const char* kvrq_last_error_string(void);
+
+/* Reads (and clears) the device status word written by bounded waits.
+ * Synchronises `stream`. Returns KVRQ_OK, KVRQ_ETIMEOUT or KVRQ_ECUDA. */
+kvrq_status kvrq_device_status(void* stream);
+
+/* ===================================================================== setup
+ * Host-only, float64, deterministic functions of their arguments. No CUDA
+ * call is made. Output arrays are caller-owned host memory.
+ */
+
+/* Number of 32-bit words holding n_codes codes of `bits` bits: ceil(n*b/32). */
+int64_t kvrq_packed_words(int64_t n_codes, int bits);
+
+/* RotorQuant group count G = ceil(d/3) [RQ "How RotorQuant Works": d=128 -> 43]. */
+int kvrq_rq_groups(int d);
+
+/* Lloyd-Max codebook for one coordinate of a uniform unit vector in R^d, density
+ * f(x) ~ (1-x^2)^((d-3)/2) on [-1,1] [TQB "Beta 分布", "MSE 标量量化（Theorem 1）"],
+ * iterated as in [PQ]: boundaries at midpoints, centroids at conditional means,
+ * until max |change| < tol or max_iter iterations. Use d_eff = d for RotorQuant
+ * too [RQ "Codebook Calibration Fix"]. Centroids are returned ascending and
+ * exactly symmetric (c[i] = -c[K-1-i]); boundaries[k] = (c[k]+c[k+1])/2.
+ *   d >= 2, 1 <= bits <= 8, tol > 0, max_iter >= 1.
+ *   centroids: [2^bits] out. boundaries: [2^bits - 1] out (may be NULL).
+ *   iterations: out (may be NULL).
+ * Returns KVRQ_ENOCONV if not converged (outputs then hold the last iterate). */
+kvrq_status tq_codebook_init(int d, int bits, double tol, int max_iter, double* centroids,
+                             double* boundaries, int* iterations);
+
+/* G = ceil(d/3) random unit rotors (s, b12, b13, b23), row-major [G][4]
+ * [RQ "How RotorQuant Works": R = [s,0,0,0,b12,b13,b23,0]]: 4 standard normals
+ * per group from the counter-based stream `seed` (splitmix64 + Box-Muller, see
+ * below), divided by their norm (uniform on the unit 3-sphere). d >= 1. */
+kvrq_status rq_rotors_init(int d, uint64_t seed, double* rotors);
+
+/* Random orthogonal Pi [d][d] row-major [TQB "随机旋转（Lemma 1）"]: Householder
+ * QR of the Gaussian matrix A[i][j] = normal(i*d+j) of stream `seed`, then
+ * Pi = Q diag(sign(diag R)) (unique, Haar distributed). 1 <= d <= 16384. */
+kvrq_status tq_rotation_init(int d, uint64_t seed, double* pi);
+
+/* QJL projection T [m][d] row-major, T[i][j] = normal(i*d+j) of stream `seed`
+ * [TQB "QJL 内积无偏估计（Theorem 2）": Gaussian S]. The sketch uses S = T Pi,
+ * which is again i.i.d. N(0,1); the kernels then work in rotated coordinates. */
+kvrq_status qjl_matrix_init(int m, int d, uint64_t seed, double* T);
+
+/* Random streams: normal number i of stream s is taken from splitmix64 outputs
+ * 2j, 2j+1 (j = i/2; output k = mix64(s + (k+1)*0x9E3779B97F4A7C15)), turned
+ * into uniforms ((out>>11)+1)*2^-53 and into two normals by Box-Muller
+ * (cos for even i, sin for odd i). Exposed for tests: out[k] = normal(first+k). */
+kvrq_status kvrq_normals(uint64_t seed, int64_t first, int64_t count, double* out);
+
+/* ================================================================ RotorQuant
+ * [RQ "How RotorQuant Works", "The Fused CUDA Kernel", "Codebook Calibration
+ * Fix"]: u = x/||x|| (norm stored separately), u zero-padded to 3G coordinates,
+ * each group g rotated by the sandwich v' = R_g v R_g~ (computed as the exact
+ * 3x3 matrix of that sandwich), each of the 3G rotated coordinates replaced by
+ * the index of its nearest centroid (ties -> lower index), codes packed.
+ * Dequantization looks the centroids up, applies the inverse sandwich
+ * R_g~ v R_g, drops coordinates >= d and multiplies by the norm.
+ *
+ *   x       [n][ldx] device, dtype xdtype, row-major, first d entries used.
+ *   rotors  [G][4] fp32 device (s, b12, b13, b23).
+ *   centroids [2^bits] fp32 device, ascending.
+ *   codes   [n][ldc] uint32 device, ldc >= kvrq_packed_words(3G, bits).
+ *   norms   [n] fp32 device (||x||, 0 for a zero row).
+ *   xhat    [n][ldo] device, dtype of x (dequantize: odtype).
+ *   1 <= bits <= 4, d >= 2. Fast path: d = 128 with 16-byte aligned rows.
+ */
+kvrq_status rq_quantize(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,
+                        const float* rotors, const float* centroids, int bits, uint32_t* codes,
+                        int64_t ldc, float* norms);
+
+kvrq_status rq_dequantize(void* stream, const uint32_t* codes, int64_t ldc, const float* norms, int64_t n,
+                          int d, const float* rotors, const float* centroids, int bits, void* xhat,
+                          kvrq_dtype odtype, int64_t ldo);
+
+/* One fused launch of quantize and dequantize [RQ "Triton Kernel Speed": the
+ * whole embed -> rotor -> quantize -> unrotor -> extract pipeline in a single
+ * launch]: writes codes, norms and xhat (same dtype as x). codes and norms may
+ * be NULL (xhat only), xhat may not. */
+kvrq_status rq_quantize_dequantize(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d,
+                                   int64_t ldx, const float* rotors, const float* centroids, int bits,
+                                   uint32_t* codes, int64_t ldc, float* norms, void* xhat, int64_t ldo);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVRQ_H */

@@ -1,0 +1,179 @@
+"""kvrq: B200-native online vector quantization of KV-cache vectors.
+
+RotorQuant (Cl(3,0) rotor sandwich on 3-dim groups) and TurboQuant (dense
+random rotation, Lloyd-Max, optional 1-bit QJL residual sketch) as
+hand-written sm_100a CUDA kernels behind a C ABI (include/kvrq.h, libkvrq.so).
+
+This module is a thin binding: it checks tensor placement, dtype and layout
+and passes raw pointers to the library. Every step of the quantization runs
+in the library's kernels; PyTorch only supplies device memory and streams.
+Parameters (codebook, rotors, Pi, QJL matrix) are produced by the library's
+host setup functions in float64 and returned as numpy arrays.
+"""
+
+import ctypes
+
+import numpy as np
+
+from . import _lib
+from ._lib import KvrqError
+
+F32, F16, BF16 = 0, 1, 2
+RQ_MSE, TQ_MSE, TQ_PROD = 0, 1, 2
+
+
+def lib():
+    return _lib.load()
+
+
+def version():
+    return lib().kvrq_version().decode()
+
+
+def _dptr(a):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+# ----------------------------------------------------------------------------- setup (host)
+
+def packed_words(n_codes, bits):
+    return int(lib().kvrq_packed_words(n_codes, bits))
+
+
+def rq_groups(d):
+    return int(lib().kvrq_rq_groups(d))
+
+
+def tq_codebook_init(d, bits, tol=1e-13, max_iter=100000):
+    """Lloyd-Max centroids and boundaries (float64 numpy) for dimension d."""
+    K = 1 << bits
+    c = np.zeros(K)
+    t = np.zeros(K - 1)
+    it = ctypes.c_int(0)
+    _lib.check("tq_codebook_init", lib().tq_codebook_init(d, bits, tol, max_iter, _dptr(c), _dptr(t), ctypes.byref(it)))
+    return c, t
+
+
+def rq_rotors_init(d, seed):
+    G = rq_groups(d)
+    r = np.zeros((G, 4))
+    _lib.check("rq_rotors_init", lib().rq_rotors_init(d, seed, _dptr(r)))
+    return r
+
+
+def tq_rotation_init(d, seed):
+    p = np.zeros((d, d))
+    _lib.check("tq_rotation_init", lib().tq_rotation_init(d, seed, _dptr(p)))
+    return p
+
+
+def qjl_matrix_init(m, d, seed):
+    t = np.zeros((m, d))
+    _lib.check("qjl_matrix_init", lib().qjl_matrix_init(m, d, seed, _dptr(t)))
+    return t
+
+
+def normals(seed, first, count):
+    out = np.zeros(count)
+    _lib.check("kvrq_normals", lib().kvrq_normals(seed, first, count, _dptr(out)))
+    return out
+
+
+# ----------------------------------------------------------------------------- device calls
+
+def _torch():
+    import torch
+
+    return torch
+
+
+def _dtype_code(t):
+    torch = _torch()
+    m = {torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}
+    if t.dtype not in m:
+        raise TypeError("unsupported dtype %s" % t.dtype)
+    return m[t.dtype]
+
+
+def _rows(t, name):
+    """(pointer, leading dimension) of a 2-D CUDA tensor with unit inner stride."""
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if t.dim() != 2 or (t.shape[1] > 1 and t.stride(1) != 1):
+        raise ValueError("%s must be 2-D with unit column stride" % name)
+    return t.data_ptr(), (t.stride(0) if t.shape[0] > 1 else t.shape[1])
+
+
+def _ptr(t, name, dtype=None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError("%s must be %s" % (name, dtype))
+    return t.data_ptr()
+
+
+def _stream(stream):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def rq_quantize(x, rotors, centroids, bits, codes=None, norms=None, stream=None):
+    """Quantize rows of x [n, d] (fp32/fp16/bf16 CUDA). Returns (codes [n, W] int32 view of uint32, norms [n])."""
+    torch = _torch()
+    n, d = x.shape
+    W = packed_words(3 * rq_groups(d), bits)
+    if codes is None:
+        codes = torch.empty((n, W), dtype=torch.int32, device=x.device)
+    if norms is None:
+        norms = torch.empty((n,), dtype=torch.float32, device=x.device)
+    xp, ldx = _rows(x, "x")
+    cp, ldc = _rows(codes, "codes")
+    _lib.check("rq_quantize", lib().rq_quantize(_stream(stream), xp, _dtype_code(x), n, d, ldx,
+                                                _ptr(rotors, "rotors", torch.float32),
+                                                _ptr(centroids, "centroids", torch.float32), bits, cp, ldc,
+                                                _ptr(norms, "norms", torch.float32)))
+    return codes, norms
+
+
+def rq_dequantize(codes, norms, d, rotors, centroids, bits, out_dtype=None, xhat=None, stream=None):
+    """Dequantize packed codes [n, W] + norms [n] into x_hat [n, d]."""
+    torch = _torch()
+    n = codes.shape[0]
+    if xhat is None:
+        xhat = torch.empty((n, d), dtype=out_dtype or torch.float16, device=codes.device)
+    cp, ldc = _rows(codes, "codes")
+    op, ldo = _rows(xhat, "xhat")
+    _lib.check("rq_dequantize", lib().rq_dequantize(_stream(stream), cp, ldc, _ptr(norms, "norms", torch.float32), n, d,
+                                                    _ptr(rotors, "rotors", torch.float32),
+                                                    _ptr(centroids, "centroids", torch.float32), bits, op,
+                                                    _dtype_code(xhat), ldo))
+    return xhat
+
+
+def rq_quantize_dequantize(x, rotors, centroids, bits, codes=None, norms=None, xhat=None, with_codes=True,
+                           stream=None):
+    """Fused roundtrip: returns (codes, norms, x_hat); codes/norms are None when with_codes is False."""
+    torch = _torch()
+    n, d = x.shape
+    W = packed_words(3 * rq_groups(d), bits)
+    if with_codes and codes is None:
+        codes = torch.empty((n, W), dtype=torch.int32, device=x.device)
+    if with_codes and norms is None:
+        norms = torch.empty((n,), dtype=torch.float32, device=x.device)
+    if xhat is None:
+        xhat = torch.empty_like(x)
+    xp, ldx = _rows(x, "x")
+    cp, ldc = _rows(codes, "codes") if codes is not None else (None, W)
+    op, ldo = _rows(xhat, "xhat")
+    _lib.check("rq_quantize_dequantize", lib().rq_quantize_dequantize(
+        _stream(stream), xp, _dtype_code(x), n, d, ldx, _ptr(rotors, "rotors", torch.float32),
+        _ptr(centroids, "centroids", torch.float32), bits, cp, ldc, _ptr(norms, "norms", torch.float32), op, ldo))
+    return codes, norms, xhat
+
+
+def device_status(stream=None):
+    """Raise if a bounded device-side wait ran out since the last check (synchronises the stream)."""
+    _lib.check("kvrq_device_status", lib().kvrq_device_status(_stream(stream)))

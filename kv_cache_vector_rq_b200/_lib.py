@@ -1,0 +1,69 @@
+"""ctypes declarations of libkvrq.so (the C ABI in include/kvrq.h).
+
+Loading fails loudly when the shared library has not been built: there is no
+fallback implementation.
+"""
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkvrq.so")
+
+c_int, c_i64, c_u64, c_f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_uint64, ctypes.c_double
+c_vp = ctypes.c_void_p
+c_dp = ctypes.POINTER(ctypes.c_double)
+c_ip = ctypes.POINTER(ctypes.c_int)
+
+# name -> (restype, argtypes); one entry per function in include/kvrq.h
+SIGNATURES = {
+    "kvrq_version": (ctypes.c_char_p, []),
+    "kvrq_last_error_string": (ctypes.c_char_p, []),
+    "kvrq_device_status": (c_int, [c_vp]),
+    "kvrq_packed_words": (c_i64, [c_i64, c_int]),
+    "kvrq_rq_groups": (c_int, [c_int]),
+    "tq_codebook_init": (c_int, [c_int, c_int, c_f64, c_int, c_dp, c_dp, c_ip]),
+    "rq_rotors_init": (c_int, [c_int, c_u64, c_dp]),
+    "tq_rotation_init": (c_int, [c_int, c_u64, c_dp]),
+    "qjl_matrix_init": (c_int, [c_int, c_int, c_u64, c_dp]),
+    "kvrq_normals": (c_int, [c_u64, c_i64, c_i64, c_dp]),
+    # stream, x, xdtype, n, d, ldx, rotors, centroids, bits, codes, ldc, norms
+    "rq_quantize": (c_int, [c_vp, c_vp, c_int, c_i64, c_int, c_i64, c_vp, c_vp, c_int, c_vp, c_i64, c_vp]),
+    # stream, codes, ldc, norms, n, d, rotors, centroids, bits, xhat, odtype, ldo
+    "rq_dequantize": (c_int, [c_vp, c_vp, c_i64, c_vp, c_i64, c_int, c_vp, c_vp, c_int, c_vp, c_int, c_i64]),
+    # stream, x, xdtype, n, d, ldx, rotors, centroids, bits, codes, ldc, norms, xhat, ldo
+    "rq_quantize_dequantize": (c_int, [c_vp, c_vp, c_int, c_i64, c_int, c_i64, c_vp, c_vp, c_int, c_vp, c_i64, c_vp,
+                                       c_vp, c_i64]),
+}
+
+_lib = None
+
+
+class KvrqError(RuntimeError):
+    """A non-OK status from the library."""
+
+    def __init__(self, name, status, message):
+        super().__init__("%s failed with status %d: %s" % (name, status, message))
+        self.status = status
+
+
+def load():
+    """Load libkvrq.so (once) and declare every function's signature."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libkvrq.so is not built (expected at %s); run __graft_entry__.build()" % LIB_PATH)
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def check(name, status):
+    if status != 0:
+        msg = load().kvrq_last_error_string().decode()
+        raise KvrqError(name, status, msg)

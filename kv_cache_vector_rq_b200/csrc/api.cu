@@ -1,0 +1,250 @@
+// C-ABI entry points of libkvrq.so: argument validation (host, before any
+// launch), TMA tensor-map encoding, kernel dispatch and status reporting.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "kvrq.h"
+#include "kvrq_internal.h"
+#include "rq_launch.h"
+
+namespace kvrq {
+
+// Device status word (see kvrq_device_status); one per device image.
+__device__ unsigned int g_device_status = 0;
+
+static thread_local std::string t_last_error;
+
+kvrq_status set_error(kvrq_status st, const char* msg) {
+  t_last_error = msg ? msg : "";
+  return st;
+}
+
+kvrq_status set_errorf(kvrq_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return st;
+}
+
+static kvrq_status cuda_fail(const char* where, cudaError_t e) {
+  return set_errorf(KVRQ_ECUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+// ------------------------------------------------------------------ per-device state
+struct DeviceInfo {
+  bool ready = false;
+  int num_sms = 0;
+  unsigned* status = nullptr;  // device address of g_device_status
+};
+
+static std::mutex g_dev_mu;
+static DeviceInfo g_dev[64];
+
+static kvrq_status current_device(DeviceInfo** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+  if (dev < 0 || dev >= 64) return set_error(KVRQ_EUNSUPPORTED, "device ordinal >= 64");
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (!di.ready) {
+    e = cudaDeviceGetAttribute(&di.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail("cudaDeviceGetAttribute", e);
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_device_status);
+    if (e != cudaSuccess) return cuda_fail("cudaGetSymbolAddress(status)", e);
+    di.status = static_cast<unsigned*>(p);
+    di.ready = true;
+  }
+  *out = &di;
+  return KVRQ_OK;
+}
+
+// ------------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static kvrq_status get_encode(EncodeTiledFn* fn) {
+  static EncodeTiledFn cached = nullptr;
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (err == cudaSuccess && q == cudaDriverEntryPointSuccess) cached = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  if (!cached) return set_error(KVRQ_ECUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  *fn = cached;
+  return KVRQ_OK;
+}
+
+static size_t dtype_size(kvrq_dtype t) { return t == KVRQ_F32 ? 4 : 2; }
+
+static CUtensorMapDataType tma_type(kvrq_dtype t) {
+  return t == KVRQ_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                       : (t == KVRQ_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+}
+
+// Row-major [rows][ld] matrix, first `cols` columns, boxes of 128 bytes x box_rows,
+// 128-byte swizzle, zero fill out of range.
+kvrq_status encode_rows_map(CUtensorMap* map, const void* ptr, kvrq_dtype dt, int64_t rows, int64_t cols, int64_t ld,
+                            int box_rows) {
+  EncodeTiledFn enc;
+  kvrq_status st = get_encode(&enc);
+  if (st != KVRQ_OK) return st;
+  const size_t es = dtype_size(dt);
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * es)};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / es), (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, tma_type(dt), 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return set_errorf(KVRQ_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return KVRQ_OK;
+}
+
+// ------------------------------------------------------------------ validation helpers
+static bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+static bool valid_dtype(int t) { return t == KVRQ_F32 || t == KVRQ_F16 || t == KVRQ_BF16; }
+
+// Rows of a [n][ld] matrix start 16-byte aligned.
+static bool rows_aligned16(const void* p, int64_t ld, kvrq_dtype dt) {
+  return aligned(p, 16) && ((ld * (int64_t)dtype_size(dt)) % 16) == 0;
+}
+
+static kvrq_status launch_status(const char* where, cudaError_t e) {
+  if (e != cudaSuccess) return cuda_fail(where, e);
+  return KVRQ_OK;
+}
+
+// Shared validation and dispatch of the three RotorQuant calls.
+static kvrq_status rq_call(const char* name, int mode, void* stream, const void* x, kvrq_dtype xdt, int64_t ldx,
+                           const uint32_t* codes_in, uint32_t* codes_out, int64_t ldc, const float* norms_in,
+                           float* norms_out, int64_t n, int d, const float* rotors, const float* centroids, int bits,
+                           void* xhat, kvrq_dtype odt, int64_t ldo) {
+  if (n < 0) return set_errorf(KVRQ_EINVAL, "%s: n < 0", name);
+  if (d < 2 || d > (1 << 20)) return set_errorf(KVRQ_EINVAL, "%s: d must be in 2..2^20", name);
+  if (bits < 1 || bits > 4) return set_errorf(KVRQ_EUNSUPPORTED, "%s: bits must be in 1..4", name);
+  const bool q_side = mode != RQ_DQ, dq_side = mode != RQ_Q;
+  if (q_side && !valid_dtype(xdt)) return set_errorf(KVRQ_EINVAL, "%s: bad input dtype", name);
+  if (dq_side && !valid_dtype(odt)) return set_errorf(KVRQ_EINVAL, "%s: bad output dtype", name);
+  const int G = (d + 2) / 3;
+  const int64_t W = kvrq_packed_words(3 * (int64_t)G, bits);
+  if (n == 0) return KVRQ_OK;
+  if (!rotors || !centroids) return set_errorf(KVRQ_EINVAL, "%s: rotors and centroids are required", name);
+  if (!aligned(rotors, 16) || !aligned(centroids, 4))
+    return set_errorf(KVRQ_EINVAL, "%s: rotors must be 16-byte aligned, centroids 4-byte aligned", name);
+  if (q_side) {
+    if (!x) return set_errorf(KVRQ_EINVAL, "%s: x is NULL", name);
+    if (ldx < d) return set_errorf(KVRQ_EINVAL, "%s: ldx < d", name);
+    if (!aligned(x, dtype_size(xdt))) return set_errorf(KVRQ_EINVAL, "%s: x misaligned", name);
+    if (mode == RQ_Q && (!codes_out || !norms_out)) return set_errorf(KVRQ_EINVAL, "%s: codes and norms are required", name);
+    if (codes_out && (ldc < W || !aligned(codes_out, 4))) return set_errorf(KVRQ_EINVAL, "%s: ldc < packed words or codes misaligned", name);
+    if (norms_out && !aligned(norms_out, 4)) return set_errorf(KVRQ_EINVAL, "%s: norms misaligned", name);
+  } else {
+    if (!codes_in || !norms_in) return set_errorf(KVRQ_EINVAL, "%s: codes and norms are required", name);
+    if (ldc < W || !aligned(codes_in, 4) || !aligned(norms_in, 4))
+      return set_errorf(KVRQ_EINVAL, "%s: ldc < packed words or codes/norms misaligned", name);
+  }
+  if (dq_side) {
+    if (!xhat) return set_errorf(KVRQ_EINVAL, "%s: xhat is NULL", name);
+    if (ldo < d) return set_errorf(KVRQ_EINVAL, "%s: ldo < d", name);
+    if (!aligned(xhat, dtype_size(odt))) return set_errorf(KVRQ_EINVAL, "%s: xhat misaligned", name);
+  }
+  if (n > ((int64_t)1 << 31) - 256) return set_errorf(KVRQ_EUNSUPPORTED, "%s: n >= 2^31", name);
+
+  DeviceInfo* di;
+  kvrq_status st = current_device(&di);
+  if (st != KVRQ_OK) return st;
+  RqArgs a{};
+  a.n = n;
+  a.d = d;
+  a.rotors = rotors;
+  a.centroids = centroids;
+  a.x = x;
+  a.ldx = ldx;
+  a.codes_out = codes_out;
+  a.norms_out = norms_out;
+  a.codes_in = codes_in;
+  a.norms_in = norms_in;
+  a.xhat = xhat;
+  a.ldo = ldo;
+  a.ldc = ldc;
+  a.status = di->status;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  const kvrq_dtype tdt = q_side ? xdt : odt;
+  bool row_path = d == 128;
+  if (q_side) row_path = row_path && rows_aligned16(x, ldx, xdt);
+  if (dq_side) row_path = row_path && rows_aligned16(xhat, ldo, odt);
+  if (mode == RQ_QDQ) row_path = row_path && xdt == odt;
+  if (row_path) {
+    CUtensorMap mx, mo;
+    memset(&mx, 0, sizeof(mx));
+    memset(&mo, 0, sizeof(mo));
+    if (q_side && (st = encode_rows_map(&mx, x, xdt, n, d, ldx, 128)) != KVRQ_OK) return st;
+    if (dq_side && (st = encode_rows_map(&mo, xhat, odt, n, d, ldo, 128)) != KVRQ_OK) return st;
+    if (!q_side) mx = mo;
+    if (!dq_side) mo = mx;
+    return launch_status(name, launch_rq_row(mode, tdt, bits, mx, mo, a, s, di->num_sms));
+  }
+  return launch_status(name, launch_rq_general(mode, xdt, odt, bits, a, s, di->num_sms));
+}
+
+}  // namespace kvrq
+
+using namespace kvrq;
+
+extern "C" {
+
+const char* kvrq_version(void) { return "kvrq 0.1.0 (sm_100a)"; }
+
+const char* kvrq_last_error_string(void) { return t_last_error.c_str(); }
+
+kvrq_status kvrq_device_status(void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned h = 0, zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&h, g_device_status, sizeof(h), 0, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemcpyToSymbolAsync(g_device_status, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail("kvrq_device_status", e);
+  if (h & 1u) return set_error(KVRQ_ETIMEOUT, "a bounded device-side wait ran out");
+  if (h) return set_errorf(KVRQ_ECUDA, "device status word 0x%x", h);
+  return KVRQ_OK;
+}
+
+kvrq_status rq_quantize(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,
+                        const float* rotors, const float* centroids, int bits, uint32_t* codes, int64_t ldc,
+                        float* norms) {
+  return rq_call("rq_quantize", RQ_Q, stream, x, xdtype, ldx, nullptr, codes, ldc, nullptr, norms, n, d, rotors,
+                 centroids, bits, nullptr, xdtype, 0);
+}
+
+kvrq_status rq_dequantize(void* stream, const uint32_t* codes, int64_t ldc, const float* norms, int64_t n, int d,
+                          const float* rotors, const float* centroids, int bits, void* xhat, kvrq_dtype odtype,
+                          int64_t ldo) {
+  return rq_call("rq_dequantize", RQ_DQ, stream, nullptr, odtype, 0, codes, nullptr, ldc, norms, nullptr, n, d,
+                 rotors, centroids, bits, xhat, odtype, ldo);
+}
+
+kvrq_status rq_quantize_dequantize(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,
+                                   const float* rotors, const float* centroids, int bits, uint32_t* codes,
+                                   int64_t ldc, float* norms, void* xhat, int64_t ldo) {
+  return rq_call("rq_quantize_dequantize", RQ_QDQ, stream, x, xdtype, ldx, nullptr, codes, ldc, nullptr, norms, n, d,
+                 rotors, centroids, bits, xhat, xdtype, ldo);
+}
+
+}  // extern "C"

@@ -1,0 +1,46 @@
+// Host-visible launch interface of the RotorQuant kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kvrq.h"
+
+namespace kvrq {
+
+enum RqMode { RQ_Q = 0, RQ_DQ = 1, RQ_QDQ = 2 };
+
+// Arguments of one RotorQuant launch (device pointers; unused ones are NULL).
+struct RqArgs {
+  int64_t n;  // rows
+  int d;
+  const float* rotors;     // [G][4]
+  const float* centroids;  // [2^bits]
+  // quantize side
+  const void* x;
+  int64_t ldx;
+  uint32_t* codes_out;
+  float* norms_out;
+  // dequantize side
+  const uint32_t* codes_in;
+  const float* norms_in;
+  void* xhat;
+  int64_t ldo;
+  int64_t ldc;  // row stride of codes (words), both directions
+  unsigned* status;  // device status word (bounded-wait time-outs)
+};
+
+// d = 128 thread-per-row kernel fed by TMA tensor maps over x and x_hat
+// (128-byte boxes of 128 rows, 128-byte swizzle).
+cudaError_t launch_rq_row(int mode, kvrq_dtype dt, int bits, const CUtensorMap& map_x, const CUtensorMap& map_o,
+                          const RqArgs& a, cudaStream_t st, int num_sms);
+
+// Dynamic shared memory the row kernel requests.
+size_t rq_row_smem_bytes(int mode, kvrq_dtype dt, int bits);
+
+// Any d / stride, warp-per-row kernel.
+cudaError_t launch_rq_general(int mode, kvrq_dtype dt_in, kvrq_dtype dt_out, int bits, const RqArgs& a,
+                              cudaStream_t st, int num_sms);
+
+}  // namespace kvrq

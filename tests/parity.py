@@ -1,0 +1,94 @@
+"""Comparison rules between the CUDA path and the float64 oracle.
+
+Codes: bit-exact, except at coordinates whose oracle decision value lies within
+MARGIN (1e-5, unit-sphere scale) of a decision boundary; there either adjacent
+code is accepted and the case is counted. Float outputs: within one unit in
+the last place of the output dtype plus a float32-arithmetic allowance, on
+rows whose codes all agree (normwise relative error is also bounded by
+1e-3 plus the output dtype's unit roundoff).
+"""
+
+import numpy as np
+import torch
+
+from oracle import codes as ocodes
+
+MARGIN = 1e-5
+
+UNIT_ROUNDOFF = {torch.float32: 2.0 ** -24, torch.float16: 2.0 ** -11, torch.bfloat16: 2.0 ** -8}
+
+
+def to_f64(t):
+    return t.detach().to("cpu").to(torch.float64).numpy()
+
+
+def words_u32(t):
+    """int32 device/host tensor of packed words -> uint32 numpy."""
+    return t.detach().to("cpu").numpy().astype(np.int64).astype(np.uint32)
+
+
+def ulp(values, dtype):
+    """Spacing of `dtype` at |values| (float64 array)."""
+    a = np.abs(values)
+    if dtype == torch.float32:
+        return np.spacing(a.astype(np.float32)).astype(np.float64)
+    if dtype == torch.float16:
+        return np.spacing(a.astype(np.float16)).astype(np.float64)
+    # bfloat16: 8 significant bits, smallest normal 2^-126
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
+    return 2.0 ** (e - 7)
+
+
+def near_boundary(y, centroids, margin=MARGIN):
+    """Boolean mask: the decision value y is within `margin` of a midpoint of the codebook."""
+    c = np.asarray(centroids, dtype=np.float64)
+    t = 0.5 * (c[:-1] + c[1:])
+    if t.size == 0:
+        return np.zeros(np.shape(y), dtype=bool)
+    return np.min(np.abs(np.asarray(y)[..., None] - t), axis=-1) < margin
+
+
+def compare_codes(gpu_words, oracle_q, n_codes, bits, centroids, decision=None, margin=MARGIN):
+    """Checks GPU packed words against the oracle's quantization dict.
+
+    Returns (n_boundary_mismatches, rows_with_any_mismatch mask). Raises
+    AssertionError on any mismatch outside the margin, on a mismatch that is
+    not to an adjacent code, or on nonzero padding bits."""
+    gw = np.asarray(gpu_words, dtype=np.uint32)
+    W = ocodes.n_words(n_codes, bits)
+    assert gw.shape[1] >= W
+    gw = gw[:, :W]
+    used = n_codes * bits - 32 * (W - 1)
+    if used < 32:
+        assert np.all((gw[:, -1].astype(np.int64) >> used) == 0), "nonzero padding bits"
+    g_codes = ocodes.unpack(gw, n_codes, bits)
+    o_codes = oracle_q["codes"]
+    y = oracle_q["y"] if decision is None else decision
+    diff = g_codes != o_codes
+    if diff.any():
+        nb = near_boundary(y, centroids, margin)
+        bad = diff & ~nb
+        assert not bad.any(), "codes differ away from a decision boundary at %s (gpu %s, oracle %s, y %s)" % (
+            np.argwhere(bad)[:5].tolist(), g_codes[bad][:5], o_codes[bad][:5], np.asarray(y)[bad][:5])
+        assert np.all(np.abs(g_codes[diff] - o_codes[diff]) == 1), "boundary mismatch to a non-adjacent code"
+    return int(diff.sum()), diff.any(axis=1)
+
+
+def compare_floats(gpu, ref, out_dtype, row_scale, skip_rows=None, arith_rtol=2e-6, name="x_hat"):
+    """Elementwise |gpu - ref| <= ulp(ref) + arith_rtol * row_scale on rows not skipped,
+    and normwise relative error <= 1e-3 + unit roundoff."""
+    g = np.asarray(gpu, dtype=np.float64)
+    r = np.asarray(ref, dtype=np.float64)
+    keep = np.ones(g.shape[0], dtype=bool) if skip_rows is None else ~np.asarray(skip_rows)
+    g, r = g[keep], r[keep]
+    sc = np.asarray(row_scale, dtype=np.float64)[keep][:, None]
+    tol = ulp(r, out_dtype) + arith_rtol * sc
+    err = np.abs(g - r)
+    assert np.all(err <= tol), "%s: max excess %g at %s" % (name, float(np.max(err - tol)),
+                                                            np.unravel_index(np.argmax(err - tol), err.shape))
+    rn = np.linalg.norm(r, axis=1)
+    ok = rn > 0
+    rel = np.linalg.norm(g - r, axis=1)[ok] / rn[ok]
+    if rel.size:
+        assert rel.max() <= 1e-3 + UNIT_ROUNDOFF[out_dtype], "%s: normwise relative error %g" % (name, rel.max())
+    return int(keep.sum())

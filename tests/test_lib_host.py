@@ -1,0 +1,152 @@
+"""Host-side checks of libkvrq.so (no GPU): symbols, parameter setup parity
+against the oracle, and argument validation that must fail before any launch."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import kv_cache_vector_rq_b200 as kvrq
+from kv_cache_vector_rq_b200 import _lib
+from oracle import codebook, params, rng
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+INCLUDE = os.path.join(ROOT, "include")
+
+
+def _declared_functions():
+    names = []
+    for fname in sorted(os.listdir(INCLUDE)):
+        if not fname.endswith(".h"):
+            continue
+        src = open(os.path.join(INCLUDE, fname)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        for m in re.finditer(r"^[A-Za-z_][\w \*]*?\b([A-Za-z_]\w*)\s*\(", src, flags=re.M):
+            if m.group(1) not in ("if", "defined"):
+                names.append(m.group(1))
+    return names
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = kvrq.lib()
+    declared = _declared_functions()
+    assert len(declared) >= 12
+    for name in declared:
+        assert hasattr(lib, name), "libkvrq.so does not export %s" % name
+        assert name in _lib.SIGNATURES, "no ctypes signature for %s" % name
+    assert set(_lib.SIGNATURES) == set(declared)
+    assert "sm_100a" in kvrq.version()
+
+
+def test_packed_words_and_groups():
+    assert kvrq.packed_words(129, 3) == 13
+    assert kvrq.packed_words(128, 3) == 12
+    assert kvrq.packed_words(128, 2) == 8
+    assert kvrq.packed_words(0, 3) == 0
+    assert kvrq.rq_groups(128) == 43 and kvrq.rq_groups(3) == 1 and kvrq.rq_groups(4096) == 1366
+
+
+# ------------------------------------------------------------------ setup parity
+
+def test_normals_match_oracle_stream():
+    for seed in (0, 1, 12345, 2 ** 63 + 7):
+        a = kvrq.normals(seed, 0, 1001)
+        b = rng.normals(seed, 1001)
+        assert np.abs(a - b).max() < 1e-13
+    # counter-based: any window of the stream
+    assert np.abs(kvrq.normals(5, 37, 10) - rng.normals(5, 47)[37:]).max() < 1e-13
+
+
+@pytest.mark.parametrize("d", [2, 3, 16, 64, 128, 129, 256, 1536, 4096])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_codebook_matches_oracle(d, bits):
+    # Both sides iterate to max |change| < 1e-14 from different starts and evaluate
+    # the cell integrals by different routes (continued fraction vs scipy), so they
+    # agree to the fixed point's conditioning: ~1e-12 absolute, ~1e-10 relative at d = 4096.
+    c_lib, t_lib = kvrq.tq_codebook_init(d, bits, tol=1e-14)
+    c_or, t_or, _ = codebook.lloyd_max(d, bits, tol=1e-14)
+    assert np.all(np.abs(c_lib - c_or) <= 1e-12 + 2e-10 * np.abs(c_or))
+    assert np.all(np.abs(t_lib - t_or) <= 1e-12 + 2e-10 * np.abs(t_or))
+    assert np.array_equal(c_lib, -c_lib[::-1])
+
+
+def test_codebook_reports_non_convergence():
+    c = np.zeros(8)
+    st = kvrq.lib().tq_codebook_init(128, 3, 1e-15, 3, kvrq._dptr(c), None, None)
+    assert st == 4  # KVRQ_ENOCONV
+
+
+@pytest.mark.parametrize("d", [1, 2, 3, 4, 128, 4096])
+def test_rotors_match_oracle(d):
+    assert np.abs(kvrq.rq_rotors_init(d, 11) - params.rotors(d, 11)).max() < 1e-14
+
+
+@pytest.mark.parametrize("d", [1, 2, 3, 17, 128, 256])
+def test_rotation_matches_oracle(d):
+    p_lib = kvrq.tq_rotation_init(d, 2)
+    p_or = params.rotation(d, 2)
+    assert np.abs(p_lib - p_or).max() < 1e-12
+    assert np.abs(p_lib @ p_lib.T - np.eye(d)).max() < 1e-13
+
+
+@pytest.mark.slow
+def test_rotation_matches_oracle_large():
+    p_lib = kvrq.tq_rotation_init(1536, 2)
+    p_or = params.rotation(1536, 2)
+    assert np.abs(p_lib - p_or).max() < 1e-11
+
+
+def test_qjl_matrix_matches_oracle():
+    assert np.abs(kvrq.qjl_matrix_init(128, 96, 3) - params.qjl_matrix(128, 96, 3)).max() < 1e-13
+
+
+def test_setup_rejects_bad_arguments():
+    lib = kvrq.lib()
+    buf = np.zeros(64)
+    assert lib.tq_codebook_init(1, 3, 1e-12, 100, kvrq._dptr(buf), None, None) == 1
+    assert lib.tq_codebook_init(128, 0, 1e-12, 100, kvrq._dptr(buf), None, None) == 1
+    assert lib.tq_codebook_init(128, 3, 0.0, 100, kvrq._dptr(buf), None, None) == 1
+    assert lib.rq_rotors_init(0, 1, kvrq._dptr(buf)) == 1
+    assert lib.tq_rotation_init(0, 1, kvrq._dptr(buf)) == 1
+    assert lib.qjl_matrix_init(0, 4, 1, kvrq._dptr(buf)) == 1
+    assert "d must be" in lib.kvrq_last_error_string().decode() or lib.kvrq_last_error_string()
+
+
+# ------------------------------------------------------------------ hot-path validation (no launch)
+
+P = 0x10000  # a fake, 16-byte aligned device address: validation fails before it is used
+
+
+def test_rq_validation_fails_before_any_launch():
+    lib = kvrq.lib()
+    EINVAL, EUNSUP = 1, 2
+    ok_args = dict(x=P, dt=1, n=10, d=128, ldx=128, rot=P, cb=P, bits=3, codes=P, ldc=13, norms=P)
+
+    def q(**kw):
+        a = dict(ok_args, **kw)
+        return lib.rq_quantize(None, a["x"], a["dt"], a["n"], a["d"], a["ldx"], a["rot"], a["cb"], a["bits"],
+                               a["codes"], a["ldc"], a["norms"])
+
+    assert q(n=-1) == EINVAL
+    assert q(d=1) == EINVAL
+    assert q(bits=0) == EUNSUP and q(bits=5) == EUNSUP
+    assert q(dt=7) == EINVAL
+    assert q(x=None) == EINVAL
+    assert q(rot=None) == EINVAL
+    assert q(rot=P + 4) == EINVAL  # rotors must be 16-byte aligned
+    assert q(ldx=100) == EINVAL
+    assert q(ldc=12) == EINVAL  # 129 codes at 3 bits need 13 words
+    assert q(codes=None) == EINVAL
+    assert q(x=P + 1) == EINVAL  # not even element aligned
+    assert q(n=0) == 0  # empty input is a no-op, no device touched
+    msg = lib.kvrq_last_error_string().decode()
+    assert isinstance(msg, str)
+    # dequantize and fused calls share the same checks
+    assert lib.rq_dequantize(None, P, 12, P, 10, 128, P, P, 3, P, 1, 128) == EINVAL
+    assert lib.rq_dequantize(None, P, 13, P, 10, 128, P, P, 3, P, 9, 128) == EINVAL
+    assert lib.rq_dequantize(None, P, 13, P, 0, 128, P, P, 3, P, 1, 128) == 0
+    assert lib.rq_quantize_dequantize(None, P, 1, 10, 128, 128, P, P, 3, P, 13, P, None, 128) == EINVAL
+    assert lib.rq_quantize_dequantize(None, P, 1, 10, 128, 128, P, P, 3, P, 13, P, P, 64) == EINVAL
