@@ -26,6 +26,9 @@
 
 #include <cuda_runtime.h>
 
+#include <cstdlib>
+#include <type_traits>
+
 #include "kvrq_device.cuh"
 #include "rq_launch.h"
 
@@ -91,19 +94,6 @@ __device__ __forceinline__ uint32_t get_code(const uint32_t (&w)[W], int j) {
   return v & ((1u << BITS) - 1u);
 }
 
-// Rotation matrices (9 floats padded to 12) for all groups, and the codebook
-// split into positive boundaries and magnitudes, built by the whole CTA.
-__device__ __forceinline__ void build_rotor_table(const float* __restrict__ rotors, int G, float4* __restrict__ mtab) {
-  for (int g = threadIdx.x; g < G; g += blockDim.x) {
-    const float4 r = __ldg(reinterpret_cast<const float4*>(rotors) + g);
-    float m[9];
-    rotor_matrix(r.x, r.y, r.z, r.w, m);
-    mtab[3 * g + 0] = make_float4(m[0], m[1], m[2], m[3]);
-    mtab[3 * g + 1] = make_float4(m[4], m[5], m[6], m[7]);
-    mtab[3 * g + 2] = make_float4(m[8], 0.f, 0.f, 0.f);
-  }
-}
-
 template <int BITS>
 __device__ __forceinline__ void build_codebook(const float* __restrict__ centroids, float* tau, float* mag, float* cfull) {
   constexpr int K = 1 << BITS, H = K / 2;
@@ -114,240 +104,420 @@ __device__ __forceinline__ void build_codebook(const float* __restrict__ centroi
 
 // ============================================================================
 // d = 128, one thread per row, TMA-streamed 128-row tiles.
+//
+// Per row: pass 1 reads the row from the swizzled shared tile and forms
+// ||x||^2; pass 2 re-reads it a group pair (6 elements) at a time, rotates
+// the pair with packed f32x2 FMAs, quantizes,
+// inverse-rotates and writes x_hat back into the same shared positions, from
+// where a TMA tensor store writes it out.
+//
+// Quantization (nearest centroid, ties to the lower index) runs on the FMA
+// pipe. With u = y/||x|| the rotated unit coordinate and B = 2^62:
+//   step_j = sat(|y'| * (B/||x||) - tau_j * B) is exactly 0 or 1 (near a
+//            boundary the exact value of that fused multiply-add is 0 or at
+//            least tau_j * B * 2^-47 >= 2^48 in magnitude, since every
+//            positive boundary at d = 128 exceeds 2^-8), and it equals
+//            [|u| > tau_j] up to the rounding of B/||x|| (relative 2^-24);
+//   cnt    = sum_j step_j, the number of positive boundaries below |u|;
+//   mag    = ||x|| c[H + cnt], accumulated as ||x|| c[H] + sum_j step_j delta_j;
+//   sign   = sign bit of y' = y - 2^-30 ||x|| (an exact zero counts as
+//            negative, as the tie rule requires; the shift is far inside the
+//            1e-5 decision margin);
+//   code   = H - 1/2 + sign (cnt + 1/2),  c_hat = sign mag.
+// Codes are added, as exact small integers, into float accumulators that
+// start at 2^23; the low 23 mantissa bits of each accumulator are a window
+// of the packed bit stream.
 // ============================================================================
+namespace row {
+
+constexpr int D = 128;
+constexpr int G = 43;         // groups of 3
+constexpr int NP = 22;        // group pairs (the last: group 42 and an all-zero group)
+constexpr int NC = 3 * G;     // 129 stored codes
+constexpr int kRows = 128;    // rows per tile = threads per CTA
+constexpr float kB = 4611686018427387904.0f;      // 2^62
+constexpr float kShift = 9.313225746154785e-10f;  // 2^-30
+constexpr float kWindow0 = 8388608.0f;            // 2^23
+
 template <typename T>
-struct RowTile {
-  static constexpr int D = 128;
-  static constexpr int kRows = 128;
-  static constexpr int kBoxElems = 128 / sizeof(T);        // elements per 128-byte box row
-  static constexpr int kBoxes = D / kBoxElems;             // boxes per tile (2 for 16-bit, 4 for fp32)
+struct Tile {
+  static constexpr int kBoxElems = 128 / (int)sizeof(T);  // elements per 128-byte box row
+  static constexpr int kBoxes = D / kBoxElems;             // 2 (16-bit) or 4 (fp32)
   static constexpr int kBoxBytes = kRows * 128;            // 16 KB
   static constexpr int kTileBytes = kBoxes * kBoxBytes;    // 32 KB (16-bit) / 64 KB (fp32)
-  static constexpr int kChunks = D * (int)sizeof(T) / 16;  // 16-byte chunks per row
-  static constexpr int kE = 16 / (int)sizeof(T);           // elements per chunk
-  static constexpr int kStages = 2;
-
-  // byte offset of 16-byte chunk j of row r inside a swizzled tile
-  __device__ __forceinline__ static uint32_t chunk_offset(int r, int j) {
-    const int box = j >> 3, c = j & 7;
-    return (uint32_t)(box * kBoxBytes + r * 128 + ((c ^ (r & 7)) << 4));
+  static constexpr int kE = 16 / (int)sizeof(T);           // elements per 16-byte chunk
+  static constexpr int kChunks = D / kE;
+  // byte offset of 16-byte chunk j of row r in the 128-byte-swizzled tile
+  __device__ __forceinline__ static uint32_t chunk(int r, int j) {
+    return (uint32_t)((j >> 3) * kBoxBytes + r * 128 + (((j & 7) ^ (r & 7)) << 4));
   }
 };
 
 template <int BITS>
-struct RowCodes {
-  static constexpr int G = 43;
-  static constexpr int NC = 3 * G;
-  static constexpr int W = (NC * BITS + 31) / 32;
-};
-
-// Shared memory layout of the row kernel (offsets from a 1024-aligned base).
-template <typename T, int BITS, int MODE>
-struct RowSmem {
-  using TL = RowTile<T>;
-  static constexpr int W = RowCodes<BITS>::W;
+struct Codes {
   static constexpr int K = 1 << BITS;
-  static constexpr bool kIn = MODE != RQ_DQ;
-  static constexpr bool kOut = MODE != RQ_Q;
-  static constexpr int in_off = 0;
-  static constexpr int in_bytes = kIn ? TL::kStages * TL::kTileBytes : 0;
-  static constexpr int out_off = in_off + in_bytes;
-  static constexpr int out_bytes = kOut ? TL::kTileBytes : 0;
-  static constexpr int codes_off = out_off + out_bytes;
-  static constexpr int codes_bytes = TL::kRows * W * 4;
-  static constexpr int lut_off = codes_off + ((codes_bytes + 15) / 16) * 16;
-  static constexpr int lut_bytes = MODE == RQ_DQ ? K * TL::kRows * 4 : 0;
-  static constexpr int mtab_off = lut_off + lut_bytes;
-  static constexpr int mtab_bytes = 3 * 43 * 16;
-  static constexpr int cb_off = mtab_off + mtab_bytes;
-  static constexpr int cb_bytes = 64 * 4;
-  static constexpr int bar_off = cb_off + cb_bytes;
-  static constexpr int bytes = bar_off + 64;
-  static constexpr int alloc = bytes + 1024;  // room to align the base
+  static constexpr int H = K / 2;
+  static constexpr int W = (NC * BITS + 31) / 32;
+  static constexpr int CPW = 23 / BITS;  // codes per float window
+  static constexpr int NWIN = (NC + CPW - 1) / CPW;
 };
 
-template <typename T, int BITS, int MODE>
-__global__ void __launch_bounds__(128) rq_row_kernel(const __grid_constant__ CUtensorMap map_x,
-                                                     const __grid_constant__ CUtensorMap map_o, RqArgs a) {
-  using TL = RowTile<T>;
-  using SM = RowSmem<T, BITS, MODE>;
-  constexpr int D = TL::D, G = RowCodes<BITS>::G, W = RowCodes<BITS>::W, K = 1 << BITS;
-  constexpr int S = TL::kStages;
+template <typename T, int BITS, int MODE, int STAGES>
+struct Smem {
+  static constexpr int W = Codes<BITS>::W;
+  static constexpr int tile_bytes = STAGES * Tile<T>::kTileBytes;
+  static constexpr int codes_off = tile_bytes;  // [2][kRows][W] words
+  static constexpr int codes_stage = ((kRows * W * 4 + 15) / 16) * 16;
+  static constexpr int lut_off = codes_off + 2 * codes_stage;  // dequantize: [K][kRows] floats
+  static constexpr int lut_bytes = MODE == RQ_DQ ? Codes<BITS>::K * kRows * 4 : 0;
+  static constexpr int mp_off = lut_off + lut_bytes;  // [NP][10] float2
+  static constexpr int mp_bytes = NP * 10 * 8;
+  static constexpr int cb_off = mp_off + mp_bytes;  // codebook constants
+  static constexpr int cb_bytes = 64 * 4;
+  static constexpr int bar_off = cb_off + cb_bytes;  // STAGES tile + 2 code-stage barriers
+  static constexpr int bytes = bar_off + 8 * (STAGES + 2);
+  static constexpr int alloc = bytes + 1024;
+};
+
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float d;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// +1.0f or -1.0f carrying the sign bit of v
+__device__ __forceinline__ float sign_one(float v) {
+  return __uint_as_float((__float_as_uint(v) & 0x80000000u) | 0x3f800000u);
+}
+
+// mp[p][3i+j] = (M_{2p}[i][j], M_{2p+1}[i][j]) for the exact sandwich matrices;
+// the all-zero group 43 has a zero matrix.
+__device__ __forceinline__ void build_pair_table(const float* __restrict__ rotors, float2* __restrict__ mp) {
+  for (int g = threadIdx.x; g < 2 * NP; g += blockDim.x) {
+    float m[9];
+    if (g < G) {
+      const float4 r = __ldg(reinterpret_cast<const float4*>(rotors) + g);
+      rotor_matrix(r.x, r.y, r.z, r.w, m);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 9; ++k) m[k] = 0.f;
+    }
+    float* dst = reinterpret_cast<float*>(mp + (g >> 1) * 10) + (g & 1);
+#pragma unroll
+    for (int k = 0; k < 9; ++k) dst[2 * k] = m[k];
+    dst[18] = 0.f;
+  }
+}
+
+// sc[j] = -tau_{j+1} B (j < H-1), mag[j] = c[H+j], cf[k] = c[k]
+template <int BITS>
+__device__ __forceinline__ void build_consts(const float* __restrict__ centroids, float* sc, float* mag, float* cf) {
+  constexpr int K = 1 << BITS, H = K / 2;
+  const int t = threadIdx.x;
+  if (t < H) mag[t] = centroids[H + t];
+  if (t < H - 1) sc[t] = -(0.5f * (centroids[H + t] + centroids[H + 1 + t])) * kB;
+  if (t < K) cf[t] = centroids[t];
+}
+
+template <typename T, int BITS, int MODE, int STAGES>
+__global__ void __launch_bounds__(kRows, MODE == RQ_Q ? 2 : 4) rq_row_kernel(const __grid_constant__ CUtensorMap map_x,
+                                                       const __grid_constant__ CUtensorMap map_o, RqArgs a) {
+  using TL = Tile<T>;
+  using CD = Codes<BITS>;
+  using SM = Smem<T, BITS, MODE, STAGES>;
+  constexpr int H = CD::H, W = CD::W, CPW = CD::CPW, NWIN = CD::NWIN;
+  constexpr int E = TL::kE;
+  constexpr bool kIn = MODE != RQ_DQ;
+  constexpr bool kOut = MODE != RQ_Q;
+  constexpr bool kScale = !std::is_same<T, __half>::value;  // fp16 norms always lie in [2^-24, 2^20]
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* s_in = smem + SM::in_off;
-  uint8_t* s_out = smem + SM::out_off;
   uint32_t* s_codes = reinterpret_cast<uint32_t*>(smem + SM::codes_off);
   float* s_lut = reinterpret_cast<float*>(smem + SM::lut_off);
-  float4* s_m = reinterpret_cast<float4*>(smem + SM::mtab_off);
-  float* s_tau = reinterpret_cast<float*>(smem + SM::cb_off);
-  float* s_mag = s_tau + 16;
-  float* s_c = s_tau + 32;
-  uint64_t* s_bar = reinterpret_cast<uint64_t*>(smem + SM::bar_off);
+  const float4* s_mp4 = reinterpret_cast<const float4*>(smem + SM::mp_off);
+  float* s_sc = reinterpret_cast<float*>(smem + SM::cb_off);
+  float* s_mag = s_sc + 16;
+  float* s_cf = s_sc + 32;
+  uint64_t* s_bar = reinterpret_cast<uint64_t*>(smem + SM::bar_off);  // [0, STAGES) tiles, [STAGES + c] codes
 
   const int tid = threadIdx.x;
   const int64_t n = a.n;
-  const int64_t ntiles = (n + TL::kRows - 1) / TL::kRows;
+  const int64_t ntiles = (n + kRows - 1) / kRows;
+  // dequantize: a full tile of packed codes is one contiguous, 16-byte aligned block
+  const bool codes_bulk = !kIn && a.ldc == W && (reinterpret_cast<uintptr_t>(a.codes_in) & 15) == 0;
 
   if (tid == 0) {
-    if (SM::kIn) tma_prefetch_desc(&map_x);
-    if (SM::kOut) tma_prefetch_desc(&map_o);
-    for (int s = 0; s < S; ++s) mbar_init(&s_bar[s], 1);
+    if (kIn) tma_prefetch_desc(&map_x);
+    if (kOut) tma_prefetch_desc(&map_o);
+    for (int s = 0; s < STAGES + 2; ++s) mbar_init(&s_bar[s], 1);
     fence_barrier_init();
   }
-  build_rotor_table(a.rotors, G, s_m);
-  build_codebook<BITS>(a.centroids, s_tau, s_mag, s_c);
+  build_pair_table(a.rotors, reinterpret_cast<float2*>(smem + SM::mp_off));
+  build_consts<BITS>(a.centroids, s_sc, s_mag, s_cf);
   __syncthreads();
 
-  // loads issued into each stage (thread 0 only); the k-th load of a stage
-  // completes that stage barrier's phase with parity k & 1
-  uint32_t issued[S];
-#pragma unroll
-  for (int s = 0; s < S; ++s) issued[s] = 0;
-  auto issue_load = [&](int64_t tile, int s) {
-    ++issued[s];
+  // bit b of `par`: parity of the next phase of barrier b (all threads);
+  // bit b of `pend`: a copy completing on barrier b is in flight (thread 0)
+  uint32_t par = 0, pend = 0;
+
+  auto tile_of = [&](int iter) -> int64_t { return blockIdx.x + (int64_t)iter * gridDim.x; };
+  auto issue_tile = [&](int64_t tile, int s) {  // thread 0
+    pend |= 1u << s;
     mbar_arrive_expect_tx(&s_bar[s], TL::kTileBytes);
 #pragma unroll
     for (int b = 0; b < TL::kBoxes; ++b)
-      tma_load_2d(s_in + s * TL::kTileBytes + b * TL::kBoxBytes, &map_x, b * TL::kBoxElems,
-                  (int32_t)(tile * TL::kRows), &s_bar[s]);
+      tma_load_2d(smem + s * TL::kTileBytes + b * TL::kBoxBytes, &map_x, b * TL::kBoxElems, (int32_t)(tile * kRows),
+                  &s_bar[s]);
+  };
+  auto codes_bulk_tile = [&](int64_t tile) { return codes_bulk && (tile + 1) * kRows <= n; };
+  auto issue_codes = [&](int64_t tile, int c) {  // thread 0
+    pend |= 1u << (STAGES + c);
+    mbar_arrive_expect_tx(&s_bar[STAGES + c], kRows * W * 4);
+    bulk_load(s_codes + c * (SM::codes_stage / 4), a.codes_in + tile * kRows * W, kRows * W * 4, &s_bar[STAGES + c]);
   };
 
-  if (SM::kIn && tid == 0) {
-    for (int s = 0; s < S; ++s) {
-      const int64_t tile = blockIdx.x + (int64_t)s * gridDim.x;
-      if (tile < ntiles) issue_load(tile, s);
+  if (tid == 0) {
+    if (kIn) {
+      for (int s = 0; s < STAGES; ++s)
+        if (tile_of(s) < ntiles) issue_tile(tile_of(s), s);
+    } else {
+      for (int c = 0; c < 2; ++c)
+        if (tile_of(c) < ntiles && codes_bulk_tile(tile_of(c))) issue_codes(tile_of(c), c);
     }
   }
 
   int it = 0;
   for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
-    const int s = it % S;
-    const uint32_t phase = (uint32_t)((it / S) & 1);
-    const int64_t row0 = tile * TL::kRows;
-    const int rows = (int)(n - row0 < (int64_t)TL::kRows ? n - row0 : (int64_t)TL::kRows);
+    const int s = it % STAGES;
+    const int cs = it & 1;
+    const int64_t row0 = tile * kRows;
+    const int rows = (int)(n - row0 < (int64_t)kRows ? n - row0 : (int64_t)kRows);
     const int64_t row = row0 + tid;
+    uint8_t* tb = smem + s * TL::kTileBytes;
+    uint32_t* stage_codes = s_codes + cs * (SM::codes_stage / 4);
 
-    float x[D];
-    uint32_t wc[W];
-#pragma unroll
-    for (int w = 0; w < W; ++w) wc[w] = 0u;
-    float nrm = 0.f;
-
+    // ---------------------------------------------------------------- inputs
     bool ok = true;
-    if constexpr (SM::kIn) {
-      ok = mbar_wait(&s_bar[s], phase, a.status);  // a time-out is recorded in the status word
-      const uint8_t* sb = s_in + s * TL::kTileBytes;
-#pragma unroll
-      for (int j = 0; j < TL::kChunks; ++j) {
-        const uint4 v = *reinterpret_cast<const uint4*>(sb + TL::chunk_offset(tid, j));
-        Elem<T>::unpack(v, &x[j * TL::kE]);
-      }
+    if constexpr (kIn) {
+      ok = mbar_wait(&s_bar[s], (par >> s) & 1, a.status);
+      par ^= 1u << s;
+      pend &= ~(1u << s);
     } else {
-      // dequantize: gather this tile's packed codes (coalesced) into shared memory
-      for (int i = tid; i < rows * W; i += TL::kRows) {
-        const int r = i / W, w = i - r * W;
-        s_codes[i] = __ldg(a.codes_in + (row0 + r) * a.ldc + w);
+      if (codes_bulk_tile(tile)) {
+        ok = mbar_wait(&s_bar[STAGES + cs], (par >> (STAGES + cs)) & 1, a.status);
+        par ^= 1u << (STAGES + cs);
+        pend &= ~(1u << (STAGES + cs));
+      } else {
+        for (int i = tid; i < rows * W; i += kRows) {
+          const int r = i / W, w = i - r * W;
+          stage_codes[i] = __ldg(a.codes_in + (row0 + r) * a.ldc + w);
+        }
       }
-      nrm = tid < rows ? __ldg(a.norms_in + row) : 0.f;
+      if (tid == 0) bulk_wait_read<0>();  // earlier x_hat stores have left the tile buffers
     }
-
-    if (SM::kOut && tid == 0) bulk_wait_read<0>();  // previous x_hat store has left s_out
     if (!__syncthreads_and(ok)) {
-      // a load timed out: wait (bounded) for this CTA's other loads before leaving
-      if (SM::kIn && tid == 0)
-        for (int s2 = 0; s2 < S; ++s2)
-          if (issued[s2]) mbar_wait(&s_bar[s2], (issued[s2] - 1) & 1, a.status);
+      // a wait ran out: wait (bounded) for this CTA's other copies, then leave
+      if (tid == 0)
+        for (int b = 0; b < STAGES + 2; ++b)
+          if ((pend >> b) & 1) mbar_wait(&s_bar[b], (par >> b) & 1, a.status);
       break;
     }
-    if (SM::kIn && tid == 0) {
-      const int64_t next = tile + (int64_t)S * gridDim.x;
-      if (next < ntiles) issue_load(next, s);
-    }
 
-    Quantizer<BITS> q;
-    if constexpr (SM::kIn) {
-      float acc[8];
+    // ---------------------------------------------------------------- per-row scale
+    float xs = 1.f;  // power-of-two prescale of the row (fp32 / bf16 rows of extreme norm only)
+    float nrm, nq;   // ||x|| and ||xs x||
+    uint32_t wc[W];
+    if constexpr (kIn) {
+      float2 acc[4];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+      for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int i = 0; i < D; ++i) acc[i & 7] = fmaf(x[i], x[i], acc[i & 7]);
-      const float ss = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-      nrm = sqrtf(ss);
-      q.scale(s_tau, s_mag, nrm);
+      for (int j = 0; j < TL::kChunks; ++j) {
+        float f[E];
+        Elem<T>::unpack(*reinterpret_cast<const uint4*>(tb + TL::chunk(tid, j)), f);
+#pragma unroll
+        for (int k = 0; k < E / 2; ++k) {
+          const float2 v = make_float2(f[2 * k], f[2 * k + 1]);
+          acc[(j * (E / 2) + k) & 3] = __ffma2_rn(v, v, acc[(j * (E / 2) + k) & 3]);
+        }
+      }
+      float ss = ((acc[0].x + acc[1].x) + (acc[2].x + acc[3].x)) + ((acc[0].y + acc[1].y) + (acc[2].y + acc[3].y));
+      if (kScale && !(ss >= 0x1p-100f && ss <= 0x1p100f)) {
+        xs = ss < 1.f ? 0x1p100f : 0x1p-100f;
+        ss = 0.f;
+#pragma unroll 1
+        for (int j = 0; j < TL::kChunks; ++j) {
+          float f[E];
+          Elem<T>::unpack(*reinterpret_cast<const uint4*>(tb + TL::chunk(tid, j)), f);
+          for (int k = 0; k < E; ++k) ss = fmaf(f[k] * xs, f[k] * xs, ss);
+        }
+      }
+      nq = sqrtf(ss);
+      nrm = kScale ? nq / xs : nq;
     } else {
+      nrm = tid < rows ? __ldg(a.norms_in + row) : 0.f;
+      nq = nrm;
 #pragma unroll
-      for (int w = 0; w < W; ++w) wc[w] = s_codes[tid * W + w];
-#pragma unroll
-      for (int k = 0; k < K; ++k) s_lut[k * TL::kRows + tid] = s_c[k] * nrm;
+      for (int w = 0; w < W; ++w) wc[w] = stage_codes[tid * W + w];
     }
 
-    float xo[TL::kE];  // the output chunk being assembled
-    uint8_t* so = s_out;
+    // scaled magnitudes as a chain: chain(0) = mag_0 ||x||, chain(j) = chain(j-1) + delta_j
+    // (explicitly rounded products and differences: never contracted, so the
+    // fused and the dequantize-only kernels build bit-identical chains)
+    const float mn0 = __fmul_rn(s_mag[0], nrm);
+    float dl[H > 1 ? H - 1 : 1];
+    {
+      float prev = mn0;
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float4 m0 = s_m[3 * g], m1 = s_m[3 * g + 1], m2 = s_m[3 * g + 2];
-      const float m[9] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w, m2.x};
-      float c[3];
-      if constexpr (SM::kIn) {
-        float v[3];
+      for (int j = 1; j < H; ++j) {
+        const float cur = __fmul_rn(s_mag[j], nrm);
+        dl[j - 1] = __fsub_rn(cur, prev);
+        prev = cur;
+      }
+    }
+    if constexpr (!kIn) {
+      float ch = mn0;
 #pragma unroll
-        for (int i = 0; i < 3; ++i) v[i] = (3 * g + i < D) ? x[3 * g + i] : 0.f;
+      for (int j = 0; j < H; ++j) {
+        if (j > 0) ch = __fadd_rn(ch, dl[j - 1]);
+        s_lut[(H + j) * kRows + tid] = ch;
+        s_lut[(H - 1 - j) * kRows + tid] = -ch;
+      }
+    }
+    const float srow = nq > 0.f ? __fdiv_rn(kB, nq) : 0.f;
+    const float2 shift2 = make_float2(-kShift * nq, -kShift * nq);
+    float sc[H > 1 ? H - 1 : 1];
+#pragma unroll
+    for (int j = 0; j < H - 1; ++j) sc[j] = s_sc[j];
+
+    float win[NWIN];
+#pragma unroll
+    for (int w = 0; w < NWIN; ++w) win[w] = kWindow0;
+
+    // ---------------------------------------------------------------- pass 2
+    // One group pair (6 elements) at a time; a 16-byte chunk is read when the
+    // pair holding its first element comes up and written back after the pair
+    // holding its last element.
+    float xe[D + 6], xo[D];
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+      if constexpr (kIn) {
+#pragma unroll
+        for (int e = 6 * p; e < 6 * p + 6; ++e) {
+          if (e < D && e % E == 0) {
+            Elem<T>::unpack(*reinterpret_cast<const uint4*>(tb + TL::chunk(tid, e / E)), &xe[e]);
+            if constexpr (kScale) {
+#pragma unroll
+              for (int k = 0; k < E; ++k) xe[e + k] *= xs;
+            }
+          }
+          if (e >= D) xe[e] = 0.f;
+        }
+      }
+      float2 M[10];
+#pragma unroll
+      for (int q = 0; q < 5; ++q) {
+        const float4 t = s_mp4[p * 5 + q];
+        M[2 * q] = make_float2(t.x, t.y);
+        M[2 * q + 1] = make_float2(t.z, t.w);
+      }
+      float2 C[3];
+      if constexpr (kIn) {
+        float2 V[3];
+#pragma unroll
+        for (int j = 0; j < 3; ++j) V[j] = make_float2(xe[6 * p + j], xe[6 * p + 3 + j]);
 #pragma unroll
         for (int i = 0; i < 3; ++i) {
-          float y = m[3 * i] * v[0];
-          if (3 * g + 1 < D) y = fmaf(m[3 * i + 1], v[1], y);
-          if (3 * g + 2 < D) y = fmaf(m[3 * i + 2], v[2], y);
-          const uint32_t code = q(y, c[i]);
-          put_code<BITS, W>(wc, 3 * g + i, code);
+          const float2 Y = __ffma2_rn(M[3 * i + 2], V[2], __ffma2_rn(M[3 * i + 1], V[1], __ffma2_rn(M[3 * i], V[0], shift2)));
+          float2 m2 = make_float2(mn0, mn0);
+          float2 cnt = make_float2(0.5f, 0.5f);
+#pragma unroll
+          for (int j = 0; j < H - 1; ++j) {
+            const float2 st = make_float2(fma_sat(fabsf(Y.x), srow, sc[j]), fma_sat(fabsf(Y.y), srow, sc[j]));
+            m2 = __ffma2_rn(st, make_float2(dl[j], dl[j]), m2);
+            cnt = __fadd2_rn(cnt, st);
+          }
+          const float2 sg = make_float2(sign_one(Y.x), sign_one(Y.y));
+          C[i] = __fmul2_rn(m2, sg);
+          const float2 code = __ffma2_rn(sg, cnt, make_float2(H - 0.5f, H - 0.5f));
+          // codes of group 2p (lane x) and 2p + 1 (lane y) into their windows
+          const int kx = 3 * (2 * p) + i, ky = 3 * (2 * p + 1) + i;
+          win[kx / CPW] = fmaf(code.x, (float)(1u << (BITS * (kx % CPW))), win[kx / CPW]);
+          if (2 * p + 1 < G) win[ky / CPW] = fmaf(code.y, (float)(1u << (BITS * (ky % CPW))), win[ky / CPW]);
         }
       } else {
 #pragma unroll
-        for (int i = 0; i < 3; ++i) c[i] = s_lut[get_code<BITS, W>(wc, 3 * g + i) * TL::kRows + tid];
+        for (int i = 0; i < 3; ++i) {
+          const int kx = 3 * (2 * p) + i, ky = 3 * (2 * p + 1) + i;
+          const float cx = s_lut[get_code<BITS, W>(wc, kx) * kRows + tid];
+          const float cy = (2 * p + 1 < G) ? s_lut[get_code<BITS, W>(wc, ky) * kRows + tid] : 0.f;
+          C[i] = make_float2(cx, cy);
+        }
       }
-      if constexpr (SM::kOut) {
+      if constexpr (kOut) {
 #pragma unroll
         for (int i = 0; i < 3; ++i) {
-          const int e = 3 * g + i;
-          if (e < D) {
-            // inverse sandwich: column i of M, i.e. row i of M^T
-            const float o = fmaf(m[6 + i], c[2], fmaf(m[3 + i], c[1], m[i] * c[0]));
-            xo[e % TL::kE] = o;
-            if (e % TL::kE == TL::kE - 1) {
-              *reinterpret_cast<uint4*>(so + TL::chunk_offset(tid, e / TL::kE)) = Elem<T>::pack(xo);
-            }
-          }
+          const float2 X = __ffma2_rn(M[6 + i], C[2], __ffma2_rn(M[3 + i], C[1], __fmul2_rn(M[i], C[0])));
+          if (6 * p + i < D) xo[6 * p + i] = X.x;
+          if (6 * p + 3 + i < D) xo[6 * p + 3 + i] = X.y;
         }
+#pragma unroll
+        for (int e = 6 * p; e < 6 * p + 6; ++e)
+          if (e < D && e % E == E - 1)
+            *reinterpret_cast<uint4*>(tb + TL::chunk(tid, e / E)) = Elem<T>::pack(&xo[e - (E - 1)]);
       }
     }
 
-    if constexpr (SM::kIn) {
+    // ---------------------------------------------------------------- outputs
+    if constexpr (kIn) {
 #pragma unroll
-      for (int w = 0; w < W; ++w) s_codes[tid * W + w] = wc[w];
+      for (int w = 0; w < W; ++w) wc[w] = 0u;
+#pragma unroll
+      for (int w = 0; w < NWIN; ++w) {
+        const uint32_t v = __float_as_uint(win[w]) & 0x7fffffu;
+        const int bo = w * CPW * BITS;
+        wc[bo >> 5] |= v << (bo & 31);
+        if ((bo & 31) + CPW * BITS > 32 && (bo >> 5) + 1 < W) wc[(bo >> 5) + 1] |= v >> (32 - (bo & 31));
+      }
+#pragma unroll
+      for (int w = 0; w < W; ++w) stage_codes[tid * W + w] = wc[w];
       if (tid < rows && a.norms_out) a.norms_out[row] = nrm;
     }
-    if constexpr (SM::kOut) fence_proxy_async_smem();
+    if constexpr (kOut) fence_proxy_async_smem();
     __syncthreads();
-    if constexpr (SM::kOut) {
-      if (tid == 0) {
+    if (tid == 0) {
+      if constexpr (kOut) {
 #pragma unroll
-        for (int b = 0; b < TL::kBoxes; ++b)
-          tma_store_2d(&map_o, b * TL::kBoxElems, (int32_t)row0, s_out + b * TL::kBoxBytes);
+        for (int b = 0; b < TL::kBoxes; ++b) tma_store_2d(&map_o, b * TL::kBoxElems, (int32_t)row0, tb + b * TL::kBoxBytes);
         bulk_commit();
       }
-    }
-    if constexpr (SM::kIn) {
-      if (a.codes_out) {
-        for (int i = tid; i < rows * W; i += TL::kRows) {
-          const int r = i / W, w = i - r * W;
-          a.codes_out[(row0 + r) * a.ldc + w] = s_codes[i];
+      if constexpr (kIn) {
+        const int64_t next = tile_of(it + STAGES);
+        if (next < ntiles) {
+          if (kOut) bulk_wait_read<0>();  // the x_hat store has read this buffer
+          issue_tile(next, s);
         }
+      } else {
+        const int64_t next = tile_of(it + 2);
+        if (next < ntiles && codes_bulk_tile(next)) issue_codes(next, cs);
       }
     }
+    if constexpr (kIn) {
+      if (a.codes_out)
+        for (int i = tid; i < rows * W; i += kRows) {
+          const int r = i / W, w = i - r * W;
+          a.codes_out[(row0 + r) * a.ldc + w] = stage_codes[i];
+        }
+    }
   }
-  if (SM::kOut && tid == 0) bulk_wait_all<0>();
+  if (kOut && tid == 0) bulk_wait_all<0>();
 }
+
+}  // namespace row
+
+using row::rq_row_kernel;
+
 
 // ============================================================================
 // Any d, any stride: one warp per row.
@@ -451,24 +621,42 @@ __global__ void __launch_bounds__(256) rq_general_kernel(RqArgs a) {
 // ============================================================================
 // Launch helpers (host)
 // ============================================================================
-template <typename T, int BITS, int MODE>
-static cudaError_t launch_row(const CUtensorMap& mx, const CUtensorMap& mo, const RqArgs& a, cudaStream_t st,
-                              int num_sms) {
-  using SM = RowSmem<T, BITS, MODE>;
-  auto kern = rq_row_kernel<T, BITS, MODE>;
+template <typename T, int BITS, int MODE, int STAGES>
+static cudaError_t launch_row_s(const CUtensorMap& mx, const CUtensorMap& mo, const RqArgs& a, cudaStream_t st,
+                                int num_sms) {
+  using SM = row::Smem<T, BITS, MODE, STAGES>;
+  auto kern = rq_row_kernel<T, BITS, MODE, STAGES>;
   static int blocks_per_sm = -1;
   if (blocks_per_sm < 0) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::alloc);
     if (e != cudaSuccess) return e;
     int b = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, 128, SM::alloc);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, row::kRows, SM::alloc);
     if (e != cudaSuccess) return e;
     blocks_per_sm = b < 1 ? 1 : b;
   }
-  const int64_t ntiles = (a.n + 127) / 128;
+  const int64_t ntiles = (a.n + row::kRows - 1) / row::kRows;
   const int64_t grid = std::min<int64_t>(ntiles, (int64_t)num_sms * blocks_per_sm);
-  kern<<<(unsigned)grid, 128, SM::alloc, st>>>(mx, mo, a);
+  kern<<<(unsigned)grid, row::kRows, SM::alloc, st>>>(mx, mo, a);
   return cudaGetLastError();
+}
+
+// Tile buffers per CTA: 1 lets four CTAs share an SM (latency hidden across
+// CTAs), 2 double-buffers within a CTA. KVRQ_RQ_STAGES overrides the default.
+static int row_stages() {
+  static int stages = -1;
+  if (stages < 0) {
+    const char* e = getenv("KVRQ_RQ_STAGES");
+    stages = (e && atoi(e) == 2) ? 2 : 1;
+  }
+  return stages;
+}
+
+template <typename T, int BITS, int MODE>
+static cudaError_t launch_row(const CUtensorMap& mx, const CUtensorMap& mo, const RqArgs& a, cudaStream_t st,
+                              int num_sms) {
+  if (row_stages() == 1) return launch_row_s<T, BITS, MODE, 1>(mx, mo, a, st, num_sms);
+  return launch_row_s<T, BITS, MODE, 2>(mx, mo, a, st, num_sms);
 }
 
 template <typename TI, typename TO, int BITS, int MODE>
@@ -507,20 +695,6 @@ cudaError_t launch_rq_row(int mode, kvrq_dtype dt, int bits, const CUtensorMap& 
     case RQ_DQ: return row_by_type<RQ_DQ>(dt, bits, mx, mo, a, st, sms);
     default: return row_by_type<RQ_QDQ>(dt, bits, mx, mo, a, st, sms);
   }
-}
-
-size_t rq_row_smem_bytes(int mode, kvrq_dtype dt, int bits) {
-#define KVRQ_SM_CASE(T)                                                   \
-  switch (bits) {                                                         \
-    case 1: return mode == RQ_Q ? RowSmem<T, 1, RQ_Q>::alloc : mode == RQ_DQ ? RowSmem<T, 1, RQ_DQ>::alloc : RowSmem<T, 1, RQ_QDQ>::alloc; \
-    case 2: return mode == RQ_Q ? RowSmem<T, 2, RQ_Q>::alloc : mode == RQ_DQ ? RowSmem<T, 2, RQ_DQ>::alloc : RowSmem<T, 2, RQ_QDQ>::alloc; \
-    case 3: return mode == RQ_Q ? RowSmem<T, 3, RQ_Q>::alloc : mode == RQ_DQ ? RowSmem<T, 3, RQ_DQ>::alloc : RowSmem<T, 3, RQ_QDQ>::alloc; \
-    default: return mode == RQ_Q ? RowSmem<T, 4, RQ_Q>::alloc : mode == RQ_DQ ? RowSmem<T, 4, RQ_DQ>::alloc : RowSmem<T, 4, RQ_QDQ>::alloc; \
-  }
-  if (dt == KVRQ_F32) { KVRQ_SM_CASE(float) }
-  if (dt == KVRQ_F16) { KVRQ_SM_CASE(__half) }
-  KVRQ_SM_CASE(__nv_bfloat16)
-#undef KVRQ_SM_CASE
 }
 
 template <typename TI, typename TO, int MODE>

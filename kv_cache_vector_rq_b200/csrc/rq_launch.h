@@ -36,9 +36,6 @@ struct RqArgs {
 cudaError_t launch_rq_row(int mode, kvrq_dtype dt, int bits, const CUtensorMap& map_x, const CUtensorMap& map_o,
                           const RqArgs& a, cudaStream_t st, int num_sms);
 
-// Dynamic shared memory the row kernel requests.
-size_t rq_row_smem_bytes(int mode, kvrq_dtype dt, int bits);
-
 // Any d / stride, warp-per-row kernel.
 cudaError_t launch_rq_general(int mode, kvrq_dtype dt_in, kvrq_dtype dt_out, int bits, const RqArgs& a,
                               cudaStream_t st, int num_sms);
