@@ -128,6 +128,10 @@ __device__ __forceinline__ void build_codebook(const float* __restrict__ centroi
 // start at 2^23; the low 23 mantissa bits of each accumulator are a window
 // of the packed bit stream.
 // ============================================================================
+#ifndef KVRQ_ROW_MIN_BLOCKS
+#define KVRQ_ROW_MIN_BLOCKS 4  // CTAs per SM the register budget is sized for
+#endif
+
 namespace row {
 
 constexpr int D = 128;
@@ -220,7 +224,7 @@ __device__ __forceinline__ void build_consts(const float* __restrict__ centroids
 }
 
 template <typename T, int BITS, int MODE, int STAGES>
-__global__ void __launch_bounds__(kRows, MODE == RQ_Q ? 2 : 4) rq_row_kernel(const __grid_constant__ CUtensorMap map_x,
+__global__ void __launch_bounds__(kRows, MODE == RQ_Q ? 2 : KVRQ_ROW_MIN_BLOCKS) rq_row_kernel(const __grid_constant__ CUtensorMap map_x,
                                                        const __grid_constant__ CUtensorMap map_o, RqArgs a) {
   using TL = Tile<T>;
   using CD = Codes<BITS>;
@@ -300,6 +304,7 @@ __global__ void __launch_bounds__(kRows, MODE == RQ_Q ? 2 : 4) rq_row_kernel(con
     // ---------------------------------------------------------------- inputs
     bool ok = true;
     if constexpr (kIn) {
+      if (tid == 0) bulk_wait_read<1>();  // the codes store from this staging buffer (two tiles ago) is done
       ok = mbar_wait(&s_bar[s], (par >> s) & 1, a.status);
       par ^= 1u << s;
       pend &= ~(1u << s);
@@ -394,6 +399,10 @@ __global__ void __launch_bounds__(kRows, MODE == RQ_Q ? 2 : 4) rq_row_kernel(con
     float win[NWIN];
 #pragma unroll
     for (int w = 0; w < NWIN; ++w) win[w] = kWindow0;
+    if constexpr (kIn) {
+#pragma unroll
+      for (int w = 0; w < W; ++w) wc[w] = 0u;
+    }
 
     // ---------------------------------------------------------------- pass 2
     // One group pair (6 elements) at a time; a 16-byte chunk is read when the
@@ -446,6 +455,26 @@ __global__ void __launch_bounds__(kRows, MODE == RQ_Q ? 2 : 4) rq_row_kernel(con
           win[kx / CPW] = fmaf(code.x, (float)(1u << (BITS * (kx % CPW))), win[kx / CPW]);
           if (2 * p + 1 < G) win[ky / CPW] = fmaf(code.y, (float)(1u << (BITS * (ky % CPW))), win[ky / CPW]);
         }
+        // windows whose codes are all in, and the words they complete, leave the registers now
+        const int done = 6 * (p + 1) < NC ? 6 * (p + 1) : NC;  // codes 0 .. done-1 are packed
+#pragma unroll
+        for (int w = 0; w < NWIN; ++w) {
+          const int last = (w + 1) * CPW < NC ? (w + 1) * CPW : NC;  // one past the window's last code
+          if (last <= done && last > 6 * p) {
+            const uint32_t v = __float_as_uint(win[w]) & 0x7fffffu;
+            const int bo = w * CPW * BITS;
+            wc[bo >> 5] |= v << (bo & 31);
+            if ((bo & 31) + CPW * BITS > 32 && (bo >> 5) + 1 < W) wc[(bo >> 5) + 1] |= v >> (32 - (bo & 31));
+          }
+        }
+#pragma unroll
+        for (int wi = 0; wi < W; ++wi) {
+          // word wi is final once every code overlapping it is packed
+          const int last_code = ((32 * wi + 31) / BITS) < NC ? (32 * wi + 31) / BITS : NC - 1;
+          const int win_end = ((last_code / CPW) + 1) * CPW < NC ? ((last_code / CPW) + 1) * CPW : NC;
+          const int prev_done = 6 * p < NC ? 6 * p : NC;
+          if (win_end <= done && win_end > prev_done) stage_codes[tid * W + wi] = wc[wi];
+        }
       } else {
 #pragma unroll
         for (int i = 0; i < 3; ++i) {
@@ -471,27 +500,20 @@ __global__ void __launch_bounds__(kRows, MODE == RQ_Q ? 2 : 4) rq_row_kernel(con
 
     // ---------------------------------------------------------------- outputs
     if constexpr (kIn) {
-#pragma unroll
-      for (int w = 0; w < W; ++w) wc[w] = 0u;
-#pragma unroll
-      for (int w = 0; w < NWIN; ++w) {
-        const uint32_t v = __float_as_uint(win[w]) & 0x7fffffu;
-        const int bo = w * CPW * BITS;
-        wc[bo >> 5] |= v << (bo & 31);
-        if ((bo & 31) + CPW * BITS > 32 && (bo >> 5) + 1 < W) wc[(bo >> 5) + 1] |= v >> (32 - (bo & 31));
-      }
-#pragma unroll
-      for (int w = 0; w < W; ++w) stage_codes[tid * W + w] = wc[w];
       if (tid < rows && a.norms_out) a.norms_out[row] = nrm;
     }
-    if constexpr (kOut) fence_proxy_async_smem();
+    // a full tile of codes leaves as one bulk copy when code rows are contiguous
+    const bool codes_bulk_out = kIn && a.codes_out && rows == kRows && a.ldc == W &&
+                                (reinterpret_cast<uintptr_t>(a.codes_out) & 15) == 0;
+    fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
       if constexpr (kOut) {
 #pragma unroll
         for (int b = 0; b < TL::kBoxes; ++b) tma_store_2d(&map_o, b * TL::kBoxElems, (int32_t)row0, tb + b * TL::kBoxBytes);
-        bulk_commit();
       }
+      if (codes_bulk_out) bulk_store(a.codes_out + row0 * W, stage_codes, kRows * W * 4);
+      if (kOut || codes_bulk_out) bulk_commit();
       if constexpr (kIn) {
         const int64_t next = tile_of(it + STAGES);
         if (next < ntiles) {
@@ -504,14 +526,14 @@ __global__ void __launch_bounds__(kRows, MODE == RQ_Q ? 2 : 4) rq_row_kernel(con
       }
     }
     if constexpr (kIn) {
-      if (a.codes_out)
+      if (a.codes_out && !codes_bulk_out)
         for (int i = tid; i < rows * W; i += kRows) {
           const int r = i / W, w = i - r * W;
           a.codes_out[(row0 + r) * a.ldc + w] = stage_codes[i];
         }
     }
   }
-  if (kOut && tid == 0) bulk_wait_all<0>();
+  if (tid == 0) bulk_wait_all<0>();
 }
 
 }  // namespace row
