@@ -151,6 +151,45 @@ kvrq_status rq_quantize_dequantize(void* stream, const void* x, kvrq_dtype xdtyp
                                    int64_t ldx, const float* rotors, const float* centroids, int bits,
                                    uint32_t* codes, int64_t ldc, float* norms, void* xhat, int64_t ldo);
 
+
+/* ================================================================ TurboQuant
+ * [TQA "方法" Algorithm 1; TQB "随机旋转（Lemma 1）"]: u = x/||x||, y = Pi u,
+ * each y_i replaced by its nearest Lloyd-Max centroid (codebook for d, ties to
+ * the lower index), codes packed; dequantize x_hat = ||x|| Pi^T c_hat.
+ * [TQA Algorithm 2; TQB "QJL 内积无偏估计（Theorem 2）"; RQ "How TurboQuant
+ * Works"] (prod, b bits): (b-1)-bit codes as above, rotated residual
+ * r = y - c_hat, gamma = ||r||, signs s = sign(T (256 r)) with the operand
+ * rounded to fp16 (S = T Pi is the pages' Gaussian projection; sign(0) = +1),
+ * x_hat = ||x|| Pi^T (c_hat + sqrt(pi/2)/m gamma T^T s).
+ *
+ * Tensor-core path: d = m = 128; x (and x_hat) fp16 or bf16 with Pi [d][d]
+ * row-major in the same type; T [m][d] row-major fp16; all 16-byte aligned;
+ * rows of x/x_hat 16-byte aligned. centroids: [2^b] (mse) or [2^(b-1)] (prod)
+ * fp32, ascending and symmetric. codes [n][ldc] uint32 with
+ * ldc >= kvrq_packed_words(d, b or b-1); signs [n][lds] uint32, lds >= m/32;
+ * norms, gammas [n] fp32. Other shapes return KVRQ_EUNSUPPORTED.
+ */
+kvrq_status tq_quantize_mse(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,
+                            const void* pi, const float* centroids, int bits, uint32_t* codes, int64_t ldc,
+                            float* norms);
+
+/* Fused quantize + dequantize (codes and norms may be NULL): one launch, two MMAs per tile. */
+kvrq_status tq_quantize_dequantize_mse(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,
+                                       const void* pi, const float* centroids, int bits, uint32_t* codes,
+                                       int64_t ldc, float* norms, void* xhat, int64_t ldo);
+
+/* TurboQuant-prod quantize, b = bits in 2..5 total bits per coordinate. */
+kvrq_status tq_quantize_prod(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,
+                             const void* pi, const uint16_t* T, int m, const float* centroids, int bits,
+                             uint32_t* codes, int64_t ldc, uint32_t* signs, int64_t lds, float* gammas,
+                             float* norms);
+
+/* Dequantize mse (signs == NULL; bits = b) or prod (signs != NULL; bits = b total). */
+kvrq_status tq_dequantize(void* stream, const uint32_t* codes, int64_t ldc, const uint32_t* signs, int64_t lds,
+                          const float* gammas, const float* norms, int64_t n, int d, int m, int bits,
+                          const void* pi, const uint16_t* T, const float* centroids, void* xhat, kvrq_dtype odtype,
+                          int64_t ldo);
+
 #ifdef __cplusplus
 }
 #endif

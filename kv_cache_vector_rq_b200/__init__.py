@@ -177,3 +177,86 @@ def rq_quantize_dequantize(x, rotors, centroids, bits, codes=None, norms=None, x
 def device_status(stream=None):
     """Raise if a bounded device-side wait ran out since the last check (synchronises the stream)."""
     _lib.check("kvrq_device_status", lib().kvrq_device_status(_stream(stream)))
+
+
+# ----------------------------------------------------------------------------- TurboQuant
+
+def _tq_outputs(x_rows, d, cbits, device, codes, norms):
+    torch = _torch()
+    W = packed_words(d, cbits)
+    if codes is None:
+        codes = torch.empty((x_rows, W), dtype=torch.int32, device=device)
+    if norms is None:
+        norms = torch.empty((x_rows,), dtype=torch.float32, device=device)
+    return codes, norms
+
+
+def tq_quantize_mse(x, pi, centroids, bits, codes=None, norms=None, stream=None):
+    """TurboQuant-mse quantize rows of x [n, d]; pi [d, d] in x's dtype. Returns (codes, norms)."""
+    torch = _torch()
+    n, d = x.shape
+    codes, norms = _tq_outputs(n, d, bits, x.device, codes, norms)
+    xp, ldx = _rows(x, "x")
+    cp, ldc = _rows(codes, "codes")
+    _lib.check("tq_quantize_mse", lib().tq_quantize_mse(_stream(stream), xp, _dtype_code(x), n, d, ldx,
+                                                        _ptr(pi, "pi", x.dtype),
+                                                        _ptr(centroids, "centroids", torch.float32), bits, cp, ldc,
+                                                        _ptr(norms, "norms", torch.float32)))
+    return codes, norms
+
+
+def tq_quantize_dequantize_mse(x, pi, centroids, bits, codes=None, norms=None, xhat=None, with_codes=True,
+                               stream=None):
+    """Fused TurboQuant-mse roundtrip: returns (codes, norms, x_hat)."""
+    torch = _torch()
+    n, d = x.shape
+    if with_codes:
+        codes, norms = _tq_outputs(n, d, bits, x.device, codes, norms)
+    if xhat is None:
+        xhat = torch.empty_like(x)
+    xp, ldx = _rows(x, "x")
+    cp, ldc = _rows(codes, "codes") if codes is not None else (None, packed_words(d, bits))
+    op, ldo = _rows(xhat, "xhat")
+    _lib.check("tq_quantize_dequantize_mse", lib().tq_quantize_dequantize_mse(
+        _stream(stream), xp, _dtype_code(x), n, d, ldx, _ptr(pi, "pi", x.dtype),
+        _ptr(centroids, "centroids", torch.float32), bits, cp, ldc, _ptr(norms, "norms", torch.float32), op, ldo))
+    return codes, norms, xhat
+
+
+def tq_quantize_prod(x, pi, T, centroids, bits, codes=None, norms=None, signs=None, gammas=None, stream=None):
+    """TurboQuant-prod quantize (bits total: bits-1 mse bits + 1 QJL bit); T [m, d] fp16.
+    Returns (codes, signs, gammas, norms)."""
+    torch = _torch()
+    n, d = x.shape
+    m = T.shape[0]
+    codes, norms = _tq_outputs(n, d, bits - 1, x.device, codes, norms)
+    if signs is None:
+        signs = torch.empty((n, m // 32), dtype=torch.int32, device=x.device)
+    if gammas is None:
+        gammas = torch.empty((n,), dtype=torch.float32, device=x.device)
+    xp, ldx = _rows(x, "x")
+    cp, ldc = _rows(codes, "codes")
+    sp, lds = _rows(signs, "signs")
+    _lib.check("tq_quantize_prod", lib().tq_quantize_prod(
+        _stream(stream), xp, _dtype_code(x), n, d, ldx, _ptr(pi, "pi", x.dtype), _ptr(T, "T", torch.float16), m,
+        _ptr(centroids, "centroids", torch.float32), bits, cp, ldc, sp, lds, _ptr(gammas, "gammas", torch.float32),
+        _ptr(norms, "norms", torch.float32)))
+    return codes, signs, gammas, norms
+
+
+def tq_dequantize(codes, norms, d, pi, centroids, bits, signs=None, gammas=None, T=None, xhat=None, stream=None):
+    """TurboQuant dequantize: mse when signs is None, prod otherwise (bits = total bits).
+    The output dtype is pi's dtype."""
+    torch = _torch()
+    n = codes.shape[0]
+    if xhat is None:
+        xhat = torch.empty((n, d), dtype=pi.dtype, device=codes.device)
+    m = T.shape[0] if T is not None else d
+    cp, ldc = _rows(codes, "codes")
+    sp, lds = _rows(signs, "signs") if signs is not None else (None, 0)
+    op, ldo = _rows(xhat, "xhat")
+    _lib.check("tq_dequantize", lib().tq_dequantize(
+        _stream(stream), cp, ldc, sp, lds, _ptr(gammas, "gammas", torch.float32), _ptr(norms, "norms", torch.float32),
+        n, d, m, bits, _ptr(pi, "pi", xhat.dtype), _ptr(T, "T", torch.float16),
+        _ptr(centroids, "centroids", torch.float32), op, _dtype_code(xhat), ldo))
+    return xhat

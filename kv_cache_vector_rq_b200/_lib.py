@@ -34,6 +34,17 @@ SIGNATURES = {
     # stream, x, xdtype, n, d, ldx, rotors, centroids, bits, codes, ldc, norms, xhat, ldo
     "rq_quantize_dequantize": (c_int, [c_vp, c_vp, c_int, c_i64, c_int, c_i64, c_vp, c_vp, c_int, c_vp, c_i64, c_vp,
                                        c_vp, c_i64]),
+    # stream, x, xdtype, n, d, ldx, pi, centroids, bits, codes, ldc, norms
+    "tq_quantize_mse": (c_int, [c_vp, c_vp, c_int, c_i64, c_int, c_i64, c_vp, c_vp, c_int, c_vp, c_i64, c_vp]),
+    # ... + xhat, ldo
+    "tq_quantize_dequantize_mse": (c_int, [c_vp, c_vp, c_int, c_i64, c_int, c_i64, c_vp, c_vp, c_int, c_vp, c_i64,
+                                           c_vp, c_vp, c_i64]),
+    # stream, x, xdtype, n, d, ldx, pi, T, m, centroids, bits, codes, ldc, signs, lds, gammas, norms
+    "tq_quantize_prod": (c_int, [c_vp, c_vp, c_int, c_i64, c_int, c_i64, c_vp, c_vp, c_int, c_vp, c_int, c_vp, c_i64,
+                                 c_vp, c_i64, c_vp, c_vp]),
+    # stream, codes, ldc, signs, lds, gammas, norms, n, d, m, bits, pi, T, centroids, xhat, odtype, ldo
+    "tq_dequantize": (c_int, [c_vp, c_vp, c_i64, c_vp, c_i64, c_vp, c_vp, c_i64, c_int, c_int, c_int, c_vp, c_vp,
+                              c_vp, c_vp, c_int, c_i64]),
 }
 
 _lib = None

@@ -13,6 +13,7 @@
 #include "kvrq.h"
 #include "kvrq_internal.h"
 #include "rq_launch.h"
+#include "tq_launch.h"
 
 namespace kvrq {
 
@@ -204,6 +205,77 @@ static kvrq_status rq_call(const char* name, int mode, void* stream, const void*
   return launch_status(name, launch_rq_general(mode, xdt, odt, bits, a, s, di->num_sms));
 }
 
+
+// Shared validation and dispatch of the TurboQuant calls (tensor-core path:
+// d = m = 128, 16-bit x and Pi of the same type, fp16 T, 16-byte aligned rows).
+static kvrq_status tq_call(const char* name, int mode, void* stream, const void* x, kvrq_dtype dt, int64_t ldx,
+                           int64_t n, int d, int m, const void* pi, const uint16_t* T, const float* centroids,
+                           int bits, uint32_t* codes_out, const uint32_t* codes_in, int64_t ldc, uint32_t* signs_out,
+                           const uint32_t* signs_in, int64_t lds, float* gammas_out, const float* gammas_in,
+                           float* norms_out, const float* norms_in, void* xhat, int64_t ldo) {
+  const bool prod = mode == TQ_PROD_Q || mode == TQ_DQ_PROD;
+  const bool q_side = mode == TQ_MSE_Q || mode == TQ_MSE_QDQ || mode == TQ_PROD_Q;
+  const bool out = mode == TQ_MSE_QDQ || mode == TQ_DQ_MSE || mode == TQ_DQ_PROD;
+  if (n < 0) return set_errorf(KVRQ_EINVAL, "%s: n < 0", name);
+  if (d < 2) return set_errorf(KVRQ_EINVAL, "%s: d must be >= 2", name);
+  if (!valid_dtype(dt)) return set_errorf(KVRQ_EINVAL, "%s: bad dtype", name);
+  if (prod ? (bits < 2 || bits > 5) : (bits < 1 || bits > 4))
+    return set_errorf(KVRQ_EUNSUPPORTED, "%s: bits must be in %s", name, prod ? "2..5" : "1..4");
+  if (d != 128) return set_errorf(KVRQ_EUNSUPPORTED, "%s: the tensor-core path supports d = 128", name);
+  if (prod && m != d) return set_errorf(KVRQ_EUNSUPPORTED, "%s: the QJL projection needs m = d", name);
+  if (dt == KVRQ_F32) return set_errorf(KVRQ_EUNSUPPORTED, "%s: fp32 vectors are not supported here", name);
+  const int cbits = prod ? bits - 1 : bits;
+  const int64_t W = kvrq_packed_words(d, cbits);
+  if (n == 0) return KVRQ_OK;
+  if (!pi || !centroids || (prod && !T)) return set_errorf(KVRQ_EINVAL, "%s: pi, centroids (and T) are required", name);
+  if (!aligned(pi, 16) || (T && !aligned(T, 16)) || !aligned(centroids, 4))
+    return set_errorf(KVRQ_EINVAL, "%s: pi and T must be 16-byte aligned", name);
+  if (q_side) {
+    if (!x || ldx < d || !rows_aligned16(x, ldx, dt)) return set_errorf(KVRQ_EINVAL, "%s: x NULL, ldx < d or rows not 16-byte aligned", name);
+    if (mode != TQ_MSE_QDQ && (!codes_out || !norms_out)) return set_errorf(KVRQ_EINVAL, "%s: codes and norms are required", name);
+    if (codes_out && (ldc < W || !aligned(codes_out, 4))) return set_errorf(KVRQ_EINVAL, "%s: ldc < packed words", name);
+    if (prod && (!signs_out || !gammas_out || lds < m / 32 || !aligned(signs_out, 4)))
+      return set_errorf(KVRQ_EINVAL, "%s: signs (lds >= m/32) and gammas are required", name);
+  } else {
+    if (!codes_in || !norms_in || ldc < W) return set_errorf(KVRQ_EINVAL, "%s: codes, norms (ldc >= packed words) are required", name);
+    if (prod && (!signs_in || !gammas_in || lds < m / 32)) return set_errorf(KVRQ_EINVAL, "%s: signs and gammas are required", name);
+  }
+  if (out && (!xhat || ldo < d || !rows_aligned16(xhat, ldo, dt)))
+    return set_errorf(KVRQ_EINVAL, "%s: xhat NULL, ldo < d or rows not 16-byte aligned", name);
+  if (n > ((int64_t)1 << 31) - 256) return set_errorf(KVRQ_EUNSUPPORTED, "%s: n >= 2^31", name);
+
+  DeviceInfo* di;
+  kvrq_status st = current_device(&di);
+  if (st != KVRQ_OK) return st;
+  CUtensorMap mx, mp, mt, mo;
+  memset(&mx, 0, sizeof(mx));
+  memset(&mp, 0, sizeof(mp));
+  memset(&mt, 0, sizeof(mt));
+  memset(&mo, 0, sizeof(mo));
+  if ((st = encode_rows_map(&mp, pi, dt, d, d, d, 128)) != KVRQ_OK) return st;
+  if (prod && (st = encode_rows_map(&mt, T, KVRQ_F16, m, d, d, 128)) != KVRQ_OK) return st;
+  if (q_side && (st = encode_rows_map(&mx, x, dt, n, d, ldx, 128)) != KVRQ_OK) return st;
+  if (out && (st = encode_rows_map(&mo, xhat, dt, n, d, ldo, 128)) != KVRQ_OK) return st;
+  TqArgs a{};
+  a.n = n;
+  a.d = d;
+  a.centroids = centroids;
+  a.qjl_scale = (float)(1.2533141373155003 / (double)m);  // sqrt(pi/2) / m
+  a.ldx = ldx;
+  a.codes_out = codes_out;
+  a.norms_out = norms_out;
+  a.signs_out = signs_out;
+  a.gammas_out = gammas_out;
+  a.codes_in = codes_in;
+  a.norms_in = norms_in;
+  a.signs_in = signs_in;
+  a.gammas_in = gammas_in;
+  a.ldc = ldc;
+  a.lds = lds;
+  a.status = di->status;
+  return launch_status(name, launch_tq(mode, dt, cbits, mx, mp, mt, mo, a, static_cast<cudaStream_t>(stream), di->num_sms));
+}
+
 }  // namespace kvrq
 
 using namespace kvrq;
@@ -245,6 +317,37 @@ kvrq_status rq_quantize_dequantize(void* stream, const void* x, kvrq_dtype xdtyp
                                    int64_t ldc, float* norms, void* xhat, int64_t ldo) {
   return rq_call("rq_quantize_dequantize", RQ_QDQ, stream, x, xdtype, ldx, nullptr, codes, ldc, nullptr, norms, n, d,
                  rotors, centroids, bits, xhat, xdtype, ldo);
+}
+
+kvrq_status tq_quantize_mse(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,
+                            const void* pi, const float* centroids, int bits, uint32_t* codes, int64_t ldc,
+                            float* norms) {
+  return tq_call("tq_quantize_mse", TQ_MSE_Q, stream, x, xdtype, ldx, n, d, d, pi, nullptr, centroids, bits, codes,
+                 nullptr, ldc, nullptr, nullptr, 0, nullptr, nullptr, norms, nullptr, nullptr, 0);
+}
+
+kvrq_status tq_quantize_dequantize_mse(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,
+                                       const void* pi, const float* centroids, int bits, uint32_t* codes,
+                                       int64_t ldc, float* norms, void* xhat, int64_t ldo) {
+  return tq_call("tq_quantize_dequantize_mse", TQ_MSE_QDQ, stream, x, xdtype, ldx, n, d, d, pi, nullptr, centroids,
+                 bits, codes, nullptr, ldc, nullptr, nullptr, 0, nullptr, nullptr, norms, nullptr, xhat, ldo);
+}
+
+kvrq_status tq_quantize_prod(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,
+                             const void* pi, const uint16_t* T, int m, const float* centroids, int bits,
+                             uint32_t* codes, int64_t ldc, uint32_t* signs, int64_t lds, float* gammas,
+                             float* norms) {
+  return tq_call("tq_quantize_prod", TQ_PROD_Q, stream, x, xdtype, ldx, n, d, m, pi, T, centroids, bits, codes,
+                 nullptr, ldc, signs, nullptr, lds, gammas, nullptr, norms, nullptr, nullptr, 0);
+}
+
+kvrq_status tq_dequantize(void* stream, const uint32_t* codes, int64_t ldc, const uint32_t* signs, int64_t lds,
+                          const float* gammas, const float* norms, int64_t n, int d, int m, int bits,
+                          const void* pi, const uint16_t* T, const float* centroids, void* xhat, kvrq_dtype odtype,
+                          int64_t ldo) {
+  const int mode = signs ? TQ_DQ_PROD : TQ_DQ_MSE;
+  return tq_call("tq_dequantize", mode, stream, nullptr, odtype, 0, n, d, m, pi, T, centroids, bits, nullptr, codes,
+                 ldc, nullptr, signs, lds, nullptr, gammas, nullptr, norms, xhat, ldo);
 }
 
 }  // extern "C"

@@ -183,17 +183,6 @@ struct Smem {
   static constexpr int alloc = bytes + 1024;
 };
 
-__device__ __forceinline__ float fma_sat(float a, float b, float c) {
-  float d;
-  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
-
-// +1.0f or -1.0f carrying the sign bit of v
-__device__ __forceinline__ float sign_one(float v) {
-  return __uint_as_float((__float_as_uint(v) & 0x80000000u) | 0x3f800000u);
-}
-
 // mp[p][3i+j] = (M_{2p}[i][j], M_{2p+1}[i][j]) for the exact sandwich matrices;
 // the all-zero group 43 has a zero matrix.
 __device__ __forceinline__ void build_pair_table(const float* __restrict__ rotors, float2* __restrict__ mp) {
@@ -391,7 +380,9 @@ __global__ void __launch_bounds__(kRows, MODE == RQ_Q ? 2 : KVRQ_ROW_MIN_BLOCKS)
       }
     }
     const float srow = nq > 0.f ? __fdiv_rn(kB, nq) : 0.f;
-    const float2 shift2 = make_float2(-kShift * nq, -kShift * nq);
+    // y' = y - (2^-30 ||x|| + 2^-126): an exact zero (also of a zero row) becomes negative
+    const float shv = -fmaf(kShift, nq, 0x1p-126f);
+    const float2 shift2 = make_float2(shv, shv);
     float sc[H > 1 ? H - 1 : 1];
 #pragma unroll
     for (int j = 0; j < H - 1; ++j) sc[j] = s_sc[j];

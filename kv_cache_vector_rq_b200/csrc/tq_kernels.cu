@@ -1,0 +1,492 @@
+// TurboQuant kernels for sm_100a: dense rotation and QJL projection on the
+// 5th-generation tensor cores (tcgen05.mma, accumulators in TMEM).
+//
+// Method (arXiv 2504.19874 summary page, "方法", Algorithms 1 and 2;
+// "TurboQuant 论文解读", "随机旋转（Lemma 1）" and "QJL 内积无偏估计（Theorem 2）";
+// "TurboQuant + RotorQuant", "How TurboQuant Works"):
+//   u = x / ||x||, y = Pi u, code_i = nearest Lloyd-Max centroid of y_i,
+//   x_hat = ||x|| Pi^T c_hat                                          (mse)
+//   (b-1)-bit mse codes, r = y - c_hat (rotated residual), gamma = ||r||,
+//   s = sign(T r) with S = T Pi, x_hat = ||x|| Pi^T (c_hat + sqrt(pi/2)/m gamma T^T s)   (prod)
+//
+// B200 design. A persistent CTA of 128 threads owns 128-row tiles; Pi (and T)
+// stay resident in shared memory as 128-byte-swizzled tiles that serve as the
+// MMA B operand both K-major (y = Pi u, T r) and MN-major (Pi^T c, T^T s).
+// The x tile arrives by TMA in the same swizzled layout and is the A operand
+// directly. One thread issues tcgen05.mma (M = 128, N = d, K = 16 steps) into
+// TMEM; every thread then reads its own row (one TMEM lane) with tcgen05.ld,
+// quantizes on the FMA pipe, and writes the next A operand (centroids, or the
+// residual for the sketch) back into the same tile buffer, which finally holds
+// x_hat for the TMA store. Two CTAs share an SM (256 TMEM columns each) so one
+// CTA's MMAs overlap the other's epilogue.
+
+#include <cuda_runtime.h>
+
+#include <cstdlib>
+#include <type_traits>
+
+#include "kvrq_device.cuh"
+#include "tq_launch.h"
+
+namespace kvrq {
+namespace tq {
+
+constexpr int kRows = 128;
+constexpr int D = 128;                            // head dimension handled by this kernel (= m)
+constexpr int kBoxBytes = kRows * 128;            // one 64-column box of 128 rows
+constexpr int kTileBytes = 2 * kBoxBytes;         // 128 x 128 16-bit elements
+constexpr float kShift = 9.313225746154785e-10f;  // 2^-30
+constexpr float kWindow0 = 8388608.0f;            // 2^23
+constexpr float kSketchScale = 256.0f;            // residual scale before rounding to fp16
+
+template <int BITS>
+struct Codes {
+  static constexpr int K = 1 << BITS;
+  static constexpr int H = K / 2;
+  static constexpr int NC = D;
+  static constexpr int W = (NC * BITS + 31) / 32;
+  static constexpr int CPW = 23 / BITS;
+  static constexpr int NWIN = (NC + CPW - 1) / CPW;
+};
+
+template <int BITS, int MODE>
+struct Smem {
+  static constexpr bool kT = MODE == TQ_PROD_Q || MODE == TQ_DQ_PROD;
+  static constexpr int W = Codes<BITS>::W;
+  static constexpr int tile_off = 0;
+  static constexpr int pi_off = kTileBytes;
+  static constexpr int t_off = pi_off + kTileBytes;
+  static constexpr int codes_off = t_off + (kT ? kTileBytes : 0);  // [kRows][W]
+  static constexpr int signs_off = codes_off + ((kRows * W * 4 + 15) / 16) * 16;  // [kRows][D/32]
+  static constexpr int cb_off = signs_off + kRows * (D / 32) * 4;
+  static constexpr int bar_off = cb_off + 64 * 4;  // x, params, mma
+  static constexpr int tmem_off = bar_off + 3 * 8;
+  static constexpr int bytes = tmem_off + 16;
+  // at least 80 KB so that at most two CTAs (2 x 256 TMEM columns) share an SM
+  static constexpr int alloc = (bytes + 1024) < 80 * 1024 ? 80 * 1024 : bytes + 1024;
+};
+
+// Positive-side quantizer constants (see rq_kernels.cu for the construction):
+// sc[j] = -tau_{j+1} * B, chain of unit centroids c[H] + sum step_j * dl[j].
+template <int BITS>
+__device__ __forceinline__ void build_consts(const float* __restrict__ centroids, float* sc, float* mag, float* cf,
+                                             float* bscale) {
+  constexpr int K = 1 << BITS, H = K / 2;
+  const int t = threadIdx.x;
+  // B = 2^(48 - floor(log2 tau_min)) keeps every step exactly 0 or 1
+  float tau_min = 1.f;
+  if (H > 1) tau_min = 0.5f * (centroids[H] + centroids[H + 1]);
+  const int e = (int)((__float_as_uint(tau_min) >> 23) & 0xFF) - 127;
+  const float B = __uint_as_float((uint32_t)(127 + 48 - e) << 23);  // exactly 2^(48 - e)
+  if (t == 0) *bscale = B;
+  if (t < H) mag[t] = centroids[H + t];
+  if (t < H - 1) sc[t] = -(0.5f * (centroids[H + t] + centroids[H + 1 + t])) * B;
+  // centroid table as the quantizer builds it: c[H + j] = c[H] + (c[H+1] - c[H]) + ... (rounded
+  // step by step), c[H - 1 - j] = -c[H + j]; so quantize-then-dequantize equals the fused path
+  if (t == 0) {
+    float ch = centroids[H];
+    for (int j = 0; j < H; ++j) {
+      if (j > 0) ch = __fadd_rn(ch, __fsub_rn(centroids[H + j], centroids[H + j - 1]));
+      cf[H + j] = ch;
+      cf[H - 1 - j] = -ch;
+    }
+  }
+}
+
+template <typename T>
+struct IsBf16 {
+  static constexpr bool value = std::is_same<T, __nv_bfloat16>::value;
+};
+
+template <typename T, int BITS, int MODE>
+__global__ void __launch_bounds__(kRows, 1)
+    tq_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_pi,
+              const __grid_constant__ CUtensorMap map_t, const __grid_constant__ CUtensorMap map_o, TqArgs a) {
+  using CD = Codes<BITS>;
+  using SM = Smem<BITS, MODE>;
+  constexpr int H = CD::H, W = CD::W, CPW = CD::CPW, NWIN = CD::NWIN;
+  constexpr int NS = D / 32;  // sign words per row
+  constexpr bool kQ = MODE == TQ_MSE_Q || MODE == TQ_MSE_QDQ || MODE == TQ_PROD_Q;
+  constexpr bool kProd = MODE == TQ_PROD_Q || MODE == TQ_DQ_PROD;
+  constexpr bool kOut = MODE == TQ_MSE_QDQ || MODE == TQ_DQ_MSE || MODE == TQ_DQ_PROD;
+  constexpr uint32_t kNcols = 256;
+  // instruction descriptors (M = 128, N = 128)
+  constexpr uint32_t kIdPi = umma_idesc_f16(IsBf16<T>::value, IsBf16<T>::value, false, D, kRows);    // X Pi^T
+  constexpr uint32_t kIdPiT = umma_idesc_f16(IsBf16<T>::value, IsBf16<T>::value, true, D, kRows);    // W Pi
+  constexpr uint32_t kIdT = umma_idesc_f16(false, false, false, D, kRows);                   // rho T^T
+  constexpr uint32_t kIdTT = umma_idesc_f16(false, false, true, D, kRows);                   // S T
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* s_tile = smem + SM::tile_off;
+  uint8_t* s_pi = smem + SM::pi_off;
+  uint8_t* s_t = smem + SM::t_off;
+  uint32_t* s_codes = reinterpret_cast<uint32_t*>(smem + SM::codes_off);
+  uint32_t* s_signs = reinterpret_cast<uint32_t*>(smem + SM::signs_off);
+  float* s_sc = reinterpret_cast<float*>(smem + SM::cb_off);
+  float* s_mag = s_sc + 16;
+  float* s_cf = s_sc + 32;
+  float* s_bscale = s_sc + 48;
+  uint64_t* bar_x = reinterpret_cast<uint64_t*>(smem + SM::bar_off);
+  uint64_t* bar_p = bar_x + 1;
+  uint64_t* bar_m = bar_x + 2;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + SM::tmem_off);
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int64_t n = a.n;
+  const int64_t ntiles = (n + kRows - 1) / kRows;
+  const uint32_t tile_s = smem_u32(s_tile), pi_s = smem_u32(s_pi), t_s = smem_u32(s_t);
+
+  if (tid == 0) {
+    if (kQ) tma_prefetch_desc(&map_x);
+    tma_prefetch_desc(&map_pi);
+    if (kProd) tma_prefetch_desc(&map_t);
+    if (kOut) tma_prefetch_desc(&map_o);
+    mbar_init(bar_x, 1);
+    mbar_init(bar_p, 1);
+    mbar_init(bar_m, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) tmem_alloc(s_tmem, kNcols);
+  build_consts<BITS>(a.centroids, s_sc, s_mag, s_cf, s_bscale);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  const uint32_t tm_y = tmem, tm_2 = tmem + 128;          // two 128-column accumulators
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;  // this warp's TMEM lanes
+
+  // resident parameters
+  if (tid == 0) {
+    mbar_arrive_expect_tx(bar_p, kTileBytes * (kProd ? 2 : 1));
+    for (int b = 0; b < 2; ++b) tma_load_2d(s_pi + b * kBoxBytes, &map_pi, b * 64, 0, bar_p);
+    if (kProd)
+      for (int b = 0; b < 2; ++b) tma_load_2d(s_t + b * kBoxBytes, &map_t, b * 64, 0, bar_p);
+  }
+  bool ok = __syncthreads_and(mbar_wait(bar_p, 0, a.status));
+
+  uint32_t par_x = 0, par_m = 0;
+  const float Bs = *s_bscale;
+
+  // MMA helpers (thread 0): A is always the tile buffer (K-major); B is Pi or T
+  auto mma_kmajor_b = [&](uint32_t tm_d, uint32_t b_s, uint32_t idesc) {
+    tc_fence_after();
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t koff = (uint32_t)((kk >> 2) * kBoxBytes + (kk & 3) * 32);
+      umma_f16(tm_d, umma_desc_sw128(tile_s + koff, 16, 1024), umma_desc_sw128(b_s + koff, 16, 1024), idesc, kk > 0);
+    }
+    umma_commit(bar_m);
+  };
+  auto mma_mnmajor_b = [&](uint32_t tm_d, uint32_t b_s, uint32_t idesc) {
+    tc_fence_after();
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t akoff = (uint32_t)((kk >> 2) * kBoxBytes + (kk & 3) * 32);
+      const uint32_t bkoff = (uint32_t)(kk * 16 * 128);  // 16 K rows of 128 bytes
+      umma_f16(tm_d, umma_desc_sw128(tile_s + akoff, 16, 1024), umma_desc_sw128(b_s + bkoff, kBoxBytes, 1024), idesc,
+               kk > 0);
+    }
+    umma_commit(bar_m);
+  };
+  auto wait_mma = [&]() {
+    const bool r = mbar_wait(bar_m, par_m, a.status);
+    par_m ^= 1;
+    tc_fence_after();
+    return r;
+  };
+  // write 8 floats as one 16-byte chunk (element type E) of this thread's row in the tile buffer
+  auto put_chunk = [&](int j, const float* v, bool as_f16) {
+    uint4 c = as_f16 ? Elem<__half>::pack(v) : Elem<T>::pack(v);
+    *reinterpret_cast<uint4*>(s_tile + sw128_chunk(tid, j, kBoxBytes)) = c;
+  };
+
+  for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+    const int64_t row0 = tile * kRows;
+    const int rows = (int)(n - row0 < (int64_t)kRows ? n - row0 : (int64_t)kRows);
+    const int64_t row = row0 + tid;
+    float nrm = 0.f;
+
+    // ------------------------------------------------------------ quantize side
+    if constexpr (kQ) {
+      if (tid == 0) {
+        bulk_wait_read<0>();  // the previous x_hat store has left the tile buffer
+        mbar_arrive_expect_tx(bar_x, kTileBytes);
+        for (int b = 0; b < 2; ++b) tma_load_2d(s_tile + b * kBoxBytes, &map_x, b * 64, (int32_t)row0, bar_x);
+      }
+      ok = mbar_wait(bar_x, par_x, a.status);
+      par_x ^= 1;
+      if (!__syncthreads_and(ok)) break;
+      if (tid == 0) mma_kmajor_b(tm_y, pi_s, kIdPi);  // y = Pi x (rows of the tile)
+      // ||x||^2 from the tile while the MMA runs
+      float2 acc[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < D / 8; ++j) {
+        float f[8];
+        Elem<T>::unpack(*reinterpret_cast<const uint4*>(s_tile + sw128_chunk(tid, j, kBoxBytes)), f);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 v = make_float2(f[2 * k], f[2 * k + 1]);
+          acc[k] = __ffma2_rn(v, v, acc[k]);
+        }
+      }
+      nrm = sqrtf(((acc[0].x + acc[1].x) + (acc[2].x + acc[3].x)) + ((acc[0].y + acc[1].y) + (acc[2].y + acc[3].y)));
+      if (!wait_mma()) ok = false;
+
+      const float srow = nrm > 0.f ? __fdiv_rn(Bs, nrm) : 0.f;
+      const float shift = -fmaf(kShift, nrm, 0x1p-126f);
+      const float rn = nrm > 0.f ? __frcp_rn(nrm) : 0.f;
+      float dl[H > 1 ? H - 1 : 1], sc[H > 1 ? H - 1 : 1];
+#pragma unroll
+      for (int j = 0; j < H - 1; ++j) {
+        dl[j] = __fsub_rn(s_mag[j + 1], s_mag[j]);
+        sc[j] = s_sc[j];
+      }
+      const float mn0 = s_mag[0];
+      float win[NWIN];
+#pragma unroll
+      for (int w = 0; w < NWIN; ++w) win[w] = kWindow0;
+      float gs = 0.f;  // ||r||^2 (prod)
+
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        float y[32];
+        tmem_ld32(tm_y + lane_off + 32 * c, y);
+        float w_out[32];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const float2 Y = make_float2(y[i] + shift, y[i + 1] + shift);
+          float2 m2 = make_float2(mn0, mn0), cnt = make_float2(0.5f, 0.5f);
+#pragma unroll
+          for (int j = 0; j < H - 1; ++j) {
+            const float2 st = make_float2(fma_sat(fabsf(Y.x), srow, sc[j]), fma_sat(fabsf(Y.y), srow, sc[j]));
+            m2 = __ffma2_rn(st, make_float2(dl[j], dl[j]), m2);
+            cnt = __fadd2_rn(cnt, st);
+          }
+          const float2 sg = make_float2(sign_one(Y.x), sign_one(Y.y));
+          const float2 chat = __fmul2_rn(m2, sg);  // unit-scale centroid
+          const float2 code = __ffma2_rn(sg, cnt, make_float2(H - 0.5f, H - 0.5f));
+          const int k0 = 32 * c + i, k1 = k0 + 1;
+          win[k0 / CPW] = fmaf(code.x, (float)(1u << (BITS * (k0 % CPW))), win[k0 / CPW]);
+          win[k1 / CPW] = fmaf(code.y, (float)(1u << (BITS * (k1 % CPW))), win[k1 / CPW]);
+          if constexpr (MODE == TQ_MSE_QDQ) {
+            w_out[i] = chat.x;
+            w_out[i + 1] = chat.y;
+          } else if constexpr (MODE == TQ_PROD_Q) {
+            // rotated unit residual r = y/||x|| - c_hat
+            const float2 r = __ffma2_rn(make_float2(y[i], y[i + 1]), make_float2(rn, rn), make_float2(-chat.x, -chat.y));
+            gs = fmaf(r.x, r.x, fmaf(r.y, r.y, gs));
+            w_out[i] = r.x * kSketchScale;
+            w_out[i + 1] = r.y * kSketchScale;
+          }
+        }
+        if constexpr (MODE == TQ_MSE_QDQ || MODE == TQ_PROD_Q) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) put_chunk(4 * c + q, &w_out[8 * q], MODE == TQ_PROD_Q);
+        }
+      }
+      // codes -> staging
+      uint32_t wc[W];
+#pragma unroll
+      for (int w = 0; w < W; ++w) wc[w] = 0u;
+#pragma unroll
+      for (int w = 0; w < NWIN; ++w) {
+        const uint32_t v = __float_as_uint(win[w]) & 0x7fffffu;
+        const int bo = w * CPW * BITS;
+        wc[bo >> 5] |= v << (bo & 31);
+        if ((bo & 31) + CPW * BITS > 32 && (bo >> 5) + 1 < W) wc[(bo >> 5) + 1] |= v >> (32 - (bo & 31));
+      }
+#pragma unroll
+      for (int w = 0; w < W; ++w) s_codes[tid * W + w] = wc[w];
+      if (tid < rows) {
+        if (a.norms_out) a.norms_out[row] = nrm;
+        if (kProd && a.gammas_out) a.gammas_out[row] = sqrtf(gs);
+      }
+
+      if constexpr (MODE == TQ_MSE_QDQ || MODE == TQ_PROD_Q) {
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+          if (MODE == TQ_MSE_QDQ) mma_mnmajor_b(tm_2, pi_s, kIdPiT);  // Pi^T c_hat
+          else mma_kmajor_b(tm_2, t_s, kIdT);                         // T rho
+        }
+        if (!wait_mma()) ok = false;
+        if constexpr (MODE == TQ_PROD_Q) {
+#pragma unroll
+          for (int c = 0; c < NS; ++c) {
+            float z[32];
+            tmem_ld32(tm_2 + lane_off + 32 * c, z);
+            uint32_t bits = 0;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) bits |= (z[i] >= 0.f ? 1u : 0u) << i;  // sign(0) = +1
+            s_signs[tid * NS + c] = bits;
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            float v[32];
+            tmem_ld32(tm_2 + lane_off + 32 * c, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= nrm;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) put_chunk(4 * c + q, &v[8 * q], false);
+          }
+        }
+      }
+    } else {
+      // ---------------------------------------------------------- dequantize side
+      for (int i = tid; i < rows * W; i += kRows) {
+        const int r = i / W, w = i - r * W;
+        s_codes[i] = __ldg(a.codes_in + (row0 + r) * a.ldc + w);
+      }
+      if (kProd)
+        for (int i = tid; i < rows * NS; i += kRows) {
+          const int r = i / NS, w = i - r * NS;
+          s_signs[i] = __ldg(a.signs_in + (row0 + r) * a.lds + w);
+        }
+      nrm = tid < rows ? __ldg(a.norms_in + row) : 0.f;
+      const float gam = (kProd && tid < rows) ? __ldg(a.gammas_in + row) : 0.f;
+      if (tid == 0) bulk_wait_read<0>();
+      if (!__syncthreads_and(ok)) break;
+      uint32_t wc[W];
+#pragma unroll
+      for (int w = 0; w < W; ++w) wc[w] = s_codes[tid * W + w];
+      auto code_at = [&](int k) -> uint32_t {
+        const int bit = k * BITS, word = bit >> 5, sh = bit & 31;
+        uint32_t v = wc[word] >> sh;
+        if (sh + BITS > 32) v |= wc[word + 1] << (32 - sh);
+        return v & ((1u << BITS) - 1u);
+      };
+      if constexpr (kProd) {
+        // S tile of +1/-1 (fp16) -> T^T s
+#pragma unroll
+        for (int c = 0; c < NS; ++c) {
+          const uint32_t sw = s_signs[tid * NS + c];
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = ((sw >> i) & 1u) ? 1.f : -1.f;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) put_chunk(4 * c + q, &v[8 * q], true);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) mma_mnmajor_b(tm_2, t_s, kIdTT);
+        if (!wait_mma()) ok = false;
+        const float qs = a.qjl_scale * gam;  // sqrt(pi/2)/m * gamma
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          float v[32];
+          tmem_ld32(tm_2 + lane_off + 32 * c, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = fmaf(qs, v[i], s_cf[code_at(32 * c + i)]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) put_chunk(4 * c + q, &v[8 * q], false);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = s_cf[code_at(32 * c + i)];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) put_chunk(4 * c + q, &v[8 * q], false);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      if (tid == 0) mma_mnmajor_b(tm_y, pi_s, kIdPiT);  // Pi^T w
+      if (!wait_mma()) ok = false;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        float v[32];
+        tmem_ld32(tm_y + lane_off + 32 * c, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] *= nrm;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) put_chunk(4 * c + q, &v[8 * q], false);
+      }
+    }
+
+    // ------------------------------------------------------------ outputs
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (kOut && tid == 0) {
+      for (int b = 0; b < 2; ++b) tma_store_2d(&map_o, b * 64, (int32_t)row0, s_tile + b * kBoxBytes);
+      bulk_commit();
+    }
+    if constexpr (kQ) {
+      if (a.codes_out)
+        for (int i = tid; i < rows * W; i += kRows) {
+          const int r = i / W, w = i - r * W;
+          a.codes_out[(row0 + r) * a.ldc + w] = s_codes[i];
+        }
+      if (kProd && a.signs_out)
+        for (int i = tid; i < rows * NS; i += kRows) {
+          const int r = i / NS, w = i - r * NS;
+          a.signs_out[(row0 + r) * a.lds + w] = s_signs[i];
+        }
+    }
+    __syncthreads();  // staging buffers are rewritten by the next tile
+  }
+  if (tid == 0) bulk_wait_all<0>();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, kNcols);
+}
+
+}  // namespace tq
+
+// ============================================================================ launch
+template <typename T, int BITS, int MODE>
+static cudaError_t launch_tq_t(const CUtensorMap& mx, const CUtensorMap& mp, const CUtensorMap& mt, const CUtensorMap& mo,
+                               const TqArgs& a, cudaStream_t st, int num_sms) {
+  using SM = tq::Smem<BITS, MODE>;
+  auto kern = tq::tq_kernel<T, BITS, MODE>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::alloc);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int64_t ntiles = (a.n + tq::kRows - 1) / tq::kRows;
+  const int64_t grid = std::min<int64_t>(ntiles, (int64_t)num_sms * 2);
+  kern<<<(unsigned)grid, tq::kRows, SM::alloc, st>>>(mx, mp, mt, mo, a);
+  return cudaGetLastError();
+}
+
+template <typename T, int MODE>
+static cudaError_t tq_by_bits(int bits, const CUtensorMap& mx, const CUtensorMap& mp, const CUtensorMap& mt,
+                              const CUtensorMap& mo, const TqArgs& a, cudaStream_t st, int sms) {
+  switch (bits) {
+    case 1: return launch_tq_t<T, 1, MODE>(mx, mp, mt, mo, a, st, sms);
+    case 2: return launch_tq_t<T, 2, MODE>(mx, mp, mt, mo, a, st, sms);
+    case 3: return launch_tq_t<T, 3, MODE>(mx, mp, mt, mo, a, st, sms);
+    default: return launch_tq_t<T, 4, MODE>(mx, mp, mt, mo, a, st, sms);
+  }
+}
+
+template <typename T>
+static cudaError_t tq_by_mode(int mode, int bits, const CUtensorMap& mx, const CUtensorMap& mp, const CUtensorMap& mt,
+                              const CUtensorMap& mo, const TqArgs& a, cudaStream_t st, int sms) {
+  switch (mode) {
+    case TQ_MSE_Q: return tq_by_bits<T, TQ_MSE_Q>(bits, mx, mp, mt, mo, a, st, sms);
+    case TQ_MSE_QDQ: return tq_by_bits<T, TQ_MSE_QDQ>(bits, mx, mp, mt, mo, a, st, sms);
+    case TQ_PROD_Q: return tq_by_bits<T, TQ_PROD_Q>(bits, mx, mp, mt, mo, a, st, sms);
+    case TQ_DQ_MSE: return tq_by_bits<T, TQ_DQ_MSE>(bits, mx, mp, mt, mo, a, st, sms);
+    default: return tq_by_bits<T, TQ_DQ_PROD>(bits, mx, mp, mt, mo, a, st, sms);
+  }
+}
+
+cudaError_t launch_tq(int mode, kvrq_dtype dt, int bits, const CUtensorMap& mx, const CUtensorMap& mp,
+                      const CUtensorMap& mt, const CUtensorMap& mo, const TqArgs& a, cudaStream_t st, int sms) {
+  if (dt == KVRQ_BF16) return tq_by_mode<__nv_bfloat16>(mode, bits, mx, mp, mt, mo, a, st, sms);
+  return tq_by_mode<__half>(mode, bits, mx, mp, mt, mo, a, st, sms);
+}
+
+}  // namespace kvrq

@@ -23,9 +23,10 @@ Readings where the pages leave a step open:
   with an orthogonal Pi this is exactly Pi r, ||r_rot|| = ||r|| and
   S r = T r_rot, so the stored gamma and signs are the pages' quantities.
   ``prod_quantize_literal`` writes the pages' form out for comparison.
-* ``sketch_operand='f16'`` rounds the unit residual direction r_rot / gamma to
-  IEEE half before the projection: the sign decision is then taken on the
-  same operand values as on a half-precision tensor-core path.
+* ``sketch_operand='f16'`` projects 2^8 * r_rot rounded to IEEE half instead
+  of r_rot: the sign decision is then taken on the same operand values as on a
+  half-precision tensor-core path (the sign of T r is unchanged by the positive
+  scale, which only keeps the operand out of the half subnormal range).
 """
 
 import numpy as np
@@ -75,7 +76,7 @@ def prod_quantize(x, Pi, T, centroids_mse, bits, sketch_operand=None):
     safe = np.where(gamma > 0, gamma, 1.0)
     rho = np.where(gamma[:, None] > 0, r_rot / safe[:, None], 0.0)
     if sketch_operand == "f16":
-        rho = rho.astype(np.float16).astype(np.float64)
+        rho = (256.0 * r_rot).astype(np.float16).astype(np.float64)
     elif sketch_operand is not None:
         raise ValueError(sketch_operand)
     p = rho @ T.T  # T r_rot / gamma, row by row
