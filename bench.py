@@ -44,6 +44,11 @@ def rq_bytes_per_vector(d, bits, in_bytes=2, out_bytes=2):
     return d * in_bytes + 4 * W + 4 + d * out_bytes
 
 
+def tq_bytes_per_vector(d, bits, in_bytes=2, out_bytes=2):
+    """TurboQuant-mse fused roundtrip: x in, d codes of b bits + norm out, x_hat out."""
+    return d * in_bytes + 4 * (-(-(d * bits) // 32)) + 4 + d * out_bytes
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -68,7 +73,7 @@ class ClockSampler:
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -146,6 +151,57 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_leg_only(args):
+    """One kernel leg on args.rows seeded vectors: a warm-up call, then args.iters timed calls."""
+    import torch
+
+    import kv_cache_vector_rq_b200 as kvrq
+    from kv_cache_vector_rq_b200 import synth
+
+    dev = torch.device("cuda", 0)
+    kind, b = args.leg.rsplit("_", 1)[0], args.leg.rsplit("_", 1)[1]
+    mode, b = b.rstrip("0123456789"), int(b.lstrip("qdmpro"))
+    rows = args.rows
+    x = synth.lognormal(rows, D, seed=1, dtype=torch.float16, device=dev)
+    xh = torch.empty_like(x)
+    if kind == "rq":
+        rot = torch.from_numpy(kvrq.rq_rotors_init(D, 1).astype(np.float32)).to(dev)
+        cb = torch.from_numpy(kvrq.tq_codebook_init(D, b)[0].astype(np.float32)).to(dev)
+        codes, norms = kvrq.rq_quantize(x, rot, cb, b)
+        calls = {"q": lambda: kvrq.rq_quantize(x, rot, cb, b, codes=codes, norms=norms),
+                 "dq": lambda: kvrq.rq_dequantize(codes, norms, D, rot, cb, b, xhat=xh),
+                 "qdq": lambda: kvrq.rq_quantize_dequantize(x, rot, cb, b, codes=codes, norms=norms, xhat=xh)}
+    else:
+        pi = torch.from_numpy(kvrq.tq_rotation_init(D, 2)).to(torch.float16).to(dev)
+        T = torch.from_numpy(kvrq.qjl_matrix_init(D, D, 3)).to(torch.float16).to(dev)
+        prod = mode in ("prod", "dqp")
+        cb = torch.from_numpy(kvrq.tq_codebook_init(D, b - 1 if prod else b)[0].astype(np.float32)).to(dev)
+        if prod:
+            codes, signs, gam, norms = kvrq.tq_quantize_prod(x, pi, T, cb, b)
+        else:
+            codes, norms = kvrq.tq_quantize_mse(x, pi, cb, b)
+        calls = {"q": lambda: kvrq.tq_quantize_mse(x, pi, cb, b, codes=codes, norms=norms),
+                 "qdq": lambda: kvrq.tq_quantize_dequantize_mse(x, pi, cb, b, codes=codes, norms=norms, xhat=xh),
+                 "dqm": lambda: kvrq.tq_dequantize(codes, norms, D, pi, cb, b, xhat=xh)}
+        if prod:
+            calls["prod"] = lambda: kvrq.tq_quantize_prod(x, pi, T, cb, b, codes=codes, norms=norms, signs=signs,
+                                                          gammas=gam)
+            calls["dqp"] = lambda: kvrq.tq_dequantize(codes, norms, D, pi, cb, b, signs=signs, gammas=gam, T=T,
+                                                      xhat=xh)
+    fn = calls[mode]
+    fn()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(args.iters):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    kvrq.device_status()
+    ms = s.elapsed_time(e) / args.iters
+    print(json.dumps({"leg": args.leg, "rows": rows, "ms": ms, "Mvec_s": rows / ms / 1e3}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -153,6 +209,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="kvrq", choices=["kvrq", "reference"])
     ap.add_argument("--no-large", action="store_true", help="skip the 1 GiB HBM-roofline leg")
+    ap.add_argument("--leg", default=None,
+                    help="time one kernel leg (rq_q3, rq_dq3, rq_qdq3, tq_q3, tq_qdq3, tq_prod3, tq_dqm3, tq_dqp3, "
+                         "any b) on --rows vectors instead of the workload; used for profiler captures")
+    ap.add_argument("--rows", type=int, default=1 << 20)
+    ap.add_argument("--iters", type=int, default=3)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -161,6 +222,9 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.leg:
+        run_leg_only(args)
         return
 
     import torch
@@ -198,14 +262,23 @@ def main():
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
-    legs = [("rq", b) for b in BITS]
+    pi = torch.from_numpy(kvrq.tq_rotation_init(D, 2)).to(torch.float16).to(dev)
+    tq_codes = {b: torch.empty((N_VEC, kvrq.packed_words(D, b)), dtype=torch.int32, device=dev) for b in BITS}
+    legs = [("rq", b) for b in BITS] + [("tq", b) for b in BITS]
 
     def run_leg(leg):
         kind, b = leg
         if kind == "rq":
             kvrq.rq_quantize_dequantize(x, rot, cbs[b], b, codes=codes[b], norms=norms, xhat=xhat, stream=stream)
+        else:
+            kvrq.tq_quantize_dequantize_mse(x, pi, cbs[b], b, codes=tq_codes[b], norms=norms, xhat=xhat,
+                                            stream=stream)
 
     # ---------------------------------------------------------------- warm-up
+    # clocks are sampled from the warm-up through the timed region and the 1 GiB leg
+    clk = ClockSampler(local)
+    clk.__enter__()
+    time.sleep(0.3)
     for _ in range(args.warmup):
         for leg in legs:
             run_leg(leg)
@@ -218,17 +291,16 @@ def main():
     barrier()
     torch.cuda.synchronize()
     t_wall = time.perf_counter()
-    with ClockSampler(local) as clk:
-        for _ in range(args.steps):
-            for leg in legs:
-                flush.zero_()
-                s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                s.record(stream)
-                run_leg(leg)
-                e.record(stream)
-                ev[leg].append((s, e))
-                launches += 1
-        torch.cuda.synchronize()
+    for _ in range(args.steps):
+        for leg in legs:
+            flush.zero_()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            run_leg(leg)
+            e.record(stream)
+            ev[leg].append((s, e))
+            launches += 1
+    torch.cuda.synchronize()
     barrier()
     wall = time.perf_counter() - t_wall
     kvrq.device_status()
@@ -244,9 +316,9 @@ def main():
     achieved = bpv * N_VEC / (head_ms * 1e-3) / 1e9
     legs_out = {}
     for (kind, b), ms in leg_ms.items():
+        bpv_leg = rq_bytes_per_vector(D, b) if kind == "rq" else tq_bytes_per_vector(D, b)
         legs_out["%s_b%d" % (kind, b)] = {
-            "ms": ms, "Mvec_s": N_VEC / (ms * 1e-3) / 1e6,
-            "GB_s": rq_bytes_per_vector(D, b) * N_VEC / (ms * 1e-3) / 1e9}
+            "ms": ms, "Mvec_s": N_VEC / (ms * 1e-3) / 1e6, "GB_s": bpv_leg * N_VEC / (ms * 1e-3) / 1e9}
 
     # ---------------------------------------------------------------- end to end through the public API
     x_host = x.to("cpu").pin_memory()
@@ -297,6 +369,7 @@ def main():
                  "frac_of_peak": gbs / peak, "frac_of_8TBs": gbs / 8000.0}
         del xl, cl, nl, ol
 
+    clk.__exit__(None, None, None)
     cpu = None
     if rank == 0:
         rate, dt = cpu_oracle_rate(1024)
@@ -313,7 +386,8 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
             "config": {"workload": "65536 x d128 fp16 KV vectors (LogNormal(0,0.5) norms, 4 outlier channels x10), "
-                                   "fused quantize+dequantize, RotorQuant b=2,3,4; headline RotorQuant b=3",
+                                   "fused quantize+dequantize, RotorQuant and TurboQuant-mse b=2,3,4; "
+                                   "headline RotorQuant b=3",
                        "n_vectors_per_gpu": N_VEC, "d": D, "io_dtype": "fp16", "l2": "flushed (256 MiB write) "
                        "before every timed launch", "parallelism": "independent shard per GPU (weak scaling)"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
