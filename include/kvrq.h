@@ -190,6 +190,30 @@ kvrq_status tq_dequantize(void* stream, const uint32_t* codes, int64_t ldc, cons
                           const void* pi, const uint16_t* T, const float* centroids, void* xhat, kvrq_dtype odtype,
                           int64_t ldo);
 
+/* ================================================================ scores from packed keys
+ * [TQB "随机旋转（Lemma 1）": rotate the query once instead of every key;
+ * RQ "How TurboQuant Works": <q,k> ~ <q,k_mse> + ||r|| sqrt(pi/2)/m <S q, sign(S r)>;
+ * RQ "When to Use Which": Q K^T straight from the compressed indices]
+ *   score[h][g][t] = ||k|| * ( <q', c_hat(k)> + [prod] sqrt(pi/2)/m * gamma(k) * <T q', s(k)> )
+ * with q' = Pi q (TurboQuant) or the per-group rotor sandwich of the zero-padded q
+ * (RotorQuant, 3G coordinates); equal to <q, x_hat(k)>.
+ *   q: [n_heads][group][ldq] (dtype qdtype), grouped-query layout: query row
+ *      (h, g) reads KV head h. n_heads counts every (layer, batch, KV head).
+ *   keys of head h, token t: codes + h*codes_head_stride + t*ldc (words),
+ *      signs + h*signs_head_stride + t*lds (prod), norms/gammas + h*tok_head_stride + t.
+ *   method KVRQ_RQ_MSE (rotors [43][4]), KVRQ_TQ_MSE or KVRQ_TQ_PROD (pi [d][d] of
+ *      pi_dtype fp16/bf16, T [m][d] fp16 for prod); bits = the quantizer's total bits
+ *      (prod stores bits-1); centroids: the stored codes' codebook.
+ *   scores: fp32 [(h*group + g)*ld_scores + t].
+ * d = 128 (m = d); group <= 64 (prod: <= 32). Scores use fp16 operands on the
+ * tensor cores with fp32 accumulation. */
+kvrq_status kv_score_packed(void* stream, kvrq_method method, const void* q, kvrq_dtype qdtype, int64_t ldq,
+                            int64_t n_heads, int group, int d, int bits, int m, const uint32_t* codes, int64_t ldc,
+                            int64_t codes_head_stride, const uint32_t* signs, int64_t lds, int64_t signs_head_stride,
+                            const float* norms, const float* gammas, int64_t tok_head_stride, int64_t n_tokens,
+                            const float* rotors, const void* pi, kvrq_dtype pi_dtype, const uint16_t* T,
+                            const float* centroids, float* scores, int64_t ld_scores);
+
 #ifdef __cplusplus
 }
 #endif

@@ -260,3 +260,39 @@ def tq_dequantize(codes, norms, d, pi, centroids, bits, signs=None, gammas=None,
         n, d, m, bits, _ptr(pi, "pi", xhat.dtype), _ptr(T, "T", torch.float16),
         _ptr(centroids, "centroids", torch.float32), op, _dtype_code(xhat), ldo))
     return xhat
+
+
+# ----------------------------------------------------------------------------- scores
+
+def kv_score_packed(method, q, codes, norms, bits, n_tokens, centroids, rotors=None, pi=None, T=None, signs=None,
+                    gammas=None, scores=None, stream=None):
+    """Scores from packed keys.
+
+    q: [n_heads, group, d] CUDA tensor. codes: [n_heads, T_max, W] (int32 view of uint32),
+    norms/gammas: [n_heads, T_max], signs: [n_heads, T_max, m/32]; the first n_tokens tokens
+    of every head are scored. method: RQ_MSE, TQ_MSE or TQ_PROD; bits: the quantizer's total
+    bits. Returns scores [n_heads, group, n_tokens] fp32."""
+    torch = _torch()
+    n_heads, group, d = q.shape
+    if q.stride(2) != 1 or q.stride(1) != q.shape[2] or q.stride(0) != group * q.shape[2]:
+        raise ValueError("q must be contiguous")
+    if scores is None:
+        scores = torch.empty((n_heads, group, n_tokens), dtype=torch.float32, device=q.device)
+    m = T.shape[0] if T is not None else d
+    def strides(t, name):
+        if t is None:
+            return None, 0, 0
+        if not t.is_cuda or t.stride(-1) != 1:
+            raise ValueError("%s must be a CUDA tensor with unit inner stride" % name)
+        return t.data_ptr(), (t.stride(1) if t.dim() == 3 else 1), t.stride(0)
+    cp, ldc, chs = strides(codes, "codes")
+    sp, lds, shs = strides(signs, "signs")
+    if norms.stride(-1) != 1 or (gammas is not None and gammas.stride() != norms.stride()):
+        raise ValueError("norms/gammas must share one [n_heads, T_max] layout")
+    pdt = _dtype_code(pi) if pi is not None else F16
+    _lib.check("kv_score_packed", lib().kv_score_packed(
+        _stream(stream), method, q.data_ptr(), _dtype_code(q), d, n_heads, group, d, bits, m, cp, ldc, chs, sp, lds,
+        shs, _ptr(norms, "norms", torch.float32), _ptr(gammas, "gammas", torch.float32), norms.stride(0), n_tokens,
+        _ptr(rotors, "rotors", torch.float32), _ptr(pi, "pi"), pdt, _ptr(T, "T", torch.float16),
+        _ptr(centroids, "centroids", torch.float32), scores.data_ptr(), scores.stride(1)))
+    return scores

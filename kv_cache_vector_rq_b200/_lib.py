@@ -45,6 +45,12 @@ SIGNATURES = {
     # stream, codes, ldc, signs, lds, gammas, norms, n, d, m, bits, pi, T, centroids, xhat, odtype, ldo
     "tq_dequantize": (c_int, [c_vp, c_vp, c_i64, c_vp, c_i64, c_vp, c_vp, c_i64, c_int, c_int, c_int, c_vp, c_vp,
                               c_vp, c_vp, c_int, c_i64]),
+    # stream, method, q, qdtype, ldq, n_heads, group, d, bits, m, codes, ldc, codes_head_stride, signs, lds,
+    # signs_head_stride, norms, gammas, tok_head_stride, n_tokens, rotors, pi, pi_dtype, T, centroids, scores,
+    # ld_scores
+    "kv_score_packed": (c_int, [c_vp, c_int, c_vp, c_int, c_i64, c_i64, c_int, c_int, c_int, c_int, c_vp, c_i64,
+                                c_i64, c_vp, c_i64, c_i64, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_vp, c_vp,
+                                c_vp, c_i64]),
 }
 
 _lib = None

@@ -14,6 +14,7 @@
 #include "kvrq_internal.h"
 #include "rq_launch.h"
 #include "tq_launch.h"
+#include "score_launch.h"
 
 namespace kvrq {
 
@@ -348,6 +349,80 @@ kvrq_status tq_dequantize(void* stream, const uint32_t* codes, int64_t ldc, cons
   const int mode = signs ? TQ_DQ_PROD : TQ_DQ_MSE;
   return tq_call("tq_dequantize", mode, stream, nullptr, odtype, 0, n, d, m, pi, T, centroids, bits, nullptr, codes,
                  ldc, nullptr, signs, lds, nullptr, gammas, nullptr, norms, xhat, ldo);
+}
+
+kvrq_status kv_score_packed(void* stream, kvrq_method method, const void* q, kvrq_dtype qdtype, int64_t ldq,
+                            int64_t n_heads, int group, int d, int bits, int m, const uint32_t* codes, int64_t ldc,
+                            int64_t codes_head_stride, const uint32_t* signs, int64_t lds, int64_t signs_head_stride,
+                            const float* norms, const float* gammas, int64_t tok_head_stride, int64_t n_tokens,
+                            const float* rotors, const void* pi, kvrq_dtype pi_dtype, const uint16_t* T,
+                            const float* centroids, float* scores, int64_t ld_scores) {
+  const char* name = "kv_score_packed";
+  const bool prod = method == KVRQ_TQ_PROD;
+  if (method != KVRQ_RQ_MSE && method != KVRQ_TQ_MSE && method != KVRQ_TQ_PROD)
+    return set_error(KVRQ_EINVAL, "kv_score_packed: unknown method");
+  if (n_heads < 0 || n_tokens < 0 || group < 1) return set_error(KVRQ_EINVAL, "kv_score_packed: bad sizes");
+  if (d != 128) return set_error(KVRQ_EUNSUPPORTED, "kv_score_packed: d = 128 is supported");
+  if (prod && m != d) return set_error(KVRQ_EUNSUPPORTED, "kv_score_packed: the QJL projection needs m = d");
+  const int cbits = prod ? bits - 1 : bits;
+  if (cbits < 1 || cbits > 4) return set_error(KVRQ_EUNSUPPORTED, "kv_score_packed: stored code width must be 1..4");
+  const int rows_needed = group * (prod ? 2 : 1);
+  if (rows_needed > 64) return set_error(KVRQ_EUNSUPPORTED, "kv_score_packed: group too large (<= 64, prod <= 32)");
+  if (!valid_dtype(qdtype) || ldq < d) return set_error(KVRQ_EINVAL, "kv_score_packed: bad query dtype or ldq");
+  const int ncode = method == KVRQ_RQ_MSE ? 3 * ((d + 2) / 3) : d;
+  const int64_t W = kvrq_packed_words(ncode, cbits);
+  if (n_heads == 0 || n_tokens == 0) return KVRQ_OK;
+  if (!q || !codes || !norms || !centroids || !scores) return set_error(KVRQ_EINVAL, "kv_score_packed: NULL argument");
+  if (ldc < W || ld_scores < n_tokens || tok_head_stride < n_tokens || codes_head_stride < n_tokens * ldc)
+    return set_error(KVRQ_EINVAL, "kv_score_packed: strides too small");
+  if (method == KVRQ_RQ_MSE && (!rotors || !aligned(rotors, 16)))
+    return set_error(KVRQ_EINVAL, "kv_score_packed: rotors (16-byte aligned) required");
+  if (method != KVRQ_RQ_MSE && (!pi || (pi_dtype != KVRQ_F16 && pi_dtype != KVRQ_BF16)))
+    return set_error(KVRQ_EINVAL, "kv_score_packed: pi (fp16 or bf16) required");
+  if (prod && (!signs || !gammas || !T || lds < m / 32 || signs_head_stride < n_tokens * lds))
+    return set_error(KVRQ_EINVAL, "kv_score_packed: signs, gammas and T required for prod");
+  if (!aligned(codes, 4) || !aligned(norms, 4) || !aligned(scores, 4))
+    return set_error(KVRQ_EINVAL, "kv_score_packed: misaligned pointer");
+  if (n_heads > 65535) return set_error(KVRQ_EUNSUPPORTED, "kv_score_packed: more than 65535 heads");
+
+  DeviceInfo* di;
+  kvrq_status st = current_device(&di);
+  if (st != KVRQ_OK) return st;
+  ScoreArgs a{};
+  a.n_heads = n_heads;
+  a.group = group;
+  a.n_tokens = n_tokens;
+  // enough CTAs to fill the GPU a few times over, at most 64 tiles each
+  int64_t tiles = (n_tokens + 127) / 128;
+  int64_t per = (tiles * n_heads + 4LL * di->num_sms - 1) / (4LL * di->num_sms);
+  if (per < 1) per = 1;
+  if (per > 64) per = 64;
+  if (per > tiles) per = tiles;
+  a.tokens_per_cta = per * 128;
+  a.q = q;
+  a.ldq = ldq;
+  a.q_f32 = qdtype == KVRQ_F32;
+  a.q_bf16 = qdtype == KVRQ_BF16;
+  a.codes = codes;
+  a.ldc = ldc;
+  a.codes_head_stride = codes_head_stride;
+  a.signs = signs;
+  a.lds = lds;
+  a.signs_head_stride = signs_head_stride;
+  a.norms = norms;
+  a.gammas = gammas;
+  a.tok_head_stride = tok_head_stride;
+  a.rotors = rotors;
+  a.pi = pi;
+  a.pi_bf16 = pi_dtype == KVRQ_BF16;
+  a.T = T;
+  a.centroids = centroids;
+  a.qjl_scale = (float)(1.2533141373155003 / (double)(prod ? m : d));
+  a.scores = scores;
+  a.ld_scores = ld_scores;
+  a.status = di->status;
+  const int nb = rows_needed <= 16 ? 16 : (rows_needed <= 32 ? 32 : 64);
+  return launch_status(name, launch_score(method, nb, cbits, a, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"
