@@ -151,6 +151,79 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def decode_step_c4(kvrq, synth, torch, dev, batch, steps, warmup, layers=36, kv_heads=2, group=8,
+                   cached=131072):
+    """Qwen2.5-3B-shaped decode step: append one K (TurboQuant-prod 3-bit) and one V
+    (RotorQuant 3-bit) per (layer, batch, KV head), then score all 16 query heads over
+    cached + 1 tokens straight from the packed keys. Returns timings and traffic."""
+    heads = layers * kv_heads * batch
+    t_max = cached + 1
+    bits_k, bits_v = 3, 3
+    pi = torch.from_numpy(kvrq.tq_rotation_init(D, 2)).to(torch.float16).to(dev)
+    T = torch.from_numpy(kvrq.qjl_matrix_init(D, D, 3)).to(torch.float16).to(dev)
+    rot = torch.from_numpy(kvrq.rq_rotors_init(D, 1).astype(np.float32)).to(dev)
+    ck = torch.from_numpy(kvrq.tq_codebook_init(D, bits_k - 1)[0].astype(np.float32)).to(dev)
+    cv = torch.from_numpy(kvrq.tq_codebook_init(D, bits_v)[0].astype(np.float32)).to(dev)
+    Wk, Wv = kvrq.packed_words(D, bits_k - 1), kvrq.packed_words(129, bits_v)
+    k_codes = torch.empty((heads, t_max, Wk), dtype=torch.int32, device=dev)
+    k_signs = torch.empty((heads, t_max, D // 32), dtype=torch.int32, device=dev)
+    k_norms = torch.empty((heads, t_max), dtype=torch.float32, device=dev)
+    k_gam = torch.empty((heads, t_max), dtype=torch.float32, device=dev)
+    v_codes = torch.empty((heads, t_max, Wv), dtype=torch.int32, device=dev)
+    v_norms = torch.empty((heads, t_max), dtype=torch.float32, device=dev)
+    # prefill (untimed): the cached tokens, quantized in chunks of heads
+    chunk = max(1, (1 << 22) // cached)
+    for h0 in range(0, heads, chunk):
+        h1 = min(heads, h0 + chunk)
+        rows = (h1 - h0) * t_max
+        kx = synth.lognormal(rows, D, seed=5000 + h0, dtype=torch.float16, device=dev)
+        kvrq.tq_quantize_prod(kx, pi, T, ck, bits_k, codes=k_codes[h0:h1].view(rows, Wk),
+                              norms=k_norms[h0:h1].reshape(rows), signs=k_signs[h0:h1].view(rows, D // 32),
+                              gammas=k_gam[h0:h1].reshape(rows))
+        vx = synth.gaussian(rows, D, seed=7000 + h0, dtype=torch.float16, device=dev)
+        kvrq.rq_quantize(vx, rot, cv, bits_v, codes=v_codes[h0:h1].view(rows, Wv), norms=v_norms[h0:h1].reshape(rows))
+        del kx, vx
+    torch.cuda.synchronize()
+    q = synth.gaussian(heads * group, D, seed=9, dtype=torch.float16, device=dev).view(heads, group, D)
+    new_k = synth.lognormal(heads, D, seed=10, dtype=torch.float16, device=dev)
+    new_v = synth.gaussian(heads, D, seed=11, dtype=torch.float16, device=dev)
+    scores = torch.empty((heads, group, t_max), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        kvrq.kv_cache_append(kvrq.TQ_PROD, new_k, cached, bits_k, ck, k_codes, k_norms, pi=pi, T=T, signs=k_signs,
+                             gammas=k_gam, stream=stream)
+        kvrq.kv_cache_append(kvrq.RQ_MSE, new_v, cached, bits_v, cv, v_codes, v_norms, rotors=rot, stream=stream)
+        ev_mid.record(stream)
+        kvrq.kv_score_packed(kvrq.TQ_PROD, q, k_codes, k_norms, bits_k, t_max, ck, pi=pi, T=T, signs=k_signs,
+                             gammas=k_gam, scores=scores, stream=stream)
+
+    ev_mid = torch.cuda.Event(enable_timing=True)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    tot, sc = [], []
+    for _ in range(steps):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev_mid = torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        step()
+        e.record(stream)
+        e.synchronize()
+        tot.append(s.elapsed_time(e))
+        sc.append(ev_mid.elapsed_time(e))
+    kvrq.device_status()
+    ms, ms_score = sum(tot) / len(tot), sum(sc) / len(sc)
+    keys = heads * t_max
+    score_bytes = keys * (4 * Wk + 4 * (D // 32) + 8) + keys * group * 4
+    out = {"batch": batch, "layers": layers, "kv_heads": kv_heads, "query_heads_per_kv": group, "tokens": t_max,
+           "ms_per_step": ms, "ms_score": ms_score, "keys_scored_per_s": keys / (ms_score * 1e-3),
+           "score_GB_s": score_bytes / (ms_score * 1e-3) / 1e9, "score_bytes_per_step": score_bytes}
+    del k_codes, k_signs, k_norms, k_gam, v_codes, v_norms, scores
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_leg_only(args):
     """One kernel leg on args.rows seeded vectors: a warm-up call, then args.iters timed calls."""
     import torch
@@ -159,8 +232,28 @@ def run_leg_only(args):
     from kv_cache_vector_rq_b200 import synth
 
     dev = torch.device("cuda", 0)
+    if args.leg.startswith("score"):
+        # packed-key scores (TurboQuant-prod 3-bit keys, 72 KV heads x 8 query heads), args.rows keys in total
+        heads, group = 72, 8
+        t = max(1, args.rows // heads)
+        pi = torch.from_numpy(kvrq.tq_rotation_init(D, 2)).to(torch.float16).to(dev)
+        T = torch.from_numpy(kvrq.qjl_matrix_init(D, D, 3)).to(torch.float16).to(dev)
+        ck = torch.from_numpy(kvrq.tq_codebook_init(D, 2)[0].astype(np.float32)).to(dev)
+        kx = synth.lognormal(heads * t, D, seed=3, dtype=torch.float16, device=dev)
+        codes, signs, gam, norms = kvrq.tq_quantize_prod(kx, pi, T, ck, 3)
+        del kx
+        q = synth.gaussian(heads * group, D, seed=4, dtype=torch.float16, device=dev).view(heads, group, D)
+        sc = torch.empty((heads, group, t), dtype=torch.float32, device=dev)
+        fn = lambda: kvrq.kv_score_packed(kvrq.TQ_PROD, q, codes.view(heads, t, -1), norms.view(heads, t), 3, t, ck,
+                                          pi=pi, T=T, signs=signs.view(heads, t, -1), gammas=gam.view(heads, t),
+                                          scores=sc)
+        rows = heads * t
+    else:
+        fn, rows = None, None
     kind, b = args.leg.rsplit("_", 1)[0], args.leg.rsplit("_", 1)[1]
     mode, b = b.rstrip("0123456789"), int(b.lstrip("qdmpro"))
+    if fn is not None:
+        return time_fn(fn, rows, args, torch, kvrq)
     rows = args.rows
     x = synth.lognormal(rows, D, seed=1, dtype=torch.float16, device=dev)
     xh = torch.empty_like(x)
@@ -188,7 +281,10 @@ def run_leg_only(args):
                                                           gammas=gam)
             calls["dqp"] = lambda: kvrq.tq_dequantize(codes, norms, D, pi, cb, b, signs=signs, gammas=gam, T=T,
                                                       xhat=xh)
-    fn = calls[mode]
+    return time_fn(calls[mode], rows, args, torch, kvrq)
+
+
+def time_fn(fn, rows, args, torch, kvrq):
     fn()
     torch.cuda.synchronize()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -368,7 +464,12 @@ def main():
         large = {"rows": LARGE_ROWS, "ms": lms, "Mvec_s": LARGE_ROWS / (lms * 1e-3) / 1e6, "GB_s": gbs,
                  "frac_of_peak": gbs / peak, "frac_of_8TBs": gbs / 8000.0}
         del xl, cl, nl, ol
+        torch.cuda.empty_cache()
 
+    decode = None
+    if not args.no_large:
+        decode = {"b1": decode_step_c4(kvrq, synth, torch, dev, 1, max(args.steps, 5), args.warmup),
+                  "b16": decode_step_c4(kvrq, synth, torch, dev, 16, 5, 3)}
     clk.__exit__(None, None, None)
     cpu = None
     if rank == 0:
@@ -395,6 +496,7 @@ def main():
                          "kernel": "rq_row_kernel<__half, 3, RQ_QDQ>", "bytes_per_vector": bpv},
             "legs": legs_out,
             "hbm_1gib": large,
+            "decode_c4": decode,
             "e2e": {"value": N_VEC * world / (e2e * 1e-3) / 1e6, "unit": "Mvec/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms": e2e},
             "gpu_launches": launches,

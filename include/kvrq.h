@@ -214,6 +214,20 @@ kvrq_status kv_score_packed(void* stream, kvrq_method method, const void* q, kvr
                             const float* rotors, const void* pi, kvrq_dtype pi_dtype, const uint16_t* T,
                             const float* centroids, float* scores, int64_t ld_scores);
 
+/* ================================================================ decode-step append
+ * [RQ "Post-Prefill Quantization": each decode step quantizes the new key (and
+ * value) for storage] Quantizes one new vector per cache row (a row = one
+ * (layer, batch, KV head)) straight into its slot of a packed cache, in one
+ * launch: row r of x goes to codes + r*codes_row_stride (words), signs +
+ * r*signs_row_stride, norms/gammas + r*norm_row_stride. The caller passes the
+ * cache pointers already advanced to the slot (e.g. codes + slot*W). method
+ * selects rq_quantize, tq_quantize_mse or tq_quantize_prod (same argument
+ * rules); unused parameters may be NULL. */
+kvrq_status kv_cache_append(void* stream, kvrq_method method, const void* x, kvrq_dtype xdtype, int64_t n_rows,
+                            int d, int64_t ldx, int bits, const float* rotors, const void* pi, const uint16_t* T, int m,
+                            const float* centroids, uint32_t* codes, int64_t codes_row_stride, uint32_t* signs,
+                            int64_t signs_row_stride, float* norms, float* gammas, int64_t norm_row_stride);
+
 #ifdef __cplusplus
 }
 #endif

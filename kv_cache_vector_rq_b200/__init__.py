@@ -296,3 +296,24 @@ def kv_score_packed(method, q, codes, norms, bits, n_tokens, centroids, rotors=N
         _ptr(rotors, "rotors", torch.float32), _ptr(pi, "pi"), pdt, _ptr(T, "T", torch.float16),
         _ptr(centroids, "centroids", torch.float32), scores.data_ptr(), scores.stride(1)))
     return scores
+
+
+def kv_cache_append(method, x, slot, bits, centroids, codes, norms, rotors=None, pi=None, T=None, signs=None,
+                    gammas=None, stream=None):
+    """Quantize x [rows, d] (one new vector per cache row) into slot `slot` of a packed cache:
+    codes [rows, T_max, W], norms/gammas [rows, T_max], signs [rows, T_max, m/32]."""
+    torch = _torch()
+    rows, d = x.shape
+    xp, ldx = _rows(x, "x")
+    W = codes.shape[2]
+    m = T.shape[0] if T is not None else d
+    cp = codes.data_ptr() + slot * codes.stride(1) * 4
+    sp = signs.data_ptr() + slot * signs.stride(1) * 4 if signs is not None else None
+    np_ = norms.data_ptr() + slot * norms.stride(1) * 4
+    gp = gammas.data_ptr() + slot * gammas.stride(1) * 4 if gammas is not None else None
+    if gammas is not None and gammas.stride() != norms.stride():
+        raise ValueError("norms and gammas must share one layout")
+    _lib.check("kv_cache_append", lib().kv_cache_append(
+        _stream(stream), method, xp, _dtype_code(x), rows, d, ldx, bits, _ptr(rotors, "rotors", torch.float32),
+        _ptr(pi, "pi"), _ptr(T, "T", torch.float16), m, _ptr(centroids, "centroids", torch.float32), cp,
+        codes.stride(0), sp, signs.stride(0) if signs is not None else 0, np_, gp, norms.stride(0)))

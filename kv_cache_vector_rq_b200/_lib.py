@@ -51,6 +51,10 @@ SIGNATURES = {
     "kv_score_packed": (c_int, [c_vp, c_int, c_vp, c_int, c_i64, c_i64, c_int, c_int, c_int, c_int, c_vp, c_i64,
                                 c_i64, c_vp, c_i64, c_i64, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_vp, c_vp,
                                 c_vp, c_i64]),
+    # stream, method, x, xdtype, n_rows, d, ldx, bits, rotors, pi, T, m, centroids, codes, codes_row_stride,
+    # signs, signs_row_stride, norms, gammas, norm_row_stride
+    "kv_cache_append": (c_int, [c_vp, c_int, c_vp, c_int, c_i64, c_int, c_i64, c_int, c_vp, c_vp, c_vp, c_int, c_vp,
+                                c_vp, c_i64, c_vp, c_i64, c_vp, c_vp, c_i64]),
 }
 
 _lib = None

@@ -136,7 +136,8 @@ static kvrq_status launch_status(const char* where, cudaError_t e) {
 static kvrq_status rq_call(const char* name, int mode, void* stream, const void* x, kvrq_dtype xdt, int64_t ldx,
                            const uint32_t* codes_in, uint32_t* codes_out, int64_t ldc, const float* norms_in,
                            float* norms_out, int64_t n, int d, const float* rotors, const float* centroids, int bits,
-                           void* xhat, kvrq_dtype odt, int64_t ldo) {
+                           void* xhat, kvrq_dtype odt, int64_t ldo, int64_t ldn = 1) {
+  if (ldn < 1) return set_errorf(KVRQ_EINVAL, "%s: norm row stride < 1", name);
   if (n < 0) return set_errorf(KVRQ_EINVAL, "%s: n < 0", name);
   if (d < 2 || d > (1 << 20)) return set_errorf(KVRQ_EINVAL, "%s: d must be in 2..2^20", name);
   if (bits < 1 || bits > 4) return set_errorf(KVRQ_EUNSUPPORTED, "%s: bits must be in 1..4", name);
@@ -185,6 +186,7 @@ static kvrq_status rq_call(const char* name, int mode, void* stream, const void*
   a.xhat = xhat;
   a.ldo = ldo;
   a.ldc = ldc;
+  a.ldn = ldn;
   a.status = di->status;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
@@ -213,8 +215,9 @@ static kvrq_status tq_call(const char* name, int mode, void* stream, const void*
                            int64_t n, int d, int m, const void* pi, const uint16_t* T, const float* centroids,
                            int bits, uint32_t* codes_out, const uint32_t* codes_in, int64_t ldc, uint32_t* signs_out,
                            const uint32_t* signs_in, int64_t lds, float* gammas_out, const float* gammas_in,
-                           float* norms_out, const float* norms_in, void* xhat, int64_t ldo) {
+                           float* norms_out, const float* norms_in, void* xhat, int64_t ldo, int64_t ldn = 1) {
   const bool prod = mode == TQ_PROD_Q || mode == TQ_DQ_PROD;
+  if (ldn < 1) return set_errorf(KVRQ_EINVAL, "%s: norm row stride < 1", name);
   const bool q_side = mode == TQ_MSE_Q || mode == TQ_MSE_QDQ || mode == TQ_PROD_Q;
   const bool out = mode == TQ_MSE_QDQ || mode == TQ_DQ_MSE || mode == TQ_DQ_PROD;
   if (n < 0) return set_errorf(KVRQ_EINVAL, "%s: n < 0", name);
@@ -273,6 +276,7 @@ static kvrq_status tq_call(const char* name, int mode, void* stream, const void*
   a.gammas_in = gammas_in;
   a.ldc = ldc;
   a.lds = lds;
+  a.ldn = ldn;
   a.status = di->status;
   return launch_status(name, launch_tq(mode, dt, cbits, mx, mp, mt, mo, a, static_cast<cudaStream_t>(stream), di->num_sms));
 }
@@ -392,11 +396,11 @@ kvrq_status kv_score_packed(void* stream, kvrq_method method, const void* q, kvr
   a.n_heads = n_heads;
   a.group = group;
   a.n_tokens = n_tokens;
-  // enough CTAs to fill the GPU a few times over, at most 64 tiles each
+  // about two CTAs per SM in total (one runs per SM): each CTA rotates its queries
+  // once, so long token ranges amortise that prologue
   int64_t tiles = (n_tokens + 127) / 128;
-  int64_t per = (tiles * n_heads + 4LL * di->num_sms - 1) / (4LL * di->num_sms);
-  if (per < 1) per = 1;
-  if (per > 64) per = 64;
+  int64_t per = (tiles * n_heads + 2LL * di->num_sms - 1) / (2LL * di->num_sms);
+  if (per < 4) per = 4;
   if (per > tiles) per = tiles;
   a.tokens_per_cta = per * 128;
   a.q = q;
@@ -423,6 +427,27 @@ kvrq_status kv_score_packed(void* stream, kvrq_method method, const void* q, kvr
   a.status = di->status;
   const int nb = rows_needed <= 16 ? 16 : (rows_needed <= 32 ? 32 : 64);
   return launch_status(name, launch_score(method, nb, cbits, a, static_cast<cudaStream_t>(stream)));
+}
+
+kvrq_status kv_cache_append(void* stream, kvrq_method method, const void* x, kvrq_dtype xdtype, int64_t n_rows,
+                            int d, int64_t ldx, int bits, const float* rotors, const void* pi, const uint16_t* T, int m,
+                            const float* centroids, uint32_t* codes, int64_t codes_row_stride, uint32_t* signs,
+                            int64_t signs_row_stride, float* norms, float* gammas, int64_t norm_row_stride) {
+  switch (method) {
+    case KVRQ_RQ_MSE:
+      return rq_call("kv_cache_append", RQ_Q, stream, x, xdtype, ldx, nullptr, codes, codes_row_stride, nullptr, norms,
+                     n_rows, d, rotors, centroids, bits, nullptr, xdtype, 0, norm_row_stride);
+    case KVRQ_TQ_MSE:
+      return tq_call("kv_cache_append", TQ_MSE_Q, stream, x, xdtype, ldx, n_rows, d, d, pi, nullptr, centroids, bits,
+                     codes, nullptr, codes_row_stride, nullptr, nullptr, 0, nullptr, nullptr, norms, nullptr, nullptr,
+                     0, norm_row_stride);
+    case KVRQ_TQ_PROD:
+      return tq_call("kv_cache_append", TQ_PROD_Q, stream, x, xdtype, ldx, n_rows, d, m, pi, T, centroids, bits, codes,
+                     nullptr, codes_row_stride, signs, nullptr, signs_row_stride, gammas, nullptr, norms, nullptr,
+                     nullptr, 0, norm_row_stride);
+    default:
+      return set_error(KVRQ_EINVAL, "kv_cache_append: unknown method");
+  }
 }
 
 }  // extern "C"

@@ -350,7 +350,7 @@ __global__ void __launch_bounds__(kRows, MODE == RQ_Q ? 2 : KVRQ_ROW_MIN_BLOCKS)
       nq = sqrtf(ss);
       nrm = kScale ? nq / xs : nq;
     } else {
-      nrm = tid < rows ? __ldg(a.norms_in + row) : 0.f;
+      nrm = tid < rows ? __ldg(a.norms_in + row * a.ldn) : 0.f;
       nq = nrm;
 #pragma unroll
       for (int w = 0; w < W; ++w) wc[w] = stage_codes[tid * W + w];
@@ -491,7 +491,7 @@ __global__ void __launch_bounds__(kRows, MODE == RQ_Q ? 2 : KVRQ_ROW_MIN_BLOCKS)
 
     // ---------------------------------------------------------------- outputs
     if constexpr (kIn) {
-      if (tid < rows && a.norms_out) a.norms_out[row] = nrm;
+      if (tid < rows && a.norms_out) a.norms_out[row * a.ldn] = nrm;
     }
     // a full tile of codes leaves as one bulk copy when code rows are contiguous
     const bool codes_bulk_out = kIn && a.codes_out && rows == kRows && a.ldc == W &&
@@ -565,9 +565,9 @@ __global__ void __launch_bounds__(256) rq_general_kernel(RqArgs a) {
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
       nrm = sqrtf(ss);
-      if (lane == 0 && a.norms_out) a.norms_out[row] = nrm;
+      if (lane == 0 && a.norms_out) a.norms_out[row * a.ldn] = nrm;
     } else {
-      nrm = __ldg(a.norms_in + row);
+      nrm = __ldg(a.norms_in + row * a.ldn);
     }
     Quantizer<BITS> q;
     q.scale(s_tau, s_mag, nrm);

@@ -28,6 +28,7 @@ struct RqArgs {
   void* xhat;
   int64_t ldo;
   int64_t ldc;  // row stride of codes (words), both directions
+  int64_t ldn;  // row stride of norms (floats), both directions
   unsigned* status;  // device status word (bounded-wait time-outs)
 };
 

@@ -8,15 +8,18 @@
 // directly from the compressed indices. For RotorQuant the same identity holds
 // per group: <q, x_hat> = ||x|| sum_g <R_g q_g R_g~, c_hat_g>, q zero-padded.
 //
-// B200 design: a CTA owns one KV head and a contiguous token range. It rotates
-// the head's query group once (Pi q and T Pi q, or the per-group sandwich) and
-// writes it as the MMA B operand (N = 16.. rows, fp16). Then, per 128-token
-// tile: packed code rows arrive by bulk copy (double-buffered), each thread
-// decodes one token through small shared-memory tables (several codes per
-// lookup) into a 128-byte-swizzled fp16 A tile (centroids, then +1/-1 signs for
-// TurboQuant-prod), one thread issues tcgen05.mma (M = 128 tokens), and the
-// epilogue reads one TMEM lane per token, applies ||k|| (and the QJL term) and
-// writes fp32 scores coalesced across tokens.
+// B200 design: a CTA of 256 threads owns one KV head and a contiguous token
+// range. It rotates the head's query group once (Pi q and T Pi q from staged
+// copies of Pi and T, or the per-group sandwich) into the MMA B operand (N = 16..
+// rows, fp16). Then, per 128-token tile: packed code rows arrive by bulk copy
+// (a ring of eight tiles in flight); the two warpgroups decode the tile's keys into a
+// 128-byte-swizzled fp16 A tile (warpgroup 0 the first half of K, warpgroup 1
+// the second: for TurboQuant-prod the centroids and the +1/-1 signs) through
+// small shared-memory tables; one thread issues tcgen05.mma (M = 128 tokens)
+// into one of two TMEM accumulators; while it runs, warpgroup 1 finishes the
+// previous tile (one TMEM lane per token: ||k|| and the QJL term, fp32 scores
+// written coalesced across tokens) and both warpgroups decode the next one into
+// the other A buffer.
 
 #include <cuda_runtime.h>
 
@@ -28,16 +31,18 @@
 namespace kvrq {
 namespace score {
 
-constexpr int kRows = 128;  // tokens per tile = threads per CTA
+constexpr int kRows = 128;     // tokens per tile
+constexpr int kThreads = 256;  // two warpgroups
+constexpr int kStages = 8;     // packed-code tiles in flight per CTA
 
 // Codes per lookup for a stored code width b: the table maps a field of
 // kPer * b bits to kPer fp16 centroids.
 template <int BITS>
 struct Dec {
   static constexpr int kPer = BITS == 1 ? 8 : BITS == 2 ? 4 : 2;
-  static constexpr int kFieldBits = kPer * BITS;      // 8, 8, 6, 8
-  static constexpr int kEntries = 1 << kFieldBits;    // 256, 256, 64, 256
-  static constexpr int kEntryBytes = kPer * 2;        // 16, 8, 4, 4
+  static constexpr int kFieldBits = kPer * BITS;    // 8, 8, 6, 8
+  static constexpr int kEntries = 1 << kFieldBits;  // 256, 256, 64, 256
+  static constexpr int kEntryBytes = kPer * 2;      // 16, 8, 4, 4
 };
 
 template <int METHOD, int BITS, int NB>
@@ -51,28 +56,34 @@ struct Cfg {
   static constexpr int W = (NCODE * BITS + 31) / 32;                // code words per key
   static constexpr int NS = kProd ? 4 : 0;                          // sign words per key (m = 128)
   static constexpr int A_BOX = kRows * 128;                         // A: box of 128 rows
+  static constexpr int A_BYTES = KBOX * A_BOX;
   static constexpr int B_BOX = NB * 128;                            // B: box of NB rows
   static constexpr int QS = D + 16;                                 // row stride of the query scratch
   static constexpr int q_bytes = 2 * NB * QS * 4;                   // fp32 rotated queries (prologue only)
-  static constexpr int a_bytes = KBOX * A_BOX > q_bytes ? KBOX * A_BOX : q_bytes;
-  static constexpr int a_off = 0;                                   // the query scratch aliases the A tile
-  static constexpr int q_off = 0;
-  static constexpr int b_off = a_off + ((a_bytes + 1023) / 1024) * 1024;
+  static constexpr int MS = 130;                                    // padded row (halves) of a staged matrix
+  static constexpr int m_off = ((q_bytes + 15) / 16) * 16;          // staged Pi or T (prologue only)
+  static constexpr int pro_bytes = m_off + D * MS * 2;
+  static constexpr int a_bytes = 2 * A_BYTES > pro_bytes ? 2 * A_BYTES : pro_bytes;
+  static constexpr int a_off = 0;  // two A buffers; the prologue scratch aliases them
+  static constexpr int b_off = ((a_bytes + 1023) / 1024) * 1024;
   static constexpr int stage_words = ((kRows * (W + NS) + 3) / 4) * 4;  // codes then signs, per tile
   static constexpr int stage_off = b_off + KBOX * B_BOX;
-  static constexpr int lut_off = stage_off + 2 * stage_words * 4;
+  static constexpr int lut_off = stage_off + kStages * stage_words * 4;
   static constexpr int lut_bytes = Dec<BITS>::kEntries * Dec<BITS>::kEntryBytes;
   static constexpr int slut_off = lut_off + lut_bytes;  // sign table: byte -> 8 x (+1/-1)
   static constexpr int slut_bytes = kProd ? 256 * 16 : 0;
-  static constexpr int bar_off = slut_off + slut_bytes;
-  static constexpr int tmem_off = bar_off + 4 * 8;
+  static constexpr int bar_off = slut_off + slut_bytes;  // [0, kStages) code stages, then 2 mma buffers
+  static constexpr int tmem_off = bar_off + (kStages + 2) * 8;
   static constexpr int bytes = tmem_off + 16;
   static constexpr int alloc = bytes + 1024;
-  static constexpr uint32_t kNcols = NB < 32 ? 32 : NB;
+  static constexpr uint32_t kNcols = 2 * NB < 32 ? 32 : 2 * NB;  // two accumulators
+  // K columns of the centroid part decoded by warpgroup 0 (the rest by warpgroup 1);
+  // for prod warpgroup 0 decodes all centroids and warpgroup 1 the signs
+  static constexpr int KSPLIT = kProd ? KC : (KC / 16) * 8;
 };
 
 template <int METHOD, int BITS, int NB>
-__global__ void __launch_bounds__(kRows, 1) score_kernel(ScoreArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs a) {
   using C = Cfg<METHOD, BITS, NB>;
   using DC = Dec<BITS>;
   constexpr int D = C::D, K = C::K, KC = C::KC, W = C::W, NS = C::NS;
@@ -86,11 +97,12 @@ __global__ void __launch_bounds__(kRows, 1) score_kernel(ScoreArgs a) {
   uint32_t* s_stage = reinterpret_cast<uint32_t*>(smem + C::stage_off);
   uint8_t* s_lut = smem + C::lut_off;
   uint8_t* s_slut = smem + C::slut_off;
-  float* s_q = reinterpret_cast<float*>(smem + C::q_off);
-  uint64_t* s_bar = reinterpret_cast<uint64_t*>(smem + C::bar_off);  // [0,1] code stages, [2] mma
+  float* s_q = reinterpret_cast<float*>(smem);
+  uint64_t* s_bar = reinterpret_cast<uint64_t*>(smem + C::bar_off);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::tmem_off);
 
   const int tid = threadIdx.x, warp = tid >> 5;
+  const int wg = tid >> 7, key = tid & 127;  // warpgroup, token within the tile
   const int G = a.group;
   const int64_t head = blockIdx.y;
   const int64_t t_begin = (int64_t)blockIdx.x * a.tokens_per_cta;
@@ -105,7 +117,7 @@ __global__ void __launch_bounds__(kRows, 1) score_kernel(ScoreArgs a) {
                     (!kProd || (reinterpret_cast<uintptr_t>(signs_h) & 15) == 0) && ((kRows * W * 4) % 16 == 0);
 
   if (tid == 0) {
-    for (int s = 0; s < 3; ++s) mbar_init(&s_bar[s], 1);
+    for (int s = 0; s < kStages + 2; ++s) mbar_init(&s_bar[s], 1);
     fence_barrier_init();
   }
   if (warp == 0) tmem_alloc(s_tmem, C::kNcols);
@@ -113,36 +125,35 @@ __global__ void __launch_bounds__(kRows, 1) score_kernel(ScoreArgs a) {
   // ---------------------------------------------------------------- decode tables
   {
     const float* cb = a.centroids;
-    for (int e = tid; e < DC::kEntries; e += kRows) {
-      __half h[DC::kPer];
+    for (int e = tid; e < DC::kEntries; e += kThreads) {
 #pragma unroll
-      for (int j = 0; j < DC::kPer; ++j) h[j] = __float2half_rn(cb[(e >> (j * BITS)) & ((1 << BITS) - 1)]);
-#pragma unroll
-      for (int j = 0; j < DC::kPer; ++j) reinterpret_cast<__half*>(s_lut + e * DC::kEntryBytes)[j] = h[j];
+      for (int j = 0; j < DC::kPer; ++j)
+        reinterpret_cast<__half*>(s_lut + e * DC::kEntryBytes)[j] =
+            __float2half_rn(cb[(e >> (j * BITS)) & ((1 << BITS) - 1)]);
     }
     if (kProd)
-      for (int e = tid; e < 256; e += kRows)
+      for (int e = tid; e < 256; e += kThreads)
 #pragma unroll
         for (int j = 0; j < 8; ++j)
           reinterpret_cast<__half*>(s_slut + e * 16)[j] = __float2half_rn(((e >> j) & 1) ? 1.f : -1.f);
   }
 
   // ---------------------------------------------------------------- rotated queries
-  // s_q[g][i] (fp32): q' = rotated query g; for prod also s_q[G + g][j] = (T q')_j
-  const int Gp = kProd ? NB / 2 : NB;  // B rows per part
-  for (int idx = tid; idx < G * D; idx += kRows) {
+  // s_q rows [0, G): q' (fp32); rows [NB, NB + G): the raw queries, later (T q')
+  const int Gp = kProd ? NB / 2 : NB;  // B rows of the centroid part
+  for (int idx = tid; idx < G * D; idx += kThreads) {
     const int g = idx / D, i = idx - g * D;
     float v = 0.f;
     const int64_t qrow = (head * G + g) * a.ldq;
     if (a.q_f32) v = reinterpret_cast<const float*>(a.q)[qrow + i];
     else if (a.q_bf16) v = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.q)[qrow + i]);
     else v = __half2float(reinterpret_cast<const __half*>(a.q)[qrow + i]);
-    s_q[(NB + g) * C::QS + i] = v;  // raw query in the spare rows
+    s_q[(NB + g) * C::QS + i] = v;
   }
   __syncthreads();
   if (METHOD == KVRQ_RQ_MSE) {
     // per group: y = M q_g (zero pad beyond d), 3G = 129 coordinates
-    for (int idx = tid; idx < G * 43; idx += kRows) {
+    for (int idx = tid; idx < G * 43; idx += kThreads) {
       const int g = idx / 43, grp = idx - g * 43;
       const float4 r = __ldg(reinterpret_cast<const float4*>(a.rotors) + grp);
       float m[9];
@@ -156,34 +167,61 @@ __global__ void __launch_bounds__(kRows, 1) score_kernel(ScoreArgs a) {
         s_q[g * C::QS + 3 * grp + i] = fmaf(m[3 * i + 2], v[2], fmaf(m[3 * i + 1], v[1], m[3 * i] * v[0]));
     }
   } else {
-    // q' = Pi q (row i of Pi times q)
-    for (int idx = tid; idx < G * D; idx += kRows) {
-      const int g = idx / D, i = idx - g * D;
-      const float* qr = s_q + (NB + g) * C::QS;
-      float acc = 0.f;
-      for (int k = 0; k < D; ++k) {
-        const float p = a.pi_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.pi)[i * D + k])
-                                  : __half2float(reinterpret_cast<const __half*>(a.pi)[i * D + k]);
-        acc = fmaf(p, qr[k], acc);
+    // q' = Pi q: Pi staged in shared memory (coalesced 16-byte loads, padded rows), then
+    // thread i < 128 forms row i of Pi against every query of the group
+    uint16_t* s_m = reinterpret_cast<uint16_t*>(smem + C::m_off);
+    auto stage = [&](const void* src) {
+      const uint4* g = reinterpret_cast<const uint4*>(src);
+      for (int i = tid; i < D * D / 8; i += kThreads) {
+        const uint4 v = __ldg(g + i);
+        uint32_t* d32 = reinterpret_cast<uint32_t*>(s_m + (i / 16) * C::MS + (i % 16) * 8);
+        d32[0] = v.x;
+        d32[1] = v.y;
+        d32[2] = v.z;
+        d32[3] = v.w;
       }
-      s_q[g * C::QS + i] = acc;
+    };
+    // out[g][i] = sum_k M[i][k] vec[g][k], one (g, i) per thread and step: a warp covers
+    // consecutive i of one g (conflict-free padded rows, broadcast vector)
+    auto mat_vec = [&](bool bf16, const float* vec_base, float* out_base) {
+      for (int idx = tid; idx < G * D; idx += kThreads) {
+        const int g = idx / D, i = idx - g * D;
+        const uint32_t* row = reinterpret_cast<const uint32_t*>(s_m + i * C::MS);
+        const float* vec = vec_base + g * C::QS;
+        float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 8
+        for (int k = 0; k < D; k += 2) {
+          const uint32_t w = row[k / 2];
+          float p0, p1;
+          if (bf16) {
+            p0 = __uint_as_float(w << 16);
+            p1 = __uint_as_float(w & 0xFFFF0000u);
+          } else {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w));
+            p0 = f.x;
+            p1 = f.y;
+          }
+          const float2 qv = *reinterpret_cast<const float2*>(vec + k);
+          acc0 = fmaf(p0, qv.x, acc0);
+          acc1 = fmaf(p1, qv.y, acc1);
+        }
+        out_base[g * C::QS + i] = acc0 + acc1;
+      }
+    };
+    stage(a.pi);
+    __syncthreads();
+    mat_vec(a.pi_bf16, s_q + NB * C::QS, s_q);
+    __syncthreads();
+    if (kProd) {
+      stage(a.T);
+      __syncthreads();
+      mat_vec(false, s_q, s_q + NB * C::QS);
     }
   }
   __syncthreads();
-  if (kProd) {
-    // (T q')_j into the spare rows (the raw queries are no longer needed)
-    for (int idx = tid; idx < G * D; idx += kRows) {
-      const int g = idx / D, j = idx - g * D;
-      const float* qp = s_q + g * C::QS;
-      float acc = 0.f;
-      for (int k = 0; k < D; ++k) acc = fmaf(__half2float(reinterpret_cast<const __half*>(a.T)[j * D + k]), qp[k], acc);
-      s_q[(NB + g) * C::QS + j] = acc;
-    }
-    __syncthreads();
-  }
   // B operand [NB rows][K] fp16, 128-byte swizzled, K-major: row g < G holds q'_g over the
   // centroid part; for prod row Gp + g holds (T q')_g over the sign part; all else zero.
-  for (int idx = tid; idx < NB * (C::KBOX * 8); idx += kRows) {
+  for (int idx = tid; idx < NB * (C::KBOX * 8); idx += kThreads) {
     const int row = idx / (C::KBOX * 8), j = idx - row * (C::KBOX * 8);  // 16-byte chunk j of the row
     float v[8];
 #pragma unroll
@@ -199,15 +237,15 @@ __global__ void __launch_bounds__(kRows, 1) score_kernel(ScoreArgs a) {
     }
     *reinterpret_cast<uint4*>(s_b + sw128_chunk(row, j, C::B_BOX)) = Elem<__half>::pack(v);
   }
-  __syncthreads();  // the query scratch (aliasing the A tile) has been read
-  // zero the A tile once (its unused K columns stay zero)
-  for (int i = tid; i < C::KBOX * C::A_BOX / 16; i += kRows) reinterpret_cast<uint4*>(s_a)[i] = make_uint4(0, 0, 0, 0);
+  __syncthreads();  // the prologue scratch (aliasing the A buffers) has been read
+  // zero both A buffers once (their unused K columns stay zero)
+  for (int i = tid; i < 2 * C::A_BYTES / 16; i += kThreads) reinterpret_cast<uint4*>(s_a)[i] = make_uint4(0, 0, 0, 0);
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
   const uint32_t a_s = smem_u32(s_a), b_s = smem_u32(s_b);
 
   auto tile_full = [&](int it) { return t_begin + (int64_t)(it + 1) * kRows <= t_end; };
@@ -220,48 +258,77 @@ __global__ void __launch_bounds__(kRows, 1) score_kernel(ScoreArgs a) {
   };
   uint32_t par = 0;  // bit s: parity of the next phase of barrier s
   if (tid == 0 && bulk)
-    for (int it = 0; it < 2 && it < ntiles; ++it)
+    for (int it = 0; it < kStages && it < ntiles; ++it)
       if (tile_full(it)) issue_stage(it, it);
 
+  // epilogue of tile `pt` (warpgroup 1): scores from accumulator pt & 1
+  auto epilogue = [&](int pt, float nrm, float gam) {
+    const int64_t t0 = t_begin + (int64_t)pt * kRows;
+    const int rows = (int)(t_end - t0 < (int64_t)kRows ? t_end - t0 : (int64_t)kRows);
+    const int64_t t = t0 + key;
+    // NB columns of accumulator pt & 1 (a multiple of 16; never past the allocation)
+    float acc[NB];
+#pragma unroll
+    for (int c = 0; c < NB / 16; ++c) tmem_ld16(tmem + lane_off + (uint32_t)((pt & 1) * NB) + 16 * c, &acc[16 * c]);
+    if (key < rows) {
+      const float qs = a.qjl_scale * gam;
+#pragma unroll
+      for (int g = 0; g < (kProd ? NB / 2 : NB); ++g) {
+        if (g < G) {
+          float s = acc[g];
+          if (kProd) s = fmaf(qs, acc[NB / 2 + g], s);
+          a.scores[(head * G + g) * a.ld_scores + t] = nrm * s;
+        }
+      }
+    }
+  };
+
   bool ok = true;
+  float prev_n = 0.f, prev_g = 0.f;  // norm / gamma of this thread's key in the previous tile
   for (int it = 0; it < ntiles; ++it) {
-    const int st = it & 1;
+    const int st = it % kStages, ab = it & 1;
+    constexpr int MB = kStages;  // first mma-buffer barrier
     const int64_t t0 = t_begin + (int64_t)it * kRows;
     const int rows = (int)(t_end - t0 < (int64_t)kRows ? t_end - t0 : (int64_t)kRows);
-    const int64_t t = t0 + tid;
     uint32_t* stg = s_stage + st * C::stage_words;
-    const float nrm = tid < rows ? __ldg(norms_h + t) : 0.f;
-    const float gam = (kProd && tid < rows) ? __ldg(gammas_h + t) : 0.f;
+    uint8_t* A = s_a + ab * C::A_BYTES;
+    const float nrm = (wg == 1 && key < rows) ? __ldg(norms_h + t0 + key) : 0.f;
+    const float gam = (kProd && wg == 1 && key < rows) ? __ldg(gammas_h + t0 + key) : 0.f;
     if (bulk && tile_full(it)) {
-      ok = mbar_wait(&s_bar[st], (par >> st) & 1, a.status);
+      ok = mbar_wait(&s_bar[st], (par >> st) & 1, a.status) && ok;
       par ^= 1u << st;
     } else {
-      for (int i = tid; i < rows * W; i += kRows) {
+      for (int i = tid; i < rows * W; i += kThreads) {
         const int r = i / W, w = i - r * W;
         stg[i] = __ldg(codes_h + (t0 + r) * a.ldc + w);
       }
       if (kProd)
-        for (int i = tid; i < rows * NS; i += kRows) {
+        for (int i = tid; i < rows * NS; i += kThreads) {
           const int r = i / NS, w = i - r * NS;
           stg[kRows * W + i] = __ldg(signs_h + (t0 + r) * a.lds + w);
         }
-      for (int i = rows * W + tid; i < kRows * W; i += kRows) stg[i] = 0u;  // ragged tail: decode zeros
+      for (int i = rows * W + tid; i < kRows * W; i += kThreads) stg[i] = 0u;  // ragged tail decodes to zero
+      if (kProd)
+        for (int i = rows * NS + tid; i < kRows * NS; i += kThreads) stg[kRows * W + i] = 0u;
     }
     if (!__syncthreads_and(ok)) break;
 
-    // ------------------------------------------------------------ decode this thread's key
-    uint32_t wc[W];
-#pragma unroll
-    for (int w = 0; w < W; ++w) wc[w] = stg[tid * W + w];
-    {
-      // fields of P codes -> P fp16 centroids (P/2 words); codes past the stored ones are zero
+    // ------------------------------------------------------------ decode key `key` into A[ab]
+    if (!kProd || wg == 0) {
       constexpr int P = DC::kPer, FB = DC::kFieldBits;
       constexpr int NF = (C::NCODE + P - 1) / P;
+      uint32_t wc[W];
+#pragma unroll
+      for (int w = 0; w < W; ++w) wc[w] = stg[key * W + w];
       uint32_t rw[KC / 2];
 #pragma unroll
       for (int k = 0; k < KC / 2; ++k) rw[k] = 0u;
+      // fields of warpgroup 0 (or, for prod, all) / of warpgroup 1
+      const int f_lo = (kProd || wg == 0) ? 0 : C::KSPLIT / P;
+      const int f_hi = (kProd || wg == 1) ? NF : C::KSPLIT / P;
 #pragma unroll
       for (int f = 0; f < NF; ++f) {
+        if (f < f_lo || f >= f_hi) continue;
         const int bit = f * FB, word = bit >> 5, sh = bit & 31;
         uint32_t v = wc[word] >> sh;
         if (sh + FB > 32 && word + 1 < W) v |= wc[word + 1] << (32 - sh);
@@ -277,18 +344,22 @@ __global__ void __launch_bounds__(kRows, 1) score_kernel(ScoreArgs a) {
         }
       }
 #pragma unroll
-      for (int j = 0; j < KC / 8; ++j)
-        *reinterpret_cast<uint4*>(s_a + sw128_chunk(tid, j, C::A_BOX)) =
-            make_uint4(rw[4 * j], rw[4 * j + 1], rw[4 * j + 2], rw[4 * j + 3]);
+      for (int j = 0; j < KC / 8; ++j) {
+        const bool mine = kProd ? true : (wg == 0 ? (8 * j < C::KSPLIT) : (8 * j >= C::KSPLIT));
+        if (mine)
+          *reinterpret_cast<uint4*>(A + sw128_chunk(key, j, C::A_BOX)) =
+              make_uint4(rw[4 * j], rw[4 * j + 1], rw[4 * j + 2], rw[4 * j + 3]);
+      }
     }
-    if constexpr (kProd) {
+    if (kProd && wg == 1) {
+      // sign part: each byte of signs -> 8 x (+1/-1) fp16
 #pragma unroll
       for (int w = 0; w < NS; ++w) {
-        const uint32_t sw = stg[kRows * W + tid * NS + w];
+        const uint32_t sw = stg[kRows * W + key * NS + w];
 #pragma unroll
         for (int bt = 0; bt < 4; ++bt) {
           const uint4 e = *reinterpret_cast<const uint4*>(s_slut + ((sw >> (8 * bt)) & 0xFF) * 16);
-          *reinterpret_cast<uint4*>(s_a + sw128_chunk(tid, KC / 8 + w * 4 + bt, C::A_BOX)) = e;
+          *reinterpret_cast<uint4*>(A + sw128_chunk(key, KC / 8 + w * 4 + bt, C::A_BOX)) = e;
         }
       }
     }
@@ -296,44 +367,37 @@ __global__ void __launch_bounds__(kRows, 1) score_kernel(ScoreArgs a) {
     tc_fence_before();
     __syncthreads();
     if (tid == 0) {
-      // refill this code stage two tiles ahead (every thread has read it)
-      if (bulk && it + 2 < ntiles && tile_full(it + 2)) issue_stage(it + 2, st);
+      // refill this code stage kStages tiles ahead (every thread has read it)
+      if (bulk && it + kStages < ntiles && tile_full(it + kStages)) issue_stage(it + kStages, st);
       tc_fence_after();
+      const uint32_t a_buf = a_s + (uint32_t)(ab * C::A_BYTES);
 #pragma unroll
       for (int kk = 0; kk < K / 16; ++kk) {
         const uint32_t off = (uint32_t)((kk >> 2) * C::A_BOX + (kk & 3) * 32);
         const uint32_t boff = (uint32_t)((kk >> 2) * C::B_BOX + (kk & 3) * 32);
-        umma_f16(tmem, umma_desc_sw128(a_s + off, 16, 1024), umma_desc_sw128(b_s + boff, 16, 1024), kIdesc, kk > 0);
+        umma_f16(tmem + (uint32_t)(ab * NB), umma_desc_sw128(a_buf + off, 16, 1024),
+                 umma_desc_sw128(b_s + boff, 16, 1024), kIdesc, kk > 0);
       }
-      umma_commit(&s_bar[2]);
+      umma_commit(&s_bar[MB + ab]);
     }
-    ok = mbar_wait(&s_bar[2], (par >> 2) & 1, a.status) && ok;
-    par ^= 4u;
-    tc_fence_after();
-
-    // ------------------------------------------------------------ epilogue: one token per thread
-    float acc[NB];
-#pragma unroll
-    for (int c = 0; c < NB / 32 + (NB % 32 ? 1 : 0); ++c) {
-      float v[32];
-      tmem_ld32(tmem + lane_off + 32 * c, v);
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (32 * c + i < NB) acc[32 * c + i] = v[i];
+    // finish the previous tile while this one's MMA runs; its MMA is complete
+    // before the next decode overwrites its A buffer
+    if (it > 0) {
+      ok = mbar_wait(&s_bar[MB + (ab ^ 1)], (par >> (MB + (ab ^ 1))) & 1, a.status) && ok;
+      par ^= 1u << (MB + (ab ^ 1));
+      tc_fence_after();
+      if (wg == 1) epilogue(it - 1, prev_n, prev_g);
     }
-    if (tid < rows) {
-      const float qs = a.qjl_scale * gam;
-#pragma unroll
-      for (int g = 0; g < (kProd ? NB / 2 : NB); ++g) {
-        if (g < G) {
-          float s = acc[g];
-          if (kProd) s = fmaf(qs, acc[NB / 2 + g], s);
-          a.scores[(head * G + g) * a.ld_scores + t] = nrm * s;
-        }
-      }
-    }
+    prev_n = nrm;
+    prev_g = gam;
     tc_fence_before();
-    __syncthreads();  // the A tile and TMEM are reused by the next tile
+  }
+  // the last tile
+  if (ok && ntiles > 0) {
+    const int lt = ntiles - 1;
+    ok = mbar_wait(&s_bar[kStages + (lt & 1)], (par >> (kStages + (lt & 1))) & 1, a.status);
+    tc_fence_after();
+    if (ok && wg == 1) epilogue(lt, prev_n, prev_g);
   }
   tc_fence_before();
   __syncthreads();
@@ -353,7 +417,7 @@ static cudaError_t launch_score_t(const ScoreArgs& a, cudaStream_t st) {
     attr = true;
   }
   dim3 grid((unsigned)((a.n_tokens + a.tokens_per_cta - 1) / a.tokens_per_cta), (unsigned)a.n_heads);
-  kern<<<grid, score::kRows, C::alloc, st>>>(a);
+  kern<<<grid, score::kThreads, C::alloc, st>>>(a);
   return cudaGetLastError();
 }
 

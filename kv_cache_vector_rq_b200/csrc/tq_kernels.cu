@@ -301,8 +301,8 @@ __global__ void __launch_bounds__(kRows, 1)
 #pragma unroll
       for (int w = 0; w < W; ++w) s_codes[tid * W + w] = wc[w];
       if (tid < rows) {
-        if (a.norms_out) a.norms_out[row] = nrm;
-        if (kProd && a.gammas_out) a.gammas_out[row] = sqrtf(gs);
+        if (a.norms_out) a.norms_out[row * a.ldn] = nrm;
+        if (kProd && a.gammas_out) a.gammas_out[row * a.ldn] = sqrtf(gs);
       }
 
       if constexpr (MODE == TQ_MSE_QDQ || MODE == TQ_PROD_Q) {
@@ -347,8 +347,8 @@ __global__ void __launch_bounds__(kRows, 1)
           const int r = i / NS, w = i - r * NS;
           s_signs[i] = __ldg(a.signs_in + (row0 + r) * a.lds + w);
         }
-      nrm = tid < rows ? __ldg(a.norms_in + row) : 0.f;
-      const float gam = (kProd && tid < rows) ? __ldg(a.gammas_in + row) : 0.f;
+      nrm = tid < rows ? __ldg(a.norms_in + row * a.ldn) : 0.f;
+      const float gam = (kProd && tid < rows) ? __ldg(a.gammas_in + row * a.ldn) : 0.f;
       if (tid == 0) bulk_wait_read<0>();
       if (!__syncthreads_and(ok)) break;
       uint32_t wc[W];

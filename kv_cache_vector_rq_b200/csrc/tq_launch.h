@@ -30,6 +30,7 @@ struct TqArgs {
   const float* gammas_in;
   int64_t ldc;  // code row stride (words)
   int64_t lds;  // sign row stride (words)
+  int64_t ldn;  // norm and gamma row stride (floats)
   unsigned* status;
 };
 
