@@ -162,33 +162,63 @@ kvrq_status rq_quantize_dequantize(void* stream, const void* x, kvrq_dtype xdtyp
  * rounded to fp16 (S = T Pi is the pages' Gaussian projection; sign(0) = +1),
  * x_hat = ||x|| Pi^T (c_hat + sqrt(pi/2)/m gamma T^T s).
  *
- * Tensor-core path: d = m = 128; x (and x_hat) fp16 or bf16 with Pi [d][d]
- * row-major in the same type; T [m][d] row-major fp16; all 16-byte aligned;
- * rows of x/x_hat 16-byte aligned. centroids: [2^b] (mse) or [2^(b-1)] (prod)
- * fp32, ascending and symmetric. codes [n][ldc] uint32 with
- * ldc >= kvrq_packed_words(d, b or b-1); signs [n][lds] uint32, lds >= m/32;
- * norms, gammas [n] fp32. Other shapes return KVRQ_EUNSUPPORTED.
+ * Two tensor-core paths, chosen by d and the vector type:
+ *  - d = m = 128, fp16 or bf16 vectors: one launch per call, Pi (and T) kept in
+ *    shared memory;
+ *  - d a multiple of 128 (fp16/bf16: d >= 256; fp32: any such d, d = 128
+ *    included), m = d: a tiled contraction that streams Pi / T, two launches
+ *    for the fused quantize + dequantize and for each prod call; the prod calls
+ *    pass the rotated residual (or the QJL-corrected centroids) between their
+ *    two launches through `workspace`, in blocks of rows.
+ * x (and x_hat) fp32, fp16 or bf16; Pi [d][d] row-major in the vector type
+ * (fp16 for fp32 vectors, which are split into fp16 hi + lo parts on the
+ * tensor cores); T [m][d] row-major fp16. Pi, T, x, x_hat and workspace
+ * 16-byte aligned, rows of x / x_hat 16-byte aligned. centroids: [2^b] (mse)
+ * or [2^(b-1)] (prod) fp32, ascending and symmetric. codes [n][ldc] uint32
+ * with ldc >= kvrq_packed_words(d, b or b-1); signs [n][lds] uint32,
+ * lds >= m/32; norms, gammas [n] fp32. Other shapes return KVRQ_EUNSUPPORTED.
  */
 kvrq_status tq_quantize_mse(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,
                             const void* pi, const float* centroids, int bits, uint32_t* codes, int64_t ldc,
                             float* norms);
 
-/* Fused quantize + dequantize (codes and norms may be NULL): one launch, two MMAs per tile. */
+/* Fused quantize + dequantize. At d = 128 (fp16/bf16) one launch with two MMAs
+ * per tile, and codes and norms may be NULL; on the tiled path the dequantize
+ * launch reads the codes and norms the quantize launch wrote, so both are
+ * required. */
 kvrq_status tq_quantize_dequantize_mse(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,
                                        const void* pi, const float* centroids, int bits, uint32_t* codes,
                                        int64_t ldc, float* norms, void* xhat, int64_t ldo);
 
-/* TurboQuant-prod quantize, b = bits in 2..5 total bits per coordinate. */
+/* Bytes of workspace the tiled prod path uses for `rows` rows at dimension d:
+ * rows * (4 d + 4 d / 128). A call given workspace_bytes processes its rows in
+ * blocks of floor(workspace_bytes / kvrq_tq_workspace_bytes(1, d) / 128) * 128
+ * rows (at least 128 rows must fit). The d = 128 fp16/bf16 path needs none. */
+size_t kvrq_tq_workspace_bytes(int64_t rows, int d);
+
+/* TurboQuant-prod quantize, b = bits in 2..5 total bits per coordinate.
+ * workspace: device buffer owned by the caller (NULL / 0 where none is needed),
+ * overwritten; calls sharing a workspace must be ordered on one stream. */
 kvrq_status tq_quantize_prod(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,
                              const void* pi, const uint16_t* T, int m, const float* centroids, int bits,
                              uint32_t* codes, int64_t ldc, uint32_t* signs, int64_t lds, float* gammas,
-                             float* norms);
+                             float* norms, void* workspace, size_t workspace_bytes);
 
-/* Dequantize mse (signs == NULL; bits = b) or prod (signs != NULL; bits = b total). */
+/* Dequantize mse (signs == NULL; bits = b) or prod (signs != NULL; bits = b
+ * total; workspace as for tq_quantize_prod). */
 kvrq_status tq_dequantize(void* stream, const uint32_t* codes, int64_t ldc, const uint32_t* signs, int64_t lds,
                           const float* gammas, const float* norms, int64_t n, int d, int m, int bits,
                           const void* pi, const uint16_t* T, const float* centroids, void* xhat, kvrq_dtype odtype,
-                          int64_t ldo);
+                          int64_t ldo, void* workspace, size_t workspace_bytes);
+
+/* The QJL map on its own [TQB "QJL 内积无偏估计（Theorem 2）"; RQ "How
+ * TurboQuant Works"]: for each row r of the [n][ldr] matrix, signs = sign(T r)
+ * (bit j = 1 for T_j . r >= 0) and gammas = ||r||. r fp32, fp16 or bf16; T [m][d]
+ * row-major in the type of r (fp16 for fp32 r, which is split into hi + lo
+ * parts). d a multiple of 64, m a multiple of 128; signs [n][lds] uint32 with
+ * lds >= m/32; gammas [n] at stride ldn. */
+kvrq_status qjl_sketch(void* stream, const void* r, kvrq_dtype rdtype, int64_t n, int d, int64_t ldr, const void* T,
+                       int m, uint32_t* signs, int64_t lds, float* gammas, int64_t ldn);
 
 /* ================================================================ scores from packed keys
  * [TQB "随机旋转（Lemma 1）": rotate the query once instead of every key;

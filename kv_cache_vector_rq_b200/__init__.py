@@ -191,15 +191,51 @@ def _tq_outputs(x_rows, d, cbits, device, codes, norms):
     return codes, norms
 
 
+def _pi_dtype(x_dtype):
+    """Operand type of Pi for vectors of x_dtype: the same 16-bit type, fp16 for fp32 vectors."""
+    torch = _torch()
+    return torch.float16 if x_dtype == torch.float32 else x_dtype
+
+
+def tq_workspace_bytes(rows, d):
+    """Bytes of workspace the tiled prod path uses for `rows` rows (kvrq_tq_workspace_bytes)."""
+    return int(lib().kvrq_tq_workspace_bytes(rows, d))
+
+
+def tq_needs_workspace(d, dtype):
+    """True when the prod calls at this d / vector dtype run on the tiled path and take a workspace."""
+    torch = _torch()
+    return d != 128 or dtype == torch.float32
+
+
+def tq_workspace(n, d, device, max_bytes=256 << 20):
+    """A workspace tensor for the prod calls: all n rows (rounded up to 128) if that fits in max_bytes,
+    else the largest multiple of 128 rows that does (at least 128)."""
+    torch = _torch()
+    per_row = tq_workspace_bytes(1, d)
+    rows = ((max(n, 1) + 127) // 128) * 128
+    rows = max(128, min(rows, (max_bytes // per_row) // 128 * 128))
+    return torch.empty((tq_workspace_bytes(rows, d),), dtype=torch.uint8, device=device)
+
+
+def _ws_args(workspace, n, d, dtype, device):
+    if not tq_needs_workspace(d, dtype):
+        return None, 0, None
+    if workspace is None:
+        workspace = tq_workspace(n, d, device)
+    return workspace.data_ptr(), workspace.numel() * workspace.element_size(), workspace
+
+
 def tq_quantize_mse(x, pi, centroids, bits, codes=None, norms=None, stream=None):
-    """TurboQuant-mse quantize rows of x [n, d]; pi [d, d] in x's dtype. Returns (codes, norms)."""
+    """TurboQuant-mse quantize rows of x [n, d]; pi [d, d] in x's dtype (fp16 for fp32 x).
+    Returns (codes, norms)."""
     torch = _torch()
     n, d = x.shape
     codes, norms = _tq_outputs(n, d, bits, x.device, codes, norms)
     xp, ldx = _rows(x, "x")
     cp, ldc = _rows(codes, "codes")
     _lib.check("tq_quantize_mse", lib().tq_quantize_mse(_stream(stream), xp, _dtype_code(x), n, d, ldx,
-                                                        _ptr(pi, "pi", x.dtype),
+                                                        _ptr(pi, "pi", _pi_dtype(x.dtype)),
                                                         _ptr(centroids, "centroids", torch.float32), bits, cp, ldc,
                                                         _ptr(norms, "norms", torch.float32)))
     return codes, norms
@@ -207,10 +243,11 @@ def tq_quantize_mse(x, pi, centroids, bits, codes=None, norms=None, stream=None)
 
 def tq_quantize_dequantize_mse(x, pi, centroids, bits, codes=None, norms=None, xhat=None, with_codes=True,
                                stream=None):
-    """Fused TurboQuant-mse roundtrip: returns (codes, norms, x_hat)."""
+    """TurboQuant-mse roundtrip: returns (codes, norms, x_hat). Outside d = 128 with 16-bit vectors the
+    codes and norms are always produced (the dequantize launch reads them)."""
     torch = _torch()
     n, d = x.shape
-    if with_codes:
+    if with_codes or tq_needs_workspace(d, x.dtype):
         codes, norms = _tq_outputs(n, d, bits, x.device, codes, norms)
     if xhat is None:
         xhat = torch.empty_like(x)
@@ -218,14 +255,16 @@ def tq_quantize_dequantize_mse(x, pi, centroids, bits, codes=None, norms=None, x
     cp, ldc = _rows(codes, "codes") if codes is not None else (None, packed_words(d, bits))
     op, ldo = _rows(xhat, "xhat")
     _lib.check("tq_quantize_dequantize_mse", lib().tq_quantize_dequantize_mse(
-        _stream(stream), xp, _dtype_code(x), n, d, ldx, _ptr(pi, "pi", x.dtype),
+        _stream(stream), xp, _dtype_code(x), n, d, ldx, _ptr(pi, "pi", _pi_dtype(x.dtype)),
         _ptr(centroids, "centroids", torch.float32), bits, cp, ldc, _ptr(norms, "norms", torch.float32), op, ldo))
     return codes, norms, xhat
 
 
-def tq_quantize_prod(x, pi, T, centroids, bits, codes=None, norms=None, signs=None, gammas=None, stream=None):
+def tq_quantize_prod(x, pi, T, centroids, bits, codes=None, norms=None, signs=None, gammas=None, workspace=None,
+                     stream=None):
     """TurboQuant-prod quantize (bits total: bits-1 mse bits + 1 QJL bit); T [m, d] fp16.
-    Returns (codes, signs, gammas, norms)."""
+    `workspace` (uint8 device tensor, see tq_workspace) is allocated here when the tiled path needs one
+    and none is given. Returns (codes, signs, gammas, norms)."""
     torch = _torch()
     n, d = x.shape
     m = T.shape[0]
@@ -237,29 +276,50 @@ def tq_quantize_prod(x, pi, T, centroids, bits, codes=None, norms=None, signs=No
     xp, ldx = _rows(x, "x")
     cp, ldc = _rows(codes, "codes")
     sp, lds = _rows(signs, "signs")
+    wp, wbytes, _keep = _ws_args(workspace, n, d, x.dtype, x.device)
     _lib.check("tq_quantize_prod", lib().tq_quantize_prod(
-        _stream(stream), xp, _dtype_code(x), n, d, ldx, _ptr(pi, "pi", x.dtype), _ptr(T, "T", torch.float16), m,
-        _ptr(centroids, "centroids", torch.float32), bits, cp, ldc, sp, lds, _ptr(gammas, "gammas", torch.float32),
-        _ptr(norms, "norms", torch.float32)))
+        _stream(stream), xp, _dtype_code(x), n, d, ldx, _ptr(pi, "pi", _pi_dtype(x.dtype)),
+        _ptr(T, "T", torch.float16), m, _ptr(centroids, "centroids", torch.float32), bits, cp, ldc, sp, lds,
+        _ptr(gammas, "gammas", torch.float32), _ptr(norms, "norms", torch.float32), wp, wbytes))
     return codes, signs, gammas, norms
 
 
-def tq_dequantize(codes, norms, d, pi, centroids, bits, signs=None, gammas=None, T=None, xhat=None, stream=None):
+def tq_dequantize(codes, norms, d, pi, centroids, bits, signs=None, gammas=None, T=None, xhat=None,
+                  out_dtype=None, workspace=None, stream=None):
     """TurboQuant dequantize: mse when signs is None, prod otherwise (bits = total bits).
-    The output dtype is pi's dtype."""
+    The output dtype is out_dtype (default: pi's dtype; fp32 output takes an fp16 pi)."""
     torch = _torch()
     n = codes.shape[0]
     if xhat is None:
-        xhat = torch.empty((n, d), dtype=pi.dtype, device=codes.device)
+        xhat = torch.empty((n, d), dtype=out_dtype or pi.dtype, device=codes.device)
     m = T.shape[0] if T is not None else d
     cp, ldc = _rows(codes, "codes")
     sp, lds = _rows(signs, "signs") if signs is not None else (None, 0)
     op, ldo = _rows(xhat, "xhat")
+    wp, wbytes, _keep = (None, 0, None) if signs is None else _ws_args(workspace, n, d, xhat.dtype, codes.device)
     _lib.check("tq_dequantize", lib().tq_dequantize(
         _stream(stream), cp, ldc, sp, lds, _ptr(gammas, "gammas", torch.float32), _ptr(norms, "norms", torch.float32),
-        n, d, m, bits, _ptr(pi, "pi", xhat.dtype), _ptr(T, "T", torch.float16),
-        _ptr(centroids, "centroids", torch.float32), op, _dtype_code(xhat), ldo))
+        n, d, m, bits, _ptr(pi, "pi", _pi_dtype(xhat.dtype)), _ptr(T, "T", torch.float16),
+        _ptr(centroids, "centroids", torch.float32), op, _dtype_code(xhat), ldo, wp, wbytes))
     return xhat
+
+
+def qjl_sketch(r, T, signs=None, gammas=None, stream=None):
+    """QJL sign sketch of the rows of r [n, d]: signs = sign(T r) packed (m/32 words per row), gammas = ||r||.
+    T [m, d] in r's dtype (fp16 for fp32 r). Returns (signs, gammas)."""
+    torch = _torch()
+    n, d = r.shape
+    m = T.shape[0]
+    if signs is None:
+        signs = torch.empty((n, m // 32), dtype=torch.int32, device=r.device)
+    if gammas is None:
+        gammas = torch.empty((n,), dtype=torch.float32, device=r.device)
+    rp, ldr = _rows(r, "r")
+    sp, lds = _rows(signs, "signs")
+    _lib.check("qjl_sketch", lib().qjl_sketch(_stream(stream), rp, _dtype_code(r), n, d, ldr,
+                                              _ptr(T, "T", _pi_dtype(r.dtype)), m, sp, lds,
+                                              _ptr(gammas, "gammas", torch.float32), 1))
+    return signs, gammas
 
 
 # ----------------------------------------------------------------------------- scores

@@ -39,12 +39,18 @@ SIGNATURES = {
     # ... + xhat, ldo
     "tq_quantize_dequantize_mse": (c_int, [c_vp, c_vp, c_int, c_i64, c_int, c_i64, c_vp, c_vp, c_int, c_vp, c_i64,
                                            c_vp, c_vp, c_i64]),
-    # stream, x, xdtype, n, d, ldx, pi, T, m, centroids, bits, codes, ldc, signs, lds, gammas, norms
+    # rows, d
+    "kvrq_tq_workspace_bytes": (ctypes.c_size_t, [c_i64, c_int]),
+    # stream, x, xdtype, n, d, ldx, pi, T, m, centroids, bits, codes, ldc, signs, lds, gammas, norms, workspace,
+    # workspace_bytes
     "tq_quantize_prod": (c_int, [c_vp, c_vp, c_int, c_i64, c_int, c_i64, c_vp, c_vp, c_int, c_vp, c_int, c_vp, c_i64,
-                                 c_vp, c_i64, c_vp, c_vp]),
-    # stream, codes, ldc, signs, lds, gammas, norms, n, d, m, bits, pi, T, centroids, xhat, odtype, ldo
+                                 c_vp, c_i64, c_vp, c_vp, c_vp, ctypes.c_size_t]),
+    # stream, codes, ldc, signs, lds, gammas, norms, n, d, m, bits, pi, T, centroids, xhat, odtype, ldo, workspace,
+    # workspace_bytes
     "tq_dequantize": (c_int, [c_vp, c_vp, c_i64, c_vp, c_i64, c_vp, c_vp, c_i64, c_int, c_int, c_int, c_vp, c_vp,
-                              c_vp, c_vp, c_int, c_i64]),
+                              c_vp, c_vp, c_int, c_i64, c_vp, ctypes.c_size_t]),
+    # stream, r, rdtype, n, d, ldr, T, m, signs, lds, gammas, ldn
+    "qjl_sketch": (c_int, [c_vp, c_vp, c_int, c_i64, c_int, c_i64, c_vp, c_int, c_vp, c_i64, c_vp, c_i64]),
     # stream, method, q, qdtype, ldq, n_heads, group, d, bits, m, codes, ldc, codes_head_stride, signs, lds,
     # signs_head_stride, norms, gammas, tok_head_stride, n_tokens, rotors, pi, pi_dtype, T, centroids, scores,
     # ld_scores

@@ -14,6 +14,7 @@
 #include "kvrq_internal.h"
 #include "rq_launch.h"
 #include "tq_launch.h"
+#include "tqg_launch.h"
 #include "score_launch.h"
 
 namespace kvrq {
@@ -209,13 +210,145 @@ static kvrq_status rq_call(const char* name, int mode, void* stream, const void*
 }
 
 
-// Shared validation and dispatch of the TurboQuant calls (tensor-core path:
-// d = m = 128, 16-bit x and Pi of the same type, fp16 T, 16-byte aligned rows).
+static int tile_n(int n_total) { return n_total % 256 == 0 ? 256 : 128; }
+
+static size_t tq_ws_row_bytes(int d) { return (size_t)4 * d + (size_t)4 * (d / 128); }
+
+// Tiled TurboQuant path (tqg_kernels.cu): every d that is a multiple of 128,
+// fp32 vectors included. Arguments are validated by tq_call.
+static kvrq_status tqg_call(const char* name, int mode, cudaStream_t s, DeviceInfo* di, const void* x, kvrq_dtype dt,
+                            int64_t ldx, int64_t n, int d, int m, const void* pi, const uint16_t* T,
+                            const float* centroids, int cbits, uint32_t* codes_out, const uint32_t* codes_in,
+                            int64_t ldc, uint32_t* signs_out, const uint32_t* signs_in, int64_t lds,
+                            float* gammas_out, const float* gammas_in, float* norms_out, const float* norms_in,
+                            void* xhat, int64_t ldo, int64_t ldn, void* ws, size_t ws_bytes) {
+  const bool f32 = dt == KVRQ_F32;
+  const kvrq_dtype pdt = f32 ? KVRQ_F16 : dt;  // operand type of Pi
+  const int bn_d = tile_n(d), bn_m = tile_n(m);
+  kvrq_status st;
+  CUtensorMap none, mx, mo;
+  memset(&none, 0, sizeof(none));
+  memset(&mx, 0, sizeof(mx));
+  memset(&mo, 0, sizeof(mo));
+  TqgArgs base{};
+  base.d = d;
+  base.n_part = d / bn_d;
+  base.centroids = centroids;
+  base.qjl_scale = (float)(1.2533141373155003 / (double)m);  // sqrt(pi/2) / m
+  base.ldx = ldx;
+  base.ldc = ldc;
+  base.lds = lds;
+  base.ldn = ldn;
+  base.status = di->status;
+  const bool q_side = mode == TQ_MSE_Q || mode == TQ_MSE_QDQ || mode == TQ_PROD_Q;
+  const bool out = mode == TQ_MSE_QDQ || mode == TQ_DQ_MSE || mode == TQ_DQ_PROD;
+  if (q_side && !f32 && (st = encode_rows_map(&mx, x, dt, n, d, ldx, 128)) != KVRQ_OK) return st;
+  if (out && (st = encode_rows_map(&mo, xhat, dt, n, d, ldo, 128)) != KVRQ_OK) return st;
+  auto launch = [&](int gmode, int bn, const CUtensorMap& ma, const CUtensorMap& mb, const TqgArgs& a) {
+    return launch_status(name, launch_tqg(gmode, dt, cbits, bn, ma, mb, mo, a, s, di->num_sms));
+  };
+
+  if (mode == TQ_MSE_Q || mode == TQ_MSE_QDQ || mode == TQ_DQ_MSE) {
+    if (mode != TQ_DQ_MSE) {
+      CUtensorMap mp;
+      if ((st = encode_rows_map(&mp, pi, pdt, d, d, d, bn_d)) != KVRQ_OK) return st;
+      TqgArgs a = base;
+      a.n = n;
+      a.k_total = d;
+      a.n_total = d;
+      a.xf = f32 ? static_cast<const float*>(x) : nullptr;
+      a.codes_out = codes_out;
+      a.norms_out = norms_out;
+      if ((st = launch(G_MSE_Q, bn_d, mx, mp, a)) != KVRQ_OK) return st;
+    }
+    if (mode != TQ_MSE_Q) {
+      CUtensorMap mpt;
+      if ((st = encode_rows_map(&mpt, pi, pdt, d, d, d, 64)) != KVRQ_OK) return st;
+      TqgArgs a = base;
+      a.n = n;
+      a.k_total = d;
+      a.n_total = d;
+      a.codes_in = mode == TQ_DQ_MSE ? codes_in : codes_out;
+      a.norms_in = mode == TQ_DQ_MSE ? norms_in : norms_out;
+      if ((st = launch(G_DQ_MSE, bn_d, none, mpt, a)) != KVRQ_OK) return st;
+    }
+    return KVRQ_OK;
+  }
+
+  // prod: blocks of rows through the workspace
+  const int64_t cap = (int64_t)(ws_bytes / tq_ws_row_bytes(d)) / 128 * 128;
+  if (!ws || cap < 128)
+    return set_errorf(KVRQ_EINVAL, "%s: workspace of %zu bytes holds fewer than 128 rows (need %zu per row)", name,
+                      ws_bytes, tq_ws_row_bytes(d));
+  if (!aligned(ws, 16)) return set_errorf(KVRQ_EINVAL, "%s: workspace must be 16-byte aligned", name);
+  float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + (size_t)cap * 4 * d);
+  if (mode == TQ_PROD_Q) {
+    CUtensorMap mp, mt, mr;
+    if ((st = encode_rows_map(&mp, pi, pdt, d, d, d, bn_d)) != KVRQ_OK) return st;
+    if ((st = encode_rows_map(&mt, T, KVRQ_F16, m, d, d, bn_m)) != KVRQ_OK) return st;
+    if ((st = encode_rows_map(&mr, ws, KVRQ_F16, cap, d, d, 128)) != KVRQ_OK) return st;
+    for (int64_t r0 = 0; r0 < n; r0 += cap) {
+      const int64_t rows = n - r0 < cap ? n - r0 : cap;
+      TqgArgs a = base;
+      a.n = rows;
+      a.k_total = d;
+      a.n_total = d;
+      a.map_row0 = r0;
+      a.xf = f32 ? static_cast<const float*>(x) + r0 * ldx : nullptr;
+      a.codes_out = codes_out + r0 * ldc;
+      a.norms_out = norms_out + r0 * ldn;
+      a.ws = ws;
+      a.part = part;
+      if ((st = launch(G_PROD_Q1, bn_d, mx, mp, a)) != KVRQ_OK) return st;
+      TqgArgs b = base;
+      b.n = rows;
+      b.k_total = d;
+      b.n_total = m;
+      b.signs_out = signs_out + r0 * lds;
+      b.gammas_out = gammas_out + r0 * ldn;
+      b.part = part;
+      if ((st = launch(G_PROD_Q2, bn_m, mr, mt, b)) != KVRQ_OK) return st;
+    }
+    return KVRQ_OK;
+  }
+  // TQ_DQ_PROD
+  CUtensorMap mtt, mpt, mw;
+  memset(&mw, 0, sizeof(mw));
+  if ((st = encode_rows_map(&mtt, T, KVRQ_F16, m, d, d, 64)) != KVRQ_OK) return st;
+  if ((st = encode_rows_map(&mpt, pi, pdt, d, d, d, 64)) != KVRQ_OK) return st;
+  if (!f32 && (st = encode_rows_map(&mw, ws, dt, cap, d, d, 128)) != KVRQ_OK) return st;
+  for (int64_t r0 = 0; r0 < n; r0 += cap) {
+    const int64_t rows = n - r0 < cap ? n - r0 : cap;
+    TqgArgs a = base;
+    a.n = rows;
+    a.k_total = m;
+    a.n_total = d;
+    a.codes_in = codes_in + r0 * ldc;
+    a.signs_in = signs_in + r0 * lds;
+    a.gammas_in = gammas_in + r0 * ldn;
+    a.ws = ws;
+    if ((st = launch(G_DQ_PROD1, bn_d, none, mtt, a)) != KVRQ_OK) return st;
+    TqgArgs b = base;
+    b.n = rows;
+    b.k_total = d;
+    b.n_total = d;
+    b.map_row0 = r0;
+    b.norms_in = norms_in + r0 * ldn;
+    b.ws = ws;
+    if ((st = launch(G_DQ_PROD2, bn_d, mw, mpt, b)) != KVRQ_OK) return st;
+  }
+  return KVRQ_OK;
+}
+
+// Shared validation and dispatch of the TurboQuant calls: d = m = 128 with
+// fp16/bf16 vectors on the resident-Pi kernels, everything else (d a multiple
+// of 128, fp32 vectors) on the tiled kernel.
 static kvrq_status tq_call(const char* name, int mode, void* stream, const void* x, kvrq_dtype dt, int64_t ldx,
                            int64_t n, int d, int m, const void* pi, const uint16_t* T, const float* centroids,
                            int bits, uint32_t* codes_out, const uint32_t* codes_in, int64_t ldc, uint32_t* signs_out,
                            const uint32_t* signs_in, int64_t lds, float* gammas_out, const float* gammas_in,
-                           float* norms_out, const float* norms_in, void* xhat, int64_t ldo, int64_t ldn = 1) {
+                           float* norms_out, const float* norms_in, void* xhat, int64_t ldo, int64_t ldn = 1,
+                           void* ws = nullptr, size_t ws_bytes = 0) {
   const bool prod = mode == TQ_PROD_Q || mode == TQ_DQ_PROD;
   if (ldn < 1) return set_errorf(KVRQ_EINVAL, "%s: norm row stride < 1", name);
   const bool q_side = mode == TQ_MSE_Q || mode == TQ_MSE_QDQ || mode == TQ_PROD_Q;
@@ -225,9 +358,10 @@ static kvrq_status tq_call(const char* name, int mode, void* stream, const void*
   if (!valid_dtype(dt)) return set_errorf(KVRQ_EINVAL, "%s: bad dtype", name);
   if (prod ? (bits < 2 || bits > 5) : (bits < 1 || bits > 4))
     return set_errorf(KVRQ_EUNSUPPORTED, "%s: bits must be in %s", name, prod ? "2..5" : "1..4");
-  if (d != 128) return set_errorf(KVRQ_EUNSUPPORTED, "%s: the tensor-core path supports d = 128", name);
+  if (d % 128 != 0 || d > 16384)
+    return set_errorf(KVRQ_EUNSUPPORTED, "%s: the tensor-core paths need d a multiple of 128 (<= 16384)", name);
   if (prod && m != d) return set_errorf(KVRQ_EUNSUPPORTED, "%s: the QJL projection needs m = d", name);
-  if (dt == KVRQ_F32) return set_errorf(KVRQ_EUNSUPPORTED, "%s: fp32 vectors are not supported here", name);
+  const bool tiled = d != 128 || dt == KVRQ_F32;
   const int cbits = prod ? bits - 1 : bits;
   const int64_t W = kvrq_packed_words(d, cbits);
   if (n == 0) return KVRQ_OK;
@@ -236,7 +370,8 @@ static kvrq_status tq_call(const char* name, int mode, void* stream, const void*
     return set_errorf(KVRQ_EINVAL, "%s: pi and T must be 16-byte aligned", name);
   if (q_side) {
     if (!x || ldx < d || !rows_aligned16(x, ldx, dt)) return set_errorf(KVRQ_EINVAL, "%s: x NULL, ldx < d or rows not 16-byte aligned", name);
-    if (mode != TQ_MSE_QDQ && (!codes_out || !norms_out)) return set_errorf(KVRQ_EINVAL, "%s: codes and norms are required", name);
+    if ((tiled || mode != TQ_MSE_QDQ) && (!codes_out || !norms_out))
+      return set_errorf(KVRQ_EINVAL, "%s: codes and norms are required", name);
     if (codes_out && (ldc < W || !aligned(codes_out, 4))) return set_errorf(KVRQ_EINVAL, "%s: ldc < packed words", name);
     if (prod && (!signs_out || !gammas_out || lds < m / 32 || !aligned(signs_out, 4)))
       return set_errorf(KVRQ_EINVAL, "%s: signs (lds >= m/32) and gammas are required", name);
@@ -247,10 +382,17 @@ static kvrq_status tq_call(const char* name, int mode, void* stream, const void*
   if (out && (!xhat || ldo < d || !rows_aligned16(xhat, ldo, dt)))
     return set_errorf(KVRQ_EINVAL, "%s: xhat NULL, ldo < d or rows not 16-byte aligned", name);
   if (n > ((int64_t)1 << 31) - 256) return set_errorf(KVRQ_EUNSUPPORTED, "%s: n >= 2^31", name);
+  if (tiled && prod && (!ws || ws_bytes / tq_ws_row_bytes(d) < 128 || !aligned(ws, 16)))
+    return set_errorf(KVRQ_EINVAL, "%s: workspace (16-byte aligned) of %zu bytes holds fewer than 128 rows (need %zu per row)",
+                      name, ws_bytes, tq_ws_row_bytes(d));
 
   DeviceInfo* di;
   kvrq_status st = current_device(&di);
   if (st != KVRQ_OK) return st;
+  if (tiled)
+    return tqg_call(name, mode, static_cast<cudaStream_t>(stream), di, x, dt, ldx, n, d, m, pi, T, centroids, cbits,
+                    codes_out, codes_in, ldc, signs_out, signs_in, lds, gammas_out, gammas_in, norms_out, norms_in,
+                    xhat, ldo, ldn, ws, ws_bytes);
   CUtensorMap mx, mp, mt, mo;
   memset(&mx, 0, sizeof(mx));
   memset(&mp, 0, sizeof(mp));
@@ -279,6 +421,46 @@ static kvrq_status tq_call(const char* name, int mode, void* stream, const void*
   a.ldn = ldn;
   a.status = di->status;
   return launch_status(name, launch_tq(mode, dt, cbits, mx, mp, mt, mo, a, static_cast<cudaStream_t>(stream), di->num_sms));
+}
+
+// The QJL sign sketch of arbitrary rows (tiled kernel, sketch epilogue).
+static kvrq_status qjl_call(void* stream, const void* r, kvrq_dtype dt, int64_t n, int d, int64_t ldr, const void* T,
+                            int m, uint32_t* signs, int64_t lds, float* gammas, int64_t ldn) {
+  const char* name = "qjl_sketch";
+  if (n < 0 || ldn < 1) return set_errorf(KVRQ_EINVAL, "%s: n < 0 or ldn < 1", name);
+  if (!valid_dtype(dt)) return set_errorf(KVRQ_EINVAL, "%s: bad dtype", name);
+  if (d < 64 || d % 64 != 0 || d > 16384 || m < 128 || m % 128 != 0)
+    return set_errorf(KVRQ_EUNSUPPORTED, "%s: d must be a multiple of 64 (<= 16384) and m a multiple of 128", name);
+  if (n == 0) return KVRQ_OK;
+  if (!r || ldr < d || !rows_aligned16(r, ldr, dt)) return set_errorf(KVRQ_EINVAL, "%s: r NULL, ldr < d or rows not 16-byte aligned", name);
+  if (!T || !aligned(T, 16)) return set_errorf(KVRQ_EINVAL, "%s: T must be a 16-byte aligned pointer", name);
+  if (!signs || lds < m / 32 || !aligned(signs, 4) || !gammas)
+    return set_errorf(KVRQ_EINVAL, "%s: signs (lds >= m/32) and gammas are required", name);
+  if (n > ((int64_t)1 << 31) - 256) return set_errorf(KVRQ_EUNSUPPORTED, "%s: n >= 2^31", name);
+  DeviceInfo* di;
+  kvrq_status st = current_device(&di);
+  if (st != KVRQ_OK) return st;
+  const bool f32 = dt == KVRQ_F32;
+  const int bn = tile_n(m);
+  CUtensorMap mr, mt, none;
+  memset(&mr, 0, sizeof(mr));
+  memset(&none, 0, sizeof(none));
+  if (!f32 && (st = encode_rows_map(&mr, r, dt, n, d, ldr, 128)) != KVRQ_OK) return st;
+  if ((st = encode_rows_map(&mt, T, f32 ? KVRQ_F16 : dt, m, d, d, bn)) != KVRQ_OK) return st;
+  TqgArgs a{};
+  a.n = n;
+  a.d = d;
+  a.k_total = d;
+  a.n_total = m;
+  a.xf = f32 ? static_cast<const float*>(r) : nullptr;
+  a.ldx = ldr;
+  a.signs_out = signs;
+  a.lds = lds;
+  a.gammas_out = gammas;
+  a.ldn = ldn;
+  a.status = di->status;
+  return launch_status(name, launch_tqg(G_SKETCH, dt, 1, bn, mr, mt, none, a, static_cast<cudaStream_t>(stream),
+                                        di->num_sms));
 }
 
 }  // namespace kvrq
@@ -341,18 +523,29 @@ kvrq_status tq_quantize_dequantize_mse(void* stream, const void* x, kvrq_dtype x
 kvrq_status tq_quantize_prod(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,
                              const void* pi, const uint16_t* T, int m, const float* centroids, int bits,
                              uint32_t* codes, int64_t ldc, uint32_t* signs, int64_t lds, float* gammas,
-                             float* norms) {
+                             float* norms, void* workspace, size_t workspace_bytes) {
   return tq_call("tq_quantize_prod", TQ_PROD_Q, stream, x, xdtype, ldx, n, d, m, pi, T, centroids, bits, codes,
-                 nullptr, ldc, signs, nullptr, lds, gammas, nullptr, norms, nullptr, nullptr, 0);
+                 nullptr, ldc, signs, nullptr, lds, gammas, nullptr, norms, nullptr, nullptr, 0, 1, workspace,
+                 workspace_bytes);
 }
 
 kvrq_status tq_dequantize(void* stream, const uint32_t* codes, int64_t ldc, const uint32_t* signs, int64_t lds,
                           const float* gammas, const float* norms, int64_t n, int d, int m, int bits,
                           const void* pi, const uint16_t* T, const float* centroids, void* xhat, kvrq_dtype odtype,
-                          int64_t ldo) {
+                          int64_t ldo, void* workspace, size_t workspace_bytes) {
   const int mode = signs ? TQ_DQ_PROD : TQ_DQ_MSE;
   return tq_call("tq_dequantize", mode, stream, nullptr, odtype, 0, n, d, m, pi, T, centroids, bits, nullptr, codes,
-                 ldc, nullptr, signs, lds, nullptr, gammas, nullptr, norms, xhat, ldo);
+                 ldc, nullptr, signs, lds, nullptr, gammas, nullptr, norms, xhat, ldo, 1, workspace, workspace_bytes);
+}
+
+size_t kvrq_tq_workspace_bytes(int64_t rows, int d) {
+  if (rows <= 0 || d <= 0) return 0;
+  return (size_t)rows * tq_ws_row_bytes(d);
+}
+
+kvrq_status qjl_sketch(void* stream, const void* r, kvrq_dtype rdtype, int64_t n, int d, int64_t ldr, const void* T,
+                       int m, uint32_t* signs, int64_t lds, float* gammas, int64_t ldn) {
+  return qjl_call(stream, r, rdtype, n, d, ldr, T, m, signs, lds, gammas, ldn);
 }
 
 kvrq_status kv_score_packed(void* stream, kvrq_method method, const void* q, kvrq_dtype qdtype, int64_t ldq,

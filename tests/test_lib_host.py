@@ -150,3 +150,40 @@ def test_rq_validation_fails_before_any_launch():
     assert lib.rq_dequantize(None, P, 13, P, 0, 128, P, P, 3, P, 1, 128) == 0
     assert lib.rq_quantize_dequantize(None, P, 1, 10, 128, 128, P, P, 3, P, 13, P, None, 128) == EINVAL
     assert lib.rq_quantize_dequantize(None, P, 1, 10, 128, 128, P, P, 3, P, 13, P, P, 64) == EINVAL
+
+
+def test_tq_validation_fails_before_any_launch():
+    lib = kvrq.lib()
+    EINVAL, EUNSUP = 1, 2
+    per_row = 4 * 256 + 4 * 2
+    assert lib.kvrq_tq_workspace_bytes(1, 256) == per_row
+    assert lib.kvrq_tq_workspace_bytes(0, 256) == 0
+
+    def prod(d=256, m=256, ws=P, wsb=per_row * 128, n=10, dt=1, bits=3, ldc=None):
+        W = -(-d * (bits - 1) // 32)
+        return lib.tq_quantize_prod(None, P, dt, n, d, d, P, P, m, P, bits, P, W if ldc is None else ldc, P, m // 32,
+                                    P, P, ws, wsb)
+
+    assert prod(ws=None) == EINVAL  # the tiled prod path needs a workspace
+    assert prod(wsb=per_row * 127) == EINVAL  # fewer than 128 rows fit
+    assert prod(ws=P + 8) == EINVAL  # not 16-byte aligned
+    assert prod(d=192, m=192) == EUNSUP  # not a multiple of 128
+    assert prod(m=128) == EUNSUP  # m = d
+    assert prod(bits=6) == EUNSUP
+    assert prod(ldc=1) == EINVAL
+    assert prod(n=0) == 0
+    # d = 128 with 16-bit vectors takes no workspace; fp32 vectors do
+    assert prod(d=128, m=128, ws=None, wsb=0, n=0) == 0
+    assert prod(d=128, m=128, dt=0, ws=None, wsb=0) == EINVAL
+    # dequantize: same workspace rule for prod, none for mse
+    assert lib.tq_dequantize(None, P, 16, P, 8, P, P, 10, 256, 256, 3, P, P, P, P, 1, 256, None, 0) == EINVAL
+
+    def sk(n=10, d=256, ldr=256, m=256, lds=8, dt=1):
+        return lib.qjl_sketch(None, P, dt, n, d, ldr, P, m, P, lds, P, 1)
+
+    assert sk(m=96) == EUNSUP
+    assert sk(d=100, ldr=100) == EUNSUP
+    assert sk(lds=7) == EINVAL
+    assert sk(ldr=200) == EINVAL
+    assert sk(n=-1) == EINVAL
+    assert sk(n=0) == 0
