@@ -204,6 +204,21 @@ kvrq_status tq_quantize_prod(void* stream, const void* x, kvrq_dtype xdtype, int
                              uint32_t* codes, int64_t ldc, uint32_t* signs, int64_t lds, float* gammas,
                              float* norms, void* workspace, size_t workspace_bytes);
 
+/* tq_quantize_prod without a workspace argument: the tiled path runs its row
+ * blocks through a static 8 MiB device array of the library (address taken
+ * once per device at set-up), so the call allocates nothing and takes no
+ * buffer beyond its outputs. The pages have no counterpart of this call; it
+ * exists for callers that may not allocate. Same arguments and results as
+ * tq_quantize_prod; returns KVRQ_EUNSUPPORTED when one 128-row block does not
+ * fit the array (128 * kvrq_tq_workspace_bytes(1, d) > 8 MiB, i.e. d = 16384).
+ * Nothing in the array has to start at zero. Calls that overlap in time on one
+ * device (other streams, other host threads) share the array and race: order
+ * them on one stream. */
+kvrq_status tq_quantize_prod_noalloc(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,
+                                     const void* pi, const uint16_t* T, int m, const float* centroids, int bits,
+                                     uint32_t* codes, int64_t ldc, uint32_t* signs, int64_t lds, float* gammas,
+                                     float* norms);
+
 /* Dequantize mse (signs == NULL; bits = b) or prod (signs != NULL; bits = b
  * total; workspace as for tq_quantize_prod). */
 kvrq_status tq_dequantize(void* stream, const uint32_t* codes, int64_t ldc, const uint32_t* signs, int64_t lds,

@@ -284,6 +284,28 @@ def tq_quantize_prod(x, pi, T, centroids, bits, codes=None, norms=None, signs=No
     return codes, signs, gammas, norms
 
 
+def tq_quantize_prod_noalloc(x, pi, T, centroids, bits, codes=None, norms=None, signs=None, gammas=None,
+                             stream=None):
+    """tq_quantize_prod through the library's static scratch instead of a workspace (the C call allocates
+    nothing; outputs are allocated here when not given). Returns (codes, signs, gammas, norms)."""
+    torch = _torch()
+    n, d = x.shape
+    m = T.shape[0]
+    codes, norms = _tq_outputs(n, d, bits - 1, x.device, codes, norms)
+    if signs is None:
+        signs = torch.empty((n, m // 32), dtype=torch.int32, device=x.device)
+    if gammas is None:
+        gammas = torch.empty((n,), dtype=torch.float32, device=x.device)
+    xp, ldx = _rows(x, "x")
+    cp, ldc = _rows(codes, "codes")
+    sp, lds = _rows(signs, "signs")
+    _lib.check("tq_quantize_prod_noalloc", lib().tq_quantize_prod_noalloc(
+        _stream(stream), xp, _dtype_code(x), n, d, ldx, _ptr(pi, "pi", _pi_dtype(x.dtype)),
+        _ptr(T, "T", torch.float16), m, _ptr(centroids, "centroids", torch.float32), bits, cp, ldc, sp, lds,
+        _ptr(gammas, "gammas", torch.float32), _ptr(norms, "norms", torch.float32)))
+    return codes, signs, gammas, norms
+
+
 def tq_dequantize(codes, norms, d, pi, centroids, bits, signs=None, gammas=None, T=None, xhat=None,
                   out_dtype=None, workspace=None, stream=None):
     """TurboQuant dequantize: mse when signs is None, prod otherwise (bits = total bits).

@@ -45,6 +45,9 @@ SIGNATURES = {
     # workspace_bytes
     "tq_quantize_prod": (c_int, [c_vp, c_vp, c_int, c_i64, c_int, c_i64, c_vp, c_vp, c_int, c_vp, c_int, c_vp, c_i64,
                                  c_vp, c_i64, c_vp, c_vp, c_vp, ctypes.c_size_t]),
+    # stream, x, xdtype, n, d, ldx, pi, T, m, centroids, bits, codes, ldc, signs, lds, gammas, norms
+    "tq_quantize_prod_noalloc": (c_int, [c_vp, c_vp, c_int, c_i64, c_int, c_i64, c_vp, c_vp, c_int, c_vp, c_int, c_vp,
+                                         c_i64, c_vp, c_i64, c_vp, c_vp]),
     # stream, codes, ldc, signs, lds, gammas, norms, n, d, m, bits, pi, T, centroids, xhat, odtype, ldo, workspace,
     # workspace_bytes
     "tq_dequantize": (c_int, [c_vp, c_vp, c_i64, c_vp, c_i64, c_vp, c_vp, c_i64, c_int, c_int, c_int, c_vp, c_vp,

@@ -44,10 +44,17 @@ static kvrq_status cuda_fail(const char* where, cudaError_t e) {
 }
 
 // ------------------------------------------------------------------ per-device state
+// Scratch of tq_quantize_prod_noalloc: one per device image, 8 MiB. Nothing in
+// it has to start at zero (each call writes every byte it later reads), and
+// calls that overlap in time on one device share it, so they race.
+constexpr size_t kNoallocScratchBytes = (size_t)8 << 20;
+static __device__ __align__(256) unsigned char g_tq_scratch[kNoallocScratchBytes];
+
 struct DeviceInfo {
   bool ready = false;
   int num_sms = 0;
   unsigned* status = nullptr;  // device address of g_device_status
+  void* scratch = nullptr;     // device address of g_tq_scratch
 };
 
 static std::mutex g_dev_mu;
@@ -67,6 +74,9 @@ static kvrq_status current_device(DeviceInfo** out) {
     e = cudaGetSymbolAddress(&p, g_device_status);
     if (e != cudaSuccess) return cuda_fail("cudaGetSymbolAddress(status)", e);
     di.status = static_cast<unsigned*>(p);
+    e = cudaGetSymbolAddress(&p, g_tq_scratch);
+    if (e != cudaSuccess) return cuda_fail("cudaGetSymbolAddress(scratch)", e);
+    di.scratch = p;
     di.ready = true;
   }
   *out = &di;
@@ -348,7 +358,7 @@ static kvrq_status tq_call(const char* name, int mode, void* stream, const void*
                            int bits, uint32_t* codes_out, const uint32_t* codes_in, int64_t ldc, uint32_t* signs_out,
                            const uint32_t* signs_in, int64_t lds, float* gammas_out, const float* gammas_in,
                            float* norms_out, const float* norms_in, void* xhat, int64_t ldo, int64_t ldn = 1,
-                           void* ws = nullptr, size_t ws_bytes = 0) {
+                           void* ws = nullptr, size_t ws_bytes = 0, bool static_scratch = false) {
   const bool prod = mode == TQ_PROD_Q || mode == TQ_DQ_PROD;
   if (ldn < 1) return set_errorf(KVRQ_EINVAL, "%s: norm row stride < 1", name);
   const bool q_side = mode == TQ_MSE_Q || mode == TQ_MSE_QDQ || mode == TQ_PROD_Q;
@@ -382,13 +392,21 @@ static kvrq_status tq_call(const char* name, int mode, void* stream, const void*
   if (out && (!xhat || ldo < d || !rows_aligned16(xhat, ldo, dt)))
     return set_errorf(KVRQ_EINVAL, "%s: xhat NULL, ldo < d or rows not 16-byte aligned", name);
   if (n > ((int64_t)1 << 31) - 256) return set_errorf(KVRQ_EUNSUPPORTED, "%s: n >= 2^31", name);
-  if (tiled && prod && (!ws || ws_bytes / tq_ws_row_bytes(d) < 128 || !aligned(ws, 16)))
+  if (tiled && prod && static_scratch && 128 * tq_ws_row_bytes(d) > kNoallocScratchBytes)
+    return set_errorf(KVRQ_EUNSUPPORTED,
+                      "%s: d = %d needs %zu bytes of scratch for one 128-row block; the static scratch holds %zu",
+                      name, d, 128 * tq_ws_row_bytes(d), kNoallocScratchBytes);
+  if (tiled && prod && !static_scratch && (!ws || ws_bytes / tq_ws_row_bytes(d) < 128 || !aligned(ws, 16)))
     return set_errorf(KVRQ_EINVAL, "%s: workspace (16-byte aligned) of %zu bytes holds fewer than 128 rows (need %zu per row)",
                       name, ws_bytes, tq_ws_row_bytes(d));
 
   DeviceInfo* di;
   kvrq_status st = current_device(&di);
   if (st != KVRQ_OK) return st;
+  if (static_scratch) {
+    ws = di->scratch;
+    ws_bytes = kNoallocScratchBytes;
+  }
   if (tiled)
     return tqg_call(name, mode, static_cast<cudaStream_t>(stream), di, x, dt, ldx, n, d, m, pi, T, centroids, cbits,
                     codes_out, codes_in, ldc, signs_out, signs_in, lds, gammas_out, gammas_in, norms_out, norms_in,
@@ -536,6 +554,15 @@ kvrq_status tq_dequantize(void* stream, const uint32_t* codes, int64_t ldc, cons
   const int mode = signs ? TQ_DQ_PROD : TQ_DQ_MSE;
   return tq_call("tq_dequantize", mode, stream, nullptr, odtype, 0, n, d, m, pi, T, centroids, bits, nullptr, codes,
                  ldc, nullptr, signs, lds, nullptr, gammas, nullptr, norms, xhat, ldo, 1, workspace, workspace_bytes);
+}
+
+kvrq_status tq_quantize_prod_noalloc(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,
+                                     const void* pi, const uint16_t* T, int m, const float* centroids, int bits,
+                                     uint32_t* codes, int64_t ldc, uint32_t* signs, int64_t lds, float* gammas,
+                                     float* norms) {
+  return tq_call("tq_quantize_prod_noalloc", TQ_PROD_Q, stream, x, xdtype, ldx, n, d, m, pi, T, centroids, bits,
+                 codes, nullptr, ldc, signs, nullptr, lds, gammas, nullptr, norms, nullptr, nullptr, 0, 1, nullptr, 0,
+                 true);
 }
 
 size_t kvrq_tq_workspace_bytes(int64_t rows, int d) {
