@@ -58,6 +58,16 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def measured_tensor_peak():
+    """Dense fp16/bf16 tensor-core peak in TFLOP/s: the measured cuBLAS bf16 burst figure (fp16 runs at the same
+    nominal rate), else the fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f).get("bf16_tflops", 1590.0))
+    return 1590.0
+
+
 class ClockSampler:
     """Samples nvidia-smi clocks and throttle reasons while running."""
 
@@ -255,47 +265,126 @@ def run_leg_only(args):
     if fn is not None:
         return time_fn(fn, rows, args, torch, kvrq)
     rows = args.rows
-    x = synth.lognormal(rows, D, seed=1, dtype=torch.float16, device=dev)
+    dd = args.dim
+    x = synth.lognormal(rows, dd, seed=1, dtype=torch.float16, device=dev, outliers=() if dd != D else
+                        synth.OUTLIER_CHANNELS)
     xh = torch.empty_like(x)
     if kind == "rq":
-        rot = torch.from_numpy(kvrq.rq_rotors_init(D, 1).astype(np.float32)).to(dev)
-        cb = torch.from_numpy(kvrq.tq_codebook_init(D, b)[0].astype(np.float32)).to(dev)
+        rot = torch.from_numpy(kvrq.rq_rotors_init(dd, 1).astype(np.float32)).to(dev)
+        cb = torch.from_numpy(kvrq.tq_codebook_init(dd, b)[0].astype(np.float32)).to(dev)
         codes, norms = kvrq.rq_quantize(x, rot, cb, b)
         calls = {"q": lambda: kvrq.rq_quantize(x, rot, cb, b, codes=codes, norms=norms),
-                 "dq": lambda: kvrq.rq_dequantize(codes, norms, D, rot, cb, b, xhat=xh),
+                 "dq": lambda: kvrq.rq_dequantize(codes, norms, dd, rot, cb, b, xhat=xh),
                  "qdq": lambda: kvrq.rq_quantize_dequantize(x, rot, cb, b, codes=codes, norms=norms, xhat=xh)}
     else:
-        pi = torch.from_numpy(kvrq.tq_rotation_init(D, 2)).to(torch.float16).to(dev)
-        T = torch.from_numpy(kvrq.qjl_matrix_init(D, D, 3)).to(torch.float16).to(dev)
+        D_ = dd
+        pi = torch.from_numpy(kvrq.tq_rotation_init(D_, 2)).to(torch.float16).to(dev)
+        T = torch.from_numpy(kvrq.qjl_matrix_init(D_, D_, 3)).to(torch.float16).to(dev)
         prod = mode in ("prod", "dqp")
-        cb = torch.from_numpy(kvrq.tq_codebook_init(D, b - 1 if prod else b)[0].astype(np.float32)).to(dev)
+        cb = torch.from_numpy(kvrq.tq_codebook_init(D_, b - 1 if prod else b)[0].astype(np.float32)).to(dev)
+        ws = kvrq.tq_workspace(rows, D_, dev) if kvrq.tq_needs_workspace(D_, x.dtype) else None
         if prod:
             codes, signs, gam, norms = kvrq.tq_quantize_prod(x, pi, T, cb, b)
         else:
             codes, norms = kvrq.tq_quantize_mse(x, pi, cb, b)
         calls = {"q": lambda: kvrq.tq_quantize_mse(x, pi, cb, b, codes=codes, norms=norms),
                  "qdq": lambda: kvrq.tq_quantize_dequantize_mse(x, pi, cb, b, codes=codes, norms=norms, xhat=xh),
-                 "dqm": lambda: kvrq.tq_dequantize(codes, norms, D, pi, cb, b, xhat=xh)}
+                 "dqm": lambda: kvrq.tq_dequantize(codes, norms, D_, pi, cb, b, xhat=xh)}
         if prod:
             calls["prod"] = lambda: kvrq.tq_quantize_prod(x, pi, T, cb, b, codes=codes, norms=norms, signs=signs,
-                                                          gammas=gam)
-            calls["dqp"] = lambda: kvrq.tq_dequantize(codes, norms, D, pi, cb, b, signs=signs, gammas=gam, T=T,
-                                                      xhat=xh)
+                                                          gammas=gam, workspace=ws)
+            calls["dqp"] = lambda: kvrq.tq_dequantize(codes, norms, D_, pi, cb, b, signs=signs, gammas=gam, T=T,
+                                                      xhat=xh, workspace=ws)
     return time_fn(calls[mode], rows, args, torch, kvrq)
 
 
+def run_dim_sweep(args):
+    """Config-5 sweep: 1 GiB of fp16 rows (N(0,1) directions, LogNormal(0, 0.5) norms, no outlier
+    channels) per d; each cell timed over args.iters calls after a warm-up call (inputs >> L2)."""
+    import torch
+
+    import kv_cache_vector_rq_b200 as kvrq
+    from kv_cache_vector_rq_b200 import synth
+
+    dev = torch.device("cuda", 0)
+    peak, peak_kind = measured_peaks()
+    tflops_peak = measured_tensor_peak()
+    clk = ClockSampler(0)
+    clk.__enter__()
+    cells = []
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        s, e = ev(), ev()
+        s.record()
+        for _ in range(args.iters):
+            fn()
+        e.record()
+        torch.cuda.synchronize()
+        kvrq.device_status()
+        return s.elapsed_time(e) / args.iters
+
+    for d in (128, 256, 1536, 4096):
+        rows = (1 << 30) // (2 * d)
+        x = synth.lognormal(rows, d, seed=5 + d, dtype=torch.float16, device=dev, outliers=())
+        xh = torch.empty_like(x)
+        rot = torch.from_numpy(kvrq.rq_rotors_init(d, 1).astype(np.float32)).to(dev)
+        pi = torch.from_numpy(kvrq.tq_rotation_init(d, 2)).to(torch.float16).to(dev)
+        T = torch.from_numpy(kvrq.qjl_matrix_init(d, d, 3)).to(torch.float16).to(dev)
+        ws = kvrq.tq_workspace(rows, d, dev) if kvrq.tq_needs_workspace(d, x.dtype) else None
+        for b in (2, 3, 4):
+            cb = torch.from_numpy(kvrq.tq_codebook_init(d, b)[0].astype(np.float32)).to(dev)
+            rc, rn = kvrq.rq_quantize(x, rot, cb, b)
+            ms = timed(lambda: kvrq.rq_quantize_dequantize(x, rot, cb, b, codes=rc, norms=rn, xhat=xh))
+            bpv = rq_bytes_per_vector(d, b)
+            cells.append({"d": d, "b": b, "path": "rq_roundtrip", "rows": rows, "ms": ms,
+                          "Mvec_s": rows / ms / 1e3, "GB_s": bpv * rows / ms / 1e6,
+                          "frac_hbm": bpv * rows / ms / 1e6 / peak})
+            del rc, rn
+            cp = torch.from_numpy(kvrq.tq_codebook_init(d, b - 1)[0].astype(np.float32)).to(dev)
+            codes, signs, gam, norms = kvrq.tq_quantize_prod(x, pi, T, cp, b, workspace=ws)
+            msq = timed(lambda: kvrq.tq_quantize_prod(x, pi, T, cp, b, codes=codes, norms=norms, signs=signs,
+                                                      gammas=gam, workspace=ws))
+            msd = timed(lambda: kvrq.tq_dequantize(codes, norms, d, pi, cp, b, signs=signs, gammas=gam, T=T,
+                                                   xhat=xh, workspace=ws))
+            flops_q = 2.0 * d * d * 2  # y = Pi x, z = T r (m = d)
+            bq = 2 * d + 4 * kvrq.packed_words(d, b - 1) + 4 * (d // 32) + 8
+            for path, t, by in (("tq_prod_quantize", msq, bq), ("tq_prod_dequantize", msd, bq),
+                                ("tq_prod_roundtrip", msq + msd, 2 * bq)):
+                fl = flops_q * (2 if path == "tq_prod_roundtrip" else 1)
+                cells.append({"d": d, "b": b, "path": path, "rows": rows, "ms": t, "Mvec_s": rows / t / 1e3,
+                              "GB_s": by * rows / t / 1e6, "TFLOP_s": fl * rows / t / 1e9,
+                              "frac_tensor": fl * rows / t / 1e9 / tflops_peak})
+            del codes, signs, gam, norms
+        del x, xh, ws
+        torch.cuda.empty_cache()
+    clk.__exit__(None, None, None)
+    print(json.dumps({"sweep": "config5", "input": "1 GiB fp16 per d", "peak_GB_s": peak, "peak_kind": peak_kind,
+                      "tensor_peak_TFLOP_s": tflops_peak, "cells": cells, "clocks": clk.summary()}), flush=True)
+
+
 def time_fn(fn, rows, args, torch, kvrq):
+    """args.iters calls timed on the device. The calls are captured once into a CUDA graph and the graph is
+    replayed, so the host cost of a call (binding, tensor-map encoding) does not pace small launches."""
     fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(args.iters):
+            fn()
+    g.replay()
     torch.cuda.synchronize()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     s.record()
-    for _ in range(args.iters):
-        fn()
+    g.replay()
     e.record()
     torch.cuda.synchronize()
     kvrq.device_status()
     ms = s.elapsed_time(e) / args.iters
-    print(json.dumps({"leg": args.leg, "rows": rows, "ms": ms, "Mvec_s": rows / ms / 1e3}), flush=True)
+    print(json.dumps({"leg": args.leg, "rows": rows, "ms": ms, "Mvec_s": rows / ms / 1e3, "timing": "graph replay"}),
+          flush=True)
 
 
 def main():
@@ -309,7 +398,12 @@ def main():
                     help="time one kernel leg (rq_q3, rq_dq3, rq_qdq3, tq_q3, tq_qdq3, tq_prod3, tq_dqm3, tq_dqp3, "
                          "any b) on --rows vectors instead of the workload; used for profiler captures")
     ap.add_argument("--rows", type=int, default=1 << 20)
+    ap.add_argument("--dim", type=int, default=D, help="head dimension of --leg (the tiled TurboQuant path "
+                                                       "and the general RotorQuant kernel run d != 128)")
     ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--c5", action="store_true",
+                    help="dimension sweep at 1 GiB fp16 input: d in {128, 256, 1536, 4096}, b in {2, 3, 4}, "
+                         "RotorQuant roundtrip vs TurboQuant-prod quantize + dequantize; one JSON line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -321,6 +415,9 @@ def main():
         return
     if args.leg:
         run_leg_only(args)
+        return
+    if args.c5:
+        run_dim_sweep(args)
         return
 
     import torch

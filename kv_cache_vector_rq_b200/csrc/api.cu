@@ -210,8 +210,8 @@ static kvrq_status rq_call(const char* name, int mode, void* stream, const void*
     CUtensorMap mx, mo;
     memset(&mx, 0, sizeof(mx));
     memset(&mo, 0, sizeof(mo));
-    if (q_side && (st = encode_rows_map(&mx, x, xdt, n, d, ldx, 128)) != KVRQ_OK) return st;
-    if (dq_side && (st = encode_rows_map(&mo, xhat, odt, n, d, ldo, 128)) != KVRQ_OK) return st;
+    if (q_side && (st = encode_rows_map(&mx, x, xdt, n, d, ldx, rq_row_box_rows())) != KVRQ_OK) return st;
+    if (dq_side && (st = encode_rows_map(&mo, xhat, odt, n, d, ldo, rq_row_box_rows())) != KVRQ_OK) return st;
     if (!q_side) mx = mo;
     if (!dq_side) mo = mx;
     return launch_status(name, launch_rq_row(mode, tdt, bits, mx, mo, a, s, di->num_sms));

@@ -8,12 +8,13 @@
 // sandwich R~ v R, drop the pad, multiply by the norm.
 //
 // B200 design (not the pages' one-thread-per-(vector, group) layout):
-//  * d = 128 rows go through `rq_row_kernel`: one thread owns one whole row, a
-//    persistent CTA streams 128-row tiles in with TMA (128-byte swizzle, so a
-//    thread reading its own row hits 8 different banks per 16-byte phase),
-//    double-buffered on mbarriers; results are written to a swizzled shared
-//    tile and leave through a TMA tensor store; codes are staged in shared
-//    memory and written out coalesced.
+//  * d = 128 rows go through `rq_row_kernel`: one thread owns one whole row and
+//    every warp is an independent pipeline over 32-row sub-tiles: its own TMA
+//    loads (128-byte swizzle, so a lane reading its own row hits 8 different
+//    banks per 16-byte phase), mbarriers, x_hat written back in place and
+//    stored by TMA, codes staged in shared memory and stored by one bulk copy.
+//    Warps whose rows arrive first compute and store first, so loads, math and
+//    stores of the warps of an SM overlap even when each warp has one sub-tile.
 //  * The sandwich is applied as its exact 3x3 matrix (9 FMA per group instead
 //    of the 48-FMA sparse product the README counts): the matrix is built once
 //    per CTA from the rotors.
@@ -103,7 +104,7 @@ __device__ __forceinline__ void build_codebook(const float* __restrict__ centroi
 }
 
 // ============================================================================
-// d = 128, one thread per row, TMA-streamed 128-row tiles.
+// d = 128, one thread per row, TMA-streamed 32-row sub-tiles per warp.
 //
 // Per row: pass 1 reads the row from the swizzled shared tile and forms
 // ||x||^2; pass 2 re-reads it a group pair (6 elements) at a time, rotates
@@ -138,7 +139,9 @@ constexpr int D = 128;
 constexpr int G = 43;         // groups of 3
 constexpr int NP = 22;        // group pairs (the last: group 42 and an all-zero group)
 constexpr int NC = 3 * G;     // 129 stored codes
-constexpr int kRows = 128;    // rows per tile = threads per CTA
+constexpr int kRows = 128;    // threads per CTA (4 warps)
+constexpr int kWR = 32;       // rows per warp sub-tile
+constexpr int kWarps = kRows / kWR;
 constexpr float kB = 4611686018427387904.0f;      // 2^62
 constexpr float kShift = 9.313225746154785e-10f;  // 2^-30
 constexpr float kWindow0 = 8388608.0f;            // 2^23
@@ -147,8 +150,8 @@ template <typename T>
 struct Tile {
   static constexpr int kBoxElems = 128 / (int)sizeof(T);  // elements per 128-byte box row
   static constexpr int kBoxes = D / kBoxElems;             // 2 (16-bit) or 4 (fp32)
-  static constexpr int kBoxBytes = kRows * 128;            // 16 KB
-  static constexpr int kTileBytes = kBoxes * kBoxBytes;    // 32 KB (16-bit) / 64 KB (fp32)
+  static constexpr int kBoxBytes = kWR * 128;              // 4 KB
+  static constexpr int kTileBytes = kBoxes * kBoxBytes;    // one warp's sub-tile: 8 KB (16-bit) / 16 KB (fp32)
   static constexpr int kE = 16 / (int)sizeof(T);           // elements per 16-byte chunk
   static constexpr int kChunks = D / kE;
   // byte offset of 16-byte chunk j of row r in the 128-byte-swizzled tile
@@ -169,17 +172,17 @@ struct Codes {
 template <typename T, int BITS, int MODE, int STAGES>
 struct Smem {
   static constexpr int W = Codes<BITS>::W;
-  static constexpr int tile_bytes = STAGES * Tile<T>::kTileBytes;
-  static constexpr int codes_off = tile_bytes;  // [2][kRows][W] words
-  static constexpr int codes_stage = ((kRows * W * 4 + 15) / 16) * 16;
-  static constexpr int lut_off = codes_off + 2 * codes_stage;  // dequantize: [K][kRows] floats
+  static constexpr int tile_bytes = kWarps * STAGES * Tile<T>::kTileBytes;  // [warp][stage] sub-tiles
+  static constexpr int codes_off = tile_bytes;                               // [warp][2][kWR][W] words
+  static constexpr int codes_stage = ((kWR * W * 4 + 15) / 16) * 16;
+  static constexpr int lut_off = codes_off + kWarps * 2 * codes_stage;  // dequantize: [K][kRows] floats
   static constexpr int lut_bytes = MODE == RQ_DQ ? Codes<BITS>::K * kRows * 4 : 0;
   static constexpr int mp_off = lut_off + lut_bytes;  // [NP][10] float2
   static constexpr int mp_bytes = NP * 10 * 8;
   static constexpr int cb_off = mp_off + mp_bytes;  // codebook constants
   static constexpr int cb_bytes = 64 * 4;
-  static constexpr int bar_off = cb_off + cb_bytes;  // STAGES tile + 2 code-stage barriers
-  static constexpr int bytes = bar_off + 8 * (STAGES + 2);
+  static constexpr int bar_off = cb_off + cb_bytes;  // per warp: STAGES sub-tile + 2 code-stage barriers
+  static constexpr int bytes = bar_off + 8 * kWarps * (STAGES + 2);
   static constexpr int alloc = bytes + 1024;
 };
 
@@ -232,89 +235,95 @@ __global__ void __launch_bounds__(kRows, MODE == RQ_Q ? 2 : KVRQ_ROW_MIN_BLOCKS)
   float* s_sc = reinterpret_cast<float*>(smem + SM::cb_off);
   float* s_mag = s_sc + 16;
   float* s_cf = s_sc + 32;
-  uint64_t* s_bar = reinterpret_cast<uint64_t*>(smem + SM::bar_off);  // [0, STAGES) tiles, [STAGES + c] codes
-
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // each warp streams its own 32-row sub-tiles: its buffers, barriers and copies
+  uint64_t* w_bar = reinterpret_cast<uint64_t*>(smem + SM::bar_off) + warp * (STAGES + 2);  // [s] tiles, [STAGES + c] codes
+  uint8_t* w_tiles = smem + warp * STAGES * TL::kTileBytes;
+  uint32_t* w_codes = s_codes + warp * 2 * (SM::codes_stage / 4);
   const int64_t n = a.n;
-  const int64_t ntiles = (n + kRows - 1) / kRows;
-  // dequantize: a full tile of packed codes is one contiguous, 16-byte aligned block
+  const int nsub = (int)((n + kWR - 1) / kWR);  // n < 2^31 (checked on the host)
+  const int gw = (int)blockIdx.x * kWarps + warp, tw = (int)gridDim.x * kWarps;
+  // dequantize: a full sub-tile of packed codes is one contiguous, 16-byte aligned block
   const bool codes_bulk = !kIn && a.ldc == W && (reinterpret_cast<uintptr_t>(a.codes_in) & 15) == 0;
 
   if (tid == 0) {
     if (kIn) tma_prefetch_desc(&map_x);
     if (kOut) tma_prefetch_desc(&map_o);
-    for (int s = 0; s < STAGES + 2; ++s) mbar_init(&s_bar[s], 1);
+    for (int s = 0; s < kWarps * (STAGES + 2); ++s)
+      mbar_init(reinterpret_cast<uint64_t*>(smem + SM::bar_off) + s, 1);
     fence_barrier_init();
   }
   build_pair_table(a.rotors, reinterpret_cast<float2*>(smem + SM::mp_off));
   build_consts<BITS>(a.centroids, s_sc, s_mag, s_cf);
   __syncthreads();
 
-  // bit b of `par`: parity of the next phase of barrier b (all threads);
-  // bit b of `pend`: a copy completing on barrier b is in flight (thread 0)
+  // bit b of `par`: parity of the next phase of barrier b (all lanes);
+  // bit b of `pend`: a copy completing on barrier b is in flight (lane 0)
   uint32_t par = 0, pend = 0;
 
-  auto tile_of = [&](int iter) -> int64_t { return blockIdx.x + (int64_t)iter * gridDim.x; };
-  auto issue_tile = [&](int64_t tile, int s) {  // thread 0
+  auto sub_of = [&](int iter) -> int { return gw + iter * tw; };
+  auto issue_tile = [&](int sub, int s) {  // lane 0
     pend |= 1u << s;
-    mbar_arrive_expect_tx(&s_bar[s], TL::kTileBytes);
+    mbar_arrive_expect_tx(&w_bar[s], TL::kTileBytes);
 #pragma unroll
     for (int b = 0; b < TL::kBoxes; ++b)
-      tma_load_2d(smem + s * TL::kTileBytes + b * TL::kBoxBytes, &map_x, b * TL::kBoxElems, (int32_t)(tile * kRows),
-                  &s_bar[s]);
+      tma_load_2d(w_tiles + s * TL::kTileBytes + b * TL::kBoxBytes, &map_x, b * TL::kBoxElems, sub * kWR,
+                  &w_bar[s]);
   };
-  auto codes_bulk_tile = [&](int64_t tile) { return codes_bulk && (tile + 1) * kRows <= n; };
-  auto issue_codes = [&](int64_t tile, int c) {  // thread 0
+  auto codes_bulk_tile = [&](int sub) { return codes_bulk && (int64_t)(sub + 1) * kWR <= n; };
+  auto issue_codes = [&](int sub, int c) {  // lane 0
     pend |= 1u << (STAGES + c);
-    mbar_arrive_expect_tx(&s_bar[STAGES + c], kRows * W * 4);
-    bulk_load(s_codes + c * (SM::codes_stage / 4), a.codes_in + tile * kRows * W, kRows * W * 4, &s_bar[STAGES + c]);
+    mbar_arrive_expect_tx(&w_bar[STAGES + c], kWR * W * 4);
+    bulk_load(w_codes + c * (SM::codes_stage / 4), a.codes_in + (int64_t)sub * kWR * W, kWR * W * 4,
+              &w_bar[STAGES + c]);
   };
 
-  if (tid == 0) {
+  if (lane == 0) {
     if (kIn) {
       for (int s = 0; s < STAGES; ++s)
-        if (tile_of(s) < ntiles) issue_tile(tile_of(s), s);
+        if (sub_of(s) < nsub) issue_tile(sub_of(s), s);
     } else {
       for (int c = 0; c < 2; ++c)
-        if (tile_of(c) < ntiles && codes_bulk_tile(tile_of(c))) issue_codes(tile_of(c), c);
+        if (sub_of(c) < nsub && codes_bulk_tile(sub_of(c))) issue_codes(sub_of(c), c);
     }
   }
 
   int it = 0;
-  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+  for (int sub = gw; sub < nsub; sub += tw, ++it) {
     const int s = it % STAGES;
     const int cs = it & 1;
-    const int64_t row0 = tile * kRows;
-    const int rows = (int)(n - row0 < (int64_t)kRows ? n - row0 : (int64_t)kRows);
-    const int64_t row = row0 + tid;
-    uint8_t* tb = smem + s * TL::kTileBytes;
-    uint32_t* stage_codes = s_codes + cs * (SM::codes_stage / 4);
+    const int64_t row0 = (int64_t)sub * kWR;
+    const int rows = (int)(n - row0 < (int64_t)kWR ? n - row0 : (int64_t)kWR);
+    const int64_t row = row0 + lane;
+    uint8_t* tb = w_tiles + s * TL::kTileBytes;
+    uint32_t* stage_codes = w_codes + cs * (SM::codes_stage / 4);
 
     // ---------------------------------------------------------------- inputs
     bool ok = true;
     if constexpr (kIn) {
-      if (tid == 0) bulk_wait_read<1>();  // the codes store from this staging buffer (two tiles ago) is done
-      ok = mbar_wait(&s_bar[s], (par >> s) & 1, a.status);
+      if (lane == 0) bulk_wait_read<1>();  // the codes store from this staging buffer (two sub-tiles ago) is done
+      ok = mbar_wait(&w_bar[s], (par >> s) & 1, a.status);
       par ^= 1u << s;
       pend &= ~(1u << s);
     } else {
-      if (codes_bulk_tile(tile)) {
-        ok = mbar_wait(&s_bar[STAGES + cs], (par >> (STAGES + cs)) & 1, a.status);
+      if (codes_bulk_tile(sub)) {
+        ok = mbar_wait(&w_bar[STAGES + cs], (par >> (STAGES + cs)) & 1, a.status);
         par ^= 1u << (STAGES + cs);
         pend &= ~(1u << (STAGES + cs));
       } else {
-        for (int i = tid; i < rows * W; i += kRows) {
+        for (int i = lane; i < rows * W; i += kWR) {
           const int r = i / W, w = i - r * W;
           stage_codes[i] = __ldg(a.codes_in + (row0 + r) * a.ldc + w);
         }
       }
-      if (tid == 0) bulk_wait_read<0>();  // earlier x_hat stores have left the tile buffers
+      if (lane == 0) bulk_wait_read<0>();  // earlier x_hat stores have left the sub-tile buffer
     }
-    if (!__syncthreads_and(ok)) {
-      // a wait ran out: wait (bounded) for this CTA's other copies, then leave
-      if (tid == 0)
+    __syncwarp();
+    if (!__all_sync(0xffffffffu, ok)) {
+      // a wait ran out: wait (bounded) for this warp's other copies, then leave
+      if (lane == 0)
         for (int b = 0; b < STAGES + 2; ++b)
-          if ((pend >> b) & 1) mbar_wait(&s_bar[b], (par >> b) & 1, a.status);
+          if ((pend >> b) & 1) mbar_wait(&w_bar[b], (par >> b) & 1, a.status);
       break;
     }
 
@@ -329,7 +338,7 @@ __global__ void __launch_bounds__(kRows, MODE == RQ_Q ? 2 : KVRQ_ROW_MIN_BLOCKS)
 #pragma unroll
       for (int j = 0; j < TL::kChunks; ++j) {
         float f[E];
-        Elem<T>::unpack(*reinterpret_cast<const uint4*>(tb + TL::chunk(tid, j)), f);
+        Elem<T>::unpack(*reinterpret_cast<const uint4*>(tb + TL::chunk(lane, j)), f);
 #pragma unroll
         for (int k = 0; k < E / 2; ++k) {
           const float2 v = make_float2(f[2 * k], f[2 * k + 1]);
@@ -343,17 +352,17 @@ __global__ void __launch_bounds__(kRows, MODE == RQ_Q ? 2 : KVRQ_ROW_MIN_BLOCKS)
 #pragma unroll 1
         for (int j = 0; j < TL::kChunks; ++j) {
           float f[E];
-          Elem<T>::unpack(*reinterpret_cast<const uint4*>(tb + TL::chunk(tid, j)), f);
+          Elem<T>::unpack(*reinterpret_cast<const uint4*>(tb + TL::chunk(lane, j)), f);
           for (int k = 0; k < E; ++k) ss = fmaf(f[k] * xs, f[k] * xs, ss);
         }
       }
       nq = sqrtf(ss);
       nrm = kScale ? nq / xs : nq;
     } else {
-      nrm = tid < rows ? __ldg(a.norms_in + row * a.ldn) : 0.f;
+      nrm = lane < rows ? __ldg(a.norms_in + row * a.ldn) : 0.f;
       nq = nrm;
 #pragma unroll
-      for (int w = 0; w < W; ++w) wc[w] = stage_codes[tid * W + w];
+      for (int w = 0; w < W; ++w) wc[w] = stage_codes[lane * W + w];
     }
 
     // scaled magnitudes as a chain: chain(0) = mag_0 ||x||, chain(j) = chain(j-1) + delta_j
@@ -406,7 +415,7 @@ __global__ void __launch_bounds__(kRows, MODE == RQ_Q ? 2 : KVRQ_ROW_MIN_BLOCKS)
 #pragma unroll
         for (int e = 6 * p; e < 6 * p + 6; ++e) {
           if (e < D && e % E == 0) {
-            Elem<T>::unpack(*reinterpret_cast<const uint4*>(tb + TL::chunk(tid, e / E)), &xe[e]);
+            Elem<T>::unpack(*reinterpret_cast<const uint4*>(tb + TL::chunk(lane, e / E)), &xe[e]);
             if constexpr (kScale) {
 #pragma unroll
               for (int k = 0; k < E; ++k) xe[e + k] *= xs;
@@ -464,7 +473,7 @@ __global__ void __launch_bounds__(kRows, MODE == RQ_Q ? 2 : KVRQ_ROW_MIN_BLOCKS)
           const int last_code = ((32 * wi + 31) / BITS) < NC ? (32 * wi + 31) / BITS : NC - 1;
           const int win_end = ((last_code / CPW) + 1) * CPW < NC ? ((last_code / CPW) + 1) * CPW : NC;
           const int prev_done = 6 * p < NC ? 6 * p : NC;
-          if (win_end <= done && win_end > prev_done) stage_codes[tid * W + wi] = wc[wi];
+          if (win_end <= done && win_end > prev_done) stage_codes[lane * W + wi] = wc[wi];
         }
       } else {
 #pragma unroll
@@ -485,51 +494,52 @@ __global__ void __launch_bounds__(kRows, MODE == RQ_Q ? 2 : KVRQ_ROW_MIN_BLOCKS)
 #pragma unroll
         for (int e = 6 * p; e < 6 * p + 6; ++e)
           if (e < D && e % E == E - 1)
-            *reinterpret_cast<uint4*>(tb + TL::chunk(tid, e / E)) = Elem<T>::pack(&xo[e - (E - 1)]);
+            *reinterpret_cast<uint4*>(tb + TL::chunk(lane, e / E)) = Elem<T>::pack(&xo[e - (E - 1)]);
       }
     }
 
     // ---------------------------------------------------------------- outputs
     if constexpr (kIn) {
-      if (tid < rows && a.norms_out) a.norms_out[row * a.ldn] = nrm;
+      if (lane < rows && a.norms_out) a.norms_out[row * a.ldn] = nrm;
     }
-    // a full tile of codes leaves as one bulk copy when code rows are contiguous
-    const bool codes_bulk_out = kIn && a.codes_out && rows == kRows && a.ldc == W &&
+    // a full sub-tile of codes leaves as one bulk copy when code rows are contiguous
+    const bool codes_bulk_out = kIn && a.codes_out && rows == kWR && a.ldc == W &&
                                 (reinterpret_cast<uintptr_t>(a.codes_out) & 15) == 0;
     fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {
+    __syncwarp();
+    if (lane == 0) {
       if constexpr (kOut) {
 #pragma unroll
         for (int b = 0; b < TL::kBoxes; ++b) tma_store_2d(&map_o, b * TL::kBoxElems, (int32_t)row0, tb + b * TL::kBoxBytes);
       }
-      if (codes_bulk_out) bulk_store(a.codes_out + row0 * W, stage_codes, kRows * W * 4);
+      if (codes_bulk_out) bulk_store(a.codes_out + row0 * W, stage_codes, kWR * W * 4);
       if (kOut || codes_bulk_out) bulk_commit();
       if constexpr (kIn) {
-        const int64_t next = tile_of(it + STAGES);
-        if (next < ntiles) {
+        const int next = sub_of(it + STAGES);
+        if (next < nsub) {
           if (kOut) bulk_wait_read<0>();  // the x_hat store has read this buffer
           issue_tile(next, s);
         }
       } else {
-        const int64_t next = tile_of(it + 2);
-        if (next < ntiles && codes_bulk_tile(next)) issue_codes(next, cs);
+        const int next = sub_of(it + 2);
+        if (next < nsub && codes_bulk_tile(next)) issue_codes(next, cs);
       }
     }
     if constexpr (kIn) {
       if (a.codes_out && !codes_bulk_out)
-        for (int i = tid; i < rows * W; i += kRows) {
+        for (int i = lane; i < rows * W; i += kWR) {
           const int r = i / W, w = i - r * W;
           a.codes_out[(row0 + r) * a.ldc + w] = stage_codes[i];
         }
     }
   }
-  if (tid == 0) bulk_wait_all<0>();
+  if (lane == 0) bulk_wait_all<0>();
 }
 
 }  // namespace row
 
 using row::rq_row_kernel;
+
 
 
 // ============================================================================
@@ -648,8 +658,8 @@ static cudaError_t launch_row_s(const CUtensorMap& mx, const CUtensorMap& mo, co
     if (e != cudaSuccess) return e;
     blocks_per_sm = b < 1 ? 1 : b;
   }
-  const int64_t ntiles = (a.n + row::kRows - 1) / row::kRows;
-  const int64_t grid = std::min<int64_t>(ntiles, (int64_t)num_sms * blocks_per_sm);
+  const int64_t nsub = (a.n + row::kWR - 1) / row::kWR;
+  const int64_t grid = std::min<int64_t>((nsub + row::kWarps - 1) / row::kWarps, (int64_t)num_sms * blocks_per_sm);
   kern<<<(unsigned)grid, row::kRows, SM::alloc, st>>>(mx, mo, a);
   return cudaGetLastError();
 }
@@ -664,6 +674,8 @@ static int row_stages() {
   }
   return stages;
 }
+
+int rq_row_box_rows() { return row::kWR; }
 
 template <typename T, int BITS, int MODE>
 static cudaError_t launch_row(const CUtensorMap& mx, const CUtensorMap& mo, const RqArgs& a, cudaStream_t st,

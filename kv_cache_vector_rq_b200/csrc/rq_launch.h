@@ -33,9 +33,12 @@ struct RqArgs {
 };
 
 // d = 128 thread-per-row kernel fed by TMA tensor maps over x and x_hat
-// (128-byte boxes of 128 rows, 128-byte swizzle).
+// (128-byte boxes of 32 rows, 128-byte swizzle: one box per warp sub-tile).
 cudaError_t launch_rq_row(int mode, kvrq_dtype dt, int bits, const CUtensorMap& map_x, const CUtensorMap& map_o,
                           const RqArgs& a, cudaStream_t st, int num_sms);
+
+// Rows per box of the tensor maps launch_rq_row expects.
+int rq_row_box_rows();
 
 // Any d / stride, warp-per-row kernel.
 cudaError_t launch_rq_general(int mode, kvrq_dtype dt_in, kvrq_dtype dt_out, int bits, const RqArgs& a,
