@@ -616,13 +616,20 @@ kvrq_status kv_score_packed(void* stream, kvrq_method method, const void* q, kvr
   a.n_heads = n_heads;
   a.group = group;
   a.n_tokens = n_tokens;
-  // about two CTAs per SM in total (one runs per SM): each CTA rotates its queries
-  // once, so long token ranges amortise that prologue
-  int64_t tiles = (n_tokens + 127) / 128;
-  int64_t per = (tiles * n_heads + 2LL * di->num_sms - 1) / (2LL * di->num_sms);
-  if (per < 4) per = 4;
-  if (per > tiles) per = tiles;
-  a.tokens_per_cta = per * 128;
+  // One CTA runs per SM. A head's tokens are cut into c ranges so that the waves
+  // of CTAs times the tiles per CTA (plus the query-rotation prologue, worth about
+  // four tiles) is smallest.
+  const int64_t tiles = (n_tokens + 127) / 128;
+  int64_t best_c = 1, best_cost = -1;
+  for (int64_t c = 1; c <= tiles && c <= 256; ++c) {
+    const int64_t waves = (n_heads * c + di->num_sms - 1) / di->num_sms;
+    const int64_t cost = waves * ((tiles + c - 1) / c + 4);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best_c = c;
+    }
+  }
+  a.tokens_per_cta = ((tiles + best_c - 1) / best_c) * 128;
   a.q = q;
   a.ldq = ldq;
   a.q_f32 = qdtype == KVRQ_F32;

@@ -8,18 +8,24 @@
 // directly from the compressed indices. For RotorQuant the same identity holds
 // per group: <q, x_hat> = ||x|| sum_g <R_g q_g R_g~, c_hat_g>, q zero-padded.
 //
-// B200 design: a CTA of 256 threads owns one KV head and a contiguous token
-// range. It rotates the head's query group once (Pi q and T Pi q from staged
-// copies of Pi and T, or the per-group sandwich) into the MMA B operand (N = 16..
-// rows, fp16). Then, per 128-token tile: packed code rows arrive by bulk copy
-// (a ring of eight tiles in flight); the two warpgroups decode the tile's keys into a
-// 128-byte-swizzled fp16 A tile (warpgroup 0 the first half of K, warpgroup 1
-// the second: for TurboQuant-prod the centroids and the +1/-1 signs) through
-// small shared-memory tables; one thread issues tcgen05.mma (M = 128 tokens)
-// into one of two TMEM accumulators; while it runs, warpgroup 1 finishes the
-// previous tile (one TMEM lane per token: ||k|| and the QJL term, fp32 scores
-// written coalesced across tokens) and both warpgroups decode the next one into
-// the other A buffer.
+// B200 design. A CTA owns one KV head and a contiguous token range. It rotates
+// the head's query group once (Pi q and T Pi q from staged copies of Pi and T,
+// or the per-group sandwich) into the MMA B operand (N = 16..64 rows, fp16, in
+// shared memory). Keys are then handled in 128-token tiles, the M = 128 rows
+// of the MMA, by two decode warpgroups that alternate tiles:
+//   * packed code rows (and sign rows) arrive by bulk copy into a ring of
+//     stages per warpgroup, issued by one control thread;
+//   * each thread decodes its key into fp16 operand words through small
+//     shared-memory tables (one lookup per 8-bit or 6-bit field of codes, and
+//     per byte of signs), replicated per lane so that the lookups of a warp
+//     never collide on a bank, and writes them with tcgen05.st straight into
+//     its lane of the warpgroup's A region in tensor memory -- the decoded keys
+//     never pass through shared memory;
+//   * the control thread issues tcgen05.mma with A in tensor memory and B in
+//     shared memory into one of the warpgroup's two accumulators;
+//   * while the next tile is being decoded the warpgroup reads the previous
+//     tile's accumulator row per thread (||k|| and the QJL term) and writes
+//     fp32 scores, coalesced across tokens.
 
 #include <cuda_runtime.h>
 
@@ -31,18 +37,26 @@
 namespace kvrq {
 namespace score {
 
-constexpr int kRows = 128;     // tokens per tile
-constexpr int kThreads = 256;  // two warpgroups
-constexpr int kStages = 8;     // packed-code tiles in flight per CTA
+constexpr int kRows = 128;                  // tokens per tile (TMEM lanes)
+constexpr int kNWG = 2;                     // decode warpgroups
+constexpr int kThreads = kNWG * 128 + 32;   // + one control warp
+constexpr int kStages = 4;                  // code stages per warpgroup
+constexpr uint32_t kTmemCols = 512;
 
-// Codes per lookup for a stored code width b: the table maps a field of
-// kPer * b bits to kPer fp16 centroids.
+// Decode table of the stored codes (width b): an f-bit field of P codes maps to
+// P fp16 centroids (EW 32-bit words); every entry is replicated R times, R
+// consecutive copies filling 128 bytes, and lane l reads copy l % R, so the
+// lanes of one shared-memory wavefront (8, 16 or 32 lanes for 16-, 8- and
+// 4-byte entries) hit distinct banks whatever the field values.
 template <int BITS>
 struct Dec {
-  static constexpr int kPer = BITS == 1 ? 8 : BITS == 2 ? 4 : 2;
-  static constexpr int kFieldBits = kPer * BITS;    // 8, 8, 6, 8
-  static constexpr int kEntries = 1 << kFieldBits;  // 256, 256, 64, 256
-  static constexpr int kEntryBytes = kPer * 2;      // 16, 8, 4, 4
+  static constexpr int FB = BITS == 3 ? 6 : 8;  // field bits
+  static constexpr int P = FB / BITS;            // codes per field: 8, 4, 2, 2
+  static constexpr int EW = P / 2;               // words per entry
+  static constexpr int EB = 4 * EW;
+  static constexpr int R = 128 / EB;             // replicas
+  static constexpr int ENT = 1 << FB;
+  static constexpr int BYTES = ENT * 128;
 };
 
 template <int METHOD, int BITS, int NB>
@@ -52,35 +66,45 @@ struct Cfg {
   static constexpr int NCODE = METHOD == KVRQ_RQ_MSE ? 129 : 128;  // stored codes per key
   static constexpr int KC = METHOD == KVRQ_RQ_MSE ? 144 : 128;     // MMA K of the centroid part
   static constexpr int K = KC + (kProd ? 128 : 0);                 // total MMA K
-  static constexpr int KBOX = (K + 63) / 64;                        // 64-element boxes per row
+  static constexpr int KA = K / 2;                                  // A columns in TMEM (fp16 pairs)
+  static constexpr int KAP = (KA + 31) / 32 * 32;                   // A region, 32-column aligned
+  static constexpr int KBOX = (K + 63) / 64;                        // 64-element B boxes per row
   static constexpr int W = (NCODE * BITS + 31) / 32;                // code words per key
   static constexpr int NS = kProd ? 4 : 0;                          // sign words per key (m = 128)
-  static constexpr int A_BOX = kRows * 128;                         // A: box of 128 rows
-  static constexpr int A_BYTES = KBOX * A_BOX;
-  static constexpr int B_BOX = NB * 128;                            // B: box of NB rows
+  static constexpr int B_BOX = NB * 128;
   static constexpr int QS = D + 16;                                 // row stride of the query scratch
-  static constexpr int q_bytes = 2 * NB * QS * 4;                   // fp32 rotated queries (prologue only)
   static constexpr int MS = 130;                                    // padded row (halves) of a staged matrix
-  static constexpr int m_off = ((q_bytes + 15) / 16) * 16;          // staged Pi or T (prologue only)
-  static constexpr int pro_bytes = m_off + D * MS * 2;
-  static constexpr int a_bytes = 2 * A_BYTES > pro_bytes ? 2 * A_BYTES : pro_bytes;
-  static constexpr int a_off = 0;  // two A buffers; the prologue scratch aliases them
-  static constexpr int b_off = ((a_bytes + 1023) / 1024) * 1024;
-  static constexpr int stage_words = ((kRows * (W + NS) + 3) / 4) * 4;  // codes then signs, per tile
-  static constexpr int stage_off = b_off + KBOX * B_BOX;
-  static constexpr int lut_off = stage_off + kStages * stage_words * 4;
-  static constexpr int lut_bytes = Dec<BITS>::kEntries * Dec<BITS>::kEntryBytes;
-  static constexpr int slut_off = lut_off + lut_bytes;  // sign table: byte -> 8 x (+1/-1)
-  static constexpr int slut_bytes = kProd ? 256 * 16 : 0;
-  static constexpr int bar_off = slut_off + slut_bytes;  // [0, kStages) code stages, then 2 mma buffers
-  static constexpr int tmem_off = bar_off + (kStages + 2) * 8;
-  static constexpr int bytes = tmem_off + 16;
-  static constexpr int alloc = bytes + 1024;
-  static constexpr uint32_t kNcols = 2 * NB < 32 ? 32 : 2 * NB;  // two accumulators
-  // K columns of the centroid part decoded by warpgroup 0 (the rest by warpgroup 1);
-  // for prod warpgroup 0 decodes all centroids and warpgroup 1 the signs
-  static constexpr int KSPLIT = kProd ? KC : (KC / 16) * 8;
+  // TMEM columns per warpgroup: A, then two accumulators
+  static constexpr int WCOLS = (KAP + 2 * NB + 31) / 32 * 32;
+  static_assert(kNWG * WCOLS <= (int)kTmemCols, "tensor memory");
+  // shared memory
+  static constexpr int stage_words = kRows * (W + NS);
+  static constexpr int lut_bytes = Dec<BITS>::BYTES;
+  static constexpr int slut_bytes = kProd ? 256 * 128 : 0;  // byte of signs -> 8 x (+1/-1), 8 replicas
+  static constexpr int lut_off = 0;
+  static constexpr int slut_off = lut_off + lut_bytes;
+  static constexpr int stage_off = slut_off + slut_bytes;
+  static constexpr int ring_end = stage_off + kNWG * kStages * stage_words * 4;
+  // prologue scratch (rotated queries, staged Pi or T) aliases tables and stages
+  static constexpr int q_bytes = 2 * NB * QS * 4;
+  static constexpr int m_off = ((q_bytes + 15) / 16) * 16;
+  static constexpr int pro_end = m_off + D * MS * 2;
+  static constexpr int b_off = (((ring_end > pro_end ? ring_end : pro_end) + 1023) / 1024) * 1024;
+  static constexpr int bar_off = b_off + KBOX * B_BOX;
+  // barriers: stage full [kNWG][kStages], A written [kNWG], accumulator full [kNWG][2], done
+  static constexpr int nbars = kNWG * kStages + kNWG + 2 * kNWG + 1;
+  static constexpr int tmem_off = bar_off + nbars * 8;
+  static constexpr int alloc = tmem_off + 16 + 1024;
 };
+
+// field of `FB` bits starting at bit `bit` of the little-endian stream in w[0..NW)
+template <int FB, int NW>
+__device__ __forceinline__ uint32_t field(const uint32_t (&w)[NW], int bit) {
+  const int wi = bit >> 5, sh = bit & 31;
+  uint32_t v = w[wi] >> sh;
+  if (sh + FB > 32 && wi + 1 < NW) v |= w[wi + 1] << (32 - sh);
+  return v & ((1u << FB) - 1u);
+}
 
 template <int METHOD, int BITS, int NB>
 __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs a) {
@@ -92,17 +116,19 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs a) {
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* s_a = smem + C::a_off;
   uint8_t* s_b = smem + C::b_off;
   uint32_t* s_stage = reinterpret_cast<uint32_t*>(smem + C::stage_off);
-  uint8_t* s_lut = smem + C::lut_off;
-  uint8_t* s_slut = smem + C::slut_off;
+  const uint8_t* s_lut = smem + C::lut_off;
+  const uint8_t* s_slut = smem + C::slut_off;
   float* s_q = reinterpret_cast<float*>(smem);
   uint64_t* s_bar = reinterpret_cast<uint64_t*>(smem + C::bar_off);
+  uint64_t* bar_stage = s_bar;                   // [w * kStages + s]
+  uint64_t* bar_afull = s_bar + kNWG * kStages;  // [w]
+  uint64_t* bar_acc = bar_afull + kNWG;          // [w * 2 + b]
+  uint64_t* bar_done = bar_acc + 2 * kNWG;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::tmem_off);
 
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int wg = tid >> 7, key = tid & 127;  // warpgroup, token within the tile
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = a.group;
   const int64_t head = blockIdx.y;
   const int64_t t_begin = (int64_t)blockIdx.x * a.tokens_per_cta;
@@ -115,28 +141,16 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs a) {
   // code rows of a tile are one contiguous, 16-byte aligned block when unpadded
   const bool bulk = a.ldc == W && (!kProd || a.lds == NS) && ((reinterpret_cast<uintptr_t>(codes_h) & 15) == 0) &&
                     (!kProd || (reinterpret_cast<uintptr_t>(signs_h) & 15) == 0) && ((kRows * W * 4) % 16 == 0);
+  auto tile_full = [&](int j) { return t_begin + (int64_t)(j + 1) * kRows <= t_end; };
 
   if (tid == 0) {
-    for (int s = 0; s < kStages + 2; ++s) mbar_init(&s_bar[s], 1);
+    for (int s = 0; s < C::nbars; ++s) {
+      const bool afull = s >= kNWG * kStages && s < kNWG * kStages + kNWG;  // every decoder arrives
+      mbar_init(&s_bar[s], afull ? 128 : 1);
+    }
     fence_barrier_init();
   }
-  if (warp == 0) tmem_alloc(s_tmem, C::kNcols);
-
-  // ---------------------------------------------------------------- decode tables
-  {
-    const float* cb = a.centroids;
-    for (int e = tid; e < DC::kEntries; e += kThreads) {
-#pragma unroll
-      for (int j = 0; j < DC::kPer; ++j)
-        reinterpret_cast<__half*>(s_lut + e * DC::kEntryBytes)[j] =
-            __float2half_rn(cb[(e >> (j * BITS)) & ((1 << BITS) - 1)]);
-    }
-    if (kProd)
-      for (int e = tid; e < 256; e += kThreads)
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          reinterpret_cast<__half*>(s_slut + e * 16)[j] = __float2half_rn(((e >> j) & 1) ? 1.f : -1.f);
-  }
+  if (warp == 0) tmem_alloc(s_tmem, kTmemCols);
 
   // ---------------------------------------------------------------- rotated queries
   // s_q rows [0, G): q' (fp32); rows [NB, NB + G): the raw queries, later (T q')
@@ -168,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs a) {
     }
   } else {
     // q' = Pi q: Pi staged in shared memory (coalesced 16-byte loads, padded rows), then
-    // thread i < 128 forms row i of Pi against every query of the group
+    // out[g][i] = sum_k M[i][k] vec[g][k] with one (g, i) per thread and step
     uint16_t* s_m = reinterpret_cast<uint16_t*>(smem + C::m_off);
     auto stage = [&](const void* src) {
       const uint4* g = reinterpret_cast<const uint4*>(src);
@@ -181,8 +195,6 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs a) {
         d32[3] = v.w;
       }
     };
-    // out[g][i] = sum_k M[i][k] vec[g][k], one (g, i) per thread and step: a warp covers
-    // consecutive i of one g (conflict-free padded rows, broadcast vector)
     auto mat_vec = [&](bool bf16, const float* vec_base, float* out_base) {
       for (int idx = tid; idx < G * D; idx += kThreads) {
         const int g = idx / D, i = idx - g * D;
@@ -237,171 +249,217 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs a) {
     }
     *reinterpret_cast<uint4*>(s_b + sw128_chunk(row, j, C::B_BOX)) = Elem<__half>::pack(v);
   }
-  __syncthreads();  // the prologue scratch (aliasing the A buffers) has been read
-  // zero both A buffers once (their unused K columns stay zero)
-  for (int i = tid; i < 2 * C::A_BYTES / 16; i += kThreads) reinterpret_cast<uint4*>(s_a)[i] = make_uint4(0, 0, 0, 0);
-  fence_proxy_async_smem();
+  __syncthreads();  // the prologue scratch (aliasing the tables and stages) has been read
+
+  // ---------------------------------------------------------------- decode tables
+  {
+    const float* cb = a.centroids;
+    // 16-bit slot s of entry e: replica s / P, code j = s % P of the field
+    for (int i = tid; i < DC::ENT * 64; i += kThreads) {
+      const int e = i >> 6, j = (i & 63) % DC::P;
+      reinterpret_cast<__half*>(smem + C::lut_off)[i] = __float2half_rn(cb[(e >> (j * BITS)) & ((1 << BITS) - 1)]);
+    }
+    if (kProd)
+      for (int i = tid; i < 256 * 64; i += kThreads) {
+        const int e = i >> 6, j = (i & 63) % 8;
+        reinterpret_cast<__half*>(smem + C::slut_off)[i] = __float2half_rn(((e >> j) & 1) ? 1.f : -1.f);
+      }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
-  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-  const uint32_t a_s = smem_u32(s_a), b_s = smem_u32(s_b);
+  const uint32_t b_s = smem_u32(s_b);
 
-  auto tile_full = [&](int it) { return t_begin + (int64_t)(it + 1) * kRows <= t_end; };
-  auto issue_stage = [&](int it, int st) {  // thread 0
-    const int64_t t0 = t_begin + (int64_t)it * kRows;
-    uint32_t* dst = s_stage + st * C::stage_words;
-    mbar_arrive_expect_tx(&s_bar[st], kRows * (W + NS) * 4);
-    bulk_load(dst, codes_h + t0 * W, kRows * W * 4, &s_bar[st]);
-    if (kProd) bulk_load(dst + kRows * W, signs_h + t0 * NS, kRows * NS * 4, &s_bar[st]);
-  };
-  uint32_t par = 0;  // bit s: parity of the next phase of barrier s
-  if (tid == 0 && bulk)
-    for (int it = 0; it < kStages && it < ntiles; ++it)
-      if (tile_full(it)) issue_stage(it, it);
+  if (warp == kNWG * 4) {
+    // ------------------------------------------------------------ control thread: copies and MMAs
+    if (lane == 0) {
+      auto issue_stage = [&](int j) {
+        const int w = j % kNWG, i = j / kNWG, s = i % kStages;
+        const int64_t t0 = t_begin + (int64_t)j * kRows;
+        uint32_t* dst = s_stage + (w * kStages + s) * C::stage_words;
+        uint64_t* bar = &bar_stage[w * kStages + s];
+        mbar_arrive_expect_tx(bar, kRows * (W + NS) * 4);
+        bulk_load(dst, codes_h + t0 * W, kRows * W * 4, bar);
+        if (kProd) bulk_load(dst + kRows * W, signs_h + t0 * NS, kRows * NS * 4, bar);
+      };
+      if (bulk)
+        for (int j = 0; j < kStages * kNWG && j < ntiles; ++j)
+          if (tile_full(j)) issue_stage(j);
+      bool ok = true;
+      for (int j = 0; j < ntiles && ok; ++j) {
+        const int w = j % kNWG, i = j / kNWG;
+        if (!(ok = mbar_wait(&bar_afull[w], (uint32_t)(i & 1), a.status))) break;
+        tc_fence_after();
+        const uint32_t a_t = tmem + (uint32_t)(w * C::WCOLS);
+        const uint32_t d_t = a_t + (uint32_t)(C::KAP + (i & 1) * NB);
+#pragma unroll
+        for (int kk = 0; kk < K / 16; ++kk) {
+          const uint32_t boff = (uint32_t)((kk >> 2) * C::B_BOX + (kk & 3) * 32);
+          umma_f16_ts(d_t, a_t + (uint32_t)(8 * kk), umma_desc_sw128(b_s + boff, 16, 1024), kIdesc, kk > 0);
+        }
+        umma_commit(&bar_acc[w * 2 + (i & 1)]);
+        // the tile's code stage has been read by the decoders: refill it
+        const int jn = j + kStages * kNWG;
+        if (bulk && jn < ntiles && tile_full(jn)) issue_stage(jn);
+      }
+      umma_commit(bar_done);  // every MMA issued has completed before TMEM is released
+      mbar_wait(bar_done, 0, a.status);
+    }
+  } else {
+    // ------------------------------------------------------------ decode warpgroups
+    const int w = warp >> 2;  // warpgroup
+    const int r = tid & 127;  // key row of the tile = TMEM lane
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t a_t = tmem + lane_off + (uint32_t)(w * C::WCOLS);
+    const uint32_t acc_t = a_t + (uint32_t)C::KAP;
+    const uint8_t* lut_l = s_lut + (lane % DC::R) * DC::EB;  // this lane's replica
+    const uint8_t* slut_l = s_slut + (lane & 7) * 16;
+    bool ok = true;
+    float prev_n = 0.f, prev_g = 0.f;
 
-  // epilogue of tile `pt` (warpgroup 1): scores from accumulator pt & 1
-  auto epilogue = [&](int pt, float nrm, float gam) {
-    const int64_t t0 = t_begin + (int64_t)pt * kRows;
-    const int rows = (int)(t_end - t0 < (int64_t)kRows ? t_end - t0 : (int64_t)kRows);
-    const int64_t t = t0 + key;
-    // NB columns of accumulator pt & 1 (a multiple of 16; never past the allocation)
-    float acc[NB];
+    auto epilogue = [&](int jp, int ip, float nrm, float gam) {
+      const int64_t t0 = t_begin + (int64_t)jp * kRows;
+      const int rows = (int)(t_end - t0 < (int64_t)kRows ? t_end - t0 : (int64_t)kRows);
+      float acc[NB];
 #pragma unroll
-    for (int c = 0; c < NB / 16; ++c) tmem_ld16(tmem + lane_off + (uint32_t)((pt & 1) * NB) + 16 * c, &acc[16 * c]);
-    if (key < rows) {
-      const float qs = a.qjl_scale * gam;
+      for (int c = 0; c < NB / 16; ++c) tmem_ld16(acc_t + (uint32_t)((ip & 1) * NB + 16 * c), &acc[16 * c]);
+      if (r < rows) {
+        const float qs = a.qjl_scale * gam;
+        const int64_t t = t0 + r;
 #pragma unroll
-      for (int g = 0; g < (kProd ? NB / 2 : NB); ++g) {
-        if (g < G) {
-          float s = acc[g];
-          if (kProd) s = fmaf(qs, acc[NB / 2 + g], s);
-          a.scores[(head * G + g) * a.ld_scores + t] = nrm * s;
+        for (int g = 0; g < (kProd ? NB / 2 : NB); ++g) {
+          if (g < G) {
+            float s = acc[g];
+            if (kProd) s = fmaf(qs, acc[NB / 2 + g], s);
+            a.scores[(head * G + g) * a.ld_scores + t] = nrm * s;
+          }
         }
       }
-    }
-  };
+    };
 
-  bool ok = true;
-  float prev_n = 0.f, prev_g = 0.f;  // norm / gamma of this thread's key in the previous tile
-  for (int it = 0; it < ntiles; ++it) {
-    const int st = it % kStages, ab = it & 1;
-    constexpr int MB = kStages;  // first mma-buffer barrier
-    const int64_t t0 = t_begin + (int64_t)it * kRows;
-    const int rows = (int)(t_end - t0 < (int64_t)kRows ? t_end - t0 : (int64_t)kRows);
-    uint32_t* stg = s_stage + st * C::stage_words;
-    uint8_t* A = s_a + ab * C::A_BYTES;
-    const float nrm = (wg == 1 && key < rows) ? __ldg(norms_h + t0 + key) : 0.f;
-    const float gam = (kProd && wg == 1 && key < rows) ? __ldg(gammas_h + t0 + key) : 0.f;
-    if (bulk && tile_full(it)) {
-      ok = mbar_wait(&s_bar[st], (par >> st) & 1, a.status) && ok;
-      par ^= 1u << st;
-    } else {
-      for (int i = tid; i < rows * W; i += kThreads) {
-        const int r = i / W, w = i - r * W;
-        stg[i] = __ldg(codes_h + (t0 + r) * a.ldc + w);
-      }
-      if (kProd)
-        for (int i = tid; i < rows * NS; i += kThreads) {
-          const int r = i / NS, w = i - r * NS;
-          stg[kRows * W + i] = __ldg(signs_h + (t0 + r) * a.lds + w);
+    int i = 0;
+    for (int j = w; j < ntiles; j += kNWG, ++i) {
+      const int s = i % kStages;
+      const int64_t t0 = t_begin + (int64_t)j * kRows;
+      const int rows = (int)(t_end - t0 < (int64_t)kRows ? t_end - t0 : (int64_t)kRows);
+      const float nrm = r < rows ? __ldg(norms_h + t0 + r) : 0.f;
+      const float gam = (kProd && r < rows) ? __ldg(gammas_h + t0 + r) : 0.f;
+      // this key's packed codes and signs
+      uint32_t wc[W], sg[NS > 0 ? NS : 1];
+      if (bulk && tile_full(j)) {
+        if (!(ok = mbar_wait(&bar_stage[w * kStages + s], (uint32_t)((i / kStages) & 1), a.status))) break;
+        const uint32_t* stg = s_stage + (w * kStages + s) * C::stage_words;
+        if constexpr (W % 4 == 0) {
+#pragma unroll
+          for (int q = 0; q < W / 4; ++q) {
+            const uint4 v = *reinterpret_cast<const uint4*>(stg + r * W + 4 * q);
+            wc[4 * q] = v.x;
+            wc[4 * q + 1] = v.y;
+            wc[4 * q + 2] = v.z;
+            wc[4 * q + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < W; ++q) wc[q] = stg[r * W + q];
         }
-      for (int i = rows * W + tid; i < kRows * W; i += kThreads) stg[i] = 0u;  // ragged tail decodes to zero
-      if (kProd)
-        for (int i = rows * NS + tid; i < kRows * NS; i += kThreads) stg[kRows * W + i] = 0u;
-    }
-    if (!__syncthreads_and(ok)) break;
+        if constexpr (kProd) {
+          const uint4 v = *reinterpret_cast<const uint4*>(stg + kRows * W + r * NS);
+          sg[0] = v.x;
+          sg[1] = v.y;
+          sg[2] = v.z;
+          sg[3] = v.w;
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < W; ++q) wc[q] = r < rows ? __ldg(codes_h + (t0 + r) * a.ldc + q) : 0u;
+        if constexpr (kProd) {
+#pragma unroll
+          for (int q = 0; q < NS; ++q) sg[q] = r < rows ? __ldg(signs_h + (t0 + r) * a.lds + q) : 0u;
+        }
+      }
+      // the previous tile's MMA has finished with A: its scores, then this tile's decode
+      if (i > 0) {
+        if (!(ok = mbar_wait(&bar_acc[w * 2 + ((i - 1) & 1)], (uint32_t)(((i - 1) >> 1) & 1), a.status))) break;
+        tc_fence_after();
+        epilogue(j - kNWG, i - 1, prev_n, prev_g);
+      }
+      prev_n = nrm;
+      prev_g = gam;
 
-    // ------------------------------------------------------------ decode key `key` into A[ab]
-    if (!kProd || wg == 0) {
-      constexpr int P = DC::kPer, FB = DC::kFieldBits;
-      constexpr int NF = (C::NCODE + P - 1) / P;
-      uint32_t wc[W];
+      // centroid part: A words [0, KC/2), 32 at a time
+      constexpr int FPC = 64 / DC::P;  // fields per 32 words
 #pragma unroll
-      for (int w = 0; w < W; ++w) wc[w] = stg[key * W + w];
-      uint32_t rw[KC / 2];
+      for (int c = 0; c < (KC / 2 + 31) / 32; ++c) {
+        uint32_t rw[32];
 #pragma unroll
-      for (int k = 0; k < KC / 2; ++k) rw[k] = 0u;
-      // fields of warpgroup 0 (or, for prod, all) / of warpgroup 1
-      const int f_lo = (kProd || wg == 0) ? 0 : C::KSPLIT / P;
-      const int f_hi = (kProd || wg == 1) ? NF : C::KSPLIT / P;
+        for (int f = 0; f < FPC; ++f) {
+          const int fi = c * FPC + f;  // field index: codes fi*P .. fi*P + P - 1
+          if (fi * DC::P < C::NCODE) {
+            const uint32_t v = field<DC::FB, W>(wc, fi * DC::FB);
+            const uint8_t* e = lut_l + v * 128;
+            if constexpr (DC::EW == 4) {
+              const uint4 x = *reinterpret_cast<const uint4*>(e);
+              rw[4 * f] = x.x;
+              rw[4 * f + 1] = x.y;
+              rw[4 * f + 2] = x.z;
+              rw[4 * f + 3] = x.w;
+            } else if constexpr (DC::EW == 2) {
+              const uint2 x = *reinterpret_cast<const uint2*>(e);
+              rw[2 * f] = x.x;
+              rw[2 * f + 1] = x.y;
+            } else {
+              rw[f] = *reinterpret_cast<const uint32_t*>(e);
+            }
+          } else {
 #pragma unroll
-      for (int f = 0; f < NF; ++f) {
-        if (f < f_lo || f >= f_hi) continue;
-        const int bit = f * FB, word = bit >> 5, sh = bit & 31;
-        uint32_t v = wc[word] >> sh;
-        if (sh + FB > 32 && word + 1 < W) v |= wc[word + 1] << (32 - sh);
-        v &= (1u << FB) - 1u;
-        const uint32_t* e = reinterpret_cast<const uint32_t*>(s_lut + v * DC::kEntryBytes);
-        const int valid = C::NCODE - f * P;  // stored codes in this field
+            for (int q = 0; q < DC::EW; ++q) rw[DC::EW * f + q] = 0u;
+          }
+          // K elements past the stored codes (the RotorQuant tail) are zero
 #pragma unroll
-        for (int k = 0; k < P / 2; ++k) {
-          uint32_t wv = e[k];
-          if (2 * k >= valid) wv = 0u;
-          else if (2 * k + 1 >= valid) wv &= 0xFFFFu;
-          rw[f * P / 2 + k] = wv;
+          for (int q = 0; q < DC::EW; ++q) {
+            const int k0 = 2 * (32 * c + DC::EW * f + q);  // first K element of this word
+            if (k0 >= C::NCODE) rw[DC::EW * f + q] = 0u;
+            else if (k0 + 1 >= C::NCODE) rw[DC::EW * f + q] &= 0xFFFFu;
+          }
+        }
+        if (32 * c + 32 <= KC / 2) tmem_st32(a_t + (uint32_t)(32 * c), rw);
+        else tmem_st8(a_t + (uint32_t)(32 * c), rw);  // RotorQuant: 72 = 2 x 32 + 8 words
+      }
+      if constexpr (kProd) {
+        // sign part: A words [KC/2, KC/2 + 64), a byte of signs per lookup
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t rw[32];
+#pragma unroll
+          for (int bq = 0; bq < 8; ++bq) {
+            const int byte = 8 * c + bq;
+            const uint32_t v = (sg[byte >> 2] >> (8 * (byte & 3))) & 0xFFu;
+            const uint4 x = *reinterpret_cast<const uint4*>(slut_l + v * 128);
+            rw[4 * bq] = x.x;
+            rw[4 * bq + 1] = x.y;
+            rw[4 * bq + 2] = x.z;
+            rw[4 * bq + 3] = x.w;
+          }
+          tmem_st32(a_t + (uint32_t)(KC / 2 + 32 * c), rw);
         }
       }
-#pragma unroll
-      for (int j = 0; j < KC / 8; ++j) {
-        const bool mine = kProd ? true : (wg == 0 ? (8 * j < C::KSPLIT) : (8 * j >= C::KSPLIT));
-        if (mine)
-          *reinterpret_cast<uint4*>(A + sw128_chunk(key, j, C::A_BOX)) =
-              make_uint4(rw[4 * j], rw[4 * j + 1], rw[4 * j + 2], rw[4 * j + 3]);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar_afull[w]);
+    }
+    // the last tile of this warpgroup
+    if (ok && i > 0) {
+      const int jl = w + (i - 1) * kNWG;
+      if (mbar_wait(&bar_acc[w * 2 + ((i - 1) & 1)], (uint32_t)(((i - 1) >> 1) & 1), a.status)) {
+        tc_fence_after();
+        epilogue(jl, i - 1, prev_n, prev_g);
       }
     }
-    if (kProd && wg == 1) {
-      // sign part: each byte of signs -> 8 x (+1/-1) fp16
-#pragma unroll
-      for (int w = 0; w < NS; ++w) {
-        const uint32_t sw = stg[kRows * W + key * NS + w];
-#pragma unroll
-        for (int bt = 0; bt < 4; ++bt) {
-          const uint4 e = *reinterpret_cast<const uint4*>(s_slut + ((sw >> (8 * bt)) & 0xFF) * 16);
-          *reinterpret_cast<uint4*>(A + sw128_chunk(key, KC / 8 + w * 4 + bt, C::A_BOX)) = e;
-        }
-      }
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      // refill this code stage kStages tiles ahead (every thread has read it)
-      if (bulk && it + kStages < ntiles && tile_full(it + kStages)) issue_stage(it + kStages, st);
-      tc_fence_after();
-      const uint32_t a_buf = a_s + (uint32_t)(ab * C::A_BYTES);
-#pragma unroll
-      for (int kk = 0; kk < K / 16; ++kk) {
-        const uint32_t off = (uint32_t)((kk >> 2) * C::A_BOX + (kk & 3) * 32);
-        const uint32_t boff = (uint32_t)((kk >> 2) * C::B_BOX + (kk & 3) * 32);
-        umma_f16(tmem + (uint32_t)(ab * NB), umma_desc_sw128(a_buf + off, 16, 1024),
-                 umma_desc_sw128(b_s + boff, 16, 1024), kIdesc, kk > 0);
-      }
-      umma_commit(&s_bar[MB + ab]);
-    }
-    // finish the previous tile while this one's MMA runs; its MMA is complete
-    // before the next decode overwrites its A buffer
-    if (it > 0) {
-      ok = mbar_wait(&s_bar[MB + (ab ^ 1)], (par >> (MB + (ab ^ 1))) & 1, a.status) && ok;
-      par ^= 1u << (MB + (ab ^ 1));
-      tc_fence_after();
-      if (wg == 1) epilogue(it - 1, prev_n, prev_g);
-    }
-    prev_n = nrm;
-    prev_g = gam;
-    tc_fence_before();
-  }
-  // the last tile
-  if (ok && ntiles > 0) {
-    const int lt = ntiles - 1;
-    ok = mbar_wait(&s_bar[kStages + (lt & 1)], (par >> (kStages + (lt & 1))) & 1, a.status);
-    tc_fence_after();
-    if (ok && wg == 1) epilogue(lt, prev_n, prev_g);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, C::kNcols);
+  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
 }  // namespace score
