@@ -282,7 +282,7 @@ def run_leg_only(args):
         T = torch.from_numpy(kvrq.qjl_matrix_init(D_, D_, 3)).to(torch.float16).to(dev)
         prod = mode in ("prod", "dqp")
         cb = torch.from_numpy(kvrq.tq_codebook_init(D_, b - 1 if prod else b)[0].astype(np.float32)).to(dev)
-        ws = kvrq.tq_workspace(rows, D_, dev) if kvrq.tq_needs_workspace(D_, x.dtype) else None
+        ws = kvrq.tq_workspace(rows, D_, dev, max_bytes=1 << 30) if kvrq.tq_needs_workspace(D_, x.dtype) else None
         if prod:
             codes, signs, gam, norms = kvrq.tq_quantize_prod(x, pi, T, cb, b)
         else:

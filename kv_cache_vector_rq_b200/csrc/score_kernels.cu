@@ -12,17 +12,19 @@
 // the head's query group once (Pi q and T Pi q from staged copies of Pi and T,
 // or the per-group sandwich) into the MMA B operand (N = 16..64 rows, fp16, in
 // shared memory). Keys are then handled in 128-token tiles, the M = 128 rows
-// of the MMA, by two decode warpgroups that alternate tiles:
-//   * packed code rows (and sign rows) arrive by bulk copy into a ring of
-//     stages per warpgroup, issued by one control thread;
+// of the MMA, by two or three decode warpgroups that take tiles in turn:
+//   * packed code rows and sign rows arrive by bulk copy into a ring of
+//     stages per warpgroup; every warpgroup is its own pipeline, its
+//     first thread issuing the copies and the MMAs of the warpgroup's tiles;
 //   * each thread decodes its key into fp16 operand words through small
 //     shared-memory tables (one lookup per 8-bit or 6-bit field of codes, and
 //     per byte of signs), replicated per lane so that the lookups of a warp
 //     never collide on a bank, and writes them with tcgen05.st straight into
 //     its lane of the warpgroup's A region in tensor memory -- the decoded keys
 //     never pass through shared memory;
-//   * the control thread issues tcgen05.mma with A in tensor memory and B in
-//     shared memory into one of the warpgroup's two accumulators;
+//   * after a warpgroup barrier that thread issues tcgen05.mma with A in
+//     tensor memory and B in shared memory into one of the warpgroup's two
+//     accumulators;
 //   * while the next tile is being decoded the warpgroup reads the previous
 //     tile's accumulator row per thread (||k|| and the QJL term) and writes
 //     fp32 scores, coalesced across tokens.
@@ -38,8 +40,6 @@ namespace kvrq {
 namespace score {
 
 constexpr int kRows = 128;                  // tokens per tile (TMEM lanes)
-constexpr int kNWG = 2;                     // decode warpgroups
-constexpr int kThreads = kNWG * 128 + 32;   // + one control warp
 constexpr int kStages = 4;                  // code stages per warpgroup
 constexpr uint32_t kTmemCols = 512;
 
@@ -74,10 +74,13 @@ struct Cfg {
   static constexpr int B_BOX = NB * 128;
   static constexpr int QS = D + 16;                                 // row stride of the query scratch
   static constexpr int MS = 130;                                    // padded row (halves) of a staged matrix
-  // TMEM columns per warpgroup: A, then two accumulators
+  // TMEM columns per warpgroup: A, then two accumulators; as many decode
+  // warpgroups (up to three) as tensor memory holds
   static constexpr int WCOLS = (KAP + 2 * NB + 31) / 32 * 32;
+  static constexpr int kNWG = 3 * WCOLS <= (int)kTmemCols ? 3 : 2;
+  static constexpr int kThreads = kNWG * 128;
   static_assert(kNWG * WCOLS <= (int)kTmemCols, "tensor memory");
-  // shared memory
+  // shared memory; a stage holds a tile's code rows and sign rows
   static constexpr int stage_words = kRows * (W + NS);
   static constexpr int lut_bytes = Dec<BITS>::BYTES;
   static constexpr int slut_bytes = kProd ? 256 * 128 : 0;  // byte of signs -> 8 x (+1/-1), 8 replicas
@@ -91,11 +94,25 @@ struct Cfg {
   static constexpr int pro_end = m_off + D * MS * 2;
   static constexpr int b_off = (((ring_end > pro_end ? ring_end : pro_end) + 1023) / 1024) * 1024;
   static constexpr int bar_off = b_off + KBOX * B_BOX;
-  // barriers: stage full [kNWG][kStages], A written [kNWG], accumulator full [kNWG][2], done
-  static constexpr int nbars = kNWG * kStages + kNWG + 2 * kNWG + 1;
+  // barriers: stage full [kNWG][kStages], accumulator full [kNWG][2]
+  static constexpr int nbars = kNWG * kStages + 2 * kNWG;
   static constexpr int tmem_off = bar_off + nbars * 8;
   static constexpr int alloc = tmem_off + 16 + 1024;
 };
+
+// Barrier `id` among the 128 threads of a warpgroup; returns the AND of `pred` over them.
+__device__ __forceinline__ bool wg_all(bool pred, int id) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred ? 1u : 0u), "r"(id)
+      : "memory");
+  return r != 0;
+}
 
 // field of `FB` bits starting at bit `bit` of the little-endian stream in w[0..NW)
 template <int FB, int NW>
@@ -107,10 +124,11 @@ __device__ __forceinline__ uint32_t field(const uint32_t (&w)[NW], int bit) {
 }
 
 template <int METHOD, int BITS, int NB>
-__global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs a) {
+__global__ void __launch_bounds__(Cfg<METHOD, BITS, NB>::kThreads, 1) score_kernel(ScoreArgs a) {
   using C = Cfg<METHOD, BITS, NB>;
   using DC = Dec<BITS>;
   constexpr int D = C::D, K = C::K, KC = C::KC, W = C::W, NS = C::NS;
+  constexpr int kNWG = C::kNWG, kThreads = C::kThreads;
   constexpr bool kProd = C::kProd;
   constexpr uint32_t kIdesc = umma_idesc_f16(false, false, false, NB, kRows);
 
@@ -122,10 +140,8 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs a) {
   const uint8_t* s_slut = smem + C::slut_off;
   float* s_q = reinterpret_cast<float*>(smem);
   uint64_t* s_bar = reinterpret_cast<uint64_t*>(smem + C::bar_off);
-  uint64_t* bar_stage = s_bar;                   // [w * kStages + s]
-  uint64_t* bar_afull = s_bar + kNWG * kStages;  // [w]
-  uint64_t* bar_acc = bar_afull + kNWG;          // [w * 2 + b]
-  uint64_t* bar_done = bar_acc + 2 * kNWG;
+  uint64_t* bar_stage = s_bar;                 // [w * kStages + s]
+  uint64_t* bar_acc = s_bar + kNWG * kStages;  // [w * 2 + b]
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::tmem_off);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -144,10 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs a) {
   auto tile_full = [&](int j) { return t_begin + (int64_t)(j + 1) * kRows <= t_end; };
 
   if (tid == 0) {
-    for (int s = 0; s < C::nbars; ++s) {
-      const bool afull = s >= kNWG * kStages && s < kNWG * kStages + kNWG;  // every decoder arrives
-      mbar_init(&s_bar[s], afull ? 128 : 1);
-    }
+    for (int s = 0; s < C::nbars; ++s) mbar_init(&s_bar[s], 1);
     fence_barrier_init();
   }
   if (warp == 0) tmem_alloc(s_tmem, kTmemCols);
@@ -271,45 +284,27 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs a) {
   const uint32_t tmem = *s_tmem;
   const uint32_t b_s = smem_u32(s_b);
 
-  if (warp == kNWG * 4) {
-    // ------------------------------------------------------------ control thread: copies and MMAs
-    if (lane == 0) {
-      auto issue_stage = [&](int j) {
-        const int w = j % kNWG, i = j / kNWG, s = i % kStages;
-        const int64_t t0 = t_begin + (int64_t)j * kRows;
-        uint32_t* dst = s_stage + (w * kStages + s) * C::stage_words;
-        uint64_t* bar = &bar_stage[w * kStages + s];
-        mbar_arrive_expect_tx(bar, kRows * (W + NS) * 4);
-        bulk_load(dst, codes_h + t0 * W, kRows * W * 4, bar);
-        if (kProd) bulk_load(dst + kRows * W, signs_h + t0 * NS, kRows * NS * 4, bar);
-      };
-      if (bulk)
-        for (int j = 0; j < kStages * kNWG && j < ntiles; ++j)
-          if (tile_full(j)) issue_stage(j);
-      bool ok = true;
-      for (int j = 0; j < ntiles && ok; ++j) {
-        const int w = j % kNWG, i = j / kNWG;
-        if (!(ok = mbar_wait(&bar_afull[w], (uint32_t)(i & 1), a.status))) break;
-        tc_fence_after();
-        const uint32_t a_t = tmem + (uint32_t)(w * C::WCOLS);
-        const uint32_t d_t = a_t + (uint32_t)(C::KAP + (i & 1) * NB);
-#pragma unroll
-        for (int kk = 0; kk < K / 16; ++kk) {
-          const uint32_t boff = (uint32_t)((kk >> 2) * C::B_BOX + (kk & 3) * 32);
-          umma_f16_ts(d_t, a_t + (uint32_t)(8 * kk), umma_desc_sw128(b_s + boff, 16, 1024), kIdesc, kk > 0);
-        }
-        umma_commit(&bar_acc[w * 2 + (i & 1)]);
-        // the tile's code stage has been read by the decoders: refill it
-        const int jn = j + kStages * kNWG;
-        if (bulk && jn < ntiles && tile_full(jn)) issue_stage(jn);
-      }
-      umma_commit(bar_done);  // every MMA issued has completed before TMEM is released
-      mbar_wait(bar_done, 0, a.status);
-    }
-  } else {
+  {
     // ------------------------------------------------------------ decode warpgroups
     const int w = warp >> 2;  // warpgroup
     const int r = tid & 127;  // key row of the tile = TMEM lane
+    // The warpgroup is its own pipeline: its thread 0 issues the bulk copies of
+    // the warpgroup's tiles and, once all 128 rows are in tensor memory, the MMAs.
+    auto issue_stage = [&](int j) {  // thread 0 of the warpgroup
+      const int i = j / kNWG, s = i % kStages;
+      const int64_t t0 = t_begin + (int64_t)j * kRows;
+      uint32_t* dst = s_stage + (w * kStages + s) * C::stage_words;
+      uint64_t* bar = &bar_stage[w * kStages + s];
+      mbar_arrive_expect_tx(bar, C::stage_words * 4);
+      bulk_load(dst, codes_h + t0 * W, kRows * W * 4, bar);
+      if (kProd) bulk_load(dst + kRows * W, signs_h + t0 * NS, kRows * NS * 4, bar);
+    };
+    if (r == 0 && bulk)
+      for (int i = 0; i < kStages; ++i) {
+        const int j = w + i * kNWG;
+        if (j < ntiles && tile_full(j)) issue_stage(j);
+      }
+    const uint32_t a_mma = tmem + (uint32_t)(w * C::WCOLS);  // lane 0 of the warpgroup's A region
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t a_t = tmem + lane_off + (uint32_t)(w * C::WCOLS);
     const uint32_t acc_t = a_t + (uint32_t)C::KAP;
@@ -338,17 +333,83 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs a) {
       }
     };
 
+    constexpr int NCC = (KC / 2 + 31) / 32;  // 32-word chunks of the centroid part
+    auto centroid_chunk = [&](int c, const uint32_t (&wc)[W]) {
+      uint32_t rw[32];
+      constexpr int FPC = 64 / DC::P;  // fields per 32 words
+#pragma unroll
+      for (int f = 0; f < FPC; ++f) {
+        const int fi = c * FPC + f;  // field index: codes fi*P .. fi*P + P - 1
+        if (fi * DC::P < C::NCODE) {
+          const uint32_t v = field<DC::FB, W>(wc, fi * DC::FB);
+          const uint8_t* e = lut_l + v * 128;
+          if constexpr (DC::EW == 4) {
+            const uint4 x = *reinterpret_cast<const uint4*>(e);
+            rw[4 * f] = x.x;
+            rw[4 * f + 1] = x.y;
+            rw[4 * f + 2] = x.z;
+            rw[4 * f + 3] = x.w;
+          } else if constexpr (DC::EW == 2) {
+            const uint2 x = *reinterpret_cast<const uint2*>(e);
+            rw[2 * f] = x.x;
+            rw[2 * f + 1] = x.y;
+          } else {
+            rw[f] = *reinterpret_cast<const uint32_t*>(e);
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < DC::EW; ++q) rw[DC::EW * f + q] = 0u;
+        }
+        // K elements past the stored codes (the RotorQuant tail) are zero
+#pragma unroll
+        for (int q = 0; q < DC::EW; ++q) {
+          const int k0 = 2 * (32 * c + DC::EW * f + q);  // first K element of this word
+          if (k0 >= C::NCODE) rw[DC::EW * f + q] = 0u;
+          else if (k0 + 1 >= C::NCODE) rw[DC::EW * f + q] &= 0xFFFFu;
+        }
+      }
+      if (32 * c + 32 <= KC / 2) tmem_st32(a_t + (uint32_t)(32 * c), rw);
+      else tmem_st8(a_t + (uint32_t)(32 * c), rw);  // RotorQuant: 72 = 2 x 32 + 8 words
+    };
+    auto sign_chunk = [&](int c, const uint32_t (&sg)[NS > 0 ? NS : 1]) {
+      uint32_t rw[32];
+#pragma unroll
+      for (int bq = 0; bq < 8; ++bq) {
+        const int byte = 8 * c + bq;
+        const uint32_t v = (sg[byte >> 2] >> (8 * (byte & 3))) & 0xFFu;
+        const uint4 x = *reinterpret_cast<const uint4*>(slut_l + v * 128);
+        rw[4 * bq] = x.x;
+        rw[4 * bq + 1] = x.y;
+        rw[4 * bq + 2] = x.z;
+        rw[4 * bq + 3] = x.w;
+      }
+      tmem_st32(a_t + (uint32_t)(KC / 2 + 32 * c), rw);
+    };
+    auto mma_steps = [&](int i, int k_lo, int k_hi) {  // thread 0 of the warpgroup
+      const uint32_t d_t = a_mma + (uint32_t)(C::KAP + (i & 1) * NB);
+      for (int kk = k_lo; kk < k_hi; ++kk) {
+        const uint32_t boff = (uint32_t)((kk >> 2) * C::B_BOX + (kk & 3) * 32);
+        umma_f16_ts(d_t, a_mma + (uint32_t)(8 * kk), umma_desc_sw128(b_s + boff, 16, 1024), kIdesc, kk > 0);
+      }
+    };
+
     int i = 0;
     for (int j = w; j < ntiles; j += kNWG, ++i) {
       const int s = i % kStages;
       const int64_t t0 = t_begin + (int64_t)j * kRows;
       const int rows = (int)(t_end - t0 < (int64_t)kRows ? t_end - t0 : (int64_t)kRows);
+      // this key's norm and gamma (used by the epilogue one iteration later), packed codes and signs
       const float nrm = r < rows ? __ldg(norms_h + t0 + r) : 0.f;
       const float gam = (kProd && r < rows) ? __ldg(gammas_h + t0 + r) : 0.f;
-      // this key's packed codes and signs
       uint32_t wc[W], sg[NS > 0 ? NS : 1];
+      // both waits of the tile first; the warpgroup leaves together if either ran out
+      if (bulk && tile_full(j)) ok = mbar_wait(&bar_stage[w * kStages + s], (uint32_t)((i / kStages) & 1), a.status);
+      if (i > 0) ok = mbar_wait(&bar_acc[w * 2 + ((i - 1) & 1)], (uint32_t)(((i - 1) >> 1) & 1), a.status) && ok;
+      if (!wg_all(ok, 1 + w)) {
+        ok = false;
+        break;
+      }
       if (bulk && tile_full(j)) {
-        if (!(ok = mbar_wait(&bar_stage[w * kStages + s], (uint32_t)((i / kStages) & 1), a.status))) break;
         const uint32_t* stg = s_stage + (w * kStages + s) * C::stage_words;
         if constexpr (W % 4 == 0) {
 #pragma unroll
@@ -380,80 +441,43 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs a) {
       }
       // the previous tile's MMA has finished with A: its scores, then this tile's decode
       if (i > 0) {
-        if (!(ok = mbar_wait(&bar_acc[w * 2 + ((i - 1) & 1)], (uint32_t)(((i - 1) >> 1) & 1), a.status))) break;
         tc_fence_after();
         epilogue(j - kNWG, i - 1, prev_n, prev_g);
       }
-      prev_n = nrm;
-      prev_g = gam;
-
-      // centroid part: A words [0, KC/2), 32 at a time
-      constexpr int FPC = 64 / DC::P;  // fields per 32 words
 #pragma unroll
-      for (int c = 0; c < (KC / 2 + 31) / 32; ++c) {
-        uint32_t rw[32];
-#pragma unroll
-        for (int f = 0; f < FPC; ++f) {
-          const int fi = c * FPC + f;  // field index: codes fi*P .. fi*P + P - 1
-          if (fi * DC::P < C::NCODE) {
-            const uint32_t v = field<DC::FB, W>(wc, fi * DC::FB);
-            const uint8_t* e = lut_l + v * 128;
-            if constexpr (DC::EW == 4) {
-              const uint4 x = *reinterpret_cast<const uint4*>(e);
-              rw[4 * f] = x.x;
-              rw[4 * f + 1] = x.y;
-              rw[4 * f + 2] = x.z;
-              rw[4 * f + 3] = x.w;
-            } else if constexpr (DC::EW == 2) {
-              const uint2 x = *reinterpret_cast<const uint2*>(e);
-              rw[2 * f] = x.x;
-              rw[2 * f + 1] = x.y;
-            } else {
-              rw[f] = *reinterpret_cast<const uint32_t*>(e);
-            }
-          } else {
-#pragma unroll
-            for (int q = 0; q < DC::EW; ++q) rw[DC::EW * f + q] = 0u;
-          }
-          // K elements past the stored codes (the RotorQuant tail) are zero
-#pragma unroll
-          for (int q = 0; q < DC::EW; ++q) {
-            const int k0 = 2 * (32 * c + DC::EW * f + q);  // first K element of this word
-            if (k0 >= C::NCODE) rw[DC::EW * f + q] = 0u;
-            else if (k0 + 1 >= C::NCODE) rw[DC::EW * f + q] &= 0xFFFFu;
-          }
-        }
-        if (32 * c + 32 <= KC / 2) tmem_st32(a_t + (uint32_t)(32 * c), rw);
-        else tmem_st8(a_t + (uint32_t)(32 * c), rw);  // RotorQuant: 72 = 2 x 32 + 8 words
-      }
+      for (int c = 0; c < NCC; ++c) centroid_chunk(c, wc);
       if constexpr (kProd) {
-        // sign part: A words [KC/2, KC/2 + 64), a byte of signs per lookup
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t rw[32];
-#pragma unroll
-          for (int bq = 0; bq < 8; ++bq) {
-            const int byte = 8 * c + bq;
-            const uint32_t v = (sg[byte >> 2] >> (8 * (byte & 3))) & 0xFFu;
-            const uint4 x = *reinterpret_cast<const uint4*>(slut_l + v * 128);
-            rw[4 * bq] = x.x;
-            rw[4 * bq + 1] = x.y;
-            rw[4 * bq + 2] = x.z;
-            rw[4 * bq + 3] = x.w;
-          }
-          tmem_st32(a_t + (uint32_t)(KC / 2 + 32 * c), rw);
-        }
+        sign_chunk(0, sg);
+        sign_chunk(1, sg);
       }
+      prev_n = nrm;  // the loads have long landed by now
+      prev_g = gam;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bar_afull[w]);
+      // all rows of the tile are in tensor memory, and every thread has read its stage
+      asm volatile("bar.sync %0, 128;" ::"r"(1 + w) : "memory");
+      if (r == 0) {
+        tc_fence_after();
+        mma_steps(i, 0, K / 16);
+        umma_commit(&bar_acc[w * 2 + (i & 1)]);
+        const int jn = j + kStages * kNWG;
+        if (bulk && jn < ntiles && tile_full(jn)) issue_stage(jn);
+      }
     }
-    // the last tile of this warpgroup
+    // the last tile of this warpgroup (also waits for its last MMA before TMEM is released)
     if (ok && i > 0) {
       const int jl = w + (i - 1) * kNWG;
       if (mbar_wait(&bar_acc[w * 2 + ((i - 1) & 1)], (uint32_t)(((i - 1) >> 1) & 1), a.status)) {
         tc_fence_after();
         epilogue(jl, i - 1, prev_n, prev_g);
+      }
+    } else if (!ok && r == 0) {
+      // a wait ran out: the MMAs and copies still in flight finish before the CTA exits
+      if (i > 0) mbar_wait(&bar_acc[w * 2 + ((i - 1) & 1)], (uint32_t)(((i - 1) >> 1) & 1), a.status);
+      for (int s2 = 0; s2 < kStages; ++s2) {
+        const int iu = i + s2;  // stages possibly still filling
+        if (bulk && w + iu * kNWG < ntiles && tile_full(w + iu * kNWG))
+          mbar_wait(&bar_stage[w * kStages + (iu % kStages)], (uint32_t)((iu / kStages) & 1), a.status);
       }
     }
   }
@@ -475,7 +499,7 @@ static cudaError_t launch_score_t(const ScoreArgs& a, cudaStream_t st) {
     attr = true;
   }
   dim3 grid((unsigned)((a.n_tokens + a.tokens_per_cta - 1) / a.tokens_per_cta), (unsigned)a.n_heads);
-  kern<<<grid, score::kThreads, C::alloc, st>>>(a);
+  kern<<<grid, C::kThreads, C::alloc, st>>>(a);
   return cudaGetLastError();
 }
 
