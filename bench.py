@@ -58,6 +58,27 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def recorded_traffic(kernel):
+    """Per-launch DRAM bytes of `kernel` from profiles/traffic.txt, or None when that record is missing or the
+    kernel's source changed since the counters were taken (the record keeps a SHA-256 prefix of the source)."""
+    import hashlib
+
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    for line in open(p):
+        if line.startswith("#") or "|" not in line:
+            continue
+        f = [x.strip() for x in line.split("|")]
+        if f[0] != kernel:
+            continue
+        src = os.path.join(ROOT, f[1])
+        if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != f[2]:
+            return None
+        return int(f[4]) + int(f[5])
+    return None
+
+
 def measured_tensor_peak():
     """Dense fp16/bf16 tensor-core peak in TFLOP/s: the measured cuBLAS bf16 burst figure (fp16 runs at the same
     nominal rate), else the fallback."""
@@ -589,7 +610,8 @@ def main():
                        "n_vectors_per_gpu": N_VEC, "d": D, "io_dtype": "fp16", "l2": "flushed (256 MiB write) "
                        "before every timed launch", "parallelism": "independent shard per GPU (weak scaling)"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+                         "frac": achieved / peak, "traffic": recorded_traffic("rq_row_kernel<__half,3,RQ_QDQ>"),
+                         "traffic_unit": "bytes per launch", "peak_kind": peak_kind,
                          "kernel": "rq_row_kernel<__half, 3, RQ_QDQ>", "bytes_per_vector": bpv},
             "legs": legs_out,
             "hbm_1gib": large,
