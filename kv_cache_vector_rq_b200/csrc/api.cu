@@ -216,6 +216,12 @@ static kvrq_status rq_call(const char* name, int mode, void* stream, const void*
     if (!dq_side) mo = mx;
     return launch_status(name, launch_rq_row(mode, tdt, bits, mx, mo, a, s, di->num_sms));
   }
+  // any d: rows streamed by bulk copy when they start 16-byte aligned and fit its row buffers
+  bool wide = true;
+  if (q_side) wide = wide && rows_aligned16(x, ldx, xdt);
+  if (dq_side) wide = wide && rows_aligned16(xhat, ldo, odt);
+  if (mode == RQ_QDQ) wide = wide && xdt == odt;
+  a.wide = wide && rq_wide_smem_bytes(d, bits, (int)dtype_size(tdt)) > 0;
   return launch_status(name, launch_rq_general(mode, xdt, odt, bits, a, s, di->num_sms));
 }
 

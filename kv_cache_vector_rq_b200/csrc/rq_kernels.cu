@@ -642,6 +642,229 @@ __global__ void __launch_bounds__(256) rq_general_kernel(RqArgs a) {
 }
 
 // ============================================================================
+// Any d with 16-byte aligned rows (d x element size a multiple of 16): rows
+// streamed by bulk copy, processed by a team of TEAM warps per row.
+//
+// The CTA (8 warps) builds the groups' exact 3x3 sandwich matrices once. A team
+// -- one warp for narrow rows, the whole CTA for wide ones (d >= 768) -- owns
+// two shared row buffers and bulk-copies blocks of rows into them, so the next
+// block is on its way while the current one is processed. Per row the norm is
+// a reduction over 16-byte chunks, thread t of the team takes groups t, t +
+// team size, ...; a group's codes are OR-ed into the team's word buffer and
+// stored coalesced; x_hat overwrites the row in the buffer and the block leaves
+// by bulk copy. The quantizer and the reconstruction are those of
+// rq_general_kernel, so quantize-then-dequantize and the fused launch agree bit
+// for bit.
+// ============================================================================
+namespace wide {
+
+constexpr int kWarps = 8;
+constexpr int kThreads = 32 * kWarps;
+
+// team of TEAM warps; dynamic shared memory:
+// [G][9] matrices | per team: 2 row buffers of BUF bytes | RB x W code words | 2 barriers | 8 partial sums
+struct Layout {
+  int G, W, RB, BUF, teams;
+  int m_off, buf_off, codes_off, bar_off, part_off, bytes;
+  __host__ __device__ Layout(int d, int bits, int row_bytes, int team) {
+    G = (d + 2) / 3;
+    W = (3 * G * bits + 31) / 32;
+    teams = kWarps / team;
+    BUF = team == 1 ? (row_bytes > 2048 ? row_bytes : 2048) : row_bytes;
+    RB = BUF / row_bytes;
+    m_off = 0;
+    buf_off = ((G * 9 * 4 + 127) / 128) * 128;
+    codes_off = buf_off + teams * 2 * BUF;
+    bar_off = codes_off + ((teams * RB * W * 4 + 15) / 16) * 16;
+    part_off = bar_off + teams * 2 * 8;
+    bytes = part_off + kWarps * 4;
+  }
+};
+
+// team size for d: the whole CTA once a row has 256 groups or more
+__host__ __device__ inline int team_of(int d) { return (d + 2) / 3 >= 256 ? kWarps : 1; }
+
+template <int TEAM>
+__device__ __forceinline__ void team_sync() {
+  if (TEAM == 1) __syncwarp();
+  else __syncthreads();
+}
+
+template <typename TI, typename TO, int BITS, int MODE, int TEAM>
+__global__ void __launch_bounds__(kThreads) rq_wide_kernel(RqArgs a) {
+  constexpr int K = 1 << BITS;
+  constexpr int TT = 32 * TEAM;  // threads per team
+  constexpr bool kIn = MODE != RQ_DQ, kOut = MODE != RQ_Q;
+  using TB = typename std::conditional<kIn, TI, TO>::type;  // element type held in the row buffers
+  __shared__ float s_tau[16], s_mag[16], s_c[16];
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int d = a.d;
+  const Layout L(d, BITS, d * (int)sizeof(TB), TEAM);
+  const int G = L.G, W = L.W, RB = L.RB;
+  float* s_m = reinterpret_cast<float*>(smem + L.m_off);
+  const int warp = threadIdx.x >> 5;
+  const int team = warp / TEAM, t = threadIdx.x % TT;
+  uint8_t* t_buf = smem + L.buf_off + team * 2 * L.BUF;
+  uint32_t* t_codes = reinterpret_cast<uint32_t*>(smem + L.codes_off) + team * RB * W;
+  uint64_t* t_bar = reinterpret_cast<uint64_t*>(smem + L.bar_off) + team * 2;
+  float* s_part = reinterpret_cast<float*>(smem + L.part_off);
+
+  build_codebook<BITS>(a.centroids, s_tau, s_mag, s_c);
+  for (int g = threadIdx.x; g < G; g += kThreads) {
+    const float4 r = __ldg(reinterpret_cast<const float4*>(a.rotors) + g);
+    rotor_matrix(r.x, r.y, r.z, r.w, s_m + g * 9);
+  }
+  for (int i = t; i < RB * W; i += TT) t_codes[i] = 0u;
+  if (t == 0) {
+    mbar_init(&t_bar[0], 1);
+    mbar_init(&t_bar[1], 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  const int64_t n = a.n;
+  const int64_t nblk = (n + RB - 1) / RB;
+  const int64_t gt = (int64_t)blockIdx.x * L.teams + team, tt = (int64_t)gridDim.x * L.teams;
+  const size_t row_bytes = (size_t)d * sizeof(TB);
+  const TI* xin = reinterpret_cast<const TI*>(a.x);
+  TO* xo = reinterpret_cast<TO*>(a.xhat);
+  auto rows_of = [&](int64_t blk) -> int { return (int)(n - blk * RB < RB ? n - blk * RB : RB); };
+  auto issue = [&](int64_t blk, int s) {  // thread 0 of the team
+    const int rows = rows_of(blk);
+    mbar_arrive_expect_tx(&t_bar[s], (uint32_t)(rows * row_bytes));
+    if (a.ldx == d) {  // contiguous rows: one copy for the block
+      bulk_load(t_buf + s * L.BUF, xin + blk * RB * a.ldx, (uint32_t)(rows * row_bytes), &t_bar[s]);
+    } else {
+      for (int r = 0; r < rows; ++r)
+        bulk_load(t_buf + s * L.BUF + r * row_bytes, xin + (blk * RB + r) * a.ldx, (uint32_t)row_bytes, &t_bar[s]);
+    }
+  };
+  if (kIn && t == 0)
+    for (int s = 0; s < 2; ++s)
+      if (gt + s * tt < nblk) issue(gt + s * tt, s);
+
+  uint32_t par = 0;
+  int it = 0;
+  bool failed = false;
+  for (int64_t blk = gt; blk < nblk; blk += tt, ++it) {
+    const int s = it & 1;
+    const int rows = rows_of(blk);
+    TB* buf = reinterpret_cast<TB*>(t_buf + s * L.BUF);
+    bool ok = true;
+    if (kIn) {
+      ok = mbar_wait(&t_bar[s], (par >> s) & 1, a.status);
+      par ^= 1u << s;
+    } else if (t == 0) {
+      bulk_wait_read<1>();  // the x_hat store that last used this buffer has read it
+    }
+    // the team leaves together if a wait ran out
+    if (TEAM == 1 ? !__all_sync(0xffffffffu, ok) : !__syncthreads_and(ok)) {
+      failed = true;
+      break;
+    }
+    for (int r = 0; r < rows; ++r) {
+      const int64_t row = blk * RB + r;
+      TB* rb = buf + (size_t)r * d;
+      float nrm;
+      if constexpr (kIn) {
+        float ss = 0.f;
+        constexpr int E = 16 / (int)sizeof(TB);
+        for (int c = t; c < d / E; c += TT) {
+          float f[E];
+          Elem<TB>::unpack(reinterpret_cast<const uint4*>(rb)[c], f);
+#pragma unroll
+          for (int e = 0; e < E; ++e) ss = fmaf(f[e], f[e], ss);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        if (TEAM > 1) {
+          if ((threadIdx.x & 31) == 0) s_part[warp] = ss;
+          __syncthreads();
+          ss = 0.f;
+#pragma unroll
+          for (int w = 0; w < TEAM; ++w) ss += s_part[w];
+        }
+        nrm = sqrtf(ss);
+        if (t == 0 && a.norms_out) a.norms_out[row * a.ldn] = nrm;
+      } else {
+        nrm = __ldg(a.norms_in + row * a.ldn);
+      }
+      Quantizer<BITS> q;
+      q.scale(s_tau, s_mag, nrm);
+      uint32_t* wc = t_codes + r * W;
+      const uint32_t* cin = kIn ? nullptr : a.codes_in + row * a.ldc;
+      for (int g = t; g < G; g += TT) {
+        const float* m = s_m + g * 9;
+        float c[3];
+        if constexpr (kIn) {
+          float v[3];
+#pragma unroll
+          for (int i = 0; i < 3; ++i) v[i] = (3 * g + i < d) ? Elem<TB>::to_float(rb[3 * g + i]) : 0.f;
+          uint32_t bits3 = 0;
+#pragma unroll
+          for (int i = 0; i < 3; ++i) {
+            const float y = fmaf(m[3 * i + 2], v[2], fmaf(m[3 * i + 1], v[1], m[3 * i] * v[0]));
+            bits3 |= q(y, c[i]) << (i * BITS);
+          }
+          const int bit = g * 3 * BITS;
+          atomicOr(&wc[bit >> 5], bits3 << (bit & 31));
+          if ((bit & 31) + 3 * BITS > 32) atomicOr(&wc[(bit >> 5) + 1], bits3 >> (32 - (bit & 31)));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 3; ++i) {
+            const int bit = (3 * g + i) * BITS;
+            uint32_t v = __ldg(cin + (bit >> 5)) >> (bit & 31);
+            if ((bit & 31) + BITS > 32) v |= __ldg(cin + (bit >> 5) + 1) << (32 - (bit & 31));
+            c[i] = s_c[v & (K - 1)] * nrm;
+          }
+        }
+        if constexpr (kOut) {
+#pragma unroll
+          for (int i = 0; i < 3; ++i)
+            if (3 * g + i < d)
+              rb[3 * g + i] = Elem<TB>::from_float(fmaf(m[6 + i], c[2], fmaf(m[3 + i], c[1], m[i] * c[0])));
+        }
+      }
+      if constexpr (kIn) {
+        team_sync<TEAM>();
+        if (a.codes_out)
+          for (int i = t; i < W; i += TT) a.codes_out[row * a.ldc + i] = wc[i];
+        team_sync<TEAM>();
+        for (int i = t; i < W; i += TT) wc[i] = 0u;
+      }
+    }
+    if constexpr (kOut) fence_proxy_async_smem();
+    team_sync<TEAM>();
+    if (t == 0) {
+      if constexpr (kOut) {
+        if (a.ldo == d) {
+          bulk_store(xo + blk * RB * a.ldo, t_buf + s * L.BUF, (uint32_t)(rows * row_bytes));
+        } else {
+          for (int r = 0; r < rows; ++r)
+            bulk_store(xo + (blk * RB + r) * a.ldo, t_buf + s * L.BUF + r * row_bytes, (uint32_t)row_bytes);
+        }
+        bulk_commit();
+      }
+      if constexpr (kIn) {
+        const int64_t next = blk + 2 * tt;
+        if (next < nblk) {
+          if (kOut) bulk_wait_read<0>();  // the x_hat store has read the buffer
+          issue(next, s);
+        }
+      }
+    }
+    team_sync<TEAM>();
+  }
+  if (t == 0) {
+    // after a failed wait, the copy into the other buffer (if any) lands before the team exits
+    if (failed && gt + (int64_t)(it + 1) * tt < nblk) mbar_wait(&t_bar[(it + 1) & 1], (par >> ((it + 1) & 1)) & 1, a.status);
+    bulk_wait_read<0>();
+  }
+}
+
+}  // namespace wide
+
+// ============================================================================
 // Launch helpers (host)
 // ============================================================================
 template <typename T, int BITS, int MODE, int STAGES>
@@ -684,6 +907,40 @@ static cudaError_t launch_row(const CUtensorMap& mx, const CUtensorMap& mo, cons
   return launch_row_s<T, BITS, MODE, 2>(mx, mo, a, st, num_sms);
 }
 
+template <typename TI, typename TO, int BITS, int MODE, int TEAM>
+static cudaError_t launch_wide_t(const RqArgs& a, cudaStream_t st, int num_sms) {
+  using TB = typename std::conditional<MODE != RQ_DQ, TI, TO>::type;
+  const wide::Layout L(a.d, BITS, a.d * (int)sizeof(TB), TEAM);
+  auto kern = wide::rq_wide_kernel<TI, TO, BITS, MODE, TEAM>;
+  static int set_bytes = 0;
+  if (L.bytes > set_bytes) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.bytes);
+    if (e != cudaSuccess) return e;
+    set_bytes = L.bytes;
+  }
+  int per_sm = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, wide::kThreads, L.bytes);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) per_sm = 1;
+  const int64_t nblk = (a.n + L.RB - 1) / L.RB;
+  const int64_t grid = std::min<int64_t>((nblk + L.teams - 1) / L.teams, (int64_t)num_sms * per_sm);
+  kern<<<(unsigned)grid, wide::kThreads, L.bytes, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename TI, typename TO, int BITS, int MODE>
+static cudaError_t launch_wide(const RqArgs& a, cudaStream_t st, int num_sms) {
+  if (wide::team_of(a.d) == 1) return launch_wide_t<TI, TO, BITS, MODE, 1>(a, st, num_sms);
+  return launch_wide_t<TI, TO, BITS, MODE, wide::kWarps>(a, st, num_sms);
+}
+
+// Shared memory the bulk-copy kernel needs for d (0 when it cannot take d).
+int rq_wide_smem_bytes(int d, int bits, int elem_bytes) {
+  if ((d * elem_bytes) % 16 != 0 || d * elem_bytes > 16384) return 0;
+  const wide::Layout L(d, bits, d * elem_bytes, wide::team_of(d));
+  return L.bytes <= 227 * 1024 ? L.bytes : 0;
+}
+
 template <typename TI, typename TO, int BITS, int MODE>
 static cudaError_t launch_general(const RqArgs& a, cudaStream_t st, int num_sms) {
   const int64_t warps = a.n;
@@ -724,6 +981,14 @@ cudaError_t launch_rq_row(int mode, kvrq_dtype dt, int bits, const CUtensorMap& 
 
 template <typename TI, typename TO, int MODE>
 static cudaError_t gen_by_bits(int bits, const RqArgs& a, cudaStream_t st, int sms) {
+  if (a.wide) {
+    switch (bits) {
+      case 1: return launch_wide<TI, TO, 1, MODE>(a, st, sms);
+      case 2: return launch_wide<TI, TO, 2, MODE>(a, st, sms);
+      case 3: return launch_wide<TI, TO, 3, MODE>(a, st, sms);
+      default: return launch_wide<TI, TO, 4, MODE>(a, st, sms);
+    }
+  }
   switch (bits) {
     case 1: return launch_general<TI, TO, 1, MODE>(a, st, sms);
     case 2: return launch_general<TI, TO, 2, MODE>(a, st, sms);

@@ -30,6 +30,7 @@ struct RqArgs {
   int64_t ldc;  // row stride of codes (words), both directions
   int64_t ldn;  // row stride of norms (floats), both directions
   unsigned* status;  // device status word (bounded-wait time-outs)
+  bool wide;         // any-d path: rows are streamed by bulk copy (rq_wide_smem_bytes > 0)
 };
 
 // d = 128 thread-per-row kernel fed by TMA tensor maps over x and x_hat
@@ -40,7 +41,12 @@ cudaError_t launch_rq_row(int mode, kvrq_dtype dt, int bits, const CUtensorMap& 
 // Rows per box of the tensor maps launch_rq_row expects.
 int rq_row_box_rows();
 
-// Any d / stride, warp-per-row kernel.
+// Dynamic shared memory of the bulk-copy any-d kernel for d, or 0 when rows of
+// d elements of elem_bytes cannot take it (row not a multiple of 16 bytes, a
+// row over 16 KB, or tables and buffers over 227 KB).
+int rq_wide_smem_bytes(int d, int bits, int elem_bytes);
+
+// Any d / stride, warp-per-row kernel (a.wide selects the bulk-copy variant).
 cudaError_t launch_rq_general(int mode, kvrq_dtype dt_in, kvrq_dtype dt_out, int bits, const RqArgs& a,
                               cudaStream_t st, int num_sms);
 

@@ -96,6 +96,20 @@ def test_general_dimensions(d, bits):
     _check_roundtrip(x, bits)
 
 
+@pytest.mark.parametrize("d,dt,n", [(4096, torch.float16, 300), (4096, torch.bfloat16, 130), (1536, torch.bfloat16, 333),
+                                    (8, torch.float16, 5000), (24, torch.float32, 1000), (2048, torch.float32, 77)])
+def test_general_dimensions_bulk_rows(d, dt, n):
+    # rows that start 16-byte aligned go through the bulk-copy kernel (several row blocks per warp)
+    x = synth.lognormal(n, d, seed=d + n, dtype=dt).cuda()
+    _check_roundtrip(x, 3)
+
+
+def test_general_bulk_rows_strided():
+    # 16-byte aligned but not contiguous rows: per-row copies
+    base = synth.lognormal(400, 264, seed=3, dtype=torch.float16).cuda()
+    _check_roundtrip(base[:, :256], 2)
+
+
 def test_general_dimension_4096_fp32():
     x = synth.gaussian(200, 4096, seed=9, dtype=torch.float32).cuda()
     _check_roundtrip(x, 3)
