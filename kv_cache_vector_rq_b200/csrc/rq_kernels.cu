@@ -833,7 +833,8 @@ __global__ void __launch_bounds__(kThreads) rq_wide_kernel(RqArgs a) {
         for (int i = t; i < W; i += TT) wc[i] = 0u;
       }
     }
-    if constexpr (kOut) fence_proxy_async_smem();
+    // generic reads (and x_hat writes) of the buffer before the bulk copies that reuse it
+    fence_proxy_async_smem();
     team_sync<TEAM>();
     if (t == 0) {
       if constexpr (kOut) {

@@ -454,6 +454,7 @@ __global__ void __launch_bounds__(Cfg<METHOD, BITS, NB>::kThreads, 1) score_kern
       prev_g = gam;
       tmem_wait_st();
       tc_fence_before();
+      fence_proxy_async_smem();  // this thread's stage reads come before the bulk copy that refills it
       // all rows of the tile are in tensor memory, and every thread has read its stage
       asm volatile("bar.sync %0, 128;" ::"r"(1 + w) : "memory");
       if (r == 0) {

@@ -287,6 +287,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               acc[k] = __ffma2_rn(v, v, acc[k]);
             }
           }
+          // The stage is refilled by TMA (async proxy) once this arrival completes the phase: without the
+          // proxy fence, loads still in flight here can return bytes of the next chunk.
+          fence_proxy_async_smem();
           mbar_arrive(&empty[s]);
         }
         if (!ok) break;

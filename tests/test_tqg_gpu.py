@@ -187,3 +187,43 @@ def test_qjl_sketch(d, m, dt, n):
     cos = ref["p"] / (np.linalg.norm(T64, axis=1)[None, :] * np.linalg.norm(r64, axis=1)[:, None])
     diff = gs != os_
     assert np.all(np.abs(cos[diff]) < SIGN_MARGIN), "sign mismatch away from zero"
+
+
+@pytest.mark.parametrize("d,dt,n", [(1536, torch.float16, 8253), (1024, torch.bfloat16, 12000),
+                                    (256, torch.float16, 60001)])
+def test_many_tiles_per_cta(d, dt, n):
+    """Several tiles per CTA (the stage ring and the norm hand-off wrap many times): every row's
+    norm, codes, gamma and sign against the oracle, for the MSE quantizer, TurboQuant-prod through
+    row blocks of a small workspace, and the QJL sketch."""
+    x = _input(n, d, dt, seed=d + n)
+    x64 = to_f64(x)
+    nrm64 = np.linalg.norm(x64, axis=1)
+    pi64, c64, T64, pi_d, c_d, T_d = _params(d, 2, dt)
+    codes, norms = kvrq.tq_quantize_mse(x, pi_d, c_d, 2)
+    torch.cuda.synchronize()
+    kvrq.device_status()
+    assert np.allclose(to_f64(norms), nrm64, rtol=1e-5)
+    ref = tq.mse_quantize(x64, pi64, c64, 2)
+    compare_codes(words_u32(codes), ref, d, 2, c64)
+
+    ws = torch.empty((kvrq.tq_workspace_bytes(2048, d),), dtype=torch.uint8, device="cuda")
+    codes, signs, gammas, norms = kvrq.tq_quantize_prod(x, pi_d, T_d, c_d, 3, workspace=ws)
+    torch.cuda.synchronize()
+    kvrq.device_status()
+    assert np.allclose(to_f64(norms), nrm64, rtol=1e-5)
+    ref = tq.prod_quantize(x64, pi64, T64, c64, 3, sketch_operand="f16")
+    nb, bad = compare_codes(words_u32(codes), ref, d, 2, c64)
+    assert np.allclose(to_f64(gammas)[~bad], ref["gammas"][~bad], rtol=1e-4, atol=1e-7)
+    diff = (ocodes.unpack(words_u32(signs), d, 1) != ocodes.unpack(ref["signs_words"], d, 1)) & ~bad[:, None]
+    assert np.all(np.abs(ref["z"][diff]) < SIGN_MARGIN), "sign mismatch away from zero"
+
+    T_s = T_d.to(dt)  # the sketch takes T in the vectors' own 16-bit type
+    signs, gammas = kvrq.qjl_sketch(x, T_s)
+    torch.cuda.synchronize()
+    kvrq.device_status()
+    assert np.allclose(to_f64(gammas), nrm64, rtol=1e-5)
+    Ts64 = to_f64(T_s)
+    sk = tq.qjl_sketch(x64, Ts64)
+    cos = sk["p"] / (np.linalg.norm(Ts64, axis=1)[None, :] * nrm64[:, None])
+    diff = ocodes.unpack(words_u32(signs), d, 1) != ocodes.unpack(sk["signs_words"], d, 1)
+    assert np.all(np.abs(cos[diff]) < SIGN_MARGIN), "sign mismatch away from zero"
