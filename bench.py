@@ -255,6 +255,49 @@ def decode_step_c4(kvrq, synth, torch, dev, batch, steps, warmup, layers=36, kv_
     return out
 
 
+def kv_stack_c3(kvrq, synth, torch, dev, steps, layers=32, kv_heads=8, tokens=32768):
+    """Llama-3.1-8B-shaped KV stack: keys from a rank-16 factor model with 4 outlier channels,
+    values N(0,1), both bf16 [layers][KV heads][tokens][128]; keys compressed with TurboQuant-prod
+    3-bit (2-bit codes + 1-bit QJL, m = 128), values with RotorQuant 3-bit. Each timed step compresses
+    the whole stack (8,388,608 keys and as many values, 4 GiB of input)."""
+    n = layers * kv_heads * tokens
+    k = synth.factor_keys(layers, kv_heads, tokens, D, seed=21, dtype=torch.bfloat16, device=dev).view(n, D)
+    v = synth.gaussian(n, D, seed=22, dtype=torch.bfloat16, device=dev)
+    pi = torch.from_numpy(kvrq.tq_rotation_init(D, 2)).to(torch.bfloat16).to(dev)
+    T = torch.from_numpy(kvrq.qjl_matrix_init(D, D, 3)).to(torch.float16).to(dev)
+    rot = torch.from_numpy(kvrq.rq_rotors_init(D, 1).astype(np.float32)).to(dev)
+    ck = torch.from_numpy(kvrq.tq_codebook_init(D, 2)[0].astype(np.float32)).to(dev)
+    cv = torch.from_numpy(kvrq.tq_codebook_init(D, 3)[0].astype(np.float32)).to(dev)
+    kc, ks, kg, kn = kvrq.tq_quantize_prod(k, pi, T, ck, 3)
+    vc, vn = kvrq.rq_quantize(v, rot, cv, 3)
+    stream = torch.cuda.current_stream()
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    tk, tv = [], []
+    for i in range(steps + 2):
+        a, b, c = ev(), ev(), ev()
+        a.record(stream)
+        kvrq.tq_quantize_prod(k, pi, T, ck, 3, codes=kc, signs=ks, gammas=kg, norms=kn, stream=stream)
+        b.record(stream)
+        kvrq.rq_quantize(v, rot, cv, 3, codes=vc, norms=vn, stream=stream)
+        c.record(stream)
+        c.synchronize()
+        if i >= 2:
+            tk.append(a.elapsed_time(b))
+            tv.append(b.elapsed_time(c))
+    kvrq.device_status()
+    mk, mv = sum(tk) / len(tk), sum(tv) / len(tv)
+    bk = 2 * D + 4 * kvrq.packed_words(D, 2) + 4 * (D // 32) + 8  # 312 B per key
+    bv = 2 * D + 4 * kvrq.packed_words(129, 3) + 4                  # 312 B per value
+    out = {"vectors_each": n, "keys_ms": mk, "values_ms": mv, "ms_per_step": mk + mv,
+           "keys_Gvec_s": n / mk / 1e6, "values_Gvec_s": n / mv / 1e6,
+           "keys_GB_s": n * bk / mk / 1e6, "values_GB_s": n * bv / mv / 1e6,
+           "stack_GB_s": n * (bk + bv) / (mk + mv) / 1e6,
+           "keys_TFLOP_s": n * 4.0 * D * D / mk / 1e9}
+    del k, v, kc, ks, kg, kn, vc, vn
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_leg_only(args):
     """One kernel leg on args.rows seeded vectors: a warm-up call, then args.iters timed calls."""
     import torch
@@ -585,9 +628,11 @@ def main():
         torch.cuda.empty_cache()
 
     decode = None
+    stack = None
     if not args.no_large:
         decode = {"b1": decode_step_c4(kvrq, synth, torch, dev, 1, max(args.steps, 5), args.warmup),
                   "b16": decode_step_c4(kvrq, synth, torch, dev, 16, 5, 3)}
+        stack = kv_stack_c3(kvrq, synth, torch, dev, 5)
     clk.__exit__(None, None, None)
     cpu = None
     if rank == 0:
@@ -616,6 +661,7 @@ def main():
             "legs": legs_out,
             "hbm_1gib": large,
             "decode_c4": decode,
+            "kv_stack_c3": stack,
             "e2e": {"value": N_VEC * world / (e2e * 1e-3) / 1e6, "unit": "Mvec/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms": e2e},
             "gpu_launches": launches,

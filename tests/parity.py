@@ -92,3 +92,59 @@ def compare_floats(gpu, ref, out_dtype, row_scale, skip_rows=None, arith_rtol=2e
     if rel.size:
         assert rel.max() <= 1e-3 + UNIT_ROUNDOFF[out_dtype], "%s: normwise relative error %g" % (name, rel.max())
     return int(keep.sum())
+
+
+# Probabilistic rounding-error model of the float32 sums on the CUDA path
+# (|error| <= LAMBDA * sqrt(n) * 2^-24 * sum |terms|, Higham & Mary 2019).
+LAMBDA = 4.0
+
+
+def residual_sketch_slack(ref, x64, Pi64, T64, centroids):
+    """(p, bound): p[i, j] = (rho_i . T_j) with rho = fp16(256 r_rot) as the oracle forms it, and a bound on
+    |p| within which the CUDA path's sign of p may differ from the oracle's.
+
+    The kernel forms y = Pi x with float32 sums of exact fp16 products, scales by 1/||x|| and subtracts the
+    centroid, so each residual coordinate may differ from the float64 one by
+    eps = LAMBDA sqrt(d) 2^-24 sum_k |Pi_ik u_k| + 2^-21 |y| + 2^-22 |c| (sums, then the norm, its
+    reciprocal, the fma and the centroid chain). A coordinate of 256 r_rot within 256 eps of an fp16
+    rounding midpoint may round to either neighbour, moving rho_k by one fp16 step; p_j then moves by at
+    most sum_k |T_jk| d_rho_k, and the sketch's own float32 sums add LAMBDA sqrt(d) 2^-24 sum_k |T_jk rho_k|."""
+    x64 = np.asarray(x64, dtype=np.float64)
+    Pi64 = np.asarray(Pi64, dtype=np.float64)
+    T64 = np.asarray(T64, dtype=np.float64)
+    d = x64.shape[1]
+    nrm = np.linalg.norm(x64, axis=1, keepdims=True)
+    u = x64 / np.where(nrm > 0, nrm, 1.0)
+    y = np.asarray(ref["y"], dtype=np.float64)
+    c_hat = np.asarray(centroids, dtype=np.float64)[ref["codes"]]
+    s = 256.0 * (y - c_hat)
+    g = LAMBDA * np.sqrt(d) * 2.0 ** -24
+    eps = g * (np.abs(u) @ np.abs(Pi64).T) + 2.0 ** -21 * np.abs(y) + 2.0 ** -22 * np.abs(c_hat)
+    rho = s.astype(np.float16).astype(np.float64)
+    lo = (s - 256.0 * eps).astype(np.float16).astype(np.float64)
+    hi = (s + 256.0 * eps).astype(np.float16).astype(np.float64)
+    d_rho = np.maximum(np.abs(hi - rho), np.abs(lo - rho))
+    aT = np.abs(T64).T
+    p = rho @ T64.T
+    bound = d_rho @ aT + g * (np.abs(rho) @ aT)
+    return p, bound
+
+
+def compare_sketch_signs(gpu_sign_words, ref, x64, Pi64, T64, centroids, skip_rows=None, max_frac=1e-4):
+    """QJL signs of TurboQuant-prod: equal to the oracle's except where |p| is within the arithmetic's bound
+    (residual_sketch_slack), and differing in at most max_frac of the signs compared (at least 8).
+    Returns the number of differing signs."""
+    T64 = np.asarray(T64, dtype=np.float64)
+    m = T64.shape[0]
+    gs = ocodes.unpack(np.asarray(gpu_sign_words, dtype=np.uint32), m, 1)
+    os_ = ocodes.unpack(ref["signs_words"], m, 1)
+    keep = np.ones(gs.shape[0], bool) if skip_rows is None else ~np.asarray(skip_rows)
+    diff = (gs != os_) & keep[:, None]
+    if diff.any():
+        p, bound = residual_sketch_slack(ref, x64, Pi64, T64, centroids)
+        far = diff & (np.abs(p) > bound)
+        assert not far.any(), "sign differs beyond the rounding bound at %s (p %s, bound %s)" % (
+            np.argwhere(far)[:5].tolist(), p[far][:5], bound[far][:5])
+    n = int(diff.sum())
+    assert n <= max(8, max_frac * keep.sum() * m), "%d of %d signs differ" % (n, keep.sum() * m)
+    return n

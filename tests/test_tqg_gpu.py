@@ -10,7 +10,7 @@ import torch
 import kv_cache_vector_rq_b200 as kvrq
 from kv_cache_vector_rq_b200 import synth
 from oracle import codebook, codes as ocodes, params, tq
-from tests.parity import compare_codes, to_f64, words_u32
+from tests.parity import compare_codes, compare_sketch_signs, to_f64, words_u32
 
 pytestmark = pytest.mark.gpu
 
@@ -129,10 +129,7 @@ def test_prod_quantize_and_dequantize_tiled(d, dt, bits, n, ws_rows):
     assert np.allclose(to_f64(norms), ref["norms"], rtol=1e-5)
     g = to_f64(gammas)
     assert np.allclose(g[~bad], ref["gammas"][~bad], rtol=1e-4, atol=1e-7)
-    gs = ocodes.unpack(words_u32(signs), d, 1)
-    os_ = ocodes.unpack(ref["signs_words"], d, 1)
-    diff = (gs != os_) & ~bad[:, None]
-    assert np.all(np.abs(ref["z"][diff]) < SIGN_MARGIN), "sign mismatch away from zero"
+    compare_sketch_signs(words_u32(signs), ref, to_f64(x), pi64, T64, c64, skip_rows=bad)
     if ws_rows is not None:  # the row blocking does not change any bit
         c1, s1, g1, n1 = kvrq.tq_quantize_prod(x, pi_d, T_d, c_d, bits)
         assert torch.equal(c1, codes) and torch.equal(s1, signs) and torch.equal(g1, gammas)
@@ -214,8 +211,7 @@ def test_many_tiles_per_cta(d, dt, n):
     ref = tq.prod_quantize(x64, pi64, T64, c64, 3, sketch_operand="f16")
     nb, bad = compare_codes(words_u32(codes), ref, d, 2, c64)
     assert np.allclose(to_f64(gammas)[~bad], ref["gammas"][~bad], rtol=1e-4, atol=1e-7)
-    diff = (ocodes.unpack(words_u32(signs), d, 1) != ocodes.unpack(ref["signs_words"], d, 1)) & ~bad[:, None]
-    assert np.all(np.abs(ref["z"][diff]) < SIGN_MARGIN), "sign mismatch away from zero"
+    compare_sketch_signs(words_u32(signs), ref, x64, pi64, T64, c64, skip_rows=bad)
 
     T_s = T_d.to(dt)  # the sketch takes T in the vectors' own 16-bit type
     signs, gammas = kvrq.qjl_sketch(x, T_s)
