@@ -129,8 +129,8 @@ __device__ __forceinline__ void build_codebook(const float* __restrict__ centroi
 // start at 2^23; the low 23 mantissa bits of each accumulator are a window
 // of the packed bit stream.
 // ============================================================================
-#ifndef KVRQ_ROW_MIN_BLOCKS
-#define KVRQ_ROW_MIN_BLOCKS 4  // CTAs per SM the register budget is sized for
+#ifndef KVRQ_ROW_MIN_WARPS
+#define KVRQ_ROW_MIN_WARPS 16  // resident warps per SM the register budget is sized for
 #endif
 
 namespace row {
@@ -139,7 +139,9 @@ constexpr int D = 128;
 constexpr int G = 43;         // groups of 3
 constexpr int NP = 22;        // group pairs (the last: group 42 and an all-zero group)
 constexpr int NC = 3 * G;     // 129 stored codes
-constexpr int kRows = 128;    // threads per CTA (4 warps)
+// Two warps per CTA: small launches (a few thousand 32-row sub-tiles) spread
+// over the SMs within one CTA of each other.
+constexpr int kRows = 64;     // threads per CTA (2 warps)
 constexpr int kWR = 32;       // rows per warp sub-tile
 constexpr int kWarps = kRows / kWR;
 constexpr float kB = 4611686018427387904.0f;      // 2^62
@@ -173,9 +175,12 @@ template <typename T, int BITS, int MODE, int STAGES>
 struct Smem {
   static constexpr int W = Codes<BITS>::W;
   static constexpr int tile_bytes = kWarps * STAGES * Tile<T>::kTileBytes;  // [warp][stage] sub-tiles
-  static constexpr int codes_off = tile_bytes;                               // [warp][2][kWR][W] words
+  // code words per warp: dequantize [2][kWR][W] (bulk loads, double-buffered); quantize [kWR][W] (one
+  // bulk store per sub-tile: before the warp's next sub-tile writes codes, that store has read them)
+  static constexpr int codes_off = tile_bytes;
   static constexpr int codes_stage = ((kWR * W * 4 + 15) / 16) * 16;
-  static constexpr int lut_off = codes_off + kWarps * 2 * codes_stage;  // dequantize: [K][kRows] floats
+  static constexpr int codes_bytes = kWarps * codes_stage * (MODE == RQ_DQ ? 2 : 1);
+  static constexpr int lut_off = codes_off + codes_bytes;  // dequantize: [K][kRows] floats
   static constexpr int lut_bytes = MODE == RQ_DQ ? Codes<BITS>::K * kRows * 4 : 0;
   static constexpr int mp_off = lut_off + lut_bytes;  // [NP][10] float2
   static constexpr int mp_bytes = NP * 10 * 8;
@@ -216,7 +221,8 @@ __device__ __forceinline__ void build_consts(const float* __restrict__ centroids
 }
 
 template <typename T, int BITS, int MODE, int STAGES>
-__global__ void __launch_bounds__(kRows, MODE == RQ_Q ? 2 : KVRQ_ROW_MIN_BLOCKS) rq_row_kernel(const __grid_constant__ CUtensorMap map_x,
+__global__ void __launch_bounds__(kRows, (MODE == RQ_Q ? KVRQ_ROW_MIN_WARPS / 2 : KVRQ_ROW_MIN_WARPS) / kWarps)
+    rq_row_kernel(const __grid_constant__ CUtensorMap map_x,
                                                        const __grid_constant__ CUtensorMap map_o, RqArgs a) {
   using TL = Tile<T>;
   using CD = Codes<BITS>;
@@ -239,23 +245,12 @@ __global__ void __launch_bounds__(kRows, MODE == RQ_Q ? 2 : KVRQ_ROW_MIN_BLOCKS)
   // each warp streams its own 32-row sub-tiles: its buffers, barriers and copies
   uint64_t* w_bar = reinterpret_cast<uint64_t*>(smem + SM::bar_off) + warp * (STAGES + 2);  // [s] tiles, [STAGES + c] codes
   uint8_t* w_tiles = smem + warp * STAGES * TL::kTileBytes;
-  uint32_t* w_codes = s_codes + warp * 2 * (SM::codes_stage / 4);
+  uint32_t* w_codes = s_codes + warp * (MODE == RQ_DQ ? 2 : 1) * (SM::codes_stage / 4);
   const int64_t n = a.n;
   const int nsub = (int)((n + kWR - 1) / kWR);  // n < 2^31 (checked on the host)
   const int gw = (int)blockIdx.x * kWarps + warp, tw = (int)gridDim.x * kWarps;
   // dequantize: a full sub-tile of packed codes is one contiguous, 16-byte aligned block
   const bool codes_bulk = !kIn && a.ldc == W && (reinterpret_cast<uintptr_t>(a.codes_in) & 15) == 0;
-
-  if (tid == 0) {
-    if (kIn) tma_prefetch_desc(&map_x);
-    if (kOut) tma_prefetch_desc(&map_o);
-    for (int s = 0; s < kWarps * (STAGES + 2); ++s)
-      mbar_init(reinterpret_cast<uint64_t*>(smem + SM::bar_off) + s, 1);
-    fence_barrier_init();
-  }
-  build_pair_table(a.rotors, reinterpret_cast<float2*>(smem + SM::mp_off));
-  build_consts<BITS>(a.centroids, s_sc, s_mag, s_cf);
-  __syncthreads();
 
   // bit b of `par`: parity of the next phase of barrier b (all lanes);
   // bit b of `pend`: a copy completing on barrier b is in flight (lane 0)
@@ -278,7 +273,13 @@ __global__ void __launch_bounds__(kRows, MODE == RQ_Q ? 2 : KVRQ_ROW_MIN_BLOCKS)
               &w_bar[STAGES + c]);
   };
 
+  // Each warp sets up its own barriers and starts its first copies before the
+  // CTA forms its tables, so the rotor loads overlap the first sub-tile's copy.
   if (lane == 0) {
+    if (kIn) tma_prefetch_desc(&map_x);
+    if (kOut) tma_prefetch_desc(&map_o);
+    for (int b = 0; b < STAGES + 2; ++b) mbar_init(&w_bar[b], 1);
+    fence_barrier_init();
     if (kIn) {
       for (int s = 0; s < STAGES; ++s)
         if (sub_of(s) < nsub) issue_tile(sub_of(s), s);
@@ -287,6 +288,9 @@ __global__ void __launch_bounds__(kRows, MODE == RQ_Q ? 2 : KVRQ_ROW_MIN_BLOCKS)
         if (sub_of(c) < nsub && codes_bulk_tile(sub_of(c))) issue_codes(sub_of(c), c);
     }
   }
+  build_pair_table(a.rotors, reinterpret_cast<float2*>(smem + SM::mp_off));
+  build_consts<BITS>(a.centroids, s_sc, s_mag, s_cf);
+  __syncthreads();
 
   int it = 0;
   for (int sub = gw; sub < nsub; sub += tw, ++it) {
@@ -296,12 +300,14 @@ __global__ void __launch_bounds__(kRows, MODE == RQ_Q ? 2 : KVRQ_ROW_MIN_BLOCKS)
     const int rows = (int)(n - row0 < (int64_t)kWR ? n - row0 : (int64_t)kWR);
     const int64_t row = row0 + lane;
     uint8_t* tb = w_tiles + s * TL::kTileBytes;
-    uint32_t* stage_codes = w_codes + cs * (SM::codes_stage / 4);
+    uint32_t* stage_codes = w_codes + (kIn ? 0 : cs * (SM::codes_stage / 4));
 
     // ---------------------------------------------------------------- inputs
     bool ok = true;
     if constexpr (kIn) {
-      if (lane == 0) bulk_wait_read<1>();  // the codes store from this staging buffer (two sub-tiles ago) is done
+      // quantize-only: the last sub-tile's codes store has read the staging words (the fused mode
+      // waited for its stores before loading this sub-tile)
+      if (!kOut && lane == 0) bulk_wait_read<0>();
       ok = mbar_wait(&w_bar[s], (par >> s) & 1, a.status);
       par ^= 1u << s;
       pend &= ~(1u << s);

@@ -454,8 +454,9 @@ __global__ void __launch_bounds__(Cfg<METHOD, BITS, NB>::kThreads, 1) score_kern
       prev_g = gam;
       tmem_wait_st();
       tc_fence_before();
-      fence_proxy_async_smem();  // this thread's stage reads come before the bulk copy that refills it
-      // all rows of the tile are in tensor memory, and every thread has read its stage
+      // All rows of the tile are in tensor memory, and every thread has read its stage: the words it
+      // loaded were decoded into the values just stored to tensor memory, so those loads have returned
+      // before the barrier that lets the leader refill the stage.
       asm volatile("bar.sync %0, 128;" ::"r"(1 + w) : "memory");
       if (r == 0) {
         tc_fence_after();
