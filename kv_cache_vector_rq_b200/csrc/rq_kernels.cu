@@ -27,7 +27,6 @@
 
 #include <cuda_runtime.h>
 
-#include <cstdlib>
 #include <type_traits>
 
 #include "kvrq_device.cuh"
@@ -139,11 +138,22 @@ constexpr int D = 128;
 constexpr int G = 43;         // groups of 3
 constexpr int NP = 22;        // group pairs (the last: group 42 and an all-zero group)
 constexpr int NC = 3 * G;     // 129 stored codes
-// Two warps per CTA: small launches (a few thousand 32-row sub-tiles) spread
-// over the SMs within one CTA of each other.
-constexpr int kRows = 64;     // threads per CTA (2 warps)
 constexpr int kWR = 32;       // rows per warp sub-tile
-constexpr int kWarps = kRows / kWR;
+
+// CTA shape. Ring (launches of at least two sub-tiles per warp, 16-bit rows,
+// quantize or fused, b <= 3): one 16-warp CTA per SM, each warp streaming its
+// sub-tiles through a ring of three half-tile boxes, so the next sub-tile's
+// halves load while the current one is computed and a box is reloaded as soon
+// as its x_hat store has read it (b = 4 code words leave no room for the third
+// box). Otherwise two-warp CTAs with one tile per warp, which also spread a
+// small launch over the SMs within one CTA of each other.
+template <typename T, int BITS, int MODE, bool RING>
+struct Shape {
+  static_assert(!RING || (MODE != RQ_DQ && sizeof(T) == 2 && BITS <= 3), "ring shape");
+  static constexpr bool kRing = RING;
+  static constexpr int kWarps = kRing ? 16 : 2;
+  static constexpr int kRows = 32 * kWarps;  // threads per CTA
+};
 constexpr float kB = 4611686018427387904.0f;      // 2^62
 constexpr float kShift = 9.313225746154785e-10f;  // 2^-30
 constexpr float kWindow0 = 8388608.0f;            // 2^23
@@ -171,10 +181,18 @@ struct Codes {
   static constexpr int NWIN = (NC + CPW - 1) / CPW;
 };
 
-template <typename T, int BITS, int MODE, int STAGES>
+template <typename T, int BITS, int MODE, bool RING>
 struct Smem {
+  using SH = Shape<T, BITS, MODE, RING>;
+  static constexpr int STAGES = 1;  // tiles per warp outside the ring
+  static constexpr int kWarps = SH::kWarps;
+  static constexpr int kRows = SH::kRows;
   static constexpr int W = Codes<BITS>::W;
-  static constexpr int tile_bytes = kWarps * STAGES * Tile<T>::kTileBytes;  // [warp][stage] sub-tiles
+  static constexpr int kRingBoxes = 3;
+  // [warp][box] half-tile boxes (ring) or [warp][stage] sub-tiles
+  static constexpr int tile_bytes = SH::kRing ? kWarps * kRingBoxes * Tile<T>::kBoxBytes
+                                              : kWarps * STAGES * Tile<T>::kTileBytes;
+  static constexpr int nbar = SH::kRing ? kRingBoxes : STAGES + 2;  // barriers per warp
   // code words per warp: dequantize [2][kWR][W] (bulk loads, double-buffered); quantize [kWR][W] (one
   // bulk store per sub-tile: before the warp's next sub-tile writes codes, that store has read them)
   static constexpr int codes_off = tile_bytes;
@@ -186,9 +204,10 @@ struct Smem {
   static constexpr int mp_bytes = NP * 10 * 8;
   static constexpr int cb_off = mp_off + mp_bytes;  // codebook constants
   static constexpr int cb_bytes = 64 * 4;
-  static constexpr int bar_off = cb_off + cb_bytes;  // per warp: STAGES sub-tile + 2 code-stage barriers
-  static constexpr int bytes = bar_off + 8 * kWarps * (STAGES + 2);
+  static constexpr int bar_off = cb_off + cb_bytes;  // per warp: ring boxes, or STAGES sub-tiles + 2 code stages
+  static constexpr int bytes = bar_off + 8 * kWarps * nbar;
   static constexpr int alloc = bytes + 1024;
+  static_assert(alloc <= 227 * 1024, "shared memory");
 };
 
 // mp[p][3i+j] = (M_{2p}[i][j], M_{2p+1}[i][j]) for the exact sandwich matrices;
@@ -308,13 +327,21 @@ struct Bisect {
   }
 };
 
-template <typename T, int BITS, int MODE, int STAGES>
-__global__ void __launch_bounds__(kRows, (MODE == RQ_Q ? KVRQ_ROW_MIN_WARPS / 2 : KVRQ_ROW_MIN_WARPS) / kWarps)
+template <typename T, int BITS, int MODE, bool RING>
+__global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
+                                  RING ? 1
+                                       : (MODE == RQ_Q ? KVRQ_ROW_MIN_WARPS / 2 : KVRQ_ROW_MIN_WARPS) /
+                                             Shape<T, BITS, MODE, RING>::kWarps)
     rq_row_kernel(const __grid_constant__ CUtensorMap map_x,
                                                        const __grid_constant__ CUtensorMap map_o, RqArgs a) {
   using TL = Tile<T>;
   using CD = Codes<BITS>;
-  using SM = Smem<T, BITS, MODE, STAGES>;
+  using SM = Smem<T, BITS, MODE, RING>;
+  using SH = Shape<T, BITS, MODE, RING>;
+  constexpr int STAGES = SM::STAGES;
+  constexpr bool kRing = SH::kRing;
+  constexpr int kWarps = SH::kWarps, kRows = SH::kRows;
+  constexpr int kNB = SM::nbar;  // barriers per warp
   constexpr int H = CD::H, W = CD::W, CPW = CD::CPW, NWIN = CD::NWIN;
   constexpr int E = TL::kE;
   constexpr bool kIn = MODE != RQ_DQ;
@@ -331,8 +358,9 @@ __global__ void __launch_bounds__(kRows, (MODE == RQ_Q ? KVRQ_ROW_MIN_WARPS / 2 
   float* s_cf = s_sc + 32;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // each warp streams its own 32-row sub-tiles: its buffers, barriers and copies
-  uint64_t* w_bar = reinterpret_cast<uint64_t*>(smem + SM::bar_off) + warp * (STAGES + 2);  // [s] tiles, [STAGES + c] codes
-  uint8_t* w_tiles = smem + warp * STAGES * TL::kTileBytes;
+  // barriers: ring [b] boxes; otherwise [s] tiles, [STAGES + c] codes
+  uint64_t* w_bar = reinterpret_cast<uint64_t*>(smem + SM::bar_off) + warp * kNB;
+  uint8_t* w_tiles = smem + warp * (kRing ? SM::kRingBoxes * TL::kBoxBytes : STAGES * TL::kTileBytes);
   uint32_t* w_codes = s_codes + warp * (MODE == RQ_DQ ? 2 : 1) * (SM::codes_stage / 4);
   const int64_t n = a.n;
   const int nsub = (int)((n + kWR - 1) / kWR);  // n < 2^31 (checked on the host)
@@ -344,7 +372,16 @@ __global__ void __launch_bounds__(kRows, (MODE == RQ_Q ? KVRQ_ROW_MIN_WARPS / 2 
   // bit b of `pend`: a copy completing on barrier b is in flight (lane 0)
   uint32_t par = 0, pend = 0;
 
-  auto sub_of = [&](int iter) -> int { return gw + iter * tw; };
+  // ring: CTA c takes sub-tiles c, c + grid, ... (warp-major), so a small launch reaches every SM;
+  // otherwise warp gw takes gw, gw + tw, ...
+  auto sub_of = [&](int iter) -> int {
+    return kRing ? (int)blockIdx.x + (int)gridDim.x * (warp + kWarps * iter) : gw + iter * tw;
+  };
+  auto issue_box = [&](int sub, int half, int bx) {  // lane 0: half `half` of sub-tile `sub` into ring box bx
+    pend |= 1u << bx;
+    mbar_arrive_expect_tx(&w_bar[bx], TL::kBoxBytes);
+    tma_load_2d(w_tiles + bx * TL::kBoxBytes, &map_x, half * TL::kBoxElems, sub * kWR, &w_bar[bx]);
+  };
   auto issue_tile = [&](int sub, int s) {  // lane 0
     pend |= 1u << s;
     mbar_arrive_expect_tx(&w_bar[s], TL::kTileBytes);
@@ -366,9 +403,15 @@ __global__ void __launch_bounds__(kRows, (MODE == RQ_Q ? KVRQ_ROW_MIN_WARPS / 2 
   if (lane == 0) {
     if (kIn) tma_prefetch_desc(&map_x);
     if (kOut) tma_prefetch_desc(&map_o);
-    for (int b = 0; b < STAGES + 2; ++b) mbar_init(&w_bar[b], 1);
+    for (int b = 0; b < kNB; ++b) mbar_init(&w_bar[b], 1);
     fence_barrier_init();
-    if (kIn) {
+    if constexpr (kRing) {  // sub-tile 0 in boxes 0 and 1, the first half of sub-tile 1 in box 2
+      if (sub_of(0) < nsub) {
+        issue_box(sub_of(0), 0, 0);
+        issue_box(sub_of(0), 1, 1);
+      }
+      if (sub_of(1) < nsub) issue_box(sub_of(1), 0, 2);
+    } else if (kIn) {
       for (int s = 0; s < STAGES; ++s)
         if (sub_of(s) < nsub) issue_tile(sub_of(s), s);
     } else {
@@ -381,18 +424,37 @@ __global__ void __launch_bounds__(kRows, (MODE == RQ_Q ? KVRQ_ROW_MIN_WARPS / 2 
   __syncthreads();
 
   int it = 0;
-  for (int sub = gw; sub < nsub; sub += tw, ++it) {
+  for (int sub = sub_of(0); sub < nsub; sub = sub_of(++it)) {
     const int s = it % STAGES;
     const int cs = it & 1;
     const int64_t row0 = (int64_t)sub * kWR;
     const int rows = (int)(n - row0 < (int64_t)kWR ? n - row0 : (int64_t)kWR);
     const int64_t row = row0 + lane;
     uint8_t* tb = w_tiles + s * TL::kTileBytes;
+    // ring: this sub-tile's halves sit in boxes blo (columns 0..63) and bhi (64..127)
+    const int blo = (2 * it) % 3, bhi = (2 * it + 1) % 3;
+    uint8_t* const box_lo = kRing ? w_tiles + blo * TL::kBoxBytes : tb;
+    uint8_t* const box_hi = kRing ? w_tiles + bhi * TL::kBoxBytes : tb + TL::kBoxBytes;
+    auto cptr = [&](int j) -> uint8_t* {  // 16-byte chunk j of this lane's row
+      if constexpr (kRing) return ((j >> 3) ? box_hi : box_lo) + lane * 128 + (((j & 7) ^ (lane & 7)) << 4);
+      else return tb + TL::chunk(lane, j);
+    };
     uint32_t* stage_codes = w_codes + (kIn ? 0 : cs * (SM::codes_stage / 4));
 
     // ---------------------------------------------------------------- inputs
     bool ok = true;
-    if constexpr (kIn) {
+    if constexpr (kRing) {
+      ok = mbar_wait(&w_bar[blo], (par >> blo) & 1, a.status);
+      if (ok) {
+        par ^= 1u << blo;
+        pend &= ~(1u << blo);
+        ok = mbar_wait(&w_bar[bhi], (par >> bhi) & 1, a.status);
+        if (ok) {
+          par ^= 1u << bhi;
+          pend &= ~(1u << bhi);
+        }
+      }
+    } else if constexpr (kIn) {
       // quantize-only: the last sub-tile's codes store has read the staging words (the fused mode
       // waited for its stores before loading this sub-tile)
       if (!kOut && lane == 0) bulk_wait_read<0>();
@@ -416,7 +478,7 @@ __global__ void __launch_bounds__(kRows, (MODE == RQ_Q ? KVRQ_ROW_MIN_WARPS / 2 
     if (!__all_sync(0xffffffffu, ok)) {
       // a wait ran out: wait (bounded) for this warp's other copies, then leave
       if (lane == 0)
-        for (int b = 0; b < STAGES + 2; ++b)
+        for (int b = 0; b < kNB; ++b)
           if ((pend >> b) & 1) mbar_wait(&w_bar[b], (par >> b) & 1, a.status);
       break;
     }
@@ -432,7 +494,7 @@ __global__ void __launch_bounds__(kRows, (MODE == RQ_Q ? KVRQ_ROW_MIN_WARPS / 2 
 #pragma unroll
       for (int j = 0; j < TL::kChunks; ++j) {
         float f[E];
-        Elem<T>::unpack(*reinterpret_cast<const uint4*>(tb + TL::chunk(lane, j)), f);
+        Elem<T>::unpack(*reinterpret_cast<const uint4*>(cptr(j)), f);
 #pragma unroll
         for (int k = 0; k < E / 2; ++k) {
           const float2 v = make_float2(f[2 * k], f[2 * k + 1]);
@@ -446,12 +508,21 @@ __global__ void __launch_bounds__(kRows, (MODE == RQ_Q ? KVRQ_ROW_MIN_WARPS / 2 
 #pragma unroll 1
         for (int j = 0; j < TL::kChunks; ++j) {
           float f[E];
-          Elem<T>::unpack(*reinterpret_cast<const uint4*>(tb + TL::chunk(lane, j)), f);
+          Elem<T>::unpack(*reinterpret_cast<const uint4*>(cptr(j)), f);
           for (int k = 0; k < E; ++k) ss = fmaf(f[k] * xs, f[k] * xs, ss);
         }
       }
       nq = sqrtf(ss);
       nrm = kScale ? nq / xs : nq;
+      if constexpr (kRing) {
+        // the previous sub-tile's stores have read their buffers: the box they left takes the next
+        // sub-tile's first half, and the code words can be staged again
+        if (lane == 0) {
+          bulk_wait_read<0>();
+          if (it > 0 && sub_of(it + 1) < nsub) issue_box(sub_of(it + 1), 0, (2 * it + 2) % 3);
+        }
+        __syncwarp();
+      }
     } else {
       nrm = lane < rows ? __ldg(a.norms_in + row * a.ldn) : 0.f;
       nq = nrm;
@@ -521,7 +592,7 @@ __global__ void __launch_bounds__(kRows, (MODE == RQ_Q ? KVRQ_ROW_MIN_WARPS / 2 
 #pragma unroll
         for (int e = 6 * p; e < 6 * p + 6; ++e) {
           if (e < D && e % E == 0) {
-            Elem<T>::unpack(*reinterpret_cast<const uint4*>(tb + TL::chunk(lane, e / E)), &xe[e]);
+            Elem<T>::unpack(*reinterpret_cast<const uint4*>(cptr(e / E)), &xe[e]);
             if constexpr (kScale) {
 #pragma unroll
               for (int k = 0; k < E; ++k) xe[e + k] *= xs;
@@ -604,7 +675,25 @@ __global__ void __launch_bounds__(kRows, (MODE == RQ_Q ? KVRQ_ROW_MIN_WARPS / 2 
 #pragma unroll
         for (int e = 6 * p; e < 6 * p + 6; ++e)
           if (e < D && e % E == E - 1)
-            *reinterpret_cast<uint4*>(tb + TL::chunk(lane, e / E)) = Elem<T>::pack(&xo[e - (E - 1)]);
+            *reinterpret_cast<uint4*>(cptr(e / E)) = Elem<T>::pack(&xo[e - (E - 1)]);
+      }
+      if constexpr (kRing) {
+        // pair 10 writes the last x_hat chunk of columns 0..63 (pair 9 read their last input chunk):
+        // that half leaves now, and once the store has read its box the box takes the next
+        // sub-tile's second half
+        static_assert(6 * 10 <= 63 && 6 * 10 + 5 >= 63 && 6 * 9 <= 56 && 6 * 9 + 5 >= 56, "half boundary");
+        if (p == 10) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (kOut && lane == 0) {
+            tma_store_2d(&map_o, 0, (int32_t)row0, box_lo);
+            bulk_commit();
+          }
+        }
+        if (p == 14 && lane == 0 && sub_of(it + 1) < nsub) {
+          if (kOut) bulk_wait_read<0>();
+          issue_box(sub_of(it + 1), 1, blo);
+        }
       }
     }
 
@@ -618,13 +707,17 @@ __global__ void __launch_bounds__(kRows, (MODE == RQ_Q ? KVRQ_ROW_MIN_WARPS / 2 
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      if constexpr (kOut) {
+      if constexpr (kOut && kRing) {
+        tma_store_2d(&map_o, TL::kBoxElems, (int32_t)row0, box_hi);
+      } else if constexpr (kOut) {
 #pragma unroll
         for (int b = 0; b < TL::kBoxes; ++b) tma_store_2d(&map_o, b * TL::kBoxElems, (int32_t)row0, tb + b * TL::kBoxBytes);
       }
       if (codes_bulk_out) bulk_store(a.codes_out + row0 * W, stage_codes, kWR * W * 4);
       if (kOut || codes_bulk_out) bulk_commit();
-      if constexpr (kIn) {
+      if constexpr (kRing) {
+        // the ring's boxes are refilled at the next sub-tile's norm pass and its pair 14
+      } else if constexpr (kIn) {
         const int next = sub_of(it + STAGES);
         if (next < nsub) {
           if (kOut) bulk_wait_read<0>();  // the x_hat store has read this buffer
@@ -978,35 +1071,27 @@ __global__ void __launch_bounds__(kThreads) rq_wide_kernel(RqArgs a) {
 // ============================================================================
 // Launch helpers (host)
 // ============================================================================
-template <typename T, int BITS, int MODE, int STAGES>
+template <typename T, int BITS, int MODE, bool RING>
 static cudaError_t launch_row_s(const CUtensorMap& mx, const CUtensorMap& mo, const RqArgs& a, cudaStream_t st,
                                 int num_sms) {
-  using SM = row::Smem<T, BITS, MODE, STAGES>;
-  auto kern = rq_row_kernel<T, BITS, MODE, STAGES>;
+  using SM = row::Smem<T, BITS, MODE, RING>;
+  using SH = row::Shape<T, BITS, MODE, RING>;
+  auto kern = rq_row_kernel<T, BITS, MODE, RING>;
   static int blocks_per_sm = -1;
   if (blocks_per_sm < 0) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::alloc);
     if (e != cudaSuccess) return e;
     int b = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, row::kRows, SM::alloc);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, SH::kRows, SM::alloc);
     if (e != cudaSuccess) return e;
     blocks_per_sm = b < 1 ? 1 : b;
   }
   const int64_t nsub = (a.n + row::kWR - 1) / row::kWR;
-  const int64_t grid = std::min<int64_t>((nsub + row::kWarps - 1) / row::kWarps, (int64_t)num_sms * blocks_per_sm);
-  kern<<<(unsigned)grid, row::kRows, SM::alloc, st>>>(mx, mo, a);
+  // ring: every CTA starts with at least one sub-tile (its warp 0 takes sub-tile blockIdx.x)
+  const int64_t want = SH::kRing ? nsub : (nsub + SH::kWarps - 1) / SH::kWarps;
+  const int64_t grid = std::min<int64_t>(want, (int64_t)num_sms * blocks_per_sm);
+  kern<<<(unsigned)grid, SH::kRows, SM::alloc, st>>>(mx, mo, a);
   return cudaGetLastError();
-}
-
-// Tile buffers per CTA: 1 lets four CTAs share an SM (latency hidden across
-// CTAs), 2 double-buffers within a CTA. KVRQ_RQ_STAGES overrides the default.
-static int row_stages() {
-  static int stages = -1;
-  if (stages < 0) {
-    const char* e = getenv("KVRQ_RQ_STAGES");
-    stages = (e && atoi(e) == 2) ? 2 : 1;
-  }
-  return stages;
 }
 
 int rq_row_box_rows() { return row::kWR; }
@@ -1014,8 +1099,13 @@ int rq_row_box_rows() { return row::kWR; }
 template <typename T, int BITS, int MODE>
 static cudaError_t launch_row(const CUtensorMap& mx, const CUtensorMap& mo, const RqArgs& a, cudaStream_t st,
                               int num_sms) {
-  if (row_stages() == 1) return launch_row_s<T, BITS, MODE, 1>(mx, mo, a, st, num_sms);
-  return launch_row_s<T, BITS, MODE, 2>(mx, mo, a, st, num_sms);
+  // the ring pays off once every warp of the GPU has two sub-tiles or more
+  constexpr bool kCanRing = MODE != RQ_DQ && sizeof(T) == 2 && BITS <= 3;
+  if constexpr (kCanRing) {
+    if ((a.n + row::kWR - 1) / row::kWR >= 2 * 16 * (int64_t)num_sms)
+      return launch_row_s<T, BITS, MODE, true>(mx, mo, a, st, num_sms);
+  }
+  return launch_row_s<T, BITS, MODE, false>(mx, mo, a, st, num_sms);
 }
 
 template <typename TI, typename TO, int BITS, int MODE, int TEAM>
