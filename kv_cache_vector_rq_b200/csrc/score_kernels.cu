@@ -308,8 +308,8 @@ __global__ void __launch_bounds__(Cfg<METHOD, BITS, NB>::kThreads, 1) score_kern
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t a_t = tmem + lane_off + (uint32_t)(w * C::WCOLS);
     const uint32_t acc_t = a_t + (uint32_t)C::KAP;
-    const uint8_t* lut_l = s_lut + (lane % DC::R) * DC::EB;  // this lane's replica
-    const uint8_t* slut_l = s_slut + (lane & 7) * 16;
+    const uint32_t lut_l = smem_u32(s_lut) + (uint32_t)((lane % DC::R) * DC::EB);  // this lane's replica
+    const uint32_t slut_l = smem_u32(s_slut) + (uint32_t)((lane & 7) * 16);
     bool ok = true;
     float prev_n = 0.f, prev_g = 0.f;
 
@@ -342,19 +342,19 @@ __global__ void __launch_bounds__(Cfg<METHOD, BITS, NB>::kThreads, 1) score_kern
         const int fi = c * FPC + f;  // field index: codes fi*P .. fi*P + P - 1
         if (fi * DC::P < C::NCODE) {
           const uint32_t v = field<DC::FB, W>(wc, fi * DC::FB);
-          const uint8_t* e = lut_l + v * 128;
+          const uint32_t e = lut_l + (v << 7);
           if constexpr (DC::EW == 4) {
-            const uint4 x = *reinterpret_cast<const uint4*>(e);
+            const uint4 x = lds_v4(e);
             rw[4 * f] = x.x;
             rw[4 * f + 1] = x.y;
             rw[4 * f + 2] = x.z;
             rw[4 * f + 3] = x.w;
           } else if constexpr (DC::EW == 2) {
-            const uint2 x = *reinterpret_cast<const uint2*>(e);
+            const uint2 x = lds_v2(e);
             rw[2 * f] = x.x;
             rw[2 * f + 1] = x.y;
           } else {
-            rw[f] = *reinterpret_cast<const uint32_t*>(e);
+            rw[f] = lds_u32(e);
           }
         } else {
 #pragma unroll
@@ -377,7 +377,7 @@ __global__ void __launch_bounds__(Cfg<METHOD, BITS, NB>::kThreads, 1) score_kern
       for (int bq = 0; bq < 8; ++bq) {
         const int byte = 8 * c + bq;
         const uint32_t v = (sg[byte >> 2] >> (8 * (byte & 3))) & 0xFFu;
-        const uint4 x = *reinterpret_cast<const uint4*>(slut_l + v * 128);
+        const uint4 x = lds_v4(slut_l + (v << 7));
         rw[4 * bq] = x.x;
         rw[4 * bq + 1] = x.y;
         rw[4 * bq + 2] = x.z;
@@ -411,10 +411,11 @@ __global__ void __launch_bounds__(Cfg<METHOD, BITS, NB>::kThreads, 1) score_kern
       }
       if (bulk && tile_full(j)) {
         const uint32_t* stg = s_stage + (w * kStages + s) * C::stage_words;
+        const uint32_t stg_a = smem_u32(stg);
         if constexpr (W % 4 == 0) {
 #pragma unroll
           for (int q = 0; q < W / 4; ++q) {
-            const uint4 v = *reinterpret_cast<const uint4*>(stg + r * W + 4 * q);
+            const uint4 v = lds_v4(stg_a + (uint32_t)((r * W + 4 * q) * 4));
             wc[4 * q] = v.x;
             wc[4 * q + 1] = v.y;
             wc[4 * q + 2] = v.z;
@@ -422,10 +423,10 @@ __global__ void __launch_bounds__(Cfg<METHOD, BITS, NB>::kThreads, 1) score_kern
           }
         } else {
 #pragma unroll
-          for (int q = 0; q < W; ++q) wc[q] = stg[r * W + q];
+          for (int q = 0; q < W; ++q) wc[q] = lds_u32(stg_a + (uint32_t)((r * W + q) * 4));
         }
         if constexpr (kProd) {
-          const uint4 v = *reinterpret_cast<const uint4*>(stg + kRows * W + r * NS);
+          const uint4 v = lds_v4(stg_a + (uint32_t)((kRows * W + r * NS) * 4));
           sg[0] = v.x;
           sg[1] = v.y;
           sg[2] = v.z;
