@@ -435,9 +435,11 @@ __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
     const int blo = (2 * it) % 3, bhi = (2 * it + 1) % 3;
     uint8_t* const box_lo = kRing ? w_tiles + blo * TL::kBoxBytes : tb;
     uint8_t* const box_hi = kRing ? w_tiles + bhi * TL::kBoxBytes : tb + TL::kBoxBytes;
-    auto cptr = [&](int j) -> uint8_t* {  // 16-byte chunk j of this lane's row
-      if constexpr (kRing) return ((j >> 3) ? box_hi : box_lo) + lane * 128 + (((j & 7) ^ (lane & 7)) << 4);
-      else return tb + TL::chunk(lane, j);
+    // shared-window address of 16-byte chunk j of this lane's row (32-bit: see lds_v4)
+    const uint32_t lo_a = smem_u32(box_lo), hi_a = smem_u32(box_hi), tb_a = smem_u32(tb);
+    auto cptr = [&](int j) -> uint32_t {
+      if constexpr (kRing) return ((j >> 3) ? hi_a : lo_a) + (uint32_t)(lane * 128 + (((j & 7) ^ (lane & 7)) << 4));
+      else return tb_a + TL::chunk(lane, j);
     };
     uint32_t* stage_codes = w_codes + (kIn ? 0 : cs * (SM::codes_stage / 4));
 
@@ -494,7 +496,7 @@ __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
 #pragma unroll
       for (int j = 0; j < TL::kChunks; ++j) {
         float f[E];
-        Elem<T>::unpack(*reinterpret_cast<const uint4*>(cptr(j)), f);
+        Elem<T>::unpack(lds_v4(cptr(j)), f);
 #pragma unroll
         for (int k = 0; k < E / 2; ++k) {
           const float2 v = make_float2(f[2 * k], f[2 * k + 1]);
@@ -508,7 +510,7 @@ __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
 #pragma unroll 1
         for (int j = 0; j < TL::kChunks; ++j) {
           float f[E];
-          Elem<T>::unpack(*reinterpret_cast<const uint4*>(cptr(j)), f);
+          Elem<T>::unpack(lds_v4(cptr(j)), f);
           for (int k = 0; k < E; ++k) ss = fmaf(f[k] * xs, f[k] * xs, ss);
         }
       }
@@ -564,6 +566,7 @@ __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
         s_lut[(H - 1 - j) * kRows + tid] = -ch;
       }
     }
+    const uint32_t lut_a = smem_u32(s_lut) + (uint32_t)(tid * 4);  // this thread's column of the table
     const float srow = nq > 0.f ? __fdiv_rn(kB, nq) : 0.f;
     // y' = y - (2^-30 ||x|| + 2^-126): an exact zero (also of a zero row) becomes negative
     const float shv = -fmaf(kShift, nq, 0x1p-126f);
@@ -592,7 +595,7 @@ __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
 #pragma unroll
         for (int e = 6 * p; e < 6 * p + 6; ++e) {
           if (e < D && e % E == 0) {
-            Elem<T>::unpack(*reinterpret_cast<const uint4*>(cptr(e / E)), &xe[e]);
+            Elem<T>::unpack(lds_v4(cptr(e / E)), &xe[e]);
             if constexpr (kScale) {
 #pragma unroll
               for (int k = 0; k < E; ++k) xe[e + k] *= xs;
@@ -660,8 +663,9 @@ __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
 #pragma unroll
         for (int i = 0; i < 3; ++i) {
           const int kx = 3 * (2 * p) + i, ky = 3 * (2 * p + 1) + i;
-          const float cx = s_lut[get_code<BITS, W>(wc, kx) * kRows + tid];
-          const float cy = (2 * p + 1 < G) ? s_lut[get_code<BITS, W>(wc, ky) * kRows + tid] : 0.f;
+          const float cx = __uint_as_float(lds_u32(lut_a + get_code<BITS, W>(wc, kx) * (kRows * 4)));
+          const float cy =
+              (2 * p + 1 < G) ? __uint_as_float(lds_u32(lut_a + get_code<BITS, W>(wc, ky) * (kRows * 4))) : 0.f;
           C[i] = make_float2(cx, cy);
         }
       }
@@ -675,7 +679,7 @@ __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
 #pragma unroll
         for (int e = 6 * p; e < 6 * p + 6; ++e)
           if (e < D && e % E == E - 1)
-            *reinterpret_cast<uint4*>(cptr(e / E)) = Elem<T>::pack(&xo[e - (E - 1)]);
+            sts_v4(cptr(e / E), Elem<T>::pack(&xo[e - (E - 1)]));
       }
       if constexpr (kRing) {
         // pair 10 writes the last x_hat chunk of columns 0..63 (pair 9 read their last input chunk):
