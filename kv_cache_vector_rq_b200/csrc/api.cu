@@ -202,7 +202,7 @@ static kvrq_status rq_call(const char* name, int mode, void* stream, const void*
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   const kvrq_dtype tdt = q_side ? xdt : odt;
-  bool row_path = d == 128;
+  bool row_path = rq_row_dims(d, xdt) && rq_row_dims(d, odt);
   if (q_side) row_path = row_path && rows_aligned16(x, ldx, xdt);
   if (dq_side) row_path = row_path && rows_aligned16(xhat, ldo, odt);
   if (mode == RQ_QDQ) row_path = row_path && xdt == odt;

@@ -134,10 +134,15 @@ __device__ __forceinline__ void build_codebook(const float* __restrict__ centroi
 
 namespace row {
 
-constexpr int D = 128;
-constexpr int G = 43;         // groups of 3
-constexpr int NP = 22;        // group pairs (the last: group 42 and an all-zero group)
-constexpr int NC = 3 * G;     // 129 stored codes
+// Row dimension (128 or 256): G groups of 3 (the last zero-padded), NP group
+// pairs (the last may pair a group with an all-zero one), NC stored codes.
+template <int DD>
+struct Dims {
+  static constexpr int D = DD;
+  static constexpr int G = (DD + 2) / 3;  // 43 / 86
+  static constexpr int NP = (G + 1) / 2;  // 22 / 43
+  static constexpr int NC = 3 * G;        // 129 / 258
+};
 constexpr int kWR = 32;       // rows per warp sub-tile
 
 // CTA shape. Ring (launches of at least two sub-tiles per warp, 16-bit rows,
@@ -158,7 +163,7 @@ constexpr float kB = 4611686018427387904.0f;      // 2^62
 constexpr float kShift = 9.313225746154785e-10f;  // 2^-30
 constexpr float kWindow0 = 8388608.0f;            // 2^23
 
-template <typename T>
+template <typename T, int D>
 struct Tile {
   static constexpr int kBoxElems = 128 / (int)sizeof(T);  // elements per 128-byte box row
   static constexpr int kBoxes = D / kBoxElems;             // 2 (16-bit) or 4 (fp32)
@@ -172,7 +177,7 @@ struct Tile {
   }
 };
 
-template <int BITS>
+template <int BITS, int NC>
 struct Codes {
   static constexpr int K = 1 << BITS;
   static constexpr int H = K / 2;
@@ -181,17 +186,18 @@ struct Codes {
   static constexpr int NWIN = (NC + CPW - 1) / CPW;
 };
 
-template <typename T, int BITS, int MODE, bool RING>
+template <typename T, int BITS, int MODE, bool RING, int DD>
 struct Smem {
   using SH = Shape<T, BITS, MODE, RING>;
+  using DM = Dims<DD>;
+  using TL = Tile<T, DD>;
   static constexpr int STAGES = 1;  // tiles per warp outside the ring
   static constexpr int kWarps = SH::kWarps;
   static constexpr int kRows = SH::kRows;
-  static constexpr int W = Codes<BITS>::W;
+  static constexpr int W = Codes<BITS, DM::NC>::W;
   static constexpr int kRingBoxes = 3;
   // [warp][box] half-tile boxes (ring) or [warp][stage] sub-tiles
-  static constexpr int tile_bytes = SH::kRing ? kWarps * kRingBoxes * Tile<T>::kBoxBytes
-                                              : kWarps * STAGES * Tile<T>::kTileBytes;
+  static constexpr int tile_bytes = SH::kRing ? kWarps * kRingBoxes * TL::kBoxBytes : kWarps * STAGES * TL::kTileBytes;
   static constexpr int nbar = SH::kRing ? kRingBoxes : STAGES + 2;  // barriers per warp
   // code words per warp: dequantize [2][kWR][W] (bulk loads, double-buffered); quantize [kWR][W] (one
   // bulk store per sub-tile: before the warp's next sub-tile writes codes, that store has read them)
@@ -199,9 +205,9 @@ struct Smem {
   static constexpr int codes_stage = ((kWR * W * 4 + 15) / 16) * 16;
   static constexpr int codes_bytes = kWarps * codes_stage * (MODE == RQ_DQ ? 2 : 1);
   static constexpr int lut_off = codes_off + codes_bytes;  // dequantize: [K][kRows] floats
-  static constexpr int lut_bytes = MODE == RQ_DQ ? Codes<BITS>::K * kRows * 4 : 0;
+  static constexpr int lut_bytes = MODE == RQ_DQ ? Codes<BITS, DM::NC>::K * kRows * 4 : 0;
   static constexpr int mp_off = lut_off + lut_bytes;  // [NP][10] float2
-  static constexpr int mp_bytes = NP * 10 * 8;
+  static constexpr int mp_bytes = DM::NP * 10 * 8;
   static constexpr int cb_off = mp_off + mp_bytes;  // codebook constants
   static constexpr int cb_bytes = 64 * 4;
   static constexpr int bar_off = cb_off + cb_bytes;  // per warp: ring boxes, or STAGES sub-tiles + 2 code stages
@@ -211,11 +217,12 @@ struct Smem {
 };
 
 // mp[p][3i+j] = (M_{2p}[i][j], M_{2p+1}[i][j]) for the exact sandwich matrices;
-// the all-zero group 43 has a zero matrix.
+// an all-zero padding group (43 at d = 128) has a zero matrix.
+template <int DD>
 __device__ __forceinline__ void build_pair_table(const float* __restrict__ rotors, float2* __restrict__ mp) {
-  for (int g = threadIdx.x; g < 2 * NP; g += blockDim.x) {
+  for (int g = threadIdx.x; g < 2 * Dims<DD>::NP; g += blockDim.x) {
     float m[9];
-    if (g < G) {
+    if (g < Dims<DD>::G) {
       const float4 r = __ldg(reinterpret_cast<const float4*>(rotors) + g);
       rotor_matrix(r.x, r.y, r.z, r.w, m);
     } else {
@@ -327,16 +334,19 @@ struct Bisect {
   }
 };
 
-template <typename T, int BITS, int MODE, bool RING>
+template <typename T, int BITS, int MODE, bool RING, int DD>
 __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
                                   RING ? 1
                                        : (MODE == RQ_Q ? KVRQ_ROW_MIN_WARPS / 2 : KVRQ_ROW_MIN_WARPS) /
                                              Shape<T, BITS, MODE, RING>::kWarps)
     rq_row_kernel(const __grid_constant__ CUtensorMap map_x,
                                                        const __grid_constant__ CUtensorMap map_o, RqArgs a) {
-  using TL = Tile<T>;
-  using CD = Codes<BITS>;
-  using SM = Smem<T, BITS, MODE, RING>;
+  using DM = Dims<DD>;
+  constexpr int D = DM::D, G = DM::G, NP = DM::NP, NC = DM::NC;
+  static_assert(!RING || DD == 128, "the ring holds half-tiles of d = 128 rows");
+  using TL = Tile<T, DD>;
+  using CD = Codes<BITS, NC>;
+  using SM = Smem<T, BITS, MODE, RING, DD>;
   using SH = Shape<T, BITS, MODE, RING>;
   constexpr int STAGES = SM::STAGES;
   constexpr bool kRing = SH::kRing;
@@ -419,7 +429,7 @@ __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
         if (sub_of(c) < nsub && codes_bulk_tile(sub_of(c))) issue_codes(sub_of(c), c);
     }
   }
-  build_pair_table(a.rotors, reinterpret_cast<float2*>(smem + SM::mp_off));
+  build_pair_table<DD>(a.rotors, reinterpret_cast<float2*>(smem + SM::mp_off));
   build_consts<BITS>(a.centroids, s_sc, s_mag, s_cf);
   __syncthreads();
 
@@ -1075,12 +1085,12 @@ __global__ void __launch_bounds__(kThreads) rq_wide_kernel(RqArgs a) {
 // ============================================================================
 // Launch helpers (host)
 // ============================================================================
-template <typename T, int BITS, int MODE, bool RING>
+template <typename T, int BITS, int MODE, bool RING, int DD>
 static cudaError_t launch_row_s(const CUtensorMap& mx, const CUtensorMap& mo, const RqArgs& a, cudaStream_t st,
                                 int num_sms) {
-  using SM = row::Smem<T, BITS, MODE, RING>;
+  using SM = row::Smem<T, BITS, MODE, RING, DD>;
   using SH = row::Shape<T, BITS, MODE, RING>;
-  auto kern = rq_row_kernel<T, BITS, MODE, RING>;
+  auto kern = rq_row_kernel<T, BITS, MODE, RING, DD>;
   static int blocks_per_sm = -1;
   if (blocks_per_sm < 0) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::alloc);
@@ -1100,16 +1110,18 @@ static cudaError_t launch_row_s(const CUtensorMap& mx, const CUtensorMap& mo, co
 
 int rq_row_box_rows() { return row::kWR; }
 
-template <typename T, int BITS, int MODE>
+bool rq_row_dims(int d, kvrq_dtype dt) { return d == 128 || (d == 256 && dt != KVRQ_F32); }
+
+template <typename T, int BITS, int MODE, int DD>
 static cudaError_t launch_row(const CUtensorMap& mx, const CUtensorMap& mo, const RqArgs& a, cudaStream_t st,
                               int num_sms) {
   // the ring pays off once every warp of the GPU has two sub-tiles or more
-  constexpr bool kCanRing = MODE != RQ_DQ && sizeof(T) == 2 && BITS <= 3;
+  constexpr bool kCanRing = DD == 128 && MODE != RQ_DQ && sizeof(T) == 2 && BITS <= 3;
   if constexpr (kCanRing) {
     if ((a.n + row::kWR - 1) / row::kWR >= 2 * 16 * (int64_t)num_sms)
-      return launch_row_s<T, BITS, MODE, true>(mx, mo, a, st, num_sms);
+      return launch_row_s<T, BITS, MODE, true, DD>(mx, mo, a, st, num_sms);
   }
-  return launch_row_s<T, BITS, MODE, false>(mx, mo, a, st, num_sms);
+  return launch_row_s<T, BITS, MODE, false, DD>(mx, mo, a, st, num_sms);
 }
 
 template <typename TI, typename TO, int BITS, int MODE, int TEAM>
@@ -1154,24 +1166,28 @@ static cudaError_t launch_general(const RqArgs& a, cudaStream_t st, int num_sms)
   return cudaGetLastError();
 }
 
-template <typename T, int MODE>
+template <typename T, int MODE, int DD>
 static cudaError_t row_by_bits(int bits, const CUtensorMap& mx, const CUtensorMap& mo, const RqArgs& a,
                                cudaStream_t st, int sms) {
   switch (bits) {
-    case 1: return launch_row<T, 1, MODE>(mx, mo, a, st, sms);
-    case 2: return launch_row<T, 2, MODE>(mx, mo, a, st, sms);
-    case 3: return launch_row<T, 3, MODE>(mx, mo, a, st, sms);
-    default: return launch_row<T, 4, MODE>(mx, mo, a, st, sms);
+    case 1: return launch_row<T, 1, MODE, DD>(mx, mo, a, st, sms);
+    case 2: return launch_row<T, 2, MODE, DD>(mx, mo, a, st, sms);
+    case 3: return launch_row<T, 3, MODE, DD>(mx, mo, a, st, sms);
+    default: return launch_row<T, 4, MODE, DD>(mx, mo, a, st, sms);
   }
 }
 
 template <int MODE>
 static cudaError_t row_by_type(kvrq_dtype dt, int bits, const CUtensorMap& mx, const CUtensorMap& mo,
                                const RqArgs& a, cudaStream_t st, int sms) {
+  if (a.d == 256) {  // 16-bit rows only (rq_row_dims)
+    if (dt == KVRQ_F16) return row_by_bits<__half, MODE, 256>(bits, mx, mo, a, st, sms);
+    return row_by_bits<__nv_bfloat16, MODE, 256>(bits, mx, mo, a, st, sms);
+  }
   switch (dt) {
-    case KVRQ_F32: return row_by_bits<float, MODE>(bits, mx, mo, a, st, sms);
-    case KVRQ_F16: return row_by_bits<__half, MODE>(bits, mx, mo, a, st, sms);
-    default: return row_by_bits<__nv_bfloat16, MODE>(bits, mx, mo, a, st, sms);
+    case KVRQ_F32: return row_by_bits<float, MODE, 128>(bits, mx, mo, a, st, sms);
+    case KVRQ_F16: return row_by_bits<__half, MODE, 128>(bits, mx, mo, a, st, sms);
+    default: return row_by_bits<__nv_bfloat16, MODE, 128>(bits, mx, mo, a, st, sms);
   }
 }
 

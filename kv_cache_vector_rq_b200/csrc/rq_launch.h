@@ -40,6 +40,9 @@ cudaError_t launch_rq_row(int mode, kvrq_dtype dt, int bits, const CUtensorMap& 
 
 // Rows per box of the tensor maps launch_rq_row expects.
 int rq_row_box_rows();
+// Row dimensions (and types) the one-thread-per-row kernel takes: d = 128, and
+// d = 256 for 16-bit rows.
+bool rq_row_dims(int d, kvrq_dtype dt);
 
 // Dynamic shared memory of the bulk-copy any-d kernel for d, or 0 when rows of
 // d elements of elem_bytes cannot take it (row not a multiple of 16 bytes, a
