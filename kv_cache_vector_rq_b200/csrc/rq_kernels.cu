@@ -898,8 +898,11 @@ struct Layout {
   }
 };
 
-// team size for d: the whole CTA once a row has 256 groups or more
-__host__ __device__ inline int team_of(int d) { return (d + 2) / 3 >= 256 ? kWarps : 1; }
+// team size: one warp per row (warp-shuffle norm, no CTA barrier per row)
+// while every warp's two row buffers fit; the whole CTA beyond that
+__host__ __device__ inline int team_of(int d, int bits, int elem_bytes) {
+  return Layout(d, bits, d * elem_bytes, 1).bytes <= 227 * 1024 ? 1 : kWarps;
+}
 
 template <int TEAM>
 __device__ __forceinline__ void team_sync() {
@@ -1147,14 +1150,15 @@ static cudaError_t launch_wide_t(const RqArgs& a, cudaStream_t st, int num_sms) 
 
 template <typename TI, typename TO, int BITS, int MODE>
 static cudaError_t launch_wide(const RqArgs& a, cudaStream_t st, int num_sms) {
-  if (wide::team_of(a.d) == 1) return launch_wide_t<TI, TO, BITS, MODE, 1>(a, st, num_sms);
+  using TB = typename std::conditional<MODE != RQ_DQ, TI, TO>::type;
+  if (wide::team_of(a.d, BITS, (int)sizeof(TB)) == 1) return launch_wide_t<TI, TO, BITS, MODE, 1>(a, st, num_sms);
   return launch_wide_t<TI, TO, BITS, MODE, wide::kWarps>(a, st, num_sms);
 }
 
 // Shared memory the bulk-copy kernel needs for d (0 when it cannot take d).
 int rq_wide_smem_bytes(int d, int bits, int elem_bytes) {
   if ((d * elem_bytes) % 16 != 0 || d * elem_bytes > 16384) return 0;
-  const wide::Layout L(d, bits, d * elem_bytes, wide::team_of(d));
+  const wide::Layout L(d, bits, d * elem_bytes, wide::team_of(d, bits, elem_bytes));
   return L.bytes <= 227 * 1024 ? L.bytes : 0;
 }
 
