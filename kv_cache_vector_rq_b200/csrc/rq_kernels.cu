@@ -873,6 +873,34 @@ __global__ void __launch_bounds__(256) rq_general_kernel(RqArgs a) {
 // rq_general_kernel, so quantize-then-dequantize and the fused launch agree bit
 // for bit.
 // ============================================================================
+// one element of a row buffer at a 32-bit shared address, as float
+template <typename TB>
+__device__ __forceinline__ float lds_elem(uint32_t addr) {
+  if constexpr (std::is_same<TB, float>::value) {
+    return __uint_as_float(lds_u32(addr));
+  } else {
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+    if constexpr (std::is_same<TB, __half>::value) return __half2float(__ushort_as_half(v));
+    else return __bfloat162float(__ushort_as_bfloat16(v));
+  }
+}
+template <typename TB>
+__device__ __forceinline__ void sts_elem(uint32_t addr, float f) {
+  if constexpr (std::is_same<TB, float>::value) {
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(f) : "memory");
+  } else {
+    const TB h = Elem<TB>::from_float(f);
+    unsigned short v;
+    if constexpr (std::is_same<TB, __half>::value) v = __half_as_ushort(h);
+    else v = __bfloat16_as_ushort(h);
+    asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+  }
+}
+__device__ __forceinline__ void red_or_shared(uint32_t addr, uint32_t v) {
+  asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
 namespace wide {
 
 constexpr int kWarps = 8;
@@ -890,7 +918,7 @@ struct Layout {
     BUF = team == 1 ? (row_bytes > 2048 ? row_bytes : 2048) : row_bytes;
     RB = BUF / row_bytes;
     m_off = 0;
-    buf_off = ((G * 9 * 4 + 127) / 128) * 128;
+    buf_off = ((G * 12 * 4 + 127) / 128) * 128;  // [G][12]: 3x3 matrix padded to 48 bytes
     codes_off = buf_off + teams * 2 * BUF;
     bar_off = codes_off + ((teams * RB * W * 4 + 15) / 16) * 16;
     part_off = bar_off + teams * 2 * 8;
@@ -932,7 +960,7 @@ __global__ void __launch_bounds__(kThreads) rq_wide_kernel(RqArgs a) {
   build_codebook<BITS>(a.centroids, s_tau, s_mag, s_c);
   for (int g = threadIdx.x; g < G; g += kThreads) {
     const float4 r = __ldg(reinterpret_cast<const float4*>(a.rotors) + g);
-    rotor_matrix(r.x, r.y, r.z, r.w, s_m + g * 9);
+    rotor_matrix(r.x, r.y, r.z, r.w, s_m + g * 12);
   }
   for (int i = t; i < RB * W; i += TT) t_codes[i] = 0u;
   if (t == 0) {
@@ -1012,14 +1040,25 @@ __global__ void __launch_bounds__(kThreads) rq_wide_kernel(RqArgs a) {
       Quantizer<BITS> q;
       q.scale(s_tau, s_mag, nrm);
       uint32_t* wc = t_codes + r * W;
-      const uint32_t* cin = kIn ? nullptr : a.codes_in + row * a.ldc;
+      const uint32_t wc_a = smem_u32(wc), rb_a = smem_u32(rb), m_a = smem_u32(s_m), c_a = smem_u32(s_c);
+      if constexpr (!kIn) {
+        // the row's code words, coalesced, into the team's code buffer
+        const uint32_t* cin = a.codes_in + row * a.ldc;
+        for (int i = t; i < W; i += TT) wc[i] = __ldg(cin + i);
+        team_sync<TEAM>();
+      }
       for (int g = t; g < G; g += TT) {
-        const float* m = s_m + g * 9;
+        // the group's matrix: three 16-byte loads of its padded row of the table
+        const uint4 m0 = lds_v4(m_a + g * 48), m1 = lds_v4(m_a + g * 48 + 16), m2 = lds_v4(m_a + g * 48 + 32);
+        const float m[9] = {__uint_as_float(m0.x), __uint_as_float(m0.y), __uint_as_float(m0.z),
+                            __uint_as_float(m0.w), __uint_as_float(m1.x), __uint_as_float(m1.y),
+                            __uint_as_float(m1.z), __uint_as_float(m1.w), __uint_as_float(m2.x)};
+        const uint32_t e_a = rb_a + (uint32_t)(3 * g * (int)sizeof(TB));
         float c[3];
         if constexpr (kIn) {
           float v[3];
 #pragma unroll
-          for (int i = 0; i < 3; ++i) v[i] = (3 * g + i < d) ? Elem<TB>::to_float(rb[3 * g + i]) : 0.f;
+          for (int i = 0; i < 3; ++i) v[i] = (3 * g + i < d) ? lds_elem<TB>(e_a + i * (int)sizeof(TB)) : 0.f;
           uint32_t bits3 = 0;
 #pragma unroll
           for (int i = 0; i < 3; ++i) {
@@ -1027,24 +1066,25 @@ __global__ void __launch_bounds__(kThreads) rq_wide_kernel(RqArgs a) {
             bits3 |= q(y, c[i]) << (i * BITS);
           }
           const int bit = g * 3 * BITS;
-          atomicOr(&wc[bit >> 5], bits3 << (bit & 31));
-          if ((bit & 31) + 3 * BITS > 32) atomicOr(&wc[(bit >> 5) + 1], bits3 >> (32 - (bit & 31)));
+          red_or_shared(wc_a + (uint32_t)((bit >> 5) * 4), bits3 << (bit & 31));
+          if ((bit & 31) + 3 * BITS > 32) red_or_shared(wc_a + (uint32_t)((bit >> 5) * 4 + 4), bits3 >> (32 - (bit & 31)));
         } else {
 #pragma unroll
           for (int i = 0; i < 3; ++i) {
             const int bit = (3 * g + i) * BITS;
-            uint32_t v = __ldg(cin + (bit >> 5)) >> (bit & 31);
-            if ((bit & 31) + BITS > 32) v |= __ldg(cin + (bit >> 5) + 1) << (32 - (bit & 31));
-            c[i] = s_c[v & (K - 1)] * nrm;
+            uint32_t v = lds_u32(wc_a + (uint32_t)((bit >> 5) * 4)) >> (bit & 31);
+            if ((bit & 31) + BITS > 32) v |= lds_u32(wc_a + (uint32_t)((bit >> 5) * 4 + 4)) << (32 - (bit & 31));
+            c[i] = __uint_as_float(lds_u32(c_a + (v & (K - 1)) * 4)) * nrm;
           }
         }
         if constexpr (kOut) {
 #pragma unroll
           for (int i = 0; i < 3; ++i)
             if (3 * g + i < d)
-              rb[3 * g + i] = Elem<TB>::from_float(fmaf(m[6 + i], c[2], fmaf(m[3 + i], c[1], m[i] * c[0])));
+              sts_elem<TB>(e_a + i * (int)sizeof(TB), fmaf(m[6 + i], c[2], fmaf(m[3 + i], c[1], m[i] * c[0])));
         }
       }
+      if constexpr (!kIn) team_sync<TEAM>();  // the code buffer is refilled by the next row
       if constexpr (kIn) {
         team_sync<TEAM>();
         if (a.codes_out)
