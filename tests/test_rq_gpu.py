@@ -110,6 +110,25 @@ def test_general_bulk_rows_strided():
     _check_roundtrip(base[:, :256], 2)
 
 
+@pytest.mark.parametrize("bits", [1, 2, 3])
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+def test_ring_sizes(dt, bits):
+    # 160,033 rows: every warp has two 32-row sub-tiles or more, so the quantizing modes take the
+    # ring of half-tile boxes; dequantize (never the ring) must reproduce the fused x_hat bit for bit
+    n = 160033
+    x = synth.lognormal(n, 128, seed=bits + 7, dtype=DT[dt]).cuda()
+    sample = np.unique(np.concatenate([np.random.default_rng(bits).choice(n, 1536, replace=False),
+                                       [0, 31, 32, 4095, n - 33, n - 1]]))
+    nb, _, _ = _check_roundtrip(x, bits, sample=np.sort(sample))
+    assert nb <= 5
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_d256_bf16_row_kernel(bits):
+    x = synth.lognormal(1000, 256, seed=bits, dtype=torch.bfloat16).cuda()
+    _check_roundtrip(x, bits)
+
+
 def test_general_dimension_4096_fp32():
     x = synth.gaussian(200, 4096, seed=9, dtype=torch.float32).cuda()
     _check_roundtrip(x, 3)
