@@ -1047,43 +1047,51 @@ __global__ void __launch_bounds__(kThreads) rq_wide_kernel(RqArgs a) {
         for (int i = t; i < W; i += TT) wc[i] = __ldg(cin + i);
         team_sync<TEAM>();
       }
-      for (int g = t; g < G; g += TT) {
-        // the group's matrix: three 16-byte loads of its padded row of the table
-        const uint4 m0 = lds_v4(m_a + g * 48), m1 = lds_v4(m_a + g * 48 + 16), m2 = lds_v4(m_a + g * 48 + 32);
+      // One group: its padded matrix row (three 16-byte loads), its three elements at e_p, its code bits
+      // at `bit`; FULL: all three elements are inside the row (every group but a zero-padded last one).
+      auto group = [&](auto full, int g, uint32_t m_p, uint32_t e_p, int bit) {
+        constexpr bool kFull = decltype(full)::value;
+        const uint4 m0 = lds_v4(m_p), m1 = lds_v4(m_p + 16), m2 = lds_v4(m_p + 32);
         const float m[9] = {__uint_as_float(m0.x), __uint_as_float(m0.y), __uint_as_float(m0.z),
                             __uint_as_float(m0.w), __uint_as_float(m1.x), __uint_as_float(m1.y),
                             __uint_as_float(m1.z), __uint_as_float(m1.w), __uint_as_float(m2.x)};
-        const uint32_t e_a = rb_a + (uint32_t)(3 * g * (int)sizeof(TB));
         float c[3];
         if constexpr (kIn) {
           float v[3];
 #pragma unroll
-          for (int i = 0; i < 3; ++i) v[i] = (3 * g + i < d) ? lds_elem<TB>(e_a + i * (int)sizeof(TB)) : 0.f;
+          for (int i = 0; i < 3; ++i) v[i] = (kFull || 3 * g + i < d) ? lds_elem<TB>(e_p + i * (int)sizeof(TB)) : 0.f;
           uint32_t bits3 = 0;
 #pragma unroll
           for (int i = 0; i < 3; ++i) {
             const float y = fmaf(m[3 * i + 2], v[2], fmaf(m[3 * i + 1], v[1], m[3 * i] * v[0]));
             bits3 |= q(y, c[i]) << (i * BITS);
           }
-          const int bit = g * 3 * BITS;
           red_or_shared(wc_a + (uint32_t)((bit >> 5) * 4), bits3 << (bit & 31));
           if ((bit & 31) + 3 * BITS > 32) red_or_shared(wc_a + (uint32_t)((bit >> 5) * 4 + 4), bits3 >> (32 - (bit & 31)));
         } else {
 #pragma unroll
           for (int i = 0; i < 3; ++i) {
-            const int bit = (3 * g + i) * BITS;
-            uint32_t v = lds_u32(wc_a + (uint32_t)((bit >> 5) * 4)) >> (bit & 31);
-            if ((bit & 31) + BITS > 32) v |= lds_u32(wc_a + (uint32_t)((bit >> 5) * 4 + 4)) << (32 - (bit & 31));
+            const int b = bit + i * BITS;
+            uint32_t v = lds_u32(wc_a + (uint32_t)((b >> 5) * 4)) >> (b & 31);
+            if ((b & 31) + BITS > 32) v |= lds_u32(wc_a + (uint32_t)((b >> 5) * 4 + 4)) << (32 - (b & 31));
             c[i] = __uint_as_float(lds_u32(c_a + (v & (K - 1)) * 4)) * nrm;
           }
         }
         if constexpr (kOut) {
 #pragma unroll
           for (int i = 0; i < 3; ++i)
-            if (3 * g + i < d)
-              sts_elem<TB>(e_a + i * (int)sizeof(TB), fmaf(m[6 + i], c[2], fmaf(m[3 + i], c[1], m[i] * c[0])));
+            if (kFull || 3 * g + i < d)
+              sts_elem<TB>(e_p + i * (int)sizeof(TB), fmaf(m[6 + i], c[2], fmaf(m[3 + i], c[1], m[i] * c[0])));
         }
-      }
+      };
+      // whole groups with addresses advanced by constant strides, then the padded last group
+      const int G_full = d / 3;
+      int g = t, bit = t * 3 * BITS;
+      uint32_t m_p = m_a + (uint32_t)(t * 48), e_p = rb_a + (uint32_t)(3 * t * (int)sizeof(TB));
+#pragma unroll 2
+      for (; g < G_full; g += TT, bit += TT * 3 * BITS, m_p += TT * 48, e_p += TT * 3 * (int)sizeof(TB))
+        group(std::true_type{}, g, m_p, e_p, bit);
+      if (g < G) group(std::false_type{}, g, m_p, e_p, bit);
       if constexpr (!kIn) team_sync<TEAM>();  // the code buffer is refilled by the next row
       if constexpr (kIn) {
         team_sync<TEAM>();
