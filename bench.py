@@ -58,11 +58,28 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def kernel_source_hash(spec):
+    """SHA-256 prefix of a kernel's source: `file#ns` hashes the text of `namespace ns { ... }  // namespace ns`
+    in that file together with the device helper header it includes; a plain path hashes the whole file."""
+    import hashlib
+
+    path, _, ns = spec.partition("#")
+    src = os.path.join(ROOT, path)
+    if not os.path.exists(src):
+        return None
+    text = open(src, "rb").read()
+    if ns:
+        a = text.find(("namespace %s {" % ns).encode())
+        b = text.find(("}  // namespace %s" % ns).encode())
+        if a < 0 or b < a:
+            return None
+        text = text[a:b] + open(os.path.join(os.path.dirname(src), "kvrq_device.cuh"), "rb").read()
+    return hashlib.sha256(text).hexdigest()[:16]
+
+
 def recorded_traffic(kernel):
     """Per-launch DRAM bytes of `kernel` from profiles/traffic.txt, or None when that record is missing or the
     kernel's source changed since the counters were taken (the record keeps a SHA-256 prefix of the source)."""
-    import hashlib
-
     p = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(p):
         return None
@@ -72,8 +89,7 @@ def recorded_traffic(kernel):
         f = [x.strip() for x in line.split("|")]
         if f[0] != kernel:
             continue
-        src = os.path.join(ROOT, f[1])
-        if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != f[2]:
+        if kernel_source_hash(f[1]) != f[2]:
             return None
         return int(f[4]) + int(f[5])
     return None
