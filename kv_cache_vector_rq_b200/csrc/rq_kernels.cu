@@ -8,22 +8,23 @@
 // sandwich R~ v R, drop the pad, multiply by the norm.
 //
 // B200 design (not the pages' one-thread-per-(vector, group) layout):
-//  * d = 128 rows go through `rq_row_kernel`: one thread owns one whole row and
-//    every warp is an independent pipeline over 32-row sub-tiles: its own TMA
-//    loads (128-byte swizzle, so a lane reading its own row hits 8 different
-//    banks per 16-byte phase), mbarriers, x_hat written back in place and
-//    stored by TMA, codes staged in shared memory and stored by one bulk copy.
-//    Warps whose rows arrive first compute and store first, so loads, math and
-//    stores of the warps of an SM overlap even when each warp has one sub-tile.
+//  * d = 128 rows (and d = 256 rows of 16-bit types) go through `rq_row_kernel`:
+//    one thread owns one whole row and every warp is an independent pipeline
+//    over 32-row sub-tiles: its own TMA loads (128-byte swizzle, so a lane
+//    reading its own row hits 8 different banks per 16-byte phase), mbarriers,
+//    x_hat written back in place and stored by TMA, codes staged in shared
+//    memory and stored by one bulk copy. Large d = 128 launches stream each
+//    warp's sub-tiles through a ring of three half-tile boxes (see Shape).
 //  * The sandwich is applied as its exact 3x3 matrix (9 FMA per group instead
 //    of the 48-FMA sparse product the README counts): the matrix is built once
 //    per CTA from the rotors.
 //  * Quantization compares |y| with the positive Lloyd-Max boundaries scaled by
 //    the row norm (so x is never divided by its norm), exploiting the exact
 //    symmetry of the codebook.
-//  * Any other d (and unaligned rows) go through `rq_general_kernel`: one warp
-//    per row, groups strided over lanes, codes assembled per warp in shared
-//    memory.
+//  * Other d with 16-byte aligned rows go through `rq_wide_kernel` (rows
+//    streamed into shared memory by bulk copy, a warp per row); anything else
+//    through `rq_general_kernel`: one warp per row, groups strided over lanes,
+//    codes assembled per warp in shared memory.
 
 #include <cuda_runtime.h>
 
