@@ -173,6 +173,27 @@ def cpu_oracle_rate(n_sample, bits=HEADLINE_BITS, seed=0):
     return n_sample / dt, dt
 
 
+def max_over_ranks(v, world, dist=None, device=None):
+    """The largest of every rank's v (times: the slowest rank sets the step), by one all-reduce."""
+    if world == 1:
+        return v
+    import torch
+
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank, world, ms):
+    """Units per second over all ranks: every rank processes its own shard of units_per_rank (weak scaling)."""
+    return units_per_rank * world / (ms * 1e-3)
+
+
+def shard_seed(rank):
+    """Seed of a rank's input shard: ranks draw different vectors."""
+    return 1000 + rank
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -517,15 +538,11 @@ def main():
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def ranks_max(v):
+        return max_over_ranks(v, world, dist, dev)
 
     # ---------------------------------------------------------------- inputs and parameters
-    x = synth.lognormal(N_VEC, D, seed=1000 + rank, dtype=torch.float16, device=dev)
+    x = synth.lognormal(N_VEC, D, seed=shard_seed(rank), dtype=torch.float16, device=dev)
     rot = torch.from_numpy(kvrq.rq_rotors_init(D, 1).astype(np.float32)).to(dev)
     cbs = {b: torch.from_numpy(kvrq.tq_codebook_init(D, b)[0].astype(np.float32)).to(dev) for b in BITS}
     W = {b: kvrq.packed_words(3 * kvrq.rq_groups(D), b) for b in BITS}
@@ -578,11 +595,11 @@ def main():
     wall = time.perf_counter() - t_wall
     kvrq.device_status()
 
-    leg_ms = {leg: max_over_ranks(sum(s.elapsed_time(e) for s, e in ev[leg]) / args.steps) for leg in legs}
+    leg_ms = {leg: ranks_max(sum(s.elapsed_time(e) for s, e in ev[leg]) / args.steps) for leg in legs}
     step_ms = sum(leg_ms.values())
     head = ("rq", HEADLINE_BITS)
     head_ms = leg_ms[head]
-    value = N_VEC * world / (head_ms * 1e-3) / 1e6
+    value = whole_job_rate(N_VEC, world, head_ms) / 1e6
 
     peak, peak_kind = measured_peaks()
     bpv = rq_bytes_per_vector(D, HEADLINE_BITS)
@@ -613,7 +630,7 @@ def main():
         e.synchronize()
         if i >= args.warmup:
             e2e_ms.append(s.elapsed_time(e))
-    e2e = max_over_ranks(sum(e2e_ms) / len(e2e_ms))
+    e2e = ranks_max(sum(e2e_ms) / len(e2e_ms))
     h2d = x_host.numel() * 2
     d2h = codes_h.numel() * 4 + norms_h.numel() * 4 + xhat_h.numel() * 2
 
@@ -636,7 +653,7 @@ def main():
             e.record(stream)
             ts.append((s, e))
         torch.cuda.synchronize()
-        lms = max_over_ranks(sum(s.elapsed_time(e) for s, e in ts) / len(ts))
+        lms = ranks_max(sum(s.elapsed_time(e) for s, e in ts) / len(ts))
         gbs = bpv * LARGE_ROWS / (lms * 1e-3) / 1e9
         large = {"rows": LARGE_ROWS, "ms": lms, "Mvec_s": LARGE_ROWS / (lms * 1e-3) / 1e6, "GB_s": gbs,
                  "frac_of_peak": gbs / peak, "frac_of_8TBs": gbs / 8000.0}
@@ -678,7 +695,7 @@ def main():
             "hbm_1gib": large,
             "decode_c4": decode,
             "kv_stack_c3": stack,
-            "e2e": {"value": N_VEC * world / (e2e * 1e-3) / 1e6, "unit": "Mvec/s", "h2d_bytes_per_step": h2d,
+            "e2e": {"value": whole_job_rate(N_VEC, world, e2e) / 1e6, "unit": "Mvec/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms": e2e},
             "gpu_launches": launches,
             "clocks": clk.summary(),
