@@ -160,17 +160,39 @@ class ClockSampler:
 
 
 def cpu_oracle_rate(n_sample, bits=HEADLINE_BITS, seed=0):
-    """Vectors/s of the oracle's RQ roundtrip on the host (bounded sample)."""
+    """Vectors/s of the oracle's RQ roundtrip on one host core (bounded sample; numpy's BLAS held to one
+    thread, so that one core is what it uses)."""
+    from threadpoolctl import threadpool_limits
+
     from kv_cache_vector_rq_b200 import synth
     from oracle import codebook, params, rq
 
     x = synth.lognormal(n_sample, D, seed=seed).float().numpy().astype(np.float64)
     rot = params.rotors(D, 1)
     c, _, _ = codebook.lloyd_max(D, bits)
-    t0 = time.perf_counter()
-    rq.roundtrip(x, rot, c, bits)
-    dt = time.perf_counter() - t0
+    with threadpool_limits(1):
+        t0 = time.perf_counter()
+        rq.roundtrip(x, rot, c, bits)
+        dt = time.perf_counter() - t0
     return n_sample / dt, dt
+
+
+def _oracle_worker(job):
+    n, seed = job
+    return cpu_oracle_rate(n, seed=seed)[1]
+
+
+def cpu_oracle_all_cores(n_per_worker, max_workers=32):
+    """(vectors/s, workers): the same oracle on every host core at once, one single-threaded worker per core
+    (a spawn pool: a forked child of a process that holds a CUDA context would hang), each on its own rows.
+    The rate is all rows over the slowest worker's oracle time."""
+    import multiprocessing
+
+    workers = max(1, min(max_workers, len(os.sched_getaffinity(0))))
+    with multiprocessing.get_context("spawn").Pool(workers) as pool:
+        pool.map(_oracle_worker, [(32, 100 + i) for i in range(workers)])  # imports and set-up
+        dts = pool.map(_oracle_worker, [(n_per_worker, 200 + i) for i in range(workers)])
+    return workers * n_per_worker / max(dts), workers
 
 
 def max_over_ranks(v, world, dist=None, device=None):
@@ -675,6 +697,10 @@ def main():
         cpu = {"value": rate / 1e6, "unit": "Mvec/s", "cores": 1, "kind": "oracle",
                "sample": "%d rows of the workload, RotorQuant 3-bit roundtrip, float64 numpy oracle (%.1f s)" % (
                    n_s, dt)}
+        per_w = int(min(8192, max(256, rate * 4)))
+        rate_all, workers = cpu_oracle_all_cores(per_w)
+        cpu["all_cores"] = {"value": rate_all / 1e6, "unit": "Mvec/s", "cores": workers,
+                            "sample": "%d rows per worker, one single-threaded oracle per core" % per_w}
 
     if rank == 0:
         line = {
