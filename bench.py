@@ -692,7 +692,7 @@ def main():
     cpu = None
     if rank == 0:
         rate, dt = cpu_oracle_rate(1024)
-        n_s = int(min(16384, max(1024, rate * 10)))
+        n_s = int(min(N_VEC, max(1024, rate * 10)))  # about 10 s of work, at most the whole workload
         rate, dt = cpu_oracle_rate(n_s)
         cpu = {"value": rate / 1e6, "unit": "Mvec/s", "cores": 1, "kind": "oracle",
                "sample": "%d rows of the workload, RotorQuant 3-bit roundtrip, float64 numpy oracle (%.1f s)" % (
