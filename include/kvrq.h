@@ -133,7 +133,9 @@ kvrq_status kvrq_normals(uint64_t seed, int64_t first, int64_t count, double* ou
  *   codes   [n][ldc] uint32 device, ldc >= kvrq_packed_words(3G, bits).
  *   norms   [n] fp32 device (||x||, 0 for a zero row).
  *   xhat    [n][ldo] device, dtype of x (dequantize: odtype).
- *   1 <= bits <= 4, d >= 2. Fast path: d = 128 with 16-byte aligned rows.
+ *   1 <= bits <= 4, d >= 2. Fast paths: d = 128 (and d = 256 for fp16/bf16) with 16-byte
+ *   aligned rows, one thread per row; other d with 16-byte aligned rows stream whole rows
+ *   through shared memory, a warp per row.
  */
 kvrq_status rq_quantize(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,
                         const float* rotors, const float* centroids, int bits, uint32_t* codes,
