@@ -314,6 +314,67 @@ def decode_step_c4(kvrq, synth, torch, dev, batch, steps, warmup, layers=36, kv_
     return out
 
 
+def decode_attention_c4(kvrq, synth, torch, dev, batch, steps, warmup, layers=36, kv_heads=2, group=8,
+                        cached=131072):
+    """Qwen2.5-3B-shaped decode attention: for every (layer, batch, KV head), the 8 query heads
+    of its group attend over cached + 1 tokens of a packed cache (keys TurboQuant-prod 3-bit,
+    values RotorQuant 3-bit), softmax(q k_hat / sqrt(d)) v_hat straight from the codes. The
+    cache is 4x L2 or more, so every call streams it from HBM."""
+    heads = layers * kv_heads * batch
+    t_max = cached + 1
+    pi = torch.from_numpy(kvrq.tq_rotation_init(D, 2)).to(torch.float16).to(dev)
+    T = torch.from_numpy(kvrq.qjl_matrix_init(D, D, 3)).to(torch.float16).to(dev)
+    rot = torch.from_numpy(kvrq.rq_rotors_init(D, 1).astype(np.float32)).to(dev)
+    ck = torch.from_numpy(kvrq.tq_codebook_init(D, 2)[0].astype(np.float32)).to(dev)
+    cv = torch.from_numpy(kvrq.tq_codebook_init(D, 3)[0].astype(np.float32)).to(dev)
+    Wk, Wv = kvrq.packed_words(D, 2), kvrq.packed_words(129, 3)
+    k_codes = torch.empty((heads, t_max, Wk), dtype=torch.int32, device=dev)
+    k_signs = torch.empty((heads, t_max, D // 32), dtype=torch.int32, device=dev)
+    k_norms = torch.empty((heads, t_max), dtype=torch.float32, device=dev)
+    k_gam = torch.empty((heads, t_max), dtype=torch.float32, device=dev)
+    v_codes = torch.empty((heads, t_max, Wv), dtype=torch.int32, device=dev)
+    v_norms = torch.empty((heads, t_max), dtype=torch.float32, device=dev)
+    chunk = max(1, (1 << 22) // t_max)
+    for h0 in range(0, heads, chunk):  # prefill (untimed)
+        h1 = min(heads, h0 + chunk)
+        rows = (h1 - h0) * t_max
+        kx = synth.lognormal(rows, D, seed=5000 + h0, dtype=torch.float16, device=dev)
+        kvrq.tq_quantize_prod(kx, pi, T, ck, 3, codes=k_codes[h0:h1].view(rows, Wk),
+                              norms=k_norms[h0:h1].reshape(rows), signs=k_signs[h0:h1].view(rows, D // 32),
+                              gammas=k_gam[h0:h1].reshape(rows))
+        vx = synth.gaussian(rows, D, seed=7000 + h0, dtype=torch.float16, device=dev)
+        kvrq.rq_quantize(vx, rot, cv, 3, codes=v_codes[h0:h1].view(rows, Wv), norms=v_norms[h0:h1].reshape(rows))
+        del kx, vx
+    q = synth.gaussian(heads * group, D, seed=9, dtype=torch.float16, device=dev).view(heads, group, D)
+    out = torch.empty((heads, group, D), dtype=torch.float32, device=dev)
+    ws = torch.empty(kvrq.attention_workspace_bytes(heads, group, t_max) // 4 + 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    fn = lambda: kvrq.kv_attention_packed(kvrq.TQ_PROD, q, k_codes, k_norms, 3, v_codes, v_norms, 3, t_max, ck, rot,
+                                          cv, pi=pi, T=T, k_signs=k_signs, k_gammas=k_gam, out=out, workspace=ws,
+                                          stream=stream)
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(steps):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        fn()
+        e.record(stream)
+        e.synchronize()
+        ts.append(s.elapsed_time(e))
+    kvrq.device_status()
+    ms = sum(ts) / len(ts)
+    tokens = heads * t_max
+    cache_bytes = tokens * (4 * Wk + 4 * (D // 32) + 8 + 4 * Wv + 4)  # keys 56 B + values 56 B per token
+    res = {"batch": batch, "layers": layers, "kv_heads": kv_heads, "query_heads_per_kv": group, "tokens": t_max,
+           "ms_per_call": ms, "tokens_per_s": tokens / (ms * 1e-3), "cache_bytes": cache_bytes,
+           "cache_GB_s": cache_bytes / (ms * 1e-3) / 1e9, "launches_per_call": 3}
+    del k_codes, k_signs, k_norms, k_gam, v_codes, v_norms, ws
+    torch.cuda.empty_cache()
+    return res
+
+
 def kv_stack_c3(kvrq, synth, torch, dev, steps, layers=32, kv_heads=8, tokens=32768):
     """Llama-3.1-8B-shaped KV stack: keys from a rank-16 factor model with 4 outlier channels,
     values N(0,1), both bf16 [layers][KV heads][tokens][128]; keys compressed with TurboQuant-prod
@@ -419,6 +480,25 @@ def run_leg_only(args):
             calls["dqp"] = lambda: kvrq.tq_dequantize(codes, norms, D_, pi, cb, b, signs=signs, gammas=gam, T=T,
                                                       xhat=xh, workspace=ws)
     return time_fn(calls[mode], rows, args, torch, kvrq)
+
+
+def run_attention(args):
+    """Decode attention at batch 1 and 16 (the packed caches of 151M tokens at batch 16 take
+    about 17 GB); one JSON line with the per-call time and the cache bytes streamed per second."""
+    import torch
+
+    import kv_cache_vector_rq_b200 as kvrq
+    from kv_cache_vector_rq_b200 import synth
+
+    dev = torch.device("cuda", 0)
+    peak, kind = measured_peaks()
+    res = {"leg": "decode_attention_c4", "timing": "CUDA events, cache >= 4x L2", "hbm_peak_gbs": peak,
+           "peak_kind": kind}
+    for b in (1, 16):
+        r = decode_attention_c4(kvrq, synth, torch, dev, b, args.steps, args.warmup)
+        r["frac_of_hbm_peak"] = r["cache_GB_s"] / peak
+        res["batch%d" % b] = r
+    print(json.dumps(res), flush=True)
 
 
 def run_dim_sweep(args):
@@ -527,6 +607,9 @@ def main():
     ap.add_argument("--c5", action="store_true",
                     help="dimension sweep at 1 GiB fp16 input: d in {128, 256, 1536, 4096}, b in {2, 3, 4}, "
                          "RotorQuant roundtrip vs TurboQuant-prod quantize + dequantize; one JSON line")
+    ap.add_argument("--attn", action="store_true",
+                    help="decode attention from the packed cache at the Qwen2.5-3B decode shape (batch 1 and 16); "
+                         "one JSON line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -541,6 +624,9 @@ def main():
         return
     if args.c5:
         run_dim_sweep(args)
+        return
+    if args.attn:
+        run_attention(args)
         return
 
     import torch

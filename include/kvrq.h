@@ -275,6 +275,46 @@ kvrq_status kv_cache_append(void* stream, kvrq_method method, const void* x, kvr
                             const float* centroids, uint32_t* codes, int64_t codes_row_stride, uint32_t* signs,
                             int64_t signs_row_stride, float* norms, float* gammas, int64_t norm_row_stride);
 
+/* ================================================================ decode attention from packed keys and values
+ * ["TurboQuant и PolarQuant: математика квантизации KV-кэша в LLM", "Проблема
+ * KV-кэша в трансформерах": attention is softmax(q K^T / sqrt(d)) V; "TurboQuant +
+ * RotorQuant", "When to Use Which": for speed, attention is computed from the
+ * compressed indices instead of a decompressed cache]
+ *   out[h][g] = sum_t softmax_t(scale * <q_(h,g), k_hat_t>) * v_hat_t
+ * for every query row (h, g) over the first n_tokens tokens of KV head h. k_hat:
+ * keys dequantized by k_method (the logits are the scores of kv_score_packed);
+ * v_hat: RotorQuant-dequantized values. Nothing is dequantized into memory.
+ *   q: [n_heads][group][ldq] of qdtype, as for kv_score_packed.
+ *   keys: k_codes + h*k_head_stride + t*ldk (words), k_signs + h*s_head_stride +
+ *     t*lds (prod), k_norms/k_gammas + h*tok_head_stride + t; parameters k_rotors
+ *     (RotorQuant keys, [43][4]) or pi (pi_dtype fp16/bf16) and T (prod, [m][d]
+ *     fp16); k_bits = the key quantizer's total bits (prod stores k_bits - 1);
+ *     k_centroids: the stored key codes' codebook.
+ *   values: RotorQuant codes v_codes + h*v_head_stride + t*ldv (3G = 129 codes of
+ *     v_bits each per row), v_norms + h*tok_head_stride + t, v_rotors [43][4],
+ *     v_centroids [2^v_bits].
+ *   scale: multiplies the logits (1/sqrt(d) for standard attention).
+ *   out: [(h*group + g)*ldo + i], i < d, of odtype.
+ *   workspace: device memory owned by the caller, at least
+ *     kvrq_attention_workspace_bytes(n_heads, group, n_tokens) bytes, 16-byte
+ *     aligned, overwritten; calls sharing it must be ordered on one stream.
+ * d = 128 (m = d); group in 1..16; k_bits 1..4 (prod 2..4); v_bits 1..4;
+ * n_heads <= 65535. n_heads = 0 is a no-op; n_tokens = 0 with n_heads > 0 is
+ * KVRQ_EINVAL (a softmax over no tokens is undefined). fp32 arithmetic on the
+ * CUDA cores; three launches (query rotation, per-chunk online softmax and value
+ * sums, chunk merge with one inverse sandwich per query row). */
+size_t kvrq_attention_workspace_bytes(int64_t n_heads, int group, int64_t n_tokens);
+
+kvrq_status kv_attention_packed(void* stream, kvrq_method k_method, const void* q, kvrq_dtype qdtype, int64_t ldq,
+                                int64_t n_heads, int group, int d, float scale, int k_bits, int m,
+                                const uint32_t* k_codes, int64_t ldk, int64_t k_head_stride, const uint32_t* k_signs,
+                                int64_t lds, int64_t s_head_stride, const float* k_norms, const float* k_gammas,
+                                const float* k_rotors, const void* pi, kvrq_dtype pi_dtype, const uint16_t* T,
+                                const float* k_centroids, const uint32_t* v_codes, int64_t ldv, int64_t v_head_stride,
+                                const float* v_norms, int v_bits, const float* v_rotors, const float* v_centroids,
+                                int64_t tok_head_stride, int64_t n_tokens, void* out, kvrq_dtype odtype, int64_t ldo,
+                                void* workspace, size_t workspace_bytes);
+
 #ifdef __cplusplus
 }
 #endif

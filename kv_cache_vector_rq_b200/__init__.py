@@ -399,3 +399,57 @@ def kv_cache_append(method, x, slot, bits, centroids, codes, norms, rotors=None,
         _stream(stream), method, xp, _dtype_code(x), rows, d, ldx, bits, _ptr(rotors, "rotors", torch.float32),
         _ptr(pi, "pi"), _ptr(T, "T", torch.float16), m, _ptr(centroids, "centroids", torch.float32), cp,
         codes.stride(0), sp, signs.stride(0) if signs is not None else 0, np_, gp, norms.stride(0)))
+
+
+def attention_workspace_bytes(n_heads, group, n_tokens):
+    return int(lib().kvrq_attention_workspace_bytes(n_heads, group, n_tokens))
+
+
+def kv_attention_packed(k_method, q, k_codes, k_norms, k_bits, v_codes, v_norms, v_bits, n_tokens, k_centroids,
+                        v_rotors, v_centroids, scale=None, k_rotors=None, pi=None, T=None, k_signs=None,
+                        k_gammas=None, out=None, out_dtype=None, workspace=None, stream=None):
+    """Decode attention from a packed KV cache.
+
+    q: [n_heads, group, d] CUDA tensor. Keys as for kv_score_packed (k_codes [n_heads, T_max, Wk],
+    k_norms/k_gammas [n_heads, T_max], k_signs [n_heads, T_max, m/32]); values RotorQuant codes
+    v_codes [n_heads, T_max, Wv] with v_norms sharing the keys' norm layout. The first n_tokens
+    tokens of every head are attended. scale defaults to 1/sqrt(d). Returns out [n_heads, group, d]
+    (fp32 unless out_dtype is given)."""
+    torch = _torch()
+    n_heads, group, d = q.shape
+    if q.stride(2) != 1 or q.stride(1) != d or q.stride(0) != group * d:
+        raise ValueError("q must be contiguous")
+    if scale is None:
+        scale = 1.0 / float(np.sqrt(d))
+    if out is None:
+        out = torch.empty((n_heads, group, d), dtype=out_dtype or torch.float32, device=q.device)
+    if out.stride(2) != 1 or out.stride(1) != out.shape[2] or out.stride(0) != group * out.shape[2]:
+        raise ValueError("out must be contiguous")
+    m = T.shape[0] if T is not None else d
+    need = attention_workspace_bytes(n_heads, group, n_tokens)
+    if workspace is None:
+        workspace = torch.empty((max(need, 16) + 15) // 16 * 4, dtype=torch.float32, device=q.device)
+
+    def strides(t, name):
+        if t is None:
+            return None, 0, 0
+        if not t.is_cuda or t.stride(-1) != 1 or t.dim() != 3:
+            raise ValueError("%s must be a 3-D CUDA tensor with unit inner stride" % name)
+        return t.data_ptr(), t.stride(1), t.stride(0)
+
+    kp, ldk, khs = strides(k_codes, "k_codes")
+    sp, lds, shs = strides(k_signs, "k_signs")
+    vp, ldv, vhs = strides(v_codes, "v_codes")
+    if k_norms.stride(-1) != 1 or v_norms.stride() != k_norms.stride() or (
+            k_gammas is not None and k_gammas.stride() != k_norms.stride()):
+        raise ValueError("k_norms, k_gammas and v_norms must share one [n_heads, T_max] layout")
+    pdt = _dtype_code(pi) if pi is not None else F16
+    _lib.check("kv_attention_packed", lib().kv_attention_packed(
+        _stream(stream), k_method, q.data_ptr(), _dtype_code(q), d, n_heads, group, d, float(scale), k_bits, m, kp,
+        ldk, khs, sp, lds, shs, _ptr(k_norms, "k_norms", torch.float32), _ptr(k_gammas, "k_gammas", torch.float32),
+        _ptr(k_rotors, "k_rotors", torch.float32), _ptr(pi, "pi"), pdt, _ptr(T, "T", torch.float16),
+        _ptr(k_centroids, "k_centroids", torch.float32), vp, ldv, vhs, _ptr(v_norms, "v_norms", torch.float32),
+        v_bits, _ptr(v_rotors, "v_rotors", torch.float32), _ptr(v_centroids, "v_centroids", torch.float32),
+        k_norms.stride(0), n_tokens, out.data_ptr(), _dtype_code(out), d, _ptr(workspace, "workspace"),
+        workspace.numel() * workspace.element_size()))
+    return out

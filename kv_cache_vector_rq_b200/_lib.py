@@ -64,6 +64,15 @@ SIGNATURES = {
     # signs, signs_row_stride, norms, gammas, norm_row_stride
     "kv_cache_append": (c_int, [c_vp, c_int, c_vp, c_int, c_i64, c_int, c_i64, c_int, c_vp, c_vp, c_vp, c_int, c_vp,
                                 c_vp, c_i64, c_vp, c_i64, c_vp, c_vp, c_i64]),
+    # n_heads, group, n_tokens
+    "kvrq_attention_workspace_bytes": (ctypes.c_size_t, [c_i64, c_int, c_i64]),
+    # stream, k_method, q, qdtype, ldq, n_heads, group, d, scale, k_bits, m, k_codes, ldk, k_head_stride, k_signs,
+    # lds, s_head_stride, k_norms, k_gammas, k_rotors, pi, pi_dtype, T, k_centroids, v_codes, ldv, v_head_stride,
+    # v_norms, v_bits, v_rotors, v_centroids, tok_head_stride, n_tokens, out, odtype, ldo, workspace, workspace_bytes
+    "kv_attention_packed": (c_int, [c_vp, c_int, c_vp, c_int, c_i64, c_i64, c_int, c_int, ctypes.c_float, c_int, c_int,
+                                    c_vp, c_i64, c_i64, c_vp, c_i64, c_i64, c_vp, c_vp, c_vp, c_vp, c_int, c_vp, c_vp,
+                                    c_vp, c_i64, c_i64, c_vp, c_int, c_vp, c_vp, c_i64, c_i64, c_vp, c_int, c_i64, c_vp,
+                                    ctypes.c_size_t]),
 }
 
 _lib = None

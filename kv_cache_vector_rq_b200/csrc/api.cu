@@ -16,6 +16,7 @@
 #include "tq_launch.h"
 #include "tqg_launch.h"
 #include "score_launch.h"
+#include "attn_launch.h"
 
 namespace kvrq {
 
@@ -660,6 +661,106 @@ kvrq_status kv_score_packed(void* stream, kvrq_method method, const void* q, kvr
   a.status = di->status;
   const int nb = rows_needed <= 16 ? 16 : (rows_needed <= 32 ? 32 : 64);
   return launch_status(name, launch_score(method, nb, cbits, a, static_cast<cudaStream_t>(stream)));
+}
+
+size_t kvrq_attention_workspace_bytes(int64_t n_heads, int group, int64_t n_tokens) {
+  if (n_heads <= 0 || group <= 0 || n_tokens <= 0) return 0;
+  return attn_workspace_bytes(n_heads, group, n_tokens);
+}
+
+kvrq_status kv_attention_packed(void* stream, kvrq_method k_method, const void* q, kvrq_dtype qdtype, int64_t ldq,
+                                int64_t n_heads, int group, int d, float scale, int k_bits, int m,
+                                const uint32_t* k_codes, int64_t ldk, int64_t k_head_stride, const uint32_t* k_signs,
+                                int64_t lds, int64_t s_head_stride, const float* k_norms, const float* k_gammas,
+                                const float* k_rotors, const void* pi, kvrq_dtype pi_dtype, const uint16_t* T,
+                                const float* k_centroids, const uint32_t* v_codes, int64_t ldv, int64_t v_head_stride,
+                                const float* v_norms, int v_bits, const float* v_rotors, const float* v_centroids,
+                                int64_t tok_head_stride, int64_t n_tokens, void* out, kvrq_dtype odtype, int64_t ldo,
+                                void* workspace, size_t workspace_bytes) {
+  const char* name = "kv_attention_packed";
+  const bool prod = k_method == KVRQ_TQ_PROD;
+  if (k_method != KVRQ_RQ_MSE && k_method != KVRQ_TQ_MSE && !prod)
+    return set_error(KVRQ_EINVAL, "kv_attention_packed: unknown key method");
+  if (n_heads < 0 || n_tokens < 0 || group < 1) return set_error(KVRQ_EINVAL, "kv_attention_packed: bad sizes");
+  if (d != 128) return set_error(KVRQ_EUNSUPPORTED, "kv_attention_packed: d = 128 is supported");
+  if (group > 16) return set_error(KVRQ_EUNSUPPORTED, "kv_attention_packed: group must be <= 16");
+  if (prod && m != d) return set_error(KVRQ_EUNSUPPORTED, "kv_attention_packed: the QJL projection needs m = d");
+  const int kcb = prod ? k_bits - 1 : k_bits;
+  if (kcb < 1 || kcb > 4) return set_error(KVRQ_EUNSUPPORTED, "kv_attention_packed: stored key code width must be 1..4");
+  if (v_bits < 1 || v_bits > 4) return set_error(KVRQ_EUNSUPPORTED, "kv_attention_packed: v_bits must be 1..4");
+  if (!valid_dtype(qdtype) || ldq < d) return set_error(KVRQ_EINVAL, "kv_attention_packed: bad query dtype or ldq");
+  if (!valid_dtype(odtype) || ldo < d) return set_error(KVRQ_EINVAL, "kv_attention_packed: bad output dtype or ldo");
+  if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f)
+    return set_error(KVRQ_EINVAL, "kv_attention_packed: scale must be finite");
+  if (n_heads == 0) return KVRQ_OK;
+  if (n_tokens == 0) return set_error(KVRQ_EINVAL, "kv_attention_packed: no tokens (the softmax is undefined)");
+  if (n_heads > 65535) return set_error(KVRQ_EUNSUPPORTED, "kv_attention_packed: more than 65535 heads");
+  const int nck = k_method == KVRQ_RQ_MSE ? 3 * ((d + 2) / 3) : d;
+  const int64_t Wk = kvrq_packed_words(nck, kcb);
+  const int64_t Wv = kvrq_packed_words(3 * ((d + 2) / 3), v_bits);
+  if (!q || !k_codes || !k_norms || !k_centroids || !v_codes || !v_norms || !v_rotors || !v_centroids || !out)
+    return set_error(KVRQ_EINVAL, "kv_attention_packed: NULL argument");
+  if (ldk < Wk || k_head_stride < n_tokens * ldk || ldv < Wv || v_head_stride < n_tokens * ldv ||
+      tok_head_stride < n_tokens)
+    return set_error(KVRQ_EINVAL, "kv_attention_packed: strides too small");
+  if (k_method == KVRQ_RQ_MSE && (!k_rotors || !aligned(k_rotors, 16)))
+    return set_error(KVRQ_EINVAL, "kv_attention_packed: key rotors (16-byte aligned) required");
+  if (k_method != KVRQ_RQ_MSE && (!pi || (pi_dtype != KVRQ_F16 && pi_dtype != KVRQ_BF16) || !aligned(pi, 2)))
+    return set_error(KVRQ_EINVAL, "kv_attention_packed: pi (fp16 or bf16) required");
+  if (prod && (!k_signs || !k_gammas || !T || !aligned(T, 2) || lds < m / 32 || s_head_stride < n_tokens * lds))
+    return set_error(KVRQ_EINVAL, "kv_attention_packed: signs, gammas and T required for prod");
+  if (!aligned(v_rotors, 16)) return set_error(KVRQ_EINVAL, "kv_attention_packed: value rotors must be 16-byte aligned");
+  if (!aligned(k_codes, 4) || !aligned(v_codes, 4) || !aligned(k_norms, 4) || !aligned(v_norms, 4) ||
+      (prod && (!aligned(k_signs, 4) || !aligned(k_gammas, 4))) || !aligned(k_centroids, 4) ||
+      !aligned(v_centroids, 4) || !aligned(q, qdtype == KVRQ_F32 ? 4 : 2) || !aligned(out, odtype == KVRQ_F32 ? 4 : 2))
+    return set_error(KVRQ_EINVAL, "kv_attention_packed: misaligned pointer");
+  const size_t need = attn_workspace_bytes(n_heads, group, n_tokens);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 16))
+    return set_errorf(KVRQ_EINVAL, "kv_attention_packed: workspace of %zu bytes (16-byte aligned) required", need);
+
+  AttnArgs a{};
+  a.n_heads = n_heads;
+  a.group = group;
+  a.n_tokens = n_tokens;
+  a.tokens_per_cta = attn_tokens_per_cta(n_heads, n_tokens);
+  a.n_chunks = (int)((n_tokens + a.tokens_per_cta - 1) / a.tokens_per_cta);
+  a.q = q;
+  a.ldq = ldq;
+  a.q_f32 = qdtype == KVRQ_F32;
+  a.q_bf16 = qdtype == KVRQ_BF16;
+  a.scale = scale;
+  a.k_codes = k_codes;
+  a.ldk = ldk;
+  a.k_head_stride = k_head_stride;
+  a.k_signs = k_signs;
+  a.lds = lds;
+  a.s_head_stride = s_head_stride;
+  a.k_norms = k_norms;
+  a.k_gammas = k_gammas;
+  a.k_rotors = k_rotors;
+  a.pi = pi;
+  a.pi_bf16 = pi_dtype == KVRQ_BF16;
+  a.T = T;
+  a.k_centroids = k_centroids;
+  a.qjl_scale = (float)(1.2533141373155003 / (double)(prod ? m : d));
+  a.v_codes = v_codes;
+  a.ldv = ldv;
+  a.v_head_stride = v_head_stride;
+  a.v_norms = v_norms;
+  a.v_rotors = v_rotors;
+  a.v_centroids = v_centroids;
+  a.v_bits = v_bits;
+  a.tok_head_stride = tok_head_stride;
+  a.out = out;
+  a.ldo = ldo;
+  a.odtype = odtype;
+  const int64_t rows = n_heads * group;
+  float* ws = static_cast<float*>(workspace);
+  a.ws_q = ws;
+  a.ws_sq = ws + rows * kAttnQS;
+  a.ws_acc = a.ws_sq + rows * 128;
+  a.ws_ml = a.ws_acc + rows * a.n_chunks * kAttnAS;
+  return launch_status(name, launch_attention(k_method, kcb, a, static_cast<cudaStream_t>(stream)));
 }
 
 kvrq_status kv_cache_append(void* stream, kvrq_method method, const void* x, kvrq_dtype xdtype, int64_t n_rows,

@@ -187,3 +187,40 @@ def test_tq_validation_fails_before_any_launch():
     assert sk(ldr=200) == EINVAL
     assert sk(n=-1) == EINVAL
     assert sk(n=0) == 0
+
+
+def test_attention_workspace_and_validation_fail_before_any_launch():
+    lib = kvrq.lib()
+    EINVAL, EUNSUP = 1, 2
+    # rows x (132 rotated-query floats + 128 sketch floats + chunks x (132 sums + max + sum)) x 4 bytes
+    assert lib.kvrq_attention_workspace_bytes(1, 8, 1000) == 8 * 4 * (260 + 4 * 134)  # 4 chunks of 256 tokens
+    assert lib.kvrq_attention_workspace_bytes(72, 8, 131073) == 576 * 4 * (260 + 33 * 134)  # 4,096-token chunks
+    assert lib.kvrq_attention_workspace_bytes(1, 1, 1000000) == 4 * (260 + 977 * 134)  # at most 1,024 chunks
+    assert lib.kvrq_attention_workspace_bytes(0, 8, 100) == 0
+    wsb = lib.kvrq_attention_workspace_bytes(2, 8, 100)
+
+    def att(method=0, n_heads=2, group=8, d=128, scale=0.088, k_bits=3, m=128, ldk=13, ldv=13, n_tokens=100,
+            ws=P, wsb=wsb, kr=P, vr=P, pi=None, T=None, ks=None, kg=None, qdt=1, odt=0, tok=100):
+        return lib.kv_attention_packed(None, method, P, qdt, 128, n_heads, group, d, scale, k_bits, m, P, ldk,
+                                       ldk * 100, ks, 4, 400, P, kg, kr, pi, 1, T, P, P, ldv, ldv * 100, P, 3, vr, P,
+                                       tok, n_tokens, P, odt, 128, ws, wsb)
+
+    assert att(method=7) == EINVAL
+    assert att(d=64) == EUNSUP
+    assert att(group=17) == EUNSUP and att(group=0) == EINVAL
+    assert att(k_bits=5) == EUNSUP
+    assert att(method=2, k_bits=1, pi=P, T=P, ks=P, kg=P) == EUNSUP  # prod stores k_bits - 1 >= 1 bits
+    assert att(method=2, m=64, pi=P, T=P, ks=P, kg=P) == EUNSUP
+    assert att(qdt=9) == EINVAL and att(odt=9) == EINVAL
+    assert att(scale=float("nan")) == EINVAL
+    assert att(n_heads=0) == 0  # no-op
+    assert att(n_tokens=0) == EINVAL  # softmax over no tokens
+    assert att(ldk=12) == EINVAL  # 129 codes at 3 bits need 13 words
+    assert att(ldv=12) == EINVAL
+    assert att(tok=99) == EINVAL
+    assert att(kr=None) == EINVAL and att(kr=P + 4) == EINVAL
+    assert att(vr=P + 8) == EINVAL
+    assert att(method=1, ldk=12) == EINVAL  # TurboQuant keys need pi
+    assert att(method=2, ldk=8, pi=P, T=P) == EINVAL  # prod needs signs and gammas
+    assert att(ws=None) == EINVAL and att(wsb=wsb - 4) == EINVAL and att(ws=P + 4) == EINVAL
+    assert att(n_heads=70000, wsb=1 << 40) == EUNSUP
