@@ -27,6 +27,24 @@ def words_u32(t):
     return t.detach().to("cpu").numpy().astype(np.int64).astype(np.uint32)
 
 
+def device_words(words, device="cuda"):
+    """An oracle's uint32 code words uploaded as an int32 device tensor (same bits): the oracle's own
+    codes become the kernel's input, so that no oracle input ever comes from the CUDA path."""
+    a = np.ascontiguousarray(np.asarray(words, dtype=np.uint32))
+    return torch.from_numpy(a.view(np.int32)).to(device)
+
+
+def oracle_prod_inputs(ref, device="cuda"):
+    """The oracle's TurboQuant-prod result `ref` as device inputs of the library's dequantize or score
+    (codes, signs, gammas, norms; gammas and norms rounded to fp32 as the library stores them) and the
+    float64 values of those rounded gammas and norms, for the oracle's side of the comparison."""
+    g32 = np.asarray(ref["gammas"], dtype=np.float32)
+    n32 = np.asarray(ref["norms"], dtype=np.float32)
+    dev = (device_words(ref["words"], device), device_words(ref["signs_words"], device),
+           torch.from_numpy(g32).to(device), torch.from_numpy(n32).to(device))
+    return dev, g32.astype(np.float64), n32.astype(np.float64)
+
+
 def ulp(values, dtype):
     """Spacing of `dtype` at |values| (float64 array)."""
     a = np.abs(values)

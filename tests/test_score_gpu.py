@@ -90,11 +90,22 @@ def test_score_of_gpu_quantized_keys_equals_dot_with_dequantized():
     assert torch.all((s[0].double() - ref).abs() <= tol)
 
 
+def _random_words(g, shape, n_codes, bits):
+    """Uniformly random packed code rows (unused high bits of the last word zero)."""
+    W = -(-n_codes * bits // 32)
+    w = g.integers(0, 1 << 32, size=shape + (W,), dtype=np.uint64).astype(np.uint32)
+    spare = W * 32 - n_codes * bits
+    if spare:
+        w[..., -1] &= np.uint32((1 << (32 - spare)) - 1)
+    return w
+
+
 @pytest.mark.parametrize("method,bits", [("tq_prod", 3), ("tq_mse", 3), ("rq", 3), ("tq_prod", 4)])
 def test_scores_many_tiles_per_cta(method, bits):
     """160 KV heads x 8,000 tokens: each CTA walks about 21 tiles, so both decode warpgroups
-    cycle their code-stage rings and accumulators several times. Keys are quantized by the
-    library; three heads are checked against the oracle's direct scores of the same codes."""
+    cycle their code-stage rings and accumulators several times. Any code pattern is a valid
+    key, so the keys are seeded random codes, norms and gammas; three heads are checked
+    against the oracle's direct scores of the same codes."""
     n_heads, n_tok, group = 160, 8000, 8
     cb_bits = bits - 1 if method == "tq_prod" else bits
     c64 = codebook.lloyd_max(D, cb_bits)[0].astype(np.float32).astype(np.float64)
@@ -102,34 +113,32 @@ def test_scores_many_tiles_per_cta(method, bits):
     rot = torch.from_numpy(params.rotors(D, 1).astype(np.float32)).cuda()
     pi = torch.from_numpy(params.rotation(D, 2)).to(torch.float16).cuda()
     T = torch.from_numpy(params.qjl_matrix(D, D, 3)).to(torch.float16).cuda()
-    k = synth.lognormal(n_heads * n_tok, D, seed=11, dtype=torch.float16, device="cuda")
+    g = np.random.default_rng(11)
+    words = _random_words(g, (n_heads, n_tok), 129 if method == "rq" else D, cb_bits)
+    nrm = np.exp(0.5 * g.standard_normal((n_heads, n_tok))).astype(np.float32).astype(np.float64)
     kw = {}
     if method == "rq":
-        codes, norms = kvrq.rq_quantize(k, rot, c, bits)
         kw["rotors"] = rot
-    elif method == "tq_mse":
-        codes, norms = kvrq.tq_quantize_mse(k, pi, c, bits)
-        kw["pi"] = pi
     else:
-        codes, signs, gam, norms = kvrq.tq_quantize_prod(k, pi, T, c, bits)
-        kw.update(pi=pi, T=T, signs=signs.view(n_heads, n_tok, -1), gammas=gam.view(n_heads, n_tok))
-    del k
+        kw["pi"] = pi
+    if method == "tq_prod":
+        swords = _random_words(g, (n_heads, n_tok), D, 1)
+        gam = (0.3 * g.random((n_heads, n_tok))).astype(np.float32).astype(np.float64)
+        kw.update(T=T, signs=_dev_words(swords), gammas=torch.from_numpy(gam.astype(np.float32)).cuda())
     q = torch.randn((n_heads, group, D), generator=torch.Generator().manual_seed(5)).to(torch.float16)
     mth = {"rq": kvrq.RQ_MSE, "tq_mse": kvrq.TQ_MSE, "tq_prod": kvrq.TQ_PROD}[method]
-    s = kvrq.kv_score_packed(mth, q.cuda(), codes.view(n_heads, n_tok, -1), norms.view(n_heads, n_tok), bits,
+    s = kvrq.kv_score_packed(mth, q.cuda(), _dev_words(words), torch.from_numpy(nrm.astype(np.float32)).cuda(), bits,
                              n_tok, c, **kw)
     torch.cuda.synchronize()
     kvrq.device_status()
     p = {"centroids": c64, "rotors": rot.double().cpu().numpy(), "Pi": pi.double().cpu().numpy(),
          "T": T.double().cpu().numpy()}
-    words = codes.view(n_heads, n_tok, -1).cpu().numpy().astype(np.int64).astype(np.uint32)
-    nrm = norms.view(n_heads, n_tok).double().cpu().numpy()
     qf = q.double().numpy()
     for h in (0, 77, 159):
         kh = {"words": words[h:h + 1], "norms": nrm[h:h + 1]}
         if method == "tq_prod":
-            kh["signs_words"] = signs.view(n_heads, n_tok, -1)[h:h + 1].cpu().numpy().astype(np.int64).astype(np.uint32)
-            kh["gammas"] = gam.view(n_heads, n_tok)[h:h + 1].double().cpu().numpy()
+            kh["signs_words"] = swords[h:h + 1]
+            kh["gammas"] = gam[h:h + 1]
         ref = score.direct(method, qf[h], kh, p, bits)
         tol = 1e-3 * np.linalg.norm(qf[h], axis=1)[:, None] * nrm[h][None, :] + 1e-6
         err = np.abs(s[h].double().cpu().numpy() - ref)

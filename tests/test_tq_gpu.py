@@ -7,7 +7,7 @@ import torch
 import kv_cache_vector_rq_b200 as kvrq
 from kv_cache_vector_rq_b200 import synth
 from oracle import codebook, codes as ocodes, params, tq
-from tests.parity import compare_codes, compare_sketch_signs, near_boundary, to_f64, words_u32
+from tests.parity import compare_codes, compare_sketch_signs, near_boundary, oracle_prod_inputs, to_f64, words_u32
 
 pytestmark = pytest.mark.gpu
 
@@ -91,10 +91,11 @@ def test_prod_quantize_and_dequantize(dt, bits, n):
     assert np.allclose(g[~bad], ref["gammas"][~bad], rtol=1e-4, atol=1e-7)
     # signs: exact except where |T rho| is within the bound of the kernel's roundings
     compare_sketch_signs(words_u32(signs), ref, to_f64(x), pi64, T64, c64, skip_rows=bad)
-    # dequantize the GPU's own codes, against the oracle's reconstruction of them
-    xh = kvrq.tq_dequantize(codes, norms, D, pi_d, c_d, bits, signs=signs, gammas=gammas, T=T_d)
+    # dequantize the oracle's codes on the GPU, against the oracle's reconstruction of the same codes
+    (oc, osg, og, on), g64, n64 = oracle_prod_inputs(ref)
+    xh = kvrq.tq_dequantize(oc, on, D, pi_d, c_d, bits, signs=osg, gammas=og, T=T_d)
     torch.cuda.synchronize()
-    xref = tq.prod_dequantize(words_u32(codes), words_u32(signs), g, to_f64(norms), pi64, T64, c64, bits, D)
+    xref = tq.prod_dequantize(ref["words"], ref["signs_words"], g64, n64, pi64, T64, c64, bits, D)
     _rows_close(to_f64(xh), xref, XHAT_RTOL[dt])
 
 

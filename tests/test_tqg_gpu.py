@@ -10,7 +10,7 @@ import torch
 import kv_cache_vector_rq_b200 as kvrq
 from kv_cache_vector_rq_b200 import synth
 from oracle import codebook, codes as ocodes, params, tq
-from tests.parity import compare_codes, compare_sketch_signs, to_f64, words_u32
+from tests.parity import compare_codes, compare_sketch_signs, oracle_prod_inputs, to_f64, words_u32
 
 pytestmark = pytest.mark.gpu
 
@@ -134,11 +134,12 @@ def test_prod_quantize_and_dequantize_tiled(d, dt, bits, n, ws_rows):
         c1, s1, g1, n1 = kvrq.tq_quantize_prod(x, pi_d, T_d, c_d, bits)
         assert torch.equal(c1, codes) and torch.equal(s1, signs) and torch.equal(g1, gammas)
         assert torch.equal(n1, norms)
-    xh = kvrq.tq_dequantize(codes, norms, d, pi_d, c_d, bits, signs=signs, gammas=gammas, T=T_d, out_dtype=dt,
-                            workspace=ws)
+    # dequantize the oracle's codes on the GPU, against the oracle's reconstruction of the same codes
+    (oc, osg, og, on), g64, n64 = oracle_prod_inputs(ref)
+    xh = kvrq.tq_dequantize(oc, on, d, pi_d, c_d, bits, signs=osg, gammas=og, T=T_d, out_dtype=dt, workspace=ws)
     torch.cuda.synchronize()
     kvrq.device_status()
-    xref = tq.prod_dequantize(words_u32(codes), words_u32(signs), g, to_f64(norms), pi64, T64, c64, bits, d)
+    xref = tq.prod_dequantize(ref["words"], ref["signs_words"], g64, n64, pi64, T64, c64, bits, d)
     _rows_close(to_f64(xh), xref, XHAT_RTOL[dt])
 
 
