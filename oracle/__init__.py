@@ -18,8 +18,9 @@ definition at a time, with numpy (float64) doing the arithmetic. The pages are:
 * The summary page of arXiv 2504.19874 (TurboQuant), section "方法"
   (Algorithm 1 and Algorithm 2 described in prose).
 * "TurboQuant и PolarQuant: математика квантизации KV-кэша в LLM" -- the
-  paragraph on building codebooks with Lloyd's algorithm, and the attention
-  formula in "Проблема KV-кэша в трансформерах".
+  paragraph on building codebooks with Lloyd's algorithm, the attention
+  formula in "Проблема KV-кэша в трансформерах", and PolarQuant
+  ("Полярное преобразование", "Алгоритм PolarQuant на практике").
 
 Modules:
   rng       counter-based splitmix64 + Box-Muller normals (parameter draws)
@@ -31,9 +32,10 @@ Modules:
   tq        TurboQuant-mse, TurboQuant-prod (QJL on the residual)
   score     inner products <q, k_hat> from packed codes, two ways
   attention decode attention softmax(q K_hat^T scale) V_hat over a packed cache
+  polar     PolarQuant: preconditioning, recursive polar transform, angle codebooks
 
 Parity status of every function: pinned (see tests/test_oracle_*.py). No
 function here is "parity unpinned".
 """
 
-from . import rng, clifford, codebook, params, codes, rq, tq, score, attention  # noqa: F401
+from . import rng, clifford, codebook, params, codes, rq, tq, score, attention, polar  # noqa: F401
