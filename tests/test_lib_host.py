@@ -224,3 +224,50 @@ def test_attention_workspace_and_validation_fail_before_any_launch():
     assert att(method=2, ldk=8, pi=P, T=P) == EINVAL  # prod needs signs and gammas
     assert att(ws=None) == EINVAL and att(wsb=wsb - 4) == EINVAL and att(ws=P + 4) == EINVAL
     assert att(n_heads=70000, wsb=1 << 40) == EUNSUP
+
+
+def test_score_and_append_validation_fail_before_any_launch():
+    lib = kvrq.lib()
+    EINVAL, EUNSUP = 1, 2
+
+    def sc(method=0, n_heads=4, group=8, d=128, bits=3, m=128, ldc=13, chs=13 * 100, lds=4, shs=400, tok=100,
+           n_tokens=100, rot=P, pi=None, pdt=1, T=None, signs=None, gam=None, qdt=1, ldq=128, lsc=100, codes=P):
+        return lib.kv_score_packed(None, method, P, qdt, ldq, n_heads, group, d, bits, m, codes, ldc, chs, signs,
+                                   lds, shs, P, gam, tok, n_tokens, rot, pi, pdt, T, P, P, lsc)
+
+    assert sc(method=5) == EINVAL
+    assert sc(group=0) == EINVAL and sc(n_tokens=-1) == EINVAL
+    assert sc(d=256) == EUNSUP
+    assert sc(bits=5) == EUNSUP and sc(method=2, bits=1, pi=P, T=P, signs=P, gam=P, ldc=4) == EUNSUP
+    assert sc(group=65) == EUNSUP and sc(method=2, group=33, pi=P, T=P, signs=P, gam=P, ldc=8) == EUNSUP
+    assert sc(method=2, m=64, pi=P, T=P, signs=P, gam=P, ldc=8) == EUNSUP  # the sketch needs m = d
+    assert sc(qdt=4) == EINVAL and sc(ldq=100) == EINVAL
+    assert sc(n_heads=0) == 0 and sc(n_tokens=0) == 0  # no-ops
+    assert sc(codes=None) == EINVAL
+    assert sc(ldc=12) == EINVAL and sc(chs=1299) == EINVAL and sc(tok=99) == EINVAL and sc(lsc=99) == EINVAL
+    assert sc(rot=None) == EINVAL and sc(rot=P + 4) == EINVAL
+    assert sc(method=1, ldc=12) == EINVAL  # TurboQuant keys need pi
+    assert sc(method=1, ldc=12, pi=P, pdt=0) == EINVAL  # pi must be fp16 or bf16
+    assert sc(method=2, ldc=8, pi=P, T=P) == EINVAL  # prod needs signs and gammas
+    assert sc(method=2, ldc=8, pi=P, T=P, signs=P, gam=P, lds=3) == EINVAL
+    assert sc(n_heads=70000, chs=1300) == EUNSUP
+
+    def ap(method=0, n=8, d=128, ldx=128, bits=3, ldc=13, lnr=1, codes=P, rot=P):
+        return lib.kv_cache_append(None, method, P, 1, n, d, ldx, bits, rot, None, None, 128, P, codes, ldc, None, 0,
+                                   P, None, lnr)
+
+    assert ap(method=9) == EINVAL
+    assert ap(bits=5) == EUNSUP
+    assert ap(ldc=12) == EINVAL  # a code row of 129 codes at 3 bits needs 13 words
+    assert ap(lnr=0) == EINVAL
+    assert ap(rot=None) == EINVAL
+    assert ap(n=0) == 0
+
+    # the no-allocation prod quantize shares the prod checks and rejects a block that does not fit its array
+    def na(d=256, m=256, n=10, bits=3):
+        W = -(-d * (bits - 1) // 32)
+        return lib.tq_quantize_prod_noalloc(None, P, 1, n, d, d, P, P, m, P, bits, P, W, P, m // 32, P, P)
+
+    assert na(d=16384, m=16384) == EUNSUP
+    assert na(m=128) == EUNSUP
+    assert na(bits=6) == EUNSUP
