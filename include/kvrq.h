@@ -17,7 +17,8 @@
  *         "QJL 内积无偏估计（Theorem 2）", "简单复现 demo".
  *   [TQA] arXiv 2504.19874 summary page, section "方法" (Algorithms 1 and 2).
  *   [PQ]  "TurboQuant и PolarQuant: математика квантизации KV-кэша в LLM",
- *         paragraph on building codebooks with Lloyd's algorithm.
+ *         paragraph on building codebooks with Lloyd's algorithm; the
+ *         attention formula in "Проблема KV-кэша в трансформерах".
  *
  * Conventions shared by all calls
  * -------------------------------
@@ -31,7 +32,8 @@
  *    kvrq_packed_words(n_codes, b) words and unused high bits are zero.
  *  - QJL signs: bit j of a row is 1 for sign +1 and 0 for -1 (sign(0) = +1),
  *    m/32 words per row.
- *  - n == 0 is a no-op returning KVRQ_OK (after argument checks).
+ *  - n == 0 is a no-op returning KVRQ_OK (after argument checks); the one
+ *    exception is kv_attention_packed with no tokens (KVRQ_EINVAL).
  *  - Arguments are validated on the host before any launch; a bad argument
  *    returns KVRQ_EINVAL / KVRQ_EUNSUPPORTED and launches nothing. A failed
  *    launch returns KVRQ_ECUDA. kvrq_last_error_string() explains the last
