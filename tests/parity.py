@@ -45,6 +45,13 @@ def oracle_prod_inputs(ref, device="cuda"):
     return dev, g32.astype(np.float64), n32.astype(np.float64)
 
 
+def attention_tolerance(ref, vmax, rel=1e-3):
+    """Allowed |error| of decode-attention outputs ref [rows, d]: rel x the largest |output| of the row
+    (the fp32 path's relative bound) plus 1e-5 x max|v_hat| (the rounding of a weighted sum of thousands
+    of fp32 terms, about sqrt(T) 2^-24 max|v_hat|)."""
+    return rel * np.abs(ref).max(axis=1, keepdims=True) + 1e-5 * vmax
+
+
 def ulp(values, dtype):
     """Spacing of `dtype` at |values| (float64 array)."""
     a = np.abs(values)

@@ -16,6 +16,7 @@ import torch
 import kv_cache_vector_rq_b200 as kvrq
 from kv_cache_vector_rq_b200 import synth
 from oracle import attention, codebook, params, rq, tq
+from tests.parity import attention_tolerance
 
 pytestmark = pytest.mark.gpu
 
@@ -119,7 +120,7 @@ def _check(k_method, k_bits, v_bits, keys, kp, values, vp, q, n_tokens, scale, g
         vh = {kk: v[h:h + 1, :n_tokens] for kk, v in values.items()}
         ref = attention.decode(k_method, qf[h], kh, kp, k_bits, vh, vp, v_bits, scale)  # [group, d]
         vmax = np.abs(attention.values_hat(vh, vp, v_bits, D)).max()
-        tol = rel * np.abs(ref).max(axis=1, keepdims=True) + 1e-5 * vmax
+        tol = attention_tolerance(ref, vmax, rel)
         err = np.abs(got[h] - ref)
         assert np.all(err <= tol), "head %d: max excess %g (max err %g)" % (h, float((err - tol).max()), err.max())
 

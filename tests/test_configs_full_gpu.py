@@ -11,8 +11,8 @@ import torch
 import kv_cache_vector_rq_b200 as kvrq
 from kv_cache_vector_rq_b200 import synth
 from oracle import attention, codebook, codes as ocodes, params, rq, score, tq
-from tests.parity import (compare_codes, compare_floats, compare_sketch_signs, device_words, oracle_prod_inputs,
-                          to_f64, words_u32)
+from tests.parity import (attention_tolerance, compare_codes, compare_floats, compare_sketch_signs, device_words,
+                          oracle_prod_inputs, to_f64, words_u32)
 
 pytestmark = pytest.mark.gpu
 
@@ -191,7 +191,7 @@ def test_config4_qwen_decode_step_sampled():
         kh, vh = planted[h]
         ref = attention.decode("tq_prod", qf[h], kh, p, bits, vh, vp, bits, 1.0 / np.sqrt(D))
         vmax = np.abs(attention.values_hat(vh, vp, bits, D)).max()
-        tol = 1e-3 * np.abs(ref).max(axis=1, keepdims=True) + 1e-5 * vmax
+        tol = attention_tolerance(ref, vmax)
         err = np.abs(out[h].double().cpu().numpy() - ref)
         assert np.all(err <= tol), "attention head %d: max excess %g" % (h, float((err - tol).max()))
     # every full-size output is a convex combination of value reconstructions: bounded by the largest one
