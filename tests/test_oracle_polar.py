@@ -7,6 +7,8 @@ density, the page's normalising constant against an independent adaptive quadrat
 Carlo angles of Gaussian sub-vectors, and the page's statement that centroids lean towards
 pi/4."""
 
+import os
+
 import numpy as np
 import pytest
 from scipy import integrate
@@ -14,6 +16,7 @@ from scipy import integrate
 from oracle import params, polar
 
 D = 128
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
 
 def test_radii_are_block_norms_and_angles_their_ratios():
@@ -40,10 +43,19 @@ def test_radii_are_block_norms_and_angles_their_ratios():
     np.testing.assert_allclose(polar.inverse_polar(angles, radii), y, atol=1e-12)
 
 
-def test_worked_bit_count():
-    # 64 x 4 + 32 x 2 + 16 x 2 + 8 x 2 + 8 x 16 = 496 bits, 2048 / 496 = 4.13x
-    assert polar.bits_per_vector(D) == 496
-    assert round(2048 / polar.bits_per_vector(D), 2) == 4.13
+def test_worked_storage_example():
+    rows = [ln.split() for ln in open(os.path.join(GOLDEN, "polarquant_storage_example.txt"))
+            if ln.strip() and not ln.startswith("#")]
+    levels = [(int(a), int(b), int(c)) for a, b, c in (r for r in rows if r[0].isdigit())]
+    extra = {r[0]: r[1:] for r in rows if not r[0].isdigit()}
+    assert tuple(b for _, _, b in levels) == polar.LEVEL_BITS_D128
+    assert [n for _, n, _ in levels] == [D >> lv for lv, _, _ in levels]  # d / 2^l angles at level l
+    assert extra["radii"] == ["8", str(polar.RADIUS_BITS)]
+    assert polar.bits_per_vector(D) == int(extra["total"][0])
+    assert round(16 * D / polar.bits_per_vector(D), 2) == float(extra["ratio"][0])
+    # the oracle's packed words hold exactly the page's angle bits (whole words per level)
+    q = polar.quantize(np.random.default_rng(0).standard_normal((3, D)), params.rotation(D, 2), polar.codebooks())
+    assert [w.shape[1] * 32 for w in q["words"]] == [n * b for _, n, b in levels]
 
 
 @pytest.mark.parametrize("level", [2, 3, 4, 5, 8])
