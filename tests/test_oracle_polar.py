@@ -53,9 +53,9 @@ def test_worked_storage_example():
     assert extra["radii"] == ["8", str(polar.RADIUS_BITS)]
     assert polar.bits_per_vector(D) == int(extra["total"][0])
     assert round(16 * D / polar.bits_per_vector(D), 2) == float(extra["ratio"][0])
-    # the oracle's packed words hold exactly the page's angle bits (whole words per level)
+    # the oracle packs each level's angle bits into ceil(bits / 32) words
     q = polar.quantize(np.random.default_rng(0).standard_normal((3, D)), params.rotation(D, 2), polar.codebooks())
-    assert [w.shape[1] * 32 for w in q["words"]] == [n * b for _, n, b in levels]
+    assert [w.shape[1] for w in q["words"]] == [-(-n * b // 32) for _, n, b in levels]
 
 
 @pytest.mark.parametrize("level", [2, 3, 4, 5, 8])
