@@ -271,3 +271,13 @@ def test_score_and_append_validation_fail_before_any_launch():
     assert na(d=16384, m=16384) == EUNSUP
     assert na(m=128) == EUNSUP
     assert na(bits=6) == EUNSUP
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    # no fallback path: without libkvrq.so the binding refuses to load, and every call goes through it
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "libkvrq.so"))
+    with pytest.raises(ImportError, match="not built"):
+        kvrq.lib()
+    with pytest.raises(ImportError):
+        kvrq.packed_words(129, 3)
