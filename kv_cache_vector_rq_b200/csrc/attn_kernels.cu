@@ -17,11 +17,11 @@
 //  3. attn_combine_kernel: merges the chunks' (max, sum, accumulator) triples of a
 //     query row and applies the inverse sandwich once. x_hat is linear in the
 //     rotated codes, so sum_t w_t v_hat_t = M(R_g)^T (sum_t w_t ||v_t|| c_hat(v_t))
-//     group by group, and the d x 3 inverse rotation runs once per query row instead
-//     of once per token.
+//     group by group, and the 43 inverse 3x3 rotations run once per query row
+//     instead of once per token.
 //
-// The contraction runs on the CUDA cores in fp32 (exact products of fp32 q' with
-// fp32 centroids, fp32 sums).
+// Both contractions run on the CUDA cores in fp32 (fused multiply-adds of the fp32
+// rotated queries with the fp32 centroids; exp and the running sums in fp32).
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
