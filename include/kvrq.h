@@ -98,6 +98,20 @@ int kvrq_rq_groups(int d);
 kvrq_status tq_codebook_init(int d, int bits, double tol, int max_iter, double* centroids,
                              double* boundaries, int* iterations);
 
+/* PolarQuant angle codebook of one level ["TurboQuant и PolarQuant: математика
+ * квантизации KV-кэша в LLM", "Полярное преобразование", "Шаг 3: построение кодовых
+ * книг"]: level-1 angles (of coordinate pairs) are uniform on [0, 2 pi); an angle of
+ * level l >= 2 pairs the norms of two k = 2^(l-1)-dimensional sub-vectors and has
+ * density Gamma(k) / (2^(k-2) Gamma(k/2)^2) sin^(k-1)(2 theta) on [0, pi/2]
+ * (sin^2 theta ~ Beta(k/2, k/2)). Lloyd iteration as for tq_codebook_init, from an
+ * even grid; level >= 2 centroids are returned exactly symmetric about pi/4.
+ *   1 <= level <= 20, 1 <= bits <= 8, tol > 0, max_iter >= 1.
+ *   centroids: [2^bits] out, ascending. boundaries: [2^bits - 1] out (may be NULL).
+ *   iterations: out (may be NULL).
+ * Returns KVRQ_ENOCONV if not converged (outputs then hold the last iterate). */
+kvrq_status pq_angle_codebook_init(int level, int bits, double tol, int max_iter, double* centroids,
+                                   double* boundaries, int* iterations);
+
 /* G = ceil(d/3) random unit rotors (s, b12, b13, b23), row-major [G][4]
  * [RQ "How RotorQuant Works": R = [s,0,0,0,b12,b13,b23,0]]: 4 standard normals
  * per group from the counter-based stream `seed` (splitmix64 + Box-Muller, see

@@ -54,6 +54,17 @@ def tq_codebook_init(d, bits, tol=1e-13, max_iter=100000):
     return c, t
 
 
+def pq_angle_codebook_init(level, bits, tol=1e-13, max_iter=100000):
+    """PolarQuant angle centroids and boundaries (float64 numpy) of one polar-transform level."""
+    K = 1 << bits
+    c = np.zeros(K)
+    t = np.zeros(K - 1)
+    it = ctypes.c_int(0)
+    _lib.check("pq_angle_codebook_init",
+               lib().pq_angle_codebook_init(level, bits, tol, max_iter, _dptr(c), _dptr(t), ctypes.byref(it)))
+    return c, t
+
+
 def rq_rotors_init(d, seed):
     G = rq_groups(d)
     r = np.zeros((G, 4))

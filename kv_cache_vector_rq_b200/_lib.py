@@ -23,6 +23,7 @@ SIGNATURES = {
     "kvrq_packed_words": (c_i64, [c_i64, c_int]),
     "kvrq_rq_groups": (c_int, [c_int]),
     "tq_codebook_init": (c_int, [c_int, c_int, c_f64, c_int, c_dp, c_dp, c_ip]),
+    "pq_angle_codebook_init": (c_int, [c_int, c_int, c_f64, c_int, c_dp, c_dp, c_ip]),
     "rq_rotors_init": (c_int, [c_int, c_u64, c_dp]),
     "tq_rotation_init": (c_int, [c_int, c_u64, c_dp]),
     "qjl_matrix_init": (c_int, [c_int, c_int, c_u64, c_dp]),

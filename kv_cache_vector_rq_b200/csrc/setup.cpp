@@ -1,5 +1,6 @@
-// Host-side parameter setup (float64): random streams, Lloyd-Max codebook,
-// unit rotors, the random orthogonal rotation Pi and the QJL matrix.
+// Host-side parameter setup (float64): random streams, Lloyd-Max codebooks (the
+// coordinate codebook and the PolarQuant angle codebooks), unit rotors, the random
+// orthogonal rotation Pi and the QJL matrix.
 //
 // These run once, off the hot path ("pack_rotors_for_triton ... one-time,
 // ~0 cost" in "TurboQuant + RotorQuant", section "Usage"); the caller rounds
@@ -112,6 +113,38 @@ struct CoordDensity {
   }
 };
 
+// ---------------------------------------------------------------- PolarQuant angle density
+// ["TurboQuant и PolarQuant", "Полярное преобразование"]: an angle of level l >= 2
+// pairs the norms of two k = 2^(l-1)-dimensional Gaussian sub-vectors and has density
+// Gamma(k) / (2^(k-2) Gamma(k/2)^2) sin^(k-1)(2 theta) on [0, pi/2]. With
+// u = sin^2 theta this is u ~ Beta(k/2, k/2), so P(Theta <= t) = I_{sin^2 t}(k/2, k/2).
+// The first moment of a cell follows by parts: int_a^b t f = [t F]_a^b - int_a^b F,
+// the last integral by adaptive Simpson quadrature of the smooth, monotone F.
+struct AngleDensity {
+  double k;
+  explicit AngleDensity(int k_) : k(k_) {}
+  double cdf(double t) const {
+    if (t <= 0.0) return 0.0;
+    if (t >= 0.5 * M_PI) return 1.0;
+    const double s = std::sin(t);
+    return ibeta(s * s, 0.5 * k, 0.5 * k);
+  }
+  double simpson(double a, double b, double fa, double fm, double fb, double whole, double eps, int depth) const {
+    const double m = 0.5 * (a + b), lm = 0.5 * (a + m), rm = 0.5 * (m + b);
+    const double flm = cdf(lm), frm = cdf(rm);
+    const double left = (m - a) / 6.0 * (fa + 4.0 * flm + fm), right = (b - m) / 6.0 * (fm + 4.0 * frm + fb);
+    const double diff = left + right - whole;
+    if (depth <= 0 || std::fabs(diff) <= 15.0 * eps) return left + right + diff / 15.0;
+    const double e2 = std::max(0.5 * eps, 1e-18);  // below rounding, halving only forces depth
+    return simpson(a, m, fa, flm, fm, left, e2, depth - 1) + simpson(m, b, fm, frm, fb, right, e2, depth - 1);
+  }
+  double first_moment(double a, double b) const {  // int_a^b t f(t) dt
+    const double fa = cdf(a), fb = cdf(b), fm = cdf(0.5 * (a + b));
+    const double whole = (b - a) / 6.0 * (fa + 4.0 * fm + fb);
+    return b * fb - a * fa - simpson(a, b, fa, fm, fb, whole, 1e-15, 24);
+  }
+};
+
 }  // namespace kvrq
 
 using namespace kvrq;
@@ -173,6 +206,57 @@ kvrq_status tq_codebook_init(int d, int bits, double tol, int max_iter, double* 
     for (int k = 0; k + 1 < K; ++k) boundaries[k] = 0.5 * (s[k] + s[k + 1]);
   if (iterations) *iterations = it;
   if (!converged) return set_error(KVRQ_ENOCONV, "tq_codebook_init: Lloyd-Max did not converge");
+  return KVRQ_OK;
+}
+
+kvrq_status pq_angle_codebook_init(int level, int bits, double tol, int max_iter, double* centroids,
+                                   double* boundaries, int* iterations) {
+  if (level < 1 || level > 20) return set_error(KVRQ_EINVAL, "pq_angle_codebook_init: level must be in 1..20");
+  if (bits < 1 || bits > 8) return set_error(KVRQ_EINVAL, "pq_angle_codebook_init: bits must be in 1..8");
+  if (!(tol > 0.0) || max_iter < 1 || !centroids)
+    return set_error(KVRQ_EINVAL, "pq_angle_codebook_init: bad tol/max_iter/centroids");
+  const int K = 1 << bits;
+  std::vector<double> c(K);
+  int it = 0;
+  bool converged = false;
+  if (level == 1) {
+    // uniform on [0, 2 pi): the cells of an even grid are their own fixed point
+    for (int k = 0; k < K; ++k) c[k] = (2.0 * k + 1.0) * M_PI / K;
+    it = 1;
+    converged = true;
+  } else {
+    const AngleDensity f(1 << (level - 1));
+    const double hi_end = 0.5 * M_PI;
+    for (int k = 0; k < K; ++k) c[k] = (k + 0.5) * hi_end / K;  // even start; the fixed point is unique
+    std::vector<double> lo(K), hi(K);
+    while (it < max_iter) {
+      ++it;
+      for (int k = 0; k < K; ++k) {
+        lo[k] = k == 0 ? 0.0 : 0.5 * (c[k - 1] + c[k]);
+        hi[k] = k == K - 1 ? hi_end : 0.5 * (c[k] + c[k + 1]);
+      }
+      double delta = 0.0;
+      for (int k = 0; k < K; ++k) {
+        const double mass = f.cdf(hi[k]) - f.cdf(lo[k]);
+        const double cn = f.first_moment(lo[k], hi[k]) / mass;
+        delta = std::max(delta, std::fabs(cn - c[k]));
+        c[k] = cn;
+      }
+      if (delta < tol) {
+        converged = true;
+        break;
+      }
+    }
+    // the density is symmetric about pi/4: make c[k] + c[K-1-k] = pi/2 exact
+    std::vector<double> s(K);
+    for (int k = 0; k < K; ++k) s[k] = 0.5 * (c[k] + (hi_end - c[K - 1 - k]));
+    c = s;
+  }
+  for (int k = 0; k < K; ++k) centroids[k] = c[k];
+  if (boundaries)
+    for (int k = 0; k + 1 < K; ++k) boundaries[k] = 0.5 * (c[k] + c[k + 1]);
+  if (iterations) *iterations = it;
+  if (!converged) return set_error(KVRQ_ENOCONV, "pq_angle_codebook_init: Lloyd iteration did not converge");
   return KVRQ_OK;
 }
 

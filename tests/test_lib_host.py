@@ -281,3 +281,28 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
         kvrq.lib()
     with pytest.raises(ImportError):
         kvrq.packed_words(129, 3)
+
+
+@pytest.mark.parametrize("level,bits", [(1, 4), (2, 2), (3, 2), (4, 2), (2, 3), (3, 4)])
+def test_polar_angle_codebook_matches_oracle(level, bits):
+    from oracle import polar
+
+    c, t = kvrq.pq_angle_codebook_init(level, bits)
+    co, _ = polar.lloyd_max_angles(level, bits)
+    np.testing.assert_allclose(c, co, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(t, 0.5 * (c[:-1] + c[1:]), rtol=0, atol=0)
+    if level >= 2:
+        np.testing.assert_allclose(c + c[::-1], np.pi / 2, rtol=0, atol=1e-15)  # symmetric about pi/4
+
+
+def test_polar_angle_codebook_errors():
+    lib = kvrq.lib()
+    c = np.zeros(16)
+    it = ctypes.c_int(0)
+    dp = lambda a: a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+    assert lib.pq_angle_codebook_init(0, 2, 1e-13, 100, dp(c), None, None) == 1
+    assert lib.pq_angle_codebook_init(2, 9, 1e-13, 100, dp(c), None, None) == 1
+    assert lib.pq_angle_codebook_init(2, 2, 0.0, 100, dp(c), None, None) == 1
+    assert lib.pq_angle_codebook_init(2, 2, 1e-13, 100, None, None, None) == 1
+    assert lib.pq_angle_codebook_init(2, 2, 1e-13, 1, dp(c), None, ctypes.byref(it)) == 4  # KVRQ_ENOCONV
+    assert it.value == 1

@@ -71,6 +71,18 @@ def test_density_constant_against_adaptive_quadrature(level):
     assert mean == pytest.approx(np.pi / 4, abs=1e-12)  # E[Theta] = pi / 4
 
 
+@pytest.mark.parametrize("level", [2, 3, 4, 6])
+def test_angle_cdf_is_the_incomplete_beta(level):
+    # u = sin^2(theta) of the lemma's density is Beta(k/2, k/2): P(Theta <= t) = I_{sin^2 t}(k/2, k/2)
+    from scipy.special import betainc
+
+    k = polar.level_dim(level)
+    for t in (0.05, 0.3, 0.6, np.pi / 4, 1.0, 1.4):
+        cdf = integrate.quad(lambda u: float(polar.angle_density(u, level)), 0, t, epsabs=1e-15, epsrel=1e-13,
+                             limit=200)[0]
+        assert cdf == pytest.approx(betainc(k / 2, k / 2, np.sin(t) ** 2), abs=1e-12)
+
+
 @pytest.mark.parametrize("level", [2, 3, 4])
 def test_density_matches_gaussian_subvector_angles(level):
     k = polar.level_dim(level)
