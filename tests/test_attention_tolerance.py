@@ -1,7 +1,9 @@
 """The decode-attention parity rule on the CPU: a float32 restatement of the kernels' algorithm
 (logits from rotated queries, online softmax over 256-token chunks, value sums in the rotated
 domain, one inverse sandwich after the merge) passes it, and each plausible kernel mistake,
-planted in that restatement, fails it."""
+planted in that restatement, fails it. A restatement with the operands of a tensor-core version
+(fp16 rotated queries, T q', centroids and weights, fp32 sums, 128-token tiles) stays inside the
+1e-2 bound of the tensor-core paths."""
 
 import numpy as np
 import pytest
@@ -100,3 +102,51 @@ def test_planted_kernel_mistake_fails(case, mistake):
     q, keys, kp, values, vp, scale, ref, tol = case
     got = _f32_kernel(q, keys, kp, values, vp, scale, mistake=mistake)
     assert np.any(np.abs(got - ref) > tol), mistake
+
+
+def _fp16_operands(q, keys, kp, values, vp, scale, tile=128):
+    """The same algorithm with fp16 operands for both contractions (fp32 sums); the rotated pad
+    coordinate stays in fp32, as it would on the CUDA cores."""
+    H = np.float16
+    Hq, Hkv = q.shape[0], keys["words"].shape[0]
+    group = Hq // Hkv
+    n_tok = keys["words"].shape[1]
+    qjl = F(np.sqrt(np.pi / 2) / D)
+    out = np.zeros((Hq, D))
+    for h in range(Hq):
+        kv = h // group
+        qp = (kp["Pi"] @ q[h]).astype(F)
+        sq = (kp["T"] @ qp.astype(np.float64)).astype(F)
+        c = kp["centroids"][ocodes.unpack(keys["words"][kv], D, 2)].astype(H).astype(F)
+        s = (2 * ocodes.unpack(keys["signs_words"][kv], D, 1) - 1).astype(F)
+        dot = c @ qp.astype(H).astype(F) + qjl * keys["gammas"][kv].astype(F) * (s @ sq.astype(H).astype(F))
+        lg = (F(scale) * keys["norms"][kv].astype(F) * dot).astype(F)
+        cv = vp["centroids"][ocodes.unpack(values["words"][kv], 129, 3)].astype(F)
+        vn = values["norms"][kv].astype(F)
+        m, l, acc = -np.inf, F(0), np.zeros(129, F)
+        for t0 in range(0, n_tok, tile):
+            lt = lg[t0:t0 + tile]
+            mn = max(m, lt.max())
+            al = np.exp(F(m - mn)) if np.isfinite(m) else F(0)
+            p = np.exp(lt - mn).astype(F)
+            l = l * al + p.sum(dtype=F)
+            pw = (p * vn[t0:t0 + tile]).astype(F)
+            acc = acc * al
+            acc[:128] += pw.astype(H).astype(F) @ cv[t0:t0 + tile, :128].astype(H).astype(F)
+            acc[128] += pw @ cv[t0:t0 + tile, 128]
+            m = mn
+        out[h] = rq.unrotate((acc / l)[None].astype(np.float64), vp["rotors"], D)[0]
+    return out
+
+
+def test_fp16_operand_restatement_within_tensor_core_bound():
+    keys, kp, values, vp = _cache(2, 2000, seed=5)
+    q = np.random.default_rng(6).standard_normal((8, D)).astype(np.float16).astype(np.float64) * 2
+    scale = 1.0 / np.sqrt(D)
+    ref = attention.decode("tq_prod", q, keys, kp, 3, values, vp, 3, scale)
+    vmax = max(np.abs(attention.values_hat({kk: v[h:h + 1] for kk, v in values.items()}, vp, 3, D)).max()
+               for h in range(2))
+    got = _fp16_operands(q, keys, kp, values, vp, scale)
+    err = np.abs(got - ref)
+    assert np.all(err <= attention_tolerance(ref, vmax, rel=1e-2))
+    assert (err / np.abs(ref).max(axis=1, keepdims=True)).max() < 5e-3
