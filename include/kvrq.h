@@ -331,6 +331,36 @@ kvrq_status kv_attention_packed(void* stream, kvrq_method k_method, const void* 
                                 int64_t tok_head_stride, int64_t n_tokens, void* out, kvrq_dtype odtype, int64_t ldo,
                                 void* workspace, size_t workspace_bytes);
 
+/* ================================================================ paged cache bookkeeping (host)
+ * ["TurboQuant + RotorQuant", "Post-Prefill Quantization": the prefill cache is
+ * quantized in bulk once, then one new key/value per decode step.] A pool of
+ * n_pages pages of page_tokens token slots each, and per sequence the block table
+ * of the pages its tokens occupy in order: logical token t of a sequence is pool slot
+ * page_tokens * table[t / page_tokens] + t % page_tokens. The packed rows (codes,
+ * signs, norms, gammas) are caller-owned device arrays indexed by slot; these calls
+ * only keep the tables (host memory, no CUDA call, thread-safe per pool).
+ *   create: n_pages in 1..2^31-1, page_tokens >= 1; destroy(NULL) is a no-op.
+ *   add_seq: a new empty sequence; its id is never reused by this pool.
+ *   append: reserves n_tokens more slots at the end of the sequence (new pages from
+ *     the free list as needed); *first_token (may be NULL) = its previous length.
+ *     KVRQ_EINVAL and nothing reserved if the free pages do not suffice.
+ *   slots: slots[k] = pool slot of logical token first + k (all below the length).
+ *   block_table: the sequence's pages in order into pages[capacity] (KVRQ_EINVAL if
+ *     capacity is too small; *n_pages and *n_tokens, either may be NULL, are set
+ *     anyway).
+ *   free_seq: returns the sequence's pages to the free list and forgets the id.
+ * Unknown sequence ids and NULL pools return KVRQ_EINVAL. */
+typedef struct kvrq_pages kvrq_pages;
+kvrq_status kvrq_pages_create(int64_t n_pages, int page_tokens, kvrq_pages** out);
+void kvrq_pages_destroy(kvrq_pages* pages);
+kvrq_status kvrq_pages_add_seq(kvrq_pages* pages, int64_t* seq_id);
+kvrq_status kvrq_pages_append(kvrq_pages* pages, int64_t seq_id, int64_t n_tokens, int64_t* first_token);
+kvrq_status kvrq_pages_slots(kvrq_pages* pages, int64_t seq_id, int64_t first, int64_t count, int64_t* slots);
+kvrq_status kvrq_pages_block_table(kvrq_pages* pages, int64_t seq_id, int32_t* table, int64_t capacity,
+                                   int64_t* n_pages, int64_t* n_tokens);
+kvrq_status kvrq_pages_free_seq(kvrq_pages* pages, int64_t seq_id);
+kvrq_status kvrq_pages_stats(kvrq_pages* pages, int64_t* free_pages, int64_t* n_seqs);
+
 #ifdef __cplusplus
 }
 #endif

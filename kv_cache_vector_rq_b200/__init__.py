@@ -464,3 +464,60 @@ def kv_attention_packed(k_method, q, k_codes, k_norms, k_bits, v_codes, v_norms,
         k_norms.stride(0), n_tokens, out.data_ptr(), _dtype_code(out), d, _ptr(workspace, "workspace"),
         workspace.numel() * workspace.element_size()))
     return out
+
+
+class PagedCache:
+    """Host bookkeeping of a paged KV cache (kvrq_pages_* in include/kvrq.h): a pool of pages of
+    page_tokens slots and per sequence its block table. Slots index the caller's packed device rows."""
+
+    def __init__(self, n_pages, page_tokens):
+        h = ctypes.c_void_p()
+        _lib.check("kvrq_pages_create", lib().kvrq_pages_create(n_pages, page_tokens, ctypes.byref(h)))
+        self._h = h
+        self.page_tokens = page_tokens
+
+    def close(self):
+        h = getattr(self, "_h", None)
+        self._h = None
+        if h is not None and h.value and _lib is not None:
+            _lib.load().kvrq_pages_destroy(h)
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:  # interpreter shutdown: the library may already be gone
+            pass
+
+    def add_seq(self):
+        sid = ctypes.c_int64(0)
+        _lib.check("kvrq_pages_add_seq", lib().kvrq_pages_add_seq(self._h, ctypes.byref(sid)))
+        return sid.value
+
+    def append(self, seq, n_tokens):
+        """Reserves n_tokens slots at the end of the sequence; returns the first new logical token."""
+        first = ctypes.c_int64(0)
+        _lib.check("kvrq_pages_append", lib().kvrq_pages_append(self._h, seq, n_tokens, ctypes.byref(first)))
+        return first.value
+
+    def slots(self, seq, first, count):
+        out = np.zeros(count, dtype=np.int64)
+        _lib.check("kvrq_pages_slots", lib().kvrq_pages_slots(self._h, seq, first, count,
+                                                              out.ctypes.data_as(ctypes.c_void_p)))
+        return out
+
+    def block_table(self, seq):
+        n_pages, n_tokens = ctypes.c_int64(0), ctypes.c_int64(0)
+        lib().kvrq_pages_block_table(self._h, seq, None, 0, ctypes.byref(n_pages), ctypes.byref(n_tokens))
+        out = np.zeros(n_pages.value, dtype=np.int32)
+        _lib.check("kvrq_pages_block_table", lib().kvrq_pages_block_table(
+            self._h, seq, out.ctypes.data_as(ctypes.c_void_p), len(out), ctypes.byref(n_pages),
+            ctypes.byref(n_tokens)))
+        return out, n_tokens.value
+
+    def free_seq(self, seq):
+        _lib.check("kvrq_pages_free_seq", lib().kvrq_pages_free_seq(self._h, seq))
+
+    def stats(self):
+        fp, ns = ctypes.c_int64(0), ctypes.c_int64(0)
+        _lib.check("kvrq_pages_stats", lib().kvrq_pages_stats(self._h, ctypes.byref(fp), ctypes.byref(ns)))
+        return fp.value, ns.value

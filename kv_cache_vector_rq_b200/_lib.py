@@ -74,6 +74,14 @@ SIGNATURES = {
                                     c_vp, c_i64, c_i64, c_vp, c_i64, c_i64, c_vp, c_vp, c_vp, c_vp, c_int, c_vp, c_vp,
                                     c_vp, c_i64, c_i64, c_vp, c_int, c_vp, c_vp, c_i64, c_i64, c_vp, c_int, c_i64, c_vp,
                                     ctypes.c_size_t]),
+    "kvrq_pages_create": (c_int, [c_i64, c_int, ctypes.POINTER(c_vp)]),
+    "kvrq_pages_destroy": (None, [c_vp]),
+    "kvrq_pages_add_seq": (c_int, [c_vp, ctypes.POINTER(c_i64)]),
+    "kvrq_pages_append": (c_int, [c_vp, c_i64, c_i64, ctypes.POINTER(c_i64)]),
+    "kvrq_pages_slots": (c_int, [c_vp, c_i64, c_i64, c_i64, c_vp]),
+    "kvrq_pages_block_table": (c_int, [c_vp, c_i64, c_vp, c_i64, ctypes.POINTER(c_i64), ctypes.POINTER(c_i64)]),
+    "kvrq_pages_free_seq": (c_int, [c_vp, c_i64]),
+    "kvrq_pages_stats": (c_int, [c_vp, ctypes.POINTER(c_i64), ctypes.POINTER(c_i64)]),
 }
 
 _lib = None
