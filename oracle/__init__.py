@@ -33,9 +33,10 @@ Modules:
   score     inner products <q, k_hat> from packed codes, two ways
   attention decode attention softmax(q K_hat^T scale) V_hat over a packed cache
   polar     PolarQuant: preconditioning, recursive polar transform, angle codebooks
+  rq4       RotorQuant in the pages' four-grade layout (172 indices per vector)
 
 Parity status of every function: pinned (see tests/test_oracle_*.py). No
 function here is "parity unpinned".
 """
 
-from . import rng, clifford, codebook, params, codes, rq, tq, score, attention, polar  # noqa: F401
+from . import rng, clifford, codebook, params, codes, rq, tq, score, attention, polar, rq4  # noqa: F401
