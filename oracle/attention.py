@@ -56,3 +56,12 @@ def decode(k_method, q, keys, k_params, k_bits, values, v_params, v_bits, scale)
     for h in range(Hq):
         out[h] = w[h] @ v_hat[h // (Hq // Hkv)]
     return out
+
+
+def decode_paged(k_method, q, pool_keys, slots, k_params, k_bits, pool_values, v_params, v_bits, scale):
+    """decode() over a paged pool: token t of KV head h is pool row slots[h][t] of every array in
+    pool_keys / pool_values (each [pool_rows, ...]); the tokens are gathered in order, then
+    attended by the plain definition."""
+    keys = {kk: np.stack([np.asarray(v)[np.asarray(s)] for s in slots]) for kk, v in pool_keys.items()}
+    values = {kk: np.stack([np.asarray(v)[np.asarray(s)] for s in slots]) for kk, v in pool_values.items()}
+    return decode(k_method, q, keys, k_params, k_bits, values, v_params, v_bits, scale)

@@ -96,3 +96,30 @@ def test_softmax_shift_and_sum():
     np.testing.assert_allclose(p.sum(axis=-1), 1.0, rtol=0, atol=1e-15)
     np.testing.assert_allclose(attention.softmax(s + 1234.5), p, rtol=1e-12, atol=0)
     np.testing.assert_allclose(p[0], np.exp(s[0]) / np.exp(s[0]).sum(), rtol=1e-12, atol=0)
+
+
+def test_paged_pool_with_shuffled_pages_equals_the_contiguous_cache():
+    import kv_cache_vector_rq_b200 as kvrq
+
+    n_kv, group, n_tok, P = 2, 4, 45, 8
+    keys, kp, values, vp, _, _ = _cache("tq_prod", 3, 3, n_kv, n_tok, seed=7)
+    q = np.random.default_rng(8).standard_normal((n_kv * group, D))
+    ref = attention.decode("tq_prod", q, keys, kp, 3, values, vp, 3, 0.1)
+    # place each head's tokens through the page manager; interleave appends so pages alternate
+    pc = kvrq.PagedCache(32, P)
+    sids = [pc.add_seq() for _ in range(n_kv)]
+    for t0 in range(0, n_tok, 5):
+        for s in sids:
+            pc.append(s, min(5, n_tok - t0))
+    slots = [pc.slots(s, 0, n_tok) for s in sids]
+    rows = 32 * P
+    pool_k = {kk: np.zeros((rows,) + v.shape[2:], dtype=v.dtype) for kk, v in keys.items()}
+    pool_v = {kk: np.zeros((rows,) + v.shape[2:], dtype=v.dtype) for kk, v in values.items()}
+    for h in range(n_kv):
+        for kk in keys:
+            pool_k[kk][slots[h]] = keys[kk][h]
+        for kk in values:
+            pool_v[kk][slots[h]] = values[kk][h]
+    assert len(set(np.concatenate(slots).tolist())) == n_kv * n_tok  # disjoint slots
+    got = attention.decode_paged("tq_prod", q, pool_k, slots, kp, 3, pool_v, vp, 3, 0.1)
+    np.testing.assert_array_equal(got, ref)
