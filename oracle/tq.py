@@ -23,10 +23,8 @@ Readings where the pages leave a step open:
   with an orthogonal Pi this is exactly Pi r, ||r_rot|| = ||r|| and
   S r = T r_rot, so the stored gamma and signs are the pages' quantities.
   ``prod_quantize_literal`` writes the pages' form out for comparison.
-* ``sketch_operand='f16'`` projects 2^8 * r_rot rounded to IEEE half instead
-  of r_rot: the sign decision is then taken on the same operand values as on a
-  half-precision tensor-core path (the sign of T r is unchanged by the positive
-  scale, which only keeps the operand out of the half subnormal range).
+* The sign decision is taken on the float64 product T r_rot itself: no
+  rounding of any implementation's operands enters the oracle.
 """
 
 import numpy as np
@@ -58,13 +56,14 @@ def _sign_bits(p):
     return (p >= 0).astype(np.int64)
 
 
-def prod_quantize(x, Pi, T, centroids_mse, bits, sketch_operand=None):
+def prod_quantize(x, Pi, T, centroids_mse, bits):
     """Algorithm 2 quantize with b = ``bits`` total (b-1 MSE bits + 1 QJL bit).
 
     Returns dict(words (MSE codes, b-1 bits), codes, signs_words [N, m/32],
-    signs (+1/-1) [N, m], gammas [N], norms [N], y, z) where z[:, j] is the
-    sketch's decision value: the cosine between row j of T and the (possibly
-    rounded) residual direction."""
+    signs (+1/-1) [N, m], gammas [N], norms [N], y, r_rot [N, d], p [N, m],
+    z [N, m]) where p = T r_rot row by row (the sketch's decision value:
+    sign bit j is p[:, j] >= 0) and z[:, j] is the cosine between row j of T
+    and the residual."""
     n, u = split_norm(x)
     Pi = np.asarray(Pi, dtype=np.float64)
     T = np.asarray(T, dtype=np.float64)
@@ -73,17 +72,10 @@ def prod_quantize(x, Pi, T, centroids_mse, bits, sketch_operand=None):
     c_hat = np.asarray(centroids_mse, dtype=np.float64)[idx]
     r_rot = y - c_hat
     gamma = np.sqrt(np.sum(r_rot * r_rot, axis=1))
-    safe = np.where(gamma > 0, gamma, 1.0)
-    rho = np.where(gamma[:, None] > 0, r_rot / safe[:, None], 0.0)
-    if sketch_operand == "f16":
-        rho = (256.0 * r_rot).astype(np.float16).astype(np.float64)
-    elif sketch_operand is not None:
-        raise ValueError(sketch_operand)
-    p = rho @ T.T  # T r_rot / gamma, row by row
+    p = r_rot @ T.T  # T r_rot, row by row
     bits_s = _sign_bits(p)
     t_norm = np.linalg.norm(T, axis=1)
-    r_norm = np.linalg.norm(rho, axis=1)
-    z = p / (t_norm[None, :] * np.where(r_norm > 0, r_norm, 1.0)[:, None])
+    z = p / (t_norm[None, :] * np.where(gamma > 0, gamma, 1.0)[:, None])
     return {
         "words": codes_mod.pack(idx, bits - 1),
         "codes": idx,
@@ -92,6 +84,8 @@ def prod_quantize(x, Pi, T, centroids_mse, bits, sketch_operand=None):
         "gammas": gamma,
         "norms": n,
         "y": y,
+        "r_rot": r_rot,
+        "p": p,
         "z": z,
     }
 

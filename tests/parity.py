@@ -96,6 +96,7 @@ def compare_codes(gpu_words, oracle_q, n_codes, bits, centroids, decision=None, 
         assert not bad.any(), "codes differ away from a decision boundary at %s (gpu %s, oracle %s, y %s)" % (
             np.argwhere(bad)[:5].tolist(), g_codes[bad][:5], o_codes[bad][:5], np.asarray(y)[bad][:5])
         assert np.all(np.abs(g_codes[diff] - o_codes[diff]) == 1), "boundary mismatch to a non-adjacent code"
+    record("code boundary ties", int(diff.sum()), int(g_codes.size))
     return int(diff.sum()), diff.any(axis=1)
 
 
@@ -125,15 +126,17 @@ LAMBDA = 4.0
 
 
 def residual_sketch_slack(ref, x64, Pi64, T64, centroids):
-    """(p, bound): p[i, j] = (rho_i . T_j) with rho = fp16(256 r_rot) as the oracle forms it, and a bound on
-    |p| within which the CUDA path's sign of p may differ from the oracle's.
+    """(p, bound): p = T r_rot in float64 (the oracle's decision values, ref["p"]) and a bound on |p| within
+    which a CUDA path that projects fp16(2^8 r) with float32 arithmetic may take the other sign.
 
     The kernel forms y = Pi x with float32 sums of exact fp16 products, scales by 1/||x|| and subtracts the
     centroid, so each residual coordinate may differ from the float64 one by
     eps = LAMBDA sqrt(d) 2^-24 sum_k |Pi_ik u_k| + 2^-21 |y| + 2^-22 |c| (sums, then the norm, its
-    reciprocal, the fma and the centroid chain). A coordinate of 256 r_rot within 256 eps of an fp16
-    rounding midpoint may round to either neighbour, moving rho_k by one fp16 step; p_j then moves by at
-    most sum_k |T_jk| d_rho_k, and the sketch's own float32 sums add LAMBDA sqrt(d) 2^-24 sum_k |T_jk rho_k|."""
+    reciprocal, the fma and the centroid chain). The tensor-core operand is then 2^8 r rounded to fp16;
+    rounding is monotone, so it lies between fp16(2^8 (r - eps)) and fp16(2^8 (r + eps)), and the operand
+    differs from 2^8 r by at most the larger distance to those two ends (this is where the fp16 step of the
+    operand, at most 2^-11 relative per coordinate, enters). p_j then moves by at most sum_k |T_jk| times
+    that distance, and the sketch's own float32 sums add LAMBDA sqrt(d) 2^-24 sum_k |T_jk 2^8 r_k|."""
     x64 = np.asarray(x64, dtype=np.float64)
     Pi64 = np.asarray(Pi64, dtype=np.float64)
     T64 = np.asarray(T64, dtype=np.float64)
@@ -145,20 +148,25 @@ def residual_sketch_slack(ref, x64, Pi64, T64, centroids):
     s = 256.0 * (y - c_hat)
     g = LAMBDA * np.sqrt(d) * 2.0 ** -24
     eps = g * (np.abs(u) @ np.abs(Pi64).T) + 2.0 ** -21 * np.abs(y) + 2.0 ** -22 * np.abs(c_hat)
-    rho = s.astype(np.float16).astype(np.float64)
     lo = (s - 256.0 * eps).astype(np.float16).astype(np.float64)
     hi = (s + 256.0 * eps).astype(np.float16).astype(np.float64)
-    d_rho = np.maximum(np.abs(hi - rho), np.abs(lo - rho))
+    d_op = np.maximum(np.abs(hi - s), np.abs(lo - s))  # |operand - 2^8 r|, worst case
     aT = np.abs(T64).T
-    p = rho @ T64.T
-    bound = d_rho @ aT + g * (np.abs(rho) @ aT)
+    p = np.asarray(ref["p"], dtype=np.float64)
+    bound = (d_op @ aT + g * (np.abs(np.maximum(np.abs(lo), np.abs(hi))) @ aT)) / 256.0
     return p, bound
 
 
-def compare_sketch_signs(gpu_sign_words, ref, x64, Pi64, T64, centroids, skip_rows=None, max_frac=1e-4):
-    """QJL signs of TurboQuant-prod: equal to the oracle's except where |p| is within the arithmetic's bound
-    (residual_sketch_slack), and differing in at most max_frac of the signs compared (at least 8).
-    Returns the number of differing signs."""
+def compare_sketch_signs(gpu_sign_words, ref, x64, Pi64, T64, centroids, skip_rows=None, max_frac=2e-4,
+                         report=True):
+    """QJL signs of TurboQuant-prod against the plain definition sign(T r_rot) of the oracle: equal except
+    where |T r_rot| is within the arithmetic's bound (residual_sketch_slack), and differing in at most
+    max_frac of the signs compared (at least 8). Records and returns the number of differing signs.
+
+    Expected rate: the fp16 operand's rounding errors are independent and uniform within half a unit in
+    the last place, so p_j moves by about N(0, (0.21 2^-10 ||2^8 r||)^2) against p_j ~ N(0, ||2^8 r||^2);
+    a sign flips with probability E|dp| phi(0) / ||2^8 r|| ~ 6.4e-5. max_frac = 2e-4 keeps a sample of
+    10^5 signs about 5 standard deviations of the count away from a false failure."""
     T64 = np.asarray(T64, dtype=np.float64)
     m = T64.shape[0]
     gs = ocodes.unpack(np.asarray(gpu_sign_words, dtype=np.uint32), m, 1)
@@ -171,5 +179,90 @@ def compare_sketch_signs(gpu_sign_words, ref, x64, Pi64, T64, centroids, skip_ro
         assert not far.any(), "sign differs beyond the rounding bound at %s (p %s, bound %s)" % (
             np.argwhere(far)[:5].tolist(), p[far][:5], bound[far][:5])
     n = int(diff.sum())
-    assert n <= max(8, max_frac * keep.sum() * m), "%d of %d signs differ" % (n, keep.sum() * m)
+    total = int(keep.sum()) * m
+    if report:
+        record("qjl sign flips", n, total)
+    assert n <= max(8, max_frac * total), "%d of %d signs differ" % (n, total)
     return n
+
+
+# ---------------------------------------------------------------- scores
+
+SCORE_RTOL = 1e-3
+SCORE_SIGMAS = 6.0  # floor multiple of the fp16 roundings' spread (each at most 2^-11 relative)
+SCORE_F32_REL = 2.0 ** -14  # float32 arithmetic: rotation, T q', tensor-core accumulation, epilogue
+
+
+def score_tolerance(method, q, keys, params, bits):
+    """Allowed |error| [Hq, T] of packed-code scores against oracle.score.direct: SCORE_RTOL |score| plus
+    an absolute floor derived from the kernel's operands.
+
+    The kernel multiplies fp16(q') by fp16(c_hat) (and, for TurboQuant-prod, fp16(T q') by the +-1 signs)
+    with float32 accumulation, where q' is the rotated query. Per key, with n = ||k||, kappa = sqrt(pi/2)/m
+    and gamma the residual norm, the floor is
+      n |sum_i q'_i (fp16(c)_i - c_i)|      the centroid rounding, exact (one table of 2^b values)
+    + n 6 2^-11 ||q' o fp16(c)||_2          the query rounding: independent, each at most 2^-11 relative
+    + n kappa gamma 6 2^-11 ||T q'||_2      the rounding of T q'
+    + n 2^-14 (sum |q'_i c_i| + kappa gamma sum_j |(T q')_j|)   float32 sums (14 significant bits kept
+                                                               through the tensor-core accumulation).
+    Six times the bound of each independent rounding is about 7 standard deviations of their sum."""
+    from oracle import codes as oc, rq as orq, tq as otq
+    from oracle.params import n_groups
+    q = np.asarray(q, dtype=np.float64)
+    Hq, d = q.shape
+    words = np.asarray(keys["words"])
+    Hkv = words.shape[0]
+    c = np.asarray(params["centroids"], dtype=np.float64)
+    c16 = c.astype(np.float16).astype(np.float64)
+    u = 2.0 ** -11
+    out = np.zeros((Hq, words.shape[1]))
+    for h in range(Hq):
+        kv = h // (Hq // Hkv)
+        norms = np.asarray(keys["norms"], dtype=np.float64)[kv]
+        if method == "rq":
+            qp = orq.rotate(q[h:h + 1], params["rotors"])[0]
+            idx = oc.unpack(words[kv], 3 * n_groups(d), bits)
+        else:
+            qp = np.asarray(params["Pi"], dtype=np.float64) @ q[h]
+            idx = oc.unpack(words[kv], d, bits if method == "tq_mse" else bits - 1)
+        a16 = c16[idx] * qp
+        f = np.abs(a16.sum(axis=1) - (c[idx] * qp).sum(axis=1))
+        f += SCORE_SIGMAS * u * np.sqrt(np.sum(a16 * a16, axis=1))
+        f += SCORE_F32_REL * np.sum(np.abs(c[idx] * qp), axis=1)
+        if method == "tq_prod":
+            T = np.asarray(params["T"], dtype=np.float64)
+            tq_ = T @ qp
+            kg = (otq.QJL_SCALE_NUM / T.shape[0]) * np.asarray(keys["gammas"], dtype=np.float64)[kv]
+            f += kg * (SCORE_SIGMAS * u * np.linalg.norm(tq_) + SCORE_F32_REL * np.sum(np.abs(tq_)))
+        out[h] = norms * f
+    return out
+
+
+def compare_scores(got, ref, floor, rtol=SCORE_RTOL, name="scores", report=True):
+    """|got - ref| <= rtol |ref| + floor elementwise; records the worst relative error over the scores of
+    at least median magnitude (a score near zero has no relative accuracy from rounded operands), and the
+    largest error as a fraction of its tolerance. Returns that worst relative error."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    tol = rtol * np.abs(ref) + floor
+    err = np.abs(got - ref)
+    big = (np.abs(ref) >= np.median(np.abs(ref))) & (ref != 0)
+    worst_rel = float(np.max(err[big] / np.abs(ref[big]))) if big.any() else 0.0
+    if report:
+        record("scores worst rel err (|s| >= median)", worst_rel, int(big.sum()))
+        record("scores max err / tol", float(np.max(err / tol)) if err.size else 0.0, int(err.size))
+    assert np.all(err <= tol), "%s: max excess %g at %s (err/tol %g)" % (
+        name, float(np.max(err - tol)), np.unravel_index(np.argmax(err - tol), err.shape), float(np.max(err / tol)))
+    return worst_rel
+
+
+# ---------------------------------------------------------------- reporting
+
+REPORT = []
+
+
+def record(kind, value, total):
+    """Keeps a count (or worst value) of one comparison for the session summary printed by conftest."""
+    import os
+    test = os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
+    REPORT.append((test, kind, value, total))

@@ -11,8 +11,8 @@ import torch
 import kv_cache_vector_rq_b200 as kvrq
 from kv_cache_vector_rq_b200 import synth
 from oracle import attention, codebook, codes as ocodes, params, rq, score, tq
-from tests.parity import (attention_tolerance, compare_codes, compare_floats, compare_sketch_signs, device_words,
-                          oracle_prod_inputs, to_f64, words_u32)
+from tests.parity import (attention_tolerance, compare_codes, compare_floats, compare_scores, compare_sketch_signs,
+                          device_words, oracle_prod_inputs, score_tolerance, to_f64, words_u32)
 
 pytestmark = pytest.mark.gpu
 
@@ -44,7 +44,7 @@ def _normwise(gpu, ref, rtol, skip=None):
 
 
 def _check_prod(x_rows64, codes, signs, gammas, norms, pi64, T64, c64, bits, d):
-    ref = tq.prod_quantize(x_rows64, pi64, T64, c64, bits, sketch_operand="f16")
+    ref = tq.prod_quantize(x_rows64, pi64, T64, c64, bits)
     nb, bad = compare_codes(codes, ref, d, bits - 1, c64)
     assert np.allclose(norms, ref["norms"], rtol=1e-5)
     assert np.allclose(gammas[~bad], ref["gammas"][~bad], rtol=1e-4, atol=1e-7)
@@ -154,7 +154,7 @@ def test_config4_qwen_decode_step_sampled():
     planted = {}
     for h in checked:
         xk[h][-1], xv[h][-1] = to_f64(new_k[h]), to_f64(new_v[h])
-        refk = tq.prod_quantize(xk[h], pi64, T64, ck64, bits, sketch_operand="f16")
+        refk = tq.prod_quantize(xk[h], pi64, T64, ck64, bits)
         g64, n64 = _plant_prod(refk, (h, tt), k_codes, k_signs, k_gam, k_norms)
         rv = rq.quantize(xv[h], rot64, cv64, bits)
         vn32 = rv["norms"].astype(np.float32)
@@ -171,9 +171,8 @@ def test_config4_qwen_decode_step_sampled():
     for h in checked:
         kh = planted[h][0]
         ref = score.direct("tq_prod", qf[h], kh, p, bits)
-        tol = 1e-3 * np.linalg.norm(qf[h], axis=1)[:, None] * kh["norms"][0][None, :] + 1e-6
-        err = np.abs(s[h][:, toks].double().cpu().numpy() - ref)
-        assert np.all(err <= tol), "head %d: max excess %g" % (h, float((err - tol).max()))
+        compare_scores(s[h][:, toks].double().cpu().numpy(), ref, score_tolerance("tq_prod", qf[h], kh, p, bits),
+                       name="head %d" % h)
     del s
     # decode attention over the full cache; checked on the three heads restricted to the sampled slots,
     # where the attention over those slots alone is a second full-size-layout launch of the same kernels

@@ -229,18 +229,6 @@ def test_prod_zero_residual_and_sign_of_zero():
     assert np.array_equal(xh, x)
 
 
-def test_sketch_operand_rounding_changes_only_near_zero():
-    d, bits = 128, 3
-    x = _gauss(300, d, 21)
-    Pi = params.rotation(d, 2)
-    T = params.qjl_matrix(d, d, 3)
-    c, _, _ = codebook.lloyd_max(d, bits - 1)
-    a = tq.prod_quantize(x, Pi, T, c, bits)
-    b = tq.prod_quantize(x, Pi, T, c, bits, sketch_operand="f16")
-    diff = a["signs"] != b["signs"]
-    assert np.all(np.abs(a["z"][diff]) < 1e-3)
-
-
 # ---------------------------------------------------------------- scores
 
 @pytest.mark.parametrize("method,bits", [("rq", 3), ("tq_mse", 3), ("tq_prod", 3), ("rq", 2), ("tq_prod", 4)])

@@ -100,6 +100,28 @@ def test_errors():
     kvrq.lib().kvrq_pages_destroy(None)  # no-op
 
 
+def test_overflow_guards():
+    """Counts near INT64_MAX are rejected before any arithmetic can wrap: slots() with a huge count must not
+    read past the block table, append() with a huge n_tokens must not reserve anything."""
+    import ctypes
+    big = (1 << 63) - 1
+    pc = kvrq.PagedCache(4, 8)
+    s = pc.add_seq()
+    pc.append(s, 10)
+    buf = np.full(4, -7, dtype=np.int64)
+    ptr = buf.ctypes.data_as(ctypes.c_void_p)
+    for first, count in ((1, big), (10, big - 9), (big, 1), (11, 0), (0, 11)):
+        assert kvrq.lib().kvrq_pages_slots(pc._h, s, first, count, ptr) == 1  # KVRQ_EINVAL
+    assert np.all(buf == -7)  # nothing written
+    assert kvrq.lib().kvrq_pages_slots(pc._h, s, 10, 0, ptr) == 0  # an empty range at the end is fine
+    for n in (big, big - 10, big - 17):
+        with pytest.raises(KvrqError):
+            pc.append(s, n)
+    table, n_tok = pc.block_table(s)
+    assert n_tok == 10 and len(table) == 2 and pc.stats()[0] == 2  # nothing reserved
+    pc.close()
+
+
 def test_concurrent_appends():
     pc = kvrq.PagedCache(4096, 8)
     seqs = [pc.add_seq() for _ in range(16)]

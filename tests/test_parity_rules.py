@@ -32,7 +32,7 @@ def test_float32_pipeline_signs_pass(d):
     Pi = _fp16(params.rotation(d, 2))
     T = _fp16(params.qjl_matrix(d, d, 3))
     c = codebook.lloyd_max(d, 2)[0].astype(np.float32).astype(np.float64)
-    ref = tq.prod_quantize(x, Pi, T, c, 3, sketch_operand="f16")
+    ref = tq.prod_quantize(x, Pi, T, c, 3)
     words, idx = _float32_prod_signs(x, Pi, T, c)
     bad_rows = np.any(idx != ref["codes"], axis=1)
     compare_sketch_signs(words, ref, x, Pi, T, c, skip_rows=bad_rows)
@@ -48,21 +48,88 @@ def test_planted_sign_error_fails():
     Pi = _fp16(params.rotation(d, 2))
     T = _fp16(params.qjl_matrix(d, d, 3))
     c = codebook.lloyd_max(d, 2)[0]
-    ref = tq.prod_quantize(x, Pi, T, c, 3, sketch_operand="f16")
+    ref = tq.prod_quantize(x, Pi, T, c, 3)
     p, bound = residual_sketch_slack(ref, x, Pi, T, c)
     s = ocodes.unpack(ref["signs_words"], d, 1)
     i, j = np.unravel_index(np.argmax(np.abs(p) - bound), p.shape)  # the sign farthest from its bound
     s[i, j] ^= 1
     with pytest.raises(AssertionError, match="beyond the rounding bound"):
-        compare_sketch_signs(ocodes.pack(s, 1), ref, x, Pi, T, c)
+        compare_sketch_signs(ocodes.pack(s, 1), ref, x, Pi, T, c, report=False)
     # many flips, each inside its bound, exceed the count limit
     x = _fp16(rng.standard_normal((2000, d)))
-    ref = tq.prod_quantize(x, Pi, T, c, 3, sketch_operand="f16")
+    ref = tq.prod_quantize(x, Pi, T, c, 3)
     p, bound = residual_sketch_slack(ref, x, Pi, T, c)
     inside = np.flatnonzero(np.abs(p).ravel() <= bound.ravel())
     assert inside.size > 8
     s = ocodes.unpack(ref["signs_words"], d, 1)
     s.ravel()[inside] ^= 1
-    compare_sketch_signs(ocodes.pack(s, 1), ref, x, Pi, T, c, max_frac=1.0)
+    compare_sketch_signs(ocodes.pack(s, 1), ref, x, Pi, T, c, max_frac=1.0, report=False)
     with pytest.raises(AssertionError, match="signs differ"):
-        compare_sketch_signs(ocodes.pack(s, 1), ref, x, Pi, T, c, max_frac=0.0)
+        compare_sketch_signs(ocodes.pack(s, 1), ref, x, Pi, T, c, max_frac=0.0, report=False)
+
+
+def _fp16_scores(method, q, keys, p, bits):
+    """Packed-code scores as the tensor-core kernel forms them: fp16 rotated query, fp16 centroids (and fp16
+    T q' against the +-1 signs), float32 sums and epilogue."""
+    from oracle import rq as orq
+    from oracle.params import n_groups
+    d = q.shape[1]
+    c16 = np.asarray(p["centroids"]).astype(np.float16).astype(np.float32)
+    out = []
+    for h in range(q.shape[0]):
+        if method == "rq":
+            qp = orq.rotate(q[h:h + 1], p["rotors"])[0]
+            idx = ocodes.unpack(keys["words"][0], 3 * n_groups(d), bits)
+        else:
+            qp = p["Pi"] @ q[h]
+            idx = ocodes.unpack(keys["words"][0], d, bits if method == "tq_mse" else bits - 1)
+        qp16 = qp.astype(np.float16).astype(np.float32)
+        s = (c16[idx] @ qp16).astype(np.float32)
+        if method == "tq_prod":
+            T = np.asarray(p["T"])
+            tq16 = (T.astype(np.float32) @ qp.astype(np.float32)).astype(np.float16).astype(np.float32)
+            sg = (2 * ocodes.unpack(keys["signs_words"][0], T.shape[0], 1) - 1).astype(np.float32)
+            s = s + np.float32(tq.QJL_SCALE_NUM / T.shape[0]) * keys["gammas"][0].astype(np.float32) * (sg @ tq16)
+        out.append(keys["norms"][0].astype(np.float32) * s)
+    return np.stack(out).astype(np.float64)
+
+
+@pytest.mark.parametrize("method,bits", [("rq", 3), ("tq_mse", 3), ("tq_prod", 3), ("tq_prod", 2)])
+def test_score_tolerance_accepts_fp16_restatement(method, bits):
+    from oracle import rq as orq, score
+    from tests.parity import compare_scores, score_tolerance
+    d, n = 128, 3000
+    rng = np.random.default_rng(5)
+    c = codebook.lloyd_max(d, bits - 1 if method == "tq_prod" else bits)[0].astype(np.float32).astype(np.float64)
+    p = {"centroids": c, "rotors": params.rotors(d, 1).astype(np.float32).astype(np.float64),
+         "Pi": _fp16(params.rotation(d, 2)), "T": _fp16(params.qjl_matrix(d, d, 3))}
+    k = rng.standard_normal((n, d)) * np.exp(0.5 * rng.standard_normal((n, 1)))
+    if method == "rq":
+        qq = orq.quantize(k, p["rotors"], c, bits)
+    elif method == "tq_mse":
+        qq = tq.mse_quantize(k, p["Pi"], c, bits)
+    else:
+        qq = tq.prod_quantize(k, p["Pi"], p["T"], c, bits)
+    keys = {"words": qq["words"][None], "norms": qq["norms"].astype(np.float32).astype(np.float64)[None]}
+    if method == "tq_prod":
+        keys["signs_words"] = qq["signs_words"][None]
+        keys["gammas"] = qq["gammas"].astype(np.float32).astype(np.float64)[None]
+    q = _fp16(rng.standard_normal((8, d)))
+    ref = score.direct(method, q, keys, p, bits)
+    floor = score_tolerance(method, q, keys, p, bits)
+    got = _fp16_scores(method, q, keys, p, bits)
+    worst = compare_scores(got, ref, floor)
+    assert worst < 1e-2  # the tensor-core bound of the scores, relative
+    assert np.median(floor) < 1e-2 * np.median(np.abs(ref))
+    # planted mistakes fail: a code moved to its neighbour, and (prod) one sign flipped
+    w = qq["words"].copy()
+    w[17, 0] ^= 1
+    bad = dict(keys, words=w[None])
+    with pytest.raises(AssertionError):
+        compare_scores(score.direct(method, q, bad, p, bits), ref, floor, report=False)
+    if method == "tq_prod":
+        sw = qq["signs_words"].copy()
+        sw[5, 1] ^= 1 << 7
+        with pytest.raises(AssertionError):
+            compare_scores(score.direct(method, q, dict(keys, signs_words=sw[None]), p, bits), ref, floor,
+                           report=False)

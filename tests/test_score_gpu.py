@@ -7,6 +7,7 @@ import torch
 import kv_cache_vector_rq_b200 as kvrq
 from kv_cache_vector_rq_b200 import synth
 from oracle import codebook, params, rq, score, tq
+from tests.parity import compare_scores, score_tolerance
 
 pytestmark = pytest.mark.gpu
 
@@ -68,9 +69,7 @@ def test_scores_match_oracle(method, bits, group, n_heads, n_tokens, t_max):
     for h in range(n_heads):
         kh = {kk: v[h:h + 1, :n_tokens] for kk, v in keys.items()}
         ref = score.direct(method, qf[h], kh, p, bits)  # [group, n_tokens]
-        tol = 1e-3 * np.linalg.norm(qf[h], axis=1)[:, None] * keys["norms"][h][None, :n_tokens] + 1e-6
-        err = np.abs(got[h] - ref)
-        assert np.all(err <= tol), "head %d: max excess %g" % (h, float((err - tol).max()))
+        compare_scores(got[h], ref, score_tolerance(method, qf[h], kh, p, bits), name="head %d" % h)
 
 
 def test_score_of_gpu_quantized_keys_equals_dot_with_dequantized():
@@ -140,6 +139,5 @@ def test_scores_many_tiles_per_cta(method, bits):
             kh["signs_words"] = swords[h:h + 1]
             kh["gammas"] = gam[h:h + 1]
         ref = score.direct(method, qf[h], kh, p, bits)
-        tol = 1e-3 * np.linalg.norm(qf[h], axis=1)[:, None] * nrm[h][None, :] + 1e-6
-        err = np.abs(s[h].double().cpu().numpy() - ref)
-        assert np.all(err <= tol), "head %d: max excess %g" % (h, float((err - tol).max()))
+        compare_scores(s[h].double().cpu().numpy(), ref, score_tolerance(method, qf[h], kh, p, bits),
+                       name="head %d" % h)

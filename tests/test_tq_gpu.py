@@ -84,7 +84,7 @@ def test_prod_quantize_and_dequantize(dt, bits, n):
     codes, signs, gammas, norms = kvrq.tq_quantize_prod(x, pi_d, T_d, c_d, bits)
     torch.cuda.synchronize()
     kvrq.device_status()
-    ref = tq.prod_quantize(to_f64(x), pi64, T64, c64, bits, sketch_operand="f16")
+    ref = tq.prod_quantize(to_f64(x), pi64, T64, c64, bits)
     nb, bad = compare_codes(words_u32(codes), ref, D, bits - 1, c64)
     assert np.allclose(to_f64(norms), ref["norms"], rtol=1e-5)
     g = to_f64(gammas)

@@ -124,7 +124,7 @@ def test_prod_quantize_and_dequantize_tiled(d, dt, bits, n, ws_rows):
     codes, signs, gammas, norms = kvrq.tq_quantize_prod(x, pi_d, T_d, c_d, bits, workspace=ws)
     torch.cuda.synchronize()
     kvrq.device_status()
-    ref = tq.prod_quantize(to_f64(x), pi64, T64, c64, bits, sketch_operand="f16")
+    ref = tq.prod_quantize(to_f64(x), pi64, T64, c64, bits)
     nb, bad = compare_codes(words_u32(codes), ref, d, bits - 1, c64)
     assert np.allclose(to_f64(norms), ref["norms"], rtol=1e-5)
     g = to_f64(gammas)
@@ -159,7 +159,7 @@ def test_zero_rows_tiled():
     codes, signs, gammas, norms = kvrq.tq_quantize_prod(x, pi_d, T_d, c_d, bits)
     torch.cuda.synchronize()
     z = [0, 131, 299]
-    ref = tq.prod_quantize(to_f64(x)[z], pi64, T64, c64, bits, sketch_operand="f16")
+    ref = tq.prod_quantize(to_f64(x)[z], pi64, T64, c64, bits)
     assert np.allclose(to_f64(gammas)[z], ref["gammas"], rtol=1e-5)
     assert np.array_equal(words_u32(signs)[z], ref["signs_words"])
     xh = kvrq.tq_dequantize(codes, norms, d, pi_d, c_d, bits, signs=signs, gammas=gammas, T=T_d)
@@ -209,7 +209,7 @@ def test_many_tiles_per_cta(d, dt, n):
     torch.cuda.synchronize()
     kvrq.device_status()
     assert np.allclose(to_f64(norms), nrm64, rtol=1e-5)
-    ref = tq.prod_quantize(x64, pi64, T64, c64, 3, sketch_operand="f16")
+    ref = tq.prod_quantize(x64, pi64, T64, c64, 3)
     nb, bad = compare_codes(words_u32(codes), ref, d, 2, c64)
     assert np.allclose(to_f64(gammas)[~bad], ref["gammas"][~bad], rtol=1e-4, atol=1e-7)
     compare_sketch_signs(words_u32(signs), ref, x64, pi64, T64, c64, skip_rows=bad)
