@@ -65,6 +65,9 @@ kvrq_status kvrq_pages_append(kvrq_pages* p, int64_t seq_id, int64_t n_tokens, i
   auto it = p->seqs.find(seq_id);
   if (it == p->seqs.end()) return set_error(KVRQ_EINVAL, "kvrq_pages_append: unknown sequence");
   kvrq_pages::Seq& s = it->second;
+  // tokens + n_tokens and its rounding up to whole pages must not overflow
+  if (n_tokens > INT64_MAX - s.tokens - p->page_tokens)
+    return set_error(KVRQ_EINVAL, "kvrq_pages_append: n_tokens too large (nothing appended)");
   const int64_t total = s.tokens + n_tokens;
   const int64_t need = (total + p->page_tokens - 1) / p->page_tokens - (int64_t)s.table.size();
   if (need > (int64_t)p->free_list.size())
@@ -85,7 +88,9 @@ kvrq_status kvrq_pages_slots(kvrq_pages* p, int64_t seq_id, int64_t first, int64
   auto it = p->seqs.find(seq_id);
   if (it == p->seqs.end()) return set_error(KVRQ_EINVAL, "kvrq_pages_slots: unknown sequence");
   const kvrq_pages::Seq& s = it->second;
-  if (first + count > s.tokens) return set_error(KVRQ_EINVAL, "kvrq_pages_slots: tokens past the sequence end");
+  // first <= tokens first, so that tokens - first cannot overflow and first + count is never formed
+  if (first > s.tokens || count > s.tokens - first)
+    return set_error(KVRQ_EINVAL, "kvrq_pages_slots: tokens past the sequence end");
   for (int64_t k = 0; k < count; ++k) {
     const int64_t t = first + k;
     slots[k] = (int64_t)s.table[(size_t)(t / p->page_tokens)] * p->page_tokens + t % p->page_tokens;
