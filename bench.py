@@ -8,9 +8,10 @@ one independent shard per rank). One step runs the fused quantize+dequantize
 roundtrip for RotorQuant (and TurboQuant-mse when built) at b = 2, 3, 4 over
 the batch. The headline `value` is the RotorQuant b = 3 roundtrip throughput
 in million vectors per second, summed over ranks (weak scaling, no
-collective on the data path). L2 is flushed (256 MiB write) before every timed
-launch; launches are timed with CUDA events on the launching stream and the
-max over ranks is taken.
+collective on the data path). L2 is flushed before every timed launch by a
+read of a 256 MiB buffer (twice L2; a read leaves clean lines, so the timed
+launch does not pay for writing back the flush's own data); launches are timed
+with CUDA events on the launching stream and the max over ranks is taken.
 
 `--impl reference` times the float64 CPU oracle on a bounded sample of the
 same workload instead (rank 0 only).
@@ -175,6 +176,26 @@ def cpu_oracle_rate(n_sample, bits=HEADLINE_BITS, seed=0):
         rq.roundtrip(x, rot, c, bits)
         dt = time.perf_counter() - t0
     return n_sample / dt, dt
+
+
+def boundary_ties(kind, bits, x_rows, gpu_words, rot, pi, centroids):
+    """Sampled oracle comparison of one leg's packed codes: (coordinates within 1e-5 of a decision boundary,
+    codes that differ from the oracle's, codes that differ away from a boundary). The parameters are the
+    device's rounded values as float64 numbers."""
+    from oracle import codes as ocodes, rq, tq
+
+    c = np.asarray(centroids, dtype=np.float64)
+    if kind == "rq":
+        ref = rq.quantize(x_rows, rot, c, bits)
+        n_codes = 3 * (-(-D // 3))
+    else:
+        ref = tq.mse_quantize(x_rows, pi, c, bits)
+        n_codes = D
+    g = ocodes.unpack(np.asarray(gpu_words, dtype=np.uint32), n_codes, bits)
+    t = 0.5 * (c[:-1] + c[1:])
+    near = np.min(np.abs(ref["y"][..., None] - t), axis=-1) < 1e-5
+    diff = g != ref["codes"]
+    return int(near.sum()), int(diff.sum()), int((diff & ~near).sum())
 
 
 def _oracle_worker(job):
@@ -657,7 +678,8 @@ def main():
     codes = {b: torch.empty((N_VEC, W[b]), dtype=torch.int32, device=dev) for b in BITS}
     norms = torch.empty(N_VEC, dtype=torch.float32, device=dev)
     xhat = torch.empty_like(x)
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    flush = torch.zeros(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    flush_out = torch.zeros((), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
     pi = torch.from_numpy(kvrq.tq_rotation_init(D, 2)).to(torch.float16).to(dev)
@@ -691,7 +713,7 @@ def main():
     t_wall = time.perf_counter()
     for _ in range(args.steps):
         for leg in legs:
-            flush.zero_()
+            torch.sum(flush, dim=0, out=flush_out)  # reads 2x L2: evicts the previous launch's lines, leaves clean ones
             s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             s.record(stream)
             run_leg(leg)
@@ -717,6 +739,20 @@ def main():
         bpv_leg = rq_bytes_per_vector(D, b) if kind == "rq" else tq_bytes_per_vector(D, b)
         legs_out["%s_b%d" % (kind, b)] = {
             "ms": ms, "Mvec_s": N_VEC / (ms * 1e-3) / 1e6, "GB_s": bpv_leg * N_VEC / (ms * 1e-3) / 1e9}
+
+    # every leg's codes for the boundary-tie count (rank 0 compares sampled rows with the oracle below)
+    tie_rows = np.unique(np.concatenate([np.random.default_rng(1).choice(N_VEC, 1024, replace=False), [0, N_VEC - 1]]))
+    tie_data = {}
+    if rank == 0:
+        idx = torch.as_tensor(tie_rows, device=dev)
+        for leg in legs:
+            run_leg(leg)
+            kind, b = leg
+            cw = (codes[b] if kind == "rq" else tq_codes[b])[idx]
+            tie_data[leg] = cw.cpu().numpy().astype(np.int64).astype(np.uint32)
+        tie_x = x[idx].double().cpu().numpy()
+        tie_params = (rot.double().cpu().numpy(), pi.double().cpu().numpy(),
+                      {b: cbs[b].double().cpu().numpy() for b in BITS})
 
     # ---------------------------------------------------------------- end to end through the public API
     x_host = x.to("cpu").pin_memory()
@@ -787,6 +823,11 @@ def main():
         rate_all, workers = cpu_oracle_all_cores(per_w)
         cpu["all_cores"] = {"value": rate_all / 1e6, "unit": "Mvec/s", "cores": workers,
                             "sample": "%d rows per worker, one single-threaded oracle per core" % per_w}
+        ties = {"rows": int(len(tie_rows)), "margin": 1e-5}
+        for (kind, b), words in tie_data.items():
+            near, diff, far = boundary_ties(kind, b, tie_x, words, tie_params[0], tie_params[1], tie_params[2][b])
+            ties["%s_b%d" % (kind, b)] = {"coords_within_margin": near, "codes_differing": diff,
+                                          "codes_differing_off_boundary": far}
 
     if rank == 0:
         line = {
@@ -797,8 +838,8 @@ def main():
             "config": {"workload": "65536 x d128 fp16 KV vectors (LogNormal(0,0.5) norms, 4 outlier channels x10), "
                                    "fused quantize+dequantize, RotorQuant and TurboQuant-mse b=2,3,4; "
                                    "headline RotorQuant b=3",
-                       "n_vectors_per_gpu": N_VEC, "d": D, "io_dtype": "fp16", "l2": "flushed (256 MiB write) "
-                       "before every timed launch", "parallelism": "independent shard per GPU (weak scaling)"},
+                       "n_vectors_per_gpu": N_VEC, "d": D, "io_dtype": "fp16", "l2": "flushed before every timed launch "
+                       "(a read of a 256 MiB buffer, twice L2)", "parallelism": "independent shard per GPU (weak scaling)"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": recorded_traffic("rq_row_kernel<__half,3,RQ_QDQ>"),
                          "traffic_unit": "bytes per launch", "peak_kind": peak_kind,
@@ -812,6 +853,7 @@ def main():
             "gpu_launches": launches,
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
+            "boundary_ties": ties if rank == 0 else None,
             "wall_s_timed_region": wall,
         }
         print(json.dumps(line), flush=True)
