@@ -169,6 +169,33 @@ kvrq_status rq_quantize_dequantize(void* stream, const void* x, kvrq_dtype xdtyp
                                    int64_t ldx, const float* rotors, const float* centroids, int bits,
                                    uint32_t* codes, int64_t ldc, float* norms, void* xhat, int64_t ldo);
 
+/* RotorQuant in the pages' four-grade storage layout [RQ "Parameter Efficiency"
+ * (rotors plus four grade codebooks), "FMA Count (d=128)" table (172 stored
+ * indices per vector, 3.7x at 3 bits), "The Fused CUDA Kernel" (a grade-1 input
+ * gives vector and trivector outputs)]: per group the stored indices are the
+ * three vector components of R v R~ and its trivector component, code k = 4g + i
+ * (i = 0, 1, 2: e1, e2, e3; i = 3: e123), 4G codes per row (172 at d = 128).
+ * The trivector component of a unit-rotor sandwich is identically zero and is
+ * stored as the code of exactly 0, 2^(bits-1) - 1 (ties to the lower index); the
+ * inverse sandwich maps a pseudoscalar to itself, so dequantization ignores it
+ * and x_hat equals that of the three-code layout. Vector and trivector share the
+ * one Lloyd-Max codebook (the pages define no other).
+ *   Arguments as rq_quantize / rq_dequantize / rq_quantize_dequantize, with
+ *   ldc >= kvrq_packed_words(4G, bits) (17 words at d = 128, 3 bits).
+ *   d = 128 only, rows 16-byte aligned (one dtype for the fused call); other
+ *   shapes return KVRQ_EUNSUPPORTED before any launch. */
+kvrq_status rq4_quantize(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,
+                         const float* rotors, const float* centroids, int bits, uint32_t* codes, int64_t ldc,
+                         float* norms);
+
+kvrq_status rq4_dequantize(void* stream, const uint32_t* codes, int64_t ldc, const float* norms, int64_t n, int d,
+                           const float* rotors, const float* centroids, int bits, void* xhat, kvrq_dtype odtype,
+                           int64_t ldo);
+
+kvrq_status rq4_quantize_dequantize(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,
+                                    const float* rotors, const float* centroids, int bits, uint32_t* codes,
+                                    int64_t ldc, float* norms, void* xhat, int64_t ldo);
+
 
 /* ================================================================ TurboQuant
  * [TQA "方法" Algorithm 1; TQB "随机旋转（Lemma 1）"]: u = x/||x||, y = Pi u,
@@ -330,6 +357,16 @@ kvrq_status kv_attention_packed(void* stream, kvrq_method k_method, const void* 
                                 const float* v_norms, int v_bits, const float* v_rotors, const float* v_centroids,
                                 int64_t tok_head_stride, int64_t n_tokens, void* out, kvrq_dtype odtype, int64_t ldo,
                                 void* workspace, size_t workspace_bytes);
+
+/* Which kernel kv_attention_packed runs for keys of k_method (k_bits total
+ * bits), values of v_bits bits and `group` query rows per KV head: 1 when both
+ * contractions run on the tensor cores (fp16 operands: decoded centroids, +-1
+ * signs, rotated queries and softmax weights, fp32 accumulation; outputs within
+ * 1e-2 of the row's largest |output|), 0 for the fp32 CUDA-core kernel (1e-3).
+ * Tensor cores take: TurboQuant-prod keys of 3 or 4 bits with group <= 8,
+ * TurboQuant-mse keys of 2..4 bits and RotorQuant keys of 2 or 3 bits with group
+ * <= 16, all with 3-bit values. Host only; no device is touched. */
+int kvrq_attention_uses_tensor_cores(kvrq_method k_method, int k_bits, int v_bits, int group);
 
 /* ================================================================ paged cache bookkeeping (host)
  * ["TurboQuant + RotorQuant", "Post-Prefill Quantization": the prefill cache is

@@ -131,25 +131,26 @@ def _stream(stream):
     return s.cuda_stream
 
 
-def rq_quantize(x, rotors, centroids, bits, codes=None, norms=None, stream=None):
+def rq_quantize(x, rotors, centroids, bits, codes=None, norms=None, stream=None, _fn="rq_quantize", _cpg=3):
     """Quantize rows of x [n, d] (fp32/fp16/bf16 CUDA). Returns (codes [n, W] int32 view of uint32, norms [n])."""
     torch = _torch()
     n, d = x.shape
-    W = packed_words(3 * rq_groups(d), bits)
+    W = packed_words(_cpg * rq_groups(d), bits)
     if codes is None:
         codes = torch.empty((n, W), dtype=torch.int32, device=x.device)
     if norms is None:
         norms = torch.empty((n,), dtype=torch.float32, device=x.device)
     xp, ldx = _rows(x, "x")
     cp, ldc = _rows(codes, "codes")
-    _lib.check("rq_quantize", lib().rq_quantize(_stream(stream), xp, _dtype_code(x), n, d, ldx,
-                                                _ptr(rotors, "rotors", torch.float32),
-                                                _ptr(centroids, "centroids", torch.float32), bits, cp, ldc,
-                                                _ptr(norms, "norms", torch.float32)))
+    _lib.check(_fn, getattr(lib(), _fn)(_stream(stream), xp, _dtype_code(x), n, d, ldx,
+                                        _ptr(rotors, "rotors", torch.float32),
+                                        _ptr(centroids, "centroids", torch.float32), bits, cp, ldc,
+                                        _ptr(norms, "norms", torch.float32)))
     return codes, norms
 
 
-def rq_dequantize(codes, norms, d, rotors, centroids, bits, out_dtype=None, xhat=None, stream=None):
+def rq_dequantize(codes, norms, d, rotors, centroids, bits, out_dtype=None, xhat=None, stream=None,
+                  _fn="rq_dequantize"):
     """Dequantize packed codes [n, W] + norms [n] into x_hat [n, d]."""
     torch = _torch()
     n = codes.shape[0]
@@ -157,19 +158,19 @@ def rq_dequantize(codes, norms, d, rotors, centroids, bits, out_dtype=None, xhat
         xhat = torch.empty((n, d), dtype=out_dtype or torch.float16, device=codes.device)
     cp, ldc = _rows(codes, "codes")
     op, ldo = _rows(xhat, "xhat")
-    _lib.check("rq_dequantize", lib().rq_dequantize(_stream(stream), cp, ldc, _ptr(norms, "norms", torch.float32), n, d,
-                                                    _ptr(rotors, "rotors", torch.float32),
-                                                    _ptr(centroids, "centroids", torch.float32), bits, op,
-                                                    _dtype_code(xhat), ldo))
+    _lib.check(_fn, getattr(lib(), _fn)(_stream(stream), cp, ldc, _ptr(norms, "norms", torch.float32), n, d,
+                                        _ptr(rotors, "rotors", torch.float32),
+                                        _ptr(centroids, "centroids", torch.float32), bits, op,
+                                        _dtype_code(xhat), ldo))
     return xhat
 
 
 def rq_quantize_dequantize(x, rotors, centroids, bits, codes=None, norms=None, xhat=None, with_codes=True,
-                           stream=None):
+                           stream=None, _fn="rq_quantize_dequantize", _cpg=3):
     """Fused roundtrip: returns (codes, norms, x_hat); codes/norms are None when with_codes is False."""
     torch = _torch()
     n, d = x.shape
-    W = packed_words(3 * rq_groups(d), bits)
+    W = packed_words(_cpg * rq_groups(d), bits)
     if with_codes and codes is None:
         codes = torch.empty((n, W), dtype=torch.int32, device=x.device)
     if with_codes and norms is None:
@@ -179,10 +180,27 @@ def rq_quantize_dequantize(x, rotors, centroids, bits, codes=None, norms=None, x
     xp, ldx = _rows(x, "x")
     cp, ldc = _rows(codes, "codes") if codes is not None else (None, W)
     op, ldo = _rows(xhat, "xhat")
-    _lib.check("rq_quantize_dequantize", lib().rq_quantize_dequantize(
+    _lib.check(_fn, getattr(lib(), _fn)(
         _stream(stream), xp, _dtype_code(x), n, d, ldx, _ptr(rotors, "rotors", torch.float32),
         _ptr(centroids, "centroids", torch.float32), bits, cp, ldc, _ptr(norms, "norms", torch.float32), op, ldo))
     return codes, norms, xhat
+
+
+def rq4_quantize(x, rotors, centroids, bits, codes=None, norms=None, stream=None):
+    """RotorQuant in the four-grade layout (4 codes per group, 172 at d = 128): (codes [n, W], norms [n])."""
+    return rq_quantize(x, rotors, centroids, bits, codes, norms, stream, _fn="rq4_quantize", _cpg=4)
+
+
+def rq4_dequantize(codes, norms, d, rotors, centroids, bits, out_dtype=None, xhat=None, stream=None):
+    """Dequantize four-grade-layout codes [n, W] + norms [n] into x_hat [n, d]."""
+    return rq_dequantize(codes, norms, d, rotors, centroids, bits, out_dtype, xhat, stream, _fn="rq4_dequantize")
+
+
+def rq4_quantize_dequantize(x, rotors, centroids, bits, codes=None, norms=None, xhat=None, with_codes=True,
+                            stream=None):
+    """Fused roundtrip in the four-grade layout: (codes, norms, x_hat)."""
+    return rq_quantize_dequantize(x, rotors, centroids, bits, codes, norms, xhat, with_codes, stream,
+                                  _fn="rq4_quantize_dequantize", _cpg=4)
 
 
 def device_status(stream=None):
@@ -414,6 +432,12 @@ def kv_cache_append(method, x, slot, bits, centroids, codes, norms, rotors=None,
 
 def attention_workspace_bytes(n_heads, group, n_tokens):
     return int(lib().kvrq_attention_workspace_bytes(n_heads, group, n_tokens))
+
+
+def attention_uses_tensor_cores(k_method, k_bits, v_bits, group):
+    """True when kv_attention_packed runs both contractions on the tensor cores for this configuration
+    (fp16 operands, outputs within 1e-2 of the row's largest |output|); False for the fp32 CUDA-core kernel."""
+    return bool(lib().kvrq_attention_uses_tensor_cores(k_method, k_bits, v_bits, group))
 
 
 def kv_attention_packed(k_method, q, k_codes, k_norms, k_bits, v_codes, v_norms, v_bits, n_tokens, k_centroids,

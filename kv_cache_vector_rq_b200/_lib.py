@@ -35,6 +35,10 @@ SIGNATURES = {
     # stream, x, xdtype, n, d, ldx, rotors, centroids, bits, codes, ldc, norms, xhat, ldo
     "rq_quantize_dequantize": (c_int, [c_vp, c_vp, c_int, c_i64, c_int, c_i64, c_vp, c_vp, c_int, c_vp, c_i64, c_vp,
                                        c_vp, c_i64]),
+    "rq4_quantize": (c_int, [c_vp, c_vp, c_int, c_i64, c_int, c_i64, c_vp, c_vp, c_int, c_vp, c_i64, c_vp]),
+    "rq4_dequantize": (c_int, [c_vp, c_vp, c_i64, c_vp, c_i64, c_int, c_vp, c_vp, c_int, c_vp, c_int, c_i64]),
+    "rq4_quantize_dequantize": (c_int, [c_vp, c_vp, c_int, c_i64, c_int, c_i64, c_vp, c_vp, c_int, c_vp, c_i64, c_vp,
+                                        c_vp, c_i64]),
     # stream, x, xdtype, n, d, ldx, pi, centroids, bits, codes, ldc, norms
     "tq_quantize_mse": (c_int, [c_vp, c_vp, c_int, c_i64, c_int, c_i64, c_vp, c_vp, c_int, c_vp, c_i64, c_vp]),
     # ... + xhat, ldo
@@ -74,6 +78,7 @@ SIGNATURES = {
                                     c_vp, c_i64, c_i64, c_vp, c_i64, c_i64, c_vp, c_vp, c_vp, c_vp, c_int, c_vp, c_vp,
                                     c_vp, c_i64, c_i64, c_vp, c_int, c_vp, c_vp, c_i64, c_i64, c_vp, c_int, c_i64, c_vp,
                                     ctypes.c_size_t]),
+    "kvrq_attention_uses_tensor_cores": (c_int, [c_int, c_int, c_int, c_int]),
     "kvrq_pages_create": (c_int, [c_i64, c_int, ctypes.POINTER(c_vp)]),
     "kvrq_pages_destroy": (None, [c_vp]),
     "kvrq_pages_add_seq": (c_int, [c_vp, ctypes.POINTER(c_i64)]),

@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -148,7 +149,7 @@ static kvrq_status launch_status(const char* where, cudaError_t e) {
 static kvrq_status rq_call(const char* name, int mode, void* stream, const void* x, kvrq_dtype xdt, int64_t ldx,
                            const uint32_t* codes_in, uint32_t* codes_out, int64_t ldc, const float* norms_in,
                            float* norms_out, int64_t n, int d, const float* rotors, const float* centroids, int bits,
-                           void* xhat, kvrq_dtype odt, int64_t ldo, int64_t ldn = 1) {
+                           void* xhat, kvrq_dtype odt, int64_t ldo, int64_t ldn = 1, int cpg = 3) {
   if (ldn < 1) return set_errorf(KVRQ_EINVAL, "%s: norm row stride < 1", name);
   if (n < 0) return set_errorf(KVRQ_EINVAL, "%s: n < 0", name);
   if (d < 2 || d > (1 << 20)) return set_errorf(KVRQ_EINVAL, "%s: d must be in 2..2^20", name);
@@ -157,7 +158,8 @@ static kvrq_status rq_call(const char* name, int mode, void* stream, const void*
   if (q_side && !valid_dtype(xdt)) return set_errorf(KVRQ_EINVAL, "%s: bad input dtype", name);
   if (dq_side && !valid_dtype(odt)) return set_errorf(KVRQ_EINVAL, "%s: bad output dtype", name);
   const int G = (d + 2) / 3;
-  const int64_t W = kvrq_packed_words(3 * (int64_t)G, bits);
+  const int64_t W = kvrq_packed_words(cpg * (int64_t)G, bits);
+  if (cpg == 4 && d != 128) return set_errorf(KVRQ_EUNSUPPORTED, "%s: the four-grade layout takes d = 128", name);
   if (n == 0) return KVRQ_OK;
   if (!rotors || !centroids) return set_errorf(KVRQ_EINVAL, "%s: rotors and centroids are required", name);
   if (!aligned(rotors, 16) || !aligned(centroids, 4))
@@ -200,6 +202,7 @@ static kvrq_status rq_call(const char* name, int mode, void* stream, const void*
   a.ldc = ldc;
   a.ldn = ldn;
   a.status = di->status;
+  a.codes_per_group = cpg;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   const kvrq_dtype tdt = q_side ? xdt : odt;
@@ -217,6 +220,9 @@ static kvrq_status rq_call(const char* name, int mode, void* stream, const void*
     if (!dq_side) mo = mx;
     return launch_status(name, launch_rq_row(mode, tdt, bits, mx, mo, a, s, di->num_sms));
   }
+  if (cpg == 4)
+    return set_errorf(KVRQ_EUNSUPPORTED, "%s: the four-grade layout needs 16-byte aligned rows (and one dtype for "
+                                         "the fused call)", name);
   // any d: rows streamed by bulk copy when they start 16-byte aligned and fit its row buffers
   bool wide = true;
   if (q_side) wide = wide && rows_aligned16(x, ldx, xdt);
@@ -531,6 +537,27 @@ kvrq_status rq_quantize_dequantize(void* stream, const void* x, kvrq_dtype xdtyp
                  rotors, centroids, bits, xhat, xdtype, ldo);
 }
 
+kvrq_status rq4_quantize(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,
+                         const float* rotors, const float* centroids, int bits, uint32_t* codes, int64_t ldc,
+                         float* norms) {
+  return rq_call("rq4_quantize", RQ_Q, stream, x, xdtype, ldx, nullptr, codes, ldc, nullptr, norms, n, d, rotors,
+                 centroids, bits, nullptr, xdtype, 0, 1, 4);
+}
+
+kvrq_status rq4_dequantize(void* stream, const uint32_t* codes, int64_t ldc, const float* norms, int64_t n, int d,
+                           const float* rotors, const float* centroids, int bits, void* xhat, kvrq_dtype odtype,
+                           int64_t ldo) {
+  return rq_call("rq4_dequantize", RQ_DQ, stream, nullptr, odtype, 0, codes, nullptr, ldc, norms, nullptr, n, d,
+                 rotors, centroids, bits, xhat, odtype, ldo, 1, 4);
+}
+
+kvrq_status rq4_quantize_dequantize(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,
+                                    const float* rotors, const float* centroids, int bits, uint32_t* codes,
+                                    int64_t ldc, float* norms, void* xhat, int64_t ldo) {
+  return rq_call("rq4_quantize_dequantize", RQ_QDQ, stream, x, xdtype, ldx, nullptr, codes, ldc, nullptr, norms, n,
+                 d, rotors, centroids, bits, xhat, xdtype, ldo, 1, 4);
+}
+
 kvrq_status tq_quantize_mse(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,
                             const void* pi, const float* centroids, int bits, uint32_t* codes, int64_t ldc,
                             float* norms) {
@@ -722,8 +749,6 @@ kvrq_status kv_attention_packed(void* stream, kvrq_method k_method, const void* 
   a.n_heads = n_heads;
   a.group = group;
   a.n_tokens = n_tokens;
-  a.tokens_per_cta = attn_tokens_per_cta(n_heads, n_tokens);
-  a.n_chunks = (int)((n_tokens + a.tokens_per_cta - 1) / a.tokens_per_cta);
   a.q = q;
   a.ldq = ldq;
   a.q_f32 = qdtype == KVRQ_F32;
@@ -759,8 +784,20 @@ kvrq_status kv_attention_packed(void* stream, kvrq_method k_method, const void* 
   a.ws_q = ws;
   a.ws_sq = ws + rows * kAttnQS;
   a.ws_acc = a.ws_sq + rows * 128;
-  a.ws_ml = a.ws_acc + rows * a.n_chunks * kAttnAS;
-  return launch_status(name, launch_attention(k_method, kcb, a, static_cast<cudaStream_t>(stream)));
+  // the chunk count (and so the offset of ws_ml) depends on the path; size both regions for the larger
+  const int64_t tpc = attn_tokens_per_cta(n_heads, n_tokens), tpi = attn_tc_tokens_per_item(n_heads, n_tokens);
+  const int64_t nc_max = std::max((n_tokens + tpc - 1) / tpc, 2 * ((n_tokens + tpi - 1) / tpi));
+  a.ws_ml = a.ws_acc + rows * nc_max * kAttnAS;
+  DeviceInfo* di;
+  kvrq_status st = current_device(&di);
+  if (st != KVRQ_OK) return st;
+  a.status = di->status;
+  return launch_status(name, launch_attention(k_method, kcb, a, static_cast<cudaStream_t>(stream), di->num_sms));
+}
+
+int kvrq_attention_uses_tensor_cores(kvrq_method k_method, int k_bits, int v_bits, int group) {
+  const int kcb = k_method == KVRQ_TQ_PROD ? k_bits - 1 : k_bits;
+  return attn_tc_supported((int)k_method, kcb, v_bits, group) ? 1 : 0;
 }
 
 kvrq_status kv_cache_append(void* stream, kvrq_method method, const void* x, kvrq_dtype xdtype, int64_t n_rows,

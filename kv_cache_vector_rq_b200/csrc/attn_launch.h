@@ -54,14 +54,26 @@ struct AttnArgs {
   float* ws_sq;             // [rows][128]     T q' (prod)
   float* ws_acc;            // [rows][n_chunks][kAttnAS] per-chunk value sums, rotated domain
   float* ws_ml;             // [rows][n_chunks][2] per-chunk (max logit, sum of weights)
+  unsigned* status;         // device status word (bounded-wait time-outs of the tensor-core path)
 };
 
-// Tokens per chunk CTA (a multiple of kAttnSub) and the workspace the call needs;
-// both depend on the sizes only, not on the device.
+// Tokens per chunk CTA of the CUDA-core path (a multiple of kAttnSub), tokens per
+// work item of the tensor-core path (a multiple of 256), and the workspace the call
+// needs (enough for either path); all depend on the sizes only, not on the device.
 int64_t attn_tokens_per_cta(int64_t n_heads, int64_t n_tokens);
+int64_t attn_tc_tokens_per_item(int64_t n_heads, int64_t n_tokens);
 size_t attn_workspace_bytes(int64_t n_heads, int group, int64_t n_tokens);
 
-// k_method: kvrq_method of the keys; k_cbits: stored key-code width.
-cudaError_t launch_attention(int k_method, int k_cbits, const AttnArgs& a, cudaStream_t st);
+// Whether the tensor-core kernel takes keys of k_method with k_cbits-bit stored codes,
+// values of v_bits bits and `group` query rows per KV head.
+bool attn_tc_supported(int k_method, int k_cbits, int v_bits, int group);
+
+// The tensor-core chunk kernel (a.tokens_per_cta = tokens per work item, a.n_chunks = 2 x
+// work items per head); persistent, at most num_sms CTAs.
+cudaError_t launch_attention_tc(int k_method, int k_cbits, const AttnArgs& a, cudaStream_t st, int num_sms);
+
+// k_method: kvrq_method of the keys; k_cbits: stored key-code width. Chooses the path
+// and sets a.tokens_per_cta and a.n_chunks for it.
+cudaError_t launch_attention(int k_method, int k_cbits, AttnArgs a, cudaStream_t st, int num_sms);
 
 }  // namespace kvrq

@@ -1,0 +1,595 @@
+// Fused decode attention from a packed KV cache on tcgen05 tensor cores.
+//   out_(h,g) = sum_t softmax_t(scale * <q_(h,g), k_hat_t>) * v_hat_t
+// ["TurboQuant и PolarQuant", "Проблема KV-кэша в трансформерах": softmax(Q K^T / sqrt(d)) V;
+//  "TurboQuant + RotorQuant", "When to Use Which": attention computed from the compressed
+//  indices; "How TurboQuant Works": <q, k> ~ <q, k_mse> + ||r|| sqrt(pi/2)/m <S q, sign(S r)>]
+//
+// Both contractions of a 128-token tile run on the tensor cores; nothing is dequantized
+// into global memory:
+//   MMA1  S[128 tokens x 16] = A1 . B1^T, K = 128 (+128 for the QJL signs, +16 padding
+//         for RotorQuant keys): A1 = the tile's decoded keys (fp16 centroids and +-1
+//         signs) written by the decoding threads straight into tensor memory, one token
+//         per lane; B1 = the head's rotated queries q' (and T q') in shared memory.
+//   MMA2  O[128 coordinates x 16] += A2 . B2^T, K = 128 tokens: A2 = the tile's decoded
+//         RotorQuant values in the rotated domain (fp16 centroids, MN-major in shared
+//         memory: token t is K row t); B2 = the softmax weights w_t ||v_t|| (fp16).
+// The softmax is online: per tile the warpgroup forms its running maximum, rescales
+// the value accumulator in tensor memory when the maximum grows, and keeps the weight
+// sums per thread (reduced once per chunk). The 129th rotated value coordinate (the
+// rotor pad) is summed on the CUDA cores. Each warpgroup leaves one partial (max,
+// weight sum, rotated value sums) per work item for the merge kernel, which applies
+// the inverse sandwich once per query row.
+//
+// B200 shape: a persistent CTA of two decode warpgroups per SM (tensor memory holds
+// A1 and both accumulators of each); work items are (KV head, token chunk) pairs.
+// A warpgroup streams its tiles' code rows, sign rows and norms by bulk copy through
+// a ring of two stages and is its own pipeline: its first thread issues the copies
+// and both MMAs. Every wait is bounded; a time-out is recorded in the device status
+// word and the CTA drains its copies and MMAs before it leaves.
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "attn_launch.h"
+#include "kvrq_device.cuh"
+#include "tc_decode.cuh"
+
+namespace kvrq {
+namespace attn_tc {
+
+constexpr int kRows = 128;  // tokens per tile = TMEM lanes
+constexpr int kNWG = 2;     // decode warpgroups per CTA
+constexpr int kThreads = 128 * kNWG;
+constexpr int kStages = 2;  // copy stages per warpgroup
+constexpr int NB = 16;      // MMA N: query rows (and, for prod, their T q' rows)
+constexpr int kNcv = 129;   // stored RotorQuant value coordinates (3G at d = 128)
+constexpr uint32_t kTmemCols = 512;
+
+template <int KM, int KB, int VB>
+struct Cfg {
+  static constexpr bool kProd = KM == KVRQ_TQ_PROD;
+  static constexpr int GMAX = kProd ? NB / 2 : NB;  // query rows per KV head
+  static constexpr int NCODE = KM == KVRQ_RQ_MSE ? 129 : 128;
+  static constexpr int KC = KM == KVRQ_RQ_MSE ? 144 : 128;  // MMA1 K of the centroid part
+  static constexpr int K = KC + (kProd ? 128 : 0);
+  static constexpr int KAP = (K / 2 + 31) / 32 * 32;        // A1 columns (fp16 pairs), 32-aligned
+  static constexpr int KBOX = (K + 63) / 64;
+  static constexpr int WK = (NCODE * KB + 31) / 32;  // key code words
+  static constexpr int NS = kProd ? 4 : 0;           // sign words (m = 128)
+  static constexpr int WV = (kNcv * VB + 31) / 32;   // value code words
+  static constexpr int B_BOX = NB * 128;             // 64 K elements x NB rows
+  static constexpr int WCOLS = KAP + 2 * NB;         // A1, S, O
+  static_assert(kNWG * WCOLS <= (int)kTmemCols, "tensor memory");
+  // a stage: key codes [128][WK], signs [128][NS], value codes [128][WV], key norms, gammas, value norms
+  static constexpr int st_s = kRows * WK;
+  static constexpr int st_v = st_s + kRows * NS;
+  static constexpr int st_kn = st_v + kRows * WV;
+  static constexpr int st_kg = st_kn + kRows;
+  static constexpr int st_vn = st_kg + kRows;
+  static constexpr int stage_words = st_vn + kRows;
+  // shared memory (from a 1024-aligned base)
+  static constexpr int klut_off = 0;
+  static constexpr int slut_off = klut_off + Dec<KB>::BYTES;
+  static constexpr int vlut_off = slut_off + (kProd ? 256 * 128 : 0);
+  static constexpr int vc_off = vlut_off + Dec<VB>::BYTES;  // fp32 value centroids [16]
+  static constexpr int b1_off = ((vc_off + 64 + 1023) / 1024) * 1024;
+  static constexpr int A2_ATOM = kRows * 128;  // 64 coordinates x 128 tokens
+  static constexpr int a2_off = b1_off + ((KBOX * B_BOX + 1023) / 1024) * 1024;  // [wg][2 atoms]
+  static constexpr int B2_BYTES = 2 * B_BOX;                                     // 128 tokens x NB rows
+  static constexpr int b2_off = a2_off + kNWG * 2 * A2_ATOM;                      // [wg]
+  static constexpr int stage_off = b2_off + kNWG * B2_BYTES;                      // [wg][stage]
+  static constexpr int red_off = stage_off + kNWG * kStages * stage_words * 4;    // [wg][warp][GMAX]
+  static constexpr int bar_off = red_off + kNWG * 4 * GMAX * 4;
+  static constexpr int nbars = kNWG * (kStages + 2);  // per wg: stages, MMA1 done, MMA2 done
+  static constexpr int tmem_off = bar_off + nbars * 8;
+  static constexpr int alloc = tmem_off + 16 + 1024;
+  static constexpr bool fits = alloc <= 227 * 1024;
+};
+
+template <int KM, int KB, int VB>
+__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
+  using C = Cfg<KM, KB, VB>;
+  static_assert(C::fits, "shared memory");
+  using DK = Dec<KB>;
+  using DV = Dec<VB>;
+  constexpr int WK = C::WK, NS = C::NS, WV = C::WV, GMAX = C::GMAX, K = C::K, KC = C::KC;
+  constexpr bool kProd = C::kProd;
+  constexpr uint32_t kId1 = umma_idesc_f16(false, false, false, NB, kRows);
+  constexpr uint32_t kId2 = umma_idesc_f16(false, false, false, NB, kRows) | (1u << 15);  // A MN-major
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* s_bar = reinterpret_cast<uint64_t*>(smem + C::bar_off);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::tmem_off);
+  float* s_vc = reinterpret_cast<float*>(smem + C::vc_off);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int w = warp >> 2, q4 = warp & 3, r = tid & 127;
+  const int group = a.group;
+
+  if (tid == 0) {
+    for (int i = 0; i < C::nbars; ++i) mbar_init(&s_bar[i], 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) tmem_alloc(s_tmem, kTmemCols);
+  // decode tables, replicated per lane group (see Dec)
+  for (int i = tid; i < DK::ENT * 64; i += kThreads) {
+    const int e = i >> 6, j = (i & 63) % DK::P;
+    reinterpret_cast<__half*>(smem + C::klut_off)[i] = __float2half_rn(a.k_centroids[(e >> (j * KB)) & ((1 << KB) - 1)]);
+  }
+  if (kProd)
+    for (int i = tid; i < 256 * 64; i += kThreads) {
+      const int e = i >> 6, j = (i & 63) % 8;
+      reinterpret_cast<__half*>(smem + C::slut_off)[i] = __float2half_rn(((e >> j) & 1) ? 1.f : -1.f);
+    }
+  for (int i = tid; i < DV::ENT * 64; i += kThreads) {
+    const int e = i >> 6, j = (i & 63) % DV::P;
+    reinterpret_cast<__half*>(smem + C::vlut_off)[i] = __float2half_rn(a.v_centroids[(e >> (j * VB)) & ((1 << VB) - 1)]);
+  }
+  if (tid < (1 << VB)) s_vc[tid] = a.v_centroids[tid];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  // this warpgroup's tensor memory, buffers and barriers
+  uint64_t* bar_st = s_bar + w * (kStages + 2);
+  uint64_t* bar1 = bar_st + kStages;
+  uint64_t* bar2 = bar1 + 1;
+  const uint32_t a1_mma = tmem + (uint32_t)(w * C::WCOLS);
+  const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+  const uint32_t a1_t = a1_mma + lane_off;
+  const uint32_t s_t = a1_t + (uint32_t)C::KAP;
+  const uint32_t o_t = s_t + (uint32_t)NB;
+  const uint32_t s_mma = a1_mma + (uint32_t)C::KAP;
+  const uint32_t o_mma = s_mma + (uint32_t)NB;
+  const uint32_t b1_s = smem_u32(smem + C::b1_off);
+  const uint32_t a2_s = smem_u32(smem + C::a2_off + w * 2 * C::A2_ATOM);
+  const uint32_t b2_s = smem_u32(smem + C::b2_off + w * C::B2_BYTES);
+  uint32_t* w_stage = reinterpret_cast<uint32_t*>(smem + C::stage_off) + w * kStages * C::stage_words;
+  const uint32_t klut_l = smem_u32(smem + C::klut_off) + (uint32_t)((lane % DK::R) * DK::EB);
+  const uint32_t slut_l = smem_u32(smem + C::slut_off) + (uint32_t)((lane & 7) * 16);
+  const uint32_t vlut_l = smem_u32(smem + C::vlut_off) + (uint32_t)((lane % DV::R) * DV::EB);
+  float* red = reinterpret_cast<float*>(smem + C::red_off) + w * 4 * GMAX;
+
+  const int64_t items_per_head = (a.n_tokens + a.tokens_per_cta - 1) / a.tokens_per_cta;
+  const int64_t n_items = a.n_heads * items_per_head;
+  uint32_t par_st = 0;  // bit s: parity of stage s's next completion
+  uint32_t n1 = 0, n2 = 0;  // MMA1 / MMA2 completions waited for so far
+  int slot = 0;             // stage of this warpgroup's next tile
+  bool ok = true;
+
+  for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
+    const int64_t head = item / items_per_head;
+    const int64_t chunk = item - head * items_per_head;
+    const int64_t row0 = head * group;
+    const int64_t t_begin = chunk * a.tokens_per_cta;
+    const int64_t t_end = a.n_tokens < t_begin + a.tokens_per_cta ? a.n_tokens : t_begin + a.tokens_per_cta;
+    const int ntiles = (int)((t_end - t_begin + kRows - 1) / kRows);
+    const uint32_t* kbase = a.k_codes + head * a.k_head_stride;
+    const uint32_t* sbase = kProd ? a.k_signs + head * a.s_head_stride : nullptr;
+    const uint32_t* vbase = a.v_codes + head * a.v_head_stride;
+    const float* knb = a.k_norms + head * a.tok_head_stride;
+    const float* kgb = kProd ? a.k_gammas + head * a.tok_head_stride : nullptr;
+    const float* vnb = a.v_norms + head * a.tok_head_stride;
+    auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+    // a full tile's rows are contiguous, 16-byte aligned blocks when the rows are unpadded
+    const bool bulk = a.ldk == WK && (!kProd || a.lds == NS) && a.ldv == WV && al16(kbase) && al16(vbase) &&
+                      al16(knb) && al16(vnb) && (!kProd || (al16(sbase) && al16(kgb))) && (t_begin % 4) == 0;
+    auto tile_full = [&](int j) { return t_begin + (int64_t)(j + 1) * kRows <= t_end; };
+
+    // ---- B1: fp16 K-major, 128-byte swizzle; row g < group: q'_g over K [0, KC);
+    //      prod row GMAX + g: (T q')_g over K [KC, KC + 128); all else zero
+    for (int idx = tid; idx < NB * (C::KBOX * 8); idx += kThreads) {
+      const int row = idx / (C::KBOX * 8), j = idx - row * (C::KBOX * 8);
+      float v[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int k = 8 * j + e;
+        float val = 0.f;
+        if (k < KC) {
+          if (row < group && k < C::NCODE) val = a.ws_q[(row0 + row) * kAttnQS + k];
+        } else if (kProd && k < K) {
+          if (row >= GMAX && row - GMAX < group) val = a.ws_sq[(row0 + row - GMAX) * 128 + (k - KC)];
+        }
+        v[e] = val;
+      }
+      *reinterpret_cast<uint4*>(smem + C::b1_off + sw128_chunk(row, j, C::B_BOX)) = Elem<__half>::pack(v);
+    }
+    fence_proxy_async_smem();  // generic writes of B1, read by the MMAs
+    __syncthreads();
+
+    auto issue = [&](int j, int s) {  // thread 0 of the warpgroup: tile j into stage s
+      const int64_t t0 = t_begin + (int64_t)j * kRows;
+      uint32_t* dst = w_stage + s * C::stage_words;
+      uint64_t* bar = &bar_st[s];
+      mbar_arrive_expect_tx(bar, (uint32_t)(kRows * 4 * (WK + NS + WV + (kProd ? 3 : 2))));
+      bulk_load(dst, kbase + t0 * WK, kRows * WK * 4, bar);
+      if (kProd) bulk_load(dst + C::st_s, sbase + t0 * NS, kRows * NS * 4, bar);
+      bulk_load(dst + C::st_v, vbase + t0 * WV, kRows * WV * 4, bar);
+      bulk_load(dst + C::st_kn, knb + t0, kRows * 4, bar);
+      if (kProd) bulk_load(dst + C::st_kg, kgb + t0, kRows * 4, bar);
+      bulk_load(dst + C::st_vn, vnb + t0, kRows * 4, bar);
+    };
+    const int nt_w = ntiles > w ? (ntiles - w + kNWG - 1) / kNWG : 0;  // this warpgroup's tiles
+    const int slot0 = slot;
+    uint32_t pend = 0;  // bit s: a copy into stage s is in flight (thread 0 of the warpgroup)
+    if (r == 0 && bulk && ok)
+      for (int q = 0; q < kStages && q < nt_w; ++q)
+        if (tile_full(w + q * kNWG)) {
+          issue(w + q * kNWG, (slot0 + q) % kStages);
+          pend |= 1u << ((slot0 + q) % kStages);
+        }
+
+    float m_run[GMAX], l_part[GMAX], a128[GMAX];
+#pragma unroll
+    for (int g = 0; g < GMAX; ++g) {
+      m_run[g] = -INFINITY;
+      l_part[g] = 0.f;
+      a128[g] = 0.f;
+    }
+    bool mma1_out = false, mma2_out = false;  // committed and not yet waited for
+    int i = 0;
+    for (; i < nt_w; ++i) {
+      const int j = w + i * kNWG;
+      const int s = (slot0 + i) % kStages;
+      const int64_t t0 = t_begin + (int64_t)j * kRows;
+      const int rows = (int)(t_end - t0 < (int64_t)kRows ? t_end - t0 : (int64_t)kRows);
+      const bool valid = r < rows;
+      const bool staged = bulk && tile_full(j);
+      if (staged) {
+        ok = mbar_wait(&bar_st[s], (par_st >> s) & 1u, a.status) && ok;
+        par_st ^= 1u << s;
+        pend &= ~(1u << s);
+      }
+      if (!wg_all(ok, 1 + w)) {
+        ok = false;
+        break;
+      }
+      uint32_t kw[WK], sg[NS > 0 ? NS : 1], vw[WV];
+      float kn, kg = 0.f, vn;
+      if (staged) {
+        const uint32_t st = smem_u32(w_stage + s * C::stage_words);
+#pragma unroll
+        for (int q = 0; q < WK; ++q) kw[q] = lds_u32(st + (uint32_t)((r * WK + q) * 4));
+        if constexpr (kProd) {
+          const uint4 v = lds_v4(st + (uint32_t)((C::st_s + r * NS) * 4));
+          sg[0] = v.x;
+          sg[1] = v.y;
+          sg[2] = v.z;
+          sg[3] = v.w;
+        }
+#pragma unroll
+        for (int q = 0; q < WV; ++q) vw[q] = lds_u32(st + (uint32_t)((C::st_v + r * WV + q) * 4));
+        kn = __uint_as_float(lds_u32(st + (uint32_t)((C::st_kn + r) * 4)));
+        if (kProd) kg = __uint_as_float(lds_u32(st + (uint32_t)((C::st_kg + r) * 4)));
+        vn = __uint_as_float(lds_u32(st + (uint32_t)((C::st_vn + r) * 4)));
+      } else {
+        const int64_t t = t0 + r;
+#pragma unroll
+        for (int q = 0; q < WK; ++q) kw[q] = valid ? __ldg(kbase + t * a.ldk + q) : 0u;
+        if constexpr (kProd) {
+#pragma unroll
+          for (int q = 0; q < NS; ++q) sg[q] = valid ? __ldg(sbase + t * a.lds + q) : 0u;
+        }
+#pragma unroll
+        for (int q = 0; q < WV; ++q) vw[q] = valid ? __ldg(vbase + t * a.ldv + q) : 0u;
+        kn = valid ? __ldg(knb + t) : 0.f;
+        if (kProd) kg = valid ? __ldg(kgb + t) : 0.f;
+        vn = valid ? __ldg(vnb + t) : 0.f;
+      }
+
+      // ---- 1. key -> A1 (tensor memory; MMA1 of the previous tile has completed: its S was read)
+      {
+        constexpr int NCC = (KC / 2 + 31) / 32;
+        constexpr int FPC = 64 / DK::P;  // fields per 32 columns
+#pragma unroll
+        for (int c = 0; c < NCC; ++c) {
+          uint32_t rw[32];
+#pragma unroll
+          for (int f = 0; f < FPC; ++f) {
+            const int fi = c * FPC + f;
+            if (fi * DK::P < C::NCODE) {
+              const uint32_t v = field<DK::FB, WK>(kw, fi * DK::FB);
+              const uint32_t e = klut_l + (v << 7);
+              if constexpr (DK::EW == 4) {
+                const uint4 x = lds_v4(e);
+                rw[4 * f] = x.x;
+                rw[4 * f + 1] = x.y;
+                rw[4 * f + 2] = x.z;
+                rw[4 * f + 3] = x.w;
+              } else if constexpr (DK::EW == 2) {
+                const uint2 x = lds_v2(e);
+                rw[2 * f] = x.x;
+                rw[2 * f + 1] = x.y;
+              } else {
+                rw[f] = lds_u32(e);
+              }
+            } else {
+#pragma unroll
+              for (int q = 0; q < DK::EW; ++q) rw[DK::EW * f + q] = 0u;
+            }
+#pragma unroll
+            for (int q = 0; q < DK::EW; ++q) {  // K elements past the stored codes are zero
+              const int k0 = 2 * (32 * c + DK::EW * f + q);
+              if (k0 >= C::NCODE) rw[DK::EW * f + q] = 0u;
+              else if (k0 + 1 >= C::NCODE) rw[DK::EW * f + q] &= 0xFFFFu;
+            }
+          }
+          if (32 * c + 32 <= KC / 2) tmem_st32(a1_t + (uint32_t)(32 * c), rw);
+          else tmem_st8(a1_t + (uint32_t)(32 * c), rw);
+        }
+        if constexpr (kProd) {
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            uint32_t rw[32];
+#pragma unroll
+            for (int bq = 0; bq < 8; ++bq) {
+              const int byte = 8 * c + bq;
+              const uint32_t v = (sg[byte >> 2] >> (8 * (byte & 3))) & 0xFFu;
+              const uint4 x = lds_v4(slut_l + (v << 7));
+              rw[4 * bq] = x.x;
+              rw[4 * bq + 1] = x.y;
+              rw[4 * bq + 2] = x.z;
+              rw[4 * bq + 3] = x.w;
+            }
+            tmem_st32(a1_t + (uint32_t)(KC / 2 + 32 * c), rw);
+          }
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      // every thread has read its stage words: the stage may be refilled
+      asm volatile("bar.sync %0, 128;" ::"r"(1 + w) : "memory");
+      if (r == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < K / 16; ++kk) {
+          const uint32_t boff = (uint32_t)((kk >> 2) * C::B_BOX + (kk & 3) * 32);
+          umma_f16_ts(s_mma, a1_mma + (uint32_t)(8 * kk), umma_desc_sw128(b1_s + boff, 16, 1024), kId1, kk > 0);
+        }
+        umma_commit(bar1);
+        const int in = i + kStages;
+        if (staged && in < nt_w && tile_full(w + in * kNWG)) {
+          issue(w + in * kNWG, s);
+          pend |= 1u << s;
+        }
+      }
+      mma1_out = true;
+
+      // ---- 2. value -> A2 (shared memory, MN-major): wait until MMA2 of the previous tile is done
+      if (mma2_out) {
+        ok = mbar_wait(bar2, n2 & 1u, a.status) && ok;
+        ++n2;
+        mma2_out = false;
+      }
+      float c128;
+      {
+        constexpr int FPCH = 8 / DV::P;  // fields per 16-byte chunk (8 coordinates)
+#pragma unroll
+        for (int at = 0; at < 2; ++at) {
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            uint32_t wv[4];
+#pragma unroll
+            for (int f = 0; f < FPCH; ++f) {
+              const int code0 = 64 * at + 8 * ch + DV::P * f;
+              const uint32_t v = field<DV::FB, WV>(vw, code0 * VB);
+              const uint32_t e = vlut_l + (v << 7);
+              if constexpr (DV::EW == 4) {
+                const uint4 x = lds_v4(e);
+                wv[0] = x.x;
+                wv[1] = x.y;
+                wv[2] = x.z;
+                wv[3] = x.w;
+              } else if constexpr (DV::EW == 2) {
+                const uint2 x = lds_v2(e);
+                wv[2 * f] = x.x;
+                wv[2 * f + 1] = x.y;
+              } else {
+                wv[f] = lds_u32(e);
+              }
+            }
+            const uint32_t addr =
+                a2_s + (uint32_t)(at * C::A2_ATOM + (r >> 3) * 1024 + (r & 7) * 128 + ((ch ^ (r & 7)) << 4));
+            sts_v4(addr, make_uint4(wv[0], wv[1], wv[2], wv[3]));
+          }
+        }
+        c128 = s_vc[field<VB, WV>(vw, 128 * VB)];
+      }
+
+      // ---- 3. logits of this tile: wait for MMA1
+      ok = mbar_wait(bar1, n1 & 1u, a.status) && ok;
+      ++n1;
+      mma1_out = false;
+      tc_fence_after();
+      float sv[NB];
+      tmem_ld16(s_t, sv);
+      float lg[GMAX];
+      const float kqs = a.qjl_scale * kg;
+#pragma unroll
+      for (int g = 0; g < GMAX; ++g) {
+        const float dot = kProd ? fmaf(kqs, sv[GMAX + g], sv[g]) : sv[g];
+        lg[g] = (valid && g < group) ? a.scale * kn * dot : -INFINITY;
+      }
+#pragma unroll
+      for (int g = 0; g < GMAX; ++g) {
+        float v = lg[g];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+        if (lane == 0) red[q4 * GMAX + g] = v;
+      }
+      asm volatile("bar.sync %0, 128;" ::"r"(1 + w) : "memory");
+      float alpha[GMAX], p[GMAX];
+      bool grew = false;
+#pragma unroll
+      for (int g = 0; g < GMAX; ++g) {
+        const float mx = fmaxf(fmaxf(red[g], red[GMAX + g]), fmaxf(red[2 * GMAX + g], red[3 * GMAX + g]));
+        const float m_new = fmaxf(m_run[g], mx);
+        alpha[g] = (m_new == m_run[g]) ? 1.f : __expf(m_run[g] - m_new);  // exp(-inf) = 0: nothing yet
+        grew = grew || (m_new != m_run[g]);
+        p[g] = (lg[g] == -INFINITY) ? 0.f : __expf(lg[g] - m_new);
+        m_run[g] = m_new;
+        l_part[g] = fmaf(l_part[g], alpha[g], p[g]);
+        a128[g] = fmaf(a128[g], alpha[g], p[g] * vn * c128);
+      }
+      // weights w_t ||v_t|| as B2 (fp16, K-major: row g, K = token r), rows >= GMAX zero
+#pragma unroll
+      for (int g = 0; g < NB; ++g) {
+        const float wv = g < GMAX ? p[g] * vn : 0.f;
+        const uint32_t addr = b2_s + (uint32_t)((r >> 6) * C::B_BOX + g * 128 +
+                                                ((((r & 63) >> 3) ^ (g & 7)) << 4) + (r & 7) * 2);
+        asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(__half_as_ushort(__float2half_rn(wv))) : "memory");
+      }
+      // the value sums so far (lane r = coordinate r) follow the new maximum
+      if (i > 0 && grew) {
+        float o[NB];
+        tmem_ld16(o_t, o);
+        uint32_t ow[NB];
+#pragma unroll
+        for (int g = 0; g < NB; ++g) ow[g] = __float_as_uint(g < GMAX ? o[g] * alpha[g] : 0.f);
+        tmem_st16(o_t, ow);
+        tmem_wait_st();
+      }
+      fence_proxy_async_smem();  // A2 and B2 were written by generic stores
+      tc_fence_before();
+      asm volatile("bar.sync %0, 128;" ::"r"(1 + w) : "memory");
+      if (r == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kRows / 16; ++kk) {
+          const uint32_t aoff = (uint32_t)(kk * 16 * 128);
+          const uint32_t boff = (uint32_t)((kk >> 2) * C::B_BOX + (kk & 3) * 32);
+          umma_f16(o_mma, umma_desc_sw128(a2_s + aoff, C::A2_ATOM, 1024), umma_desc_sw128(b2_s + boff, 16, 1024),
+                   kId2, i > 0 || kk > 0);
+        }
+        umma_commit(bar2);
+      }
+      mma2_out = true;
+    }
+
+    // ---- this warpgroup's partial of the item: chunk 2 * chunk + w of each query row
+    const int64_t nck = a.n_chunks;
+    const int64_t cidx = 2 * chunk + w;
+    float o[NB];
+    if (mma2_out) {
+      ok = mbar_wait(bar2, n2 & 1u, a.status) && ok;
+      ++n2;
+      mma2_out = false;
+    }
+    if (mma1_out) {  // a time-out between MMA1 and its wait
+      ok = mbar_wait(bar1, n1 & 1u, a.status) && ok;
+      ++n1;
+      mma1_out = false;
+    }
+    // copies still in flight exist only after a time-out broke the tile loop: they land before the
+    // CTA leaves (the CTA stops after such an item, so the stage parities need no update)
+    if (r == 0)
+      for (int s2 = 0; s2 < kStages; ++s2)
+        if ((pend >> s2) & 1u) {
+          mbar_wait(&bar_st[s2], (par_st >> s2) & 1u, a.status);
+          ok = false;
+        }
+    slot = (slot0 + nt_w) % kStages;
+    ok = wg_all(ok, 1 + w);  // uniform before the warp-collective tensor-memory load
+    tc_fence_after();
+    if (i > 0 && ok) {
+      tmem_ld16(o_t, o);
+#pragma unroll
+      for (int g = 0; g < GMAX; ++g)
+        if (g < group) a.ws_acc[((row0 + g) * nck + cidx) * kAttnAS + r] = o[g];
+    }
+#pragma unroll
+    for (int g = 0; g < GMAX; ++g) {
+      float v = l_part[g], u = a128[g];
+#pragma unroll
+      for (int of = 16; of > 0; of >>= 1) {
+        v += __shfl_xor_sync(0xffffffffu, v, of);
+        u += __shfl_xor_sync(0xffffffffu, u, of);
+      }
+      l_part[g] = v;
+      a128[g] = u;
+    }
+    if (lane == 0)
+#pragma unroll
+      for (int g = 0; g < GMAX; ++g) red[q4 * GMAX + g] = l_part[g];
+    asm volatile("bar.sync %0, 128;" ::"r"(1 + w) : "memory");
+    float lsum[GMAX];
+#pragma unroll
+    for (int g = 0; g < GMAX; ++g) lsum[g] = (red[g] + red[GMAX + g]) + (red[2 * GMAX + g] + red[3 * GMAX + g]);
+    asm volatile("bar.sync %0, 128;" ::"r"(1 + w) : "memory");
+    if (lane == 0)
+#pragma unroll
+      for (int g = 0; g < GMAX; ++g) red[q4 * GMAX + g] = a128[g];
+    asm volatile("bar.sync %0, 128;" ::"r"(1 + w) : "memory");
+#pragma unroll
+    for (int g = 0; g < GMAX; ++g) {
+      if (g < group && r == g) {
+        const int64_t base = (row0 + g) * nck + cidx;
+        const float asum = (red[g] + red[GMAX + g]) + (red[2 * GMAX + g] + red[3 * GMAX + g]);
+        // a warpgroup without tiles leaves an empty partial: weight zero in the merge
+        a.ws_ml[base * 2] = i > 0 ? m_run[g] : -INFINITY;
+        a.ws_ml[base * 2 + 1] = lsum[g];
+        a.ws_acc[base * kAttnAS + 128] = i > 0 ? asum : 0.f;
+      }
+    }
+    if (i == 0 || !ok)
+      for (int g = 0; g < group && g < GMAX; ++g) a.ws_acc[((row0 + g) * nck + cidx) * kAttnAS + r] = 0.f;
+    tc_fence_before();
+    __syncthreads();  // both warpgroups are done with B1 and with this item's buffers
+    if (!__syncthreads_and(ok)) break;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int KM, int KB, int VB>
+static cudaError_t launch_t(const AttnArgs& a, cudaStream_t st, int num_sms) {
+  using C = Cfg<KM, KB, VB>;
+  auto kern = attn_tc_kernel<KM, KB, VB>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::alloc);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int64_t items = a.n_heads * ((a.n_tokens + a.tokens_per_cta - 1) / a.tokens_per_cta);
+  const int64_t grid = items < num_sms ? items : num_sms;
+  kern<<<(unsigned)grid, kThreads, C::alloc, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace attn_tc
+
+bool attn_tc_supported(int k_method, int k_cbits, int v_bits, int group) {
+  if (v_bits != 3) return false;
+  switch (k_method) {
+    case KVRQ_TQ_PROD: return (k_cbits == 2 || k_cbits == 3) && group <= attn_tc::NB / 2;
+    case KVRQ_TQ_MSE: return (k_cbits == 2 || k_cbits == 3 || k_cbits == 4) && group <= attn_tc::NB;
+    case KVRQ_RQ_MSE: return (k_cbits == 2 || k_cbits == 3) && group <= attn_tc::NB;
+    default: return false;
+  }
+}
+
+cudaError_t launch_attention_tc(int k_method, int k_cbits, const AttnArgs& a, cudaStream_t st, int num_sms) {
+  using namespace attn_tc;
+  switch (k_method) {
+    case KVRQ_TQ_PROD:
+      return k_cbits == 2 ? launch_t<KVRQ_TQ_PROD, 2, 3>(a, st, num_sms) : launch_t<KVRQ_TQ_PROD, 3, 3>(a, st, num_sms);
+    case KVRQ_TQ_MSE:
+      if (k_cbits == 2) return launch_t<KVRQ_TQ_MSE, 2, 3>(a, st, num_sms);
+      if (k_cbits == 3) return launch_t<KVRQ_TQ_MSE, 3, 3>(a, st, num_sms);
+      return launch_t<KVRQ_TQ_MSE, 4, 3>(a, st, num_sms);
+    default:
+      return k_cbits == 2 ? launch_t<KVRQ_RQ_MSE, 2, 3>(a, st, num_sms) : launch_t<KVRQ_RQ_MSE, 3, 3>(a, st, num_sms);
+  }
+}
+
+}  // namespace kvrq

@@ -187,15 +187,16 @@ struct Codes {
   static constexpr int NWIN = (NC + CPW - 1) / CPW;
 };
 
-template <typename T, int BITS, int MODE, bool RING, int DD>
+template <typename T, int BITS, int MODE, bool RING, int DD, int L>
 struct Smem {
   using SH = Shape<T, BITS, MODE, RING>;
   using DM = Dims<DD>;
   using TL = Tile<T, DD>;
+  static constexpr int NC = L * DM::G;  // stored codes per row
   static constexpr int STAGES = 1;  // tiles per warp outside the ring
   static constexpr int kWarps = SH::kWarps;
   static constexpr int kRows = SH::kRows;
-  static constexpr int W = Codes<BITS, DM::NC>::W;
+  static constexpr int W = Codes<BITS, NC>::W;
   static constexpr int kRingBoxes = 3;
   // [warp][box] half-tile boxes (ring) or [warp][stage] sub-tiles
   static constexpr int tile_bytes = SH::kRing ? kWarps * kRingBoxes * TL::kBoxBytes : kWarps * STAGES * TL::kTileBytes;
@@ -206,7 +207,7 @@ struct Smem {
   static constexpr int codes_stage = ((kWR * W * 4 + 15) / 16) * 16;
   static constexpr int codes_bytes = kWarps * codes_stage * (MODE == RQ_DQ ? 2 : 1);
   static constexpr int lut_off = codes_off + codes_bytes;  // dequantize: [K][kRows] floats
-  static constexpr int lut_bytes = MODE == RQ_DQ ? Codes<BITS, DM::NC>::K * kRows * 4 : 0;
+  static constexpr int lut_bytes = MODE == RQ_DQ ? Codes<BITS, NC>::K * kRows * 4 : 0;
   static constexpr int mp_off = lut_off + lut_bytes;  // [NP][10] float2
   static constexpr int mp_bytes = DM::NP * 10 * 8;
   static constexpr int cb_off = mp_off + mp_bytes;  // codebook constants
@@ -214,7 +215,7 @@ struct Smem {
   static constexpr int bar_off = cb_off + cb_bytes;  // per warp: ring boxes, or STAGES sub-tiles + 2 code stages
   static constexpr int bytes = bar_off + 8 * kWarps * nbar;
   static constexpr int alloc = bytes + 1024;
-  static_assert(alloc <= 227 * 1024, "shared memory");
+  static constexpr bool fits = alloc <= 227 * 1024;
 };
 
 // mp[p][3i+j] = (M_{2p}[i][j], M_{2p+1}[i][j]) for the exact sandwich matrices;
@@ -335,7 +336,7 @@ struct Bisect {
   }
 };
 
-template <typename T, int BITS, int MODE, bool RING, int DD>
+template <typename T, int BITS, int MODE, bool RING, int DD, int L>
 __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
                                   RING ? 1
                                        : (MODE == RQ_Q ? KVRQ_ROW_MIN_WARPS / 2 : KVRQ_ROW_MIN_WARPS) /
@@ -343,11 +344,16 @@ __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
     rq_row_kernel(const __grid_constant__ CUtensorMap map_x,
                                                        const __grid_constant__ CUtensorMap map_o, RqArgs a) {
   using DM = Dims<DD>;
-  constexpr int D = DM::D, G = DM::G, NP = DM::NP, NC = DM::NC;
+  // L codes per group: 3 (the vector part) or 4 (the pages' four-grade layout: the vector part and
+  // the trivector part, which is identically zero for a unit rotor and stored as the code of 0)
+  static_assert(L == 3 || (L == 4 && DD == 128), "codes per group");
+  constexpr int D = DM::D, G = DM::G, NP = DM::NP, NC = L * G;
+  constexpr int PC = 2 * L;  // codes per group pair
   static_assert(!RING || DD == 128, "the ring holds half-tiles of d = 128 rows");
   using TL = Tile<T, DD>;
   using CD = Codes<BITS, NC>;
-  using SM = Smem<T, BITS, MODE, RING, DD>;
+  using SM = Smem<T, BITS, MODE, RING, DD, L>;
+  static_assert(SM::fits, "shared memory");
   using SH = Shape<T, BITS, MODE, RING>;
   constexpr int STAGES = SM::STAGES;
   constexpr bool kRing = SH::kRing;
@@ -590,6 +596,13 @@ __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
     float win[NWIN];
 #pragma unroll
     for (int w = 0; w < NWIN; ++w) win[w] = kWindow0;
+    if constexpr (L == 4) {
+      // trivector codes: the code of exactly 0, H - 1 by the tie rule (integers < 2^23: exact sums)
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        win[(4 * g + 3) / CPW] += (float)((H - 1) << (BITS * ((4 * g + 3) % CPW)));
+      }
+    }
     if constexpr (kIn) {
 #pragma unroll
       for (int w = 0; w < W; ++w) wc[w] = 0u;
@@ -646,16 +659,16 @@ __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
           C[i] = __fmul2_rn(m2, sg);
           const float2 code = __ffma2_rn(sg, cnt, make_float2(H - 0.5f, H - 0.5f));
           // codes of group 2p (lane x) and 2p + 1 (lane y) into their windows
-          const int kx = 3 * (2 * p) + i, ky = 3 * (2 * p + 1) + i;
+          const int kx = L * (2 * p) + i, ky = L * (2 * p + 1) + i;
           win[kx / CPW] = fmaf(code.x, (float)(1u << (BITS * (kx % CPW))), win[kx / CPW]);
           if (2 * p + 1 < G) win[ky / CPW] = fmaf(code.y, (float)(1u << (BITS * (ky % CPW))), win[ky / CPW]);
         }
         // windows whose codes are all in, and the words they complete, leave the registers now
-        const int done = 6 * (p + 1) < NC ? 6 * (p + 1) : NC;  // codes 0 .. done-1 are packed
+        const int done = PC * (p + 1) < NC ? PC * (p + 1) : NC;  // codes 0 .. done-1 are packed
 #pragma unroll
         for (int w = 0; w < NWIN; ++w) {
           const int last = (w + 1) * CPW < NC ? (w + 1) * CPW : NC;  // one past the window's last code
-          if (last <= done && last > 6 * p) {
+          if (last <= done && last > PC * p) {
             const uint32_t v = __float_as_uint(win[w]) & 0x7fffffu;
             const int bo = w * CPW * BITS;
             wc[bo >> 5] |= v << (bo & 31);
@@ -667,13 +680,13 @@ __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
           // word wi is final once every code overlapping it is packed
           const int last_code = ((32 * wi + 31) / BITS) < NC ? (32 * wi + 31) / BITS : NC - 1;
           const int win_end = ((last_code / CPW) + 1) * CPW < NC ? ((last_code / CPW) + 1) * CPW : NC;
-          const int prev_done = 6 * p < NC ? 6 * p : NC;
+          const int prev_done = PC * p < NC ? PC * p : NC;
           if (win_end <= done && win_end > prev_done) stage_codes[lane * W + wi] = wc[wi];
         }
       } else {
 #pragma unroll
         for (int i = 0; i < 3; ++i) {
-          const int kx = 3 * (2 * p) + i, ky = 3 * (2 * p + 1) + i;
+          const int kx = L * (2 * p) + i, ky = L * (2 * p + 1) + i;
           const float cx = __uint_as_float(lds_u32(lut_a + get_code<BITS, W>(wc, kx) * (kRows * 4)));
           const float cy =
               (2 * p + 1 < G) ? __uint_as_float(lds_u32(lut_a + get_code<BITS, W>(wc, ky) * (kRows * 4))) : 0.f;
@@ -1137,12 +1150,12 @@ __global__ void __launch_bounds__(kThreads) rq_wide_kernel(RqArgs a) {
 // ============================================================================
 // Launch helpers (host)
 // ============================================================================
-template <typename T, int BITS, int MODE, bool RING, int DD>
+template <typename T, int BITS, int MODE, bool RING, int DD, int L>
 static cudaError_t launch_row_s(const CUtensorMap& mx, const CUtensorMap& mo, const RqArgs& a, cudaStream_t st,
                                 int num_sms) {
-  using SM = row::Smem<T, BITS, MODE, RING, DD>;
+  using SM = row::Smem<T, BITS, MODE, RING, DD, L>;
   using SH = row::Shape<T, BITS, MODE, RING>;
-  auto kern = rq_row_kernel<T, BITS, MODE, RING, DD>;
+  auto kern = rq_row_kernel<T, BITS, MODE, RING, DD, L>;
   static int blocks_per_sm = -1;
   if (blocks_per_sm < 0) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::alloc);
@@ -1164,16 +1177,24 @@ int rq_row_box_rows() { return row::kWR; }
 
 bool rq_row_dims(int d, kvrq_dtype dt) { return d == 128 || (d == 256 && dt != KVRQ_F32); }
 
-template <typename T, int BITS, int MODE, int DD>
+// The ring shape exists for d = 128, 16-bit rows, quantize or fused, b <= 3, and buffers that fit.
+template <typename T, int BITS, int MODE, int DD, int L>
+constexpr bool can_ring() {
+  if constexpr (DD == 128 && MODE != RQ_DQ && sizeof(T) == 2 && BITS <= 3)
+    return row::Smem<T, BITS, MODE, true, DD, L>::fits;
+  else
+    return false;
+}
+
+template <typename T, int BITS, int MODE, int DD, int L>
 static cudaError_t launch_row(const CUtensorMap& mx, const CUtensorMap& mo, const RqArgs& a, cudaStream_t st,
                               int num_sms) {
   // the ring pays off once every warp of the GPU has two sub-tiles or more
-  constexpr bool kCanRing = DD == 128 && MODE != RQ_DQ && sizeof(T) == 2 && BITS <= 3;
-  if constexpr (kCanRing) {
+  if constexpr (can_ring<T, BITS, MODE, DD, L>()) {
     if ((a.n + row::kWR - 1) / row::kWR >= 2 * 16 * (int64_t)num_sms)
-      return launch_row_s<T, BITS, MODE, true, DD>(mx, mo, a, st, num_sms);
+      return launch_row_s<T, BITS, MODE, true, DD, L>(mx, mo, a, st, num_sms);
   }
-  return launch_row_s<T, BITS, MODE, false, DD>(mx, mo, a, st, num_sms);
+  return launch_row_s<T, BITS, MODE, false, DD, L>(mx, mo, a, st, num_sms);
 }
 
 template <typename TI, typename TO, int BITS, int MODE, int TEAM>
@@ -1219,14 +1240,14 @@ static cudaError_t launch_general(const RqArgs& a, cudaStream_t st, int num_sms)
   return cudaGetLastError();
 }
 
-template <typename T, int MODE, int DD>
+template <typename T, int MODE, int DD, int L = 3>
 static cudaError_t row_by_bits(int bits, const CUtensorMap& mx, const CUtensorMap& mo, const RqArgs& a,
                                cudaStream_t st, int sms) {
   switch (bits) {
-    case 1: return launch_row<T, 1, MODE, DD>(mx, mo, a, st, sms);
-    case 2: return launch_row<T, 2, MODE, DD>(mx, mo, a, st, sms);
-    case 3: return launch_row<T, 3, MODE, DD>(mx, mo, a, st, sms);
-    default: return launch_row<T, 4, MODE, DD>(mx, mo, a, st, sms);
+    case 1: return launch_row<T, 1, MODE, DD, L>(mx, mo, a, st, sms);
+    case 2: return launch_row<T, 2, MODE, DD, L>(mx, mo, a, st, sms);
+    case 3: return launch_row<T, 3, MODE, DD, L>(mx, mo, a, st, sms);
+    default: return launch_row<T, 4, MODE, DD, L>(mx, mo, a, st, sms);
   }
 }
 
@@ -1236,6 +1257,13 @@ static cudaError_t row_by_type(kvrq_dtype dt, int bits, const CUtensorMap& mx, c
   if (a.d == 256) {  // 16-bit rows only (rq_row_dims)
     if (dt == KVRQ_F16) return row_by_bits<__half, MODE, 256>(bits, mx, mo, a, st, sms);
     return row_by_bits<__nv_bfloat16, MODE, 256>(bits, mx, mo, a, st, sms);
+  }
+  if (a.codes_per_group == 4) {  // the four-grade layout (d = 128 only, checked on the host)
+    switch (dt) {
+      case KVRQ_F32: return row_by_bits<float, MODE, 128, 4>(bits, mx, mo, a, st, sms);
+      case KVRQ_F16: return row_by_bits<__half, MODE, 128, 4>(bits, mx, mo, a, st, sms);
+      default: return row_by_bits<__nv_bfloat16, MODE, 128, 4>(bits, mx, mo, a, st, sms);
+    }
   }
   switch (dt) {
     case KVRQ_F32: return row_by_bits<float, MODE, 128>(bits, mx, mo, a, st, sms);

@@ -31,6 +31,7 @@ struct RqArgs {
   int64_t ldn;  // row stride of norms (floats), both directions
   unsigned* status;  // device status word (bounded-wait time-outs)
   bool wide;         // any-d path: rows are streamed by bulk copy (rq_wide_smem_bytes > 0)
+  int codes_per_group;  // 4: the four-grade layout (row kernel, d = 128); anything else: 3
 };
 
 // d = 128 thread-per-row kernel fed by TMA tensor maps over x and x_hat

@@ -52,6 +52,17 @@ def attention_tolerance(ref, vmax, rel=1e-3):
     return rel * np.abs(ref).max(axis=1, keepdims=True) + 1e-5 * vmax
 
 
+def random_words(g, shape, n_codes, bits):
+    """Seeded uniformly random packed code rows [*shape, W] (unused high bits of the last word zero): any bit
+    pattern is a valid row of codes, so these are inputs that no implementation produced."""
+    W = -(-n_codes * bits // 32)
+    w = g.integers(0, 1 << 32, size=tuple(shape) + (W,), dtype=np.uint64).astype(np.uint32)
+    spare = W * 32 - n_codes * bits
+    if spare:
+        w[..., -1] &= np.uint32((1 << (32 - spare)) - 1)
+    return w
+
+
 def ulp(values, dtype):
     """Spacing of `dtype` at |values| (float64 array)."""
     a = np.abs(values)

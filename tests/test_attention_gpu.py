@@ -1,12 +1,17 @@
 """GPU parity of decode attention from a packed KV cache against the oracle.
 
-Tolerance: the kernel computes in fp32 from the same rounded parameters (Pi and T
-in fp16, rotors and centroids in fp32) that the oracle reads as float64. Logit
-errors are ~1e-6 relative, so the softmax weights agree to ~1e-6; the weighted
-sum of up to a few thousand fp32 terms adds at most ~sqrt(T) * 2^-24 * max|v_hat|
-in the typical case. Every output element must lie within
-1e-3 * (largest |output| of its row) + 1e-5 * max|v_hat|, which is the 1e-3
-relative bound of the fp32 path with an absolute floor for that accumulation.
+Tolerance, by the kernel that runs (kvrq.attention_uses_tensor_cores):
+* CUDA-core kernel: fp32 from the same rounded parameters (Pi and T in fp16, rotors
+  and centroids in fp32) that the oracle reads as float64. Logit errors are ~1e-6
+  relative, so the softmax weights agree to ~1e-6; the weighted sum of up to a few
+  thousand fp32 terms adds at most ~sqrt(T) * 2^-24 * max|v_hat| in the typical
+  case. Every output element must lie within 1e-3 * (largest |output| of its row)
+  + 1e-5 * max|v_hat|: the 1e-3 relative bound of the fp32 path with an absolute
+  floor for that accumulation.
+* Tensor-core kernel: the rotated queries, T q', the centroids and the softmax
+  weights enter the MMAs as fp16; a CPU restatement of that arithmetic
+  (tests/test_attention_tolerance.py) reaches 1-2e-3 of the row's largest output, so
+  the bound is 1e-2 of it (the tensor-core paths' relative bound) with the same floor.
 """
 
 import numpy as np
@@ -16,7 +21,7 @@ import torch
 import kv_cache_vector_rq_b200 as kvrq
 from kv_cache_vector_rq_b200 import synth
 from oracle import attention, codebook, params, rq, tq
-from tests.parity import attention_tolerance
+from tests.parity import attention_tolerance, random_words
 
 pytestmark = pytest.mark.gpu
 
@@ -113,8 +118,14 @@ def _run(k_method, k_bits, v_bits, keys, kp, values, vp, pi, T, q, n_tokens, sca
     return out.double().cpu().numpy()
 
 
-def _check(k_method, k_bits, v_bits, keys, kp, values, vp, q, n_tokens, scale, got, heads, rel=1e-3):
+def _rel(k_method, k_bits, v_bits, group):
+    return 1e-2 if kvrq.attention_uses_tensor_cores(METHODS[k_method], k_bits, v_bits, group) else 1e-3
+
+
+def _check(k_method, k_bits, v_bits, keys, kp, values, vp, q, n_tokens, scale, got, heads, rel=None):
     qf = q.double().numpy()
+    if rel is None:
+        rel = _rel(k_method, k_bits, v_bits, q.shape[1])
     for h in heads:
         kh = {kk: v[h:h + 1, :n_tokens] for kk, v in keys.items()}
         vh = {kk: v[h:h + 1, :n_tokens] for kk, v in values.items()}
@@ -159,3 +170,64 @@ def test_attention_bf16_output_and_sharp_softmax():
     q = torch.randn((2, 8, D), generator=torch.Generator().manual_seed(2)).to(torch.float16)
     got = _run("tq_mse", 3, 3, keys, kp, values, vp, pi, T, q, 500, 2.0, out_dtype=torch.bfloat16)
     _check("tq_mse", 3, 3, keys, kp, values, vp, q, 500, 2.0, got, (0, 1), rel=1e-2)
+
+
+# ---------------------------------------------------------------- tensor-core kernel
+
+def test_tensor_core_path_selection():
+    assert kvrq.attention_uses_tensor_cores(kvrq.TQ_PROD, 3, 3, 8)
+    assert not kvrq.attention_uses_tensor_cores(kvrq.TQ_PROD, 3, 3, 9)  # the QJL rows need N = 2 x group
+    assert kvrq.attention_uses_tensor_cores(kvrq.TQ_MSE, 3, 3, 16)
+    assert kvrq.attention_uses_tensor_cores(kvrq.RQ_MSE, 3, 3, 16)
+    assert not kvrq.attention_uses_tensor_cores(kvrq.RQ_MSE, 3, 4, 8)  # 4-bit values: CUDA cores
+    assert not kvrq.attention_uses_tensor_cores(kvrq.TQ_MSE, 1, 3, 8)
+
+
+@pytest.mark.parametrize("n_tokens", [1, 127, 128, 129, 255, 256, 257, 3001])
+def test_tc_ragged_token_counts(n_tokens):
+    """TurboQuant-prod 3-bit keys, RotorQuant 3-bit values, 8 query rows per KV head (the decode config):
+    partial first tiles, exact tile multiples, one warpgroup without tiles, and a ragged last tile."""
+    keys, kp, values, vp, pi, T = _quantized_cache("tq_prod", 3, 3, 3, n_tokens + 5, seed=n_tokens % 97)
+    q = (2.0 * torch.randn((3, 8, D), generator=torch.Generator().manual_seed(n_tokens))).to(torch.float16)
+    got = _run("tq_prod", 3, 3, keys, kp, values, vp, pi, T, q, n_tokens, 1.0 / np.sqrt(D))
+    _check("tq_prod", 3, 3, keys, kp, values, vp, q, n_tokens, 1.0 / np.sqrt(D), got, range(3))
+
+
+@pytest.mark.parametrize("k_method,k_bits,group", [("tq_prod", 3, 5), ("tq_prod", 4, 8), ("tq_mse", 2, 16),
+                                                   ("tq_mse", 4, 3), ("rq", 2, 16), ("rq", 3, 7)])
+def test_tc_key_methods(k_method, k_bits, group):
+    keys, kp, values, vp, pi, T = _random_cache(k_method, k_bits, 3, 2, 2000, seed=group)
+    q = (2.0 * torch.randn((2, group, D), generator=torch.Generator().manual_seed(group))).to(torch.bfloat16)
+    assert kvrq.attention_uses_tensor_cores(METHODS[k_method], k_bits, 3, group)
+    got = _run(k_method, k_bits, 3, keys, kp, values, vp, pi, T, q, 1999, 1.0 / np.sqrt(D))
+    _check(k_method, k_bits, 3, keys, kp, values, vp, q, 1999, 1.0 / np.sqrt(D), got, (0, 1))
+
+
+def test_tc_persistent_many_items():
+    """More (head, chunk) work items than CTAs: every CTA rebuilds its query operand for several heads and
+    keeps its stage ring and barrier phases across items."""
+    n_heads, n_tok = 400, 1500
+    keys, kp, values, vp, pi, T = _random_cache("tq_prod", 3, 3, n_heads, n_tok, seed=31)
+    q = (3.0 * torch.randn((n_heads, 8, D), generator=torch.Generator().manual_seed(3))).to(torch.float16)
+    got = _run("tq_prod", 3, 3, keys, kp, values, vp, pi, T, q, n_tok, 1.0 / np.sqrt(D))
+    _check("tq_prod", 3, 3, keys, kp, values, vp, q, n_tok, 1.0 / np.sqrt(D), got, (0, 149, 150, 399))
+
+
+def test_tc_padded_rows_take_per_thread_loads():
+    """Code rows padded beyond their packed width (no contiguous tile blocks): every tile is loaded per
+    thread instead of by bulk copy; same results."""
+    n_heads, n_tok = 3, 1000
+    keys, kp, values, vp, pi, T = _random_cache("tq_prod", 3, 3, n_heads, n_tok, seed=41)
+    q = torch.randn((n_heads, 8, D), generator=torch.Generator().manual_seed(4)).to(torch.float16)
+    pad = lambda w: np.concatenate([w, np.zeros(w.shape[:-1] + (3,), dtype=w.dtype)], axis=-1)
+    kw = dict(pi=pi.cuda(), T=T.cuda(), k_signs=_dev_words(pad(keys["signs_words"])), k_gammas=_dev_f32(keys["gammas"]))
+    out = kvrq.kv_attention_packed(kvrq.TQ_PROD, q.cuda(), _dev_words(pad(keys["words"])), _dev_f32(keys["norms"]), 3,
+                                   _dev_words(pad(values["words"])), _dev_f32(values["norms"]), 3, n_tok,
+                                   _dev_f32(kp["centroids"]), _dev_f32(vp["rotors"]), _dev_f32(vp["centroids"]), **kw)
+    torch.cuda.synchronize()
+    kvrq.device_status()
+    got = out.double().cpu().numpy()
+    _check("tq_prod", 3, 3, keys, kp, values, vp, q, n_tok, 1.0 / np.sqrt(D), got, range(n_heads))
+    # and equal to the unpadded launch up to the order of the fp32 sums (the same tiles, the same MMAs)
+    ref = _run("tq_prod", 3, 3, keys, kp, values, vp, pi, T, q, n_tok, 1.0 / np.sqrt(D))
+    assert np.allclose(got, ref, rtol=0, atol=1e-6 * np.abs(ref).max())

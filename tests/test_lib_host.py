@@ -150,6 +150,15 @@ def test_rq_validation_fails_before_any_launch():
     assert lib.rq_dequantize(None, P, 13, P, 0, 128, P, P, 3, P, 1, 128) == 0
     assert lib.rq_quantize_dequantize(None, P, 1, 10, 128, 128, P, P, 3, P, 13, P, None, 128) == EINVAL
     assert lib.rq_quantize_dequantize(None, P, 1, 10, 128, 128, P, P, 3, P, 13, P, P, 64) == EINVAL
+    # the four-grade layout: 172 codes at d = 128 (17 words at 3 bits), d = 128 only
+    assert lib.rq4_quantize(None, P, 1, 10, 128, 128, P, P, 3, P, 16, P) == EINVAL
+    assert lib.rq4_quantize(None, P, 1, 10, 64, 64, P, P, 3, P, 17, P) == EUNSUP
+    assert lib.rq4_quantize(None, P, 1, 0, 64, 64, P, P, 3, P, 17, P) == EUNSUP
+    assert lib.rq4_quantize(None, P, 1, 0, 128, 128, P, P, 3, P, 17, P) == 0
+    assert lib.rq4_dequantize(None, P, 16, P, 10, 128, P, P, 3, P, 1, 128) == EINVAL
+    assert lib.rq4_dequantize(None, P, 11, P, 10, 128, P, P, 2, P, 1, 127) == EINVAL
+    assert lib.rq4_quantize_dequantize(None, P, 1, 10, 128, 128, P, P, 4, P, 21, P, P, 128) == EINVAL
+    assert kvrq.packed_words(172, 3) == 17 and kvrq.packed_words(172, 2) == 11 and kvrq.packed_words(172, 4) == 22
 
 
 def test_tq_validation_fails_before_any_launch():
@@ -192,10 +201,12 @@ def test_tq_validation_fails_before_any_launch():
 def test_attention_workspace_and_validation_fail_before_any_launch():
     lib = kvrq.lib()
     EINVAL, EUNSUP = 1, 2
-    # rows x (132 rotated-query floats + 128 sketch floats + chunks x (132 sums + max + sum)) x 4 bytes
-    assert lib.kvrq_attention_workspace_bytes(1, 8, 1000) == 8 * 4 * (260 + 4 * 134)  # 4 chunks of 256 tokens
-    assert lib.kvrq_attention_workspace_bytes(72, 8, 131073) == 576 * 4 * (260 + 33 * 134)  # 4,096-token chunks
-    assert lib.kvrq_attention_workspace_bytes(1, 1, 1000000) == 4 * (260 + 977 * 134)  # at most 1,024 chunks
+    # rows x (132 rotated-query floats + 128 sketch floats + chunks x (132 sums + max + sum)) x 4 bytes, with
+    # chunks the larger of the CUDA-core kernel's (token chunks) and the tensor-core kernel's (two partials per
+    # work item; work items of a multiple of 256 tokens, about 16 per SM of a 148-SM GPU)
+    assert lib.kvrq_attention_workspace_bytes(1, 8, 1000) == 8 * 4 * (260 + 8 * 134)  # 4 items of 256 tokens
+    assert lib.kvrq_attention_workspace_bytes(72, 8, 131073) == 576 * 4 * (260 + 66 * 134)  # 33 items of 4,096
+    assert lib.kvrq_attention_workspace_bytes(1, 1, 1000000) == 4 * (260 + 978 * 134)  # 489 items, 1,024 at most
     assert lib.kvrq_attention_workspace_bytes(0, 8, 100) == 0
     wsb = lib.kvrq_attention_workspace_bytes(2, 8, 100)
 
