@@ -515,8 +515,8 @@ def run_attention(args):
     peak, kind = measured_peaks()
     res = {"leg": "decode_attention_c4", "timing": "CUDA events, cache >= 4x L2", "hbm_peak_gbs": peak,
            "peak_kind": kind}
-    for b in (1, 16):
-        r = decode_attention_c4(kvrq, synth, torch, dev, b, args.steps, args.warmup)
+    for b in [int(v) for v in args.attn_batches.split(",")]:
+        r = decode_attention_c4(kvrq, synth, torch, dev, b, args.steps, args.warmup, cached=args.attn_tokens)
         r["frac_of_hbm_peak"] = r["cache_GB_s"] / peak
         res["batch%d" % b] = r
     print(json.dumps(res), flush=True)
@@ -631,6 +631,8 @@ def main():
     ap.add_argument("--attn", action="store_true",
                     help="decode attention from the packed cache at the Qwen2.5-3B decode shape (batch 1 and 16); "
                          "one JSON line")
+    ap.add_argument("--attn-batches", default="1,16", help="batches of --attn (comma separated)")
+    ap.add_argument("--attn-tokens", type=int, default=131072, help="cached tokens of --attn (one more is appended)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 

@@ -20,11 +20,11 @@
 // weight sum, rotated value sums) per work item for the merge kernel, which applies
 // the inverse sandwich once per query row.
 //
-// B200 shape: a persistent CTA of two decode warpgroups per SM (tensor memory holds
-// A1 and both accumulators of each); work items are (KV head, token chunk) pairs.
-// A warpgroup streams its tiles' code rows, sign rows and norms by bulk copy through
-// a ring of two stages and is its own pipeline: its first thread issues the copies
-// and both MMAs. Every wait is bounded; a time-out is recorded in the device status
+// B200 shape: a persistent CTA of three decode warpgroups per SM (tensor memory holds
+// A1 and both accumulators of each; 168 registers per thread); work items are (KV head,
+// token chunk) pairs. A warpgroup streams its tiles' code rows, sign rows and norms by
+// bulk copy into its own stage (the next tile's copy lands while the current tile is
+// computed) and is its own pipeline: its first thread issues the copies and both MMAs. Every wait is bounded; a time-out is recorded in the device status
 // word and the CTA drains its copies and MMAs before it leaves.
 
 #include <cuda_bf16.h>
@@ -40,16 +40,30 @@
 namespace kvrq {
 namespace attn_tc {
 
-constexpr int kRows = 128;  // tokens per tile = TMEM lanes
-constexpr int kNWG = 2;     // decode warpgroups per CTA
+constexpr int kRows = 128;         // tokens per tile = TMEM lanes
+constexpr int kNWG = kAttnTcParts;  // decode warpgroups per CTA (one partial each per work item)
 constexpr int kThreads = 128 * kNWG;
-constexpr int kStages = 2;  // copy stages per warpgroup
+constexpr int kStages = 1;          // copy stages per warpgroup (a refill lands while the tile is computed)
 constexpr int NB = 16;      // MMA N: query rows (and, for prod, their T q' rows)
 constexpr int kNcv = 129;   // stored RotorQuant value coordinates (3G at d = 128)
 constexpr uint32_t kTmemCols = 512;
 
+// A decode table with `RDIV` times fewer replicas than Dec (lanes l and l + R share one, a 2-way bank
+// conflict for RDIV = 2): line = the R replicas of one entry.
+template <int BITS, int RDIV>
+struct Lut {
+  using D = Dec<BITS>;
+  static constexpr int R = D::R / RDIV;
+  static constexpr int LINE = R * D::EB;     // bytes per entry
+  static constexpr int LSH = LINE == 128 ? 7 : (LINE == 64 ? 6 : 5);
+  static_assert((1 << LSH) == LINE, "line");
+  static constexpr int BYTES = D::ENT * LINE;
+};
+
 template <int KM, int KB, int VB>
 struct Cfg {
+  using KL = Lut<KB, 2>;
+  using VL = Lut<VB, 1>;
   static constexpr bool kProd = KM == KVRQ_TQ_PROD;
   static constexpr int GMAX = kProd ? NB / 2 : NB;  // query rows per KV head
   static constexpr int NCODE = KM == KVRQ_RQ_MSE ? 129 : 128;
@@ -72,9 +86,10 @@ struct Cfg {
   static constexpr int stage_words = st_vn + kRows;
   // shared memory (from a 1024-aligned base)
   static constexpr int klut_off = 0;
-  static constexpr int slut_off = klut_off + Dec<KB>::BYTES;
-  static constexpr int vlut_off = slut_off + (kProd ? 256 * 128 : 0);
-  static constexpr int vc_off = vlut_off + Dec<VB>::BYTES;  // fp32 value centroids [16]
+  static constexpr int slut_off = klut_off + KL::BYTES;
+  static constexpr int SLINE = 64;  // signs: byte -> 8 x (+1/-1) (16 bytes), 4 replicas
+  static constexpr int vlut_off = slut_off + (kProd ? 256 * SLINE : 0);
+  static constexpr int vc_off = vlut_off + VL::BYTES;  // fp32 value centroids [16]
   static constexpr int b1_off = ((vc_off + 64 + 1023) / 1024) * 1024;
   static constexpr int A2_ATOM = kRows * 128;  // 64 coordinates x 128 tokens
   static constexpr int a2_off = b1_off + ((KBOX * B_BOX + 1023) / 1024) * 1024;  // [wg][2 atoms]
@@ -95,6 +110,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
   static_assert(C::fits, "shared memory");
   using DK = Dec<KB>;
   using DV = Dec<VB>;
+  using KL = typename C::KL;
+  using VL = typename C::VL;
   constexpr int WK = C::WK, NS = C::NS, WV = C::WV, GMAX = C::GMAX, K = C::K, KC = C::KC;
   constexpr bool kProd = C::kProd;
   constexpr uint32_t kId1 = umma_idesc_f16(false, false, false, NB, kRows);
@@ -116,20 +133,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
   }
   if (warp == 0) tmem_alloc(s_tmem, kTmemCols);
   // decode tables, replicated per lane group (see Dec)
-  for (int i = tid; i < DK::ENT * 64; i += kThreads) {
-    const int e = i >> 6, j = (i & 63) % DK::P;
+  for (int i = tid; i < KL::BYTES / 2; i += kThreads) {  // half j of an entry line: code j % P of the field
+    const int e = i / (KL::LINE / 2), j = (i % (KL::LINE / 2)) % DK::P;
     reinterpret_cast<__half*>(smem + C::klut_off)[i] = __float2half_rn(a.k_centroids[(e >> (j * KB)) & ((1 << KB) - 1)]);
   }
   if (kProd)
-    for (int i = tid; i < 256 * 64; i += kThreads) {
-      const int e = i >> 6, j = (i & 63) % 8;
+    for (int i = tid; i < 256 * C::SLINE / 2; i += kThreads) {
+      const int e = i / (C::SLINE / 2), j = (i % (C::SLINE / 2)) % 8;
       reinterpret_cast<__half*>(smem + C::slut_off)[i] = __float2half_rn(((e >> j) & 1) ? 1.f : -1.f);
     }
-  for (int i = tid; i < DV::ENT * 64; i += kThreads) {
-    const int e = i >> 6, j = (i & 63) % DV::P;
+  for (int i = tid; i < VL::BYTES / 2; i += kThreads) {
+    const int e = i / (VL::LINE / 2), j = (i % (VL::LINE / 2)) % DV::P;
     reinterpret_cast<__half*>(smem + C::vlut_off)[i] = __float2half_rn(a.v_centroids[(e >> (j * VB)) & ((1 << VB) - 1)]);
   }
   if (tid < (1 << VB)) s_vc[tid] = a.v_centroids[tid];
+  // B2 rows >= GMAX (the QJL rows of the logit operand have no weights) stay zero for the whole kernel
+  if (GMAX < NB)
+    for (int i = tid; i < kNWG * 2 * (NB - GMAX) * 32; i += kThreads) {
+      const int wg = i / (2 * (NB - GMAX) * 32), rem = i - wg * 2 * (NB - GMAX) * 32;
+      const int box = rem / ((NB - GMAX) * 32), rr = rem - box * (NB - GMAX) * 32;
+      reinterpret_cast<uint32_t*>(smem + C::b2_off + wg * C::B2_BYTES + box * C::B_BOX + GMAX * 128)[rr] = 0u;
+    }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -150,9 +174,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
   const uint32_t a2_s = smem_u32(smem + C::a2_off + w * 2 * C::A2_ATOM);
   const uint32_t b2_s = smem_u32(smem + C::b2_off + w * C::B2_BYTES);
   uint32_t* w_stage = reinterpret_cast<uint32_t*>(smem + C::stage_off) + w * kStages * C::stage_words;
-  const uint32_t klut_l = smem_u32(smem + C::klut_off) + (uint32_t)((lane % DK::R) * DK::EB);
-  const uint32_t slut_l = smem_u32(smem + C::slut_off) + (uint32_t)((lane & 7) * 16);
-  const uint32_t vlut_l = smem_u32(smem + C::vlut_off) + (uint32_t)((lane % DV::R) * DV::EB);
+  const uint32_t klut_l = smem_u32(smem + C::klut_off) + (uint32_t)((lane % KL::R) * DK::EB);
+  const uint32_t slut_l = smem_u32(smem + C::slut_off) + (uint32_t)((lane & 3) * 16);
+  const uint32_t vlut_l = smem_u32(smem + C::vlut_off) + (uint32_t)((lane % VL::R) * DV::EB);
   float* red = reinterpret_cast<float*>(smem + C::red_off) + w * 4 * GMAX;
 
   const int64_t items_per_head = (a.n_tokens + a.tokens_per_cta - 1) / a.tokens_per_cta;
@@ -253,8 +277,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
       float kn, kg = 0.f, vn;
       if (staged) {
         const uint32_t st = smem_u32(w_stage + s * C::stage_words);
+        if constexpr (WK % 4 == 0) {  // 16-byte rows: vector loads (a 32-bit stride of WK words would conflict)
 #pragma unroll
-        for (int q = 0; q < WK; ++q) kw[q] = lds_u32(st + (uint32_t)((r * WK + q) * 4));
+          for (int q = 0; q < WK / 4; ++q) {
+            const uint4 v = lds_v4(st + (uint32_t)((r * WK + 4 * q) * 4));
+            kw[4 * q] = v.x;
+            kw[4 * q + 1] = v.y;
+            kw[4 * q + 2] = v.z;
+            kw[4 * q + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < WK; ++q) kw[q] = lds_u32(st + (uint32_t)((r * WK + q) * 4));
+        }
         if constexpr (kProd) {
           const uint4 v = lds_v4(st + (uint32_t)((C::st_s + r * NS) * 4));
           sg[0] = v.x;
@@ -282,19 +317,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
         vn = valid ? __ldg(vnb + t) : 0.f;
       }
 
-      // ---- 1. key -> A1 (tensor memory; MMA1 of the previous tile has completed: its S was read)
+      // ---- 1. key -> A1 (tensor memory; MMA1 of the previous tile has completed: its S was read),
+      //      16 columns (32 K elements) per tensor-memory store
       {
-        constexpr int NCC = (KC / 2 + 31) / 32;
-        constexpr int FPC = 64 / DK::P;  // fields per 32 columns
+        constexpr int NCH = (KC / 2 + 15) / 16;
+        constexpr int FPH = 16 / DK::EW;  // fields per 16 columns
 #pragma unroll
-        for (int c = 0; c < NCC; ++c) {
-          uint32_t rw[32];
+        for (int c = 0; c < NCH; ++c) {
+          uint32_t rw[16];
 #pragma unroll
-          for (int f = 0; f < FPC; ++f) {
-            const int fi = c * FPC + f;
+          for (int f = 0; f < FPH; ++f) {
+            const int fi = c * FPH + f;
             if (fi * DK::P < C::NCODE) {
               const uint32_t v = field<DK::FB, WK>(kw, fi * DK::FB);
-              const uint32_t e = klut_l + (v << 7);
+              const uint32_t e = klut_l + (v << KL::LSH);
               if constexpr (DK::EW == 4) {
                 const uint4 x = lds_v4(e);
                 rw[4 * f] = x.x;
@@ -314,29 +350,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
             }
 #pragma unroll
             for (int q = 0; q < DK::EW; ++q) {  // K elements past the stored codes are zero
-              const int k0 = 2 * (32 * c + DK::EW * f + q);
+              const int k0 = 2 * (16 * c + DK::EW * f + q);
               if (k0 >= C::NCODE) rw[DK::EW * f + q] = 0u;
               else if (k0 + 1 >= C::NCODE) rw[DK::EW * f + q] &= 0xFFFFu;
             }
           }
-          if (32 * c + 32 <= KC / 2) tmem_st32(a1_t + (uint32_t)(32 * c), rw);
-          else tmem_st8(a1_t + (uint32_t)(32 * c), rw);
+          if (16 * c + 16 <= KC / 2) tmem_st16(a1_t + (uint32_t)(16 * c), rw);
+          else tmem_st8(a1_t + (uint32_t)(16 * c), rw);  // RotorQuant: 72 = 4 x 16 + 8 columns
         }
         if constexpr (kProd) {
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            uint32_t rw[32];
+          for (int c = 0; c < 4; ++c) {  // 32 signs (4 bytes) per 16 columns
+            uint32_t rw[16];
 #pragma unroll
-            for (int bq = 0; bq < 8; ++bq) {
-              const int byte = 8 * c + bq;
-              const uint32_t v = (sg[byte >> 2] >> (8 * (byte & 3))) & 0xFFu;
-              const uint4 x = lds_v4(slut_l + (v << 7));
+            for (int bq = 0; bq < 4; ++bq) {
+              const uint32_t v = (sg[c] >> (8 * bq)) & 0xFFu;
+              const uint4 x = lds_v4(slut_l + (v << 6));
               rw[4 * bq] = x.x;
               rw[4 * bq + 1] = x.y;
               rw[4 * bq + 2] = x.z;
               rw[4 * bq + 3] = x.w;
             }
-            tmem_st32(a1_t + (uint32_t)(KC / 2 + 32 * c), rw);
+            tmem_st16(a1_t + (uint32_t)(KC / 2 + 16 * c), rw);
           }
         }
       }
@@ -378,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
             for (int f = 0; f < FPCH; ++f) {
               const int code0 = 64 * at + 8 * ch + DV::P * f;
               const uint32_t v = field<DV::FB, WV>(vw, code0 * VB);
-              const uint32_t e = vlut_l + (v << 7);
+              const uint32_t e = vlut_l + (v << VL::LSH);
               if constexpr (DV::EW == 4) {
                 const uint4 x = lds_v4(e);
                 wv[0] = x.x;
@@ -415,48 +450,83 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
         const float dot = kProd ? fmaf(kqs, sv[GMAX + g], sv[g]) : sv[g];
         lg[g] = (valid && g < group) ? a.scale * kn * dot : -INFINITY;
       }
+      // Weights against the running maximum m (lazy rescaling): while every weight stays <= 256 and
+      // every w ||v|| <= 8192 (inside fp16) the maximum is left as it is; otherwise (always on the first
+      // tile, where m = -inf) the warpgroup forms the exact maximum, rescales what it has accumulated and
+      // recomputes the weights. Either way all sums refer to the same m.
+      float p[GMAX];
+      bool need = false;
 #pragma unroll
       for (int g = 0; g < GMAX; ++g) {
-        float v = lg[g];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-        if (lane == 0) red[q4 * GMAX + g] = v;
+        p[g] = (lg[g] == -INFINITY) ? 0.f : __expf(lg[g] - m_run[g]);
+        need = need || !(p[g] <= 256.f) || !(p[g] * vn <= 8192.f);
       }
-      asm volatile("bar.sync %0, 128;" ::"r"(1 + w) : "memory");
-      float alpha[GMAX], p[GMAX];
-      bool grew = false;
+      auto write_b2 = [&]() {
+        // weights w_t ||v_t|| as B2 (fp16, K-major: row g, K = token r): neighbouring tokens share a
+        // 4-byte word; the even thread of a pair writes the first half of the rows, the odd one the rest
+        constexpr int HR = GMAX / 2;
+        const bool odd = (r & 1) != 0;
+        const int rb = r & ~1;
 #pragma unroll
-      for (int g = 0; g < GMAX; ++g) {
-        const float mx = fmaxf(fmaxf(red[g], red[GMAX + g]), fmaxf(red[2 * GMAX + g], red[3 * GMAX + g]));
-        const float m_new = fmaxf(m_run[g], mx);
-        alpha[g] = (m_new == m_run[g]) ? 1.f : __expf(m_run[g] - m_new);  // exp(-inf) = 0: nothing yet
-        grew = grew || (m_new != m_run[g]);
-        p[g] = (lg[g] == -INFINITY) ? 0.f : __expf(lg[g] - m_new);
-        m_run[g] = m_new;
-        l_part[g] = fmaf(l_part[g], alpha[g], p[g]);
-        a128[g] = fmaf(a128[g], alpha[g], p[g] * vn * c128);
-      }
-      // weights w_t ||v_t|| as B2 (fp16, K-major: row g, K = token r), rows >= GMAX zero
-#pragma unroll
-      for (int g = 0; g < NB; ++g) {
-        const float wv = g < GMAX ? p[g] * vn : 0.f;
-        const uint32_t addr = b2_s + (uint32_t)((r >> 6) * C::B_BOX + g * 128 +
-                                                ((((r & 63) >> 3) ^ (g & 7)) << 4) + (r & 7) * 2);
-        asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(__half_as_ushort(__float2half_rn(wv))) : "memory");
-      }
-      // the value sums so far (lane r = coordinate r) follow the new maximum
-      if (i > 0 && grew) {
-        float o[NB];
-        tmem_ld16(o_t, o);
-        uint32_t ow[NB];
-#pragma unroll
-        for (int g = 0; g < NB; ++g) ow[g] = __float_as_uint(g < GMAX ? o[g] * alpha[g] : 0.f);
-        tmem_st16(o_t, ow);
-        tmem_wait_st();
-      }
+        for (int k = 0; k < HR; ++k) {
+          const float lo = p[k] * vn, hi = p[HR + k] * vn;  // compile-time indices: p stays in registers
+          const float mine = odd ? hi : lo;
+          const float give = odd ? lo : hi;
+          const float other = __shfl_xor_sync(0xffffffffu, give, 1);
+          const int g = odd ? HR + k : k;
+          const __half2 h = odd ? __floats2half2_rn(other, mine) : __floats2half2_rn(mine, other);
+          const uint32_t addr = b2_s + (uint32_t)((rb >> 6) * C::B_BOX + g * 128 +
+                                                  ((((rb & 63) >> 3) ^ (g & 7)) << 4) + (rb & 7) * 2);
+          asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(*reinterpret_cast<const uint32_t*>(&h))
+                       : "memory");
+        }
+      };
+      write_b2();
       fence_proxy_async_smem();  // A2 and B2 were written by generic stores
       tc_fence_before();
-      asm volatile("bar.sync %0, 128;" ::"r"(1 + w) : "memory");
+      if (wg_any(need, 1 + w)) {  // (the barrier before MMA2 when no rescaling is needed)
+#pragma unroll
+        for (int g = 0; g < GMAX; ++g) {
+          float v = lg[g];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+          if (lane == 0) red[q4 * GMAX + g] = v;
+        }
+        asm volatile("bar.sync %0, 128;" ::"r"(1 + w) : "memory");
+        float alpha[GMAX];
+        bool grew = false;
+#pragma unroll
+        for (int g = 0; g < GMAX; ++g) {
+          const float mx = fmaxf(fmaxf(red[g], red[GMAX + g]), fmaxf(red[2 * GMAX + g], red[3 * GMAX + g]));
+          const float m_new = fmaxf(m_run[g], mx);
+          alpha[g] = (m_new == m_run[g]) ? 1.f : __expf(m_run[g] - m_new);  // exp(-inf) = 0: nothing yet
+          grew = grew || (m_new != m_run[g]);
+          p[g] = (lg[g] == -INFINITY) ? 0.f : __expf(lg[g] - m_new);
+          m_run[g] = m_new;
+          l_part[g] *= alpha[g];
+          a128[g] *= alpha[g];
+        }
+        // the value sums so far (lane r = coordinate r) follow the new maximum
+        if (i > 0 && grew) {
+          float o[NB];
+          tmem_ld16(o_t, o);
+          uint32_t ow[NB];
+#pragma unroll
+          for (int g = 0; g < NB; ++g) ow[g] = __float_as_uint(g < GMAX ? o[g] * alpha[g] : 0.f);
+          tmem_st16(o_t, ow);
+          tmem_wait_st();
+        }
+        // every thread has read red and the old B2 words are no longer needed: rewrite them
+        write_b2();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        asm volatile("bar.sync %0, 128;" ::"r"(1 + w) : "memory");
+      }
+#pragma unroll
+      for (int g = 0; g < GMAX; ++g) {
+        l_part[g] += p[g];
+        a128[g] = fmaf(p[g] * vn, c128, a128[g]);
+      }
       if (r == 0) {
         tc_fence_after();
 #pragma unroll
@@ -473,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
 
     // ---- this warpgroup's partial of the item: chunk 2 * chunk + w of each query row
     const int64_t nck = a.n_chunks;
-    const int64_t cidx = 2 * chunk + w;
+    const int64_t cidx = kNWG * chunk + w;
     float o[NB];
     if (mma2_out) {
       ok = mbar_wait(bar2, n2 & 1u, a.status) && ok;

@@ -39,6 +39,20 @@ __device__ __forceinline__ bool wg_all(bool pred, int id) {
   return r != 0;
 }
 
+// Barrier `id` among the 128 threads of a warpgroup; returns the OR of `pred` over them.
+__device__ __forceinline__ bool wg_any(bool pred, int id) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred ? 1u : 0u), "r"(id)
+      : "memory");
+  return r != 0;
+}
+
 // field of `FB` bits starting at bit `bit` of the little-endian stream in w[0..NW)
 template <int FB, int NW>
 __device__ __forceinline__ uint32_t field(const uint32_t (&w)[NW], int bit) {
