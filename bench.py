@@ -8,10 +8,11 @@ one independent shard per rank). One step runs the fused quantize+dequantize
 roundtrip for RotorQuant (and TurboQuant-mse when built) at b = 2, 3, 4 over
 the batch. The headline `value` is the RotorQuant b = 3 roundtrip throughput
 in million vectors per second, summed over ranks (weak scaling, no
-collective on the data path). L2 is flushed before every timed launch by a
-read of a 256 MiB buffer (twice L2; a read leaves clean lines, so the timed
-launch does not pay for writing back the flush's own data); launches are timed
-with CUDA events on the launching stream and the max over ranks is taken.
+collective on the data path). Step k runs on batch set k mod 8 (8 independent
+batches, ~306 MB with their outputs: over twice L2, so no launch finds its inputs
+in L2); each leg's K launches are captured into a CUDA graph and replayed back to
+back between two CUDA events on the launching stream, and the max over ranks is
+taken.
 
 `--impl reference` times the float64 CPU oracle on a bounded sample of the
 same workload instead (rank 0 only).
@@ -32,6 +33,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 N_VEC = 65536
+NSETS = 8  # independent batches the timed steps rotate over (inputs and outputs over twice L2)
 D = 128
 BITS = (2, 3, 4)
 HEADLINE_BITS = 3
@@ -673,61 +675,82 @@ def main():
         return max_over_ranks(v, world, dist, dev)
 
     # ---------------------------------------------------------------- inputs and parameters
-    x = synth.lognormal(N_VEC, D, seed=shard_seed(rank), dtype=torch.float16, device=dev)
+    # NSETS independent batches of the workload (inputs and outputs ~306 MB, over twice L2): step k runs on
+    # set k mod NSETS, so no launch finds its inputs in L2 (the previous NSETS - 1 launches streamed ~268 MB)
+    xs = [synth.lognormal(N_VEC, D, seed=shard_seed(rank) * 16 + k, dtype=torch.float16, device=dev)
+          for k in range(NSETS)]
+    x = xs[0]
     rot = torch.from_numpy(kvrq.rq_rotors_init(D, 1).astype(np.float32)).to(dev)
     cbs = {b: torch.from_numpy(kvrq.tq_codebook_init(D, b)[0].astype(np.float32)).to(dev) for b in BITS}
     W = {b: kvrq.packed_words(3 * kvrq.rq_groups(D), b) for b in BITS}
-    codes = {b: torch.empty((N_VEC, W[b]), dtype=torch.int32, device=dev) for b in BITS}
-    norms = torch.empty(N_VEC, dtype=torch.float32, device=dev)
-    xhat = torch.empty_like(x)
-    flush = torch.zeros(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
-    flush_out = torch.zeros((), dtype=torch.float32, device=dev)
+    WMAX = max(max(W.values()), max(kvrq.packed_words(D, b) for b in BITS))
+    codes_all = [torch.empty((N_VEC, WMAX), dtype=torch.int32, device=dev) for _ in range(NSETS)]
+    norms_all = [torch.empty(N_VEC, dtype=torch.float32, device=dev) for _ in range(NSETS)]
+    xhats = [torch.empty_like(x) for _ in range(NSETS)]
+    codes = {b: codes_all[0][:, :W[b]] for b in BITS}
+    norms, xhat = norms_all[0], xhats[0]
     stream = torch.cuda.current_stream()
 
     pi = torch.from_numpy(kvrq.tq_rotation_init(D, 2)).to(torch.float16).to(dev)
-    tq_codes = {b: torch.empty((N_VEC, kvrq.packed_words(D, b)), dtype=torch.int32, device=dev) for b in BITS}
+    tq_codes = {b: codes_all[0][:, :kvrq.packed_words(D, b)] for b in BITS}
     legs = [("rq", b) for b in BITS] + [("tq", b) for b in BITS]
 
-    def run_leg(leg):
+    def run_leg(leg, k=0):
         kind, b = leg
+        st = torch.cuda.current_stream()  # the capture stream while a graph is recorded
         if kind == "rq":
-            kvrq.rq_quantize_dequantize(x, rot, cbs[b], b, codes=codes[b], norms=norms, xhat=xhat, stream=stream)
+            kvrq.rq_quantize_dequantize(xs[k], rot, cbs[b], b, codes=codes_all[k][:, :W[b]], norms=norms_all[k],
+                                        xhat=xhats[k], stream=st)
         else:
-            kvrq.tq_quantize_dequantize_mse(x, pi, cbs[b], b, codes=tq_codes[b], norms=norms, xhat=xhat,
-                                            stream=stream)
+            kvrq.tq_quantize_dequantize_mse(xs[k], pi, cbs[b], b, codes=codes_all[k][:, :kvrq.packed_words(D, b)],
+                                            norms=norms_all[k], xhat=xhats[k], stream=st)
 
     # ---------------------------------------------------------------- warm-up
     # clocks are sampled from the warm-up through the timed region and the 1 GiB leg
     clk = ClockSampler(local)
     clk.__enter__()
     time.sleep(0.3)
-    for _ in range(args.warmup):
+    for i in range(args.warmup):
         for leg in legs:
-            run_leg(leg)
+            for k in range(NSETS):
+                run_leg(leg, k)
+    torch.cuda.synchronize()
+    kvrq.device_status()
+    # Each leg's K launches of the timed region, step k on set k mod NSETS, are captured once into a CUDA
+    # graph: a replay issues them back to back on the device, so neither the host cost of a call (binding,
+    # tensor-map encoding) nor an event pair per launch enters the time of a launch.
+    graphs = {}
+    for leg in legs:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for k in range(args.steps):
+                run_leg(leg, k % NSETS)
+        graphs[leg] = g
+    for leg in legs:
+        graphs[leg].replay()  # one untimed replay (the warm-up of the captured launches)
     torch.cuda.synchronize()
     kvrq.device_status()
 
     # ---------------------------------------------------------------- timed region
-    ev = {leg: [] for leg in legs}
+    ev = {}
     launches = 0
     barrier()
     torch.cuda.synchronize()
     t_wall = time.perf_counter()
-    for _ in range(args.steps):
-        for leg in legs:
-            torch.sum(flush, dim=0, out=flush_out)  # reads 2x L2: evicts the previous launch's lines, leaves clean ones
-            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            s.record(stream)
-            run_leg(leg)
-            e.record(stream)
-            ev[leg].append((s, e))
-            launches += 1
+    for leg in legs:
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        graphs[leg].replay()
+        e.record(stream)
+        ev[leg] = (s, e)
+        launches += args.steps
     torch.cuda.synchronize()
     barrier()
     wall = time.perf_counter() - t_wall
     kvrq.device_status()
+    del graphs
 
-    leg_ms = {leg: ranks_max(sum(s.elapsed_time(e) for s, e in ev[leg]) / args.steps) for leg in legs}
+    leg_ms = {leg: ranks_max(ev[leg][0].elapsed_time(ev[leg][1]) / args.steps) for leg in legs}
     step_ms = sum(leg_ms.values())
     head = ("rq", HEADLINE_BITS)
     head_ms = leg_ms[head]
@@ -783,7 +806,8 @@ def main():
     # ---------------------------------------------------------------- 1 GiB leg (HBM roofline, inputs >> L2)
     large = None
     if not args.no_large:
-        del flush
+        del xs, xhats, codes_all, norms_all
+        torch.cuda.empty_cache()
         xl = synth.lognormal(LARGE_ROWS, D, seed=2000 + rank, dtype=torch.float16, device=dev)
         cl = torch.empty((LARGE_ROWS, W[HEADLINE_BITS]), dtype=torch.int32, device=dev)
         nl = torch.empty(LARGE_ROWS, dtype=torch.float32, device=dev)
@@ -840,8 +864,10 @@ def main():
             "config": {"workload": "65536 x d128 fp16 KV vectors (LogNormal(0,0.5) norms, 4 outlier channels x10), "
                                    "fused quantize+dequantize, RotorQuant and TurboQuant-mse b=2,3,4; "
                                    "headline RotorQuant b=3",
-                       "n_vectors_per_gpu": N_VEC, "d": D, "io_dtype": "fp16", "l2": "flushed before every timed launch "
-                       "(a read of a 256 MiB buffer, twice L2)", "parallelism": "independent shard per GPU (weak scaling)"},
+                       "n_vectors_per_gpu": N_VEC, "d": D, "io_dtype": "fp16",
+                       "l2": "inputs larger than L2: step k runs on batch set k mod %d (%d independent batches, "
+                             "%.0f MB with outputs); each leg's K launches replayed back to back from a CUDA graph"
+                             % (NSETS, NSETS, NSETS * N_VEC * (4 * D + 4 * 17 + 4) / 1e6), "parallelism": "independent shard per GPU (weak scaling)"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": recorded_traffic("rq_row_kernel<__half,3,RQ_QDQ>"),
                          "traffic_unit": "bytes per launch", "peak_kind": peak_kind,
