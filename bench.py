@@ -47,6 +47,17 @@ def rq_bytes_per_vector(d, bits, in_bytes=2, out_bytes=2):
     return d * in_bytes + 4 * W + 4 + d * out_bytes
 
 
+def leg_name(leg):
+    """JSON key of a leg: rq_b3, tq_b2, ... and pq_4222 (PolarQuant's four levels of 4, 2, 2, 2 bits)."""
+    kind, b = leg
+    return "pq_4222" if kind == "pq" else "%s_b%d" % (kind, b)
+
+
+def pq_bytes_per_vector(d=128, in_bytes=2, out_bytes=2):
+    """PolarQuant fused roundtrip at d = 128: x in, 496 bits of angle codes and fp16 radii out, x_hat out."""
+    return d * in_bytes + 62 + d * out_bytes
+
+
 def tq_bytes_per_vector(d, bits, in_bytes=2, out_bytes=2):
     """TurboQuant-mse fused roundtrip: x in, d codes of b bits + norm out, x_hat out."""
     return d * in_bytes + 4 * (-(-(d * bits) // 32)) + 4 + d * out_bytes
@@ -184,9 +195,25 @@ def boundary_ties(kind, bits, x_rows, gpu_words, rot, pi, centroids):
     """Sampled oracle comparison of one leg's packed codes: (coordinates within 1e-5 of a decision boundary,
     codes that differ from the oracle's, codes that differ away from a boundary). The parameters are the
     device's rounded values as float64 numbers."""
-    from oracle import codes as ocodes, rq, tq
+    from oracle import codes as ocodes, polar, rq, tq
 
     c = np.asarray(centroids, dtype=np.float64)
+    if kind == "pq":
+        books = [c[:16], c[16:20], c[20:24], c[24:28]]
+        ref = polar.quantize(x_rows, pi, books)
+        gw = np.asarray(gpu_words, dtype=np.uint32)
+        near = diff = far_ = 0
+        for lv, (w0, w1, b) in enumerate([(0, 8, 4), (8, 10, 2), (10, 11, 2), (11, 12, 2)]):
+            g = ocodes.unpack(gw[:, w0:w1], 64 >> lv, b)
+            t = 0.5 * (books[lv][:-1] + books[lv][1:])
+            if lv == 0:
+                t = np.concatenate([[0.0, 2.0 * np.pi], t])
+            dist = np.min(np.abs(np.asarray(ref["angles"][lv])[..., None] - t), axis=-1)
+            d_ = g != ref["codes"][lv]
+            near += int((dist < 1e-5).sum())
+            diff += int(d_.sum())
+            far_ += int((d_ & ~(dist < 1e-5)).sum())
+        return near, diff, far_
     if kind == "rq":
         ref = rq.quantize(x_rows, rot, c, bits)
         n_codes = 3 * (-(-D // 3))
@@ -693,7 +720,8 @@ def main():
 
     pi = torch.from_numpy(kvrq.tq_rotation_init(D, 2)).to(torch.float16).to(dev)
     tq_codes = {b: codes_all[0][:, :kvrq.packed_words(D, b)] for b in BITS}
-    legs = [("rq", b) for b in BITS] + [("tq", b) for b in BITS]
+    pq_c = torch.from_numpy(kvrq.pq_codebooks()).to(dev)
+    legs = [("rq", b) for b in BITS] + [("tq", b) for b in BITS] + [("pq", 4)]
 
     def run_leg(leg, k=0):
         kind, b = leg
@@ -701,6 +729,9 @@ def main():
         if kind == "rq":
             kvrq.rq_quantize_dequantize(xs[k], rot, cbs[b], b, codes=codes_all[k][:, :W[b]], norms=norms_all[k],
                                         xhat=xhats[k], stream=st)
+        elif kind == "pq":
+            kvrq.pq_quantize_dequantize(xs[k], pi, pq_c, codes=codes_all[k][:, :kvrq.PQ_WORDS], xhat=xhats[k],
+                                        stream=st)
         else:
             kvrq.tq_quantize_dequantize_mse(xs[k], pi, cbs[b], b, codes=codes_all[k][:, :kvrq.packed_words(D, b)],
                                             norms=norms_all[k], xhat=xhats[k], stream=st)
@@ -761,8 +792,9 @@ def main():
     achieved = bpv * N_VEC / (head_ms * 1e-3) / 1e9
     legs_out = {}
     for (kind, b), ms in leg_ms.items():
-        bpv_leg = rq_bytes_per_vector(D, b) if kind == "rq" else tq_bytes_per_vector(D, b)
-        legs_out["%s_b%d" % (kind, b)] = {
+        bpv_leg = (rq_bytes_per_vector(D, b) if kind == "rq" else
+                   pq_bytes_per_vector(D) if kind == "pq" else tq_bytes_per_vector(D, b))
+        legs_out[leg_name((kind, b))] = {
             "ms": ms, "Mvec_s": N_VEC / (ms * 1e-3) / 1e6, "GB_s": bpv_leg * N_VEC / (ms * 1e-3) / 1e9}
 
     # every leg's codes for the boundary-tie count (rank 0 compares sampled rows with the oracle below)
@@ -773,11 +805,11 @@ def main():
         for leg in legs:
             run_leg(leg)
             kind, b = leg
-            cw = (codes[b] if kind == "rq" else tq_codes[b])[idx]
+            cw = (codes[b] if kind == "rq" else codes_all[0][:, :kvrq.PQ_WORDS] if kind == "pq" else tq_codes[b])[idx]
             tie_data[leg] = cw.cpu().numpy().astype(np.int64).astype(np.uint32)
         tie_x = x[idx].double().cpu().numpy()
         tie_params = (rot.double().cpu().numpy(), pi.double().cpu().numpy(),
-                      {b: cbs[b].double().cpu().numpy() for b in BITS})
+                      dict({b: cbs[b].double().cpu().numpy() for b in BITS}, pq=pq_c.double().cpu().numpy()))
 
     # ---------------------------------------------------------------- end to end through the public API
     x_host = x.to("cpu").pin_memory()
@@ -851,8 +883,9 @@ def main():
                             "sample": "%d rows per worker, one single-threaded oracle per core" % per_w}
         ties = {"rows": int(len(tie_rows)), "margin": 1e-5}
         for (kind, b), words in tie_data.items():
-            near, diff, far = boundary_ties(kind, b, tie_x, words, tie_params[0], tie_params[1], tie_params[2][b])
-            ties["%s_b%d" % (kind, b)] = {"coords_within_margin": near, "codes_differing": diff,
+            cb_leg = tie_params[2]["pq"] if kind == "pq" else tie_params[2][b]
+            near, diff, far = boundary_ties(kind, b, tie_x, words, tie_params[0], tie_params[1], cb_leg)
+            ties[leg_name((kind, b))] = {"coords_within_margin": near, "codes_differing": diff,
                                           "codes_differing_off_boundary": far}
 
     if rank == 0:

@@ -197,6 +197,40 @@ kvrq_status rq4_quantize_dequantize(void* stream, const void* x, kvrq_dtype xdty
                                     int64_t ldc, float* norms, void* xhat, int64_t ldo);
 
 
+/* ================================================================ PolarQuant
+ * ["TurboQuant и PolarQuant: математика квантизации KV-кэша в LLM": "Шаг 1:
+ * предобусловливание" (a fixed random rotation), "Полярное преобразование" (level 1
+ * pairs consecutive coordinates (a, b) into a radius and an angle atan2(b, a) in
+ * [0, 2 pi); every further level pairs consecutive radii of the level below, angles
+ * in [0, pi/2]), "Шаг 3: построение кодовых книг" (one Lloyd-Max codebook per level,
+ * nearest centroid), "Степень сжатия" (d = 128: four levels of 4, 2, 2, 2 bits and the
+ * 8 last radii as 16-bit floats, 496 bits per vector)]:
+ *   y = Pi x, the polar transform of y, every angle replaced by the index of its
+ *   nearest centroid (ties to the lower index; a zero pair has angle 0), the 8
+ *   level-4 radii rounded to fp16; x_hat = Pi^T y_hat, y_hat rebuilt from the
+ *   codes and the 16-bit radii (r cos c_hat, r sin c_hat, level by level).
+ *   x, x_hat: [n][ldx], [n][ldo] fp16 or bf16 (xdtype / odtype), rows 16-byte aligned.
+ *   pi: [128][128] row-major in the vector type, 16-byte aligned (Pi of tq_rotation_init).
+ *   centroids: [28] fp32 device: level 1 (16; the Lloyd-Max codebook of the uniform
+ *     angle, (2i + 1) pi/16, whose boundaries are the multiples of pi/8: the kernel
+ *     decides level-1 codes against those boundaries), then 4 for each of levels 2,
+ *     3, 4 ascending (pq_angle_codebook_init(level, 2)); the boundaries of levels
+ *     2..4 are the midpoints of neighbouring centroids.
+ *   codes: [n][ldc] uint32, ldc >= 16: words 0..7 the 64 level-1 codes (4 bits,
+ *     LSB first), 8..9 the 32 level-2 codes, 10 the 16 level-3 codes, 11 the 8
+ *     level-4 codes (bits 0..15; bits 16..31 zero), 12..15 the 8 level-4 radii as
+ *     fp16 pairs (radius 2c in the low half of word 12 + c).
+ *   d = 128 only; other shapes and dtypes return KVRQ_EUNSUPPORTED before any
+ *   launch. The rotations run on the tensor cores (16-bit operands, fp32
+ *   accumulation). pq_quantize_dequantize: codes may be NULL (x_hat only). */
+kvrq_status pq_quantize_dequantize(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,
+                                   const void* pi, const float* centroids, uint32_t* codes, int64_t ldc, void* xhat,
+                                   int64_t ldo);
+
+kvrq_status pq_dequantize(void* stream, const uint32_t* codes, int64_t ldc, int64_t n, int d, const void* pi,
+                          const float* centroids, void* xhat, kvrq_dtype odtype, int64_t ldo);
+
+
 /* ================================================================ TurboQuant
  * [TQA "方法" Algorithm 1; TQB "随机旋转（Lemma 1）"]: u = x/||x||, y = Pi u,
  * each y_i replaced by its nearest Lloyd-Max centroid (codebook for d, ties to

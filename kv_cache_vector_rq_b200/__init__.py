@@ -434,6 +434,50 @@ def attention_workspace_bytes(n_heads, group, n_tokens):
     return int(lib().kvrq_attention_workspace_bytes(n_heads, group, n_tokens))
 
 
+# ----------------------------------------------------------------------------- PolarQuant
+
+PQ_WORDS = 16  # code words per d = 128 row: 496 bits of angle codes and fp16 radii
+
+
+def pq_codebooks(level_bits=(4, 2, 2, 2)):
+    """The [28] fp32 centroid table of pq_quantize_dequantize: the Lloyd-Max angle codebook of every level
+    (pq_angle_codebook_init), level 1 first."""
+    return np.concatenate([pq_angle_codebook_init(level, b)[0] for level, b in enumerate(level_bits, start=1)]
+                          ).astype(np.float32)
+
+
+def pq_quantize_dequantize(x, pi, centroids, codes=None, xhat=None, with_codes=True, stream=None):
+    """PolarQuant fused roundtrip of rows x [n, 128] (fp16/bf16 CUDA): returns (codes [n, 16] int32 view of
+    uint32, x_hat); codes is None when with_codes is False."""
+    torch = _torch()
+    n, d = x.shape
+    if with_codes and codes is None:
+        codes = torch.empty((n, PQ_WORDS), dtype=torch.int32, device=x.device)
+    if xhat is None:
+        xhat = torch.empty_like(x)
+    xp, ldx = _rows(x, "x")
+    cp, ldc = _rows(codes, "codes") if codes is not None else (None, PQ_WORDS)
+    op, ldo = _rows(xhat, "xhat")
+    _lib.check("pq_quantize_dequantize", lib().pq_quantize_dequantize(
+        _stream(stream), xp, _dtype_code(x), n, d, ldx, _ptr(pi, "pi", pi.dtype),
+        _ptr(centroids, "centroids", torch.float32), cp, ldc, op, ldo))
+    return codes, xhat
+
+
+def pq_dequantize(codes, d, pi, centroids, out_dtype=None, xhat=None, stream=None):
+    """x_hat [n, d] from PolarQuant code rows [n, 16]."""
+    torch = _torch()
+    n = codes.shape[0]
+    if xhat is None:
+        xhat = torch.empty((n, d), dtype=out_dtype or pi.dtype, device=codes.device)
+    cp, ldc = _rows(codes, "codes")
+    op, ldo = _rows(xhat, "xhat")
+    _lib.check("pq_dequantize", lib().pq_dequantize(_stream(stream), cp, ldc, n, d, _ptr(pi, "pi", pi.dtype),
+                                                    _ptr(centroids, "centroids", torch.float32), op,
+                                                    _dtype_code(xhat), ldo))
+    return xhat
+
+
 def attention_uses_tensor_cores(k_method, k_bits, v_bits, group):
     """True when kv_attention_packed runs both contractions on the tensor cores for this configuration
     (fp16 operands, outputs within 1e-2 of the row's largest |output|); False for the fp32 CUDA-core kernel."""

@@ -78,6 +78,10 @@ SIGNATURES = {
                                     c_vp, c_i64, c_i64, c_vp, c_i64, c_i64, c_vp, c_vp, c_vp, c_vp, c_int, c_vp, c_vp,
                                     c_vp, c_i64, c_i64, c_vp, c_int, c_vp, c_vp, c_i64, c_i64, c_vp, c_int, c_i64, c_vp,
                                     ctypes.c_size_t]),
+    # stream, x, xdtype, n, d, ldx, pi, centroids, codes, ldc, xhat, ldo
+    "pq_quantize_dequantize": (c_int, [c_vp, c_vp, c_int, c_i64, c_int, c_i64, c_vp, c_vp, c_vp, c_i64, c_vp, c_i64]),
+    # stream, codes, ldc, n, d, pi, centroids, xhat, odtype, ldo
+    "pq_dequantize": (c_int, [c_vp, c_vp, c_i64, c_i64, c_int, c_vp, c_vp, c_vp, c_int, c_i64]),
     "kvrq_attention_uses_tensor_cores": (c_int, [c_int, c_int, c_int, c_int]),
     "kvrq_pages_create": (c_int, [c_i64, c_int, ctypes.POINTER(c_vp)]),
     "kvrq_pages_destroy": (None, [c_vp]),

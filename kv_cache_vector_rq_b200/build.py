@@ -18,7 +18,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libkvrq.so")
 
 SOURCES = ["setup.cpp", "pages.cpp", "api.cu", "rq_kernels.cu", "tq_kernels.cu", "tqg_kernels.cu",
-           "score_kernels.cu", "attn_kernels.cu", "attn_tc_kernels.cu"]
+           "score_kernels.cu", "attn_kernels.cu", "attn_tc_kernels.cu", "pq_kernels.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-I" + INCLUDE, "-I" + CSRC]
 

@@ -18,6 +18,7 @@
 #include "tqg_launch.h"
 #include "score_launch.h"
 #include "attn_launch.h"
+#include "pq_launch.h"
 
 namespace kvrq {
 
@@ -454,6 +455,45 @@ static kvrq_status tq_call(const char* name, int mode, void* stream, const void*
   return launch_status(name, launch_tq(mode, dt, cbits, mx, mp, mt, mo, a, static_cast<cudaStream_t>(stream), di->num_sms));
 }
 
+// PolarQuant at d = 128 (fused roundtrip, or dequantize of stored code rows).
+static kvrq_status pq_call(const char* name, int mode, void* stream, const void* x, kvrq_dtype dt, int64_t ldx,
+                           int64_t n, int d, const void* pi, const float* centroids, uint32_t* codes_out,
+                           const uint32_t* codes_in, int64_t ldc, void* xhat, int64_t ldo) {
+  if (n < 0) return set_errorf(KVRQ_EINVAL, "%s: n < 0", name);
+  if (d != 128) return set_errorf(KVRQ_EUNSUPPORTED, "%s: d = 128 is supported (four levels of 4, 2, 2, 2 bits)", name);
+  if (dt != KVRQ_F16 && dt != KVRQ_BF16) return set_errorf(KVRQ_EUNSUPPORTED, "%s: fp16 or bf16 vectors", name);
+  if (n == 0) return KVRQ_OK;
+  if (!pi || !aligned(pi, 16) || !centroids || !aligned(centroids, 4))
+    return set_errorf(KVRQ_EINVAL, "%s: pi (16-byte aligned) and centroids are required", name);
+  if (mode == PQ_QDQ && (!x || ldx < d || !rows_aligned16(x, ldx, dt)))
+    return set_errorf(KVRQ_EINVAL, "%s: x NULL, ldx < d or rows not 16-byte aligned", name);
+  if (mode == PQ_DQ && !codes_in) return set_errorf(KVRQ_EINVAL, "%s: codes are required", name);
+  if ((codes_in || codes_out) && (ldc < kPqWords || !aligned(codes_in ? (const void*)codes_in : codes_out, 4)))
+    return set_errorf(KVRQ_EINVAL, "%s: ldc must be >= %d code words", name, kPqWords);
+  if (!xhat || ldo < d || !rows_aligned16(xhat, ldo, dt))
+    return set_errorf(KVRQ_EINVAL, "%s: xhat NULL, ldo < d or rows not 16-byte aligned", name);
+  if (n > ((int64_t)1 << 31) - 256) return set_errorf(KVRQ_EUNSUPPORTED, "%s: n >= 2^31", name);
+  DeviceInfo* di;
+  kvrq_status st = current_device(&di);
+  if (st != KVRQ_OK) return st;
+  CUtensorMap mx, mp, mo;
+  memset(&mx, 0, sizeof(mx));
+  memset(&mp, 0, sizeof(mp));
+  memset(&mo, 0, sizeof(mo));
+  if ((st = encode_rows_map(&mp, pi, dt, d, d, d, 128)) != KVRQ_OK) return st;
+  if (mode == PQ_QDQ && (st = encode_rows_map(&mx, x, dt, n, d, ldx, 128)) != KVRQ_OK) return st;
+  if ((st = encode_rows_map(&mo, xhat, dt, n, d, ldo, 128)) != KVRQ_OK) return st;
+  if (mode != PQ_QDQ) mx = mo;
+  PqArgs a{};
+  a.n = n;
+  a.centroids = centroids;
+  a.codes_out = codes_out;
+  a.codes_in = codes_in;
+  a.ldc = ldc;
+  a.status = di->status;
+  return launch_status(name, launch_pq(mode, dt, mx, mp, mo, a, static_cast<cudaStream_t>(stream), di->num_sms));
+}
+
 // The QJL sign sketch of arbitrary rows (tiled kernel, sketch epilogue).
 static kvrq_status qjl_call(void* stream, const void* r, kvrq_dtype dt, int64_t n, int d, int64_t ldr, const void* T,
                             int m, uint32_t* signs, int64_t lds, float* gammas, int64_t ldn) {
@@ -535,6 +575,19 @@ kvrq_status rq_quantize_dequantize(void* stream, const void* x, kvrq_dtype xdtyp
                                    int64_t ldc, float* norms, void* xhat, int64_t ldo) {
   return rq_call("rq_quantize_dequantize", RQ_QDQ, stream, x, xdtype, ldx, nullptr, codes, ldc, nullptr, norms, n, d,
                  rotors, centroids, bits, xhat, xdtype, ldo);
+}
+
+kvrq_status pq_quantize_dequantize(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,
+                                   const void* pi, const float* centroids, uint32_t* codes, int64_t ldc, void* xhat,
+                                   int64_t ldo) {
+  return pq_call("pq_quantize_dequantize", PQ_QDQ, stream, x, xdtype, ldx, n, d, pi, centroids, codes, nullptr, ldc,
+                 xhat, ldo);
+}
+
+kvrq_status pq_dequantize(void* stream, const uint32_t* codes, int64_t ldc, int64_t n, int d, const void* pi,
+                          const float* centroids, void* xhat, kvrq_dtype odtype, int64_t ldo) {
+  return pq_call("pq_dequantize", PQ_DQ, stream, nullptr, odtype, 0, n, d, pi, centroids, nullptr, codes, ldc, xhat,
+                 ldo);
 }
 
 kvrq_status rq4_quantize(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,

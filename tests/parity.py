@@ -277,3 +277,71 @@ def record(kind, value, total):
     import os
     test = os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
     REPORT.append((test, kind, value, total))
+
+
+# ---------------------------------------------------------------- PolarQuant
+
+def polar_angle_margins(x64, Pi64, ref):
+    """Per level, a margin (radians) per angle within which the CUDA path may take the neighbouring code.
+
+    The kernel forms y = Pi x with float32 sums of exact 16-bit products: |dy_i| <= e_i = LAMBDA sqrt(d) 2^-24
+    sum_k |Pi_ik x_k|. A level-1 angle atan2(b, a) of a pair of radius r moves by at most (e_a + e_b) / r; a
+    float32 radius carries the errors of its pair plus two roundings (2^-22 r), and a level-l angle of radii
+    (r_a, r_b) moves by (dr_a + dr_b) / r. The decision itself (products of float32 cosines and sines)
+    adds 2^-21. Margin = max(1e-5, 2 x that bound)."""
+    x64 = np.asarray(x64, dtype=np.float64)
+    Pi64 = np.asarray(Pi64, dtype=np.float64)
+    d = x64.shape[1]
+    e = LAMBDA * np.sqrt(d) * 2.0 ** -24 * (np.abs(x64) @ np.abs(Pi64).T)
+    y = x64 @ Pi64.T
+    r = y
+    dr = e
+    out = []
+    for level in range(len(ref["angles"])):
+        a, b = r[:, 0::2], r[:, 1::2]
+        da, db = dr[:, 0::2], dr[:, 1::2]
+        rad = np.sqrt(a * a + b * b)
+        with np.errstate(divide="ignore", invalid="ignore"):
+            dth = np.where(rad > 0, (da + db) / rad, np.inf) + 2.0 ** -21
+        out.append(np.maximum(1e-5, 2.0 * dth))
+        dr = da + db + 2.0 ** -22 * rad
+        r = rad
+    return out
+
+
+def compare_polar_codes(gpu_words, ref, books, margins):
+    """GPU PolarQuant code rows [N, 16] against the oracle's quantization `ref`: every level's codes equal
+    except where the oracle's angle is within its margin of a boundary (then the neighbouring code, modulo
+    16 at level 1 whose boundaries include 0 = 2 pi), and the 16-bit radii equal or one fp16 step apart.
+    Records the mismatches; returns the mask of rows with any."""
+    gw = np.asarray(gpu_words, dtype=np.uint32)
+    level_words = [(0, 8, 4), (8, 10, 2), (10, 11, 2), (11, 12, 2)]
+    bad_rows = np.zeros(gw.shape[0], dtype=bool)
+    total = 0
+    for lv, (w0, w1, bits) in enumerate(level_words):
+        n_codes = 64 >> lv
+        g = ocodes.unpack(gw[:, w0:w1], n_codes, bits)
+        o = np.asarray(ref["codes"][lv])
+        diff = g != o
+        if diff.any():
+            c = np.asarray(books[lv], dtype=np.float64)
+            t = 0.5 * (c[:-1] + c[1:])
+            if lv == 0:
+                t = np.concatenate([[0.0, 2.0 * np.pi], t])
+            th = np.asarray(ref["angles"][lv])
+            dist = np.min(np.abs(th[..., None] - t), axis=-1)
+            far = diff & ~(dist < margins[lv])
+            assert not far.any(), "level %d codes differ away from a boundary at %s (gpu %s, oracle %s)" % (
+                lv + 1, np.argwhere(far)[:5].tolist(), g[far][:5], o[far][:5])
+            step = np.abs(g[diff] - o[diff])
+            if lv == 0:
+                step = np.minimum(step, 16 - step)
+            assert np.all(step == 1), "level %d: boundary mismatch to a non-adjacent code" % (lv + 1)
+            bad_rows |= diff.any(axis=1)
+        total += int(diff.sum())
+    assert np.all((gw[:, 11] >> 16) == 0), "nonzero padding bits"
+    rad = gw[:, 12:16].view(np.uint16).astype(np.int64)
+    orad = np.asarray(ref["radii"]).astype(np.float16).view(np.uint16).astype(np.int64)
+    assert np.all(np.abs(rad - orad) <= 1), "fp16 radii differ by more than one step"
+    record("polar code boundary ties", total, int(gw.shape[0]) * 120)
+    return bad_rows

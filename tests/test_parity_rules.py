@@ -133,3 +133,69 @@ def test_score_tolerance_accepts_fp16_restatement(method, bits):
         with pytest.raises(AssertionError):
             compare_scores(score.direct(method, q, dict(keys, signs_words=sw[None]), p, bits), ref, floor,
                            report=False)
+
+
+def _float32_polar_words(x, Pi, books32):
+    """PolarQuant code rows as a float32 pipeline forms them: y = Pi x in float32, level-1 sectors against
+    tan(pi/8), 1, tan(3 pi/8), level >= 2 codes by comparing b cos t with a sin t, float32 radii."""
+    F = np.float32
+    y = (x.astype(F) @ Pi.astype(F).T).astype(F)
+    t8, t38 = F(np.tan(np.pi / 8)), F(np.tan(3 * np.pi / 8))
+    n = x.shape[0]
+    words = np.zeros((n, 16), dtype=np.uint32)
+    a, b = y[:, 0::2], y[:, 1::2]
+    q = np.where(b >= 0, np.where((a > 0) | (b == 0), 0, 1), np.where(a < 0, 2, 3))
+    xx = np.choose(q, [a, b, -a, -b]).astype(F)
+    yy = np.choose(q, [b, -a, -b, a]).astype(F)
+    k1 = 4 * q + (yy > (xx * t8).astype(F)) + (yy > xx) + (yy > (xx * t38).astype(F))
+    r = np.sqrt((a * a + b * b).astype(F)).astype(F)
+    codes = [k1]
+    for lv in range(1, 4):
+        c = books32[lv]
+        t = (F(0.5) * (c[:-1] + c[1:])).astype(F)
+        ct, st = np.cos(t).astype(F), np.sin(t).astype(F)
+        ra, rb = r[:, 0::2], r[:, 1::2]
+        h1 = (rb * ct[1]).astype(F) > (ra * st[1]).astype(F)
+        hi = (rb * ct[2]).astype(F) > (ra * st[2]).astype(F)
+        lo = (rb * ct[0]).astype(F) > (ra * st[0]).astype(F)
+        codes.append(np.where(h1, 2 + hi, lo.astype(int)))
+        r = np.sqrt((ra * ra + rb * rb).astype(F)).astype(F)
+    words[:, 0:8] = ocodes.pack(codes[0], 4)
+    words[:, 8:10] = ocodes.pack(codes[1], 2)
+    words[:, 10:11] = ocodes.pack(codes[2], 2)
+    words[:, 11:12] = ocodes.pack(codes[3], 2)
+    h = r.astype(np.float16).view(np.uint16).astype(np.uint32)
+    words[:, 12:16] = h[:, 0::2] | (h[:, 1::2] << 16)
+    return words
+
+
+def test_polar_rule_accepts_float32_restatement_and_rejects_planted_errors():
+    from oracle import polar
+    from tests.parity import compare_polar_codes, polar_angle_margins
+    d = 128
+    rng = np.random.default_rng(3)
+    x = _fp16(rng.standard_normal((2000, d)) * np.exp(0.5 * rng.standard_normal((2000, 1))))
+    x[10] = 0
+    Pi = _fp16(params.rotation(d, 2))
+    books32 = [polar.lloyd_max_angles(lv, b)[0].astype(np.float32) for lv, b in enumerate((4, 2, 2, 2), 1)]
+    books = [b.astype(np.float64) for b in books32]
+    ref = polar.quantize(x, Pi, books)
+    margins = polar_angle_margins(x, Pi, ref)
+    words = _float32_polar_words(x, Pi, books32)
+    compare_polar_codes(words, ref, books, margins)
+    assert np.median(margins[0]) < 1e-4  # the margins stay small for typical pairs
+    # a level-2 code moved away from its boundary, and a radius moved by two fp16 steps, fail
+    th = np.asarray(ref["angles"][1])
+    t = 0.5 * (books[1][:-1] + books[1][1:])
+    far = np.min(np.abs(th[..., None] - t), axis=-1) > 1e-2
+    i, j = np.argwhere(far)[0]
+    bad = words.copy()
+    cd = ocodes.unpack(bad[:, 8:10], 32, 2)
+    cd[i, j] = (cd[i, j] + 1) % 4
+    bad[:, 8:10] = ocodes.pack(cd, 2)
+    with pytest.raises(AssertionError):
+        compare_polar_codes(bad, ref, books, margins)
+    bad = words.copy()
+    bad[5, 12] += 2
+    with pytest.raises(AssertionError):
+        compare_polar_codes(bad, ref, books, margins)
