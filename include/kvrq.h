@@ -338,6 +338,71 @@ kvrq_status kv_score_packed(void* stream, kvrq_method method, const void* q, kvr
                             const float* rotors, const void* pi, kvrq_dtype pi_dtype, const uint16_t* T,
                             const float* centroids, float* scores, int64_t ld_scores);
 
+/* ================================================================ paged KV cache
+ * ["TurboQuant + RotorQuant", "Post-Prefill Quantization": the prefill cache is
+ * quantized in bulk, then one new key and value per decode step; with many sequences
+ * of different lengths the packed rows live in pages of a pool]
+ * A paged cache keeps, for every pool head p = layer * kv_heads + k (one per layer
+ * and KV head), its packed rows in slots of a pool: codes + p * codes_pool_stride +
+ * slot * ldc, signs + p * signs_pool_stride + slot * lds, norms / gammas (and value
+ * norms) + p * tok_pool_stride + slot. Sequence s owns pages of page_tokens slots
+ * listed by its block table (the kvrq_pages_* bookkeeping below hands them out):
+ * token t < seq_lens[s] sits at slot page_tokens * block_tables[s * ld_table +
+ * t / page_tokens] + t % page_tokens. Head h of a call is (layer, sequence, KV
+ * head), h = (layer * n_seqs + s) * kv_heads + k, so n_heads is a multiple of n_seqs
+ * x kv_heads. block_tables and seq_lens are device int32 arrays the kernels read;
+ * the caller keeps every slot they name inside the pools. */
+typedef struct kvrq_paged {
+  const int32_t* block_tables; /* device [n_seqs][ld_table] */
+  int64_t ld_table;            /* >= ceil(max_tokens / page_tokens) */
+  const int32_t* seq_lens;     /* device [n_seqs], tokens of each sequence (<= max_tokens) */
+  int32_t page_tokens;         /* slots per page, >= 1 (a power of two >= 16 keeps bulk copies) */
+  int32_t n_seqs;
+  int32_t kv_heads;
+} kvrq_paged;
+
+/* kv_score_packed over a paged cache: scores [(h*group + g)*ld_scores + t] for
+ * t < seq_lens[s] of head h's sequence (others untouched); max_tokens bounds the
+ * sequence lengths (it sizes the launch, ld_scores >= max_tokens). Other arguments
+ * as kv_score_packed, the head strides stepping pool heads. */
+kvrq_status kv_score_packed_paged(void* stream, kvrq_method method, const void* q, kvrq_dtype qdtype, int64_t ldq,
+                                  int64_t n_heads, int group, int d, int bits, int m, const uint32_t* codes,
+                                  int64_t ldc, int64_t codes_pool_stride, const uint32_t* signs, int64_t lds,
+                                  int64_t signs_pool_stride, const float* norms, const float* gammas,
+                                  int64_t tok_pool_stride, const kvrq_paged* paged, int64_t max_tokens,
+                                  const float* rotors, const void* pi, kvrq_dtype pi_dtype, const uint16_t* T,
+                                  const float* centroids, float* scores, int64_t ld_scores);
+
+/* kv_attention_packed over a paged cache (keys and values share the slots): every
+ * query row of head h attends over the seq_lens[s] tokens of its sequence (a
+ * sequence of no tokens gives a zero output). Runs where
+ * kvrq_attention_uses_tensor_cores is 1; other configurations return
+ * KVRQ_EUNSUPPORTED. workspace: kvrq_attention_workspace_bytes(n_heads, group,
+ * max_tokens) bytes. Other arguments as kv_attention_packed, the head strides
+ * stepping pool heads. */
+kvrq_status kv_attention_packed_paged(void* stream, kvrq_method k_method, const void* q, kvrq_dtype qdtype,
+                                      int64_t ldq, int64_t n_heads, int group, int d, float scale, int k_bits, int m,
+                                      const uint32_t* k_codes, int64_t ldk, int64_t k_pool_stride,
+                                      const uint32_t* k_signs, int64_t lds, int64_t s_pool_stride,
+                                      const float* k_norms, const float* k_gammas, const float* k_rotors,
+                                      const void* pi, kvrq_dtype pi_dtype, const uint16_t* T,
+                                      const float* k_centroids, const uint32_t* v_codes, int64_t ldv,
+                                      int64_t v_pool_stride, const float* v_norms, int v_bits,
+                                      const float* v_rotors, const float* v_centroids, int64_t tok_pool_stride,
+                                      const kvrq_paged* paged, int64_t max_tokens, void* out, kvrq_dtype odtype,
+                                      int64_t ldo, void* workspace, size_t workspace_bytes);
+
+/* Quantizes row r of x into pool row dst_rows[r] (device int64 [n_rows], e.g.
+ * p * slots_per_pool + slot of the new token): codes + dst_rows[r] * ldc, signs +
+ * dst_rows[r] * lds, norms / gammas + dst_rows[r] * ldn, in one launch; the decode
+ * step of a paged cache. method and parameters as kv_cache_append; d = 128 with
+ * 16-byte aligned rows (TurboQuant: fp16 or bf16), else KVRQ_EUNSUPPORTED. */
+kvrq_status kv_cache_append_rows(void* stream, kvrq_method method, const void* x, kvrq_dtype xdtype, int64_t n_rows,
+                                 int d, int64_t ldx, int bits, const float* rotors, const void* pi, const uint16_t* T,
+                                 int m, const float* centroids, const int64_t* dst_rows, uint32_t* codes,
+                                 int64_t ldc, uint32_t* signs, int64_t lds, float* norms, float* gammas,
+                                 int64_t ldn);
+
 /* ================================================================ decode-step append
  * [RQ "Post-Prefill Quantization": each decode step quantizes the new key (and
  * value) for storage] Quantizes one new vector per cache row (a row = one

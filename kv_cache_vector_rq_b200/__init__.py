@@ -430,6 +430,115 @@ def kv_cache_append(method, x, slot, bits, centroids, codes, norms, rotors=None,
         codes.stride(0), sp, signs.stride(0) if signs is not None else 0, np_, gp, norms.stride(0)))
 
 
+# ----------------------------------------------------------------------------- paged cache
+
+def _paged(block_tables, seq_lens, page_tokens, n_seqs, kv_heads):
+    torch = _torch()
+    if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32 or not block_tables.is_cuda:
+        raise TypeError("block_tables and seq_lens must be int32 CUDA tensors")
+    if block_tables.dim() != 2 or block_tables.stride(1) != 1 or not seq_lens.is_contiguous():
+        raise ValueError("block_tables must be [n_seqs, ld_table] with unit inner stride")
+    return _lib.KvrqPaged(block_tables.data_ptr(), block_tables.stride(0), seq_lens.data_ptr(), page_tokens, n_seqs,
+                          kv_heads)
+
+
+def _pool(t, name):
+    """(pointer, row stride, pool-head stride) of a pool tensor [pool_heads, slots, W] (or [pool_heads, slots])."""
+    if t is None:
+        return None, 0, 0
+    if not t.is_cuda or t.stride(-1) != 1:
+        raise ValueError("%s must be a CUDA tensor with unit inner stride" % name)
+    return t.data_ptr(), (t.stride(1) if t.dim() == 3 else 1), t.stride(0)
+
+
+def kv_score_packed_paged(method, q, codes, norms, bits, block_tables, seq_lens, page_tokens, n_seqs, kv_heads,
+                          max_tokens, centroids, rotors=None, pi=None, T=None, signs=None, gammas=None, scores=None,
+                          stream=None):
+    """Scores from a paged packed cache (kv_score_packed_paged in include/kvrq.h).
+
+    q: [n_heads, group, d], head h = (layer * n_seqs + s) * kv_heads + k. Pools: codes [pool_heads, slots, W],
+    norms/gammas [pool_heads, slots], signs [pool_heads, slots, m/32], pool head = layer * kv_heads + k.
+    block_tables [n_seqs, ld_table] and seq_lens [n_seqs] int32 CUDA. Returns scores [n_heads, group,
+    max_tokens] (entries t >= seq_lens[s] are left as they were)."""
+    torch = _torch()
+    n_heads, group, d = q.shape
+    if not q.is_contiguous():
+        raise ValueError("q must be contiguous")
+    if scores is None:
+        scores = torch.zeros((n_heads, group, max_tokens), dtype=torch.float32, device=q.device)
+    m = T.shape[0] if T is not None else d
+    cp, ldc, cps = _pool(codes, "codes")
+    sp, lds, sps = _pool(signs, "signs")
+    if norms.stride(-1) != 1 or (gammas is not None and gammas.stride() != norms.stride()):
+        raise ValueError("norms/gammas must share one [pool_heads, slots] layout")
+    pg = _paged(block_tables, seq_lens, page_tokens, n_seqs, kv_heads)
+    pdt = _dtype_code(pi) if pi is not None else F16
+    _lib.check("kv_score_packed_paged", lib().kv_score_packed_paged(
+        _stream(stream), method, q.data_ptr(), _dtype_code(q), d, n_heads, group, d, bits, m, cp, ldc, cps, sp, lds,
+        sps, _ptr(norms, "norms", torch.float32), _ptr(gammas, "gammas", torch.float32), norms.stride(0),
+        ctypes.byref(pg), max_tokens, _ptr(rotors, "rotors", torch.float32), _ptr(pi, "pi"), pdt,
+        _ptr(T, "T", torch.float16), _ptr(centroids, "centroids", torch.float32), scores.data_ptr(),
+        scores.stride(1)))
+    return scores
+
+
+def kv_attention_packed_paged(k_method, q, k_codes, k_norms, k_bits, v_codes, v_norms, v_bits, block_tables,
+                              seq_lens, page_tokens, n_seqs, kv_heads, max_tokens, k_centroids, v_rotors,
+                              v_centroids, scale=None, k_rotors=None, pi=None, T=None, k_signs=None, k_gammas=None,
+                              out=None, out_dtype=None, workspace=None, stream=None):
+    """Decode attention over a paged packed cache (kv_attention_packed_paged in include/kvrq.h); pools and
+    heads as kv_score_packed_paged, values v_codes [pool_heads, slots, Wv] and v_norms sharing the key norms'
+    layout. Returns out [n_heads, group, d]."""
+    torch = _torch()
+    n_heads, group, d = q.shape
+    if not q.is_contiguous():
+        raise ValueError("q must be contiguous")
+    if scale is None:
+        scale = 1.0 / float(np.sqrt(d))
+    if out is None:
+        out = torch.empty((n_heads, group, d), dtype=out_dtype or torch.float32, device=q.device)
+    m = T.shape[0] if T is not None else d
+    need = attention_workspace_bytes(n_heads, group, max_tokens)
+    if workspace is None:
+        workspace = torch.empty((max(need, 16) + 15) // 16 * 4, dtype=torch.float32, device=q.device)
+    kp, ldk, kps = _pool(k_codes, "k_codes")
+    sp, lds, sps = _pool(k_signs, "k_signs")
+    vp, ldv, vps = _pool(v_codes, "v_codes")
+    if k_norms.stride(-1) != 1 or v_norms.stride() != k_norms.stride() or (
+            k_gammas is not None and k_gammas.stride() != k_norms.stride()):
+        raise ValueError("k_norms, k_gammas and v_norms must share one [pool_heads, slots] layout")
+    pg = _paged(block_tables, seq_lens, page_tokens, n_seqs, kv_heads)
+    pdt = _dtype_code(pi) if pi is not None else F16
+    _lib.check("kv_attention_packed_paged", lib().kv_attention_packed_paged(
+        _stream(stream), k_method, q.data_ptr(), _dtype_code(q), d, n_heads, group, d, float(scale), k_bits, m, kp,
+        ldk, kps, sp, lds, sps, _ptr(k_norms, "k_norms", torch.float32), _ptr(k_gammas, "k_gammas", torch.float32),
+        _ptr(k_rotors, "k_rotors", torch.float32), _ptr(pi, "pi"), pdt, _ptr(T, "T", torch.float16),
+        _ptr(k_centroids, "k_centroids", torch.float32), vp, ldv, vps, _ptr(v_norms, "v_norms", torch.float32),
+        v_bits, _ptr(v_rotors, "v_rotors", torch.float32), _ptr(v_centroids, "v_centroids", torch.float32),
+        k_norms.stride(0), ctypes.byref(pg), max_tokens, out.data_ptr(), _dtype_code(out), out.stride(1),
+        workspace.data_ptr(), workspace.numel() * workspace.element_size()))
+    return out
+
+
+def kv_cache_append_rows(method, x, dst_rows, bits, centroids, codes, norms, rotors=None, pi=None, T=None,
+                         signs=None, gammas=None, stream=None):
+    """Quantize row r of x [n, d] into pool row dst_rows[r] (int64 CUDA [n]) of flat pools: codes [rows, W],
+    norms/gammas [rows], signs [rows, m/32] (e.g. a [pool_heads, slots, W] pool viewed as [pool_heads * slots,
+    W], dst = pool_head * slots + slot)."""
+    torch = _torch()
+    n, d = x.shape
+    if dst_rows.dtype != torch.int64 or not dst_rows.is_cuda or not dst_rows.is_contiguous():
+        raise TypeError("dst_rows must be a contiguous int64 CUDA tensor")
+    xp, ldx = _rows(x, "x")
+    m = T.shape[0] if T is not None else d
+    _lib.check("kv_cache_append_rows", lib().kv_cache_append_rows(
+        _stream(stream), method, xp, _dtype_code(x), n, d, ldx, bits, _ptr(rotors, "rotors", torch.float32),
+        _ptr(pi, "pi"), _ptr(T, "T", torch.float16), m, _ptr(centroids, "centroids", torch.float32),
+        dst_rows.data_ptr(), codes.data_ptr(), codes.stride(0), signs.data_ptr() if signs is not None else None,
+        signs.stride(0) if signs is not None else 0, norms.data_ptr(), gammas.data_ptr() if gammas is not None else None,
+        norms.stride(0)))
+
+
 def attention_workspace_bytes(n_heads, group, n_tokens):
     return int(lib().kvrq_attention_workspace_bytes(n_heads, group, n_tokens))
 

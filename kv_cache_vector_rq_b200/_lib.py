@@ -82,6 +82,21 @@ SIGNATURES = {
     "pq_quantize_dequantize": (c_int, [c_vp, c_vp, c_int, c_i64, c_int, c_i64, c_vp, c_vp, c_vp, c_i64, c_vp, c_i64]),
     # stream, codes, ldc, n, d, pi, centroids, xhat, odtype, ldo
     "pq_dequantize": (c_int, [c_vp, c_vp, c_i64, c_i64, c_int, c_vp, c_vp, c_vp, c_int, c_i64]),
+    # stream, method, q, qdtype, ldq, n_heads, group, d, bits, m, codes, ldc, codes_pool_stride, signs, lds,
+    # signs_pool_stride, norms, gammas, tok_pool_stride, paged, max_tokens, rotors, pi, pi_dtype, T, centroids,
+    # scores, ld_scores
+    "kv_score_packed_paged": (c_int, [c_vp, c_int, c_vp, c_int, c_i64, c_i64, c_int, c_int, c_int, c_int, c_vp,
+                                      c_i64, c_i64, c_vp, c_i64, c_i64, c_vp, c_vp, c_i64, c_vp, c_i64, c_vp, c_vp,
+                                      c_int, c_vp, c_vp, c_vp, c_i64]),
+    # as kv_attention_packed with pool strides, then paged, max_tokens before out
+    "kv_attention_packed_paged": (c_int, [c_vp, c_int, c_vp, c_int, c_i64, c_i64, c_int, c_int, ctypes.c_float,
+                                          c_int, c_int, c_vp, c_i64, c_i64, c_vp, c_i64, c_i64, c_vp, c_vp, c_vp,
+                                          c_vp, c_int, c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_int, c_vp, c_vp,
+                                          c_i64, c_vp, c_i64, c_vp, c_int, c_i64, c_vp, ctypes.c_size_t]),
+    # stream, method, x, xdtype, n_rows, d, ldx, bits, rotors, pi, T, m, centroids, dst_rows, codes, ldc, signs,
+    # lds, norms, gammas, ldn
+    "kv_cache_append_rows": (c_int, [c_vp, c_int, c_vp, c_int, c_i64, c_int, c_i64, c_int, c_vp, c_vp, c_vp, c_int,
+                                     c_vp, c_vp, c_vp, c_i64, c_vp, c_i64, c_vp, c_vp, c_i64]),
     "kvrq_attention_uses_tensor_cores": (c_int, [c_int, c_int, c_int, c_int]),
     "kvrq_pages_create": (c_int, [c_i64, c_int, ctypes.POINTER(c_vp)]),
     "kvrq_pages_destroy": (None, [c_vp]),
@@ -124,3 +139,9 @@ def check(name, status):
     if status != 0:
         msg = load().kvrq_last_error_string().decode()
         raise KvrqError(name, status, msg)
+
+
+class KvrqPaged(ctypes.Structure):
+    """struct kvrq_paged of include/kvrq.h."""
+    _fields_ = [("block_tables", ctypes.c_void_p), ("ld_table", ctypes.c_int64), ("seq_lens", ctypes.c_void_p),
+                ("page_tokens", ctypes.c_int32), ("n_seqs", ctypes.c_int32), ("kv_heads", ctypes.c_int32)]

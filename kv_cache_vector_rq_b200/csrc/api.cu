@@ -150,7 +150,8 @@ static kvrq_status launch_status(const char* where, cudaError_t e) {
 static kvrq_status rq_call(const char* name, int mode, void* stream, const void* x, kvrq_dtype xdt, int64_t ldx,
                            const uint32_t* codes_in, uint32_t* codes_out, int64_t ldc, const float* norms_in,
                            float* norms_out, int64_t n, int d, const float* rotors, const float* centroids, int bits,
-                           void* xhat, kvrq_dtype odt, int64_t ldo, int64_t ldn = 1, int cpg = 3) {
+                           void* xhat, kvrq_dtype odt, int64_t ldo, int64_t ldn = 1, int cpg = 3,
+                           const int64_t* out_rows = nullptr) {
   if (ldn < 1) return set_errorf(KVRQ_EINVAL, "%s: norm row stride < 1", name);
   if (n < 0) return set_errorf(KVRQ_EINVAL, "%s: n < 0", name);
   if (d < 2 || d > (1 << 20)) return set_errorf(KVRQ_EINVAL, "%s: d must be in 2..2^20", name);
@@ -204,6 +205,7 @@ static kvrq_status rq_call(const char* name, int mode, void* stream, const void*
   a.ldn = ldn;
   a.status = di->status;
   a.codes_per_group = cpg;
+  a.out_rows = out_rows;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   const kvrq_dtype tdt = q_side ? xdt : odt;
@@ -224,6 +226,7 @@ static kvrq_status rq_call(const char* name, int mode, void* stream, const void*
   if (cpg == 4)
     return set_errorf(KVRQ_EUNSUPPORTED, "%s: the four-grade layout needs 16-byte aligned rows (and one dtype for "
                                          "the fused call)", name);
+  if (out_rows) return set_errorf(KVRQ_EUNSUPPORTED, "%s: destination rows need d = 128 and 16-byte aligned rows", name);
   // any d: rows streamed by bulk copy when they start 16-byte aligned and fit its row buffers
   bool wide = true;
   if (q_side) wide = wide && rows_aligned16(x, ldx, xdt);
@@ -372,7 +375,8 @@ static kvrq_status tq_call(const char* name, int mode, void* stream, const void*
                            int bits, uint32_t* codes_out, const uint32_t* codes_in, int64_t ldc, uint32_t* signs_out,
                            const uint32_t* signs_in, int64_t lds, float* gammas_out, const float* gammas_in,
                            float* norms_out, const float* norms_in, void* xhat, int64_t ldo, int64_t ldn = 1,
-                           void* ws = nullptr, size_t ws_bytes = 0, bool static_scratch = false) {
+                           void* ws = nullptr, size_t ws_bytes = 0, bool static_scratch = false,
+                           const int64_t* out_rows = nullptr) {
   const bool prod = mode == TQ_PROD_Q || mode == TQ_DQ_PROD;
   if (ldn < 1) return set_errorf(KVRQ_EINVAL, "%s: norm row stride < 1", name);
   const bool q_side = mode == TQ_MSE_Q || mode == TQ_MSE_QDQ || mode == TQ_PROD_Q;
@@ -386,6 +390,8 @@ static kvrq_status tq_call(const char* name, int mode, void* stream, const void*
     return set_errorf(KVRQ_EUNSUPPORTED, "%s: the tensor-core paths need d a multiple of 128 (<= 16384)", name);
   if (prod && m != d) return set_errorf(KVRQ_EUNSUPPORTED, "%s: the QJL projection needs m = d", name);
   const bool tiled = d != 128 || dt == KVRQ_F32;
+  if (out_rows && tiled)
+    return set_errorf(KVRQ_EUNSUPPORTED, "%s: destination rows need d = 128 and fp16 or bf16 vectors", name);
   const int cbits = prod ? bits - 1 : bits;
   const int64_t W = kvrq_packed_words(d, cbits);
   if (n == 0) return KVRQ_OK;
@@ -452,6 +458,7 @@ static kvrq_status tq_call(const char* name, int mode, void* stream, const void*
   a.lds = lds;
   a.ldn = ldn;
   a.status = di->status;
+  a.out_rows = out_rows;
   return launch_status(name, launch_tq(mode, dt, cbits, mx, mp, mt, mo, a, static_cast<cudaStream_t>(stream), di->num_sms));
 }
 
@@ -662,13 +669,28 @@ kvrq_status qjl_sketch(void* stream, const void* r, kvrq_dtype rdtype, int64_t n
   return qjl_call(stream, r, rdtype, n, d, ldr, T, m, signs, lds, gammas, ldn);
 }
 
-kvrq_status kv_score_packed(void* stream, kvrq_method method, const void* q, kvrq_dtype qdtype, int64_t ldq,
-                            int64_t n_heads, int group, int d, int bits, int m, const uint32_t* codes, int64_t ldc,
-                            int64_t codes_head_stride, const uint32_t* signs, int64_t lds, int64_t signs_head_stride,
-                            const float* norms, const float* gammas, int64_t tok_head_stride, int64_t n_tokens,
-                            const float* rotors, const void* pi, kvrq_dtype pi_dtype, const uint16_t* T,
-                            const float* centroids, float* scores, int64_t ld_scores) {
-  const char* name = "kv_score_packed";
+}  // extern "C"
+
+// Checks of a paged-cache descriptor shared by the paged calls (tables on the device are not read).
+static kvrq_status check_paged(const char* name, const kvrq_paged* pg, int64_t n_heads, int64_t max_tokens) {
+  if (!pg->block_tables || !pg->seq_lens || !aligned(pg->block_tables, 4) || !aligned(pg->seq_lens, 4))
+    return set_errorf(KVRQ_EINVAL, "%s: block_tables and seq_lens are required", name);
+  if (pg->page_tokens < 1 || pg->n_seqs < 1 || pg->kv_heads < 1)
+    return set_errorf(KVRQ_EINVAL, "%s: page_tokens, n_seqs and kv_heads must be >= 1", name);
+  if (n_heads % ((int64_t)pg->n_seqs * pg->kv_heads) != 0)
+    return set_errorf(KVRQ_EINVAL, "%s: n_heads must be a multiple of n_seqs x kv_heads", name);
+  if (pg->ld_table < (max_tokens + pg->page_tokens - 1) / pg->page_tokens)
+    return set_errorf(KVRQ_EINVAL, "%s: ld_table holds fewer pages than max_tokens needs", name);
+  return KVRQ_OK;
+}
+
+static kvrq_status score_call(const char* name, void* stream, kvrq_method method, const void* q, kvrq_dtype qdtype,
+                              int64_t ldq, int64_t n_heads, int group, int d, int bits, int m, const uint32_t* codes,
+                              int64_t ldc, int64_t codes_head_stride, const uint32_t* signs, int64_t lds,
+                              int64_t signs_head_stride, const float* norms, const float* gammas,
+                              int64_t tok_head_stride, int64_t n_tokens, const kvrq_paged* pg, const float* rotors,
+                              const void* pi, kvrq_dtype pi_dtype, const uint16_t* T, const float* centroids,
+                              float* scores, int64_t ld_scores) {
   const bool prod = method == KVRQ_TQ_PROD;
   if (method != KVRQ_RQ_MSE && method != KVRQ_TQ_MSE && method != KVRQ_TQ_PROD)
     return set_error(KVRQ_EINVAL, "kv_score_packed: unknown method");
@@ -684,17 +706,21 @@ kvrq_status kv_score_packed(void* stream, kvrq_method method, const void* q, kvr
   const int64_t W = kvrq_packed_words(ncode, cbits);
   if (n_heads == 0 || n_tokens == 0) return KVRQ_OK;
   if (!q || !codes || !norms || !centroids || !scores) return set_error(KVRQ_EINVAL, "kv_score_packed: NULL argument");
-  if (ldc < W || ld_scores < n_tokens || tok_head_stride < n_tokens || codes_head_stride < n_tokens * ldc)
+  // (a paged pool's rows are named by the tables: its strides are the caller's)
+  if (ldc < W || ld_scores < n_tokens ||
+      (!pg && (tok_head_stride < n_tokens || codes_head_stride < n_tokens * ldc)))
     return set_error(KVRQ_EINVAL, "kv_score_packed: strides too small");
   if (method == KVRQ_RQ_MSE && (!rotors || !aligned(rotors, 16)))
     return set_error(KVRQ_EINVAL, "kv_score_packed: rotors (16-byte aligned) required");
   if (method != KVRQ_RQ_MSE && (!pi || (pi_dtype != KVRQ_F16 && pi_dtype != KVRQ_BF16)))
     return set_error(KVRQ_EINVAL, "kv_score_packed: pi (fp16 or bf16) required");
-  if (prod && (!signs || !gammas || !T || lds < m / 32 || signs_head_stride < n_tokens * lds))
+  if (prod && (!signs || !gammas || !T || lds < m / 32 || (!pg && signs_head_stride < n_tokens * lds)))
     return set_error(KVRQ_EINVAL, "kv_score_packed: signs, gammas and T required for prod");
   if (!aligned(codes, 4) || !aligned(norms, 4) || !aligned(scores, 4))
     return set_error(KVRQ_EINVAL, "kv_score_packed: misaligned pointer");
   if (n_heads > 65535) return set_error(KVRQ_EUNSUPPORTED, "kv_score_packed: more than 65535 heads");
+  kvrq_status pst;
+  if (pg && (pst = check_paged(name, pg, n_heads, n_tokens)) != KVRQ_OK) return pst;
 
   DeviceInfo* di;
   kvrq_status st = current_device(&di);
@@ -739,8 +765,42 @@ kvrq_status kv_score_packed(void* stream, kvrq_method method, const void* q, kvr
   a.scores = scores;
   a.ld_scores = ld_scores;
   a.status = di->status;
+  if (pg) {
+    a.block_tables = pg->block_tables;
+    a.ld_table = pg->ld_table;
+    a.seq_lens = pg->seq_lens;
+    a.page_tokens = pg->page_tokens;
+    a.n_seqs = pg->n_seqs;
+    a.kv_heads = pg->kv_heads;
+  }
   const int nb = rows_needed <= 16 ? 16 : (rows_needed <= 32 ? 32 : 64);
   return launch_status(name, launch_score(method, nb, cbits, a, static_cast<cudaStream_t>(stream)));
+}
+
+extern "C" {
+
+kvrq_status kv_score_packed(void* stream, kvrq_method method, const void* q, kvrq_dtype qdtype, int64_t ldq,
+                            int64_t n_heads, int group, int d, int bits, int m, const uint32_t* codes, int64_t ldc,
+                            int64_t codes_head_stride, const uint32_t* signs, int64_t lds, int64_t signs_head_stride,
+                            const float* norms, const float* gammas, int64_t tok_head_stride, int64_t n_tokens,
+                            const float* rotors, const void* pi, kvrq_dtype pi_dtype, const uint16_t* T,
+                            const float* centroids, float* scores, int64_t ld_scores) {
+  return score_call("kv_score_packed", stream, method, q, qdtype, ldq, n_heads, group, d, bits, m, codes, ldc,
+                    codes_head_stride, signs, lds, signs_head_stride, norms, gammas, tok_head_stride, n_tokens,
+                    nullptr, rotors, pi, pi_dtype, T, centroids, scores, ld_scores);
+}
+
+kvrq_status kv_score_packed_paged(void* stream, kvrq_method method, const void* q, kvrq_dtype qdtype, int64_t ldq,
+                                  int64_t n_heads, int group, int d, int bits, int m, const uint32_t* codes,
+                                  int64_t ldc, int64_t codes_pool_stride, const uint32_t* signs, int64_t lds,
+                                  int64_t signs_pool_stride, const float* norms, const float* gammas,
+                                  int64_t tok_pool_stride, const kvrq_paged* paged, int64_t max_tokens,
+                                  const float* rotors, const void* pi, kvrq_dtype pi_dtype, const uint16_t* T,
+                                  const float* centroids, float* scores, int64_t ld_scores) {
+  if (!paged) return set_error(KVRQ_EINVAL, "kv_score_packed_paged: paged is NULL");
+  return score_call("kv_score_packed_paged", stream, method, q, qdtype, ldq, n_heads, group, d, bits, m, codes, ldc,
+                    codes_pool_stride, signs, lds, signs_pool_stride, norms, gammas, tok_pool_stride, max_tokens,
+                    paged, rotors, pi, pi_dtype, T, centroids, scores, ld_scores);
 }
 
 size_t kvrq_attention_workspace_bytes(int64_t n_heads, int group, int64_t n_tokens) {
@@ -748,16 +808,18 @@ size_t kvrq_attention_workspace_bytes(int64_t n_heads, int group, int64_t n_toke
   return attn_workspace_bytes(n_heads, group, n_tokens);
 }
 
-kvrq_status kv_attention_packed(void* stream, kvrq_method k_method, const void* q, kvrq_dtype qdtype, int64_t ldq,
-                                int64_t n_heads, int group, int d, float scale, int k_bits, int m,
-                                const uint32_t* k_codes, int64_t ldk, int64_t k_head_stride, const uint32_t* k_signs,
-                                int64_t lds, int64_t s_head_stride, const float* k_norms, const float* k_gammas,
-                                const float* k_rotors, const void* pi, kvrq_dtype pi_dtype, const uint16_t* T,
-                                const float* k_centroids, const uint32_t* v_codes, int64_t ldv, int64_t v_head_stride,
-                                const float* v_norms, int v_bits, const float* v_rotors, const float* v_centroids,
-                                int64_t tok_head_stride, int64_t n_tokens, void* out, kvrq_dtype odtype, int64_t ldo,
-                                void* workspace, size_t workspace_bytes) {
-  const char* name = "kv_attention_packed";
+}  // extern "C"
+
+static kvrq_status attention_call(const char* name, void* stream, kvrq_method k_method, const void* q,
+                                  kvrq_dtype qdtype, int64_t ldq, int64_t n_heads, int group, int d, float scale,
+                                  int k_bits, int m, const uint32_t* k_codes, int64_t ldk, int64_t k_head_stride,
+                                  const uint32_t* k_signs, int64_t lds, int64_t s_head_stride, const float* k_norms,
+                                  const float* k_gammas, const float* k_rotors, const void* pi, kvrq_dtype pi_dtype,
+                                  const uint16_t* T, const float* k_centroids, const uint32_t* v_codes, int64_t ldv,
+                                  int64_t v_head_stride, const float* v_norms, int v_bits, const float* v_rotors,
+                                  const float* v_centroids, int64_t tok_head_stride, int64_t n_tokens,
+                                  const kvrq_paged* pg, void* out, kvrq_dtype odtype, int64_t ldo, void* workspace,
+                                  size_t workspace_bytes) {
   const bool prod = k_method == KVRQ_TQ_PROD;
   if (k_method != KVRQ_RQ_MSE && k_method != KVRQ_TQ_MSE && !prod)
     return set_error(KVRQ_EINVAL, "kv_attention_packed: unknown key method");
@@ -780,20 +842,28 @@ kvrq_status kv_attention_packed(void* stream, kvrq_method k_method, const void* 
   const int64_t Wv = kvrq_packed_words(3 * ((d + 2) / 3), v_bits);
   if (!q || !k_codes || !k_norms || !k_centroids || !v_codes || !v_norms || !v_rotors || !v_centroids || !out)
     return set_error(KVRQ_EINVAL, "kv_attention_packed: NULL argument");
-  if (ldk < Wk || k_head_stride < n_tokens * ldk || ldv < Wv || v_head_stride < n_tokens * ldv ||
-      tok_head_stride < n_tokens)
+  if (ldk < Wk || ldv < Wv ||
+      (!pg && (k_head_stride < n_tokens * ldk || v_head_stride < n_tokens * ldv || tok_head_stride < n_tokens)))
     return set_error(KVRQ_EINVAL, "kv_attention_packed: strides too small");
   if (k_method == KVRQ_RQ_MSE && (!k_rotors || !aligned(k_rotors, 16)))
     return set_error(KVRQ_EINVAL, "kv_attention_packed: key rotors (16-byte aligned) required");
   if (k_method != KVRQ_RQ_MSE && (!pi || (pi_dtype != KVRQ_F16 && pi_dtype != KVRQ_BF16) || !aligned(pi, 2)))
     return set_error(KVRQ_EINVAL, "kv_attention_packed: pi (fp16 or bf16) required");
-  if (prod && (!k_signs || !k_gammas || !T || !aligned(T, 2) || lds < m / 32 || s_head_stride < n_tokens * lds))
+  if (prod && (!k_signs || !k_gammas || !T || !aligned(T, 2) || lds < m / 32 ||
+               (!pg && s_head_stride < n_tokens * lds)))
     return set_error(KVRQ_EINVAL, "kv_attention_packed: signs, gammas and T required for prod");
   if (!aligned(v_rotors, 16)) return set_error(KVRQ_EINVAL, "kv_attention_packed: value rotors must be 16-byte aligned");
   if (!aligned(k_codes, 4) || !aligned(v_codes, 4) || !aligned(k_norms, 4) || !aligned(v_norms, 4) ||
       (prod && (!aligned(k_signs, 4) || !aligned(k_gammas, 4))) || !aligned(k_centroids, 4) ||
       !aligned(v_centroids, 4) || !aligned(q, qdtype == KVRQ_F32 ? 4 : 2) || !aligned(out, odtype == KVRQ_F32 ? 4 : 2))
     return set_error(KVRQ_EINVAL, "kv_attention_packed: misaligned pointer");
+  if (pg) {
+    kvrq_status pst = check_paged(name, pg, n_heads, n_tokens);
+    if (pst != KVRQ_OK) return pst;
+    if (!attn_tc_supported(k_method, kcb, v_bits, group))
+      return set_errorf(KVRQ_EUNSUPPORTED, "%s: a paged cache is read by the tensor-core kernel only "
+                                           "(kvrq_attention_uses_tensor_cores)", name);
+  }
   const size_t need = attn_workspace_bytes(n_heads, group, n_tokens);
   if (!workspace || workspace_bytes < need || !aligned(workspace, 16))
     return set_errorf(KVRQ_EINVAL, "kv_attention_packed: workspace of %zu bytes (16-byte aligned) required", need);
@@ -845,7 +915,76 @@ kvrq_status kv_attention_packed(void* stream, kvrq_method k_method, const void* 
   kvrq_status st = current_device(&di);
   if (st != KVRQ_OK) return st;
   a.status = di->status;
+  if (pg) {
+    a.block_tables = pg->block_tables;
+    a.ld_table = pg->ld_table;
+    a.seq_lens = pg->seq_lens;
+    a.page_tokens = pg->page_tokens;
+    a.n_seqs = pg->n_seqs;
+    a.kv_heads = pg->kv_heads;
+  }
   return launch_status(name, launch_attention(k_method, kcb, a, static_cast<cudaStream_t>(stream), di->num_sms));
+}
+
+extern "C" {
+
+kvrq_status kv_attention_packed(void* stream, kvrq_method k_method, const void* q, kvrq_dtype qdtype, int64_t ldq,
+                                int64_t n_heads, int group, int d, float scale, int k_bits, int m,
+                                const uint32_t* k_codes, int64_t ldk, int64_t k_head_stride, const uint32_t* k_signs,
+                                int64_t lds, int64_t s_head_stride, const float* k_norms, const float* k_gammas,
+                                const float* k_rotors, const void* pi, kvrq_dtype pi_dtype, const uint16_t* T,
+                                const float* k_centroids, const uint32_t* v_codes, int64_t ldv, int64_t v_head_stride,
+                                const float* v_norms, int v_bits, const float* v_rotors, const float* v_centroids,
+                                int64_t tok_head_stride, int64_t n_tokens, void* out, kvrq_dtype odtype, int64_t ldo,
+                                void* workspace, size_t workspace_bytes) {
+  return attention_call("kv_attention_packed", stream, k_method, q, qdtype, ldq, n_heads, group, d, scale, k_bits, m,
+                        k_codes, ldk, k_head_stride, k_signs, lds, s_head_stride, k_norms, k_gammas, k_rotors, pi,
+                        pi_dtype, T, k_centroids, v_codes, ldv, v_head_stride, v_norms, v_bits, v_rotors, v_centroids,
+                        tok_head_stride, n_tokens, nullptr, out, odtype, ldo, workspace, workspace_bytes);
+}
+
+kvrq_status kv_attention_packed_paged(void* stream, kvrq_method k_method, const void* q, kvrq_dtype qdtype,
+                                      int64_t ldq, int64_t n_heads, int group, int d, float scale, int k_bits, int m,
+                                      const uint32_t* k_codes, int64_t ldk, int64_t k_pool_stride,
+                                      const uint32_t* k_signs, int64_t lds, int64_t s_pool_stride,
+                                      const float* k_norms, const float* k_gammas, const float* k_rotors,
+                                      const void* pi, kvrq_dtype pi_dtype, const uint16_t* T,
+                                      const float* k_centroids, const uint32_t* v_codes, int64_t ldv,
+                                      int64_t v_pool_stride, const float* v_norms, int v_bits,
+                                      const float* v_rotors, const float* v_centroids, int64_t tok_pool_stride,
+                                      const kvrq_paged* paged, int64_t max_tokens, void* out, kvrq_dtype odtype,
+                                      int64_t ldo, void* workspace, size_t workspace_bytes) {
+  if (!paged) return set_error(KVRQ_EINVAL, "kv_attention_packed_paged: paged is NULL");
+  return attention_call("kv_attention_packed_paged", stream, k_method, q, qdtype, ldq, n_heads, group, d, scale,
+                        k_bits, m, k_codes, ldk, k_pool_stride, k_signs, lds, s_pool_stride, k_norms, k_gammas,
+                        k_rotors, pi, pi_dtype, T, k_centroids, v_codes, ldv, v_pool_stride, v_norms, v_bits,
+                        v_rotors, v_centroids, tok_pool_stride, max_tokens, paged, out, odtype, ldo, workspace,
+                        workspace_bytes);
+}
+
+kvrq_status kv_cache_append_rows(void* stream, kvrq_method method, const void* x, kvrq_dtype xdtype, int64_t n_rows,
+                                 int d, int64_t ldx, int bits, const float* rotors, const void* pi, const uint16_t* T,
+                                 int m, const float* centroids, const int64_t* dst_rows, uint32_t* codes,
+                                 int64_t ldc, uint32_t* signs, int64_t lds, float* norms, float* gammas,
+                                 int64_t ldn) {
+  const char* name = "kv_cache_append_rows";
+  if (n_rows > 0 && (!dst_rows || !aligned(dst_rows, 8)))
+    return set_error(KVRQ_EINVAL, "kv_cache_append_rows: dst_rows (8-byte aligned) is required");
+  switch (method) {
+    case KVRQ_RQ_MSE:
+      return rq_call(name, RQ_Q, stream, x, xdtype, ldx, nullptr, codes, ldc, nullptr, norms, n_rows, d, rotors,
+                     centroids, bits, nullptr, xdtype, 0, ldn, 3, dst_rows);
+    case KVRQ_TQ_MSE:
+      return tq_call(name, TQ_MSE_Q, stream, x, xdtype, ldx, n_rows, d, d, pi, nullptr, centroids, bits, codes,
+                     nullptr, ldc, nullptr, nullptr, 0, nullptr, nullptr, norms, nullptr, nullptr, 0, ldn, nullptr,
+                     0, false, dst_rows);
+    case KVRQ_TQ_PROD:
+      return tq_call(name, TQ_PROD_Q, stream, x, xdtype, ldx, n_rows, d, m, pi, T, centroids, bits, codes, nullptr,
+                     ldc, signs, nullptr, lds, gammas, nullptr, norms, nullptr, nullptr, 0, ldn, nullptr, 0, false,
+                     dst_rows);
+    default:
+      return set_error(KVRQ_EINVAL, "kv_cache_append_rows: unknown method");
+  }
 }
 
 int kvrq_attention_uses_tensor_cores(kvrq_method k_method, int k_bits, int v_bits, int group) {

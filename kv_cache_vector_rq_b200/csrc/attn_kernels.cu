@@ -329,7 +329,7 @@ __global__ void __launch_bounds__(kThreads) attn_combine_kernel(AttnArgs a) {
 
   float sum = 0.f;
   for (int c = tid; c < nc; c += kThreads) {
-    const float w = expf(ml[2 * c] - M);
+    const float w = ml[2 * c] == -INFINITY ? 0.f : expf(ml[2 * c] - M);  // an empty chunk weighs nothing
     s_w[c] = w;
     sum = fmaf(w, ml[2 * c + 1], sum);
   }
@@ -339,7 +339,7 @@ __global__ void __launch_bounds__(kThreads) attn_combine_kernel(AttnArgs a) {
   float L = 0.f;
 #pragma unroll
   for (int w = 0; w < kWarps; ++w) L += s_red[w];  // >= 1: the chunk holding the largest logit adds >= 1
-  const float inv = 1.f / L;
+  const float inv = L > 0.f ? 1.f / L : 0.f;        // (0 only for a paged sequence with no tokens: output 0)
 
   if (tid < kNcv) {
     const float* acc = a.ws_acc + row * nc * kAttnAS + tid;

@@ -56,6 +56,13 @@ struct AttnArgs {
   float* ws_acc;            // [rows][n_chunks][kAttnAS] per-chunk value sums, rotated domain
   float* ws_ml;             // [rows][n_chunks][2] per-chunk (max logit, sum of weights)
   unsigned* status;         // device status word (bounded-wait time-outs of the tensor-core path)
+  // paged cache (block_tables != NULL, tensor-core path): as ScoreArgs; the head strides then step pool heads
+  const int32_t* block_tables;
+  int64_t ld_table;
+  const int32_t* seq_lens;
+  int page_tokens;
+  int n_seqs;
+  int kv_heads;
 };
 
 // Tokens per chunk CTA of the CUDA-core path (a multiple of kAttnSub), tokens per

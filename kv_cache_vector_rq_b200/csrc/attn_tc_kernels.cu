@@ -35,6 +35,7 @@
 
 #include "attn_launch.h"
 #include "kvrq_device.cuh"
+#include "score_launch.h"
 #include "tc_decode.cuh"
 
 namespace kvrq {
@@ -191,17 +192,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
     const int64_t chunk = item - head * items_per_head;
     const int64_t row0 = head * group;
     const int64_t t_begin = chunk * a.tokens_per_cta;
-    const int64_t t_end = a.n_tokens < t_begin + a.tokens_per_cta ? a.n_tokens : t_begin + a.tokens_per_cta;
-    const int ntiles = (int)((t_end - t_begin + kRows - 1) / kRows);
-    const uint32_t* kbase = a.k_codes + head * a.k_head_stride;
-    const uint32_t* sbase = kProd ? a.k_signs + head * a.s_head_stride : nullptr;
-    const uint32_t* vbase = a.v_codes + head * a.v_head_stride;
-    const float* knb = a.k_norms + head * a.tok_head_stride;
-    const float* kgb = kProd ? a.k_gammas + head * a.tok_head_stride : nullptr;
-    const float* vnb = a.v_norms + head * a.tok_head_stride;
+    const PagedHead ph = paged_head(head, a.n_tokens, a.block_tables, a.ld_table, a.seq_lens, a.page_tokens,
+                                    a.n_seqs, a.kv_heads);
+    const int64_t t_end = ph.n_tokens < t_begin + a.tokens_per_cta ? ph.n_tokens : t_begin + a.tokens_per_cta;
+    const int ntiles = t_end > t_begin ? (int)((t_end - t_begin + kRows - 1) / kRows) : 0;
+    const uint32_t* kbase = a.k_codes + ph.pool_head * a.k_head_stride;
+    const uint32_t* sbase = kProd ? a.k_signs + ph.pool_head * a.s_head_stride : nullptr;
+    const uint32_t* vbase = a.v_codes + ph.pool_head * a.v_head_stride;
+    const float* knb = a.k_norms + ph.pool_head * a.tok_head_stride;
+    const float* kgb = kProd ? a.k_gammas + ph.pool_head * a.tok_head_stride : nullptr;
+    const float* vnb = a.v_norms + ph.pool_head * a.tok_head_stride;
+    // a paged tile is copied one page segment (min(page, 128) rows) at a time: pages of a power of two >= 16
+    // slots start 16-byte aligned and split a 128-token tile evenly
+    const int seg = !ph.table ? kRows : (ph.ptok < kRows ? ph.ptok : kRows);
     auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
     // a full tile's rows are contiguous, 16-byte aligned blocks when the rows are unpadded
-    const bool bulk = a.ldk == WK && (!kProd || a.lds == NS) && a.ldv == WV && al16(kbase) && al16(vbase) &&
+    const bool bulk = (!ph.table || ph.shift >= 4) && a.ldk == WK && (!kProd || a.lds == NS) && a.ldv == WV &&
+                      al16(kbase) && al16(vbase) &&
                       al16(knb) && al16(vnb) && (!kProd || (al16(sbase) && al16(kgb))) && (t_begin % 4) == 0;
     auto tile_full = [&](int j) { return t_begin + (int64_t)(j + 1) * kRows <= t_end; };
 
@@ -231,12 +238,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
       uint32_t* dst = w_stage + s * C::stage_words;
       uint64_t* bar = &bar_st[s];
       mbar_arrive_expect_tx(bar, (uint32_t)(kRows * 4 * (WK + NS + WV + (kProd ? 3 : 2))));
-      bulk_load(dst, kbase + t0 * WK, kRows * WK * 4, bar);
-      if (kProd) bulk_load(dst + C::st_s, sbase + t0 * NS, kRows * NS * 4, bar);
-      bulk_load(dst + C::st_v, vbase + t0 * WV, kRows * WV * 4, bar);
-      bulk_load(dst + C::st_kn, knb + t0, kRows * 4, bar);
-      if (kProd) bulk_load(dst + C::st_kg, kgb + t0, kRows * 4, bar);
-      bulk_load(dst + C::st_vn, vnb + t0, kRows * 4, bar);
+      for (int g0 = 0; g0 < kRows; g0 += seg) {  // one copy per page segment (the whole tile when unpaged)
+        const int64_t sl = ph.slot(t0 + g0);
+        bulk_load(dst + g0 * WK, kbase + sl * WK, seg * WK * 4, bar);
+        if (kProd) bulk_load(dst + C::st_s + g0 * NS, sbase + sl * NS, seg * NS * 4, bar);
+        bulk_load(dst + C::st_v + g0 * WV, vbase + sl * WV, seg * WV * 4, bar);
+        bulk_load(dst + C::st_kn + g0, knb + sl, seg * 4, bar);
+        if (kProd) bulk_load(dst + C::st_kg + g0, kgb + sl, seg * 4, bar);
+        bulk_load(dst + C::st_vn + g0, vnb + sl, seg * 4, bar);
+      }
     };
     const int nt_w = ntiles > w ? (ntiles - w + kNWG - 1) / kNWG : 0;  // this warpgroup's tiles
     const int slot0 = slot;
@@ -303,18 +313,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
         if (kProd) kg = __uint_as_float(lds_u32(st + (uint32_t)((C::st_kg + r) * 4)));
         vn = __uint_as_float(lds_u32(st + (uint32_t)((C::st_vn + r) * 4)));
       } else {
-        const int64_t t = t0 + r;
+        const int64_t sl = valid ? ph.slot(t0 + r) : 0;  // this token's row in its pool
 #pragma unroll
-        for (int q = 0; q < WK; ++q) kw[q] = valid ? __ldg(kbase + t * a.ldk + q) : 0u;
+        for (int q = 0; q < WK; ++q) kw[q] = valid ? __ldg(kbase + sl * a.ldk + q) : 0u;
         if constexpr (kProd) {
 #pragma unroll
-          for (int q = 0; q < NS; ++q) sg[q] = valid ? __ldg(sbase + t * a.lds + q) : 0u;
+          for (int q = 0; q < NS; ++q) sg[q] = valid ? __ldg(sbase + sl * a.lds + q) : 0u;
         }
 #pragma unroll
-        for (int q = 0; q < WV; ++q) vw[q] = valid ? __ldg(vbase + t * a.ldv + q) : 0u;
-        kn = valid ? __ldg(knb + t) : 0.f;
-        if (kProd) kg = valid ? __ldg(kgb + t) : 0.f;
-        vn = valid ? __ldg(vnb + t) : 0.f;
+        for (int q = 0; q < WV; ++q) vw[q] = valid ? __ldg(vbase + sl * a.ldv + q) : 0u;
+        kn = valid ? __ldg(knb + sl) : 0.f;
+        if (kProd) kg = valid ? __ldg(kgb + sl) : 0.f;
+        vn = valid ? __ldg(vnb + sl) : 0.f;
       }
 
       // ---- 1. key -> A1 (tensor memory; MMA1 of the previous tile has completed: its S was read),

@@ -727,10 +727,10 @@ __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
 
     // ---------------------------------------------------------------- outputs
     if constexpr (kIn) {
-      if (lane < rows && a.norms_out) a.norms_out[row * a.ldn] = nrm;
+      if (lane < rows && a.norms_out) a.norms_out[(a.out_rows ? a.out_rows[row] : row) * a.ldn] = nrm;
     }
     // a full sub-tile of codes leaves as one bulk copy when code rows are contiguous
-    const bool codes_bulk_out = kIn && a.codes_out && rows == kWR && a.ldc == W &&
+    const bool codes_bulk_out = kIn && a.codes_out && !a.out_rows && rows == kWR && a.ldc == W &&
                                 (reinterpret_cast<uintptr_t>(a.codes_out) & 15) == 0;
     fence_proxy_async_smem();
     __syncwarp();
@@ -760,7 +760,7 @@ __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
       if (a.codes_out && !codes_bulk_out)
         for (int i = lane; i < rows * W; i += kWR) {
           const int r = i / W, w = i - r * W;
-          a.codes_out[(row0 + r) * a.ldc + w] = stage_codes[i];
+          a.codes_out[(a.out_rows ? a.out_rows[row0 + r] : row0 + r) * a.ldc + w] = stage_codes[i];
         }
     }
   }

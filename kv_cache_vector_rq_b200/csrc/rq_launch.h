@@ -32,6 +32,7 @@ struct RqArgs {
   unsigned* status;  // device status word (bounded-wait time-outs)
   bool wide;         // any-d path: rows are streamed by bulk copy (rq_wide_smem_bytes > 0)
   int codes_per_group;  // 4: the four-grade layout (row kernel, d = 128); anything else: 3
+  const int64_t* out_rows;  // quantize, d = 128: row r's outputs go to row out_rows[r] (NULL: row r)
 };
 
 // d = 128 thread-per-row kernel fed by TMA tensor maps over x and x_hat

@@ -110,14 +110,20 @@ __global__ void __launch_bounds__(Cfg<METHOD, BITS, NB>::kThreads, 1) score_kern
   const int G = a.group;
   const int64_t head = blockIdx.y;
   const int64_t t_begin = (int64_t)blockIdx.x * a.tokens_per_cta;
-  const int64_t t_end = a.n_tokens < t_begin + a.tokens_per_cta ? a.n_tokens : t_begin + a.tokens_per_cta;
-  const int ntiles = (int)((t_end - t_begin + kRows - 1) / kRows);
-  const uint32_t* codes_h = a.codes + head * a.codes_head_stride;
-  const uint32_t* signs_h = kProd ? a.signs + head * a.signs_head_stride : nullptr;
-  const float* norms_h = a.norms + head * a.tok_head_stride;
-  const float* gammas_h = kProd ? a.gammas + head * a.tok_head_stride : nullptr;
+  const PagedHead ph = paged_head(head, a.n_tokens, a.block_tables, a.ld_table, a.seq_lens, a.page_tokens, a.n_seqs,
+                                  a.kv_heads);
+  const int64_t t_end = ph.n_tokens < t_begin + a.tokens_per_cta ? ph.n_tokens : t_begin + a.tokens_per_cta;
+  const int ntiles = t_end > t_begin ? (int)((t_end - t_begin + kRows - 1) / kRows) : 0;
+  const uint32_t* codes_h = a.codes + ph.pool_head * a.codes_head_stride;
+  const uint32_t* signs_h = kProd ? a.signs + ph.pool_head * a.signs_head_stride : nullptr;
+  const float* norms_h = a.norms + ph.pool_head * a.tok_head_stride;
+  const float* gammas_h = kProd ? a.gammas + ph.pool_head * a.tok_head_stride : nullptr;
+  // a paged tile is copied one page segment (min(page, 128) rows) at a time: pages of a power of two >= 16
+  // slots start 16-byte aligned and split a 128-token tile evenly
+  const int seg = !ph.table ? kRows : (ph.ptok < kRows ? ph.ptok : kRows);
+  const bool seg_ok = !ph.table || (ph.shift >= 4);
   // code rows of a tile are one contiguous, 16-byte aligned block when unpadded
-  const bool bulk = a.ldc == W && (!kProd || a.lds == NS) && ((reinterpret_cast<uintptr_t>(codes_h) & 15) == 0) &&
+  const bool bulk = seg_ok && a.ldc == W && (!kProd || a.lds == NS) && ((reinterpret_cast<uintptr_t>(codes_h) & 15) == 0) &&
                     (!kProd || (reinterpret_cast<uintptr_t>(signs_h) & 15) == 0) && ((kRows * W * 4) % 16 == 0);
   auto tile_full = [&](int j) { return t_begin + (int64_t)(j + 1) * kRows <= t_end; };
 
@@ -258,8 +264,11 @@ __global__ void __launch_bounds__(Cfg<METHOD, BITS, NB>::kThreads, 1) score_kern
       uint32_t* dst = s_stage + (w * kStages + s) * C::stage_words;
       uint64_t* bar = &bar_stage[w * kStages + s];
       mbar_arrive_expect_tx(bar, C::stage_words * 4);
-      bulk_load(dst, codes_h + t0 * W, kRows * W * 4, bar);
-      if (kProd) bulk_load(dst + kRows * W, signs_h + t0 * NS, kRows * NS * 4, bar);
+      for (int g0 = 0; g0 < kRows; g0 += seg) {  // one copy per page segment (the whole tile when unpaged)
+        const int64_t sl = ph.slot(t0 + g0);
+        bulk_load(dst + g0 * W, codes_h + sl * W, seg * W * 4, bar);
+        if (kProd) bulk_load(dst + kRows * W + g0 * NS, signs_h + sl * NS, seg * NS * 4, bar);
+      }
     };
     if (r == 0 && bulk)
       for (int i = 0; i < kStages; ++i) {
@@ -361,8 +370,9 @@ __global__ void __launch_bounds__(Cfg<METHOD, BITS, NB>::kThreads, 1) score_kern
       const int64_t t0 = t_begin + (int64_t)j * kRows;
       const int rows = (int)(t_end - t0 < (int64_t)kRows ? t_end - t0 : (int64_t)kRows);
       // this key's norm and gamma (used by the epilogue one iteration later), packed codes and signs
-      const float nrm = r < rows ? __ldg(norms_h + t0 + r) : 0.f;
-      const float gam = (kProd && r < rows) ? __ldg(gammas_h + t0 + r) : 0.f;
+      const int64_t sl = r < rows ? ph.slot(t0 + r) : 0;  // this key's row in its pool
+      const float nrm = r < rows ? __ldg(norms_h + sl) : 0.f;
+      const float gam = (kProd && r < rows) ? __ldg(gammas_h + sl) : 0.f;
       uint32_t wc[W], sg[NS > 0 ? NS : 1];
       // both waits of the tile first; the warpgroup leaves together if either ran out
       if (bulk && tile_full(j)) ok = mbar_wait(&bar_stage[w * kStages + s], (uint32_t)((i / kStages) & 1), a.status);
@@ -396,10 +406,10 @@ __global__ void __launch_bounds__(Cfg<METHOD, BITS, NB>::kThreads, 1) score_kern
         }
       } else {
 #pragma unroll
-        for (int q = 0; q < W; ++q) wc[q] = r < rows ? __ldg(codes_h + (t0 + r) * a.ldc + q) : 0u;
+        for (int q = 0; q < W; ++q) wc[q] = r < rows ? __ldg(codes_h + sl * a.ldc + q) : 0u;
         if constexpr (kProd) {
 #pragma unroll
-          for (int q = 0; q < NS; ++q) sg[q] = r < rows ? __ldg(signs_h + (t0 + r) * a.lds + q) : 0u;
+          for (int q = 0; q < NS; ++q) sg[q] = r < rows ? __ldg(signs_h + sl * a.lds + q) : 0u;
         }
       }
       // the previous tile's MMA has finished with A: its scores, then this tile's decode

@@ -36,7 +36,50 @@ struct ScoreArgs {
   float* scores;
   int64_t ld_scores;
   unsigned* status;
+  // paged cache (block_tables != NULL): head h = (layer * n_seqs + s) * kv_heads + k reads the rows of pool
+  // head layer * kv_heads + k (the strides above then step pool heads), token t < seq_lens[s] at slot
+  // page_tokens * block_tables[s * ld_table + t / page_tokens] + t % page_tokens
+  const int32_t* block_tables;
+  int64_t ld_table;
+  const int32_t* seq_lens;
+  int page_tokens;
+  int n_seqs;
+  int kv_heads;
 };
+
+// Pool head, block-table row and token count of head `head` of a paged call, or of a contiguous one
+// (head itself, no table, n_tokens).
+struct PagedHead {
+  int64_t pool_head;
+  const int32_t* table;
+  int64_t n_tokens;
+  int shift;   // log2(page_tokens) when it is a power of two, else -1
+  int ptok;
+  __device__ __forceinline__ int64_t slot(int64_t t) const {
+    if (!table) return t;
+    if (shift >= 0) return ((int64_t)__ldg(table + (t >> shift)) << shift) + (t & (ptok - 1));
+    return (int64_t)__ldg(table + t / ptok) * ptok + t % ptok;
+  }
+};
+
+__device__ __forceinline__ PagedHead paged_head(int64_t head, int64_t n_tokens, const int32_t* tables, int64_t ld_table,
+                                                const int32_t* seq_lens, int page_tokens, int n_seqs, int kv_heads) {
+  PagedHead p;
+  p.pool_head = head;
+  p.table = nullptr;
+  p.n_tokens = n_tokens;
+  p.ptok = page_tokens;
+  p.shift = -1;
+  if (tables) {
+    const int64_t k = head % kv_heads, s = (head / kv_heads) % n_seqs, layer = head / ((int64_t)kv_heads * n_seqs);
+    p.pool_head = layer * kv_heads + k;
+    p.table = tables + s * ld_table;
+    const int64_t len = __ldg(seq_lens + s);
+    p.n_tokens = len < n_tokens ? (len > 0 ? len : 0) : n_tokens;
+    if ((page_tokens & (page_tokens - 1)) == 0) p.shift = __ffs(page_tokens) - 1;
+  }
+  return p;
+}
 
 // nb: MMA N (16, 32 or 64); cbits: stored code width.
 cudaError_t launch_score(int method, int nb, int cbits, const ScoreArgs& a, cudaStream_t st);

@@ -301,8 +301,9 @@ __global__ void __launch_bounds__(kRows, 1)
 #pragma unroll
       for (int w = 0; w < W; ++w) s_codes[tid * W + w] = wc[w];
       if (tid < rows) {
-        if (a.norms_out) a.norms_out[row * a.ldn] = nrm;
-        if (kProd && a.gammas_out) a.gammas_out[row * a.ldn] = sqrtf(gs);
+        const int64_t orow = a.out_rows ? a.out_rows[row] : row;
+        if (a.norms_out) a.norms_out[orow * a.ldn] = nrm;
+        if (kProd && a.gammas_out) a.gammas_out[orow * a.ldn] = sqrtf(gs);
       }
 
       if constexpr (MODE == TQ_MSE_QDQ || MODE == TQ_PROD_Q) {
@@ -424,12 +425,12 @@ __global__ void __launch_bounds__(kRows, 1)
       if (a.codes_out)
         for (int i = tid; i < rows * W; i += kRows) {
           const int r = i / W, w = i - r * W;
-          a.codes_out[(row0 + r) * a.ldc + w] = s_codes[i];
+          a.codes_out[(a.out_rows ? a.out_rows[row0 + r] : row0 + r) * a.ldc + w] = s_codes[i];
         }
       if (kProd && a.signs_out)
         for (int i = tid; i < rows * NS; i += kRows) {
           const int r = i / NS, w = i - r * NS;
-          a.signs_out[(row0 + r) * a.lds + w] = s_signs[i];
+          a.signs_out[(a.out_rows ? a.out_rows[row0 + r] : row0 + r) * a.lds + w] = s_signs[i];
         }
     }
     __syncthreads();  // staging buffers are rewritten by the next tile

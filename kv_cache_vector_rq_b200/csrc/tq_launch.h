@@ -32,6 +32,7 @@ struct TqArgs {
   int64_t lds;  // sign row stride (words)
   int64_t ldn;  // norm and gamma row stride (floats)
   unsigned* status;
+  const int64_t* out_rows;  // quantize, d = 128: row r's outputs go to row out_rows[r] (NULL: row r)
 };
 
 // map_x: input rows (quantize), map_pi: Pi [d][d], map_t: T [m][d] (fp16),
