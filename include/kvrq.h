@@ -57,7 +57,9 @@ typedef enum {
   KVRQ_EUNSUPPORTED = 2, /* valid but not implemented (e.g. bits outside 1..4) */
   KVRQ_ECUDA = 3,        /* a CUDA runtime/driver call failed */
   KVRQ_ENOCONV = 4,      /* Lloyd-Max did not converge within max_iter */
-  KVRQ_ETIMEOUT = 5      /* a bounded device-side wait ran out */
+  KVRQ_ETIMEOUT = 5,     /* a bounded device-side wait ran out */
+  KVRQ_ENOMEM = 6,       /* host memory could not be allocated (the call changed nothing) */
+  KVRQ_ECHECKSUM = 7     /* a parameter file's contents do not match its checksum */
 } kvrq_status;
 
 typedef enum { KVRQ_F32 = 0, KVRQ_F16 = 1, KVRQ_BF16 = 2 } kvrq_dtype;
@@ -337,6 +339,42 @@ kvrq_status kv_score_packed(void* stream, kvrq_method method, const void* q, kvr
                             const float* norms, const float* gammas, int64_t tok_head_stride, int64_t n_tokens,
                             const float* rotors, const void* pi, kvrq_dtype pi_dtype, const uint16_t* T,
                             const float* centroids, float* scores, int64_t ld_scores);
+
+/* Parameter files: the seed-derived parameters of one configuration (d, bits, m,
+ * seed) written once and read back, verified ["TurboQuant 论文解读", "简单复现 demo";
+ * "TurboQuant + RotorQuant", "How RotorQuant Works", "Codebook Calibration Fix": the
+ * rotation, the Gaussian projection, the rotors and the codebook are fixed functions
+ * of the seed and the sizes]. The file is a magic line "KVRQ-PARAMS 1", a one-line
+ * JSON header (d, bits, m, seed, the array lengths and "fnv1a64", the FNV-1a 64-bit
+ * hash of the payload in hex) and the float64 arrays little-endian: rotors [G][4]
+ * (rq_rotors_init, seed + 1), pi [d][d] (tq_rotation_init, seed + 2), T [m][d]
+ * (qjl_matrix_init, seed + 3), centroids [2^bits] (tq_codebook_init, tol 1e-13).
+ *   export: 2 <= d <= 16384, 1 <= bits <= 8, 1 <= m <= 16384; KVRQ_EINVAL if the
+ *     file cannot be written.
+ *   import: the file must hold exactly that (d, bits, m) (else KVRQ_EINVAL, as for a
+ *     missing, malformed or wrong-length file); payload bytes that do not hash to the
+ *     header's checksum return KVRQ_ECHECKSUM and write nothing. Output arrays may
+ *     be NULL (skipped); seed receives the file's seed (may be NULL). Host only. */
+kvrq_status kvrq_params_export(const char* path, int d, int bits, int m, uint64_t seed);
+kvrq_status kvrq_params_import(const char* path, int d, int bits, int m, uint64_t* seed, double* rotors, double* pi,
+                               double* T, double* centroids);
+
+/* Time-out path of the device waits: every wait of a kernel on a copy or a
+ * tensor-core product polls a bounded number of times, then records KVRQ_ETIMEOUT
+ * in the device status word (read and cleared by kvrq_device_status), waits at the
+ * default limit for its own copies and products still in flight, frees its tensor
+ * memory and returns (its outputs are then incomplete). kvrq_set_wait_limit sets
+ * the polls of the packed-score kernel's main-loop waits for the calls that follow
+ * in this process (negative: the default, 2^24 polls), so a test can make a wait
+ * run out with no fault: with 0 those waits give up without polling (a single poll
+ * may itself block until a copy lands). */
+void kvrq_set_wait_limit(int64_t polls);
+
+/* Test hook of the host failure path: the next `count` host allocations made by
+ * the library's entry points (parameter setup work vectors, page-manager tables)
+ * fail as if memory were exhausted; each such call returns KVRQ_ENOMEM and changes
+ * nothing. count <= 0 disarms the hook. No device memory is involved. */
+void kvrq_test_fail_allocations(int count);
 
 /* ================================================================ paged KV cache
  * ["TurboQuant + RotorQuant", "Post-Prefill Quantization": the prefill cache is

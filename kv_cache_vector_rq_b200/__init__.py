@@ -12,6 +12,7 @@ host setup functions in float64 and returned as numpy arrays.
 """
 
 import ctypes
+import os
 
 import numpy as np
 
@@ -63,6 +64,23 @@ def pq_angle_codebook_init(level, bits, tol=1e-13, max_iter=100000):
     _lib.check("pq_angle_codebook_init",
                lib().pq_angle_codebook_init(level, bits, tol, max_iter, _dptr(c), _dptr(t), ctypes.byref(it)))
     return c, t
+
+
+def params_export(path, d, bits, m, seed):
+    """Write the parameters of (d, bits, m, seed) to a checksummed file (kvrq_params_export)."""
+    _lib.check("kvrq_params_export", lib().kvrq_params_export(os.fsencode(path), d, bits, m, seed))
+
+
+def params_import(path, d, bits, m):
+    """Read and verify a parameter file: returns dict(seed, rotors [G, 4], pi [d, d], T [m, d], centroids)."""
+    G = rq_groups(d)
+    out = {"rotors": np.zeros((G, 4)), "pi": np.zeros((d, d)), "T": np.zeros((m, d)), "centroids": np.zeros(1 << bits)}
+    seed = ctypes.c_uint64(0)
+    _lib.check("kvrq_params_import", lib().kvrq_params_import(
+        os.fsencode(path), d, bits, m, ctypes.byref(seed), _dptr(out["rotors"]), _dptr(out["pi"]), _dptr(out["T"]),
+        _dptr(out["centroids"])))
+    out["seed"] = seed.value
+    return out
 
 
 def rq_rotors_init(d, seed):

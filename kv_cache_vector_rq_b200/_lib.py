@@ -97,6 +97,11 @@ SIGNATURES = {
     # lds, norms, gammas, ldn
     "kv_cache_append_rows": (c_int, [c_vp, c_int, c_vp, c_int, c_i64, c_int, c_i64, c_int, c_vp, c_vp, c_vp, c_int,
                                      c_vp, c_vp, c_vp, c_i64, c_vp, c_i64, c_vp, c_vp, c_i64]),
+    "kvrq_test_fail_allocations": (None, [c_int]),
+    "kvrq_set_wait_limit": (None, [c_i64]),
+    "kvrq_params_export": (c_int, [ctypes.c_char_p, c_int, c_int, c_int, ctypes.c_uint64]),
+    "kvrq_params_import": (c_int, [ctypes.c_char_p, c_int, c_int, c_int, ctypes.POINTER(ctypes.c_uint64), c_vp, c_vp,
+                                   c_vp, c_vp]),
     "kvrq_attention_uses_tensor_cores": (c_int, [c_int, c_int, c_int, c_int]),
     "kvrq_pages_create": (c_int, [c_i64, c_int, ctypes.POINTER(c_vp)]),
     "kvrq_pages_destroy": (None, [c_vp]),

@@ -17,7 +17,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libkvrq.so")
 
-SOURCES = ["setup.cpp", "pages.cpp", "api.cu", "rq_kernels.cu", "tq_kernels.cu", "tqg_kernels.cu",
+SOURCES = ["setup.cpp", "pages.cpp", "params.cpp", "api.cu", "rq_kernels.cu", "tq_kernels.cu", "tqg_kernels.cu",
            "score_kernels.cu", "attn_kernels.cu", "attn_tc_kernels.cu", "pq_kernels.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-I" + INCLUDE, "-I" + CSRC]

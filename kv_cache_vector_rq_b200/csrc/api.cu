@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -26,6 +27,19 @@ namespace kvrq {
 __device__ unsigned int g_device_status = 0;
 
 static thread_local std::string t_last_error;
+
+// Allocation failures the test hook still has to inject (kvrq_test_fail_allocations).
+static std::atomic<int> g_fail_allocs{0};
+
+// Polls after which the packed-score kernel's main-loop waits give up (kvrq_set_wait_limit; < 0: default).
+static std::atomic<int32_t> g_wait_limit{-1};
+
+void alloc_check() {
+  int left = g_fail_allocs.load();
+  while (left > 0) {
+    if (g_fail_allocs.compare_exchange_weak(left, left - 1)) throw std::bad_alloc();
+  }
+}
 
 kvrq_status set_error(kvrq_status st, const char* msg) {
   t_last_error = msg ? msg : "";
@@ -184,6 +198,8 @@ static kvrq_status rq_call(const char* name, int mode, void* stream, const void*
     if (!aligned(xhat, dtype_size(odt))) return set_errorf(KVRQ_EINVAL, "%s: xhat misaligned", name);
   }
   if (n > ((int64_t)1 << 31) - 256) return set_errorf(KVRQ_EUNSUPPORTED, "%s: n >= 2^31", name);
+  if (out_rows && !(mode == RQ_Q && d == 128 && rows_aligned16(x, ldx, xdt)))
+    return set_errorf(KVRQ_EUNSUPPORTED, "%s: destination rows need d = 128 and 16-byte aligned rows", name);
 
   DeviceInfo* di;
   kvrq_status st = current_device(&di);
@@ -226,7 +242,7 @@ static kvrq_status rq_call(const char* name, int mode, void* stream, const void*
   if (cpg == 4)
     return set_errorf(KVRQ_EUNSUPPORTED, "%s: the four-grade layout needs 16-byte aligned rows (and one dtype for "
                                          "the fused call)", name);
-  if (out_rows) return set_errorf(KVRQ_EUNSUPPORTED, "%s: destination rows need d = 128 and 16-byte aligned rows", name);
+
   // any d: rows streamed by bulk copy when they start 16-byte aligned and fit its row buffers
   bool wide = true;
   if (q_side) wide = wide && rows_aligned16(x, ldx, xdt);
@@ -773,6 +789,7 @@ static kvrq_status score_call(const char* name, void* stream, kvrq_method method
     a.n_seqs = pg->n_seqs;
     a.kv_heads = pg->kv_heads;
   }
+  a.spin_limit = g_wait_limit.load();
   const int nb = rows_needed <= 16 ? 16 : (rows_needed <= 32 ? 32 : 64);
   return launch_status(name, launch_score(method, nb, cbits, a, static_cast<cudaStream_t>(stream)));
 }
@@ -985,6 +1002,12 @@ kvrq_status kv_cache_append_rows(void* stream, kvrq_method method, const void* x
     default:
       return set_error(KVRQ_EINVAL, "kv_cache_append_rows: unknown method");
   }
+}
+
+void kvrq_test_fail_allocations(int count) { g_fail_allocs.store(count > 0 ? count : 0); }
+
+void kvrq_set_wait_limit(int64_t polls) {
+  g_wait_limit.store(polls < 0 ? -1 : (int32_t)(polls < INT32_MAX ? polls : INT32_MAX));
 }
 
 int kvrq_attention_uses_tensor_cores(kvrq_method k_method, int k_bits, int v_bits, int group) {

@@ -85,9 +85,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
 }
 
 // Bounded wait for the phase with parity `phase` to complete. Returns false
-// (and records a time-out) if it did not complete within kSpinLimit polls.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, unsigned* status) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i)
+// (and records a time-out) if it did not complete within `limit` polls.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, unsigned* status,
+                                          uint32_t limit = kSpinLimit) {
+  for (uint32_t i = 0; i < limit; ++i)
     if (mbar_try_wait(bar, phase)) return true;
   record_status(status, kStatusTimeout);
   return false;

@@ -11,6 +11,7 @@
 // indexed by these slot numbers.
 
 #include <cstdint>
+#include <memory>
 #include <mutex>
 #include <unordered_map>
 #include <vector>
@@ -40,13 +41,17 @@ kvrq_status kvrq_pages_create(int64_t n_pages, int page_tokens, kvrq_pages** out
   *out = nullptr;
   if (n_pages < 1 || n_pages > INT32_MAX || page_tokens < 1)
     return set_error(KVRQ_EINVAL, "kvrq_pages_create: n_pages in 1..2^31-1 and page_tokens >= 1");
-  kvrq_pages* p = new kvrq_pages();
-  p->n_pages = n_pages;
-  p->page_tokens = page_tokens;
-  p->free_list.reserve((size_t)n_pages);
-  for (int64_t i = n_pages - 1; i >= 0; --i) p->free_list.push_back((int32_t)i);  // page 0 is handed out first
-  *out = p;
-  return KVRQ_OK;
+  return guarded("kvrq_pages_create", [&] {
+    alloc_check();
+    std::unique_ptr<kvrq_pages> p(new kvrq_pages());
+    p->n_pages = n_pages;
+    p->page_tokens = page_tokens;
+    // the free list never holds more than n_pages pages: later pushes never reallocate
+    p->free_list.reserve((size_t)n_pages);
+    for (int64_t i = n_pages - 1; i >= 0; --i) p->free_list.push_back((int32_t)i);  // page 0 is handed out first
+    *out = p.release();
+    return KVRQ_OK;
+  });
 }
 
 void kvrq_pages_destroy(kvrq_pages* p) { delete p; }
@@ -54,9 +59,12 @@ void kvrq_pages_destroy(kvrq_pages* p) { delete p; }
 kvrq_status kvrq_pages_add_seq(kvrq_pages* p, int64_t* seq_id) {
   if (!p || !seq_id) return set_error(KVRQ_EINVAL, "kvrq_pages_add_seq: NULL argument");
   std::lock_guard<std::mutex> lk(p->mu);
-  *seq_id = p->next_id++;
-  p->seqs.emplace(*seq_id, kvrq_pages::Seq());
-  return KVRQ_OK;
+  return guarded("kvrq_pages_add_seq", [&] {
+    alloc_check();
+    p->seqs.emplace(p->next_id, kvrq_pages::Seq());  // the id is taken only once the entry exists
+    *seq_id = p->next_id++;
+    return KVRQ_OK;
+  });
 }
 
 kvrq_status kvrq_pages_append(kvrq_pages* p, int64_t seq_id, int64_t n_tokens, int64_t* first_token) {
@@ -72,13 +80,19 @@ kvrq_status kvrq_pages_append(kvrq_pages* p, int64_t seq_id, int64_t n_tokens, i
   const int64_t need = (total + p->page_tokens - 1) / p->page_tokens - (int64_t)s.table.size();
   if (need > (int64_t)p->free_list.size())
     return set_error(KVRQ_EINVAL, "kvrq_pages_append: not enough free pages (nothing appended)");
-  for (int64_t i = 0; i < need; ++i) {
-    s.table.push_back(p->free_list.back());
-    p->free_list.pop_back();
-  }
-  if (first_token) *first_token = s.tokens;
-  s.tokens = total;
-  return KVRQ_OK;
+  return guarded("kvrq_pages_append", [&] {
+    if (need > 0) {
+      alloc_check();
+      s.table.reserve(s.table.size() + (size_t)need);  // may throw: nothing has moved yet
+    }
+    for (int64_t i = 0; i < need; ++i) {  // no allocation from here on
+      s.table.push_back(p->free_list.back());
+      p->free_list.pop_back();
+    }
+    if (first_token) *first_token = s.tokens;
+    s.tokens = total;
+    return KVRQ_OK;
+  });
 }
 
 kvrq_status kvrq_pages_slots(kvrq_pages* p, int64_t seq_id, int64_t first, int64_t count, int64_t* slots) {

@@ -126,6 +126,7 @@ __global__ void __launch_bounds__(Cfg<METHOD, BITS, NB>::kThreads, 1) score_kern
   const bool bulk = seg_ok && a.ldc == W && (!kProd || a.lds == NS) && ((reinterpret_cast<uintptr_t>(codes_h) & 15) == 0) &&
                     (!kProd || (reinterpret_cast<uintptr_t>(signs_h) & 15) == 0) && ((kRows * W * 4) % 16 == 0);
   auto tile_full = [&](int j) { return t_begin + (int64_t)(j + 1) * kRows <= t_end; };
+  const uint32_t lim = a.spin_limit < 0 ? kSpinLimit : (uint32_t)a.spin_limit;  // main loop (the drain: default)
 
   if (tid == 0) {
     for (int s = 0; s < C::nbars; ++s) mbar_init(&s_bar[s], 1);
@@ -375,8 +376,9 @@ __global__ void __launch_bounds__(Cfg<METHOD, BITS, NB>::kThreads, 1) score_kern
       const float gam = (kProd && r < rows) ? __ldg(gammas_h + sl) : 0.f;
       uint32_t wc[W], sg[NS > 0 ? NS : 1];
       // both waits of the tile first; the warpgroup leaves together if either ran out
-      if (bulk && tile_full(j)) ok = mbar_wait(&bar_stage[w * kStages + s], (uint32_t)((i / kStages) & 1), a.status);
-      if (i > 0) ok = mbar_wait(&bar_acc[w * 2 + ((i - 1) & 1)], (uint32_t)(((i - 1) >> 1) & 1), a.status) && ok;
+      if (bulk && tile_full(j))
+        ok = mbar_wait(&bar_stage[w * kStages + s], (uint32_t)((i / kStages) & 1), a.status, lim);
+      if (i > 0) ok = mbar_wait(&bar_acc[w * 2 + ((i - 1) & 1)], (uint32_t)(((i - 1) >> 1) & 1), a.status, lim) && ok;
       if (!wg_all(ok, 1 + w)) {
         ok = false;
         break;

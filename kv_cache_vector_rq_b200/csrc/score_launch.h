@@ -45,6 +45,9 @@ struct ScoreArgs {
   int page_tokens;
   int n_seqs;
   int kv_heads;
+  // polls of the tile and MMA waits of the main loop before they give up (negative: the default;
+  // 0: they give up at once); the waits that drain copies and MMAs in flight always use the default
+  int32_t spin_limit;
 };
 
 // Pool head, block-table row and token count of head `head` of a paged call, or of a contiguous one

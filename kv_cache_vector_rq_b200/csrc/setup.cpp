@@ -164,7 +164,7 @@ kvrq_status kvrq_normals(uint64_t seed, int64_t first, int64_t count, double* ou
   return KVRQ_OK;
 }
 
-kvrq_status tq_codebook_init(int d, int bits, double tol, int max_iter, double* centroids,
+static kvrq_status tq_codebook_init_body(int d, int bits, double tol, int max_iter, double* centroids,
                              double* boundaries, int* iterations) {
   if (d < 2) return set_error(KVRQ_EINVAL, "tq_codebook_init: d must be >= 2");
   if (bits < 1 || bits > 8) return set_error(KVRQ_EINVAL, "tq_codebook_init: bits must be in 1..8");
@@ -209,7 +209,7 @@ kvrq_status tq_codebook_init(int d, int bits, double tol, int max_iter, double* 
   return KVRQ_OK;
 }
 
-kvrq_status pq_angle_codebook_init(int level, int bits, double tol, int max_iter, double* centroids,
+static kvrq_status pq_angle_codebook_init_body(int level, int bits, double tol, int max_iter, double* centroids,
                                    double* boundaries, int* iterations) {
   if (level < 1 || level > 20) return set_error(KVRQ_EINVAL, "pq_angle_codebook_init: level must be in 1..20");
   if (bits < 1 || bits > 8) return set_error(KVRQ_EINVAL, "pq_angle_codebook_init: bits must be in 1..8");
@@ -287,7 +287,7 @@ kvrq_status qjl_matrix_init(int m, int d, uint64_t seed, double* T) {
 // trailing block is updated as A <- (I - 2 v v^T / v^T v) A. R_kk = alpha.
 // Q = H_0 H_1 ... H_{d-1} is formed by applying the reflectors to I in
 // reverse order. Pi = Q diag(sign(R_kk)).
-kvrq_status tq_rotation_init(int d, uint64_t seed, double* pi) {
+static kvrq_status tq_rotation_init_body(int d, uint64_t seed, double* pi) {
   if (d < 1 || d > 16384 || !pi) return set_error(KVRQ_EINVAL, "tq_rotation_init: 1 <= d <= 16384, pi != NULL");
   const int64_t n = d;
   std::vector<double> A((size_t)(n * n));
@@ -366,6 +366,30 @@ kvrq_status tq_rotation_init(int d, uint64_t seed, double* pi) {
   for (int64_t i = 0; i < n; ++i)
     for (int64_t j = 0; j < n; ++j) pi[i * n + j] = Q[(size_t)(i * n + j)] * (rdiag[(size_t)j] >= 0.0 ? 1.0 : -1.0);
   return KVRQ_OK;
+}
+
+// The entry points that allocate host memory (work vectors, threads) run their bodies guarded.
+kvrq_status tq_codebook_init(int d, int bits, double tol, int max_iter, double* centroids, double* boundaries,
+                             int* iterations) {
+  return guarded("tq_codebook_init", [&] {
+    alloc_check();
+    return tq_codebook_init_body(d, bits, tol, max_iter, centroids, boundaries, iterations);
+  });
+}
+
+kvrq_status pq_angle_codebook_init(int level, int bits, double tol, int max_iter, double* centroids,
+                                   double* boundaries, int* iterations) {
+  return guarded("pq_angle_codebook_init", [&] {
+    alloc_check();
+    return pq_angle_codebook_init_body(level, bits, tol, max_iter, centroids, boundaries, iterations);
+  });
+}
+
+kvrq_status tq_rotation_init(int d, uint64_t seed, double* pi) {
+  return guarded("tq_rotation_init", [&] {
+    alloc_check();
+    return tq_rotation_init_body(d, seed, pi);
+  });
 }
 
 }  // extern "C"
