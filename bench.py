@@ -494,10 +494,18 @@ def run_leg_only(args):
         rows = heads * t
     else:
         fn, rows = None, None
-    kind, b = args.leg.rsplit("_", 1)[0], args.leg.rsplit("_", 1)[1]
-    mode, b = b.rstrip("0123456789"), int(b.lstrip("qdmpro"))
+    if args.leg == "pq_qdq":  # PolarQuant fused roundtrip at d = 128 (levels of 4, 2, 2, 2 bits)
+        x = synth.lognormal(args.rows, D, seed=1, dtype=torch.float16, device=dev)
+        pi = torch.from_numpy(kvrq.tq_rotation_init(D, 2)).to(torch.float16).to(dev)
+        pc = torch.from_numpy(kvrq.pq_codebooks()).to(dev)
+        codes = torch.empty((args.rows, kvrq.PQ_WORDS), dtype=torch.int32, device=dev)
+        xh = torch.empty_like(x)
+        fn = lambda: kvrq.pq_quantize_dequantize(x, pi, pc, codes=codes, xhat=xh)
+        rows = args.rows
     if fn is not None:
         return time_fn(fn, rows, args, torch, kvrq)
+    kind, b = args.leg.rsplit("_", 1)[0], args.leg.rsplit("_", 1)[1]
+    mode, b = b.rstrip("0123456789"), int(b.lstrip("qdmpro"))
     rows = args.rows
     dd = args.dim
     x = synth.lognormal(rows, dd, seed=1, dtype=torch.float16, device=dev, outliers=() if dd != D else
@@ -649,7 +657,8 @@ def main():
     ap.add_argument("--no-large", action="store_true", help="skip the 1 GiB HBM-roofline leg")
     ap.add_argument("--leg", default=None,
                     help="time one kernel leg (rq_q3, rq_dq3, rq_qdq3, tq_q3, tq_qdq3, tq_prod3, tq_dqm3, tq_dqp3, "
-                         "any b) on --rows vectors instead of the workload; used for profiler captures")
+                         "any b; score_prod3; pq_qdq) on --rows vectors instead of the workload; used for profiler "
+                         "captures")
     ap.add_argument("--rows", type=int, default=1 << 20)
     ap.add_argument("--dim", type=int, default=D, help="head dimension of --leg (the tiled TurboQuant path "
                                                        "and the general RotorQuant kernel run d != 128)")
