@@ -287,8 +287,8 @@ def polar_angle_margins(x64, Pi64, ref):
     The kernel forms y = Pi x with float32 sums of exact 16-bit products: |dy_i| <= e_i = LAMBDA sqrt(d) 2^-24
     sum_k |Pi_ik x_k|. A level-1 angle atan2(b, a) of a pair of radius r moves by at most (e_a + e_b) / r; a
     float32 radius carries the errors of its pair plus two roundings (2^-22 r), and a level-l angle of radii
-    (r_a, r_b) moves by (dr_a + dr_b) / r. The decision itself (products of float32 cosines and sines)
-    adds 2^-21. Margin = max(1e-5, 2 x that bound)."""
+    (r_a, r_b) moves by (dr_a + dr_b) / r. The decision itself (float32 products of the coordinates or
+    squared radii with float32 tangents of the boundaries) adds 2^-21. Margin = max(1e-5, 2 x that bound)."""
     x64 = np.asarray(x64, dtype=np.float64)
     Pi64 = np.asarray(Pi64, dtype=np.float64)
     d = x64.shape[1]

@@ -129,3 +129,57 @@ def test_unsupported_shapes_are_rejected():
         kvrq.pq_quantize_dequantize(torch.zeros((4, 256), dtype=torch.float16, device="cuda"), pi_d, c_d)
     with pytest.raises(kvrq.KvrqError):
         kvrq.pq_quantize_dequantize(torch.zeros((4, D), dtype=torch.float32, device="cuda"), pi_d, c_d)
+
+
+def test_axis_and_diagonal_pairs_with_identity_rotation():
+    """Pi = I makes y = x exactly, so pairs can sit on the axes and the diagonals (boundaries of the level-1
+    cells, and of the middle level-2 cell by the symmetry of its density): every quadrant's sign pattern,
+    zeros of either sign, and equal radii. The angle of a boundary pair may take either neighbouring code; a
+    zero pair takes code 0."""
+    books64, _, _, c_d = _params(torch.float16)
+    eye = torch.eye(D, dtype=torch.float16)
+    g = np.random.default_rng(21)
+    n = 512
+    x = np.exp(0.5 * g.standard_normal((n, D))) * np.where(g.random((n, D)) < 0.5, -1.0, 1.0)
+    pats = np.array([[1, 0], [0, 1], [-1, 0], [0, -1], [1, 1], [-1, 1], [-1, -1], [1, -1], [0, 0]], dtype=np.float64)
+    for i in range(n):
+        for p in range(D // 2):
+            if g.random() < 0.6:
+                x[i, 2 * p:2 * p + 2] = pats[g.integers(len(pats))] * x[i, 2 * p]
+    x[5] = 0.0
+    x[6, 0::2] = 2.0  # every pair (2, 1): equal radii at every level >= 2
+    x[6, 1::2] = 1.0
+    x[7, 0::2], x[7, 1::2] = -0.0, 3.0  # signed zeros against nonzero partners
+    x[8, 0::2], x[8, 1::2] = 3.0, -0.0
+    xt = torch.from_numpy(x).to(torch.float16)
+    codes, xhat = kvrq.pq_quantize_dequantize(xt.cuda(), eye.cuda(), c_d)
+    torch.cuda.synchronize()
+    kvrq.device_status()
+    x64 = xt.double().numpy()
+    ref = polar.quantize(x64, np.eye(D), books64)
+    w = words_u32(codes)
+    bad = compare_polar_codes(w, ref, books64, polar_angle_margins(x64, np.eye(D), ref))
+    assert np.all(w[5] == 0)
+    _normwise(to_f64(xhat), polar.dequantize(ref, np.eye(D), books64), XHAT_RTOL[torch.float16], skip=bad)
+    xd = kvrq.pq_dequantize(codes, D, eye.cuda(), c_d, out_dtype=torch.float16)
+    torch.cuda.synchronize()
+    assert torch.equal(xd.view(torch.int16), xhat.view(torch.int16))
+
+
+@pytest.mark.parametrize("ld,off", [(17, 0), (20, 1)])
+def test_strided_code_rows(ld, off):
+    """Code rows with a stride that is not a multiple of four words, or not 16-byte aligned, take the
+    word-by-word path: the same words as the contiguous layout, and the same x_hat from them."""
+    books64, pi64, pi_d, c_d = _params(torch.float16)
+    x = synth.lognormal(1000, D, seed=31, dtype=torch.float16).cuda()
+    c0, x0 = kvrq.pq_quantize_dequantize(x, pi_d, c_d)
+    buf = torch.full((1000, ld), -1, dtype=torch.int32, device="cuda")
+    view = buf[:, off:off + 16]
+    _, x1 = kvrq.pq_quantize_dequantize(x, pi_d, c_d, codes=view)
+    torch.cuda.synchronize()
+    assert torch.equal(view, c0) and torch.equal(x1.view(torch.int16), x0.view(torch.int16))
+    rest = torch.cat([buf[:, :off], buf[:, off + 16:]], dim=1)
+    assert torch.all(rest == -1)  # nothing outside the 16 words of a row is written
+    xd = kvrq.pq_dequantize(view, D, pi_d, c_d, out_dtype=torch.float16)
+    torch.cuda.synchronize()
+    assert torch.equal(xd.view(torch.int16), x0.view(torch.int16))
