@@ -441,6 +441,315 @@ __global__ void __launch_bounds__(kRows, 1)
   if (warp == 0) tmem_dealloc(tmem, kNcols);
 }
 
+// ============================================================================ mse, two threads per row
+// TurboQuant-mse at d = 128 (quantize, roundtrip, dequantize) with 256-thread CTAs: thread (row r,
+// half h = warp / 4) owns columns 64h .. 64h + 63 of its row (TMEM lane r), so a warp's chain is
+// half as long and an SM holds twice the warps. The row norm is the sum of the two halves' sums of
+// squares, exchanged through shared memory under a barrier of the two warps that share the rows.
+// Two tile buffers alternate: the next tile's x is loaded as soon as this tile's first product has
+// read its own, and lands while this tile is quantized; the centroid operand of the second product
+// is written over x, and x_hat over the centroids. A half row holds 64 codes, whole code words.
+constexpr int kThreadsM = 256;
+
+template <int BITS>
+struct HalfRow {
+  static constexpr int CPW = 23 / BITS;                 // codes per mantissa window
+  static constexpr int NWH = (64 + CPW - 1) / CPW;      // windows of a half row
+  static constexpr int WH = 2 * BITS;                   // code words of a half row
+};
+
+struct SmemM {
+  static constexpr int buf_off = 0;                         // two tiles
+  static constexpr int pi_off = 2 * kTileBytes;
+  static constexpr int cb_off = pi_off + kTileBytes;        // 64 floats: sc, mag, cf, bscale
+  static constexpr int part_off = cb_off + 64 * 4;          // float [2][kRows]: the halves' sums of squares
+  static constexpr int bar_off = part_off + 2 * kRows * 4;  // x[2], params, mma
+  static constexpr int tmem_off = bar_off + 4 * 8;
+  static constexpr int bytes = tmem_off + 16;
+  static constexpr int alloc = bytes + 1024;
+};
+static_assert(2 * (SmemM::alloc + 1024) <= 228 * 1024, "two CTAs per SM");
+
+// barrier of the two warps (w, w + 4) whose threads share the rows 32 (w & 3) ..
+__device__ __forceinline__ void pair_sync(int warp) {
+  asm volatile("bar.sync %0, %1;" ::"r"(1 + (warp & 3)), "r"(64) : "memory");
+}
+
+template <typename T, int BITS, int MODE>
+__global__ void __launch_bounds__(kThreadsM, 2)
+    tq_mse_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_pi,
+                  const __grid_constant__ CUtensorMap map_o, TqArgs a) {
+  using HR = HalfRow<BITS>;
+  using SM = SmemM;
+  constexpr int H = Codes<BITS>::H, CPW = HR::CPW, NWH = HR::NWH, WH = HR::WH;
+  constexpr bool kQ = MODE != TQ_DQ_MSE;
+  constexpr bool kOut = MODE != TQ_MSE_Q;
+  constexpr uint32_t kNcols = 256;
+  constexpr uint32_t kIdPi = umma_idesc_f16(IsBf16<T>::value, IsBf16<T>::value, false, D, kRows);  // X Pi^T
+  constexpr uint32_t kIdPiT = umma_idesc_f16(IsBf16<T>::value, IsBf16<T>::value, true, D, kRows);  // C Pi
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* s_buf = smem + SM::buf_off;
+  uint8_t* s_pi = smem + SM::pi_off;
+  float* s_sc = reinterpret_cast<float*>(smem + SM::cb_off);
+  float* s_mag = s_sc + 16;
+  float* s_cf = s_sc + 32;
+  float* s_bscale = s_sc + 48;
+  float* s_part = reinterpret_cast<float*>(smem + SM::part_off);
+  uint64_t* bar_x = reinterpret_cast<uint64_t*>(smem + SM::bar_off);  // [2]
+  uint64_t* bar_p = bar_x + 2;
+  uint64_t* bar_m = bar_x + 3;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + SM::tmem_off);
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int r = tid & (kRows - 1);  // row in the tile = TMEM lane
+  const int h = warp >> 2;          // half of the columns
+  const int64_t n = a.n;
+  const int64_t ntiles = (n + kRows - 1) / kRows;
+  const uint32_t buf_s = smem_u32(s_buf), pi_s = smem_u32(s_pi);
+  // 8-byte code-word accesses when every half row's words start 8-byte aligned
+  const bool vec = (a.ldc & 1) == 0 &&
+                   ((reinterpret_cast<uintptr_t>(kQ ? (const void*)a.codes_out : (const void*)a.codes_in) & 7u) == 0);
+
+  if (tid == 0) {
+    if (kQ) tma_prefetch_desc(&map_x);
+    tma_prefetch_desc(&map_pi);
+    if (kOut) tma_prefetch_desc(&map_o);
+    mbar_init(bar_x, 1);
+    mbar_init(bar_x + 1, 1);
+    mbar_init(bar_p, 1);
+    mbar_init(bar_m, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) tmem_alloc(s_tmem, kNcols);
+  build_consts<BITS>(a.centroids, s_sc, s_mag, s_cf, s_bscale);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+  const uint32_t tm_y = tmem + lane_off + 64u * (uint32_t)h, tm_x = tmem + 128u + lane_off + 64u * (uint32_t)h;
+
+  if (tid == 0) {
+    mbar_arrive_expect_tx(bar_p, kTileBytes);
+    for (int b = 0; b < 2; ++b) tma_load_2d(s_pi + b * kBoxBytes, &map_pi, b * 64, 0, bar_p);
+    if (kQ && (int64_t)blockIdx.x < ntiles) {
+      mbar_arrive_expect_tx(bar_x, kTileBytes);
+      for (int b = 0; b < 2; ++b)
+        tma_load_2d(s_buf + b * kBoxBytes, &map_x, b * 64, (int32_t)((int64_t)blockIdx.x * kRows), bar_x);
+    }
+  }
+  bool ok = __syncthreads_and(mbar_wait(bar_p, 0, a.status));
+  uint32_t par_m = 0;
+  const float Bs = *s_bscale;
+  float dl[H > 1 ? H - 1 : 1], sc[H > 1 ? H - 1 : 1];
+#pragma unroll
+  for (int j = 0; j < H - 1; ++j) {
+    dl[j] = __fsub_rn(s_mag[j + 1], s_mag[j]);
+    sc[j] = s_sc[j];
+  }
+  const float mn0 = s_mag[0];
+
+  auto mma = [&](uint32_t a_s, uint32_t tm_d, uint32_t idesc, bool mn_b) {  // thread 0
+    tc_fence_after();
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t akoff = (uint32_t)((kk >> 2) * kBoxBytes + (kk & 3) * 32);
+      const uint32_t bkoff = mn_b ? (uint32_t)(kk * 16 * 128) : akoff;
+      umma_f16(tm_d, umma_desc_sw128(a_s + akoff, 16, 1024),
+               umma_desc_sw128(pi_s + bkoff, mn_b ? kBoxBytes : 16, 1024), idesc, kk > 0);
+    }
+    umma_commit(bar_m);
+  };
+  auto wait_mma = [&]() {
+    const bool w = mbar_wait(bar_m, par_m, a.status);
+    par_m ^= 1;
+    tc_fence_after();
+    return w;
+  };
+
+  int k = 0;
+  for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++k) {
+    const int s = k & 1;
+    uint8_t* tbuf = s_buf + s * kTileBytes;
+    const uint32_t tbuf_s = buf_s + (uint32_t)(s * kTileBytes);
+    const int64_t row0 = tile * kRows;
+    const int rows = (int)(n - row0 < (int64_t)kRows ? n - row0 : (int64_t)kRows);
+    const int64_t next = tile + gridDim.x;
+    const bool live = r < rows;
+    const int64_t row = row0 + r;
+    float nrm = 0.f;
+    uint32_t wc[WH];
+#pragma unroll
+    for (int w = 0; w < WH; ++w) wc[w] = 0u;
+    auto put = [&](int j, const float* v) {
+      *reinterpret_cast<uint4*>(tbuf + sw128_chunk(r, j, kBoxBytes)) = Elem<T>::pack(v);
+    };
+    auto store_outputs = [&]() {  // code words and norm of this half row
+      if (!kQ || !live) return;
+      const int64_t orow = a.out_rows ? a.out_rows[row] : row;
+      if (a.codes_out) {
+        uint32_t* dst = a.codes_out + orow * a.ldc + WH * h;
+        if (vec) {
+#pragma unroll
+          for (int w = 0; w < WH; w += 2) *reinterpret_cast<uint2*>(dst + w) = make_uint2(wc[w], wc[w + 1]);
+        } else {
+#pragma unroll
+          for (int w = 0; w < WH; ++w) dst[w] = wc[w];
+        }
+      }
+      if (h == 0 && a.norms_out) a.norms_out[orow * a.ldn] = nrm;
+    };
+
+    if constexpr (kQ) {
+      // every thread reads x from the tile (its half's sum of squares), so every thread waits for it
+      const bool landed = mbar_wait(bar_x + s, (uint32_t)(k >> 1) & 1u, a.status);
+      if (!landed) ok = false;
+      if (tid == 0 && landed) mma(tbuf_s, tmem, kIdPi, false);  // y = Pi x per row
+      // this half's sum of squares from the tile while the MMA runs
+      float2 acc[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float f[8];
+        Elem<T>::unpack(*reinterpret_cast<const uint4*>(tbuf + sw128_chunk(r, 8 * h + j, kBoxBytes)), f);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 v = make_float2(f[2 * q], f[2 * q + 1]);
+          acc[q] = __ffma2_rn(v, v, acc[q]);
+        }
+      }
+      s_part[h * kRows + r] =
+          ((acc[0].x + acc[1].x) + (acc[2].x + acc[3].x)) + ((acc[0].y + acc[1].y) + (acc[2].y + acc[3].y));
+      if (!wait_mma()) ok = false;
+      pair_sync(warp);
+      nrm = sqrtf(s_part[r] + s_part[kRows + r]);
+      if (tid == 0 && next < ntiles) {
+        // the other buffer's x_hat store (previous tile) has been read: load the next tile's x into it
+        bulk_wait_read<0>();
+        mbar_arrive_expect_tx(bar_x + (s ^ 1), kTileBytes);
+        for (int b = 0; b < 2; ++b)
+          tma_load_2d(s_buf + (s ^ 1) * kTileBytes + b * kBoxBytes, &map_x, b * 64, (int32_t)(next * kRows),
+                      bar_x + (s ^ 1));
+      }
+      const float srow = nrm > 0.f ? __fdiv_rn(Bs, nrm) : 0.f;
+      const float shift = -fmaf(kShift, nrm, 0x1p-126f);
+      float win[NWH];
+#pragma unroll
+      for (int w = 0; w < NWH; ++w) win[w] = kWindow0;
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        float y[32];
+        tmem_ld32(tm_y + 32u * (uint32_t)cc, y);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+        float w_out[8];
+#pragma unroll
+        for (int i = 8 * q; i < 8 * q + 8; i += 2) {
+          const float2 Y = make_float2(y[i] + shift, y[i + 1] + shift);
+          float2 m2 = make_float2(mn0, mn0), cnt = make_float2(0.5f, 0.5f);
+#pragma unroll
+          for (int j = 0; j < H - 1; ++j) {
+            const float2 st = make_float2(fma_sat(fabsf(Y.x), srow, sc[j]), fma_sat(fabsf(Y.y), srow, sc[j]));
+            m2 = __ffma2_rn(st, make_float2(dl[j], dl[j]), m2);
+            cnt = __fadd2_rn(cnt, st);
+          }
+          const float2 sg = make_float2(sign_one(Y.x), sign_one(Y.y));
+          const float2 code = __ffma2_rn(sg, cnt, make_float2(H - 0.5f, H - 0.5f));
+          const int k0 = 32 * cc + i, k1 = k0 + 1;  // code index in the half row
+          win[k0 / CPW] = fmaf(code.x, (float)(1u << (BITS * (k0 % CPW))), win[k0 / CPW]);
+          win[k1 / CPW] = fmaf(code.y, (float)(1u << (BITS * (k1 % CPW))), win[k1 / CPW]);
+          if constexpr (kOut) {
+            const float2 chat = __fmul2_rn(m2, sg);  // unit-scale centroid
+            w_out[i - 8 * q] = chat.x;
+            w_out[i + 1 - 8 * q] = chat.y;
+          }
+        }
+        if constexpr (kOut) put(8 * h + 4 * cc + q, w_out);
+        }
+      }
+#pragma unroll
+      for (int w = 0; w < NWH; ++w) {
+        const uint32_t v = __float_as_uint(win[w]) & 0x7fffffu;
+        const int bo = w * CPW * BITS;
+        wc[bo >> 5] |= v << (bo & 31);
+        if ((bo & 31) + CPW * BITS > 32 && (bo >> 5) + 1 < WH) wc[(bo >> 5) + 1] |= v >> (32 - (bo & 31));
+      }
+    } else {
+      if (tid == 0) bulk_wait_read<1>();  // this buffer's store (two tiles back) has been read
+      if (live) {
+        const uint32_t* src = a.codes_in + row * a.ldc + WH * h;
+        if (vec) {
+#pragma unroll
+          for (int w = 0; w < WH; w += 2) {
+            const uint2 v = __ldg(reinterpret_cast<const uint2*>(src + w));
+            wc[w] = v.x, wc[w + 1] = v.y;
+          }
+        } else {
+#pragma unroll
+          for (int w = 0; w < WH; ++w) wc[w] = __ldg(src + w);
+        }
+        nrm = __ldg(a.norms_in + row * a.ldn);
+      }
+      auto code_at = [&](int kl) -> uint32_t {
+        const int bit = kl * BITS, word = bit >> 5, sh = bit & 31;
+        uint32_t v = wc[word] >> sh;
+        if (sh + BITS > 32) v |= wc[word + 1] << (32 - sh);
+        return v & ((1u << BITS) - 1u);
+      };
+      __syncthreads();  // the buffer is free
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = s_cf[code_at(32 * cc + i)];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) put(8 * h + 4 * cc + q, &v[8 * q]);
+      }
+    }
+
+    if constexpr (kOut) {
+      fence_proxy_async_smem();
+      tc_fence_before();
+      ok = __syncthreads_and(ok);
+      if (!ok) break;
+      if (tid == 0) mma(tbuf_s, tmem + 128u, kIdPiT, true);  // Pi^T c_hat per row
+      store_outputs();
+      if (!wait_mma()) ok = false;
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        float v[32];
+        tmem_ld32(tm_x + 32u * (uint32_t)cc, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] *= nrm;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) put(8 * h + 4 * cc + q, &v[8 * q]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      ok = __syncthreads_and(ok);
+      if (!ok) break;
+      if (tid == 0) {
+        for (int b = 0; b < 2; ++b) tma_store_2d(&map_o, b * 64, (int32_t)row0, tbuf + b * kBoxBytes);
+        bulk_commit();
+      }
+    } else {
+      store_outputs();
+      tc_fence_before();  // this tile's TMEM reads precede the next tile's product
+      ok = __syncthreads_and(ok);
+    }
+  }
+  if (tid == 0) bulk_wait_all<0>();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kNcols);
+  }
+}
+
 }  // namespace tq
 
 // ============================================================================ launch
@@ -461,6 +770,33 @@ static cudaError_t launch_tq_t(const CUtensorMap& mx, const CUtensorMap& mp, con
   return cudaGetLastError();
 }
 
+template <typename T, int BITS, int MODE>
+static cudaError_t launch_tq_mse_t(const CUtensorMap& mx, const CUtensorMap& mp, const CUtensorMap& mo,
+                                   const TqArgs& a, cudaStream_t st, int num_sms) {
+  auto kern = tq::tq_mse_kernel<T, BITS, MODE>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, tq::SmemM::alloc);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int64_t ntiles = (a.n + tq::kRows - 1) / tq::kRows;
+  const int64_t grid = std::min<int64_t>(ntiles, (int64_t)num_sms * 2);
+  kern<<<(unsigned)grid, tq::kThreadsM, tq::SmemM::alloc, st>>>(mx, mp, mo, a);
+  return cudaGetLastError();
+}
+
+template <typename T, int MODE>
+static cudaError_t tq_mse_by_bits(int bits, const CUtensorMap& mx, const CUtensorMap& mp, const CUtensorMap& mo,
+                                  const TqArgs& a, cudaStream_t st, int sms) {
+  switch (bits) {
+    case 1: return launch_tq_mse_t<T, 1, MODE>(mx, mp, mo, a, st, sms);
+    case 2: return launch_tq_mse_t<T, 2, MODE>(mx, mp, mo, a, st, sms);
+    case 3: return launch_tq_mse_t<T, 3, MODE>(mx, mp, mo, a, st, sms);
+    default: return launch_tq_mse_t<T, 4, MODE>(mx, mp, mo, a, st, sms);
+  }
+}
+
 template <typename T, int MODE>
 static cudaError_t tq_by_bits(int bits, const CUtensorMap& mx, const CUtensorMap& mp, const CUtensorMap& mt,
                               const CUtensorMap& mo, const TqArgs& a, cudaStream_t st, int sms) {
@@ -476,10 +812,10 @@ template <typename T>
 static cudaError_t tq_by_mode(int mode, int bits, const CUtensorMap& mx, const CUtensorMap& mp, const CUtensorMap& mt,
                               const CUtensorMap& mo, const TqArgs& a, cudaStream_t st, int sms) {
   switch (mode) {
-    case TQ_MSE_Q: return tq_by_bits<T, TQ_MSE_Q>(bits, mx, mp, mt, mo, a, st, sms);
-    case TQ_MSE_QDQ: return tq_by_bits<T, TQ_MSE_QDQ>(bits, mx, mp, mt, mo, a, st, sms);
+    case TQ_MSE_Q: return tq_mse_by_bits<T, TQ_MSE_Q>(bits, mx, mp, mo, a, st, sms);
+    case TQ_MSE_QDQ: return tq_mse_by_bits<T, TQ_MSE_QDQ>(bits, mx, mp, mo, a, st, sms);
     case TQ_PROD_Q: return tq_by_bits<T, TQ_PROD_Q>(bits, mx, mp, mt, mo, a, st, sms);
-    case TQ_DQ_MSE: return tq_by_bits<T, TQ_DQ_MSE>(bits, mx, mp, mt, mo, a, st, sms);
+    case TQ_DQ_MSE: return tq_mse_by_bits<T, TQ_DQ_MSE>(bits, mx, mp, mo, a, st, sms);
     default: return tq_by_bits<T, TQ_DQ_PROD>(bits, mx, mp, mt, mo, a, st, sms);
   }
 }

@@ -183,3 +183,10 @@ def test_strided_code_rows(ld, off):
     xd = kvrq.pq_dequantize(view, D, pi_d, c_d, out_dtype=torch.float16)
     torch.cuda.synchronize()
     assert torch.equal(xd.view(torch.int16), x0.view(torch.int16))
+
+
+def test_many_tiles_per_cta():
+    """200,003 rows: five or six tiles per CTA through both tile buffers, ragged last tile."""
+    x = synth.lognormal(200003, D, seed=13, dtype=torch.float16).cuda()
+    rows = np.unique(np.concatenate([np.random.default_rng(4).choice(200003, 2048, replace=False), [0, 200002]]))
+    _check(x, rows)

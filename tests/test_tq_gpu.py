@@ -110,3 +110,28 @@ def test_zero_rows_tq():
     zc = ocodes.unpack(words_u32(codes)[[3, 130]], D, bits)
     assert np.all(zc == (1 << (bits - 1)) - 1)  # y = 0 takes the lower middle code
     assert np.all(to_f64(xhat)[[3, 130]] == 0) and np.all(to_f64(norms)[[3, 130]] == 0)
+
+
+@pytest.mark.parametrize("dt", [torch.float16, torch.bfloat16])
+def test_mse_many_tiles_per_cta(dt):
+    """200,003 rows: every CTA of the d = 128 kernel takes five or six 128-row tiles, so both tile buffers
+    and the loads issued during the previous tile are exercised, with a ragged last tile. Quantize-only and
+    dequantize-only launches must reproduce the fused one bit for bit."""
+    bits = 3
+    n = 200003
+    pi64, c64, _, pi_d, c_d, _ = _params(bits, dt)
+    x = synth.lognormal(n, D, seed=12, dtype=dt).cuda()
+    codes, norms, xhat = kvrq.tq_quantize_dequantize_mse(x, pi_d, c_d, bits)
+    torch.cuda.synchronize()
+    kvrq.device_status()
+    rows = np.unique(np.concatenate([np.random.default_rng(9).choice(n, 3000, replace=False), [0, 127, 128, n - 1]]))
+    ref = tq.mse_quantize(to_f64(x)[rows], pi64, c64, bits)
+    nb, bad = compare_codes(words_u32(codes)[rows], ref, D, bits, c64)
+    assert np.allclose(to_f64(norms)[rows], ref["norms"], rtol=1e-5)
+    xref = tq.mse_dequantize(ref["words"], ref["norms"], pi64, c64, bits, D)
+    _rows_close(to_f64(xhat)[rows], xref, XHAT_RTOL[dt], skip=bad)
+    c2, n2 = kvrq.tq_quantize_mse(x, pi_d, c_d, bits)
+    assert torch.equal(c2, codes) and torch.equal(n2, norms)
+    xd = kvrq.tq_dequantize(codes, norms, D, pi_d, c_d, bits)
+    torch.cuda.synchronize()
+    assert torch.equal(xd, xhat)
