@@ -9,16 +9,19 @@
 //   (b-1)-bit mse codes, r = y - c_hat (rotated residual), gamma = ||r||,
 //   s = sign(T r) with S = T Pi, x_hat = ||x|| Pi^T (c_hat + sqrt(pi/2)/m gamma T^T s)   (prod)
 //
-// B200 design. A persistent CTA of 128 threads owns 128-row tiles; Pi (and T)
-// stay resident in shared memory as 128-byte-swizzled tiles that serve as the
-// MMA B operand both K-major (y = Pi u, T r) and MN-major (Pi^T c, T^T s).
-// The x tile arrives by TMA in the same swizzled layout and is the A operand
-// directly. One thread issues tcgen05.mma (M = 128, N = d, K = 16 steps) into
-// TMEM; every thread then reads its own row (one TMEM lane) with tcgen05.ld,
-// quantizes on the FMA pipe, and writes the next A operand (centroids, or the
-// residual for the sketch) back into the same tile buffer, which finally holds
-// x_hat for the TMA store. Two CTAs share an SM (256 TMEM columns each) so one
-// CTA's MMAs overlap the other's epilogue.
+// B200 design. Pi (and T) stay resident in shared memory as 128-byte-swizzled tiles
+// that serve as the MMA B operand both K-major (y = Pi u, T r) and MN-major (Pi^T c,
+// T^T s). The x tile arrives by TMA in the same swizzled layout and is the A operand
+// directly. One thread issues tcgen05.mma (M = 128, N = d, K = 16 steps) into TMEM;
+// the threads then read their rows (one TMEM lane per row) with tcgen05.ld, quantize
+// on the FMA pipe, and write the next A operand (centroids, or the residual for the
+// sketch) back into the tile buffer, which finally holds x_hat for the TMA store.
+//  * tq_mse_kernel (the mse modes): 256 threads, two per row (64 columns each), two
+//    tile buffers so the next tile's load lands while this tile is quantized.
+//  * tq_kernel (the prod modes, whose Pi and T leave room for one tile buffer at two
+//    CTAs per SM): 128 threads, one per row, one tile at a time.
+// Two CTAs share an SM (256 TMEM columns each), so one CTA's MMAs overlap the other's
+// epilogue.
 
 #include <cuda_runtime.h>
 
