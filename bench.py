@@ -91,6 +91,29 @@ def kernel_source_hash(spec):
     return hashlib.sha256(text).hexdigest()[:16]
 
 
+def build_identity():
+    """What was measured: the git commit when the tree has its history (a snapshot copied without .git has
+    none), and a SHA-256 prefix of the library's sources, the public header and this script, which names
+    the build either way."""
+    import hashlib
+    import subprocess
+
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "kv_cache_vector_rq_b200", "csrc")
+    files = sorted(os.path.join(csrc, f) for f in os.listdir(csrc) if f.endswith((".cu", ".cuh", ".h", ".cpp")))
+    files += [os.path.join(ROOT, "include", "kvrq.h"), os.path.abspath(__file__)]
+    for f in files:
+        h.update(os.path.relpath(f, ROOT).encode() + b"\0" + open(f, "rb").read())
+    sha = None
+    try:
+        out = subprocess.run(["git", "-C", ROOT, "rev-parse", "HEAD"], capture_output=True, text=True, timeout=10)
+        if out.returncode == 0:
+            sha = out.stdout.strip() or None
+    except (OSError, subprocess.SubprocessError):
+        sha = None
+    return {"git_sha": sha, "source_sha256": h.hexdigest()[:16]}
+
+
 def recorded_traffic(kernel):
     """Per-launch DRAM bytes of `kernel` from profiles/traffic.txt, or None when that record is missing or the
     kernel's source changed since the counters were taken (the record keeps a SHA-256 prefix of the source)."""
@@ -904,8 +927,8 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
             "config": {"workload": "65536 x d128 fp16 KV vectors (LogNormal(0,0.5) norms, 4 outlier channels x10), "
-                                   "fused quantize+dequantize, RotorQuant and TurboQuant-mse b=2,3,4; "
-                                   "headline RotorQuant b=3",
+                                   "fused quantize+dequantize, RotorQuant and TurboQuant-mse b=2,3,4, PolarQuant "
+                                   "4-2-2-2; headline RotorQuant b=3",
                        "n_vectors_per_gpu": N_VEC, "d": D, "io_dtype": "fp16",
                        "l2": "inputs larger than L2: step k runs on batch set k mod %d (%d independent batches, "
                              "%.0f MB with outputs); each leg's K launches replayed back to back from a CUDA graph"
@@ -921,6 +944,7 @@ def main():
             "e2e": {"value": whole_job_rate(N_VEC, world, e2e) / 1e6, "unit": "Mvec/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms": e2e},
             "gpu_launches": launches,
+            "build": build_identity(),
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
             "boundary_ties": ties if rank == 0 else None,
