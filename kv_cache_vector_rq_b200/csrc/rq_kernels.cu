@@ -369,7 +369,7 @@ __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint32_t* s_codes = reinterpret_cast<uint32_t*>(smem + SM::codes_off);
   float* s_lut = reinterpret_cast<float*>(smem + SM::lut_off);
-  const float4* s_mp4 = reinterpret_cast<const float4*>(smem + SM::mp_off);
+  const uint32_t mp_a = smem_u32(smem + SM::mp_off);  // the group pairs' sandwich matrices
   float* s_sc = reinterpret_cast<float*>(smem + SM::cb_off);
   float* s_mag = s_sc + 16;
   float* s_cf = s_sc + 32;
@@ -415,6 +415,10 @@ __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
               &w_bar[STAGES + c]);
   };
 
+  // Launched with programmatic stream serialization: the CTA may be resident before the previous
+  // kernel of the stream has finished; every global access below follows this wait.
+  grid_dep_wait();
+  grid_dep_launch();
   // Each warp sets up its own barriers and starts its first copies before the
   // CTA forms its tables, so the rotor loads overlap the first sub-tile's copy.
   if (lane == 0) {
@@ -459,6 +463,7 @@ __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
       else return tb_a + TL::chunk(lane, j);
     };
     uint32_t* stage_codes = w_codes + (kIn ? 0 : cs * (SM::codes_stage / 4));
+    const uint32_t stage_a = smem_u32(stage_codes) + (uint32_t)(lane * W * 4);  // this lane's staged words
 
     // ---------------------------------------------------------------- inputs
     bool ok = true;
@@ -631,9 +636,9 @@ __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
       float2 M[10];
 #pragma unroll
       for (int q = 0; q < 5; ++q) {
-        const float4 t = s_mp4[p * 5 + q];
-        M[2 * q] = make_float2(t.x, t.y);
-        M[2 * q + 1] = make_float2(t.z, t.w);
+        const uint4 t = lds_v4(mp_a + (uint32_t)((p * 5 + q) * 16));
+        M[2 * q] = make_float2(__uint_as_float(t.x), __uint_as_float(t.y));
+        M[2 * q + 1] = make_float2(__uint_as_float(t.z), __uint_as_float(t.w));
       }
       float2 C[3];
       if constexpr (kIn) {
@@ -681,7 +686,7 @@ __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
           const int last_code = ((32 * wi + 31) / BITS) < NC ? (32 * wi + 31) / BITS : NC - 1;
           const int win_end = ((last_code / CPW) + 1) * CPW < NC ? ((last_code / CPW) + 1) * CPW : NC;
           const int prev_done = PC * p < NC ? PC * p : NC;
-          if (win_end <= done && win_end > prev_done) stage_codes[lane * W + wi] = wc[wi];
+          if (win_end <= done && win_end > prev_done) sts_u32(stage_a + (uint32_t)(wi * 4), wc[wi]);
         }
       } else {
 #pragma unroll
@@ -1169,8 +1174,7 @@ static cudaError_t launch_row_s(const CUtensorMap& mx, const CUtensorMap& mo, co
   // ring: every CTA starts with at least one sub-tile (its warp 0 takes sub-tile blockIdx.x)
   const int64_t want = SH::kRing ? nsub : (nsub + SH::kWarps - 1) / SH::kWarps;
   const int64_t grid = std::min<int64_t>(want, (int64_t)num_sms * blocks_per_sm);
-  kern<<<(unsigned)grid, SH::kRows, SM::alloc, st>>>(mx, mo, a);
-  return cudaGetLastError();
+  return launch_pdl(kern, (unsigned)grid, SH::kRows, SM::alloc, st, mx, mo, a);
 }
 
 int rq_row_box_rows() { return row::kWR; }

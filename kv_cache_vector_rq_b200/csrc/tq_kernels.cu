@@ -515,6 +515,9 @@ __global__ void __launch_bounds__(kThreadsM, 2)
   const bool vec = (a.ldc & 1) == 0 &&
                    ((reinterpret_cast<uintptr_t>(kQ ? (const void*)a.codes_out : (const void*)a.codes_in) & 7u) == 0);
 
+  // launched with programmatic stream serialization: every global access follows this wait
+  grid_dep_wait();
+  grid_dep_launch();
   if (tid == 0) {
     if (kQ) tma_prefetch_desc(&map_x);
     tma_prefetch_desc(&map_pi);
@@ -785,8 +788,7 @@ static cudaError_t launch_tq_mse_t(const CUtensorMap& mx, const CUtensorMap& mp,
   }
   const int64_t ntiles = (a.n + tq::kRows - 1) / tq::kRows;
   const int64_t grid = std::min<int64_t>(ntiles, (int64_t)num_sms * 2);
-  kern<<<(unsigned)grid, tq::kThreadsM, tq::SmemM::alloc, st>>>(mx, mp, mo, a);
-  return cudaGetLastError();
+  return launch_pdl(kern, (unsigned)grid, tq::kThreadsM, tq::SmemM::alloc, st, mx, mp, mo, a);
 }
 
 template <typename T, int MODE>
