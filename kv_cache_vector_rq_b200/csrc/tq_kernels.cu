@@ -28,6 +28,7 @@
 #include <cstdlib>
 #include <type_traits>
 
+#include "bisect.cuh"
 #include "kvrq_device.cuh"
 #include "tq_launch.h"
 
@@ -546,8 +547,6 @@ __global__ void __launch_bounds__(kThreadsM, 2)
         tma_load_2d(s_buf + b * kBoxBytes, &map_x, b * 64, (int32_t)((int64_t)blockIdx.x * kRows), bar_x);
     }
   }
-  bool ok = __syncthreads_and(mbar_wait(bar_p, 0, a.status));
-  uint32_t par_m = 0;
   const float Bs = *s_bscale;
   float dl[H > 1 ? H - 1 : 1], sc[H > 1 ? H - 1 : 1];
 #pragma unroll
@@ -556,6 +555,24 @@ __global__ void __launch_bounds__(kThreadsM, 2)
     sc[j] = s_sc[j];
   }
   const float mn0 = s_mag[0];
+  // b >= 3: binary search over the boundaries (one saturating step per code bit); the centroid table
+  // of the dequantize side is rebuilt from the same magnitude sequence, so both sides give the same bits
+  constexpr bool kBisect = BITS >= 3;
+  Bisect<kBisect ? BITS : 3> bs;
+  if constexpr (kBisect) {
+    bs.thresholds(sc);
+    bs.magnitudes(s_mag);
+  }
+  bool ok = mbar_wait(bar_p, 0, a.status);
+  if constexpr (kBisect) {
+    if (tid < H) {
+      const float m = bs.mag(tid);
+      s_cf[H + tid] = m;
+      s_cf[H - 1 - tid] = -m;
+    }
+  }
+  ok = __syncthreads_and(ok);
+  uint32_t par_m = 0;
 
   auto mma = [&](uint32_t a_s, uint32_t tm_d, uint32_t idesc, bool mn_b) {  // thread 0
     tc_fence_after();
@@ -656,11 +673,15 @@ __global__ void __launch_bounds__(kThreadsM, 2)
         for (int i = 8 * q; i < 8 * q + 8; i += 2) {
           const float2 Y = make_float2(y[i] + shift, y[i + 1] + shift);
           float2 m2 = make_float2(mn0, mn0), cnt = make_float2(0.5f, 0.5f);
+          if constexpr (kBisect) {
+            bs(make_float2(fabsf(Y.x), fabsf(Y.y)), srow, m2, cnt);
+          } else {
 #pragma unroll
-          for (int j = 0; j < H - 1; ++j) {
-            const float2 st = make_float2(fma_sat(fabsf(Y.x), srow, sc[j]), fma_sat(fabsf(Y.y), srow, sc[j]));
-            m2 = __ffma2_rn(st, make_float2(dl[j], dl[j]), m2);
-            cnt = __fadd2_rn(cnt, st);
+            for (int j = 0; j < H - 1; ++j) {
+              const float2 st = make_float2(fma_sat(fabsf(Y.x), srow, sc[j]), fma_sat(fabsf(Y.y), srow, sc[j]));
+              m2 = __ffma2_rn(st, make_float2(dl[j], dl[j]), m2);
+              cnt = __fadd2_rn(cnt, st);
+            }
           }
           const float2 sg = make_float2(sign_one(Y.x), sign_one(Y.y));
           const float2 code = __ffma2_rn(sg, cnt, make_float2(H - 0.5f, H - 0.5f));
