@@ -74,7 +74,8 @@ def measured_peaks():
 
 def kernel_source_hash(spec):
     """SHA-256 prefix of a kernel's source: `file#ns` hashes the text of `namespace ns { ... }  // namespace ns`
-    in that file together with the device helper header it includes; a plain path hashes the whole file."""
+    in that file together with the device headers it includes (helpers and the bisection quantizer); a plain
+    path hashes the whole file."""
     import hashlib
 
     path, _, ns = spec.partition("#")
@@ -87,7 +88,9 @@ def kernel_source_hash(spec):
         b = text.find(("}  // namespace %s" % ns).encode())
         if a < 0 or b < a:
             return None
-        text = text[a:b] + open(os.path.join(os.path.dirname(src), "kvrq_device.cuh"), "rb").read()
+        text = text[a:b]
+        for hdr in ("kvrq_device.cuh", "bisect.cuh"):
+            text += open(os.path.join(os.path.dirname(src), hdr), "rb").read()
     return hashlib.sha256(text).hexdigest()[:16]
 
 

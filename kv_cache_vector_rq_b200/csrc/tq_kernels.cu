@@ -777,6 +777,272 @@ __global__ void __launch_bounds__(kThreadsM, 2)
   }
 }
 
+// ============================================================================ prod, two threads per row
+// TurboQuant-prod quantize at d = 128 with 256-thread CTAs, two threads per row as in tq_mse_kernel.
+// Pi and T stay resident (64 KB), which leaves one tile buffer at two CTAs per SM; the sketch's A
+// operand, fp16(2^8 r), goes to tensor memory (64 columns beside the 128 of y), so the x buffer is
+// free as soon as the first product and the norm pass have read it, and the next tile's load is
+// issued then: it lands while this tile is quantized, sketched and stored. T r reuses y's columns.
+struct SmemP {
+  static constexpr int buf_off = 0;                          // one tile
+  static constexpr int pi_off = kTileBytes;
+  static constexpr int t_off = 2 * kTileBytes;
+  static constexpr int cb_off = 3 * kTileBytes;              // 64 floats: sc, mag, cf, bscale
+  static constexpr int part_off = cb_off + 64 * 4;           // float [2][kRows]: halves' sums of squares
+  static constexpr int gpart_off = part_off + 2 * kRows * 4;  // float [2][kRows]: halves' ||r||^2
+  static constexpr int bar_off = gpart_off + 2 * kRows * 4;  // x, params, mma
+  static constexpr int tmem_off = bar_off + 3 * 8;
+  static constexpr int bytes = tmem_off + 16;
+  static constexpr int alloc = bytes + 1024;
+};
+static_assert(2 * (SmemP::alloc + 1024) <= 228 * 1024, "two CTAs per SM");
+
+template <typename T, int BITS>
+__global__ void __launch_bounds__(kThreadsM, 2)
+    tq_prod_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_pi,
+                   const __grid_constant__ CUtensorMap map_t, TqArgs a) {
+  using HR = HalfRow<BITS>;
+  using SM = SmemP;
+  constexpr int H = Codes<BITS>::H, CPW = HR::CPW, NWH = HR::NWH, WH = HR::WH;
+  constexpr uint32_t kNcols = 256;  // y (then T r): 0 .. 127; the sketch operand: 128 .. 191
+  constexpr uint32_t kIdPi = umma_idesc_f16(IsBf16<T>::value, IsBf16<T>::value, false, D, kRows);  // X Pi^T
+  constexpr uint32_t kIdT = umma_idesc_f16(false, false, false, D, kRows);                          // rho T^T
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* s_buf = smem + SM::buf_off;
+  uint8_t* s_pi = smem + SM::pi_off;
+  uint8_t* s_t = smem + SM::t_off;
+  float* s_sc = reinterpret_cast<float*>(smem + SM::cb_off);
+  float* s_mag = s_sc + 16;
+  float* s_cf = s_sc + 32;
+  float* s_bscale = s_sc + 48;
+  float* s_part = reinterpret_cast<float*>(smem + SM::part_off);
+  float* s_gpart = reinterpret_cast<float*>(smem + SM::gpart_off);
+  uint64_t* bar_x = reinterpret_cast<uint64_t*>(smem + SM::bar_off);
+  uint64_t* bar_p = bar_x + 1;
+  uint64_t* bar_m = bar_x + 2;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + SM::tmem_off);
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int r = tid & (kRows - 1);  // row in the tile = TMEM lane
+  const int h = warp >> 2;          // half of the columns
+  const int64_t n = a.n;
+  const int64_t ntiles = (n + kRows - 1) / kRows;
+  const uint32_t buf_s = smem_u32(s_buf), pi_s = smem_u32(s_pi), t_s = smem_u32(s_t);
+  constexpr int NS = D / 32;  // sign words per row
+  const bool vec = (a.ldc & 1) == 0 && (reinterpret_cast<uintptr_t>(a.codes_out) & 7u) == 0;
+  const bool svec = (a.lds & 1) == 0 && (reinterpret_cast<uintptr_t>(a.signs_out) & 7u) == 0;
+
+  // launched with programmatic stream serialization: every global access follows this wait
+  grid_dep_wait();
+  grid_dep_launch();
+  if (tid == 0) {
+    tma_prefetch_desc(&map_x);
+    tma_prefetch_desc(&map_pi);
+    tma_prefetch_desc(&map_t);
+    mbar_init(bar_x, 1);
+    mbar_init(bar_p, 1);
+    mbar_init(bar_m, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) tmem_alloc(s_tmem, kNcols);
+  build_consts<BITS>(a.centroids, s_sc, s_mag, s_cf, s_bscale);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+  const uint32_t tm_y = tmem + lane_off + 64u * (uint32_t)h;                // this half's y (then T r) columns
+  const uint32_t tm_rho = tmem + 128u + lane_off + 32u * (uint32_t)h;       // this half's sketch operand words
+
+  if (tid == 0) {
+    mbar_arrive_expect_tx(bar_p, 2 * kTileBytes);
+    for (int b = 0; b < 2; ++b) tma_load_2d(s_pi + b * kBoxBytes, &map_pi, b * 64, 0, bar_p);
+    for (int b = 0; b < 2; ++b) tma_load_2d(s_t + b * kBoxBytes, &map_t, b * 64, 0, bar_p);
+    if ((int64_t)blockIdx.x < ntiles) {
+      mbar_arrive_expect_tx(bar_x, kTileBytes);
+      for (int b = 0; b < 2; ++b)
+        tma_load_2d(s_buf + b * kBoxBytes, &map_x, b * 64, (int32_t)((int64_t)blockIdx.x * kRows), bar_x);
+    }
+  }
+  const float Bs = *s_bscale;
+  float dl[H > 1 ? H - 1 : 1], sc[H > 1 ? H - 1 : 1];
+#pragma unroll
+  for (int j = 0; j < H - 1; ++j) {
+    dl[j] = __fsub_rn(s_mag[j + 1], s_mag[j]);
+    sc[j] = s_sc[j];
+  }
+  const float mn0 = s_mag[0];
+  constexpr bool kBisect = BITS >= 3;
+  Bisect<kBisect ? BITS : 3> bs;
+  if constexpr (kBisect) {
+    bs.thresholds(sc);
+    bs.magnitudes(s_mag);
+  }
+  bool ok = __syncthreads_and(mbar_wait(bar_p, 0, a.status));
+  uint32_t par_m = 0;
+
+  auto wait_mma = [&]() {
+    const bool w = mbar_wait(bar_m, par_m, a.status);
+    par_m ^= 1;
+    tc_fence_after();
+    return w;
+  };
+
+  int k = 0;
+  for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++k) {
+    const int64_t row0 = tile * kRows;
+    const int rows = (int)(n - row0 < (int64_t)kRows ? n - row0 : (int64_t)kRows);
+    const int64_t next = tile + gridDim.x;
+    const bool live = r < rows;
+    const int64_t row = row0 + r;
+
+    // every thread reads x from the tile (its half's sum of squares), so every thread waits for it
+    const bool landed = mbar_wait(bar_x, (uint32_t)k & 1u, a.status);
+    if (!landed) ok = false;
+    if (tid == 0 && landed) {  // y = Pi x per row
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t koff = (uint32_t)((kk >> 2) * kBoxBytes + (kk & 3) * 32);
+        umma_f16(tmem, umma_desc_sw128(buf_s + koff, 16, 1024), umma_desc_sw128(pi_s + koff, 16, 1024), kIdPi,
+                 kk > 0);
+      }
+      umma_commit(bar_m);
+    }
+    float2 acc[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float f[8];
+      Elem<T>::unpack(*reinterpret_cast<const uint4*>(s_buf + sw128_chunk(r, 8 * h + j, kBoxBytes)), f);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 v = make_float2(f[2 * q], f[2 * q + 1]);
+        acc[q] = __ffma2_rn(v, v, acc[q]);
+      }
+    }
+    s_part[h * kRows + r] =
+        ((acc[0].x + acc[1].x) + (acc[2].x + acc[3].x)) + ((acc[0].y + acc[1].y) + (acc[2].y + acc[3].y));
+    if (!wait_mma()) ok = false;
+    __syncthreads();  // every half's sum is in, and no thread reads x any more
+    const float nrm = sqrtf(s_part[r] + s_part[kRows + r]);
+    if (tid == 0 && next < ntiles) {  // the product and the norm pass have read the buffer
+      mbar_arrive_expect_tx(bar_x, kTileBytes);
+      for (int b = 0; b < 2; ++b)
+        tma_load_2d(s_buf + b * kBoxBytes, &map_x, b * 64, (int32_t)(next * kRows), bar_x);
+    }
+
+    const float srow = nrm > 0.f ? __fdiv_rn(Bs, nrm) : 0.f;
+    const float shift = -fmaf(kShift, nrm, 0x1p-126f);
+    const float rn = nrm > 0.f ? __frcp_rn(nrm) : 0.f;
+    float win[NWH];
+#pragma unroll
+    for (int w = 0; w < NWH; ++w) win[w] = kWindow0;
+    float gs = 0.f;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {  // 16 columns at a time
+      float y[16];
+      tmem_ld16(tm_y + 16u * (uint32_t)cc, y);
+      uint32_t rho[8];  // fp16(2^8 r) pairs of these columns
+#pragma unroll
+      for (int i = 0; i < 16; i += 2) {
+        const float2 Y = make_float2(y[i] + shift, y[i + 1] + shift);
+        float2 m2 = make_float2(mn0, mn0), cnt = make_float2(0.5f, 0.5f);
+        if constexpr (kBisect) {
+          bs(make_float2(fabsf(Y.x), fabsf(Y.y)), srow, m2, cnt);
+        } else {
+#pragma unroll
+          for (int j = 0; j < H - 1; ++j) {
+            const float2 st = make_float2(fma_sat(fabsf(Y.x), srow, sc[j]), fma_sat(fabsf(Y.y), srow, sc[j]));
+            m2 = __ffma2_rn(st, make_float2(dl[j], dl[j]), m2);
+            cnt = __fadd2_rn(cnt, st);
+          }
+        }
+        const float2 sg = make_float2(sign_one(Y.x), sign_one(Y.y));
+        const float2 chat = __fmul2_rn(m2, sg);  // unit-scale centroid
+        const float2 code = __ffma2_rn(sg, cnt, make_float2(H - 0.5f, H - 0.5f));
+        const int k0 = 16 * cc + i, k1 = k0 + 1;  // code index in the half row
+        win[k0 / CPW] = fmaf(code.x, (float)(1u << (BITS * (k0 % CPW))), win[k0 / CPW]);
+        win[k1 / CPW] = fmaf(code.y, (float)(1u << (BITS * (k1 % CPW))), win[k1 / CPW]);
+        // rotated unit residual r = y / ||x|| - c_hat
+        const float2 rr = __ffma2_rn(make_float2(y[i], y[i + 1]), make_float2(rn, rn), make_float2(-chat.x, -chat.y));
+        gs = fmaf(rr.x, rr.x, fmaf(rr.y, rr.y, gs));
+        const __half2 hp = __floats2half2_rn(rr.x * kSketchScale, rr.y * kSketchScale);
+        rho[i / 2] = *reinterpret_cast<const uint32_t*>(&hp);
+      }
+      tmem_st8(tm_rho + 8u * (uint32_t)cc, rho);
+    }
+    s_gpart[h * kRows + r] = gs;
+    uint32_t wc[WH];
+#pragma unroll
+    for (int w = 0; w < WH; ++w) wc[w] = 0u;
+#pragma unroll
+    for (int w = 0; w < NWH; ++w) {
+      const uint32_t v = __float_as_uint(win[w]) & 0x7fffffu;
+      const int bo = w * CPW * BITS;
+      wc[bo >> 5] |= v << (bo & 31);
+      if ((bo & 31) + CPW * BITS > 32 && (bo >> 5) + 1 < WH) wc[(bo >> 5) + 1] |= v >> (32 - (bo & 31));
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    ok = __syncthreads_and(ok);  // the operand is complete and y has been read
+    if (!ok) break;
+    if (tid == 0) {  // T r per row, into y's columns
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t koff = (uint32_t)((kk >> 2) * kBoxBytes + (kk & 3) * 32);
+        umma_f16_ts(tmem, tmem + 128u + (uint32_t)(8 * kk), umma_desc_sw128(t_s + koff, 16, 1024), kIdT, kk > 0);
+      }
+      umma_commit(bar_m);
+    }
+    const int64_t orow = live ? (a.out_rows ? a.out_rows[row] : row) : 0;
+    if (live) {
+      if (a.codes_out) {
+        uint32_t* dst = a.codes_out + orow * a.ldc + WH * h;
+        if (vec) {
+#pragma unroll
+          for (int w = 0; w < WH; w += 2) *reinterpret_cast<uint2*>(dst + w) = make_uint2(wc[w], wc[w + 1]);
+        } else {
+#pragma unroll
+          for (int w = 0; w < WH; ++w) dst[w] = wc[w];
+        }
+      }
+      if (h == 0) {
+        if (a.norms_out) a.norms_out[orow * a.ldn] = nrm;
+        if (a.gammas_out) a.gammas_out[orow * a.ldn] = sqrtf(s_gpart[r] + s_gpart[kRows + r]);
+      }
+    }
+    if (!wait_mma()) ok = false;
+    uint32_t sw[2];
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      float z[32];
+      tmem_ld32(tm_y + 32u * (uint32_t)cc, z);
+      uint32_t bits = 0;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) bits |= (z[i] >= 0.f ? 1u : 0u) << i;  // sign(0) = +1
+      sw[cc] = bits;
+    }
+    if (live && a.signs_out) {
+      uint32_t* dst = a.signs_out + orow * a.lds + (NS / 2) * h;
+      if (svec) *reinterpret_cast<uint2*>(dst) = make_uint2(sw[0], sw[1]);
+      else dst[0] = sw[0], dst[1] = sw[1];
+    }
+    tc_fence_before();
+    ok = __syncthreads_and(ok);  // T r has been read before the next tile's product overwrites it
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kNcols);
+  }
+}
+
 }  // namespace tq
 
 // ============================================================================ launch
@@ -823,6 +1089,32 @@ static cudaError_t tq_mse_by_bits(int bits, const CUtensorMap& mx, const CUtenso
   }
 }
 
+template <typename T, int BITS>
+static cudaError_t launch_tq_prod_t(const CUtensorMap& mx, const CUtensorMap& mp, const CUtensorMap& mt,
+                                    const TqArgs& a, cudaStream_t st, int num_sms) {
+  auto kern = tq::tq_prod_kernel<T, BITS>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, tq::SmemP::alloc);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int64_t ntiles = (a.n + tq::kRows - 1) / tq::kRows;
+  const int64_t grid = std::min<int64_t>(ntiles, (int64_t)num_sms * 2);
+  return launch_pdl(kern, (unsigned)grid, tq::kThreadsM, tq::SmemP::alloc, st, mx, mp, mt, a);
+}
+
+template <typename T>
+static cudaError_t tq_prod_by_bits(int bits, const CUtensorMap& mx, const CUtensorMap& mp, const CUtensorMap& mt,
+                                   const TqArgs& a, cudaStream_t st, int sms) {
+  switch (bits) {
+    case 1: return launch_tq_prod_t<T, 1>(mx, mp, mt, a, st, sms);
+    case 2: return launch_tq_prod_t<T, 2>(mx, mp, mt, a, st, sms);
+    case 3: return launch_tq_prod_t<T, 3>(mx, mp, mt, a, st, sms);
+    default: return launch_tq_prod_t<T, 4>(mx, mp, mt, a, st, sms);
+  }
+}
+
 template <typename T, int MODE>
 static cudaError_t tq_by_bits(int bits, const CUtensorMap& mx, const CUtensorMap& mp, const CUtensorMap& mt,
                               const CUtensorMap& mo, const TqArgs& a, cudaStream_t st, int sms) {
@@ -840,7 +1132,7 @@ static cudaError_t tq_by_mode(int mode, int bits, const CUtensorMap& mx, const C
   switch (mode) {
     case TQ_MSE_Q: return tq_mse_by_bits<T, TQ_MSE_Q>(bits, mx, mp, mo, a, st, sms);
     case TQ_MSE_QDQ: return tq_mse_by_bits<T, TQ_MSE_QDQ>(bits, mx, mp, mo, a, st, sms);
-    case TQ_PROD_Q: return tq_by_bits<T, TQ_PROD_Q>(bits, mx, mp, mt, mo, a, st, sms);
+    case TQ_PROD_Q: return tq_prod_by_bits<T>(bits, mx, mp, mt, a, st, sms);
     case TQ_DQ_MSE: return tq_mse_by_bits<T, TQ_DQ_MSE>(bits, mx, mp, mo, a, st, sms);
     default: return tq_by_bits<T, TQ_DQ_PROD>(bits, mx, mp, mt, mo, a, st, sms);
   }
