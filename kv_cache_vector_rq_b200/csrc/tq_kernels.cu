@@ -18,8 +18,10 @@
 // sketch) back into the tile buffer, which finally holds x_hat for the TMA store.
 //  * tq_mse_kernel (the mse modes): 256 threads, two per row (64 columns each), two
 //    tile buffers so the next tile's load lands while this tile is quantized.
-//  * tq_kernel (the prod modes, whose Pi and T leave room for one tile buffer at two
-//    CTAs per SM): 128 threads, one per row, one tile at a time.
+//  * tq_prod_kernel (prod quantize): 256 threads, two per row; Pi and T leave room for
+//    one tile buffer at two CTAs per SM, so the sketch operand goes to tensor memory
+//    and the buffer takes the next tile's x as soon as the first product has read it.
+//  * tq_dq_prod_kernel (prod dequantize): 128 threads, one per row, one tile at a time.
 // Two CTAs share an SM (256 TMEM columns each), so one CTA's MMAs overlap the other's
 // epilogue.
 
@@ -53,22 +55,19 @@ struct Codes {
   static constexpr int NWIN = (NC + CPW - 1) / CPW;
 };
 
-template <int BITS, int MODE>
-struct Smem {
-  static constexpr bool kT = MODE == TQ_PROD_Q || MODE == TQ_DQ_PROD;
-  static constexpr int W = Codes<BITS>::W;
+struct SmemD {
   static constexpr int tile_off = 0;
   static constexpr int pi_off = kTileBytes;
   static constexpr int t_off = pi_off + kTileBytes;
-  static constexpr int codes_off = t_off + (kT ? kTileBytes : 0);  // [kRows][W]
-  static constexpr int signs_off = codes_off + ((kRows * W * 4 + 15) / 16) * 16;  // [kRows][D/32]
+  static constexpr int codes_off = t_off + kTileBytes;  // [kRows][W], W <= 16
+  static constexpr int signs_off = codes_off + kRows * 16 * 4;  // [kRows][D/32]
   static constexpr int cb_off = signs_off + kRows * (D / 32) * 4;
-  static constexpr int bar_off = cb_off + 64 * 4;  // x, params, mma
-  static constexpr int tmem_off = bar_off + 3 * 8;
+  static constexpr int bar_off = cb_off + 64 * 4;  // params, mma
+  static constexpr int tmem_off = bar_off + 2 * 8;
   static constexpr int bytes = tmem_off + 16;
-  // at least 80 KB so that at most two CTAs (2 x 256 TMEM columns) share an SM
-  static constexpr int alloc = (bytes + 1024) < 80 * 1024 ? 80 * 1024 : bytes + 1024;
+  static constexpr int alloc = bytes + 1024;
 };
+static_assert(2 * (SmemD::alloc + 1024) <= 228 * 1024, "two CTAs per SM");
 
 // Positive-side quantizer constants (see rq_kernels.cu for the construction):
 // sc[j] = -tau_{j+1} * B, chain of unit centroids c[H] + sum step_j * dl[j].
@@ -102,23 +101,20 @@ struct IsBf16 {
   static constexpr bool value = std::is_same<T, __nv_bfloat16>::value;
 };
 
-template <typename T, int BITS, int MODE>
+// TurboQuant-prod dequantize at d = 128: x_hat = ||x|| Pi^T (c_hat + sqrt(pi/2)/m gamma T^T s). One
+// thread per row (TMEM lane); per tile the +-1 sign operand S goes through the tile buffer into
+// T^T s (MN-major T), the corrected centroids w into Pi^T w, and x_hat leaves by TMA.
+template <typename T, int BITS>
 __global__ void __launch_bounds__(kRows, 1)
-    tq_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_pi,
-              const __grid_constant__ CUtensorMap map_t, const __grid_constant__ CUtensorMap map_o, TqArgs a) {
-  using CD = Codes<BITS>;
-  using SM = Smem<BITS, MODE>;
-  constexpr int H = CD::H, W = CD::W, CPW = CD::CPW, NWIN = CD::NWIN;
+    tq_dq_prod_kernel(const __grid_constant__ CUtensorMap map_pi, const __grid_constant__ CUtensorMap map_t,
+                      const __grid_constant__ CUtensorMap map_o, TqArgs a) {
+  using SM = SmemD;
+  constexpr int W = Codes<BITS>::W;
+  static_assert(W <= 16, "code staging");
   constexpr int NS = D / 32;  // sign words per row
-  constexpr bool kQ = MODE == TQ_MSE_Q || MODE == TQ_MSE_QDQ || MODE == TQ_PROD_Q;
-  constexpr bool kProd = MODE == TQ_PROD_Q || MODE == TQ_DQ_PROD;
-  constexpr bool kOut = MODE == TQ_MSE_QDQ || MODE == TQ_DQ_MSE || MODE == TQ_DQ_PROD;
   constexpr uint32_t kNcols = 256;
-  // instruction descriptors (M = 128, N = 128)
-  constexpr uint32_t kIdPi = umma_idesc_f16(IsBf16<T>::value, IsBf16<T>::value, false, D, kRows);    // X Pi^T
-  constexpr uint32_t kIdPiT = umma_idesc_f16(IsBf16<T>::value, IsBf16<T>::value, true, D, kRows);    // W Pi
-  constexpr uint32_t kIdT = umma_idesc_f16(false, false, false, D, kRows);                   // rho T^T
-  constexpr uint32_t kIdTT = umma_idesc_f16(false, false, true, D, kRows);                   // S T
+  constexpr uint32_t kIdPiT = umma_idesc_f16(IsBf16<T>::value, IsBf16<T>::value, true, D, kRows);  // W Pi
+  constexpr uint32_t kIdTT = umma_idesc_f16(false, false, true, D, kRows);                          // S T
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -131,9 +127,8 @@ __global__ void __launch_bounds__(kRows, 1)
   float* s_mag = s_sc + 16;
   float* s_cf = s_sc + 32;
   float* s_bscale = s_sc + 48;
-  uint64_t* bar_x = reinterpret_cast<uint64_t*>(smem + SM::bar_off);
-  uint64_t* bar_p = bar_x + 1;
-  uint64_t* bar_m = bar_x + 2;
+  uint64_t* bar_p = reinterpret_cast<uint64_t*>(smem + SM::bar_off);
+  uint64_t* bar_m = bar_p + 1;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + SM::tmem_off);
 
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -142,11 +137,9 @@ __global__ void __launch_bounds__(kRows, 1)
   const uint32_t tile_s = smem_u32(s_tile), pi_s = smem_u32(s_pi), t_s = smem_u32(s_t);
 
   if (tid == 0) {
-    if (kQ) tma_prefetch_desc(&map_x);
     tma_prefetch_desc(&map_pi);
-    if (kProd) tma_prefetch_desc(&map_t);
-    if (kOut) tma_prefetch_desc(&map_o);
-    mbar_init(bar_x, 1);
+    tma_prefetch_desc(&map_t);
+    tma_prefetch_desc(&map_o);
     mbar_init(bar_p, 1);
     mbar_init(bar_m, 1);
     fence_barrier_init();
@@ -162,26 +155,14 @@ __global__ void __launch_bounds__(kRows, 1)
 
   // resident parameters
   if (tid == 0) {
-    mbar_arrive_expect_tx(bar_p, kTileBytes * (kProd ? 2 : 1));
+    mbar_arrive_expect_tx(bar_p, 2 * kTileBytes);
     for (int b = 0; b < 2; ++b) tma_load_2d(s_pi + b * kBoxBytes, &map_pi, b * 64, 0, bar_p);
-    if (kProd)
-      for (int b = 0; b < 2; ++b) tma_load_2d(s_t + b * kBoxBytes, &map_t, b * 64, 0, bar_p);
+    for (int b = 0; b < 2; ++b) tma_load_2d(s_t + b * kBoxBytes, &map_t, b * 64, 0, bar_p);
   }
   bool ok = __syncthreads_and(mbar_wait(bar_p, 0, a.status));
+  uint32_t par_m = 0;
 
-  uint32_t par_x = 0, par_m = 0;
-  const float Bs = *s_bscale;
-
-  // MMA helpers (thread 0): A is always the tile buffer (K-major); B is Pi or T
-  auto mma_kmajor_b = [&](uint32_t tm_d, uint32_t b_s, uint32_t idesc) {
-    tc_fence_after();
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t koff = (uint32_t)((kk >> 2) * kBoxBytes + (kk & 3) * 32);
-      umma_f16(tm_d, umma_desc_sw128(tile_s + koff, 16, 1024), umma_desc_sw128(b_s + koff, 16, 1024), idesc, kk > 0);
-    }
-    umma_commit(bar_m);
-  };
+  // MMA (thread 0): A is the tile buffer (K-major), B = Pi or T (MN-major)
   auto mma_mnmajor_b = [&](uint32_t tm_d, uint32_t b_s, uint32_t idesc) {
     tc_fence_after();
 #pragma unroll
@@ -199,7 +180,7 @@ __global__ void __launch_bounds__(kRows, 1)
     tc_fence_after();
     return r;
   };
-  // write 8 floats as one 16-byte chunk (element type E) of this thread's row in the tile buffer
+  // write 8 floats as one 16-byte chunk of this thread's row in the tile buffer
   auto put_chunk = [&](int j, const float* v, bool as_f16) {
     uint4 c = as_f16 ? Elem<__half>::pack(v) : Elem<T>::pack(v);
     *reinterpret_cast<uint4*>(s_tile + sw128_chunk(tid, j, kBoxBytes)) = c;
@@ -209,235 +190,74 @@ __global__ void __launch_bounds__(kRows, 1)
     const int64_t row0 = tile * kRows;
     const int rows = (int)(n - row0 < (int64_t)kRows ? n - row0 : (int64_t)kRows);
     const int64_t row = row0 + tid;
-    float nrm = 0.f;
-
-    // ------------------------------------------------------------ quantize side
-    if constexpr (kQ) {
-      if (tid == 0) {
-        bulk_wait_read<0>();  // the previous x_hat store has left the tile buffer
-        mbar_arrive_expect_tx(bar_x, kTileBytes);
-        for (int b = 0; b < 2; ++b) tma_load_2d(s_tile + b * kBoxBytes, &map_x, b * 64, (int32_t)row0, bar_x);
-      }
-      ok = mbar_wait(bar_x, par_x, a.status);
-      par_x ^= 1;
-      if (!__syncthreads_and(ok)) break;
-      if (tid == 0) mma_kmajor_b(tm_y, pi_s, kIdPi);  // y = Pi x (rows of the tile)
-      // ||x||^2 from the tile while the MMA runs
-      float2 acc[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int j = 0; j < D / 8; ++j) {
-        float f[8];
-        Elem<T>::unpack(*reinterpret_cast<const uint4*>(s_tile + sw128_chunk(tid, j, kBoxBytes)), f);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 v = make_float2(f[2 * k], f[2 * k + 1]);
-          acc[k] = __ffma2_rn(v, v, acc[k]);
-        }
-      }
-      nrm = sqrtf(((acc[0].x + acc[1].x) + (acc[2].x + acc[3].x)) + ((acc[0].y + acc[1].y) + (acc[2].y + acc[3].y)));
-      if (!wait_mma()) ok = false;
-
-      const float srow = nrm > 0.f ? __fdiv_rn(Bs, nrm) : 0.f;
-      const float shift = -fmaf(kShift, nrm, 0x1p-126f);
-      const float rn = nrm > 0.f ? __frcp_rn(nrm) : 0.f;
-      float dl[H > 1 ? H - 1 : 1], sc[H > 1 ? H - 1 : 1];
-#pragma unroll
-      for (int j = 0; j < H - 1; ++j) {
-        dl[j] = __fsub_rn(s_mag[j + 1], s_mag[j]);
-        sc[j] = s_sc[j];
-      }
-      const float mn0 = s_mag[0];
-      float win[NWIN];
-#pragma unroll
-      for (int w = 0; w < NWIN; ++w) win[w] = kWindow0;
-      float gs = 0.f;  // ||r||^2 (prod)
-
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        float y[32];
-        tmem_ld32(tm_y + lane_off + 32 * c, y);
-        float w_out[32];
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const float2 Y = make_float2(y[i] + shift, y[i + 1] + shift);
-          float2 m2 = make_float2(mn0, mn0), cnt = make_float2(0.5f, 0.5f);
-#pragma unroll
-          for (int j = 0; j < H - 1; ++j) {
-            const float2 st = make_float2(fma_sat(fabsf(Y.x), srow, sc[j]), fma_sat(fabsf(Y.y), srow, sc[j]));
-            m2 = __ffma2_rn(st, make_float2(dl[j], dl[j]), m2);
-            cnt = __fadd2_rn(cnt, st);
-          }
-          const float2 sg = make_float2(sign_one(Y.x), sign_one(Y.y));
-          const float2 chat = __fmul2_rn(m2, sg);  // unit-scale centroid
-          const float2 code = __ffma2_rn(sg, cnt, make_float2(H - 0.5f, H - 0.5f));
-          const int k0 = 32 * c + i, k1 = k0 + 1;
-          win[k0 / CPW] = fmaf(code.x, (float)(1u << (BITS * (k0 % CPW))), win[k0 / CPW]);
-          win[k1 / CPW] = fmaf(code.y, (float)(1u << (BITS * (k1 % CPW))), win[k1 / CPW]);
-          if constexpr (MODE == TQ_MSE_QDQ) {
-            w_out[i] = chat.x;
-            w_out[i + 1] = chat.y;
-          } else if constexpr (MODE == TQ_PROD_Q) {
-            // rotated unit residual r = y/||x|| - c_hat
-            const float2 r = __ffma2_rn(make_float2(y[i], y[i + 1]), make_float2(rn, rn), make_float2(-chat.x, -chat.y));
-            gs = fmaf(r.x, r.x, fmaf(r.y, r.y, gs));
-            w_out[i] = r.x * kSketchScale;
-            w_out[i + 1] = r.y * kSketchScale;
-          }
-        }
-        if constexpr (MODE == TQ_MSE_QDQ || MODE == TQ_PROD_Q) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) put_chunk(4 * c + q, &w_out[8 * q], MODE == TQ_PROD_Q);
-        }
-      }
-      // codes -> staging
-      uint32_t wc[W];
-#pragma unroll
-      for (int w = 0; w < W; ++w) wc[w] = 0u;
-#pragma unroll
-      for (int w = 0; w < NWIN; ++w) {
-        const uint32_t v = __float_as_uint(win[w]) & 0x7fffffu;
-        const int bo = w * CPW * BITS;
-        wc[bo >> 5] |= v << (bo & 31);
-        if ((bo & 31) + CPW * BITS > 32 && (bo >> 5) + 1 < W) wc[(bo >> 5) + 1] |= v >> (32 - (bo & 31));
-      }
-#pragma unroll
-      for (int w = 0; w < W; ++w) s_codes[tid * W + w] = wc[w];
-      if (tid < rows) {
-        const int64_t orow = a.out_rows ? a.out_rows[row] : row;
-        if (a.norms_out) a.norms_out[orow * a.ldn] = nrm;
-        if (kProd && a.gammas_out) a.gammas_out[orow * a.ldn] = sqrtf(gs);
-      }
-
-      if constexpr (MODE == TQ_MSE_QDQ || MODE == TQ_PROD_Q) {
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-          if (MODE == TQ_MSE_QDQ) mma_mnmajor_b(tm_2, pi_s, kIdPiT);  // Pi^T c_hat
-          else mma_kmajor_b(tm_2, t_s, kIdT);                         // T rho
-        }
-        if (!wait_mma()) ok = false;
-        if constexpr (MODE == TQ_PROD_Q) {
-#pragma unroll
-          for (int c = 0; c < NS; ++c) {
-            float z[32];
-            tmem_ld32(tm_2 + lane_off + 32 * c, z);
-            uint32_t bits = 0;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) bits |= (z[i] >= 0.f ? 1u : 0u) << i;  // sign(0) = +1
-            s_signs[tid * NS + c] = bits;
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            float v[32];
-            tmem_ld32(tm_2 + lane_off + 32 * c, v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] *= nrm;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) put_chunk(4 * c + q, &v[8 * q], false);
-          }
-        }
-      }
-    } else {
-      // ---------------------------------------------------------- dequantize side
-      for (int i = tid; i < rows * W; i += kRows) {
-        const int r = i / W, w = i - r * W;
-        s_codes[i] = __ldg(a.codes_in + (row0 + r) * a.ldc + w);
-      }
-      if (kProd)
-        for (int i = tid; i < rows * NS; i += kRows) {
-          const int r = i / NS, w = i - r * NS;
-          s_signs[i] = __ldg(a.signs_in + (row0 + r) * a.lds + w);
-        }
-      nrm = tid < rows ? __ldg(a.norms_in + row * a.ldn) : 0.f;
-      const float gam = (kProd && tid < rows) ? __ldg(a.gammas_in + row * a.ldn) : 0.f;
-      if (tid == 0) bulk_wait_read<0>();
-      if (!__syncthreads_and(ok)) break;
-      uint32_t wc[W];
-#pragma unroll
-      for (int w = 0; w < W; ++w) wc[w] = s_codes[tid * W + w];
-      auto code_at = [&](int k) -> uint32_t {
-        const int bit = k * BITS, word = bit >> 5, sh = bit & 31;
-        uint32_t v = wc[word] >> sh;
-        if (sh + BITS > 32) v |= wc[word + 1] << (32 - sh);
-        return v & ((1u << BITS) - 1u);
-      };
-      if constexpr (kProd) {
-        // S tile of +1/-1 (fp16) -> T^T s
-#pragma unroll
-        for (int c = 0; c < NS; ++c) {
-          const uint32_t sw = s_signs[tid * NS + c];
-          float v[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = ((sw >> i) & 1u) ? 1.f : -1.f;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) put_chunk(4 * c + q, &v[8 * q], true);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) mma_mnmajor_b(tm_2, t_s, kIdTT);
-        if (!wait_mma()) ok = false;
-        const float qs = a.qjl_scale * gam;  // sqrt(pi/2)/m * gamma
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          float v[32];
-          tmem_ld32(tm_2 + lane_off + 32 * c, v);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = fmaf(qs, v[i], s_cf[code_at(32 * c + i)]);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) put_chunk(4 * c + q, &v[8 * q], false);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          float v[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = s_cf[code_at(32 * c + i)];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) put_chunk(4 * c + q, &v[8 * q], false);
-        }
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncthreads();
-      if (tid == 0) mma_mnmajor_b(tm_y, pi_s, kIdPiT);  // Pi^T w
-      if (!wait_mma()) ok = false;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        float v[32];
-        tmem_ld32(tm_y + lane_off + 32 * c, v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] *= nrm;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) put_chunk(4 * c + q, &v[8 * q], false);
-      }
+    for (int i = tid; i < rows * W; i += kRows) {
+      const int r = i / W, w = i - r * W;
+      s_codes[i] = __ldg(a.codes_in + (row0 + r) * a.ldc + w);
     }
-
-    // ------------------------------------------------------------ outputs
+    for (int i = tid; i < rows * NS; i += kRows) {
+      const int r = i / NS, w = i - r * NS;
+      s_signs[i] = __ldg(a.signs_in + (row0 + r) * a.lds + w);
+    }
+    const float nrm = tid < rows ? __ldg(a.norms_in + row * a.ldn) : 0.f;
+    const float gam = tid < rows ? __ldg(a.gammas_in + row * a.ldn) : 0.f;
+    if (tid == 0) bulk_wait_read<0>();  // the previous x_hat store has left the tile buffer
+    if (!__syncthreads_and(ok)) break;
+    uint32_t wc[W];
+#pragma unroll
+    for (int w = 0; w < W; ++w) wc[w] = tid < rows ? s_codes[tid * W + w] : 0u;
+    auto code_at = [&](int k) -> uint32_t {
+      const int bit = k * BITS, word = bit >> 5, sh = bit & 31;
+      uint32_t v = wc[word] >> sh;
+      if (sh + BITS > 32) v |= wc[word + 1] << (32 - sh);
+      return v & ((1u << BITS) - 1u);
+    };
+    // S tile of +1/-1 (fp16) -> T^T s
+#pragma unroll
+    for (int c = 0; c < NS; ++c) {
+      const uint32_t sw = tid < rows ? s_signs[tid * NS + c] : 0u;
+      float v[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = ((sw >> i) & 1u) ? 1.f : -1.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) put_chunk(4 * c + q, &v[8 * q], true);
+    }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (kOut && tid == 0) {
+    if (tid == 0) mma_mnmajor_b(tm_2, t_s, kIdTT);
+    if (!wait_mma()) ok = false;
+    const float qs = a.qjl_scale * gam;  // sqrt(pi/2)/m * gamma
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      float v[32];
+      tmem_ld32(tm_2 + lane_off + 32 * c, v);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = fmaf(qs, v[i], s_cf[code_at(32 * c + i)]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) put_chunk(4 * c + q, &v[8 * q], false);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) mma_mnmajor_b(tm_y, pi_s, kIdPiT);  // Pi^T w
+    if (!wait_mma()) ok = false;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      float v[32];
+      tmem_ld32(tm_y + lane_off + 32 * c, v);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] *= nrm;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) put_chunk(4 * c + q, &v[8 * q], false);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
       for (int b = 0; b < 2; ++b) tma_store_2d(&map_o, b * 64, (int32_t)row0, s_tile + b * kBoxBytes);
       bulk_commit();
     }
-    if constexpr (kQ) {
-      if (a.codes_out)
-        for (int i = tid; i < rows * W; i += kRows) {
-          const int r = i / W, w = i - r * W;
-          a.codes_out[(a.out_rows ? a.out_rows[row0 + r] : row0 + r) * a.ldc + w] = s_codes[i];
-        }
-      if (kProd && a.signs_out)
-        for (int i = tid; i < rows * NS; i += kRows) {
-          const int r = i / NS, w = i - r * NS;
-          a.signs_out[(a.out_rows ? a.out_rows[row0 + r] : row0 + r) * a.lds + w] = s_signs[i];
-        }
-    }
-    __syncthreads();  // staging buffers are rewritten by the next tile
+    __syncthreads();  // the staged words are rewritten by the next tile
   }
   if (tid == 0) bulk_wait_all<0>();
   tc_fence_before();
@@ -1046,20 +866,19 @@ __global__ void __launch_bounds__(kThreadsM, 2)
 }  // namespace tq
 
 // ============================================================================ launch
-template <typename T, int BITS, int MODE>
-static cudaError_t launch_tq_t(const CUtensorMap& mx, const CUtensorMap& mp, const CUtensorMap& mt, const CUtensorMap& mo,
-                               const TqArgs& a, cudaStream_t st, int num_sms) {
-  using SM = tq::Smem<BITS, MODE>;
-  auto kern = tq::tq_kernel<T, BITS, MODE>;
+template <typename T, int BITS>
+static cudaError_t launch_tq_dq_prod_t(const CUtensorMap& mp, const CUtensorMap& mt, const CUtensorMap& mo,
+                                       const TqArgs& a, cudaStream_t st, int num_sms) {
+  auto kern = tq::tq_dq_prod_kernel<T, BITS>;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::alloc);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, tq::SmemD::alloc);
     if (e != cudaSuccess) return e;
     attr = true;
   }
   const int64_t ntiles = (a.n + tq::kRows - 1) / tq::kRows;
   const int64_t grid = std::min<int64_t>(ntiles, (int64_t)num_sms * 2);
-  kern<<<(unsigned)grid, tq::kRows, SM::alloc, st>>>(mx, mp, mt, mo, a);
+  kern<<<(unsigned)grid, tq::kRows, tq::SmemD::alloc, st>>>(mp, mt, mo, a);
   return cudaGetLastError();
 }
 
@@ -1115,14 +934,14 @@ static cudaError_t tq_prod_by_bits(int bits, const CUtensorMap& mx, const CUtens
   }
 }
 
-template <typename T, int MODE>
-static cudaError_t tq_by_bits(int bits, const CUtensorMap& mx, const CUtensorMap& mp, const CUtensorMap& mt,
-                              const CUtensorMap& mo, const TqArgs& a, cudaStream_t st, int sms) {
+template <typename T>
+static cudaError_t tq_dq_prod_by_bits(int bits, const CUtensorMap& mp, const CUtensorMap& mt, const CUtensorMap& mo,
+                                      const TqArgs& a, cudaStream_t st, int sms) {
   switch (bits) {
-    case 1: return launch_tq_t<T, 1, MODE>(mx, mp, mt, mo, a, st, sms);
-    case 2: return launch_tq_t<T, 2, MODE>(mx, mp, mt, mo, a, st, sms);
-    case 3: return launch_tq_t<T, 3, MODE>(mx, mp, mt, mo, a, st, sms);
-    default: return launch_tq_t<T, 4, MODE>(mx, mp, mt, mo, a, st, sms);
+    case 1: return launch_tq_dq_prod_t<T, 1>(mp, mt, mo, a, st, sms);
+    case 2: return launch_tq_dq_prod_t<T, 2>(mp, mt, mo, a, st, sms);
+    case 3: return launch_tq_dq_prod_t<T, 3>(mp, mt, mo, a, st, sms);
+    default: return launch_tq_dq_prod_t<T, 4>(mp, mt, mo, a, st, sms);
   }
 }
 
@@ -1134,7 +953,7 @@ static cudaError_t tq_by_mode(int mode, int bits, const CUtensorMap& mx, const C
     case TQ_MSE_QDQ: return tq_mse_by_bits<T, TQ_MSE_QDQ>(bits, mx, mp, mo, a, st, sms);
     case TQ_PROD_Q: return tq_prod_by_bits<T>(bits, mx, mp, mt, a, st, sms);
     case TQ_DQ_MSE: return tq_mse_by_bits<T, TQ_DQ_MSE>(bits, mx, mp, mo, a, st, sms);
-    default: return tq_by_bits<T, TQ_DQ_PROD>(bits, mx, mp, mt, mo, a, st, sms);
+    default: return tq_dq_prod_by_bits<T>(bits, mp, mt, mo, a, st, sms);
   }
 }
 
