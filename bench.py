@@ -398,22 +398,25 @@ def decode_attention_c4(kvrq, synth, torch, dev, batch, steps, warmup, layers=36
     cache is 4x L2 or more, so every call streams it from HBM."""
     heads = layers * kv_heads * batch
     t_max = cached + 1
+    # capacity in whole 16-token blocks, as a cache allocator (or a page pool) gives it: every head's
+    # rows then start 16-byte aligned, which the kernel's bulk copies need for 52-byte value rows
+    cap = -(-t_max // 16) * 16
     pi = torch.from_numpy(kvrq.tq_rotation_init(D, 2)).to(torch.float16).to(dev)
     T = torch.from_numpy(kvrq.qjl_matrix_init(D, D, 3)).to(torch.float16).to(dev)
     rot = torch.from_numpy(kvrq.rq_rotors_init(D, 1).astype(np.float32)).to(dev)
     ck = torch.from_numpy(kvrq.tq_codebook_init(D, 2)[0].astype(np.float32)).to(dev)
     cv = torch.from_numpy(kvrq.tq_codebook_init(D, 3)[0].astype(np.float32)).to(dev)
     Wk, Wv = kvrq.packed_words(D, 2), kvrq.packed_words(129, 3)
-    k_codes = torch.empty((heads, t_max, Wk), dtype=torch.int32, device=dev)
-    k_signs = torch.empty((heads, t_max, D // 32), dtype=torch.int32, device=dev)
-    k_norms = torch.empty((heads, t_max), dtype=torch.float32, device=dev)
-    k_gam = torch.empty((heads, t_max), dtype=torch.float32, device=dev)
-    v_codes = torch.empty((heads, t_max, Wv), dtype=torch.int32, device=dev)
-    v_norms = torch.empty((heads, t_max), dtype=torch.float32, device=dev)
-    chunk = max(1, (1 << 22) // t_max)
+    k_codes = torch.empty((heads, cap, Wk), dtype=torch.int32, device=dev)
+    k_signs = torch.empty((heads, cap, D // 32), dtype=torch.int32, device=dev)
+    k_norms = torch.empty((heads, cap), dtype=torch.float32, device=dev)
+    k_gam = torch.empty((heads, cap), dtype=torch.float32, device=dev)
+    v_codes = torch.empty((heads, cap, Wv), dtype=torch.int32, device=dev)
+    v_norms = torch.empty((heads, cap), dtype=torch.float32, device=dev)
+    chunk = max(1, (1 << 22) // cap)
     for h0 in range(0, heads, chunk):  # prefill (untimed)
         h1 = min(heads, h0 + chunk)
-        rows = (h1 - h0) * t_max
+        rows = (h1 - h0) * cap
         kx = synth.lognormal(rows, D, seed=5000 + h0, dtype=torch.float16, device=dev)
         kvrq.tq_quantize_prod(kx, pi, T, ck, 3, codes=k_codes[h0:h1].view(rows, Wk),
                               norms=k_norms[h0:h1].reshape(rows), signs=k_signs[h0:h1].view(rows, D // 32),
@@ -444,6 +447,7 @@ def decode_attention_c4(kvrq, synth, torch, dev, batch, steps, warmup, layers=36
     tokens = heads * t_max
     cache_bytes = tokens * (4 * Wk + 4 * (D // 32) + 8 + 4 * Wv + 4)  # keys 56 B + values 56 B per token
     res = {"batch": batch, "layers": layers, "kv_heads": kv_heads, "query_heads_per_kv": group, "tokens": t_max,
+           "capacity": cap,
            "ms_per_call": ms, "tokens_per_s": tokens / (ms * 1e-3), "cache_bytes": cache_bytes,
            "cache_GB_s": cache_bytes / (ms * 1e-3) / 1e9, "launches_per_call": 3}
     del k_codes, k_signs, k_norms, k_gam, v_codes, v_norms, ws
