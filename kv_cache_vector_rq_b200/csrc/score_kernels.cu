@@ -305,10 +305,10 @@ __global__ void __launch_bounds__(Cfg<METHOD, BITS, NB>::kThreads, 1) score_kern
       }
     };
 
-    constexpr int NCC = (KC / 2 + 31) / 32;  // 32-word chunks of the centroid part
+    constexpr int NCC = (KC / 2 + 15) / 16;  // 16-word chunks of the centroid part
     auto centroid_chunk = [&](int c, const uint32_t (&wc)[W]) {
-      uint32_t rw[32];
-      constexpr int FPC = 64 / DC::P;  // fields per 32 words
+      uint32_t rw[16];
+      constexpr int FPC = 32 / DC::P;  // fields per 16 words
 #pragma unroll
       for (int f = 0; f < FPC; ++f) {
         const int fi = c * FPC + f;  // field index: codes fi*P .. fi*P + P - 1
@@ -335,19 +335,19 @@ __global__ void __launch_bounds__(Cfg<METHOD, BITS, NB>::kThreads, 1) score_kern
         // K elements past the stored codes (the RotorQuant tail) are zero
 #pragma unroll
         for (int q = 0; q < DC::EW; ++q) {
-          const int k0 = 2 * (32 * c + DC::EW * f + q);  // first K element of this word
+          const int k0 = 2 * (16 * c + DC::EW * f + q);  // first K element of this word
           if (k0 >= C::NCODE) rw[DC::EW * f + q] = 0u;
           else if (k0 + 1 >= C::NCODE) rw[DC::EW * f + q] &= 0xFFFFu;
         }
       }
-      if (32 * c + 32 <= KC / 2) tmem_st32(a_t + (uint32_t)(32 * c), rw);
-      else tmem_st8(a_t + (uint32_t)(32 * c), rw);  // RotorQuant: 72 = 2 x 32 + 8 words
+      if (16 * c + 16 <= KC / 2) tmem_st16(a_t + (uint32_t)(16 * c), rw);
+      else tmem_st8(a_t + (uint32_t)(16 * c), rw);  // RotorQuant: 72 = 4 x 16 + 8 words
     };
-    auto sign_chunk = [&](int c, const uint32_t (&sg)[NS > 0 ? NS : 1]) {
-      uint32_t rw[32];
+    auto sign_chunk = [&](int c, const uint32_t (&sg)[NS > 0 ? NS : 1]) {  // 16 words: 4 bytes of signs
+      uint32_t rw[16];
 #pragma unroll
-      for (int bq = 0; bq < 8; ++bq) {
-        const int byte = 8 * c + bq;
+      for (int bq = 0; bq < 4; ++bq) {
+        const int byte = 4 * c + bq;
         const uint32_t v = (sg[byte >> 2] >> (8 * (byte & 3))) & 0xFFu;
         const uint4 x = lds_v4(slut_l + (v << 7));
         rw[4 * bq] = x.x;
@@ -355,7 +355,7 @@ __global__ void __launch_bounds__(Cfg<METHOD, BITS, NB>::kThreads, 1) score_kern
         rw[4 * bq + 2] = x.z;
         rw[4 * bq + 3] = x.w;
       }
-      tmem_st32(a_t + (uint32_t)(KC / 2 + 32 * c), rw);
+      tmem_st16(a_t + (uint32_t)(KC / 2 + 16 * c), rw);
     };
     auto mma_steps = [&](int i, int k_lo, int k_hi) {  // thread 0 of the warpgroup
       const uint32_t d_t = a_mma + (uint32_t)(C::KAP + (i & 1) * NB);
@@ -422,8 +422,8 @@ __global__ void __launch_bounds__(Cfg<METHOD, BITS, NB>::kThreads, 1) score_kern
 #pragma unroll
       for (int c = 0; c < NCC; ++c) centroid_chunk(c, wc);
       if constexpr (kProd) {
-        sign_chunk(0, sg);
-        sign_chunk(1, sg);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) sign_chunk(c, sg);
       }
       prev_n = nrm;  // the loads have long landed by now
       prev_g = gam;
