@@ -497,9 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
       if (wg_any(need, 1 + w)) {  // (the barrier before MMA2 when no rescaling is needed)
 #pragma unroll
         for (int g = 0; g < GMAX; ++g) {
-          float v = lg[g];
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+          const float v = warp_max_f32(lg[g]);
           if (lane == 0) red[q4 * GMAX + g] = v;
         }
         asm volatile("bar.sync %0, 128;" ::"r"(1 + w) : "memory");
