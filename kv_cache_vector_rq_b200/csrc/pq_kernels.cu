@@ -356,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       rebuild_chunk(hw, cc, cs_s, yh);
 #pragma unroll
       for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<uint4*>(tbuf + sw128_chunk(r, 8 * h + 4 * cc + q, kBoxBytes)) = Elem<T>::pack(&yh[8 * q]);
+        sts_v4(tbuf_s + sw128_chunk(r, 8 * h + 4 * cc + q, kBoxBytes), Elem<T>::pack(&yh[8 * q]));
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -391,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       tmem_ld32(tm_x + 32u * (uint32_t)cc, v);
 #pragma unroll
       for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<uint4*>(tbuf + sw128_chunk(r, 8 * h + 4 * cc + q, kBoxBytes)) = Elem<T>::pack(&v[8 * q]);
+        sts_v4(tbuf_s + sw128_chunk(r, 8 * h + 4 * cc + q, kBoxBytes), Elem<T>::pack(&v[8 * q]));
     }
     fence_proxy_async_smem();
     tc_fence_before();

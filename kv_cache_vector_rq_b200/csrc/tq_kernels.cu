@@ -427,7 +427,7 @@ __global__ void __launch_bounds__(kThreadsM, 2)
 #pragma unroll
     for (int w = 0; w < WH; ++w) wc[w] = 0u;
     auto put = [&](int j, const float* v) {
-      *reinterpret_cast<uint4*>(tbuf + sw128_chunk(r, j, kBoxBytes)) = Elem<T>::pack(v);
+      sts_v4(tbuf_s + sw128_chunk(r, j, kBoxBytes), Elem<T>::pack(v));
     };
     auto store_outputs = [&]() {  // code words and norm of this half row
       if (!kQ || !live) return;
@@ -457,7 +457,7 @@ __global__ void __launch_bounds__(kThreadsM, 2)
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         float f[8];
-        Elem<T>::unpack(*reinterpret_cast<const uint4*>(tbuf + sw128_chunk(r, 8 * h + j, kBoxBytes)), f);
+        Elem<T>::unpack(lds_v4(tbuf_s + sw128_chunk(r, 8 * h + j, kBoxBytes)), f);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const float2 v = make_float2(f[2 * q], f[2 * q + 1]);
@@ -737,7 +737,7 @@ __global__ void __launch_bounds__(kThreadsM, 2)
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       float f[8];
-      Elem<T>::unpack(*reinterpret_cast<const uint4*>(s_buf + sw128_chunk(r, 8 * h + j, kBoxBytes)), f);
+      Elem<T>::unpack(lds_v4(buf_s + sw128_chunk(r, 8 * h + j, kBoxBytes)), f);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const float2 v = make_float2(f[2 * q], f[2 * q + 1]);
