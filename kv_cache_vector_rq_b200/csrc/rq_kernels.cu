@@ -1066,6 +1066,370 @@ __global__ void __launch_bounds__(kThreads) rq_wide_kernel(RqArgs a) {
 }  // namespace wide
 
 // ============================================================================
+// d > 256 with 16-bit rows: a warp per row, each lane a contiguous run of R groups.
+// ============================================================================
+// Rows stream into shared memory by bulk copy (two buffers per warp). Lane t owns groups
+// R t .. R t + R - 1 (R a multiple of 8, so its 3R elements start on a 16-byte boundary and
+// d, a multiple of 8, ends on a chunk boundary): it reads its elements as 16-byte chunks,
+// rotates group pairs with packed f32x2 FMAs on the pairs' exact sandwich matrices,
+// quantizes with the row kernel's binary search (b >= 3) or saturating steps (b <= 2),
+// writes x_hat back in place, and ORs its contiguous code bits into the warp's staged code
+// words. The pair matrices sit in a per-lane table whose lane stride is padded by 16 bytes,
+// so the lanes' 16-byte loads of their own matrices spread over the banks.
+namespace run {
+
+constexpr int kWarps = 8;
+constexpr int kThreads = 32 * kWarps;
+
+struct Layout {
+  int G, W, lane_bytes, row_bytes, buf_off, codes_off, lut_off, bar_off, cb_off, bytes;
+  __host__ __device__ Layout(int d, int bits, int R) {
+    G = (d + 2) / 3;
+    W = (3 * G * bits + 31) / 32;
+    lane_bytes = (R / 2) * 80 + 16;
+    row_bytes = d * 2;
+    buf_off = ((32 * lane_bytes + 127) / 128) * 128;
+    codes_off = buf_off + kWarps * 2 * row_bytes;
+    lut_off = codes_off + ((kWarps * W * 4 + 15) / 16) * 16;  // dequantize: [warp][16] centroids
+    bar_off = lut_off + kWarps * 16 * 4;
+    cb_off = bar_off + kWarps * 2 * 8;
+    bytes = cb_off + 64 * 4;
+  }
+};
+
+// run length (groups per lane) for d, 0 when the run kernel does not take d
+__host__ __device__ inline int run_groups(int d) {
+  if (d <= 256 || d % 8 != 0) return 0;
+  const int G = (d + 2) / 3;
+  for (int R = 8; R <= 48; R += 8)
+    if (32 * R >= G) return R;
+  return 0;
+}
+
+// two CTAs per SM where their row buffers fit (R <= 24: d <= 2304), so registers are capped at 128
+template <typename T, int BITS, int MODE, int R>
+__global__ void __launch_bounds__(kThreads, R <= 24 ? 2 : 1) rq_run_kernel(RqArgs a) {
+  constexpr int K = 1 << BITS, H = K / 2;
+  constexpr bool kIn = MODE != RQ_DQ, kOut = MODE != RQ_Q;
+  constexpr bool kScale = !std::is_same<T, __half>::value;  // fp16 norms always lie in [2^-24, 2^20]
+  constexpr int E = 8;                 // elements per 16-byte chunk
+  constexpr int NE = 3 * R;            // elements (and codes) of a lane's run
+  constexpr int NCH = NE / E;          // chunks of the run
+  constexpr int NP = R / 2;            // group pairs of the run
+  constexpr int CPW = 23 / BITS;       // codes per float window
+  constexpr int NWIN = (NE + CPW - 1) / CPW;
+  constexpr int WLOC = (NE * BITS + 31) / 32;  // words of the run's own bit stream
+  constexpr bool kBisect = BITS >= 3;
+  static_assert(R % 8 == 0 && NE % E == 0, "run");
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int d = a.d;
+  const Layout L(d, BITS, R);
+  const int G = L.G, W = L.W;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* s_sc = reinterpret_cast<float*>(smem + L.cb_off);
+  float* s_mag = s_sc + 16;
+  float* s_cf = s_sc + 32;
+
+  // the per-lane table of pair matrices: lane t, pair p at t * lane_bytes + 80 p, (M_2p, M_2p+1) interleaved
+  for (int idx = threadIdx.x; idx < 32 * R; idx += kThreads) {
+    const int t = idx / R, gl = idx - t * R, g = R * t + gl;
+    float m[9];
+    if (g < G) {
+      const float4 r4 = __ldg(reinterpret_cast<const float4*>(a.rotors) + g);
+      rotor_matrix(r4.x, r4.y, r4.z, r4.w, m);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 9; ++k) m[k] = 0.f;
+    }
+    float* dst = reinterpret_cast<float*>(smem + t * L.lane_bytes + (gl >> 1) * 80) + (gl & 1);
+#pragma unroll
+    for (int k = 0; k < 9; ++k) dst[2 * k] = m[k];
+    dst[18] = 0.f;
+  }
+  row::build_consts<BITS>(a.centroids, s_sc, s_mag, s_cf);
+  uint8_t* w_buf = smem + L.buf_off + warp * 2 * L.row_bytes;
+  uint64_t* w_bar = reinterpret_cast<uint64_t*>(smem + L.bar_off) + warp * 2;
+  uint32_t* w_codes = reinterpret_cast<uint32_t*>(smem + L.codes_off) + warp * W;
+  float* w_lut = reinterpret_cast<float*>(smem + L.lut_off) + warp * 16;
+  for (int i = lane; i < W; i += 32) w_codes[i] = 0u;
+  if (lane == 0) {
+    mbar_init(&w_bar[0], 1);
+    mbar_init(&w_bar[1], 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  const int64_t n = a.n;
+  const int64_t gw = (int64_t)blockIdx.x * kWarps + warp, tw = (int64_t)gridDim.x * kWarps;
+  const T* xin = reinterpret_cast<const T*>(a.x);
+  T* xo_g = reinterpret_cast<T*>(a.xhat);
+  const uint32_t rb_bytes = (uint32_t)L.row_bytes;
+  auto issue = [&](int64_t row, int s) {  // lane 0
+    mbar_arrive_expect_tx(&w_bar[s], rb_bytes);
+    bulk_load(w_buf + s * L.row_bytes, xin + row * a.ldx, rb_bytes, &w_bar[s]);
+  };
+  if (kIn && lane == 0)
+    for (int s = 0; s < 2; ++s)
+      if (gw + s * tw < n) issue(gw + s * tw, s);
+
+  const int e0 = NE * lane;  // the run's first element
+  const uint32_t tab_a = smem_u32(smem) + (uint32_t)(lane * L.lane_bytes);
+  const uint32_t codes_a = smem_u32(w_codes);
+  const int base = NE * BITS * lane;  // the run's first code bit in the row's stream
+  float sc[H > 1 ? H - 1 : 1];
+#pragma unroll
+  for (int j = 0; j < H - 1; ++j) sc[j] = s_sc[j];
+  uint32_t par = 0;
+  int it = 0;
+  bool failed = false;
+  for (int64_t row = gw; row < n; row += tw, ++it) {
+    const int s = it & 1;
+    uint8_t* rb = w_buf + s * L.row_bytes;
+    const uint32_t run_a = smem_u32(rb) + (uint32_t)(e0 * 2);
+    bool ok = true;
+    if constexpr (kIn) {
+      ok = mbar_wait(&w_bar[s], (par >> s) & 1, a.status);
+      par ^= 1u << s;
+    } else if (lane == 0) {
+      bulk_wait_read<1>();  // the x_hat store that last used this buffer has read it
+    }
+    if (!__all_sync(0xffffffffu, ok)) {
+      failed = true;
+      break;
+    }
+    auto chunk_in = [&](int c) { return e0 + E * c < d; };  // d and e0 are multiples of 8
+
+    // ---------------------------------------------------------------- per-row scale
+    float xs = 1.f, nrm, nq;
+    if constexpr (kIn) {
+      float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) {
+        if (chunk_in(c)) {
+          float f[E];
+          Elem<T>::unpack(lds_v4(run_a + 16u * c), f);
+#pragma unroll
+          for (int k = 0; k < E / 2; ++k) {
+            const float2 v = make_float2(f[2 * k], f[2 * k + 1]);
+            acc[k & 1] = __ffma2_rn(v, v, acc[k & 1]);
+          }
+        }
+      }
+      float ss = (acc[0].x + acc[1].x) + (acc[0].y + acc[1].y);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      if (kScale && !(ss >= 0x1p-100f && ss <= 0x1p100f)) {
+        xs = ss < 1.f ? 0x1p100f : 0x1p-100f;
+        ss = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < NCH; ++c) {
+          if (chunk_in(c)) {
+            float f[E];
+            Elem<T>::unpack(lds_v4(run_a + 16u * c), f);
+            for (int k = 0; k < E; ++k) ss = fmaf(f[k] * xs, f[k] * xs, ss);
+          }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      }
+      nq = sqrtf(ss);
+      nrm = kScale ? nq / xs : nq;
+    } else {
+      nrm = __ldg(a.norms_in + row * a.ldn);
+      nq = nrm;
+      const uint32_t* cin = a.codes_in + row * a.ldc;
+      for (int i = lane; i < W; i += 32) w_codes[i] = __ldg(cin + i);
+    }
+
+    // scaled magnitudes (the row kernel's sequence, so that quantize and dequantize agree bit for bit)
+    const float mn0 = __fmul_rn(s_mag[0], nrm);
+    float dl[H > 1 ? H - 1 : 1];
+    Bisect<kBisect ? BITS : 3> bs;
+    if constexpr (kBisect) {
+      float Mj[H];
+#pragma unroll
+      for (int j = 0; j < H; ++j) Mj[j] = __fmul_rn(s_mag[j], nrm);
+      bs.magnitudes(Mj);
+      bs.thresholds(sc);
+    } else {
+      float prev = mn0;
+#pragma unroll
+      for (int j = 1; j < H; ++j) {
+        const float cur = __fmul_rn(s_mag[j], nrm);
+        dl[j - 1] = __fsub_rn(cur, prev);
+        prev = cur;
+      }
+    }
+    uint32_t lw[WLOC + 1];  // dequantize: the run's code words, aligned to its first code
+    if constexpr (!kIn) {
+      if (lane < H) {
+        float ch;
+        if constexpr (kBisect) {
+          ch = bs.mag(lane);
+        } else {
+          ch = mn0;
+#pragma unroll
+          for (int j = 0; j < H - 1; ++j)
+            if (j < lane) ch = __fadd_rn(ch, dl[j]);
+        }
+        w_lut[H + lane] = ch;
+        w_lut[H - 1 - lane] = -ch;
+      }
+      __syncwarp();
+      const int w0 = base >> 5, sh = base & 31;
+      uint32_t raw[WLOC + 1];
+#pragma unroll
+      for (int j = 0; j <= WLOC; ++j) raw[j] = (w0 + j < W) ? lds_u32(codes_a + 4u * (uint32_t)(w0 + j)) : 0u;
+#pragma unroll
+      for (int j = 0; j <= WLOC; ++j)
+        lw[j] = sh == 0 ? raw[j] : ((raw[j] >> sh) | (j < WLOC ? raw[j + 1] << (32 - sh) : 0u));
+    }
+    const uint32_t lut_a = smem_u32(w_lut);
+    const float srow = nq > 0.f ? __fdiv_rn(row::kB, nq) : 0.f;
+    const float shv = -fmaf(row::kShift, nq, 0x1p-126f);
+    const float2 shift2 = make_float2(shv, shv);
+    float win[NWIN];
+#pragma unroll
+    for (int w = 0; w < NWIN; ++w) win[w] = row::kWindow0;
+
+    // ---------------------------------------------------------------- group pairs of the run
+    float xe[NE + 6], xo[NE];
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+      if constexpr (kIn) {
+#pragma unroll
+        for (int e = 6 * p; e < 6 * p + 6; ++e)
+          if (e % E == 0) {
+            if (chunk_in(e / E)) {
+              Elem<T>::unpack(lds_v4(run_a + 16u * (uint32_t)(e / E)), &xe[e]);
+              if constexpr (kScale) {
+#pragma unroll
+                for (int k = 0; k < E; ++k) xe[e + k] *= xs;
+              }
+            } else {
+#pragma unroll
+              for (int k = 0; k < E; ++k) xe[e + k] = 0.f;
+            }
+          }
+      }
+      float2 M[10];
+#pragma unroll
+      for (int q = 0; q < 5; ++q) {
+        const uint4 t4 = lds_v4(tab_a + (uint32_t)((p * 5 + q) * 16));
+        M[2 * q] = make_float2(__uint_as_float(t4.x), __uint_as_float(t4.y));
+        M[2 * q + 1] = make_float2(__uint_as_float(t4.z), __uint_as_float(t4.w));
+      }
+      // groups R lane + 2p (lane x) and R lane + 2p + 1 (lane y); beyond G neither codes nor elements
+      const bool gx = R * lane + 2 * p < G, gy = R * lane + 2 * p + 1 < G;
+      float2 C[3];
+      if constexpr (kIn) {
+        float2 V[3];
+#pragma unroll
+        for (int j = 0; j < 3; ++j) V[j] = make_float2(xe[6 * p + j], xe[6 * p + 3 + j]);
+#pragma unroll
+        for (int i = 0; i < 3; ++i) {
+          const float2 Y =
+              __ffma2_rn(M[3 * i + 2], V[2], __ffma2_rn(M[3 * i + 1], V[1], __ffma2_rn(M[3 * i], V[0], shift2)));
+          float2 m2 = make_float2(mn0, mn0);
+          float2 cnt = make_float2(0.5f, 0.5f);
+          if constexpr (kBisect) {
+            bs(make_float2(fabsf(Y.x), fabsf(Y.y)), srow, m2, cnt);
+          } else {
+#pragma unroll
+            for (int j = 0; j < H - 1; ++j) {
+              const float2 st = make_float2(fma_sat(fabsf(Y.x), srow, sc[j]), fma_sat(fabsf(Y.y), srow, sc[j]));
+              m2 = __ffma2_rn(st, make_float2(dl[j], dl[j]), m2);
+              cnt = __fadd2_rn(cnt, st);
+            }
+          }
+          const float2 sg = make_float2(sign_one(Y.x), sign_one(Y.y));
+          C[i] = __fmul2_rn(m2, sg);
+          const float2 code = __ffma2_rn(sg, cnt, make_float2(H - 0.5f, H - 0.5f));
+          const int kx = 6 * p + i, ky = 6 * p + 3 + i;  // code indices in the run
+          if (gx) win[kx / CPW] = fmaf(code.x, (float)(1u << (BITS * (kx % CPW))), win[kx / CPW]);
+          if (gy) win[ky / CPW] = fmaf(code.y, (float)(1u << (BITS * (ky % CPW))), win[ky / CPW]);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 3; ++i) {
+          const int kx = 6 * p + i, ky = 6 * p + 3 + i;
+          const float cx = gx ? __uint_as_float(lds_u32(lut_a + 4u * get_code<BITS, WLOC + 1>(lw, kx))) : 0.f;
+          const float cy = gy ? __uint_as_float(lds_u32(lut_a + 4u * get_code<BITS, WLOC + 1>(lw, ky))) : 0.f;
+          C[i] = make_float2(cx, cy);
+        }
+      }
+      if constexpr (kOut) {
+#pragma unroll
+        for (int i = 0; i < 3; ++i) {
+          const float2 X = __ffma2_rn(M[6 + i], C[2], __ffma2_rn(M[3 + i], C[1], __fmul2_rn(M[i], C[0])));
+          xo[6 * p + i] = X.x;
+          xo[6 * p + 3 + i] = X.y;
+        }
+#pragma unroll
+        for (int e = 6 * p; e < 6 * p + 6; ++e)
+          if (e % E == E - 1 && chunk_in(e / E)) sts_v4(run_a + 16u * (uint32_t)(e / E), Elem<T>::pack(&xo[e - (E - 1)]));
+      }
+    }
+
+    // ---------------------------------------------------------------- outputs
+    if constexpr (kIn) {
+      // the run's bit stream (codes past the row's 3G left at zero), shifted to its place in the row's words
+      uint32_t wl[WLOC];
+#pragma unroll
+      for (int w = 0; w < WLOC; ++w) wl[w] = 0u;
+#pragma unroll
+      for (int w = 0; w < NWIN; ++w) {
+        const uint32_t v = __float_as_uint(win[w]) & 0x7fffffu;
+        const int bo = w * CPW * BITS;
+        wl[bo >> 5] |= v << (bo & 31);
+        if ((bo & 31) + CPW * BITS > 32 && (bo >> 5) + 1 < WLOC) wl[(bo >> 5) + 1] |= v >> (32 - (bo & 31));
+      }
+      const int w0 = base >> 5, sh = base & 31;
+#pragma unroll
+      for (int j = 0; j <= WLOC; ++j) {
+        const uint32_t lo = j < WLOC ? wl[j] << sh : 0u;
+        const uint32_t hi = (j > 0 && sh != 0) ? wl[j - 1] >> (32 - sh) : 0u;
+        const uint32_t v = lo | hi;
+        if (v != 0u && w0 + j < W) red_or_shared(codes_a + 4u * (uint32_t)(w0 + j), v);
+      }
+      if (lane == 0 && a.norms_out) a.norms_out[row * a.ldn] = nrm;
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if constexpr (kIn) {
+      if (a.codes_out) {
+        uint32_t* cout = a.codes_out + row * a.ldc;
+        for (int i = lane; i < W; i += 32) cout[i] = w_codes[i];
+      }
+      __syncwarp();
+      for (int i = lane; i < W; i += 32) w_codes[i] = 0u;
+    }
+    if (lane == 0) {
+      if constexpr (kOut) {
+        bulk_store(xo_g + row * a.ldo, rb, rb_bytes);
+        bulk_commit();
+      }
+      if constexpr (kIn) {
+        const int64_t next = row + 2 * tw;
+        if (next < n) {
+          if (kOut) bulk_wait_read<0>();  // the x_hat store has read the buffer
+          issue(next, s);
+        }
+      }
+    }
+    __syncwarp();
+  }
+  if (lane == 0) {
+    // after a failed wait, the copy into the other buffer (if any) lands before the warp exits
+    if (failed && gw + (int64_t)(it + 1) * tw < n) mbar_wait(&w_bar[(it + 1) & 1], (par >> ((it + 1) & 1)) & 1, a.status);
+    bulk_wait_all<0>();
+  }
+}
+
+}  // namespace run
+
+// ============================================================================
 // Launch helpers (host)
 // ============================================================================
 template <typename T, int BITS, int MODE, bool RING, int DD, int L>
@@ -1198,8 +1562,58 @@ cudaError_t launch_rq_row(int mode, kvrq_dtype dt, int bits, const CUtensorMap& 
   }
 }
 
+template <typename T, int BITS, int MODE, int R>
+static cudaError_t launch_run_t(const RqArgs& a, cudaStream_t st, int num_sms) {
+  const run::Layout L(a.d, BITS, R);
+  auto kern = run::rq_run_kernel<T, BITS, MODE, R>;
+  static int set_bytes = 0;
+  if (L.bytes > set_bytes) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.bytes);
+    if (e != cudaSuccess) return e;
+    set_bytes = L.bytes;
+  }
+  int per_sm = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, run::kThreads, L.bytes);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) per_sm = 1;
+  const int64_t grid = std::min<int64_t>((a.n + run::kWarps - 1) / run::kWarps, (int64_t)num_sms * per_sm);
+  kern<<<(unsigned)grid, run::kThreads, L.bytes, st>>>(a);
+  return cudaGetLastError();
+}
+
+// Run length of the run kernel for 16-bit rows of d, or 0 (the bulk-copy kernel takes d).
+static int run_length(int d, int bits) {
+  int R = run::run_groups(d);
+  if (R == 32 || R == 40) R = 48;  // instantiated lengths: 8, 16, 24, 48
+  if (R == 0 || run::Layout(d, bits, R).bytes > 227 * 1024) return 0;
+  return R;
+}
+
+template <typename T, int BITS, int MODE>
+static cudaError_t launch_run(int R, const RqArgs& a, cudaStream_t st, int sms) {
+  switch (R) {
+    case 8: return launch_run_t<T, BITS, MODE, 8>(a, st, sms);
+    case 16: return launch_run_t<T, BITS, MODE, 16>(a, st, sms);
+    case 24: return launch_run_t<T, BITS, MODE, 24>(a, st, sms);
+    default: return launch_run_t<T, BITS, MODE, 48>(a, st, sms);
+  }
+}
+
 template <typename TI, typename TO, int MODE>
 static cudaError_t gen_by_bits(int bits, const RqArgs& a, cudaStream_t st, int sms) {
+  using TB = typename std::conditional<MODE != RQ_DQ, TI, TO>::type;
+  if constexpr (sizeof(TB) == 2) {
+    // 16-bit rows of d > 256: a warp per row, a contiguous run of groups per lane
+    const int R = a.wide ? run_length(a.d, bits) : 0;
+    if (R > 0) {
+      switch (bits) {
+        case 1: return launch_run<TB, 1, MODE>(R, a, st, sms);
+        case 2: return launch_run<TB, 2, MODE>(R, a, st, sms);
+        case 3: return launch_run<TB, 3, MODE>(R, a, st, sms);
+        default: return launch_run<TB, 4, MODE>(R, a, st, sms);
+      }
+    }
+  }
   if (a.wide) {
     switch (bits) {
       case 1: return launch_wide<TI, TO, 1, MODE>(a, st, sms);

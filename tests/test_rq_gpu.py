@@ -186,3 +186,26 @@ def test_output_canaries_untouched_on_ragged_tail():
     assert norms_buf[0].item() == -1.0 and norms_buf[n + 1].item() == -1.0
     assert torch.all(xh_buf[0] == -3.0) and torch.all(xh_buf[n + 1] == -3.0)
     kvrq.device_status()
+
+
+@pytest.mark.parametrize("d,bits,dt", [(264, 2, torch.float16), (384, 3, torch.bfloat16), (1000, 3, torch.float16),
+                                       (1000, 1, torch.bfloat16), (3072, 4, torch.float16), (4608, 3, torch.float16),
+                                       (4608, 2, torch.bfloat16)])
+def test_run_lengths(d, bits, dt):
+    """16-bit rows of d > 256 (a multiple of 8) take the warp-per-row kernel whose lanes own contiguous runs
+    of 8, 16, 24 or 48 groups: lanes past the last group, a zero-padded last group (d = 1000), and the
+    largest d the run table and row buffers fit (4608)."""
+    x = synth.lognormal(97, d, seed=d + bits, dtype=dt).cuda()
+    _check_roundtrip(x, bits)
+
+
+@pytest.mark.parametrize("dt", [torch.float16, torch.bfloat16])
+def test_run_zero_rows_and_extreme_norms(dt):
+    d = 1536
+    x = synth.lognormal(64, d, seed=4, dtype=torch.float32)
+    x[3] = 0.0
+    if dt == torch.bfloat16:
+        x[5] *= 1e30  # norms beyond fp32's square range: the power-of-two prescale
+        x[6] *= 1e-30
+    _, _, xhat = _check_roundtrip(x.to(dt).cuda(), 3)
+    assert np.all(to_f64(xhat)[3] == 0.0)
