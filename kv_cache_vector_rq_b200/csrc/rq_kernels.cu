@@ -21,10 +21,13 @@
 //  * Quantization compares |y| with the positive Lloyd-Max boundaries scaled by
 //    the row norm (so x is never divided by its norm), exploiting the exact
 //    symmetry of the codebook.
+//  * 16-bit rows of d > 256 (a multiple of 8, up to 4,608) go through
+//    `rq_run_kernel`: rows streamed into shared memory by bulk copy, a warp per
+//    row, each lane a contiguous run of groups on packed f32x2 FMAs.
 //  * Other d with 16-byte aligned rows go through `rq_wide_kernel` (rows
-//    streamed into shared memory by bulk copy, a warp per row); anything else
-//    through `rq_general_kernel`: one warp per row, groups strided over lanes,
-//    codes assembled per warp in shared memory.
+//    streamed into shared memory by bulk copy, a warp per row, groups strided
+//    over the lanes); anything else through `rq_general_kernel`: one warp per
+//    row, groups strided over lanes, codes assembled per warp in shared memory.
 
 #include <cuda_runtime.h>
 
