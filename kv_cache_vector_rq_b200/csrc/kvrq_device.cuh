@@ -327,6 +327,16 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {  
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
+// a0 += lo * lo, a1 += hi * hi for the two fp16 halves of w, each one fused multiply-add with
+// fp16 operands and an fp32 accumulator (sm_100a): the product of two fp16 values is exact in
+// fp32, so this rounds exactly as converting first and using an fp32 fma
+__device__ __forceinline__ void sq_acc_f16x2(uint32_t w, float& a0, float& a1) {
+  asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "fma.rn.f32.f16 %0, l, l, %0;\n\tfma.rn.f32.f16 %1, h, h, %1;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "r"(w));
+}
+
 // Maximum of v over the 32 lanes of a fully active warp, in one instruction (sm_100a); exact, as
 // the butterfly of shuffles and fmaxf it replaces.
 __device__ __forceinline__ float warp_max_f32(float v) {

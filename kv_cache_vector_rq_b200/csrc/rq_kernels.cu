@@ -433,12 +433,20 @@ __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
       for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int j = 0; j < TL::kChunks; ++j) {
-        float f[E];
-        Elem<T>::unpack(lds_v4(cptr(j)), f);
+        if constexpr (std::is_same<T, __half>::value) {
+          // fp16 squares straight into the fp32 sums (the same roundings as converting first)
+          const uint4 c = lds_v4(cptr(j));
+          const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-        for (int k = 0; k < E / 2; ++k) {
-          const float2 v = make_float2(f[2 * k], f[2 * k + 1]);
-          acc[(j * (E / 2) + k) & 3] = __ffma2_rn(v, v, acc[(j * (E / 2) + k) & 3]);
+          for (int k = 0; k < 4; ++k) sq_acc_f16x2(cw[k], acc[(j * 4 + k) & 3].x, acc[(j * 4 + k) & 3].y);
+        } else {
+          float f[E];
+          Elem<T>::unpack(lds_v4(cptr(j)), f);
+#pragma unroll
+          for (int k = 0; k < E / 2; ++k) {
+            const float2 v = make_float2(f[2 * k], f[2 * k + 1]);
+            acc[(j * (E / 2) + k) & 3] = __ffma2_rn(v, v, acc[(j * (E / 2) + k) & 3]);
+          }
         }
       }
       float ss = ((acc[0].x + acc[1].x) + (acc[2].x + acc[3].x)) + ((acc[0].y + acc[1].y) + (acc[2].y + acc[3].y));
