@@ -1218,12 +1218,19 @@ __global__ void __launch_bounds__(kThreads, R <= 24 ? 2 : 1) rq_run_kernel(RqArg
 #pragma unroll
       for (int c = 0; c < NCH; ++c) {
         if (chunk_in(c)) {
-          float f[E];
-          Elem<T>::unpack(lds_v4(run_a + 16u * c), f);
+          if constexpr (std::is_same<T, __half>::value) {  // fp16 squares straight into the fp32 sums
+            const uint4 c4 = lds_v4(run_a + 16u * c);
+            const uint32_t cw[4] = {c4.x, c4.y, c4.z, c4.w};
 #pragma unroll
-          for (int k = 0; k < E / 2; ++k) {
-            const float2 v = make_float2(f[2 * k], f[2 * k + 1]);
-            acc[k & 1] = __ffma2_rn(v, v, acc[k & 1]);
+            for (int k = 0; k < 4; ++k) sq_acc_f16x2(cw[k], acc[k & 1].x, acc[k & 1].y);
+          } else {
+            float f[E];
+            Elem<T>::unpack(lds_v4(run_a + 16u * c), f);
+#pragma unroll
+            for (int k = 0; k < E / 2; ++k) {
+              const float2 v = make_float2(f[2 * k], f[2 * k + 1]);
+              acc[k & 1] = __ffma2_rn(v, v, acc[k & 1]);
+            }
           }
         }
       }

@@ -456,12 +456,19 @@ __global__ void __launch_bounds__(kThreadsM, 2)
       for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        float f[8];
-        Elem<T>::unpack(lds_v4(tbuf_s + sw128_chunk(r, 8 * h + j, kBoxBytes)), f);
+        if constexpr (std::is_same<T, __half>::value) {  // fp16 squares straight into the fp32 sums
+          const uint4 c = lds_v4(tbuf_s + sw128_chunk(r, 8 * h + j, kBoxBytes));
+          const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 v = make_float2(f[2 * q], f[2 * q + 1]);
-          acc[q] = __ffma2_rn(v, v, acc[q]);
+          for (int q = 0; q < 4; ++q) sq_acc_f16x2(cw[q], acc[q].x, acc[q].y);
+        } else {
+          float f[8];
+          Elem<T>::unpack(lds_v4(tbuf_s + sw128_chunk(r, 8 * h + j, kBoxBytes)), f);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 v = make_float2(f[2 * q], f[2 * q + 1]);
+            acc[q] = __ffma2_rn(v, v, acc[q]);
+          }
         }
       }
       s_part[h * kRows + r] =
@@ -736,12 +743,19 @@ __global__ void __launch_bounds__(kThreadsM, 2)
     for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      float f[8];
-      Elem<T>::unpack(lds_v4(buf_s + sw128_chunk(r, 8 * h + j, kBoxBytes)), f);
+      if constexpr (std::is_same<T, __half>::value) {  // fp16 squares straight into the fp32 sums
+        const uint4 c = lds_v4(buf_s + sw128_chunk(r, 8 * h + j, kBoxBytes));
+        const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 v = make_float2(f[2 * q], f[2 * q + 1]);
-        acc[q] = __ffma2_rn(v, v, acc[q]);
+        for (int q = 0; q < 4; ++q) sq_acc_f16x2(cw[q], acc[q].x, acc[q].y);
+      } else {
+        float f[8];
+        Elem<T>::unpack(lds_v4(buf_s + sw128_chunk(r, 8 * h + j, kBoxBytes)), f);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 v = make_float2(f[2 * q], f[2 * q + 1]);
+          acc[q] = __ffma2_rn(v, v, acc[q]);
+        }
       }
     }
     s_part[h * kRows + r] =
