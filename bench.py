@@ -855,17 +855,15 @@ def main():
     codes_h = torch.empty((N_VEC, W[HEADLINE_BITS]), dtype=torch.int32).pin_memory()
     norms_h = torch.empty(N_VEC, dtype=torch.float32).pin_memory()
     xhat_h = torch.empty_like(x_host).pin_memory()
-    xd = torch.empty_like(x)
+    # the host-buffer call: chunks of 16,384 rows whose copy-in, kernel and copy-out overlap (smaller chunks pay
+    # the fixed cost of each copy more often: 4,096-row chunks measured 0.82 ms a step, 16,384-row ones 0.62 ms)
+    ws = torch.empty(kvrq.host_workspace_bytes(D, HEADLINE_BITS, torch.float16, 16384), dtype=torch.uint8, device=dev)
     e2e_ms = []
     for i in range(args.warmup + args.steps):
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s.record(stream)
-        xd.copy_(x_host, non_blocking=True)
-        kvrq.rq_quantize_dequantize(xd, rot, cbs[HEADLINE_BITS], HEADLINE_BITS, codes=codes[HEADLINE_BITS],
-                                    norms=norms, xhat=xhat, stream=stream)
-        codes_h.copy_(codes[HEADLINE_BITS], non_blocking=True)
-        norms_h.copy_(norms, non_blocking=True)
-        xhat_h.copy_(xhat, non_blocking=True)
+        kvrq.rq_quantize_dequantize_host(x_host, rot, cbs[HEADLINE_BITS], HEADLINE_BITS, ws, codes=codes_h,
+                                         norms=norms_h, xhat=xhat_h, stream=stream)
         e.record(stream)
         e.synchronize()
         if i >= args.warmup:

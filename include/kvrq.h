@@ -171,6 +171,36 @@ kvrq_status rq_quantize_dequantize(void* stream, const void* x, kvrq_dtype xdtyp
                                    int64_t ldx, const float* rotors, const float* centroids, int bits,
                                    uint32_t* codes, int64_t ldc, float* norms, void* xhat, int64_t ldo);
 
+/* RotorQuant fused roundtrip of rows in HOST memory ["TurboQuant + RotorQuant", "Post-Prefill
+ * Quantization" (a prefill cache quantized in bulk) and "Triton Kernel Speed" (one fused launch per
+ * block of vectors)]: the rows are copied to the device in chunks, each chunk is quantized and
+ * dequantized there by rq_quantize_dequantize, and its codes, norms and x_hat are copied back; the
+ * copy-in of one chunk, the kernel of the previous one and the copy-out of the one before run at
+ * once, on three streams the library creates per device. The call is ordered after the work queued
+ * on `stream` before it (and after the copy-outs of earlier calls of this function on the device),
+ * work queued on `stream` after it waits for its last copy-out, and it returns without waiting.
+ *   x      [n][ldx] host rows (fp32, fp16 or bf16), xhat [n][ldo] host rows of the same dtype;
+ *   codes  [n][ldc] host uint32 (may be NULL), norms [n] host fp32 (may be NULL);
+ *   rotors, centroids: device arrays as for rq_quantize_dequantize.
+ *   workspace: device memory, 256-byte aligned, of workspace_bytes >= kvrq_host_workspace_bytes(d,
+ *   bits, xdtype, 32); the call takes the largest chunk (32 rows times a power of two) whose three
+ *   slots fit, at most the input rounded up to 32 rows. Host arrays should be page-locked
+ *   (cudaHostAlloc, cudaHostRegister): pageable memory gives the same results with the copies
+ *   serialised by the driver. Nothing is allocated by the call.
+ *   KVRQ_EINVAL: NULL pointers, ldx, ldo < d, ldc below the code words of a row, a misaligned or
+ *   too small workspace; these are checked before anything is queued. KVRQ_ECUDA: a copy, event
+ *   or launch failed; copies and kernels queued before the failure may still run, so the caller
+ *   synchronizes the device before reusing the buffers. */
+kvrq_status rq_quantize_dequantize_host(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d,
+                                        int64_t ldx, const float* rotors, const float* centroids, int bits,
+                                        uint32_t* codes, int64_t ldc, float* norms, void* xhat, int64_t ldo,
+                                        void* workspace, size_t workspace_bytes);
+
+/* Device workspace bytes rq_quantize_dequantize_host needs for chunks of chunk_rows rows (rounded up
+ * to a multiple of 32; at least 32): three slots of x and x_hat rows padded to 16 bytes, code words
+ * and norms. 0 for arguments the call rejects. */
+size_t kvrq_host_workspace_bytes(int d, int bits, kvrq_dtype dtype, int64_t chunk_rows);
+
 /* RotorQuant in the pages' four-grade storage layout [RQ "Parameter Efficiency"
  * (rotors plus four grade codebooks), "FMA Count (d=128)" table (172 stored
  * indices per vector, 3.7x at 3 bits), "The Fused CUDA Kernel" (a grade-1 input

@@ -204,6 +204,51 @@ def rq_quantize_dequantize(x, rotors, centroids, bits, codes=None, norms=None, x
     return codes, norms, xhat
 
 
+def host_workspace_bytes(d, bits, dtype, chunk_rows=4096):
+    """Device workspace bytes of rq_quantize_dequantize_host for chunks of chunk_rows rows."""
+    torch = _torch()
+    code = {torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}[dtype]
+    return int(lib().kvrq_host_workspace_bytes(d, bits, code, chunk_rows))
+
+
+def _host_rows(t, name):
+    """(pointer, leading dimension) of a 2-D host tensor with unit inner stride."""
+    if t.is_cuda:
+        raise ValueError("%s must be a host tensor" % name)
+    if t.dim() != 2 or (t.shape[1] > 1 and t.stride(1) != 1):
+        raise ValueError("%s must be 2-D with unit column stride" % name)
+    return t.data_ptr(), (t.stride(0) if t.shape[0] > 1 else t.shape[1])
+
+
+def rq_quantize_dequantize_host(x, rotors, centroids, bits, workspace, codes=None, norms=None, xhat=None,
+                                stream=None):
+    """Fused roundtrip of host rows x [n, d] (ideally pinned) through the device, in chunks whose copy-in, kernel
+    and copy-out overlap: returns host (codes [n, W], norms [n], x_hat [n, d]) (pinned when allocated here).
+    workspace: a CUDA tensor of at least host_workspace_bytes(d, bits, x.dtype, 32) bytes. Asynchronous on
+    `stream`, like the device calls: synchronize before reading the outputs."""
+    torch = _torch()
+    n, d = x.shape
+    W = packed_words(3 * rq_groups(d), bits)
+    if codes is None:
+        codes = torch.empty((n, W), dtype=torch.int32).pin_memory()
+    if norms is None:
+        norms = torch.empty((n,), dtype=torch.float32).pin_memory()
+    if xhat is None:
+        xhat = torch.empty((n, d), dtype=x.dtype).pin_memory()
+    if not workspace.is_cuda:
+        raise ValueError("workspace must be a CUDA tensor")
+    xp, ldx = _host_rows(x, "x")
+    cp, ldc = _host_rows(codes, "codes")
+    op, ldo = _host_rows(xhat, "xhat")
+    if norms.is_cuda or not norms.is_contiguous() or norms.dtype != torch.float32:
+        raise ValueError("norms must be a contiguous fp32 host tensor")
+    _lib.check("rq_quantize_dequantize_host", lib().rq_quantize_dequantize_host(
+        _stream(stream), xp, _dtype_code(x), n, d, ldx, _ptr(rotors, "rotors", torch.float32),
+        _ptr(centroids, "centroids", torch.float32), bits, cp, ldc, norms.data_ptr(), op, ldo, workspace.data_ptr(),
+        workspace.numel() * workspace.element_size()))
+    return codes, norms, xhat
+
+
 def rq4_quantize(x, rotors, centroids, bits, codes=None, norms=None, stream=None):
     """RotorQuant in the four-grade layout (4 codes per group, 172 at d = 128): (codes [n, W], norms [n])."""
     return rq_quantize(x, rotors, centroids, bits, codes, norms, stream, _fn="rq4_quantize", _cpg=4)

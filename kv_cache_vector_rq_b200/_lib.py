@@ -35,6 +35,11 @@ SIGNATURES = {
     # stream, x, xdtype, n, d, ldx, rotors, centroids, bits, codes, ldc, norms, xhat, ldo
     "rq_quantize_dequantize": (c_int, [c_vp, c_vp, c_int, c_i64, c_int, c_i64, c_vp, c_vp, c_int, c_vp, c_i64, c_vp,
                                        c_vp, c_i64]),
+    # stream, x (host), xdtype, n, d, ldx, rotors, centroids, bits, codes (host), ldc, norms (host), xhat (host),
+    # ldo, workspace (device), workspace bytes
+    "rq_quantize_dequantize_host": (c_int, [c_vp, c_vp, c_int, c_i64, c_int, c_i64, c_vp, c_vp, c_int, c_vp, c_i64,
+                                            c_vp, c_vp, c_i64, c_vp, ctypes.c_size_t]),
+    "kvrq_host_workspace_bytes": (ctypes.c_size_t, [c_int, c_int, c_int, c_i64]),
     "rq4_quantize": (c_int, [c_vp, c_vp, c_int, c_i64, c_int, c_i64, c_vp, c_vp, c_int, c_vp, c_i64, c_vp]),
     "rq4_dequantize": (c_int, [c_vp, c_vp, c_i64, c_vp, c_i64, c_int, c_vp, c_vp, c_int, c_vp, c_int, c_i64]),
     "rq4_quantize_dequantize": (c_int, [c_vp, c_vp, c_int, c_i64, c_int, c_i64, c_vp, c_vp, c_int, c_vp, c_i64, c_vp,

@@ -67,11 +67,21 @@ static kvrq_status cuda_fail(const char* where, cudaError_t e) {
 constexpr size_t kNoallocScratchBytes = (size_t)8 << 20;
 static __device__ __align__(256) unsigned char g_tq_scratch[kNoallocScratchBytes];
 
+constexpr int kHostSlots = 3;  // chunks in flight in the host-buffer pipeline
+
 struct DeviceInfo {
   bool ready = false;
   int num_sms = 0;
   unsigned* status = nullptr;  // device address of g_device_status
   void* scratch = nullptr;     // device address of g_tq_scratch
+  // host-buffer pipeline (created at its first call): copy-in, compute and copy-out streams,
+  // per-slot events, the start and end events of a call, and a lock that keeps one call's
+  // issue sequence whole
+  bool pipe_ready = false;
+  cudaStream_t pipe[3] = {nullptr, nullptr, nullptr};
+  cudaEvent_t in_done[kHostSlots] = {}, comp_done[kHostSlots] = {}, out_done[kHostSlots] = {};
+  cudaEvent_t ev_start = nullptr, ev_end = nullptr;
+  std::mutex pipe_mu;
 };
 
 static std::mutex g_dev_mu;
@@ -598,6 +608,131 @@ kvrq_status rq_quantize_dequantize(void* stream, const void* x, kvrq_dtype xdtyp
                                    int64_t ldc, float* norms, void* xhat, int64_t ldo) {
   return rq_call("rq_quantize_dequantize", RQ_QDQ, stream, x, xdtype, ldx, nullptr, codes, ldc, nullptr, norms, n, d,
                  rotors, centroids, bits, xhat, xdtype, ldo);
+}
+
+// ------------------------------------------------------------------ host-buffer roundtrip
+// Device bytes of one chunk slot: x and x_hat rows padded to 16 bytes, code words, norms.
+static size_t host_slot_bytes(int d, int bits, kvrq_dtype dt, int64_t rows) {
+  const size_t es = dtype_size(dt);
+  const size_t row = ((size_t)d * es + 15) / 16 * 16;
+  const size_t W = (size_t)kvrq_packed_words(3 * (int64_t)((d + 2) / 3), bits);
+  const size_t bytes = (size_t)rows * (2 * row + 4 * W + 4) + 4 * 256;
+  return (bytes + 255) / 256 * 256;
+}
+
+static kvrq_status pipe_init(DeviceInfo* di) {
+  if (di->pipe_ready) return KVRQ_OK;
+  cudaError_t e;
+  for (int i = 0; i < 3; ++i)
+    if ((e = cudaStreamCreateWithFlags(&di->pipe[i], cudaStreamNonBlocking)) != cudaSuccess)
+      return cuda_fail("cudaStreamCreateWithFlags", e);
+  for (int sl = 0; sl < kHostSlots; ++sl)
+    for (cudaEvent_t* ev : {&di->in_done[sl], &di->comp_done[sl], &di->out_done[sl]})
+      if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess)
+        return cuda_fail("cudaEventCreateWithFlags", e);
+  for (cudaEvent_t* ev : {&di->ev_start, &di->ev_end})
+    if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess)
+      return cuda_fail("cudaEventCreateWithFlags", e);
+  di->pipe_ready = true;
+  return KVRQ_OK;
+}
+
+static kvrq_status copy_rows(void* dst, size_t dpitch, const void* src, size_t spitch, size_t width, int64_t rows,
+                             cudaMemcpyKind kind, cudaStream_t st) {
+  cudaError_t e = dpitch == width && spitch == width
+                      ? cudaMemcpyAsync(dst, src, width * (size_t)rows, kind, st)
+                      : cudaMemcpy2DAsync(dst, dpitch, src, spitch, width, (size_t)rows, kind, st);
+  return e == cudaSuccess ? KVRQ_OK : cuda_fail("cudaMemcpyAsync", e);
+}
+
+static kvrq_status ev_chain(cudaEvent_t ev, cudaStream_t from, cudaStream_t to) {
+  cudaError_t e = cudaEventRecord(ev, from);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(to, ev, 0);
+  return e == cudaSuccess ? KVRQ_OK : cuda_fail("cudaEventRecord / cudaStreamWaitEvent", e);
+}
+
+static kvrq_status rq_host_pipeline(DeviceInfo* di, cudaStream_t caller, const uint8_t* x, kvrq_dtype dt,
+                                    int64_t n, int d, int64_t ldx, const float* rotors, const float* centroids,
+                                    int bits, uint32_t* codes, int64_t ldc, float* norms, uint8_t* xhat,
+                                    int64_t ldo, uint8_t* ws, int64_t chunk) {
+  const size_t es = dtype_size(dt);
+  const int64_t ld_dev = (int64_t)(((size_t)d * es + 15) / 16 * 16 / es);
+  const int64_t W = kvrq_packed_words(3 * (int64_t)((d + 2) / 3), bits);
+  const size_t slot = host_slot_bytes(d, bits, dt, chunk);
+  cudaStream_t in = di->pipe[0], comp = di->pipe[1], out = di->pipe[2];
+  kvrq_status st;
+  // everything queued on the caller's stream before this call comes first, and so do the copy-outs
+  // of earlier calls (the workspace slots may be the same memory)
+  for (cudaStream_t s2 : {in, comp, out})
+    if ((st = ev_chain(di->ev_start, caller, s2)) != KVRQ_OK) return st;
+  if ((st = ev_chain(di->ev_end, out, in)) != KVRQ_OK) return st;
+  for (int64_t r0 = 0, k = 0; r0 < n; r0 += chunk, ++k) {
+    const int sl = (int)(k % kHostSlots);
+    const int64_t rows = n - r0 < chunk ? n - r0 : chunk;
+    uint8_t* b = ws + (size_t)sl * slot;
+    uint8_t* dx = b;
+    uint8_t* dxh = dx + (size_t)chunk * ld_dev * es;
+    uint32_t* dc = reinterpret_cast<uint32_t*>(dxh + (size_t)chunk * ld_dev * es);
+    float* dn = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(dc) + ((size_t)chunk * W * 4 + 255) / 256 * 256);
+    cudaError_t e;
+    if (k >= kHostSlots && (e = cudaStreamWaitEvent(in, di->out_done[sl], 0)) != cudaSuccess)
+      return cuda_fail("cudaStreamWaitEvent", e);  // the slot's last copy-out has finished
+    if ((st = copy_rows(dx, ld_dev * es, x + (size_t)r0 * ldx * es, ldx * es, d * es, rows, cudaMemcpyHostToDevice,
+                        in)) != KVRQ_OK)
+      return st;
+    if ((st = ev_chain(di->in_done[sl], in, comp)) != KVRQ_OK) return st;
+    if ((st = rq_quantize_dequantize(comp, dx, dt, rows, d, ld_dev, rotors, centroids, bits, codes ? dc : nullptr, W,
+                                     norms ? dn : nullptr, dxh, ld_dev)) != KVRQ_OK)
+      return st;
+    if ((st = ev_chain(di->comp_done[sl], comp, out)) != KVRQ_OK) return st;
+    if (codes && (st = copy_rows(codes + r0 * ldc, ldc * 4, dc, W * 4, W * 4, rows, cudaMemcpyDeviceToHost, out)) !=
+                     KVRQ_OK)
+      return st;
+    if (norms && (st = copy_rows(norms + r0, 4 * rows, dn, 4 * rows, 4 * rows, 1, cudaMemcpyDeviceToHost, out)) !=
+                     KVRQ_OK)
+      return st;
+    if ((st = copy_rows(xhat + (size_t)r0 * ldo * es, ldo * es, dxh, ld_dev * es, d * es, rows,
+                        cudaMemcpyDeviceToHost, out)) != KVRQ_OK)
+      return st;
+    if ((e = cudaEventRecord(di->out_done[sl], out)) != cudaSuccess) return cuda_fail("cudaEventRecord", e);
+  }
+  // work queued on the caller's stream after this call waits for the last copy-out
+  return ev_chain(di->ev_end, out, caller);
+}
+
+size_t kvrq_host_workspace_bytes(int d, int bits, kvrq_dtype dtype, int64_t chunk_rows) {
+  if (d < 2 || bits < 1 || bits > 4 || !valid_dtype(dtype) || chunk_rows < 32) return 0;
+  return kHostSlots * host_slot_bytes(d, bits, dtype, (chunk_rows + 31) / 32 * 32);
+}
+
+kvrq_status rq_quantize_dequantize_host(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,
+                                        const float* rotors, const float* centroids, int bits, uint32_t* codes,
+                                        int64_t ldc, float* norms, void* xhat, int64_t ldo, void* workspace,
+                                        size_t workspace_bytes) {
+  const char* name = "rq_quantize_dequantize_host";
+  if (n < 0) return set_errorf(KVRQ_EINVAL, "%s: n < 0", name);
+  if (d < 2 || d > (1 << 20)) return set_errorf(KVRQ_EINVAL, "%s: d must be in 2..2^20", name);
+  if (bits < 1 || bits > 4) return set_errorf(KVRQ_EUNSUPPORTED, "%s: bits must be in 1..4", name);
+  if (!valid_dtype(xdtype)) return set_errorf(KVRQ_EINVAL, "%s: bad dtype", name);
+  if (n == 0) return KVRQ_OK;
+  if (!x || ldx < d || !xhat || ldo < d) return set_errorf(KVRQ_EINVAL, "%s: x, xhat NULL or ldx, ldo < d", name);
+  if (codes && ldc < kvrq_packed_words(3 * (int64_t)((d + 2) / 3), bits))
+    return set_errorf(KVRQ_EINVAL, "%s: ldc < the code words of a row", name);
+  if (!workspace || !aligned(workspace, 256)) return set_errorf(KVRQ_EINVAL, "%s: workspace NULL or not 256-byte aligned", name);
+  // the largest chunk of 32-row multiples whose slots fit (at most the whole input)
+  int64_t chunk = 32;
+  if (kHostSlots * host_slot_bytes(d, bits, xdtype, chunk) > workspace_bytes)
+    return set_errorf(KVRQ_EINVAL, "%s: workspace below kvrq_host_workspace_bytes(d, bits, dtype, 32)", name);
+  const int64_t cap = (n + 31) / 32 * 32;
+  while (chunk * 2 <= cap && kHostSlots * host_slot_bytes(d, bits, xdtype, chunk * 2) <= workspace_bytes) chunk *= 2;
+  DeviceInfo* di;
+  kvrq_status st = current_device(&di);
+  if (st != KVRQ_OK) return st;
+  std::lock_guard<std::mutex> lk(di->pipe_mu);
+  if ((st = pipe_init(di)) != KVRQ_OK) return st;
+  return rq_host_pipeline(di, static_cast<cudaStream_t>(stream), static_cast<const uint8_t*>(x), xdtype, n, d, ldx,
+                          rotors, centroids, bits, codes, ldc, norms, static_cast<uint8_t*>(xhat), ldo,
+                          static_cast<uint8_t*>(workspace), chunk);
 }
 
 kvrq_status pq_quantize_dequantize(void* stream, const void* x, kvrq_dtype xdtype, int64_t n, int d, int64_t ldx,

@@ -146,3 +146,34 @@ def test_paged_calls_validate_before_any_launch():
                                     1) == EUNSUP
     assert lib.kv_cache_append_rows(None, 1, P, 0, 4, 128, 128, 3, None, P, None, 128, P, P, P, 12, None, 0, P, None,
                                     1) == EUNSUP  # fp32 TurboQuant rows run the tiled kernel: no destination rows
+
+
+def test_host_roundtrip_validates_before_anything_is_queued():
+    """rq_quantize_dequantize_host checks its pointers, strides and workspace before it touches a device
+    (these run without one): NULL host arrays, ldx below d, a misaligned or too small workspace."""
+    lib = kvrq.lib()
+    d, bits = 128, 3
+    ws_min = lib.kvrq_host_workspace_bytes(d, bits, kvrq.F16, 32)
+    assert ws_min > 0 and ws_min % 256 == 0
+    assert lib.kvrq_host_workspace_bytes(d, bits, kvrq.F16, 33) == lib.kvrq_host_workspace_bytes(d, bits, kvrq.F16, 64)
+    assert lib.kvrq_host_workspace_bytes(d, bits, kvrq.F16, 31) == 0  # below one 32-row chunk
+    assert lib.kvrq_host_workspace_bytes(d, 5, kvrq.F16, 64) == 0
+    big = lib.kvrq_host_workspace_bytes(d, bits, kvrq.F16, 4096)
+    assert big > 100 * ws_min  # three slots of 4096 rows against three of 32
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: every call below fails its checks first
+    args = dict(stream=None, x=fake, dt=kvrq.F16, n=100, d=d, ldx=d, rot=fake, cb=fake, bits=bits, codes=fake, ldc=13,
+                norms=fake, xhat=fake, ldo=d, ws=fake, wsb=ws_min)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return lib.rq_quantize_dequantize_host(a["stream"], a["x"], a["dt"], a["n"], a["d"], a["ldx"], a["rot"], a["cb"],
+                                               a["bits"], a["codes"], a["ldc"], a["norms"], a["xhat"], a["ldo"],
+                                               a["ws"], a["wsb"])
+    assert call(x=None) == EINVAL
+    assert call(xhat=None) == EINVAL
+    assert call(ldx=d - 1) == EINVAL
+    assert call(ldc=12) == EINVAL  # 129 3-bit codes need 13 words
+    assert call(ws=ctypes.c_void_p((1 << 20) + 16)) == EINVAL  # not 256-byte aligned
+    assert call(wsb=ws_min - 256) == EINVAL
+    assert call(bits=5) == EUNSUP
+    assert call(n=0) == 0  # nothing to do
