@@ -151,17 +151,17 @@ struct Dims {
 constexpr int kWR = 32;       // rows per warp sub-tile
 
 // CTA shape. Ring (launches of at least two sub-tiles per warp, 16-bit rows,
-// quantize or fused, b <= 3): one 16-warp CTA per SM, each warp streaming its
-// sub-tiles through a ring of three half-tile boxes, so the next sub-tile's
-// halves load while the current one is computed and a box is reloaded as soon
-// as its x_hat store has read it (b = 4 code words leave no room for the third
-// box). Otherwise two-warp CTAs with one tile per warp, which also spread a
+// quantize or fused): one CTA per SM of 16 warps (14 at b = 4, whose code words
+// leave room for fewer warps' boxes), each warp streaming its sub-tiles through
+// a ring of three half-tile boxes, so the next sub-tile's halves load while the
+// current one is computed and a box is reloaded as soon as its x_hat store has
+// read it. Otherwise two-warp CTAs with one tile per warp, which also spread a
 // small launch over the SMs within one CTA of each other.
 template <typename T, int BITS, int MODE, bool RING>
 struct Shape {
-  static_assert(!RING || (MODE != RQ_DQ && sizeof(T) == 2 && BITS <= 3), "ring shape");
+  static_assert(!RING || (MODE != RQ_DQ && sizeof(T) == 2 && BITS <= 4), "ring shape");
   static constexpr bool kRing = RING;
-  static constexpr int kWarps = kRing ? 16 : 2;
+  static constexpr int kWarps = kRing ? (BITS == 4 ? 14 : 16) : 2;
   static constexpr int kRows = 32 * kWarps;  // threads per CTA
 };
 constexpr float kB = 4611686018427387904.0f;      // 2^62
@@ -1476,10 +1476,10 @@ int rq_row_box_rows() { return row::kWR; }
 
 bool rq_row_dims(int d, kvrq_dtype dt) { return d == 128 || (d == 256 && dt != KVRQ_F32); }
 
-// The ring shape exists for d = 128, 16-bit rows, quantize or fused, b <= 3, and buffers that fit.
+// The ring shape exists for d = 128, 16-bit rows, quantize or fused, and buffers that fit.
 template <typename T, int BITS, int MODE, int DD, int L>
 constexpr bool can_ring() {
-  if constexpr (DD == 128 && MODE != RQ_DQ && sizeof(T) == 2 && BITS <= 3)
+  if constexpr (DD == 128 && MODE != RQ_DQ && sizeof(T) == 2)
     return row::Smem<T, BITS, MODE, true, DD, L>::fits;
   else
     return false;
@@ -1490,7 +1490,7 @@ static cudaError_t launch_row(const CUtensorMap& mx, const CUtensorMap& mo, cons
                               int num_sms) {
   // the ring pays off once every warp of the GPU has two sub-tiles or more
   if constexpr (can_ring<T, BITS, MODE, DD, L>()) {
-    if ((a.n + row::kWR - 1) / row::kWR >= 2 * 16 * (int64_t)num_sms)
+    if ((a.n + row::kWR - 1) / row::kWR >= 2 * row::Shape<T, BITS, MODE, true>::kWarps * (int64_t)num_sms)
       return launch_row_s<T, BITS, MODE, true, DD, L>(mx, mo, a, st, num_sms);
   }
   return launch_row_s<T, BITS, MODE, false, DD, L>(mx, mo, a, st, num_sms);

@@ -84,10 +84,10 @@ def test_ragged_and_dtypes(dt, n):
     _check(synth.lognormal(n, D, seed=n, dtype=dt).cuda(), 3)
 
 
-@pytest.mark.parametrize("bits", [1, 2])
+@pytest.mark.parametrize("bits", [1, 2, 4])
 def test_ring_shape_large_launch(bits):
     # 200,000 rows is over two 32-row sub-tiles per warp of the GPU: the ring-buffered shape (b <= 2 in this
-    # layout, where its code words fit)
+    # layout with 16-warp CTAs, b = 4 with 14; at b = 3 the code words of 16 warps do not fit)
     n = 200000
     x = synth.lognormal(n, D, seed=77, dtype=torch.float16).cuda()
     rows = np.unique(np.concatenate([np.random.default_rng(5).choice(n, 1500, replace=False), [0, n - 1]]))

@@ -110,11 +110,12 @@ def test_general_bulk_rows_strided():
     _check_roundtrip(base[:, :256], 2)
 
 
-@pytest.mark.parametrize("bits", [1, 2, 3])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
 @pytest.mark.parametrize("dt", ["f16", "bf16"])
 def test_ring_sizes(dt, bits):
-    # 160,033 rows: every warp has two 32-row sub-tiles or more, so the quantizing modes take the
-    # ring of half-tile boxes; dequantize (never the ring) must reproduce the fused x_hat bit for bit
+    # 160,033 rows: every warp has two 32-row sub-tiles or more (16-warp CTAs, 14 at b = 4), so the
+    # quantizing modes take the ring of half-tile boxes; dequantize (never the ring) must reproduce the
+    # fused x_hat bit for bit
     n = 160033
     x = synth.lognormal(n, 128, seed=bits + 7, dtype=DT[dt]).cuda()
     sample = np.unique(np.concatenate([np.random.default_rng(bits).choice(n, 1536, replace=False),
