@@ -21,7 +21,8 @@
 //  * tq_prod_kernel (prod quantize): 256 threads, two per row; Pi and T leave room for
 //    one tile buffer at two CTAs per SM, so the sketch operand goes to tensor memory
 //    and the buffer takes the next tile's x as soon as the first product has read it.
-//  * tq_dq_prod_kernel (prod dequantize): 128 threads, one per row, one tile at a time.
+//  * tq_dq_prod_kernel (prod dequantize): 256 threads, two per row; the sign operand in tensor
+//    memory, the corrected centroids in the tile buffer, one tile at a time.
 // Two CTAs share an SM (256 TMEM columns each), so one CTA's MMAs overlap the other's
 // epilogue.
 
@@ -55,19 +56,6 @@ struct Codes {
   static constexpr int NWIN = (NC + CPW - 1) / CPW;
 };
 
-struct SmemD {
-  static constexpr int tile_off = 0;
-  static constexpr int pi_off = kTileBytes;
-  static constexpr int t_off = pi_off + kTileBytes;
-  static constexpr int codes_off = t_off + kTileBytes;  // [kRows][W], W <= 16
-  static constexpr int signs_off = codes_off + kRows * 16 * 4;  // [kRows][D/32]
-  static constexpr int cb_off = signs_off + kRows * (D / 32) * 4;
-  static constexpr int bar_off = cb_off + 64 * 4;  // params, mma
-  static constexpr int tmem_off = bar_off + 2 * 8;
-  static constexpr int bytes = tmem_off + 16;
-  static constexpr int alloc = bytes + 1024;
-};
-static_assert(2 * (SmemD::alloc + 1024) <= 228 * 1024, "two CTAs per SM");
 
 // Positive-side quantizer constants (see rq_kernels.cu for the construction):
 // sc[j] = -tau_{j+1} * B, chain of unit centroids c[H] + sum step_j * dl[j].
@@ -100,170 +88,6 @@ template <typename T>
 struct IsBf16 {
   static constexpr bool value = std::is_same<T, __nv_bfloat16>::value;
 };
-
-// TurboQuant-prod dequantize at d = 128: x_hat = ||x|| Pi^T (c_hat + sqrt(pi/2)/m gamma T^T s). One
-// thread per row (TMEM lane); per tile the +-1 sign operand S goes through the tile buffer into
-// T^T s (MN-major T), the corrected centroids w into Pi^T w, and x_hat leaves by TMA.
-template <typename T, int BITS>
-__global__ void __launch_bounds__(kRows, 1)
-    tq_dq_prod_kernel(const __grid_constant__ CUtensorMap map_pi, const __grid_constant__ CUtensorMap map_t,
-                      const __grid_constant__ CUtensorMap map_o, TqArgs a) {
-  using SM = SmemD;
-  constexpr int W = Codes<BITS>::W;
-  static_assert(W <= 16, "code staging");
-  constexpr int NS = D / 32;  // sign words per row
-  constexpr uint32_t kNcols = 256;
-  constexpr uint32_t kIdPiT = umma_idesc_f16(IsBf16<T>::value, IsBf16<T>::value, true, D, kRows);  // W Pi
-  constexpr uint32_t kIdTT = umma_idesc_f16(false, false, true, D, kRows);                          // S T
-
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* s_tile = smem + SM::tile_off;
-  uint8_t* s_pi = smem + SM::pi_off;
-  uint8_t* s_t = smem + SM::t_off;
-  uint32_t* s_codes = reinterpret_cast<uint32_t*>(smem + SM::codes_off);
-  uint32_t* s_signs = reinterpret_cast<uint32_t*>(smem + SM::signs_off);
-  float* s_sc = reinterpret_cast<float*>(smem + SM::cb_off);
-  float* s_mag = s_sc + 16;
-  float* s_cf = s_sc + 32;
-  float* s_bscale = s_sc + 48;
-  uint64_t* bar_p = reinterpret_cast<uint64_t*>(smem + SM::bar_off);
-  uint64_t* bar_m = bar_p + 1;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + SM::tmem_off);
-
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int64_t n = a.n;
-  const int64_t ntiles = (n + kRows - 1) / kRows;
-  const uint32_t tile_s = smem_u32(s_tile), pi_s = smem_u32(s_pi), t_s = smem_u32(s_t);
-
-  if (tid == 0) {
-    tma_prefetch_desc(&map_pi);
-    tma_prefetch_desc(&map_t);
-    tma_prefetch_desc(&map_o);
-    mbar_init(bar_p, 1);
-    mbar_init(bar_m, 1);
-    fence_barrier_init();
-  }
-  if (warp == 0) tmem_alloc(s_tmem, kNcols);
-  build_consts<BITS>(a.centroids, s_sc, s_mag, s_cf, s_bscale);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *s_tmem;
-  const uint32_t tm_y = tmem, tm_2 = tmem + 128;          // two 128-column accumulators
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;  // this warp's TMEM lanes
-
-  // resident parameters
-  if (tid == 0) {
-    mbar_arrive_expect_tx(bar_p, 2 * kTileBytes);
-    for (int b = 0; b < 2; ++b) tma_load_2d(s_pi + b * kBoxBytes, &map_pi, b * 64, 0, bar_p);
-    for (int b = 0; b < 2; ++b) tma_load_2d(s_t + b * kBoxBytes, &map_t, b * 64, 0, bar_p);
-  }
-  bool ok = __syncthreads_and(mbar_wait(bar_p, 0, a.status));
-  uint32_t par_m = 0;
-
-  // MMA (thread 0): A is the tile buffer (K-major), B = Pi or T (MN-major)
-  auto mma_mnmajor_b = [&](uint32_t tm_d, uint32_t b_s, uint32_t idesc) {
-    tc_fence_after();
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t akoff = (uint32_t)((kk >> 2) * kBoxBytes + (kk & 3) * 32);
-      const uint32_t bkoff = (uint32_t)(kk * 16 * 128);  // 16 K rows of 128 bytes
-      umma_f16(tm_d, umma_desc_sw128(tile_s + akoff, 16, 1024), umma_desc_sw128(b_s + bkoff, kBoxBytes, 1024), idesc,
-               kk > 0);
-    }
-    umma_commit(bar_m);
-  };
-  auto wait_mma = [&]() {
-    const bool r = mbar_wait(bar_m, par_m, a.status);
-    par_m ^= 1;
-    tc_fence_after();
-    return r;
-  };
-  // write 8 floats as one 16-byte chunk of this thread's row in the tile buffer
-  auto put_chunk = [&](int j, const float* v, bool as_f16) {
-    uint4 c = as_f16 ? Elem<__half>::pack(v) : Elem<T>::pack(v);
-    *reinterpret_cast<uint4*>(s_tile + sw128_chunk(tid, j, kBoxBytes)) = c;
-  };
-
-  for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
-    const int64_t row0 = tile * kRows;
-    const int rows = (int)(n - row0 < (int64_t)kRows ? n - row0 : (int64_t)kRows);
-    const int64_t row = row0 + tid;
-    for (int i = tid; i < rows * W; i += kRows) {
-      const int r = i / W, w = i - r * W;
-      s_codes[i] = __ldg(a.codes_in + (row0 + r) * a.ldc + w);
-    }
-    for (int i = tid; i < rows * NS; i += kRows) {
-      const int r = i / NS, w = i - r * NS;
-      s_signs[i] = __ldg(a.signs_in + (row0 + r) * a.lds + w);
-    }
-    const float nrm = tid < rows ? __ldg(a.norms_in + row * a.ldn) : 0.f;
-    const float gam = tid < rows ? __ldg(a.gammas_in + row * a.ldn) : 0.f;
-    if (tid == 0) bulk_wait_read<0>();  // the previous x_hat store has left the tile buffer
-    if (!__syncthreads_and(ok)) break;
-    uint32_t wc[W];
-#pragma unroll
-    for (int w = 0; w < W; ++w) wc[w] = tid < rows ? s_codes[tid * W + w] : 0u;
-    auto code_at = [&](int k) -> uint32_t {
-      const int bit = k * BITS, word = bit >> 5, sh = bit & 31;
-      uint32_t v = wc[word] >> sh;
-      if (sh + BITS > 32) v |= wc[word + 1] << (32 - sh);
-      return v & ((1u << BITS) - 1u);
-    };
-    // S tile of +1/-1 (fp16) -> T^T s
-#pragma unroll
-    for (int c = 0; c < NS; ++c) {
-      const uint32_t sw = tid < rows ? s_signs[tid * NS + c] : 0u;
-      float v[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = ((sw >> i) & 1u) ? 1.f : -1.f;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) put_chunk(4 * c + q, &v[8 * q], true);
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) mma_mnmajor_b(tm_2, t_s, kIdTT);
-    if (!wait_mma()) ok = false;
-    const float qs = a.qjl_scale * gam;  // sqrt(pi/2)/m * gamma
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      float v[32];
-      tmem_ld32(tm_2 + lane_off + 32 * c, v);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = fmaf(qs, v[i], s_cf[code_at(32 * c + i)]);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) put_chunk(4 * c + q, &v[8 * q], false);
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) mma_mnmajor_b(tm_y, pi_s, kIdPiT);  // Pi^T w
-    if (!wait_mma()) ok = false;
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      float v[32];
-      tmem_ld32(tm_y + lane_off + 32 * c, v);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] *= nrm;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) put_chunk(4 * c + q, &v[8 * q], false);
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      for (int b = 0; b < 2; ++b) tma_store_2d(&map_o, b * 64, (int32_t)row0, s_tile + b * kBoxBytes);
-      bulk_commit();
-    }
-    __syncthreads();  // the staged words are rewritten by the next tile
-  }
-  if (tid == 0) bulk_wait_all<0>();
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, kNcols);
-}
 
 // ============================================================================ mse, two threads per row
 // TurboQuant-mse at d = 128 (quantize, roundtrip, dequantize) with 256-thread CTAs: thread (row r,
@@ -877,6 +701,201 @@ __global__ void __launch_bounds__(kThreadsM, 2)
   }
 }
 
+// ============================================================================ prod dequantize, two threads per row
+// x_hat = ||x|| Pi^T (c_hat + sqrt(pi/2)/m gamma T^T s) at d = 128 with 256-thread CTAs, two threads per
+// row. Per tile each thread writes its half of the +-1 sign operand (fp16 pairs) into tensor memory,
+// the A of T^T s (MN-major T); reads T^T s back, adds its centroids (the quantizer's magnitude
+// sequence), and writes the corrected centroids w into the tile buffer, the A of Pi^T w; x_hat goes
+// back over w and leaves by TMA. Pi and T resident (64 KB) and one tile buffer: two CTAs per SM.
+template <typename T, int BITS>
+__global__ void __launch_bounds__(kThreadsM, 2)
+    tq_dq_prod_kernel(const __grid_constant__ CUtensorMap map_pi, const __grid_constant__ CUtensorMap map_t,
+                      const __grid_constant__ CUtensorMap map_o, TqArgs a) {
+  using HR = HalfRow<BITS>;
+  using SM = SmemP;
+  constexpr int H = Codes<BITS>::H, WH = HR::WH;
+  constexpr int NS = D / 32;  // sign words per row
+  constexpr uint32_t kNcols = 256;  // T^T s, then Pi^T w: 0 .. 127; the sign operand: 128 .. 191
+  constexpr uint32_t kIdPiT = umma_idesc_f16(IsBf16<T>::value, IsBf16<T>::value, true, D, kRows);  // W Pi
+  constexpr uint32_t kIdTT = umma_idesc_f16(false, false, true, D, kRows);                          // S T
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* s_pi = smem + SM::pi_off;
+  uint8_t* s_t = smem + SM::t_off;
+  float* s_sc = reinterpret_cast<float*>(smem + SM::cb_off);
+  float* s_mag = s_sc + 16;
+  float* s_cf = s_sc + 32;
+  float* s_bscale = s_sc + 48;
+  uint64_t* bar_p = reinterpret_cast<uint64_t*>(smem + SM::bar_off) + 1;
+  uint64_t* bar_m = bar_p + 1;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + SM::tmem_off);
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int r = tid & (kRows - 1);  // row in the tile = TMEM lane
+  const int h = warp >> 2;          // half of the columns
+  const int64_t n = a.n;
+  const int64_t ntiles = (n + kRows - 1) / kRows;
+  const uint32_t buf_s = smem_u32(smem + SM::buf_off), pi_s = smem_u32(s_pi), t_s = smem_u32(s_t);
+  const bool vec = (a.ldc & 1) == 0 && (reinterpret_cast<uintptr_t>(a.codes_in) & 7u) == 0;
+  const bool svec = (a.lds & 1) == 0 && (reinterpret_cast<uintptr_t>(a.signs_in) & 7u) == 0;
+
+  if (tid == 0) {
+    tma_prefetch_desc(&map_pi);
+    tma_prefetch_desc(&map_t);
+    tma_prefetch_desc(&map_o);
+    mbar_init(bar_p, 1);
+    mbar_init(bar_m, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) tmem_alloc(s_tmem, kNcols);
+  build_consts<BITS>(a.centroids, s_sc, s_mag, s_cf, s_bscale);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+  const uint32_t tm_z = tmem + lane_off + 64u * (uint32_t)h;            // this half's T^T s, then Pi^T w
+  const uint32_t tm_s = tmem + 128u + lane_off + 32u * (uint32_t)h;     // this half's sign operand words
+  if (tid == 0) {
+    mbar_arrive_expect_tx(bar_p, 2 * kTileBytes);
+    for (int b = 0; b < 2; ++b) tma_load_2d(s_pi + b * kBoxBytes, &map_pi, b * 64, 0, bar_p);
+    for (int b = 0; b < 2; ++b) tma_load_2d(s_t + b * kBoxBytes, &map_t, b * 64, 0, bar_p);
+  }
+  // the centroid table of the quantizer's magnitude sequence (b >= 3 codes: the binary search's)
+  if constexpr (BITS >= 3) {
+    Bisect<BITS> bs;
+    bs.magnitudes(s_mag);
+    if (tid < H) {
+      const float m = bs.mag(tid);
+      s_cf[H + tid] = m;
+      s_cf[H - 1 - tid] = -m;
+    }
+  }
+  bool ok = __syncthreads_and(mbar_wait(bar_p, 0, a.status));
+  uint32_t par_m = 0;
+  auto wait_mma = [&]() {
+    const bool w = mbar_wait(bar_m, par_m, a.status);
+    par_m ^= 1;
+    tc_fence_after();
+    return w;
+  };
+
+  for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+    const int64_t row0 = tile * kRows;
+    const int rows = (int)(n - row0 < (int64_t)kRows ? n - row0 : (int64_t)kRows);
+    const bool live = r < rows;
+    const int64_t row = row0 + r;
+    uint32_t wc[WH], sw[2] = {0u, 0u};
+#pragma unroll
+    for (int w = 0; w < WH; ++w) wc[w] = 0u;
+    float nrm = 0.f, gam = 0.f;
+    if (live) {
+      const uint32_t* src = a.codes_in + row * a.ldc + WH * h;
+      if (vec) {
+#pragma unroll
+        for (int w = 0; w < WH; w += 2) {
+          const uint2 v = __ldg(reinterpret_cast<const uint2*>(src + w));
+          wc[w] = v.x, wc[w + 1] = v.y;
+        }
+      } else {
+#pragma unroll
+        for (int w = 0; w < WH; ++w) wc[w] = __ldg(src + w);
+      }
+      const uint32_t* ssrc = a.signs_in + row * a.lds + (NS / 2) * h;
+      if (svec) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(ssrc));
+        sw[0] = v.x, sw[1] = v.y;
+      } else {
+        sw[0] = __ldg(ssrc), sw[1] = __ldg(ssrc + 1);
+      }
+      nrm = __ldg(a.norms_in + row * a.ldn);
+      gam = __ldg(a.gammas_in + row * a.ldn);
+    }
+    // +-1 (fp16) sign operand of this half: bit 1 = +1, a pair of coordinates per word
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      uint32_t so[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const uint32_t t2 = sw[cc] >> (2 * i);
+        so[i] = 0xBC00BC00u ^ ((t2 & 1u) << 15) ^ ((t2 & 2u) << 30);
+      }
+      tmem_st16(tm_s + 16u * (uint32_t)cc, so);
+    }
+    tmem_wait_st();
+    if (tid == 0) bulk_wait_read<0>();  // the previous tile's x_hat store has left the tile buffer
+    tc_fence_before();
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
+    if (tid == 0) {  // T^T s per row
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk)
+        umma_f16_ts(tmem, tmem + 128u + (uint32_t)(8 * kk), umma_desc_sw128(t_s + (uint32_t)(kk * 16 * 128), kBoxBytes, 1024),
+                    kIdTT, kk > 0);
+      umma_commit(bar_m);
+    }
+    if (!wait_mma()) ok = false;
+    auto code_at = [&](int kl) -> uint32_t {
+      const int bit = kl * BITS, word = bit >> 5, sh = bit & 31;
+      uint32_t v = wc[word] >> sh;
+      if (sh + BITS > 32) v |= wc[word + 1] << (32 - sh);
+      return v & ((1u << BITS) - 1u);
+    };
+    const float qs = a.qjl_scale * gam;  // sqrt(pi/2)/m * gamma
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      float v[32];
+      tmem_ld32(tm_z + 32u * (uint32_t)cc, v);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = fmaf(qs, v[i], s_cf[code_at(32 * cc + i)]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) sts_v4(buf_s + sw128_chunk(r, 8 * h + 4 * cc + q, kBoxBytes), Elem<T>::pack(&v[8 * q]));
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
+    if (tid == 0) {  // Pi^T w per row
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t akoff = (uint32_t)((kk >> 2) * kBoxBytes + (kk & 3) * 32);
+        umma_f16(tmem, umma_desc_sw128(buf_s + akoff, 16, 1024),
+                 umma_desc_sw128(pi_s + (uint32_t)(kk * 16 * 128), kBoxBytes, 1024), kIdPiT, kk > 0);
+      }
+      umma_commit(bar_m);
+    }
+    if (!wait_mma()) ok = false;
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      float v[32];
+      tmem_ld32(tm_z + 32u * (uint32_t)cc, v);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] *= nrm;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) sts_v4(buf_s + sw128_chunk(r, 8 * h + 4 * cc + q, kBoxBytes), Elem<T>::pack(&v[8 * q]));
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
+    if (tid == 0) {
+      for (int b = 0; b < 2; ++b)
+        tma_store_2d(&map_o, b * 64, (int32_t)row0, smem + SM::buf_off + b * kBoxBytes);
+      bulk_commit();
+    }
+  }
+  if (tid == 0) bulk_wait_all<0>();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kNcols);
+  }
+}
+
 }  // namespace tq
 
 // ============================================================================ launch
@@ -886,13 +905,13 @@ static cudaError_t launch_tq_dq_prod_t(const CUtensorMap& mp, const CUtensorMap&
   auto kern = tq::tq_dq_prod_kernel<T, BITS>;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, tq::SmemD::alloc);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, tq::SmemP::alloc);
     if (e != cudaSuccess) return e;
     attr = true;
   }
   const int64_t ntiles = (a.n + tq::kRows - 1) / tq::kRows;
   const int64_t grid = std::min<int64_t>(ntiles, (int64_t)num_sms * 2);
-  kern<<<(unsigned)grid, tq::kRows, tq::SmemD::alloc, st>>>(mp, mt, mo, a);
+  kern<<<(unsigned)grid, tq::kThreadsM, tq::SmemP::alloc, st>>>(mp, mt, mo, a);
   return cudaGetLastError();
 }
 
