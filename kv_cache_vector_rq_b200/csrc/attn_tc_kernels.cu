@@ -149,7 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
   }
   if (tid < (1 << VB)) s_vc[tid] = a.v_centroids[tid];
   // B2 rows >= GMAX (the QJL rows of the logit operand have no weights) stay zero for the whole kernel
-  if (GMAX < NB)
+  if constexpr (GMAX < NB)
     for (int i = tid; i < kNWG * 2 * (NB - GMAX) * 32; i += kThreads) {
       const int wg = i / (2 * (NB - GMAX) * 32), rem = i - wg * 2 * (NB - GMAX) * 32;
       const int box = rem / ((NB - GMAX) * 32), rr = rem - box * (NB - GMAX) * 32;
