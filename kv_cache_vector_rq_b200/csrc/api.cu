@@ -1061,7 +1061,7 @@ static kvrq_status attention_call(const char* name, void* stream, kvrq_method k_
   a.ws_acc = a.ws_sq + rows * 128;
   // the chunk count (and so the offset of ws_ml) depends on the path; size both regions for the larger
   const int64_t tpc = attn_tokens_per_cta(n_heads, n_tokens), tpi = attn_tc_tokens_per_item(n_heads, n_tokens);
-  const int64_t nc_max = std::max((n_tokens + tpc - 1) / tpc, kAttnTcParts * ((n_tokens + tpi - 1) / tpi));
+  const int64_t nc_max = std::max((n_tokens + tpc - 1) / tpc, (n_tokens + tpi - 1) / tpi);
   a.ws_ml = a.ws_acc + rows * nc_max * kAttnAS;
   DeviceInfo* di;
   kvrq_status st = current_device(&di);

@@ -398,16 +398,26 @@ int64_t attn_tokens_per_cta(int64_t n_heads, int64_t n_tokens) {
 }
 
 int64_t attn_tc_tokens_per_item(int64_t n_heads, int64_t n_tokens) {
-  // about 16 work items per SM of a 148-SM B200 (a sizing rule, not a device query), at
-  // least 256 tokens, and at most kAttnMaxChunks / kAttnTcParts items per head (the merge's limit)
-  const int64_t want_per_head = (16 * 148 + n_heads - 1) / n_heads;
-  int64_t tpi = (n_tokens + want_per_head - 1) / want_per_head;
-  tpi = ((tpi + 255) / 256) * 256;
-  constexpr int64_t kMaxItems = kAttnMaxChunks / kAttnTcParts;
-  const int64_t min_tpi = ((n_tokens + kMaxItems - 1) / kMaxItems + 255) / 256 * 256;
-  if (tpi < min_tpi) tpi = min_tpi;
-  if (tpi < 256) tpi = 256;
-  return tpi;
+  // Every decode warpgroup of the persistent kernel takes whole items in turn: 444 workers (three
+  // per SM of a 148-SM B200; a sizing rule, not a device query). A head's T tiles are cut into
+  // items of k tiles (the last one shorter); the slowest worker runs ceil(items / 444) items of
+  // k tiles plus about one tile's worth of set-up each, and k is chosen to make that smallest
+  // (ties: fewer items, so fewer partials to merge), with at most kAttnMaxChunks items per head.
+  constexpr int64_t kWorkers = 148 * kAttnTcParts;
+  const int64_t T = (n_tokens + 127) / 128;
+  if (T <= 1) return 128;
+  int64_t best_k = T, best_cost = -1;
+  for (int64_t ip = 1; ip <= T && ip <= kAttnMaxChunks; ++ip) {
+    const int64_t k = (T + ip - 1) / ip;
+    const int64_t items = (T + k - 1) / k;
+    if (items != ip) continue;  // the same k as a smaller ip
+    const int64_t cost = ((n_heads * items + kWorkers - 1) / kWorkers) * (k + 1);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best_k = k;
+    }
+  }
+  return best_k * 128;
 }
 
 size_t attn_workspace_bytes(int64_t n_heads, int group, int64_t n_tokens) {
@@ -415,7 +425,7 @@ size_t attn_workspace_bytes(int64_t n_heads, int group, int64_t n_tokens) {
   const int64_t tpc = attn_tokens_per_cta(n_heads, n_tokens);
   const int64_t nc_cuda = (n_tokens + tpc - 1) / tpc;
   const int64_t tpi = attn_tc_tokens_per_item(n_heads, n_tokens);
-  const int64_t nc_tc = kAttnTcParts * ((n_tokens + tpi - 1) / tpi);
+  const int64_t nc_tc = (n_tokens + tpi - 1) / tpi;
   const int64_t nc = nc_cuda > nc_tc ? nc_cuda : nc_tc;
   return (size_t)rows * 4 * (kAttnQS + 128 + nc * (kAttnAS + 2));
 }
@@ -425,7 +435,7 @@ cudaError_t launch_attention(int k_method, int k_cbits, AttnArgs a, cudaStream_t
   const bool tc = attn_tc_supported(k_method, k_cbits, a.v_bits, a.group);
   if (tc) {
     a.tokens_per_cta = attn_tc_tokens_per_item(a.n_heads, a.n_tokens);
-    a.n_chunks = (int)(kAttnTcParts * ((a.n_tokens + a.tokens_per_cta - 1) / a.tokens_per_cta));
+    a.n_chunks = (int)((a.n_tokens + a.tokens_per_cta - 1) / a.tokens_per_cta);
   } else {
     a.tokens_per_cta = attn_tokens_per_cta(a.n_heads, a.n_tokens);
     a.n_chunks = (int)((a.n_tokens + a.tokens_per_cta - 1) / a.tokens_per_cta);

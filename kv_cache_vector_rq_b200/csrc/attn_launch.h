@@ -12,7 +12,7 @@ constexpr int kAttnQS = 132;   // floats per rotated-query row (3G = 129 used fo
 constexpr int kAttnAS = 132;   // floats per value-accumulator row (3G = 129 rotated value coordinates used)
 constexpr int kAttnSub = 256;  // tokens per sub-chunk: one per thread of the chunk kernel
 constexpr int kAttnMaxChunks = 1024;
-constexpr int kAttnTcParts = 3;  // tensor-core path: partials per work item (its decode warpgroups)
+constexpr int kAttnTcParts = 3;  // tensor-core path: decode warpgroups per CTA, each taking its own work items
 
 struct AttnArgs {
   int64_t n_heads;          // KV heads (layers x batch x KV heads, flattened)
@@ -66,7 +66,7 @@ struct AttnArgs {
 };
 
 // Tokens per chunk CTA of the CUDA-core path (a multiple of kAttnSub), tokens per
-// work item of the tensor-core path (a multiple of 256), and the workspace the call
+// work item of the tensor-core path (a multiple of 128), and the workspace the call
 // needs (enough for either path); all depend on the sizes only, not on the device.
 int64_t attn_tokens_per_cta(int64_t n_heads, int64_t n_tokens);
 int64_t attn_tc_tokens_per_item(int64_t n_heads, int64_t n_tokens);
@@ -77,7 +77,7 @@ size_t attn_workspace_bytes(int64_t n_heads, int group, int64_t n_tokens);
 bool attn_tc_supported(int k_method, int k_cbits, int v_bits, int group);
 
 // The tensor-core chunk kernel (a.tokens_per_cta = tokens per work item, a.n_chunks =
-// kAttnTcParts x work items per head); persistent, at most num_sms CTAs.
+// work items per head, one partial each); persistent, at most num_sms CTAs.
 cudaError_t launch_attention_tc(int k_method, int k_cbits, const AttnArgs& a, cudaStream_t st, int num_sms);
 
 // k_method: kvrq_method of the keys; k_cbits: stored key-code width. Chooses the path

@@ -21,11 +21,14 @@
 // the inverse sandwich once per query row.
 //
 // B200 shape: a persistent CTA of three decode warpgroups per SM (tensor memory holds
-// A1 and both accumulators of each; 168 registers per thread); work items are (KV head,
-// token chunk) pairs. A warpgroup streams its tiles' code rows, sign rows and norms by
-// bulk copy into its own stage (the next tile's copy lands while the current tile is
-// computed) and is its own pipeline: its first thread issues the copies and both MMAs. Every wait is bounded; a time-out is recorded in the device status
-// word and the CTA drains its copies and MMAs before it leaves.
+// A1 and both accumulators of each; 168 registers per thread). Each warpgroup is a
+// worker of its own: it takes (KV head, token range) work items in turn, writes the
+// head's query operand B1 into its own buffer, streams the item's code rows, sign rows
+// and norms by bulk copy into its own stage (the next tile's copy lands while the
+// current tile is computed; an item's first copy while B1 is written), and leaves one
+// partial per item. Its first thread issues the copies and both MMAs. Every wait is
+// bounded; a time-out is recorded in the device status word and the warpgroup drains
+// its copies and MMAs and stops.
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -92,8 +95,9 @@ struct Cfg {
   static constexpr int vlut_off = slut_off + (kProd ? 256 * SLINE : 0);
   static constexpr int vc_off = vlut_off + VL::BYTES;  // fp32 value centroids [16]
   static constexpr int b1_off = ((vc_off + 64 + 1023) / 1024) * 1024;
+  static constexpr int B1_BYTES = ((KBOX * B_BOX + 1023) / 1024) * 1024;       // per wg
   static constexpr int A2_ATOM = kRows * 128;  // 64 coordinates x 128 tokens
-  static constexpr int a2_off = b1_off + ((KBOX * B_BOX + 1023) / 1024) * 1024;  // [wg][2 atoms]
+  static constexpr int a2_off = b1_off + kNWG * B1_BYTES;                         // [wg][2 atoms]
   static constexpr int B2_BYTES = 2 * B_BOX;                                     // 128 tokens x NB rows
   static constexpr int b2_off = a2_off + kNWG * 2 * A2_ATOM;                      // [wg]
   static constexpr int stage_off = b2_off + kNWG * B2_BYTES;                      // [wg][stage]
@@ -171,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
   const uint32_t o_t = s_t + (uint32_t)NB;
   const uint32_t s_mma = a1_mma + (uint32_t)C::KAP;
   const uint32_t o_mma = s_mma + (uint32_t)NB;
-  const uint32_t b1_s = smem_u32(smem + C::b1_off);
+  const uint32_t b1_s = smem_u32(smem + C::b1_off + w * C::B1_BYTES);
   const uint32_t a2_s = smem_u32(smem + C::a2_off + w * 2 * C::A2_ATOM);
   const uint32_t b2_s = smem_u32(smem + C::b2_off + w * C::B2_BYTES);
   uint32_t* w_stage = reinterpret_cast<uint32_t*>(smem + C::stage_off) + w * kStages * C::stage_words;
@@ -187,7 +191,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
   int slot = 0;             // stage of this warpgroup's next tile
   bool ok = true;
 
-  for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
+  // each warpgroup is a worker of its own: items w * gridDim.x + blockIdx.x, then every
+  // kNWG * gridDim.x-th one
+  const int64_t n_workers = (int64_t)kNWG * gridDim.x;
+  for (int64_t item = (int64_t)w * gridDim.x + blockIdx.x; item < n_items; item += n_workers) {
     const int64_t head = item / items_per_head;
     const int64_t chunk = item - head * items_per_head;
     const int64_t row0 = head * group;
@@ -212,27 +219,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
                       al16(knb) && al16(vnb) && (!kProd || (al16(sbase) && al16(kgb))) && (t_begin % 4) == 0;
     auto tile_full = [&](int j) { return t_begin + (int64_t)(j + 1) * kRows <= t_end; };
 
-    // ---- B1: fp16 K-major, 128-byte swizzle; row g < group: q'_g over K [0, KC);
-    //      prod row GMAX + g: (T q')_g over K [KC, KC + 128); all else zero
-    for (int idx = tid; idx < NB * (C::KBOX * 8); idx += kThreads) {
-      const int row = idx / (C::KBOX * 8), j = idx - row * (C::KBOX * 8);
-      float v[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int k = 8 * j + e;
-        float val = 0.f;
-        if (k < KC) {
-          if (row < group && k < C::NCODE) val = a.ws_q[(row0 + row) * kAttnQS + k];
-        } else if (kProd && k < K) {
-          if (row >= GMAX && row - GMAX < group) val = a.ws_sq[(row0 + row - GMAX) * 128 + (k - KC)];
-        }
-        v[e] = val;
-      }
-      *reinterpret_cast<uint4*>(smem + C::b1_off + sw128_chunk(row, j, C::B_BOX)) = Elem<__half>::pack(v);
-    }
-    fence_proxy_async_smem();  // generic writes of B1, read by the MMAs
-    __syncthreads();
-
     auto issue = [&](int j, int s) {  // thread 0 of the warpgroup: tile j into stage s
       const int64_t t0 = t_begin + (int64_t)j * kRows;
       uint32_t* dst = w_stage + s * C::stage_words;
@@ -248,15 +234,39 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
         bulk_load(dst + C::st_vn + g0, vnb + sl, seg * 4, bar);
       }
     };
-    const int nt_w = ntiles > w ? (ntiles - w + kNWG - 1) / kNWG : 0;  // this warpgroup's tiles
+    const int nt_w = ntiles;  // this warpgroup's tiles: all of the item's
     const int slot0 = slot;
     uint32_t pend = 0;  // bit s: a copy into stage s is in flight (thread 0 of the warpgroup)
+    // the first tiles' copies (the stages are free: the last item's tiles have been read) land
+    // while B1 is written
     if (r == 0 && bulk && ok)
       for (int q = 0; q < kStages && q < nt_w; ++q)
-        if (tile_full(w + q * kNWG)) {
-          issue(w + q * kNWG, (slot0 + q) % kStages);
+        if (tile_full(q)) {
+          issue(q, (slot0 + q) % kStages);
           pend |= 1u << ((slot0 + q) % kStages);
         }
+
+    // ---- B1: fp16 K-major, 128-byte swizzle; row g < group: q'_g over K [0, KC);
+    //      prod row GMAX + g: (T q')_g over K [KC, KC + 128); all else zero
+    for (int idx = r; idx < NB * (C::KBOX * 8); idx += 128) {
+      const int row = idx / (C::KBOX * 8), j = idx - row * (C::KBOX * 8);
+      float v[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int k = 8 * j + e;
+        float val = 0.f;
+        if (k < KC) {
+          if (row < group && k < C::NCODE) val = a.ws_q[(row0 + row) * kAttnQS + k];
+        } else if (kProd && k < K) {
+          if (row >= GMAX && row - GMAX < group) val = a.ws_sq[(row0 + row - GMAX) * 128 + (k - KC)];
+        }
+        v[e] = val;
+      }
+      *reinterpret_cast<uint4*>(smem + C::b1_off + w * C::B1_BYTES + sw128_chunk(row, j, C::B_BOX)) =
+          Elem<__half>::pack(v);
+    }
+    fence_proxy_async_smem();  // generic writes of B1, read by the MMAs
+    asm volatile("bar.sync %0, 128;" ::"r"(1 + w) : "memory");
 
     float m_run[GMAX], l_part[GMAX], a128[GMAX];
 #pragma unroll
@@ -268,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
     bool mma1_out = false, mma2_out = false;  // committed and not yet waited for
     int i = 0;
     for (; i < nt_w; ++i) {
-      const int j = w + i * kNWG;
+      const int j = i;
       const int s = (slot0 + i) % kStages;
       const int64_t t0 = t_begin + (int64_t)j * kRows;
       const int rows = (int)(t_end - t0 < (int64_t)kRows ? t_end - t0 : (int64_t)kRows);
@@ -398,8 +408,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
         }
         umma_commit(bar1);
         const int in = i + kStages;
-        if (staged && in < nt_w && tile_full(w + in * kNWG)) {
-          issue(w + in * kNWG, s);
+        if (staged && in < nt_w && tile_full(in)) {
+          issue(in, s);
           pend |= 1u << s;
         }
       }
@@ -549,9 +559,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
       mma2_out = true;
     }
 
-    // ---- this warpgroup's partial of the item: chunk 2 * chunk + w of each query row
+    // ---- this warpgroup's partial of the item: chunk `chunk` of each query row
     const int64_t nck = a.n_chunks;
-    const int64_t cidx = kNWG * chunk + w;
+    const int64_t cidx = chunk;
     float o[NB];
     if (mma2_out) {
       ok = mbar_wait(bar2, n2 & 1u, a.status) && ok;
@@ -617,8 +627,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
     if (i == 0 || !ok)
       for (int g = 0; g < group && g < GMAX; ++g) a.ws_acc[((row0 + g) * nck + cidx) * kAttnAS + r] = 0.f;
     tc_fence_before();
-    __syncthreads();  // both warpgroups are done with B1 and with this item's buffers
-    if (!__syncthreads_and(ok)) break;
+    // the warpgroup is done with its B1, red and this item's buffers; it stops after a time-out
+    if (!wg_all(ok, 1 + w)) break;
   }
   tc_fence_before();
   __syncthreads();

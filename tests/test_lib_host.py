@@ -202,11 +202,14 @@ def test_attention_workspace_and_validation_fail_before_any_launch():
     lib = kvrq.lib()
     EINVAL, EUNSUP = 1, 2
     # rows x (132 rotated-query floats + 128 sketch floats + chunks x (132 sums + max + sum)) x 4 bytes, with
-    # chunks the larger of the CUDA-core kernel's (token chunks) and the tensor-core kernel's (three partials per
-    # work item; work items of a multiple of 256 tokens, about 16 per SM of a 148-SM GPU, at most 341 per head)
-    assert lib.kvrq_attention_workspace_bytes(1, 8, 1000) == 8 * 4 * (260 + 12 * 134)  # 4 items of 256 tokens
-    assert lib.kvrq_attention_workspace_bytes(72, 8, 131073) == 576 * 4 * (260 + 99 * 134)  # 33 items of 4,096
-    assert lib.kvrq_attention_workspace_bytes(1, 1, 1000000) == 4 * (260 + 978 * 134)  # 326 items of 3,072
+    # chunks the larger of the CUDA-core kernel's (token chunks of a multiple of 256 tokens) and the tensor-core
+    # kernel's (one partial per work item: items of k 128-token tiles, k making ceil(items / 444) * (k + 1)
+    # smallest for 444 warpgroup workers, at most 1,024 items per head)
+    assert lib.kvrq_attention_workspace_bytes(1, 8, 1000) == 8 * 4 * (260 + 8 * 134)  # 8 items of 128 tokens
+    # 33 CUDA-core chunks of 4,096 tokens (the tensor-core path: 6 items of 171 tiles)
+    assert lib.kvrq_attention_workspace_bytes(72, 8, 131073) == 576 * 4 * (260 + 33 * 134)
+    # 977 CUDA-core chunks of 1,024 tokens (the tensor-core path: 435 items of 18 tiles)
+    assert lib.kvrq_attention_workspace_bytes(1, 1, 1000000) == 4 * (260 + 977 * 134)
     assert lib.kvrq_attention_workspace_bytes(0, 8, 100) == 0
     wsb = lib.kvrq_attention_workspace_bytes(2, 8, 100)
 
