@@ -402,7 +402,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       bulk_commit();
     }
   }
-  if (tid == 0) bulk_wait_all<0>();
+  // the stores have read their shared-memory sources; their writes complete with the grid
+  if (tid == 0) bulk_wait_read<0>();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {

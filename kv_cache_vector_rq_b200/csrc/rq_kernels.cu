@@ -651,6 +651,19 @@ __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
           if (kOut) bulk_wait_read<0>();
           issue_box(sub_of(it + 1), 1, blo);
         }
+      } else if constexpr (kOut) {
+        // every box but the last leaves as soon as the pair writing its last x_hat chunk is done
+        // (the pairs before it have read its input chunks), so its store overlaps the rest
+#pragma unroll
+        for (int b = 0; b + 1 < TL::kBoxes; ++b)
+          if (p == ((b + 1) * TL::kBoxElems - 1) / 6) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&map_o, b * TL::kBoxElems, (int32_t)row0, tb + b * TL::kBoxBytes);
+              bulk_commit();
+            }
+          }
       }
     }
 
@@ -667,8 +680,8 @@ __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
       if constexpr (kOut && kRing) {
         tma_store_2d(&map_o, TL::kBoxElems, (int32_t)row0, box_hi);
       } else if constexpr (kOut) {
-#pragma unroll
-        for (int b = 0; b < TL::kBoxes; ++b) tma_store_2d(&map_o, b * TL::kBoxElems, (int32_t)row0, tb + b * TL::kBoxBytes);
+        constexpr int b = TL::kBoxes - 1;  // the others left during pass 2
+        tma_store_2d(&map_o, b * TL::kBoxElems, (int32_t)row0, tb + b * TL::kBoxBytes);
       }
       if (codes_bulk_out) bulk_store(a.codes_out + row0 * W, stage_codes, kWR * W * 4);
       if (kOut || codes_bulk_out) bulk_commit();
@@ -693,7 +706,8 @@ __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
         }
     }
   }
-  if (lane == 0) bulk_wait_all<0>();
+  // the stores have read their shared-memory sources; their writes complete with the grid
+  if (lane == 0) bulk_wait_read<0>();
 }
 
 }  // namespace row

@@ -419,7 +419,8 @@ __global__ void __launch_bounds__(kThreadsM, 2)
       ok = __syncthreads_and(ok);
     }
   }
-  if (tid == 0) bulk_wait_all<0>();
+  // the stores have read their shared-memory sources; their writes complete with the grid
+  if (tid == 0) bulk_wait_read<0>();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -887,7 +888,8 @@ __global__ void __launch_bounds__(kThreadsM, 2)
       bulk_commit();
     }
   }
-  if (tid == 0) bulk_wait_all<0>();
+  // the stores have read their shared-memory sources; their writes complete with the grid
+  if (tid == 0) bulk_wait_read<0>();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
