@@ -394,8 +394,9 @@ kvrq_status kvrq_params_import(const char* path, int d, int bits, int m, uint64_
  * in the device status word (read and cleared by kvrq_device_status), waits at the
  * default limit for its own copies and products still in flight, frees its tensor
  * memory and returns (its outputs are then incomplete). kvrq_set_wait_limit sets
- * the polls of the packed-score kernel's main-loop waits for the calls that follow
- * in this process (negative: the default, 2^24 polls), so a test can make a wait
+ * the polls of the packed-score kernel's main-loop waits and of the tensor-core
+ * attention kernel's tile-copy waits for the calls that follow in this process
+ * (negative: the default, 2^24 polls), so a test can make a wait
  * run out with no fault: with 0 those waits give up without polling (a single poll
  * may itself block until a copy lands). */
 void kvrq_set_wait_limit(int64_t polls);

@@ -1067,6 +1067,7 @@ static kvrq_status attention_call(const char* name, void* stream, kvrq_method k_
   kvrq_status st = current_device(&di);
   if (st != KVRQ_OK) return st;
   a.status = di->status;
+  a.spin_limit = g_wait_limit.load();
   if (pg) {
     a.block_tables = pg->block_tables;
     a.ld_table = pg->ld_table;

@@ -56,6 +56,7 @@ struct AttnArgs {
   float* ws_acc;            // [rows][n_chunks][kAttnAS] per-chunk value sums, rotated domain
   float* ws_ml;             // [rows][n_chunks][2] per-chunk (max logit, sum of weights)
   unsigned* status;         // device status word (bounded-wait time-outs of the tensor-core path)
+  int32_t spin_limit;       // polls of the tensor-core path's tile-copy waits (< 0: the default)
   // paged cache (block_tables != NULL, tensor-core path): as ScoreArgs; the head strides then step pool heads
   const int32_t* block_tables;
   int64_t ld_table;

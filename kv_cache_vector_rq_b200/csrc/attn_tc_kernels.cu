@@ -186,6 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
 
   const int64_t items_per_head = (a.n_tokens + a.tokens_per_cta - 1) / a.tokens_per_cta;
   const int64_t n_items = a.n_heads * items_per_head;
+  const uint32_t lim = a.spin_limit < 0 ? kSpinLimit : (uint32_t)a.spin_limit;  // tile-copy waits (the drain: default)
   uint32_t par_st = 0;  // bit s: parity of stage s's next completion
   uint32_t n1 = 0, n2 = 0;  // MMA1 / MMA2 completions waited for so far
   int slot = 0;             // stage of this warpgroup's next tile
@@ -285,9 +286,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
       const bool valid = r < rows;
       const bool staged = bulk && tile_full(j);
       if (staged) {
-        ok = mbar_wait(&bar_st[s], (par_st >> s) & 1u, a.status) && ok;
-        par_st ^= 1u << s;
-        pend &= ~(1u << s);
+        // a copy whose wait ran out stays pending: the drain below waits for it again
+        if (mbar_wait(&bar_st[s], (par_st >> s) & 1u, a.status, lim)) {
+          par_st ^= 1u << s;
+          pend &= ~(1u << s);
+        } else {
+          ok = false;
+        }
       }
       if (!wg_all(ok, 1 + w)) {
         ok = false;
@@ -574,7 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
       mma1_out = false;
     }
     // copies still in flight exist only after a time-out broke the tile loop: they land before the
-    // CTA leaves (the CTA stops after such an item, so the stage parities need no update)
+    // warpgroup leaves (it stops after such an item, so the stage parities need no update)
     if (r == 0)
       for (int s2 = 0; s2 < kStages; ++s2)
         if ((pend >> s2) & 1u) {

@@ -48,3 +48,45 @@ def test_wait_runs_out_and_the_context_recovers():
     torch.cuda.synchronize()
     kvrq.device_status()
     assert torch.equal(again, ref)
+
+
+def test_attention_copy_wait_runs_out_and_the_context_recovers():
+    """The tensor-core attention kernel under the same zero limit: every warpgroup's first tile-copy wait gives
+    up, the warpgroup writes nothing to tensor memory, waits (at the default limit) for the copy it issued and
+    stops; the status reads KVRQ_ETIMEOUT once, and the next call reproduces the reference bit for bit."""
+    heads, tokens = 16, 4096
+    pi = torch.from_numpy(params.rotation(D, 2)).to(torch.float16).cuda()
+    T = torch.from_numpy(params.qjl_matrix(D, D, 3)).to(torch.float16).cuda()
+    ck = torch.from_numpy(codebook.lloyd_max(D, 2)[0].astype(np.float32)).cuda()
+    cv = torch.from_numpy(codebook.lloyd_max(D, 3)[0].astype(np.float32)).cuda()
+    rot = torch.from_numpy(params.rotors(D, 5).astype(np.float32)).cuda()
+    k = synth.lognormal(heads * tokens, D, seed=6, dtype=torch.float16, device="cuda")
+    v = synth.lognormal(heads * tokens, D, seed=7, dtype=torch.float16, device="cuda")
+    kc, ks, kg, kn = kvrq.tq_quantize_prod(k, pi, T, ck, 3)
+    vc, vn = kvrq.rq_quantize(v, rot, cv, 3)
+    q = synth.gaussian(heads * 8, D, seed=8, dtype=torch.float16, device="cuda").view(heads, 8, D)
+    assert kvrq.attention_uses_tensor_cores(kvrq.TQ_PROD, 3, 3, 8)
+
+    def run():
+        return kvrq.kv_attention_packed(kvrq.TQ_PROD, q, kc.view(heads, tokens, -1), kn.view(heads, tokens), 3,
+                                        vc.view(heads, tokens, -1), vn.view(heads, tokens), 3, tokens, ck, rot, cv,
+                                        pi=pi, T=T, k_signs=ks.view(heads, tokens, -1),
+                                        k_gammas=kg.view(heads, tokens))
+
+    ref = run()
+    torch.cuda.synchronize()
+    kvrq.device_status()
+    try:
+        kvrq.lib().kvrq_set_wait_limit(0)
+        run()
+        torch.cuda.synchronize()  # the kernel returned: no hang, no fault
+    finally:
+        kvrq.lib().kvrq_set_wait_limit(-1)
+    with pytest.raises(KvrqError) as e:
+        kvrq.device_status()
+    assert e.value.status == 5  # KVRQ_ETIMEOUT
+    kvrq.device_status()
+    again = run()
+    torch.cuda.synchronize()
+    kvrq.device_status()
+    assert torch.equal(again, ref)
