@@ -58,6 +58,58 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// y = M x for a row-major 128 x 128 matrix M (fp16, or bf16) and x, y in shared memory, by the
+// 128 threads of the CTA: warp w takes rows 32w .. 32w + 31. With M 16-byte aligned, lane l reads
+// 16 bytes (columns 8 (l mod 16) .. + 7) of rows 32w + 2i + l / 16, i < 16, all sixteen loads issued
+// before the first is used; a row's eight-term partial sums are added across its half-warp.
+// Otherwise lane l reads columns l, l + 32, l + 64, l + 96 of each row, and the warp adds them.
+__device__ __forceinline__ void mat_vec128(const void* M, bool bf16, const float* x, float* y) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if ((reinterpret_cast<uintptr_t>(M) & 15) == 0) {
+    const int c0 = 8 * (lane & 15);
+    float xv[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) xv[e] = x[c0 + e];
+    const uint4* base = reinterpret_cast<const uint4*>(M);
+    uint4 w[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) w[i] = __ldg(base + (32 * warp + 2 * i + (lane >> 4)) * 16 + (lane & 15));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t u[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+      float acc = 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float2 f;
+        if (bf16) f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u[k]));
+        else f = __half22float2(*reinterpret_cast<const __half2*>(&u[k]));
+        acc = fmaf(f.x, xv[2 * k], acc);
+        acc = fmaf(f.y, xv[2 * k + 1], acc);
+      }
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if ((lane & 15) == 0) y[32 * warp + 2 * i + (lane >> 4)] = acc;
+    }
+    return;
+  }
+  float xv[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) xv[j] = x[lane + 32 * j];
+#pragma unroll 4
+  for (int i = 32 * warp; i < 32 * warp + 32; ++i) {
+    float acc = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t off = (int64_t)i * 128 + lane + 32 * j;
+      const float m = bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(M)[off])
+                           : __half2float(reinterpret_cast<const __half*>(M)[off]);
+      acc = fmaf(m, xv[j], acc);
+    }
+    acc = warp_sum(acc);
+    if (lane == 0) y[i] = acc;
+  }
+}
+
 // ------------------------------------------------------------------ 1. rotated queries
 // One CTA of 128 threads per query row.
 __global__ void __launch_bounds__(128) attn_rotate_q_kernel(AttnArgs a, int k_method) {
@@ -83,28 +135,15 @@ __global__ void __launch_bounds__(128) attn_rotate_q_kernel(AttnArgs a, int k_me
     }
     return;
   }
-  // q'_i = sum_k Pi[i][k] q_k
-  float acc = 0.f;
-  if (a.pi_bf16) {
-    const __nv_bfloat16* p = reinterpret_cast<const __nv_bfloat16*>(a.pi) + (int64_t)tid * 128;
-#pragma unroll 8
-    for (int k = 0; k < 128; ++k) acc = fmaf(__bfloat162float(p[k]), s_in[k], acc);
-  } else {
-    const __half* p = reinterpret_cast<const __half*>(a.pi) + (int64_t)tid * 128;
-#pragma unroll 8
-    for (int k = 0; k < 128; ++k) acc = fmaf(__half2float(p[k]), s_in[k], acc);
-  }
-  wq[tid] = acc;
+  // q' = Pi q, then (prod) T q'
+  mat_vec128(a.pi, a.pi_bf16, s_in, s_qp);
+  __syncthreads();
+  wq[tid] = s_qp[tid];
   if (tid < kAttnQS - 128) wq[128 + tid] = 0.f;
   if (k_method != KVRQ_TQ_PROD) return;
-  s_qp[tid] = acc;
+  mat_vec128(a.T, false, s_qp, s_in);  // s_in is no longer read: it takes T q'
   __syncthreads();
-  // (T q')_i = sum_k T[i][k] q'_k
-  const __half* t = reinterpret_cast<const __half*>(a.T) + (int64_t)tid * 128;
-  float acc2 = 0.f;
-#pragma unroll 8
-  for (int k = 0; k < 128; ++k) acc2 = fmaf(__half2float(t[k]), s_qp[k], acc2);
-  a.ws_sq[row * 128 + tid] = acc2;
+  a.ws_sq[row * 128 + tid] = s_in[tid];
 }
 
 // ------------------------------------------------------------------ 2. chunk partials

@@ -231,3 +231,35 @@ def test_tc_padded_rows_take_per_thread_loads():
     # and equal to the unpadded launch up to the order of the fp32 sums (the same tiles, the same MMAs)
     ref = _run("tq_prod", 3, 3, keys, kp, values, vp, pi, T, q, n_tok, 1.0 / np.sqrt(D))
     assert np.allclose(got, ref, rtol=0, atol=1e-6 * np.abs(ref).max())
+
+
+@pytest.mark.parametrize("pi_dtype", [torch.float16, torch.bfloat16])
+def test_query_rotation_with_two_byte_aligned_pi_and_T(pi_dtype):
+    """Pi and T only 2-byte aligned (the call accepts that): the query rotation reads them element by element
+    instead of in 16-byte vectors. The outputs match the oracle (fp16 Pi), and the aligned call within 2e-3 of
+    the largest |output|: the two paths add the rotation's products in different orders, and a q' coordinate
+    whose fp32 value moves by that rounding can round to a neighbouring fp16 value in the MMA operand (2^-11
+    relative), which moves its logits and so the softmax weights by about that much."""
+    n_heads, n_tok = 6, 700
+    keys, kp, values, vp, pi, T = _random_cache("tq_prod", 3, 3, n_heads, n_tok, seed=53)
+    q = (2.0 * torch.randn((n_heads, 8, D), generator=torch.Generator().manual_seed(5))).to(torch.float16)
+    pi_buf = torch.zeros(D * D + 1, dtype=pi_dtype, device="cuda")
+    pi_buf[1:] = pi.to(pi_dtype).cuda().reshape(-1)
+    t_buf = torch.zeros(D * D + 1, dtype=torch.float16, device="cuda")
+    t_buf[1:] = T.cuda().reshape(-1)
+    pi_u, t_u = pi_buf[1:].view(D, D), t_buf[1:].view(D, D)
+    assert pi_u.data_ptr() % 16 == 2 and t_u.data_ptr() % 16 == 2
+    kw = dict(k_signs=_dev_words(keys["signs_words"]), k_gammas=_dev_f32(keys["gammas"]))
+    args = (kvrq.TQ_PROD, q.cuda(), _dev_words(keys["words"]), _dev_f32(keys["norms"]), 3, _dev_words(values["words"]),
+            _dev_f32(values["norms"]), 3, n_tok, _dev_f32(kp["centroids"]), _dev_f32(vp["rotors"]),
+            _dev_f32(vp["centroids"]))
+    out_u = kvrq.kv_attention_packed(*args, pi=pi_u, T=t_u, **kw)
+    out_a = kvrq.kv_attention_packed(*args, pi=pi_u.clone(), T=t_u.clone(), **kw)
+    torch.cuda.synchronize()
+    kvrq.device_status()
+    got = out_u.double().cpu().numpy()
+    ref = out_a.double().cpu().numpy()
+    if pi_dtype == torch.float16:
+        _check("tq_prod", 3, 3, keys, kp, values, vp, q, n_tok, 1.0 / np.sqrt(D), got, range(n_heads))
+    err = np.abs(got - ref).max() / np.abs(ref).max()
+    assert err <= 2e-3, err
