@@ -236,6 +236,30 @@ __global__ void __launch_bounds__(kThreadsM, 2)
     return w;
   };
 
+  // dequantize: this thread's half row of tile `t` (zeros past the last row), loaded one tile ahead
+  auto load_codes = [&](int64_t t, uint32_t (&wc_)[WH], float& nrm_) {
+#pragma unroll
+    for (int w = 0; w < WH; ++w) wc_[w] = 0u;
+    nrm_ = 0.f;
+    const int64_t row_ = t * kRows + r;
+    if (t >= ntiles || row_ >= n) return;
+    const uint32_t* src = a.codes_in + row_ * a.ldc + WH * h;
+    if (vec) {
+#pragma unroll
+      for (int w = 0; w < WH; w += 2) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(src + w));
+        wc_[w] = v.x, wc_[w + 1] = v.y;
+      }
+    } else {
+#pragma unroll
+      for (int w = 0; w < WH; ++w) wc_[w] = __ldg(src + w);
+    }
+    nrm_ = __ldg(a.norms_in + row_ * a.ldn);
+  };
+  uint32_t wc_p[WH];
+  float nrm_p = 0.f;
+  if constexpr (!kQ) load_codes(blockIdx.x, wc_p, nrm_p);
+
   int k = 0;
   for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++k) {
     const int s = k & 1;
@@ -357,20 +381,11 @@ __global__ void __launch_bounds__(kThreadsM, 2)
       }
     } else {
       if (tid == 0) bulk_wait_read<1>();  // this buffer's store (two tiles back) has been read
-      if (live) {
-        const uint32_t* src = a.codes_in + row * a.ldc + WH * h;
-        if (vec) {
+      // this tile's codes and norm (loaded during the previous tile); the next tile's load starts now
 #pragma unroll
-          for (int w = 0; w < WH; w += 2) {
-            const uint2 v = __ldg(reinterpret_cast<const uint2*>(src + w));
-            wc[w] = v.x, wc[w + 1] = v.y;
-          }
-        } else {
-#pragma unroll
-          for (int w = 0; w < WH; ++w) wc[w] = __ldg(src + w);
-        }
-        nrm = __ldg(a.norms_in + row * a.ldn);
-      }
+      for (int w = 0; w < WH; ++w) wc[w] = wc_p[w];
+      nrm = nrm_p;
+      load_codes(next, wc_p, nrm_p);
       auto code_at = [&](int kl) -> uint32_t {
         const int bit = kl * BITS, word = bit >> 5, sh = bit & 31;
         uint32_t v = wc[word] >> sh;
@@ -782,37 +797,45 @@ __global__ void __launch_bounds__(kThreadsM, 2)
     return w;
   };
 
+  // this thread's half row of tile `t` (zeros past the last row): code words, sign words, norm, gamma
+  auto load_half_row = [&](int64_t t, uint32_t (&wc_)[WH], uint32_t (&sw_)[2], float& nrm_, float& gam_) {
+#pragma unroll
+    for (int w = 0; w < WH; ++w) wc_[w] = 0u;
+    sw_[0] = sw_[1] = 0u;
+    nrm_ = gam_ = 0.f;
+    const int64_t row = t * kRows + r;
+    if (t >= ntiles || row >= n) return;
+    const uint32_t* src = a.codes_in + row * a.ldc + WH * h;
+    if (vec) {
+#pragma unroll
+      for (int w = 0; w < WH; w += 2) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(src + w));
+        wc_[w] = v.x, wc_[w + 1] = v.y;
+      }
+    } else {
+#pragma unroll
+      for (int w = 0; w < WH; ++w) wc_[w] = __ldg(src + w);
+    }
+    const uint32_t* ssrc = a.signs_in + row * a.lds + (NS / 2) * h;
+    if (svec) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(ssrc));
+      sw_[0] = v.x, sw_[1] = v.y;
+    } else {
+      sw_[0] = __ldg(ssrc), sw_[1] = __ldg(ssrc + 1);
+    }
+    nrm_ = __ldg(a.norms_in + row * a.ldn);
+    gam_ = __ldg(a.gammas_in + row * a.ldn);
+  };
+  uint32_t wc[WH], sw[2];
+  float nrm, gam;
+  load_half_row(blockIdx.x, wc, sw, nrm, gam);
+
   for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
     const int64_t row0 = tile * kRows;
-    const int rows = (int)(n - row0 < (int64_t)kRows ? n - row0 : (int64_t)kRows);
-    const bool live = r < rows;
-    const int64_t row = row0 + r;
-    uint32_t wc[WH], sw[2] = {0u, 0u};
-#pragma unroll
-    for (int w = 0; w < WH; ++w) wc[w] = 0u;
-    float nrm = 0.f, gam = 0.f;
-    if (live) {
-      const uint32_t* src = a.codes_in + row * a.ldc + WH * h;
-      if (vec) {
-#pragma unroll
-        for (int w = 0; w < WH; w += 2) {
-          const uint2 v = __ldg(reinterpret_cast<const uint2*>(src + w));
-          wc[w] = v.x, wc[w + 1] = v.y;
-        }
-      } else {
-#pragma unroll
-        for (int w = 0; w < WH; ++w) wc[w] = __ldg(src + w);
-      }
-      const uint32_t* ssrc = a.signs_in + row * a.lds + (NS / 2) * h;
-      if (svec) {
-        const uint2 v = __ldg(reinterpret_cast<const uint2*>(ssrc));
-        sw[0] = v.x, sw[1] = v.y;
-      } else {
-        sw[0] = __ldg(ssrc), sw[1] = __ldg(ssrc + 1);
-      }
-      nrm = __ldg(a.norms_in + row * a.ldn);
-      gam = __ldg(a.gammas_in + row * a.ldn);
-    }
+    // the next tile's inputs are loaded while this one is computed
+    uint32_t wc_n[WH], sw_n[2];
+    float nrm_n, gam_n;
+    load_half_row(tile + gridDim.x, wc_n, sw_n, nrm_n, gam_n);
     // +-1 (fp16) sign operand of this half: bit 1 = +1, a pair of coordinates per word
 #pragma unroll
     for (int cc = 0; cc < 2; ++cc) {
@@ -887,6 +910,10 @@ __global__ void __launch_bounds__(kThreadsM, 2)
         tma_store_2d(&map_o, b * 64, (int32_t)row0, smem + SM::buf_off + b * kBoxBytes);
       bulk_commit();
     }
+#pragma unroll
+    for (int w = 0; w < WH; ++w) wc[w] = wc_n[w];
+    sw[0] = sw_n[0], sw[1] = sw_n[1];
+    nrm = nrm_n, gam = gam_n;
   }
   // the stores have read their shared-memory sources; their writes complete with the grid
   if (tid == 0) bulk_wait_read<0>();
