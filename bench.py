@@ -549,13 +549,17 @@ def run_leg_only(args):
         rows = heads * t
     else:
         fn, rows = None, None
-    if args.leg == "pq_qdq":  # PolarQuant fused roundtrip at d = 128 (levels of 4, 2, 2, 2 bits)
+    if args.leg in ("pq_qdq", "pq_dq"):  # PolarQuant at d = 128 (levels of 4, 2, 2, 2 bits): roundtrip, dequantize
         x = synth.lognormal(args.rows, D, seed=1, dtype=torch.float16, device=dev)
         pi = torch.from_numpy(kvrq.tq_rotation_init(D, 2)).to(torch.float16).to(dev)
         pc = torch.from_numpy(kvrq.pq_codebooks()).to(dev)
         codes = torch.empty((args.rows, kvrq.PQ_WORDS), dtype=torch.int32, device=dev)
         xh = torch.empty_like(x)
-        fn = lambda: kvrq.pq_quantize_dequantize(x, pi, pc, codes=codes, xhat=xh)
+        if args.leg == "pq_qdq":
+            fn = lambda: kvrq.pq_quantize_dequantize(x, pi, pc, codes=codes, xhat=xh)
+        else:
+            kvrq.pq_quantize_dequantize(x, pi, pc, codes=codes, xhat=xh)
+            fn = lambda: kvrq.pq_dequantize(codes, D, pi, pc, xhat=xh)
         rows = args.rows
     if fn is not None:
         return time_fn(fn, rows, args, torch, kvrq)
@@ -713,7 +717,7 @@ def main():
     ap.add_argument("--no-large", action="store_true", help="skip the 1 GiB HBM-roofline leg")
     ap.add_argument("--leg", default=None,
                     help="time one kernel leg (rq_q3, rq_dq3, rq_qdq3, tq_q3, tq_qdq3, tq_prod3, tq_dqm3, tq_dqp3, "
-                         "any b; score_prod3; pq_qdq) on --rows vectors instead of the workload; used for profiler "
+                         "any b; score_prod3; pq_qdq, pq_dq) on --rows vectors instead of the workload; used for profiler "
                          "captures")
     ap.add_argument("--rows", type=int, default=1 << 20)
     ap.add_argument("--dim", type=int, default=D, help="head dimension of --leg (the tiled TurboQuant path "

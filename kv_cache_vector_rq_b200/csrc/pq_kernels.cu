@@ -288,6 +288,37 @@ __global__ void __launch_bounds__(kThreads, 2)
     return w;
   };
 
+  // dequantize: the code words of this thread's half row of tile `t` (zeros past the last row), loaded
+  // one tile ahead
+  struct Raw {
+    uint32_t l1[4], l2, w10, w11, r[2];
+  };
+  auto load_raw = [&](int64_t t, Raw& o) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o.l1[i] = 0u;
+    o.l2 = o.w10 = o.w11 = o.r[0] = o.r[1] = 0u;
+    const int64_t row_ = t * kRows + r;
+    if (t >= ntiles || row_ >= n) return;
+    const uint32_t* src = a.codes_in + row_ * ldc;
+    if (vec) {
+      const uint4 l = __ldg(reinterpret_cast<const uint4*>(src + 4 * h));
+      o.l1[0] = l.x, o.l1[1] = l.y, o.l1[2] = l.z, o.l1[3] = l.w;
+      o.l2 = __ldg(src + 8 + h);
+      const uint2 m = __ldg(reinterpret_cast<const uint2*>(src + 10));
+      o.w10 = m.x, o.w11 = m.y;
+      const uint2 q = __ldg(reinterpret_cast<const uint2*>(src + 12 + 2 * h));
+      o.r[0] = q.x, o.r[1] = q.y;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o.l1[i] = __ldg(src + 4 * h + i);
+      o.l2 = __ldg(src + 8 + h);
+      o.w10 = __ldg(src + 10), o.w11 = __ldg(src + 11);
+      o.r[0] = __ldg(src + 12 + 2 * h), o.r[1] = __ldg(src + 13 + 2 * h);
+    }
+  };
+  Raw raw_p;
+  if constexpr (!kQ) load_raw(blockIdx.x, raw_p);
+
   int k = 0;
   for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++k) {
     const int s = k & 1;
@@ -323,30 +354,15 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (h == 1) s_xchg[r] = hw.l3 | (hw.l4 << 16);
     } else {
       if (tid == 0) bulk_wait_read<1>();  // this buffer's store (two tiles back) has been read
-      const bool live = r < rows;
-      const uint32_t* src = a.codes_in + (row0 + r) * ldc;
-      uint32_t w10 = 0u, w11 = 0u;
-      if (live && vec) {
-        const uint4 l = __ldg(reinterpret_cast<const uint4*>(src + 4 * h));
-        hw.l1[0] = l.x, hw.l1[1] = l.y, hw.l1[2] = l.z, hw.l1[3] = l.w;
-        hw.l2 = __ldg(src + 8 + h);
-        const uint2 m = __ldg(reinterpret_cast<const uint2*>(src + 10));
-        w10 = m.x, w11 = m.y;
-        const uint2 q = __ldg(reinterpret_cast<const uint2*>(src + 12 + 2 * h));
-        hw.r[0] = q.x, hw.r[1] = q.y;
-      } else if (live) {
+      // this tile's words (loaded during the previous tile); the next tile's load starts now
+      const Raw cur = raw_p;
+      load_raw(next, raw_p);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) hw.l1[i] = __ldg(src + 4 * h + i);
-        hw.l2 = __ldg(src + 8 + h);
-        w10 = __ldg(src + 10), w11 = __ldg(src + 11);
-        hw.r[0] = __ldg(src + 12 + 2 * h), hw.r[1] = __ldg(src + 13 + 2 * h);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) hw.l1[i] = 0u;
-        hw.r[0] = hw.r[1] = 0u;
-      }
-      hw.l3 = (w10 >> (16 * h)) & 0xFFFFu;
-      hw.l4 = (w11 >> (8 * h)) & 0xFFu;
+      for (int i = 0; i < 4; ++i) hw.l1[i] = cur.l1[i];
+      hw.l2 = cur.l2;
+      hw.r[0] = cur.r[0], hw.r[1] = cur.r[1];
+      hw.l3 = (cur.w10 >> (16 * h)) & 0xFFFFu;
+      hw.l4 = (cur.w11 >> (8 * h)) & 0xFFu;
       __syncthreads();  // the buffer is free
     }
     // y_hat (the inverse transform of the codes and the 16-bit radii) as the second A operand
