@@ -360,6 +360,14 @@ __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
   build_consts<BITS>(a.centroids, s_sc, s_mag, s_cf);
   __syncthreads();
 
+  // dequantize: this lane's norm of sub-tile `sub`, loaded one sub-tile ahead (0 past the last row)
+  auto load_norm = [&](int sub) -> float {
+    const int64_t rw = (int64_t)sub * kWR + lane;
+    return (sub < nsub && rw < n) ? __ldg(a.norms_in + rw * a.ldn) : 0.f;
+  };
+  float nrm_pf = 0.f;
+  if constexpr (!kIn) nrm_pf = load_norm(sub_of(0));
+
   int it = 0;
   for (int sub = sub_of(0); sub < nsub; sub = sub_of(++it)) {
     const int s = it % STAGES;
@@ -472,7 +480,8 @@ __global__ void __launch_bounds__(Shape<T, BITS, MODE, RING>::kRows,
         __syncwarp();
       }
     } else {
-      nrm = lane < rows ? __ldg(a.norms_in + row * a.ldn) : 0.f;
+      nrm = nrm_pf;  // (0 for lanes past the last row)
+      nrm_pf = load_norm(sub_of(it + 1));
       nq = nrm;
 #pragma unroll
       for (int w = 0; w < W; ++w) wc[w] = stage_codes[lane * W + w];
