@@ -511,9 +511,11 @@ kvrq_status kv_cache_append(void* stream, kvrq_method method, const void* x, kvr
  *     aligned, overwritten; calls sharing it must be ordered on one stream.
  * d = 128 (m = d); group in 1..16; k_bits 1..4 (prod 2..4); v_bits 1..4;
  * n_heads <= 65535. n_heads = 0 is a no-op; n_tokens = 0 with n_heads > 0 is
- * KVRQ_EINVAL (a softmax over no tokens is undefined). fp32 arithmetic on the
- * CUDA cores; three launches (query rotation, per-chunk online softmax and value
- * sums, chunk merge with one inverse sandwich per query row). */
+ * KVRQ_EINVAL (a softmax over no tokens is undefined). Where
+ * kvrq_attention_uses_tensor_cores is 1 both contractions run on the tensor cores
+ * (fp16 operands, fp32 accumulation), else in fp32 on the CUDA cores; three
+ * launches either way (query rotation, per-chunk online softmax and value sums,
+ * chunk merge with one inverse sandwich per query row). */
 size_t kvrq_attention_workspace_bytes(int64_t n_heads, int group, int64_t n_tokens);
 
 kvrq_status kv_attention_packed(void* stream, kvrq_method k_method, const void* q, kvrq_dtype qdtype, int64_t ldq,
