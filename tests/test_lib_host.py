@@ -198,6 +198,20 @@ def test_tq_validation_fails_before_any_launch():
     assert sk(n=0) == 0
 
 
+def test_attention_chunk_count_stays_within_the_merge_limit():
+    """The merge kernel holds at most 1,024 partials per query row: whatever the head count and length, the
+    workspace is rows x 4 x (260 + chunks x 134) bytes with 1 <= chunks <= 1,024, and chunks covers the
+    tokens (at least one 128-token tile per chunk of the tensor-core path, at most 1,024 of them)."""
+    lib = kvrq.lib()
+    for heads in (1, 3, 72, 148, 1152, 65535):
+        for tokens in (1, 127, 128, 129, 4097, 131073, 1000000, 20000000):
+            b = lib.kvrq_attention_workspace_bytes(heads, 8, tokens)
+            per_row = b // (heads * 8 * 4)
+            assert b == heads * 8 * 4 * per_row and (per_row - 260) % 134 == 0
+            chunks = (per_row - 260) // 134
+            assert 1 <= chunks <= 1024, (heads, tokens, chunks)
+
+
 def test_attention_workspace_and_validation_fail_before_any_launch():
     lib = kvrq.lib()
     EINVAL, EUNSUP = 1, 2
